@@ -1,0 +1,182 @@
+"""fp64 CPU oracle for the RG-LRU recurrent block -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the cpu_baseline / reference leg of
+``bench.py`` may import this package.  The product (the CUDA library and its binding) never
+imports, links or runs it, and it shares no code with the product: the arithmetic lives in
+``rglru_oracle.c`` (plain C, fp64), and this file only marshals numpy arrays into it.
+
+Inputs are the exact values handed to the GPU: fp32 arrays, or bf16 stored as their 16 bits
+in uint16 arrays (widened exactly inside the C code).  Outputs and state are fp64.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rglru_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "librglru_oracle.so")
+_lib = None
+
+F32, BF16 = 0, 1
+HIST = 3  # conv width 4 -> 3 past inputs
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (fp64, no fast-math, no FP contraction, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O3", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+                               "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def load_library(path: str):
+    """Open an oracle build at ``path`` and declare its entry points."""
+    lib = ctypes.CDLL(path)
+    P, I, D, L = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_long
+    lib.rglru_oracle_gelu.restype = D
+    lib.rglru_oracle_gelu.argtypes = [D, I]
+    lib.rglru_oracle_prefill_unit.restype = I
+    lib.rglru_oracle_prefill_unit.argtypes = [I, I, D, I, I, P, L, P, P, P, I, P, P, P,
+                                              P, P, L, P, P, P, L, P, L, P]
+    lib.rglru_oracle_prefill.restype = I
+    lib.rglru_oracle_prefill.argtypes = [I, I, I, I, D, I, I, P, P, P, P, P, P, P,
+                                         P, P, P, P, P, P, P, I, I]
+    lib.rglru_oracle_decode.restype = I
+    lib.rglru_oracle_decode.argtypes = [I, I, I, D, I, I, P, P, P, P, P, P, P,
+                                        P, P, P, P, P, P, I]
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = load_library(build())
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _act(a: np.ndarray):
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray(a), BF16
+    return np.ascontiguousarray(a, dtype=np.float32), F32
+
+
+def _f32(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+
+
+def gelu(v: float, tanh_form: int = 0) -> float:
+    return _load().rglru_oracle_gelu(float(v), int(tanh_form))
+
+
+def prefill(params: dict, x: np.ndarray, y: np.ndarray, heads: int,
+            reset: Optional[np.ndarray] = None, h0: Optional[np.ndarray] = None,
+            tail0: Optional[np.ndarray] = None, c: float = 8.0, gelu_tanh: int = 0,
+            units: Optional[Sequence] = None, threads: int = 0):
+    """Full-sequence prefill of x, y [B, T, W].
+
+    Returns (out [B, T, W] fp64, h [B, W] fp64, tail [B, 3, W] fp64).  h0 / tail0 default to
+    zero.  ``units`` = list of (b, head): only those sequences are computed (others stay 0).
+    """
+    lib = _load()
+    x, dt = _act(x)
+    y, dty = _act(y)
+    assert dt == dty and x.shape == y.shape and x.ndim == 3
+    B, T, W = x.shape
+    dh = W // heads
+    w_a, dtw = _act(params["w_a"])
+    w_x, _ = _act(params["w_x"])
+    assert dtw == dt, "gate weights are stored in the activation dtype"
+    conv_w, conv_b = _f32(params["conv_w"]), _f32(params.get("conv_b"))
+    b_a, b_x, lam = _f32(params.get("b_a")), _f32(params.get("b_x")), _f32(params["lam"])
+    h = np.zeros((B, W)) if h0 is None else np.array(h0, dtype=np.float64, copy=True)
+    tail = np.zeros((B, HIST, W)) if tail0 is None else tail_from_act(tail0).copy()
+    out = np.zeros((B, T, W))
+    rst = None if reset is None else np.ascontiguousarray(reset, dtype=np.uint8)
+    uarr = None
+    n_units = 0
+    if units is not None:
+        uarr = np.ascontiguousarray(np.array(units, dtype=np.int32).reshape(-1, 2))
+        n_units = uarr.shape[0]
+    rc = lib.rglru_oracle_prefill(B, T, heads, dh, c, gelu_tanh, dt, _p(conv_w), _p(conv_b),
+                                  _p(w_a), _p(w_x), _p(b_a), _p(b_x), _p(lam), _p(x), _p(y),
+                                  _p(rst), _p(h), _p(tail), _p(out), _p(uarr), n_units, threads)
+    if rc != 0:
+        raise RuntimeError("oracle prefill failed")
+    return out, h, tail
+
+
+def prefill_unit_decay(params: dict, x: np.ndarray, y: np.ndarray, heads: int, b: int, head: int,
+                       reset: Optional[np.ndarray] = None, c: float = 8.0):
+    """One (b, head) sequence from zero state; returns (out [T, dh], a_t [T, dh])."""
+    lib = _load()
+    x, dt = _act(x)
+    y, _ = _act(y)
+    B, T, W = x.shape
+    dh = W // heads
+    w_a, _ = _act(params["w_a"])
+    w_x, _ = _act(params["w_x"])
+    es = 4 if dt == F32 else 2
+    ch0 = head * dh
+    conv_w = _f32(params["conv_w"])
+    conv_b, b_a, b_x, lam = (_f32(params.get(k)) for k in ("conv_b", "b_a", "b_x", "lam"))
+    h = np.zeros(dh)
+    tail = np.zeros((HIST, dh))
+    out = np.zeros((T, dh))
+    a_out = np.zeros((T, dh))
+    base = lambda arr, off, size: ctypes.c_void_p(arr.ctypes.data + off * size)  # noqa: E731
+    rst = None if reset is None else np.ascontiguousarray(reset[b], dtype=np.uint8)
+    rc = lib.rglru_oracle_prefill_unit(
+        T, dh, c, 0, dt, base(conv_w, ch0, 4), W,
+        None if conv_b is None else base(conv_b, ch0, 4),
+        base(w_a, head * dh * dh, es), base(w_x, head * dh * dh, es), dt,
+        None if b_a is None else base(b_a, ch0, 4), None if b_x is None else base(b_x, ch0, 4),
+        base(lam, ch0, 4), base(x, b * T * W + ch0, es), base(y, b * T * W + ch0, es), W,
+        _p(rst), _p(h), _p(tail), dh, _p(out), dh, _p(a_out))
+    if rc != 0:
+        raise RuntimeError("oracle prefill_unit failed")
+    return out, a_out
+
+
+def decode(params: dict, x: np.ndarray, y: np.ndarray, heads: int, h: np.ndarray,
+           tail: np.ndarray, reset: Optional[np.ndarray] = None, c: float = 8.0,
+           gelu_tanh: int = 0, threads: int = 0):
+    """One decode step for x, y [B, W]; h [B, W] and tail [B, 3, W] (fp64) are updated in
+    place.  Returns out [B, W] fp64."""
+    lib = _load()
+    x, dt = _act(x)
+    y, _ = _act(y)
+    B, W = x.shape
+    dh = W // heads
+    w_a, _ = _act(params["w_a"])
+    w_x, _ = _act(params["w_x"])
+    assert h.dtype == np.float64 and h.flags.c_contiguous
+    assert tail.dtype == np.float64 and tail.flags.c_contiguous
+    conv_w, conv_b = _f32(params["conv_w"]), _f32(params.get("conv_b"))
+    b_a, b_x, lam = _f32(params.get("b_a")), _f32(params.get("b_x")), _f32(params["lam"])
+    rst = None if reset is None else np.ascontiguousarray(reset, dtype=np.uint8)
+    out = np.zeros((B, W))
+    rc = lib.rglru_oracle_decode(B, heads, dh, c, gelu_tanh, dt, _p(conv_w), _p(conv_b),
+                                 _p(w_a), _p(w_x), _p(b_a), _p(b_x), _p(lam), _p(x), _p(y),
+                                 _p(rst), _p(h), _p(tail), _p(out), threads)
+    if rc != 0:
+        raise RuntimeError("oracle decode failed")
+    return out
+
+
+def tail_from_act(tail0: np.ndarray) -> np.ndarray:
+    """fp64 copy of an act-dtype conv history (bf16 bits or fp32)."""
+    if tail0.dtype == np.uint16:
+        return np.ascontiguousarray((tail0.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    return np.ascontiguousarray(tail0, dtype=np.float64)

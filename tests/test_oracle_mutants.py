@@ -1,0 +1,69 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case copies the oracle source, plants one mistake (a dropped term, a wrong sign, a
+swapped index, a transposed operand, a shifted tap, a missed reset), builds it on the CPU and
+runs the pin suite against it: at least one pin has to fail.  Nothing here touches a GPU.
+"""
+
+import os
+import shutil
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "rglru_oracle.c")
+
+MUTANTS = {
+    "transposed_gate_weights": ("widen(w_a, (long)i * dh + o, w_dtype)", "widen(w_a, (long)o * dh + i, w_dtype)"),
+    "dropped_sqrt_normaliser": ("h[o] = a * h[o] + beta * (ig * xc[o]);", "h[o] = a * h[o] + (ig * xc[o]);"),
+    "sign_of_log_decay": ("double log_a = c * r * log_a_base[o];", "double log_a = -c * r * log_a_base[o];"),
+    "raw_x_instead_of_conv": ("h[o] = a * h[o] + beta * (ig * xc[o]);", "h[o] = a * h[o] + beta * (ig * widen(x, (long)t * ld + o, act_dtype));"),
+    "tap_order_reversed": ("acc += (double)conv_w[k * conv_ld + j] * tail[k * tail_ld + j];", "acc += (double)conv_w[(2 - k) * conv_ld + j] * tail[k * tail_ld + j];"),
+    "dropped_conv_bias": ("double acc = conv_b ? (double)conv_b[j] : 0.0;", "double acc = 0.0;"),
+    "reset_keeps_state": ("for (int j = 0; j < dh; ++j) h[j] = 0.0;", "(void)0;"),
+    "gate_bias_swapped": ("ga[o] = b_a ? (double)b_a[o] : 0.0;", "ga[o] = b_x ? (double)b_x[o] : 0.0;"),
+    "input_gate_from_recurrence_weights": ("gx[o] += xi * widen(w_x, (long)i * dh + o, w_dtype);", "gx[o] += xi * widen(w_a, (long)i * dh + o, w_dtype);"),
+    "gelu_tanh_by_default": ("    return 0.5 * v * erfc(-v / sqrt(2.0));", "    return 0.5 * v * (1.0 + tanh(0.7978845608028654 * (v + 0.044715 * v * v * v)));"),
+}
+
+PIN_TESTS = [
+    pins.test_gelu_spot_values,
+    pins.test_closed_form_geometric_sum,
+    pins.test_freeze_when_recurrence_gate_is_zero,
+    pins.test_decay_strictly_inside_unit_interval,
+    lambda: pins.test_bruteforce_unrolling_T8("f32"),
+    pins.test_gate_orientation_is_in_major,
+    pins.test_conv_identity_and_single_taps,
+    pins.test_conv_matches_torch_conv1d_listing_form,
+    pins.test_packed_rows_equal_separate_documents,
+    pins.test_reset_cuts_all_dependence_on_the_past,
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    tmp = tempfile.mkdtemp(prefix="oracle_mutant_")
+    try:
+        path = os.path.join(tmp, "mutant.c")
+        with open(path, "w") as f:
+            f.write(src.replace(old, new))
+        lib_path = os.path.join(tmp, "libmutant.so")
+        subprocess.check_call(["gcc", "-O1", "-std=c11", "-ffp-contract=off", "-fopenmp", "-fPIC",
+                               "-shared", "-o", lib_path, path, "-lm"])
+        monkeypatch.setattr(oracle, "_lib", oracle.load_library(lib_path))
+        failed = []
+        for t in PIN_TESTS:
+            try:
+                t()
+            except AssertionError:
+                failed.append(getattr(t, "__name__", "bruteforce"))
+        assert failed, f"no pin caught the planted mistake '{name}'"
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
