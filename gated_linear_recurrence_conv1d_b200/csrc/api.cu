@@ -1,0 +1,177 @@
+// api.cu -- the C ABI of librglru.so: host-side validation, workspace sizing, dispatch.
+//
+// Every check runs on the host before anything is enqueued; a failed check returns its code
+// and launches nothing.  Device-side conditions are latched in the workspace status word.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "rglru.h"
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;   // status word area at the start of every workspace
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t act_size(int dtype) { return dtype == RGLRU_F32 ? 4 : 2; }
+
+rglru_status check_dims(const rglru_dims* d, bool prefill) {
+    if (!d) return RGLRU_ERR_INVALID_ARG;
+    if (d->batch <= 0 || d->heads <= 0 || d->head_dim <= 0) return RGLRU_ERR_INVALID_ARG;
+    if (prefill && d->seq_len <= 0) return RGLRU_ERR_INVALID_ARG;
+    if (d->act_dtype != RGLRU_F32 && d->act_dtype != RGLRU_BF16) return RGLRU_ERR_INVALID_ARG;
+    if (!(d->c > 0.0f) || d->c != d->c) return RGLRU_ERR_INVALID_ARG;
+    if (d->gelu_tanh != 0 && d->gelu_tanh != 1) return RGLRU_ERR_INVALID_ARG;
+    if (d->conv_width != rglru::kConvWidth) return RGLRU_ERR_UNSUPPORTED;
+    if (d->head_dim % 16 != 0 || d->head_dim > 256) return RGLRU_ERR_UNSUPPORTED;
+    const long long W = (long long)d->heads * d->head_dim;
+    if ((W * (long long)act_size(d->act_dtype)) % 16 != 0) return RGLRU_ERR_UNSUPPORTED;
+    // every [B, T, W] index must fit comfortably in 63 bits; grid dims in 31 bits
+    if (d->heads > 65535 || d->batch > (1 << 30)) return RGLRU_ERR_UNSUPPORTED;
+    if (prefill && (long long)d->batch * d->seq_len * W > (1LL << 40)) return RGLRU_ERR_UNSUPPORTED;
+    return RGLRU_OK;
+}
+
+rglru_status check_params(const rglru_params* p) {
+    if (!p || !p->conv_w || !p->w_a || !p->w_x || !p->lambda) return RGLRU_ERR_INVALID_ARG;
+    if (!aligned(p->conv_w, 4) || !aligned(p->lambda, 4)) return RGLRU_ERR_INVALID_ARG;
+    if ((p->conv_b && !aligned(p->conv_b, 4)) || (p->b_a && !aligned(p->b_a, 4)) ||
+        (p->b_x && !aligned(p->b_x, 4)))
+        return RGLRU_ERR_INVALID_ARG;
+    if (!aligned(p->w_a, 16) || !aligned(p->w_x, 16)) return RGLRU_ERR_INVALID_ARG;
+    return RGLRU_OK;
+}
+
+rglru_status check_state(const rglru_state* s) {
+    if (!s || !s->h || !s->conv_tail) return RGLRU_ERR_INVALID_ARG;
+    if (!aligned(s->h, 4) || !aligned(s->conv_tail, 16)) return RGLRU_ERR_INVALID_ARG;
+    return RGLRU_OK;
+}
+
+rglru_status check_io(const void* x, const void* y, const void* out) {
+    if (!x || !y || !out) return RGLRU_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(out, 16)) return RGLRU_ERR_INVALID_ARG;
+    if (out == x || out == y) return RGLRU_ERR_INVALID_ARG;
+    return RGLRU_OK;
+}
+
+rglru_status check_workspace(void* ws, size_t bytes, size_t need) {
+    if (!ws || bytes < need) return RGLRU_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return RGLRU_ERR_INVALID_ARG;
+    return RGLRU_OK;
+}
+
+rglru_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return RGLRU_OK;
+    cudaGetLastError();   // clear a sticky launch-configuration error for the caller
+    return RGLRU_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rglru_abi_version(void) { return RGLRU_ABI_VERSION; }
+
+const char* rglru_status_string(rglru_status s) {
+    switch (s) {
+        case RGLRU_OK: return "RGLRU_OK";
+        case RGLRU_ERR_INVALID_ARG: return "RGLRU_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
+        case RGLRU_ERR_UNSUPPORTED: return "RGLRU_ERR_UNSUPPORTED: shape outside the supported set";
+        case RGLRU_ERR_WORKSPACE: return "RGLRU_ERR_WORKSPACE: workspace missing or too small";
+        case RGLRU_ERR_CUDA: return "RGLRU_ERR_CUDA: a CUDA runtime call or launch failed";
+        case RGLRU_ERR_TIMEOUT: return "RGLRU_ERR_TIMEOUT: a bounded device-side wait expired";
+        case RGLRU_ERR_DEVICE: return "RGLRU_ERR_DEVICE: a device-side consistency check failed";
+    }
+    return "RGLRU_ERR_UNKNOWN";
+}
+
+rglru_status rglru_state_init(const rglru_dims* dims, rglru_state* state, void* stream) {
+    rglru_status st = check_dims(dims, false);
+    if (st != RGLRU_OK) return st;
+    if ((st = check_state(state)) != RGLRU_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t W = (size_t)dims->heads * dims->head_dim;
+    cudaError_t e = cudaMemsetAsync(state->h, 0, (size_t)dims->batch * W * sizeof(float), s);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(state->conv_tail, 0,
+                            (size_t)dims->batch * rglru::kHist * W * act_size(dims->act_dtype), s);
+    return cuda_status(e);
+}
+
+size_t rglru_prefill_workspace_size(const rglru_dims* dims) {
+    if (check_dims(dims, true) != RGLRU_OK) return 0;
+    return kStatusBytes;
+}
+
+size_t rglru_decode_workspace_size(const rglru_dims* dims) {
+    if (check_dims(dims, false) != RGLRU_OK) return 0;
+    return kStatusBytes;
+}
+
+rglru_status rglru_block_prefill(const rglru_dims* dims, const rglru_params* params,
+                                 const void* x, const void* y, const uint8_t* reset,
+                                 rglru_state* state, void* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    rglru_status st = check_dims(dims, true);
+    if (st != RGLRU_OK) return st;
+    if ((st = check_params(params)) != RGLRU_OK) return st;
+    if ((st = check_io(x, y, out)) != RGLRU_OK) return st;
+    if (state && (st = check_state(state)) != RGLRU_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes, rglru_prefill_workspace_size(dims))) != RGLRU_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cuda_status(rglru::launch_prefill_generic(dims, params, x, y, reset, state, out, s));
+}
+
+rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_params* params,
+                                const void* x, const void* y, const uint8_t* reset,
+                                rglru_state* state, void* out, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    rglru_status st = check_dims(dims, false);
+    if (st != RGLRU_OK) return st;
+    if ((st = check_params(params)) != RGLRU_OK) return st;
+    if ((st = check_io(x, y, out)) != RGLRU_OK) return st;
+    if ((st = check_state(state)) != RGLRU_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes, rglru_decode_workspace_size(dims))) != RGLRU_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cuda_status(rglru::launch_decode_generic(dims, params, x, y, reset, state, out, s));
+}
+
+rglru_status rglru_prefill_plan(const rglru_dims* dims, int* kernel, int* launches) {
+    rglru_status st = check_dims(dims, true);
+    if (st != RGLRU_OK) return st;
+    if (!kernel || !launches) return RGLRU_ERR_INVALID_ARG;
+    *kernel = RGLRU_KERNEL_GENERIC;
+    *launches = 1;
+    return RGLRU_OK;
+}
+
+rglru_status rglru_decode_plan(const rglru_dims* dims, int* kernel, int* launches) {
+    rglru_status st = check_dims(dims, false);
+    if (st != RGLRU_OK) return st;
+    if (!kernel || !launches) return RGLRU_ERR_INVALID_ARG;
+    *kernel = RGLRU_KERNEL_GENERIC;
+    *launches = 1;
+    return RGLRU_OK;
+}
+
+rglru_status rglru_read_device_status(void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace || workspace_bytes < sizeof(rglru::DeviceStatus) || !aligned(workspace, 256))
+        return RGLRU_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    rglru::DeviceStatus host{};
+    cudaError_t e = cudaMemcpyAsync(&host, workspace, sizeof host, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof host, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (host.code == 0) return RGLRU_OK;
+    if (host.code == RGLRU_ERR_TIMEOUT) return RGLRU_ERR_TIMEOUT;
+    return RGLRU_ERR_DEVICE;
+}
+
+}  // extern "C"

@@ -1,0 +1,174 @@
+/*
+ * rglru.h -- C ABI of the B200 (sm_100a) RG-LRU recurrent-block library (librglru.so).
+ *
+ * The block, per batch row b, head h, channel ch = h * head_dim + j and token t:
+ *
+ *   xc_t  = conv_b + sum_{k=0..3} conv_w[k] * x~_{t-3+k}          causal depthwise conv
+ *   r_t   = sigmoid(xc_t(head) @ W_a[h] + b_a)                     recurrence gate
+ *   i_t   = sigmoid(xc_t(head) @ W_x[h] + b_x)                     input gate
+ *   log a_t = c * r_t * log sigmoid(Lambda)                        dynamic diagonal decay
+ *   h_t   = a_t * h_{t-1} + sqrt(1 - a_t^2) * (i_t * xc_t)          diagonal linear scan
+ *   out_t = h_t * GeLU(y_t)                                         multiplicative merge
+ *
+ * Sources ("Griffin Guide: RecurrentGemma, RG-LRU & Hybrid Attention"): the four governing
+ * equations and the log-space decay in "1. Formulation of the RG-LRU Gating Mechanism"; the
+ * sqrt(1 - a^2) factor in "2. The Role of Square-Root Variance Normalization"; the width-4
+ * depthwise conv before the RG-LRU in "1. Temporal Filtering via Separable 1D Convolutions";
+ * the GeLU merge in "2. Non-Linear Multiplicative Gating with GeLU"; per-head block-diagonal
+ * W_a / W_x in "3. Block-Diagonal Sharding for Zero-Communication Tensor Parallelism"; the
+ * conv padding (left K-1, truncated to T), the carried (y, last_state) and the zero initial
+ * state in the listing "1. PyTorch Implementation of RG-LRU and the Griffin Block"
+ * (RGLRU.forward / RGLRU.step / RecurrentBlock.forward).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library allocates no
+ *     memory, keeps no per-call state on the host and never synchronises unless stated.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) in
+ *     stream order; outputs are valid once the stream reaches that point.
+ *   - Arguments are validated on the host before anything is launched; on any error nothing
+ *     is launched and no output is touched.
+ *   - Layouts are row-major.  W = heads * head_dim.  Activations ("act dtype": fp32 or bf16)
+ *       x, y, out        [B, T, W]  (prefill)   /  [B, W]  (decode)
+ *       w_a, w_x         [heads, head_dim(in), head_dim(out)], act dtype:
+ *                        gate_o = b_o + sum_i xc_i * W[h][i][o]
+ *       conv_w           [4, W] fp32, tap-major, tap 3 multiplies the current token
+ *       conv_b, b_a, b_x [W] fp32, each may be NULL (= zeros)
+ *       lambda           [W] fp32 (a = sigmoid(lambda))
+ *       reset            [B, T] uint8 (prefill) / [B] (decode) or NULL; nonzero = that
+ *                        token starts a new segment (document): the conv history is emptied
+ *                        and h_{t-1} := 0 before the normal update
+ *       state.h          [B, W] fp32;  state.conv_tail [B, 3, W] act dtype: the last three
+ *                        x-branch inputs (pre-conv) of the current segment, oldest first
+ *   - x, y, out, w_a, w_x, conv_tail must be 16-byte aligned; fp32 parameter vectors and
+ *     state.h must be 4-byte aligned.  Outputs must not alias inputs (the state is in/out).
+ *   - Supported shapes: conv_width == 4; head_dim a multiple of 16 in [16, 256]; batch >= 1;
+ *     seq_len >= 1 (prefill); heads >= 1; W * sizeof(act) a multiple of 16.
+ *   - GeLU is exact, v * Phi(v), unless dims.gelu_tanh = 1 selects the tanh approximation.
+ *   - There is no CPU fallback: without a usable CUDA device every launching call returns
+ *     RGLRU_ERR_CUDA.
+ */
+#ifndef RGLRU_H
+#define RGLRU_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RGLRU_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define RGLRU_API __attribute__((visibility("default")))
+#else
+#define RGLRU_API
+#endif
+
+typedef enum { RGLRU_F32 = 0, RGLRU_BF16 = 1 } rglru_dtype;
+
+typedef enum {
+    RGLRU_OK = 0,
+    RGLRU_ERR_INVALID_ARG = 1,  /* NULL / misaligned pointer, non-positive size, bad enum */
+    RGLRU_ERR_UNSUPPORTED = 2,  /* valid but outside the supported shapes above */
+    RGLRU_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than the queried size */
+    RGLRU_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    RGLRU_ERR_TIMEOUT = 5,      /* device side: a bounded wait expired (see read_device_status) */
+    RGLRU_ERR_DEVICE = 6        /* device side: an internal consistency check failed */
+} rglru_status;
+
+/* Problem description.  `flags` is 0 in normal use; bit RGLRU_FLAG_GENERIC forces the
+ * portable (non-tensor-core) kernels, bit RGLRU_FLAG_TEST_WITHHOLD makes the fused prefill
+ * kernel withhold the carry of its first time chunk so that its successors' bounded waits
+ * expire (a test hook for the timeout path; results are then undefined). */
+typedef struct {
+    int batch;        /* B */
+    int seq_len;      /* T (prefill); ignored by decode */
+    int heads;        /* H */
+    int head_dim;     /* dh */
+    int conv_width;   /* must be 4 */
+    int act_dtype;    /* rglru_dtype of x, y, out, w_a, w_x, conv_tail */
+    float c;          /* decay scale c (8 on the pages) */
+    int gelu_tanh;    /* 0 = exact GeLU, 1 = tanh approximation */
+    unsigned flags;
+} rglru_dims;
+
+#define RGLRU_FLAG_GENERIC 1u
+#define RGLRU_FLAG_TEST_WITHHOLD 2u
+
+typedef struct {
+    const float* conv_w;  /* [4, W] */
+    const float* conv_b;  /* [W] or NULL */
+    const void* w_a;      /* [H, dh, dh] act dtype */
+    const void* w_x;      /* [H, dh, dh] act dtype */
+    const float* b_a;     /* [W] or NULL */
+    const float* b_x;     /* [W] or NULL */
+    const float* lambda;  /* [W] */
+} rglru_params;
+
+typedef struct {
+    float* h;          /* [B, W] fp32 */
+    void* conv_tail;   /* [B, 3, W] act dtype */
+} rglru_state;
+
+/* Zero-fills state->h and state->conv_tail (the listing's "no prev_state" start).
+ * Enqueued on `stream`.  Errors: INVALID_ARG (NULL/misaligned), CUDA. */
+RGLRU_API rglru_status rglru_state_init(const rglru_dims* dims, rglru_state* state, void* stream);
+
+/* Bytes of device workspace rglru_block_prefill needs for `dims` (0 on invalid dims).
+ * The workspace is scratch owned by the caller; it must be 256-byte aligned, it may be
+ * reused across calls on the same stream, and two calls in flight at once (on different
+ * streams) need different workspaces.  Its first 16 bytes hold the device status word. */
+RGLRU_API size_t rglru_prefill_workspace_size(const rglru_dims* dims);
+
+/* Full-sequence prefill: out = block(x, y) over T tokens for every row.
+ *   state == NULL: start from zero state, final state discarded.
+ *   state != NULL: start from *state, and overwrite *state with the state after token T-1
+ *                  (h_{T-1} and the last three x inputs of the final segment).
+ * Follows RGLRU.forward / RecurrentBlock.forward of the listing, with the conv's history
+ * taken from conv_tail instead of zero padding when a state is given.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA (host side, nothing launched).  Device
+ * side conditions (TIMEOUT, DEVICE) are latched in the workspace status word: read them
+ * with rglru_read_device_status. */
+RGLRU_API rglru_status rglru_block_prefill(const rglru_dims* dims, const rglru_params* params,
+                                 const void* x, const void* y, const uint8_t* reset,
+                                 rglru_state* state, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace rglru_block_decode needs (at least 16: the status word). */
+RGLRU_API size_t rglru_decode_workspace_size(const rglru_dims* dims);
+
+/* One single-token decode step for every row (RGLRU.step of the listing, plus the conv):
+ * conv over conv_tail[0..2] and x, gates, state update in place, out = h * GeLU(y), then the
+ * conv history shifts left by one and appends x.  reset[b] != 0 empties row b's state first.
+ * state is required (in/out).  dims.seq_len is ignored.  Errors as for prefill. */
+RGLRU_API rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_params* params,
+                                const void* x, const void* y, const uint8_t* reset,
+                                rglru_state* state, void* out,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* How a call with `dims` runs: *kernel receives RGLRU_KERNEL_GENERIC (CUDA-core kernels) or
+ * RGLRU_KERNEL_TENSOR (tcgen05 / TMEM kernels), *launches the number of kernel launches one
+ * call enqueues.  The choice depends on dims only (the library targets sm_100a alone).
+ * Errors: INVALID_ARG / UNSUPPORTED exactly as the corresponding call would return them. */
+#define RGLRU_KERNEL_GENERIC 0
+#define RGLRU_KERNEL_TENSOR 1
+RGLRU_API rglru_status rglru_prefill_plan(const rglru_dims* dims, int* kernel, int* launches);
+RGLRU_API rglru_status rglru_decode_plan(const rglru_dims* dims, int* kernel, int* launches);
+
+/* Synchronises `stream`, reads and clears the device status word at the start of
+ * `workspace`, and returns RGLRU_OK, RGLRU_ERR_TIMEOUT or RGLRU_ERR_DEVICE (or
+ * INVALID_ARG / CUDA for a bad argument or a failed copy). */
+RGLRU_API rglru_status rglru_read_device_status(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Static, human-readable name of a status code. */
+RGLRU_API const char* rglru_status_string(rglru_status status);
+
+/* RGLRU_ABI_VERSION of the built library. */
+RGLRU_API int rglru_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RGLRU_H */

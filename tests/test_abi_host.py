@@ -1,0 +1,113 @@
+"""Host-side checks of the C ABI (no GPU needed, nothing is launched).
+
+The library must load on a machine without a GPU, export every entry point that
+include/rglru.h declares, and reject bad arguments on the host with the documented codes.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_linear_recurrence_conv1d_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "rglru.h")).read()
+    return re.findall(r"RGLRU_API\s+[\w\s\*]+?\b(rglru_\w+)\s*\(", src)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = binding.load()
+    names = _declared()
+    assert len(names) >= 8
+    assert set(names) == set(binding.EXPORTED)
+    for n in names:
+        assert getattr(lib, n) is not None
+    assert lib.rglru_abi_version() == 1
+
+
+def test_status_strings():
+    lib = binding.load()
+    for code, name in binding.STATUS_NAMES.items():
+        assert lib.rglru_status_string(code).decode().startswith(name)
+    assert lib.rglru_status_string(99).decode() == "RGLRU_ERR_UNKNOWN"
+
+
+def _dims(**kw):
+    d = dict(batch=2, seq_len=16, heads=2, head_dim=64, act_dtype=binding.RGLRU_BF16)
+    d.update(kw)
+    return binding.make_dims(**d)
+
+
+def test_workspace_size_queries():
+    assert binding.prefill_workspace_size(_dims()) >= 16
+    assert binding.decode_workspace_size(_dims()) >= 16
+    assert binding.prefill_workspace_size(_dims(seq_len=0)) == 0
+    assert binding.prefill_workspace_size(_dims(head_dim=24)) == 0
+    d = _dims()
+    d.conv_width = 3
+    assert binding.prefill_workspace_size(d) == 0
+
+
+FAKE = 0x10000  # a 256-aligned non-null address: never dereferenced, validation fails first
+
+
+def _params(**over):
+    p = dict(conv_w=FAKE, conv_b=None, w_a=FAKE, w_x=FAKE, b_a=None, b_x=None, lambda_=FAKE)
+    p.update(over)
+    return binding.Params(*(ctypes.c_void_p(v) if v is not None else None for v in p.values()))
+
+
+def _prefill(d, p=None, x=FAKE, y=FAKE + 0x100, out=FAKE + 0x200, ws=FAKE, ws_bytes=1 << 20,
+             state=None):
+    lib = binding.load()
+    p = p or _params()
+    st = ctypes.byref(state) if state is not None else None
+    return lib.rglru_block_prefill(ctypes.byref(d), ctypes.byref(p), ctypes.c_void_p(x) if x else None,
+                                   ctypes.c_void_p(y) if y else None, None, st,
+                                   ctypes.c_void_p(out) if out else None,
+                                   ctypes.c_void_p(ws) if ws else None, ws_bytes, None)
+
+
+@pytest.mark.parametrize("case,code", [
+    (dict(batch=0), 1), (dict(seq_len=0), 1), (dict(heads=-1), 1), (dict(act_dtype=7), 1),
+    (dict(head_dim=24), 2), (dict(head_dim=512), 2), (dict(gelu_tanh=2), 1),
+])
+def test_bad_dims_are_rejected(case, code):
+    assert _prefill(_dims(**case)) == code
+
+
+def test_bad_pointers_are_rejected():
+    d = _dims()
+    assert _prefill(d, x=None) == 1
+    assert _prefill(d, x=FAKE + 2) == 1                      # misaligned activation
+    assert _prefill(d, out=FAKE) == 1                          # out aliases x
+    assert _prefill(d, p=_params(w_a=None)) == 1
+    assert _prefill(d, p=_params(w_x=FAKE + 8)) == 1          # gate weights need 16 B
+    assert _prefill(d, ws=None) == 3
+    assert _prefill(d, ws_bytes=8) == 3
+    assert _prefill(d, ws=FAKE + 16) == 1                     # workspace needs 256 B
+    st = binding.State(ctypes.c_void_p(FAKE), None)
+    assert _prefill(d, state=st) == 1
+    d.c = 0.0
+    assert _prefill(d) == 1
+
+
+def test_decode_requires_state():
+    lib = binding.load()
+    d = _dims(seq_len=1)
+    p = _params()
+    rc = lib.rglru_block_decode(ctypes.byref(d), ctypes.byref(p), ctypes.c_void_p(FAKE),
+                                ctypes.c_void_p(FAKE + 0x100), None, None,
+                                ctypes.c_void_p(FAKE + 0x200), ctypes.c_void_p(FAKE), 1 << 20, None)
+    assert rc == 1
+
+
+def test_read_status_rejects_bad_workspace():
+    lib = binding.load()
+    assert lib.rglru_read_device_status(None, 256, None) == 1
+    assert lib.rglru_read_device_status(ctypes.c_void_p(FAKE + 4), 256, None) == 1
