@@ -17,6 +17,8 @@ import torch
 from . import build as _build
 
 RGLRU_OK = 0
+RGLRU_ERR_TIMEOUT = 5
+RGLRU_ERR_DEVICE = 6
 RGLRU_F32, RGLRU_BF16 = 0, 1
 FLAG_GENERIC = 1
 FLAG_TEST_WITHHOLD = 2

@@ -103,6 +103,7 @@ rglru_status rglru_state_init(const rglru_dims* dims, rglru_state* state, void* 
 
 size_t rglru_prefill_workspace_size(const rglru_dims* dims) {
     if (check_dims(dims, true) != RGLRU_OK) return 0;
+    if (rglru::fused_prefill_supported(dims)) return rglru::fused_prefill_workspace(dims);
     return kStatusBytes;
 }
 
@@ -123,6 +124,9 @@ rglru_status rglru_block_prefill(const rglru_dims* dims, const rglru_params* par
     if ((st = check_workspace(workspace, workspace_bytes, rglru_prefill_workspace_size(dims))) != RGLRU_OK)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (rglru::fused_prefill_supported(dims))
+        return cuda_status(rglru::launch_fused_prefill(dims, params, x, y, reset, state, out, workspace,
+                                                       workspace_bytes, s));
     return cuda_status(rglru::launch_prefill_generic(dims, params, x, y, reset, state, out, s));
 }
 
@@ -145,8 +149,9 @@ rglru_status rglru_prefill_plan(const rglru_dims* dims, int* kernel, int* launch
     rglru_status st = check_dims(dims, true);
     if (st != RGLRU_OK) return st;
     if (!kernel || !launches) return RGLRU_ERR_INVALID_ARG;
-    *kernel = RGLRU_KERNEL_GENERIC;
-    *launches = 1;
+    const bool tc = rglru::fused_prefill_supported(dims);
+    *kernel = tc ? RGLRU_KERNEL_TENSOR : RGLRU_KERNEL_GENERIC;
+    *launches = tc ? rglru::fused_prefill_launches(dims) : 1;
     return RGLRU_OK;
 }
 

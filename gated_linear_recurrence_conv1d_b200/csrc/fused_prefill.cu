@@ -1,0 +1,856 @@
+// fused_prefill.cu -- tensor-core RG-LRU prefill for bf16 activations, head_dim 256 (sm_100a).
+//
+// One kernel does the whole block (conv -> gates -> decay -> scan -> GeLU merge -> state):
+//
+//   * a persistent CTA owns one (head, 128-channel half) "group" for its whole life; its
+//     block-diagonal gate weights W_a[h][:, half], W_x[h][:, half] are written once into
+//     tensor memory (TMEM) and used as the A operand of tcgen05.mma (TS form), so shared
+//     memory only holds streamed tiles;
+//   * work items are (batch row, 64-token chunk) of the group, handed out by a per-group
+//     atomic ticket so every CTA of a group stays busy and an item's predecessor is always
+//     held by a running CTA;
+//   * warp roles: an x producer (TMA: x tile with a 3-token halo, and the ticket), a y producer
+//     (TMA: y tile, issued once the previous out store of that stage has left shared memory),
+//     8 conv warps (causal width-4 depthwise conv in fp32, written as the bf16 B operand in the
+//     128-byte swizzled K-major layout), 1 MMA thread (gates^T[128 ch x 64 tok] = W^T . xc^T for
+//     both gates, K = 256 in 16 steps, fp32 accumulators in TMEM), and 2 epilogue groups of 4
+//     warps, group g owning TMEM stage g, so one group's look-back wait overlaps the other
+//     group's math;
+//   * transposed orientation: a TMEM lane is an output channel and the 64 columns are tokens,
+//     so an epilogue thread owns one channel and runs the diagonal scan along its registers
+//     (no shuffles);
+//   * chunks of one sequence handled by different CTAs chain through a look-back in the spirit
+//     of Merrill & Garland ("Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016):
+//     after its first pass a chunk publishes its aggregate (prod a, local h) per channel; its
+//     carry is the inclusive state of an anchor chunk (every 32nd chunk of the row) followed by
+//     the aggregates of the chunks in between, applied in a fixed order so the result does not
+//     depend on timing; it then publishes its own inclusive state and replays the scan from
+//     TMEM with the true carry.  Every wait is bounded by %globaltimer; on expiry the kernel
+//     latches RGLRU_ERR_TIMEOUT in the workspace status word and drains.
+//
+// Arithmetic follows "Griffin Guide: RecurrentGemma, RG-LRU & Hybrid Attention": recurrence /
+// input gates, a_t = a^(c r_t) in log space, h_t = a_t h_{t-1} + sqrt(1 - a_t^2)(i_t x_t)
+// ("1. Formulation of the RG-LRU Gating Mechanism"), the width-4 conv before the RG-LRU and
+// the GeLU merge ("1. Temporal Filtering via Separable 1D Convolutions", "2. Non-Linear
+// Multiplicative Gating with GeLU"), per-head block-diagonal gates ("3. Block-Diagonal
+// Sharding for Zero-Communication Tensor Parallelism").  The conv output feeding the MMA and
+// the i_t * x_t product is rounded to bf16 (the tensor-core operand); state and all
+// element-wise math stay in fp32.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace rglru {
+namespace tc {
+
+using namespace sm100;
+
+constexpr int DH = 256;                 // head dim (K of the gate contraction)
+constexpr int HALF = 128;               // output channels per CTA (= TMEM lanes = MMA M)
+constexpr int L = 64;                   // tokens per chunk (= MMA N)
+constexpr int LH = L / 2;               // tokens per conv warp
+constexpr int XROWS = L + kHist;        // x tile rows incl. the 3-token halo
+constexpr int KSTEPS = DH / 16;         // MMA K steps
+constexpr int STAGES = 2;
+constexpr int SLOTS = 8;                // ring of item ids, indexed by iteration
+constexpr int kSub = 8;                 // tokens per TMEM load in the epilogue
+
+// warp roles: 0-7 conv (K block = warp % 4, token half = warp / 4), 8-15 epilogue (TMEM lane
+// quarter = warp % 4, group = stage = (warp - 8) / 4), 16 x producer, 17 y producer, 18 MMA.
+constexpr int kConvWarps = 8, kEpiWarps = 8, kEpiGroup = 4;
+constexpr int kWarpEpi0 = 8, kWarpProdX = 16, kWarpProdY = 17, kWarpMma = 18;
+constexpr int kThreads = 19 * 32;
+
+constexpr uint32_t X_BYTES = XROWS * DH * 2;      // 34304
+constexpr uint32_t Y_BYTES = L * HALF * 2;        // 16384
+constexpr uint32_t B_BYTES = L * DH * 2;          // 32768 (4 K-blocks of L x 128 B)
+constexpr uint32_t KBLK_BYTES = L * 128;          // one 64-wide K block
+
+// shared memory map (offsets from a 1024-aligned base)
+constexpr uint32_t OFF_B = 0;                                   // STAGES x B_BYTES
+constexpr uint32_t OFF_X = OFF_B + STAGES * B_BYTES;            // STAGES x X_BYTES
+constexpr uint32_t OFF_Y = OFF_X + STAGES * X_BYTES;            // STAGES x Y_BYTES
+constexpr uint32_t OFF_BAR = OFF_Y + STAGES * Y_BYTES;
+constexpr int NBAR = 9 * STAGES + 2;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;               // slots, TMEM base, abort flag
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;          // + slack for 1024 alignment
+static_assert(2 * HALF * DH * 2 <= OFF_Y, "weight staging reuses the B and x tiles");
+
+// TMEM columns: [0,128) A = W_a^T (bf16 pairs), [128,256) A = W_x^T, then per stage
+// 128 columns: gate a accumulators [0,64) and gate x accumulators [64,128).
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_A = 0, TM_D = 256;
+
+constexpr unsigned FLAG_AGG = 1, FLAG_INCL = 2;
+constexpr int LBW = 32;                 // look-back block: anchors every LBW chunks
+
+struct Args {
+    int B, T, H, NC, items;          // items = B * NC per group
+    int groups;                      // 2 * H
+    int base, extra;                 // CTAs per group: base (+1 for the first `extra` groups)
+    float c;
+    int gelu_tanh;
+    unsigned flags;
+    unsigned long long timeout_ns;
+    const float* conv_w;
+    const float* conv_b;
+    const __nv_bfloat16* w_a;
+    const __nv_bfloat16* w_x;
+    const float* b_a;
+    const float* b_x;
+    const float* lambda;
+    const uint8_t* reset;
+    float* h_state;                  // nullptr: zero initial state, no write-back
+    __nv_bfloat16* tail_state;
+    DeviceStatus* status;
+    unsigned* counters;              // [groups] tickets
+    unsigned* lb_flags;              // [groups][items][4]
+    float2* lb_agg;                  // [groups][items][128]
+    float* lb_incl;                  // [groups][items][128]
+};
+
+struct Bars {
+    uint32_t x_full[STAGES], x_empty[STAGES], y_full[STAGES], y_empty[STAGES], b_full[STAGES],
+        b_empty[STAGES], acc_full[STAGES], acc_empty[STAGES], out_ready[STAGES], w_ready, mma_done;
+};
+
+__device__ __forceinline__ Bars make_bars(uint32_t base) {
+    Bars b;
+    uint32_t o = base;
+    auto next = [&]() { uint32_t r = o; o += 8; return r; };
+    for (int s = 0; s < STAGES; ++s) {
+        b.x_full[s] = next(); b.x_empty[s] = next(); b.y_full[s] = next(); b.y_empty[s] = next();
+        b.b_full[s] = next(); b.b_empty[s] = next(); b.acc_full[s] = next(); b.acc_empty[s] = next();
+        b.out_ready[s] = next();
+    }
+    b.w_ready = next();
+    b.mma_done = next();
+    return b;
+}
+
+// Context of the bounded waits: they give up after timeout_ns, or as soon as another thread of
+// the grid has latched a failure, so that every role drains instead of hanging.
+struct WaitCtx {
+    DeviceStatus* status;
+    unsigned long long timeout_ns;
+    volatile int* abort;
+};
+
+__device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, WaitCtx w, unsigned where) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 255) == 0) {
+            if (*w.abort) return false;
+            if (*(volatile unsigned*)&w.status->code != 0) {
+                *w.abort = 1;
+                return false;
+            }
+            if (globaltimer_ns() - t0 > w.timeout_ns) {
+                latch_status(w.status, RGLRU_ERR_TIMEOUT, where, blockIdx.x, parity);
+                *w.abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, WaitCtx w, unsigned where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bar_slow(bar, parity, w, where);
+}
+
+// Bounded wait for a look-back flag to reach at least `want`; returns the flag (0 on failure).
+__device__ __noinline__ unsigned wait_flag(const unsigned* f, unsigned want, WaitCtx w, unsigned where) {
+    unsigned v = ld_acquire_gpu(f);
+    if (v >= want) return v;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(20);
+        v = ld_acquire_gpu(f);
+        if (v >= want) return v;
+        if ((i & 63) == 0) {
+            if (*w.abort || *(volatile unsigned*)&w.status->code != 0) {
+                *w.abort = 1;
+                return 0;
+            }
+            if (globaltimer_ns() - t0 > w.timeout_ns) {
+                latch_status(w.status, RGLRU_ERR_TIMEOUT, where, blockIdx.x, 0);
+                *w.abort = 1;
+                return 0;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t b_tile_offset(int t, int k) {
+    // element (token t, channel k) of the 128-byte swizzled K-major B tile
+    const int kb = k >> 6, kk = k & 63;
+    const int chunk = (kk >> 3) ^ (t & 7);
+    return kb * KBLK_BYTES + (t >> 3) * 1024 + (t & 7) * 128 + chunk * 16 + (kk & 7) * 2;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&p);
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float rsqrt_approx(float x) {
+    float r;
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// sigma(z) = 1 / (1 + 2^(-z log2 e)) with the ex2 / rcp approximations: relative error of a
+// few ulp over the whole range (the recurrence gate needs it: sqrt(1 - a^2) ~ sqrt(r) for
+// small r).
+__device__ __forceinline__ float sigmoid_fast(float z) {
+    return rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * z));
+}
+// sigma(z) = (1 + tanh(z / 2)) / 2: absolute error ~2.5e-4, enough for the input gate, whose
+// error enters h only additively through i_t x_t.
+__device__ __forceinline__ float sigmoid_tanh(float z) {
+    return fmaf(0.5f, tanh_approx(0.5f * z), 0.5f);
+}
+
+// Decay a = e^l and sqrt(1 - a^2) for l = c r log sigma(Lambda) <= 0.  When the channel's
+// |c log sigma(Lambda)| <= 1/8 (so |l| <= 1/8): em = expm1(l) from its Taylor series (terms
+// l^k / k!, truncation below 1e-8 relative), a = 1 + em, 1 - a^2 = -em (2 + em) without
+// cancellation.  Otherwise a = 2^(l log2 e) and 1 - a^2 directly, switching to the series when
+// |l| < 1/8.
+__device__ __forceinline__ void decay_beta(float l, bool small_range, float& a, float& beta) {
+    float v;
+    if (small_range || l > -0.125f) {
+        float p = fmaf(l, 1.0f / 720.0f, 1.0f / 120.0f);
+        p = fmaf(l, p, 1.0f / 24.0f);
+        p = fmaf(l, p, 1.0f / 6.0f);
+        p = fmaf(l, p, 0.5f);
+        p = fmaf(l, p, 1.0f);
+        const float em = l * p;
+        a = 1.0f + em;
+        v = -em * (2.0f + em);
+    } else {
+        a = ex2_approx(l * 1.4426950408889634f);
+        v = fmaf(-a, a, 1.0f);
+    }
+    beta = v > 0.0f ? v * rsqrt_approx(v) : 0.0f;
+}
+
+// GeLU(v) = v Phi(v).  Exact form: Phi from erf of Abramowitz & Stegun 7.1.28,
+// erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 for x >= 0 (|error| <= 3e-7), one reciprocal.
+// Tanh form: 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))).
+__device__ __forceinline__ float gelu_fast(float v, int tanh_form) {
+    if (tanh_form) {
+        const float k = 0.79788456080286535588f;
+        return 0.5f * v * (1.0f + tanh_approx(k * fmaf(0.044715f * v, v * v, v)));
+    }
+    const float x = fabsf(v) * 0.70710678118654752f;
+    float p = fmaf(x, 0.0000430638f, 0.0002765672f);
+    p = fmaf(x, p, 0.0001520143f);
+    p = fmaf(x, p, 0.0092705272f);
+    p = fmaf(x, p, 0.0422820123f);
+    p = fmaf(x, p, 0.0705230784f);
+    p = fmaf(x, p, 1.0f);
+    p = p * p;
+    p = p * p;
+    p = p * p;
+    p = p * p;                                        // (1 + ...)^16
+    const float half_erfc = 0.5f * rcp_approx(p);     // (1 - erf(x)) / 2
+    return v * (v >= 0.0f ? 1.0f - half_erfc : half_erfc);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_y,
+                     const __grid_constant__ CUtensorMap map_out, const Args a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const Bars bars = make_bars(sbase + OFF_BAR);
+    volatile int* slot = reinterpret_cast<volatile int*>(smem + OFF_MISC);        // [SLOTS]
+    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 32);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 48);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- group of this CTA -----------------------------------------------------------------
+    int group;
+    {
+        const int cta = blockIdx.x, big = a.extra * (a.base + 1);
+        group = cta < big ? cta / (a.base + 1) : a.extra + (cta - big) / a.base;
+    }
+    const int head = group >> 1, half = group & 1;
+    const int W = a.H * DH;
+    const size_t lb_base = (size_t)group * a.items;
+
+    // ---- set-up ------------------------------------------------------------------------------
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bars.x_full[s], 1);
+            mbar_init(bars.x_empty[s], kConvWarps);
+            mbar_init(bars.y_full[s], 1);
+            mbar_init(bars.y_empty[s], 1);
+            mbar_init(bars.b_full[s], kConvWarps);
+            mbar_init(bars.b_empty[s], 1 + kEpiGroup);
+            mbar_init(bars.acc_full[s], 1);
+            mbar_init(bars.acc_empty[s], kEpiGroup);
+            mbar_init(bars.out_ready[s], kEpiGroup);
+        }
+        mbar_init(bars.w_ready, kEpiWarps);
+        mbar_init(bars.mma_done, 1);
+        *abort = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32((const void*)tmem_base_s), TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == kWarpProdX && lane == 0) {
+        prefetch_tensormap(&map_x);
+        prefetch_tensormap(&map_y);
+        prefetch_tensormap(&map_out);
+    }
+    // stage this CTA's gate weights W_g[head][i][half*128 + o] (o contiguous) in shared memory
+    // with coalesced 16-byte loads: gate a at byte 0, gate x at byte 65536 (B and x tiles are
+    // still unused)
+    if (warp < kConvWarps + kEpiWarps) {
+        const int tid = threadIdx.x;                       // 0..511
+        for (int e = tid; e < 2 * DH * (HALF / 8); e += (kConvWarps + kEpiWarps) * 32) {
+            const int g = e / (DH * (HALF / 8)), r = e % (DH * (HALF / 8));
+            const int i = r / (HALF / 8), o8 = r % (HALF / 8);
+            const __nv_bfloat16* src = (g ? a.w_x : a.w_a) + ((size_t)head * DH + i) * DH + half * HALF + o8 * 8;
+            *reinterpret_cast<uint4*>(smem + g * (HALF * DH * 2) + (i * HALF + o8 * 8) * 2) =
+                __ldg(reinterpret_cast<const uint4*>(src));
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_s;
+    const WaitCtx wc{a.status, a.timeout_ns, abort};
+
+    if (warp >= kWarpEpi0 && warp < kWarpEpi0 + kEpiWarps) {
+        // weights -> TMEM A operand: lane m, column j holds (W[2j][m], W[2j+1][m]); group 0 of
+        // each lane quarter writes gate a, group 1 gate x
+        const int q = warp & 3, g = (warp - kWarpEpi0) >> 2, m = q * 32 + lane;
+        const unsigned short* ws = reinterpret_cast<const unsigned short*>(smem + g * (HALF * DH * 2)) + m;
+#pragma unroll 1
+        for (int j0 = 0; j0 < DH / 2; j0 += 16) {
+            uint32_t r[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int i = 2 * (j0 + j);
+                r[j] = (uint32_t)ws[i * HALF] | ((uint32_t)ws[(i + 1) * HALF] << 16);
+            }
+            tmem_st16(tmem + ((uint32_t)(q * 32) << 16) + TM_A + g * 128 + j0, r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.w_ready);
+    }
+    __syncthreads();   // the staging area is free again before any TMA load lands in it
+
+    if (warp == kWarpProdX) {
+        // ================================ x producer (and tickets) ============================
+        if (lane == 0) {
+            int issued[STAGES] = {0, 0};
+            for (int n = 0;; ++n) {
+                const int st = n & 1;
+                const uint32_t ph = (n >> 1) & 1;
+                if (!wait_bar(bars.x_empty[st], ph ^ 1, wc, 1)) break;
+                int k = (int)atomicAdd(&a.counters[group], 1u);
+                if (k >= a.items) {
+                    slot[n & (SLOTS - 1)] = -1;            // terminal item for the stage-n group
+                    slot[(n + 1) & (SLOTS - 1)] = -1;      // ... and for the other group
+                    mbar_arrive(bars.x_full[st]);
+                    issued[st] = 0;   // that phase completing implies the earlier load landed
+                    break;
+                }
+                slot[n & (SLOTS - 1)] = k;
+                const int b = k / a.NC, c = k % a.NC;
+                mbar_arrive_expect_tx(bars.x_full[st], X_BYTES);
+                tma_load_3d(sbase + OFF_X + st * X_BYTES, &map_x, head * DH, c * L - kHist, b,
+                            bars.x_full[st]);
+                issued[st] = n + 1;
+            }
+            // never leave the CTA with a bulk copy still writing its shared memory
+            for (int st = 0; st < STAGES; ++st)
+                if (issued[st]) {
+                    const int n = issued[st] - 1;
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(bars.x_full[st], (n >> 1) & 1) &&
+                           globaltimer_ns() - t0 < a.timeout_ns) {
+                    }
+                }
+        }
+    } else if (warp == kWarpProdY) {
+        // ================================ y producer ==========================================
+        if (lane == 0) {
+            int issued[STAGES] = {0, 0};
+            for (int n = 0;; ++n) {
+                const int st = n & 1;
+                const uint32_t ph = (n >> 1) & 1;
+                // b_full (the conv warps arrive after reading item n's slot, which the x producer
+                // wrote before x_full) orders the slot read for this thread too
+                if (!wait_bar(bars.b_full[st], ph, wc, 15)) break;
+                const int k = slot[n & (SLOTS - 1)];
+                if (!wait_bar(bars.y_empty[st], ph ^ 1, wc, 2)) break;
+                if (k < 0) {
+                    mbar_arrive(bars.y_full[st]);
+                    issued[st] = 0;
+                    break;
+                }
+                const int b = k / a.NC, c = k % a.NC;
+                mbar_arrive_expect_tx(bars.y_full[st], Y_BYTES);
+                tma_load_3d(sbase + OFF_Y + st * Y_BYTES, &map_y, head * DH + half * HALF, c * L, b,
+                            bars.y_full[st]);
+                issued[st] = n + 1;
+            }
+            for (int st = 0; st < STAGES; ++st)
+                if (issued[st]) {
+                    const int n = issued[st] - 1;
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(bars.y_full[st], (n >> 1) & 1) &&
+                           globaltimer_ns() - t0 < a.timeout_ns) {
+                    }
+                }
+        }
+    } else if (warp == kWarpMma) {
+        // ================================ MMA issuer ===========================================
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(HALF, L);
+            bool ok = wait_bar(bars.w_ready, 0, wc, 3);
+            tc_fence_after();
+            for (int n = 0; ok; ++n) {
+                const int st = n & 1;
+                const uint32_t ph = (n >> 1) & 1;
+                if (!wait_bar(bars.b_full[st], ph, wc, 4)) break;
+                if (!wait_bar(bars.acc_empty[st], ph ^ 1, wc, 5)) break;
+                if (slot[n & (SLOTS - 1)] < 0) {
+                    // hand the terminal item to both epilogue groups: group st now, group st^1
+                    // once it has released its previous item (so that no phase is skipped)
+                    mbar_arrive(bars.acc_full[st]);
+                    const uint32_t ph1 = ((n + 1) >> 1) & 1;
+                    if (wait_bar(bars.acc_empty[st ^ 1], ph1 ^ 1, wc, 17)) mbar_arrive(bars.acc_full[st ^ 1]);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t bt = sbase + OFF_B + st * B_BYTES;
+#pragma unroll 1
+                for (int g = 0; g < 2; ++g) {
+                    const uint32_t d = tmem + TM_D + st * 128 + g * L;
+#pragma unroll
+                    for (int ks = 0; ks < KSTEPS; ++ks) {
+                        const uint64_t bd = desc_k_sw128(bt + (ks >> 2) * KBLK_BYTES + (ks & 3) * 32);
+                        mma_ts(d, tmem + TM_A + g * 128 + ks * 8, bd, idesc, ks > 0 ? 1u : 0u);
+                    }
+                }
+                mma_commit(bars.acc_full[st]);
+                mma_commit(bars.b_empty[st]);
+            }
+            // every MMA this thread issued has finished before TMEM is released
+            mma_commit(bars.mma_done);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(bars.mma_done, 0) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+        }
+    } else if (warp < kConvWarps) {
+        // ================================ conv warps ==========================================
+        const int kb = warp & 3, th = warp >> 2;          // K block, token half
+        const int p = kb * 32 + lane;                     // channel pair 2p, 2p+1 of the head
+        const int chg = head * DH + 2 * p;                // global channel of the pair
+        float w0[kConvWidth], w1[kConvWidth];
+#pragma unroll
+        for (int k = 0; k < kConvWidth; ++k) {
+            w0[k] = a.conv_w[(size_t)k * W + chg];
+            w1[k] = a.conv_w[(size_t)k * W + chg + 1];
+        }
+        const float cb0 = a.conv_b ? a.conv_b[chg] : 0.f;
+        const float cb1 = a.conv_b ? a.conv_b[chg + 1] : 0.f;
+        const bool own_tail = (p >> 6) == half;          // this CTA writes these tail channels
+        for (int n = 0;; ++n) {
+            const int st = n & 1;
+            const uint32_t ph = (n >> 1) & 1;
+            if (!wait_bar(bars.x_full[st], ph, wc, 6)) break;
+            if (!wait_bar(bars.b_empty[st], ph ^ 1, wc, 7)) break;
+            const int k = slot[n & (SLOTS - 1)];
+            if (k < 0) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars.b_full[st]);
+                break;
+            }
+            const int b = k / a.NC, c = k % a.NC, t0 = c * L;
+            const int nt = min(L, a.T - t0);
+            const int tb = th * LH;                        // first token of this warp's half
+            const int ts = t0 + tb;                        // its sequence position
+            const uint8_t* rst = a.reset ? a.reset + (size_t)b * a.T : nullptr;
+            const uint8_t* xt = smem + OFF_X + st * X_BYTES + 4 * p;
+            uint8_t* bt = smem + OFF_B + st * B_BYTES;
+            float h0a, h1a, h2a, h0b, h1b, h2b;          // window x_{t-3}, x_{t-2}, x_{t-1}
+            if (ts == 0) {
+                if (a.tail_state) {
+                    const __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
+                    uint32_t v0 = *reinterpret_cast<const uint32_t*>(tl);
+                    uint32_t v1 = *reinterpret_cast<const uint32_t*>(tl + W);
+                    uint32_t v2 = *reinterpret_cast<const uint32_t*>(tl + 2 * W);
+                    h0a = bf16lo(v0); h0b = bf16hi(v0);
+                    h1a = bf16lo(v1); h1b = bf16hi(v1);
+                    h2a = bf16lo(v2); h2b = bf16hi(v2);
+                } else {
+                    h0a = h1a = h2a = h0b = h1b = h2b = 0.f;
+                }
+            } else {
+                uint32_t v0 = *reinterpret_cast<const uint32_t*>(xt + (tb + 0) * DH * 2);
+                uint32_t v1 = *reinterpret_cast<const uint32_t*>(xt + (tb + 1) * DH * 2);
+                uint32_t v2 = *reinterpret_cast<const uint32_t*>(xt + (tb + 2) * DH * 2);
+                h0a = bf16lo(v0); h0b = bf16hi(v0);
+                h1a = bf16lo(v1); h1b = bf16hi(v1);
+                h2a = bf16lo(v2); h2b = bf16hi(v2);
+                if (rst && ts < a.T) {
+                    if (rst[ts - 1]) { h0a = h0b = h1a = h1b = 0.f; }
+                    if (rst[ts - 2]) { h0a = h0b = 0.f; }
+                }
+            }
+            float ta0 = 0.f, ta1 = 0.f, ta2 = 0.f, tb0 = 0.f, tb1 = 0.f, tb2 = 0.f;   // final window
+#pragma unroll 8
+            for (int j = 0; j < LH; ++j) {
+                const int t = tb + j;
+                const uint32_t v = *reinterpret_cast<const uint32_t*>(xt + (t + kHist) * DH * 2);
+                const float xa = bf16lo(v), xb = bf16hi(v);
+                if (rst && t < nt && rst[t0 + t]) { h0a = h1a = h2a = h0b = h1b = h2b = 0.f; }
+                float ya = fmaf(w0[3], xa, fmaf(w0[2], h2a, fmaf(w0[1], h1a, fmaf(w0[0], h0a, cb0))));
+                float yb = fmaf(w1[3], xb, fmaf(w1[2], h2b, fmaf(w1[1], h1b, fmaf(w1[0], h0b, cb1))));
+                *reinterpret_cast<uint32_t*>(bt + b_tile_offset(t, 2 * p)) = pack_bf16x2(ya, yb);
+                h0a = h1a; h1a = h2a; h2a = xa;
+                h0b = h1b; h1b = h2b; h2b = xb;
+                if (t == nt - 1) { ta0 = h0a; ta1 = h1a; ta2 = h2a; tb0 = h0b; tb1 = h1b; tb2 = h2b; }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bars.x_empty[st]);
+                mbar_arrive(bars.b_full[st]);
+            }
+            // final conv history of the sequence, once its first chunk has read the old one
+            if (a.tail_state && c == a.NC - 1 && own_tail && nt - 1 >= tb && nt - 1 < tb + LH) {
+                bool ok = true;
+                if (c > 0) ok = wait_flag(a.lb_flags + (lb_base + (size_t)b * a.NC) * 4, FLAG_AGG, wc, 8) != 0;
+                if (ok) {
+                    __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
+                    *reinterpret_cast<uint32_t*>(tl) = pack_bf16x2(ta0, tb0);
+                    *reinterpret_cast<uint32_t*>(tl + W) = pack_bf16x2(ta1, tb1);
+                    *reinterpret_cast<uint32_t*>(tl + 2 * W) = pack_bf16x2(ta2, tb2);
+                }
+            }
+        }
+    } else if (warp < kWarpEpi0 + kEpiWarps) {
+        // ================================ epilogue groups ======================================
+        const int q = warp & 3;                          // TMEM lane quarter
+        const int eg = (warp - kWarpEpi0) >> 2;          // group = TMEM stage it owns
+        const int st = eg;
+        const int m = q * 32 + lane;                     // local output channel = TMEM lane
+        const int chl = half * HALF + m;                 // channel within the head
+        const int ch = head * DH + chl;                  // global channel
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const float lab = log_sigmoid_acc(a.lambda[ch]);
+        const float c_lab = a.c * lab;                   // log a_t = c_lab * r_t
+        const bool small_range = c_lab >= -0.125f;
+        const float ba = a.b_a ? a.b_a[ch] : 0.f;
+        const float bx = a.b_x ? a.b_x[ch] : 0.f;
+        const int tanh_form = a.gelu_tanh;
+        const bool withhold_hook = (a.flags & RGLRU_FLAG_TEST_WITHHOLD) && group == 0;
+        const uint8_t* bt = smem + OFF_B + st * B_BYTES;
+        uint8_t* yt = smem + OFF_Y + st * Y_BYTES + 2 * m;
+        const uint32_t dcol = tmem + lane_off + TM_D + st * 128;
+
+        for (int n = eg;; n += 2) {
+            const uint32_t ph = (n >> 1) & 1;
+            if (!wait_bar(bars.acc_full[st], ph, wc, 9)) break;
+            const int k = slot[n & (SLOTS - 1)];
+            if (k < 0) break;
+            tc_fence_after();
+            const int b = k / a.NC, c = k % a.NC, t0 = c * L;
+            const int nt = min(L, a.T - t0);
+            const uint8_t* rst = a.reset ? a.reset + (size_t)b * a.T + t0 : nullptr;
+            const size_t kb_item = lb_base + (size_t)b * a.NC;       // first chunk of this row
+            const bool withhold = withhold_hook && k == 0;
+            unsigned* myflag = a.lb_flags + (lb_base + k) * 4 + q;
+
+            // ---- pass 1: gates, decay and normalised input of the chunk -> TMEM (a, u)
+            float aggA = 1.f, aggH = 0.f;
+#pragma unroll 1
+            for (int j0 = 0; j0 < L; j0 += kSub) {
+                float ga[kSub], gx[kSub];
+                tmem_ld8(dcol + j0, ga);
+                tmem_ld8(dcol + L + j0, gx);
+                tmem_wait_ld();
+                uint32_t ra[kSub], ru[kSub];
+#pragma unroll
+                for (int j = 0; j < kSub; ++j) {
+                    const int t = j0 + j;
+                    const float xc = __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(
+                                                         bt + b_tile_offset(t, chl)) << 16);
+                    const float r = sigmoid_fast(ga[j] + ba);
+                    float at, beta;
+                    decay_beta(c_lab * r, small_range, at, beta);
+                    const float ig = sigmoid_tanh(gx[j] + bx);
+                    float u = beta * (ig * xc);
+                    if (rst && t < nt && rst[t]) at = 0.f;                // h_{t-1} := 0
+                    if (t >= nt) { at = 1.f; u = 0.f; }                   // padding: identity
+                    aggH = fmaf(at, aggH, u);
+                    aggA *= at;
+                    ra[j] = __float_as_uint(at);
+                    ru[j] = __float_as_uint(u);
+                }
+                tmem_st8(dcol + j0, ra);
+                tmem_st8(dcol + L + j0, ru);
+            }
+            // the B tile (xc) is no longer read by this warp
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.b_empty[st]);
+            if (c > 0 && !withhold) {                    // chunk aggregate, as early as possible
+                a.lb_agg[(lb_base + k) * HALF + m] = make_float2(aggA, aggH);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_gpu(myflag, FLAG_AGG);
+            }
+
+            // ---- carry: initial state for the first chunk, else the look-back
+            float carry = 0.f;
+            if (c == 0) {
+                carry = a.h_state ? a.h_state[(size_t)b * W + ch] : 0.f;
+            } else {
+                // fixed association, so results do not depend on timing: the anchor is the
+                // nearest earlier chunk whose index is a multiple of LBW; carry = the anchor's
+                // inclusive state, then the aggregates of the chunks in between, in order
+                const int anc = ((c - 1) / LBW) * LBW;
+                const int nagg = c - 1 - anc;                       // < LBW <= 32
+                const unsigned* fa = a.lb_flags + (kb_item + anc) * 4 + q;
+                const bool mine = lane < nagg;
+                const unsigned* fl = fa + (size_t)(lane + 1) * 4;
+                const uint64_t tw = globaltimer_ns();
+                bool ready = false;
+                for (uint32_t it = 0;; ++it) {
+                    bool okl = mine ? ld_acquire_gpu(fl) >= FLAG_AGG : true;
+                    if (lane == 0) okl = okl && ld_acquire_gpu(fa) >= FLAG_INCL;
+                    if (__all_sync(0xffffffffu, okl)) { ready = true; break; }
+                    __nanosleep(20);
+                    if ((it & 63) == 63) {
+                        int give_up = 0;
+                        if (lane == 0) {
+                            if (*abort || *(volatile unsigned*)&a.status->code != 0) give_up = 1;
+                            else if (globaltimer_ns() - tw > a.timeout_ns) {
+                                latch_status(a.status, RGLRU_ERR_TIMEOUT, 10, blockIdx.x, (unsigned)k);
+                                give_up = 1;
+                            }
+                            if (give_up) *abort = 1;
+                        }
+                        if (__shfl_sync(0xffffffffu, give_up, 0)) break;
+                    }
+                }
+                if (ready) {
+                    float hc = __ldcg(a.lb_incl + (kb_item + anc) * HALF + m);
+                    for (int i = 0; i < nagg; ++i) {
+                        const float2 g = __ldcg(a.lb_agg + (kb_item + anc + 1 + i) * HALF + m);
+                        hc = fmaf(g.x, hc, g.y);
+                    }
+                    carry = hc;
+                }
+            }
+            const float incl = fmaf(aggA, carry, aggH);             // state after the chunk
+            if (!withhold) {
+                a.lb_incl[(lb_base + k) * HALF + m] = incl;
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release_gpu(myflag, FLAG_INCL);
+            }
+            // final state of the row, once its first chunk has read the old one
+            if (a.h_state && c == a.NC - 1) {
+                bool okw = true;
+                if (c > 0) {
+                    unsigned f = 0;
+                    if (lane == 0) f = wait_flag(a.lb_flags + kb_item * 4 + q, FLAG_INCL, wc, 11);
+                    okw = __shfl_sync(0xffffffffu, f, 0) != 0;
+                }
+                if (okw) a.h_state[(size_t)b * W + ch] = incl;
+            }
+
+            // ---- pass 2: replay the scan from TMEM, merge with GeLU(y)
+            if (!wait_bar(bars.y_full[st], ph, wc, 16)) break;
+            tmem_wait_st();
+            float h = carry;
+#pragma unroll 1
+            for (int j0 = 0; j0 < L; j0 += kSub) {
+                float av[kSub], uv[kSub];
+                tmem_ld8(dcol + j0, av);
+                tmem_ld8(dcol + L + j0, uv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < kSub; ++j) {
+                    const int t = j0 + j;
+                    h = fmaf(av[j], h, uv[j]);
+                    if (t < nt) {
+                        __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(yt + t * HALF * 2);
+                        *yp = __float2bfloat16_rn(h * gelu_fast(__bfloat162float(*yp), tanh_form));
+                    }
+                }
+            }
+            // TMEM accumulators of this stage are free again
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.acc_empty[st]);
+
+            // ---- out tile -> global (TMA store clips the ragged tail)
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.out_ready[st]);
+            if (q == 0 && lane == 0) {
+                if (wait_bar(bars.out_ready[st], ph, wc, 12)) {
+                    tma_store_3d(&map_out, sbase + OFF_Y + st * Y_BYTES, head * DH + half * HALF, t0, b);
+                    bulk_commit();
+                    bulk_wait_read0();
+                }
+                mbar_arrive(bars.y_empty[st]);
+            }
+        }
+        if (q == 0 && lane == 0) bulk_wait0();
+    }
+
+    // ---- teardown: all tensor-core work has drained (MMA thread waited on mma_done) ----------
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// --------------------------------------------------------------------------- host side ------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map_3d(CUtensorMap* m, const void* base, int W, int T, int B, int box_c, int box_t) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)W * 2, (cuuint64_t)T * W * 2};
+    cuuint32_t box[3] = {(cuuint32_t)box_c, (cuuint32_t)box_t, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Plan {
+    int NC, items, groups, ctas, base, extra;
+    size_t off_counters, off_flags, off_agg, off_incl, total;
+};
+
+Plan make_plan(const rglru_dims* d, int sms) {
+    Plan p{};
+    p.NC = (d->seq_len + L - 1) / L;
+    p.items = d->batch * p.NC;
+    p.groups = 2 * d->heads;
+    p.ctas = p.groups >= sms ? p.groups : sms;
+    p.base = p.ctas / p.groups;
+    p.extra = p.ctas % p.groups;
+    auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
+    p.off_counters = 256;
+    p.off_flags = up(p.off_counters + (size_t)p.groups * 4);
+    p.off_agg = up(p.off_flags + (size_t)p.groups * p.items * 16);
+    p.off_incl = up(p.off_agg + (size_t)p.groups * p.items * HALF * 8);
+    p.total = up(p.off_incl + (size_t)p.groups * p.items * HALF * 4);
+    return p;
+}
+
+}  // namespace tc
+
+bool fused_prefill_supported(const rglru_dims* d) {
+    return d->act_dtype == RGLRU_BF16 && d->head_dim == tc::DH && !(d->flags & RGLRU_FLAG_GENERIC);
+}
+
+// The workspace layout is sized for the largest grid the kernel may use (one CTA per SM up to
+// 1024 SMs, so the size does not depend on the device); only the parts in use are touched.
+size_t fused_prefill_workspace(const rglru_dims* d) { return tc::make_plan(d, 1024).total; }
+
+int fused_prefill_launches(const rglru_dims* d) {
+    (void)d;
+    return 2;   // one memset of the tickets / look-back flags, one kernel
+}
+
+cudaError_t launch_fused_prefill(const rglru_dims* d, const rglru_params* p, const void* x, const void* y,
+                                 const uint8_t* reset, rglru_state* st, void* out, void* ws, size_t ws_bytes,
+                                 cudaStream_t s) {
+    using namespace tc;
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (sms > 1024) sms = 1024;
+    Plan pl = make_plan(d, sms);
+    if (pl.total > ws_bytes) return cudaErrorInvalidValue;
+    const int W = d->heads * d->head_dim;
+    CUtensorMap mx, my, mo;
+    if (!make_map_3d(&mx, x, W, d->seq_len, d->batch, DH, XROWS) ||
+        !make_map_3d(&my, y, W, d->seq_len, d->batch, HALF, L) ||
+        !make_map_3d(&mo, out, W, d->seq_len, d->batch, HALF, L))
+        return cudaErrorInvalidValue;
+    static cudaError_t attr = cudaFuncSetAttribute(fused_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)SMEM_BYTES);
+    if (attr != cudaSuccess) return attr;
+
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    Args a;
+    a.B = d->batch; a.T = d->seq_len; a.H = d->heads; a.NC = pl.NC; a.items = pl.items;
+    a.groups = pl.groups; a.base = pl.base; a.extra = pl.extra;
+    a.c = d->c; a.gelu_tanh = d->gelu_tanh; a.flags = d->flags;
+    a.timeout_ns = (d->flags & RGLRU_FLAG_TEST_WITHHOLD) ? 2000000ull : 1000000000ull;
+    a.conv_w = p->conv_w; a.conv_b = p->conv_b;
+    a.w_a = static_cast<const __nv_bfloat16*>(p->w_a); a.w_x = static_cast<const __nv_bfloat16*>(p->w_x);
+    a.b_a = p->b_a; a.b_x = p->b_x; a.lambda = p->lambda; a.reset = reset;
+    a.h_state = st ? st->h : nullptr;
+    a.tail_state = st ? static_cast<__nv_bfloat16*>(st->conv_tail) : nullptr;
+    a.status = reinterpret_cast<DeviceStatus*>(w);
+    a.counters = reinterpret_cast<unsigned*>(w + pl.off_counters);
+    a.lb_flags = reinterpret_cast<unsigned*>(w + pl.off_flags);
+    a.lb_agg = reinterpret_cast<float2*>(w + pl.off_agg);
+    a.lb_incl = reinterpret_cast<float*>(w + pl.off_incl);
+    const size_t clear = pl.off_agg - pl.off_counters;      // tickets and look-back flags
+    e = cudaMemsetAsync(w + pl.off_counters, 0, clear, s);
+    if (e != cudaSuccess) return e;
+    fused_prefill_kernel<<<pl.ctas, kThreads, SMEM_BYTES, s>>>(mx, my, mo, a);
+    return cudaGetLastError();
+}
+
+}  // namespace rglru

@@ -239,14 +239,32 @@ GenericArgs make_args(const rglru_dims* d, const rglru_params* p, const void* x,
     return a;
 }
 
-// The dynamic shared-memory limit is raised once per kernel to its largest possible need
+// The dynamic shared-memory limits of all four kernels are raised once, to their largest need
 // (head_dim 256), so that no attribute call is made while a stream is being captured.
+cudaError_t raise_smem_limits() {
+    static cudaError_t once = [] {
+        const int pre = 3 * kTile * 256 * (int)sizeof(float);
+        const int dec = kRows * 256 * (int)sizeof(float);
+        cudaError_t e = cudaFuncSetAttribute(prefill_generic_kernel<float>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, pre);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_generic_kernel<__nv_bfloat16>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, pre);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(decode_generic_kernel<float>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dec);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(decode_generic_kernel<__nv_bfloat16>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dec);
+        return e;
+    }();
+    return once;
+}
+
 template <typename K>
-cudaError_t launch(K kernel, dim3 grid, size_t smem, size_t smem_max, cudaStream_t s,
-                   const GenericArgs& a) {
-    static cudaError_t once = cudaFuncSetAttribute(
-        kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
-    if (once != cudaSuccess) return once;
+cudaError_t launch(K kernel, dim3 grid, size_t smem, cudaStream_t s, const GenericArgs& a) {
+    cudaError_t e = raise_smem_limits();
+    if (e != cudaSuccess) return e;
     kernel<<<grid, kThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
@@ -259,9 +277,8 @@ cudaError_t launch_prefill_generic(const rglru_dims* d, const rglru_params* p, c
     GenericArgs a = make_args(d, p, x, y, reset, st, out);
     dim3 grid(d->heads, d->batch);
     size_t smem = (size_t)3 * kTile * d->head_dim * sizeof(float);
-    size_t smax = (size_t)3 * kTile * 256 * sizeof(float);
-    if (d->act_dtype == RGLRU_F32) return launch(prefill_generic_kernel<float>, grid, smem, smax, s, a);
-    return launch(prefill_generic_kernel<__nv_bfloat16>, grid, smem, smax, s, a);
+    if (d->act_dtype == RGLRU_F32) return launch(prefill_generic_kernel<float>, grid, smem, s, a);
+    return launch(prefill_generic_kernel<__nv_bfloat16>, grid, smem, s, a);
 }
 
 cudaError_t launch_decode_generic(const rglru_dims* d, const rglru_params* p, const void* x,
@@ -271,9 +288,8 @@ cudaError_t launch_decode_generic(const rglru_dims* d, const rglru_params* p, co
     a.T = 1;
     dim3 grid(d->heads, (d->batch + kRows - 1) / kRows);
     size_t smem = (size_t)kRows * d->head_dim * sizeof(float);
-    size_t smax = (size_t)kRows * 256 * sizeof(float);
-    if (d->act_dtype == RGLRU_F32) return launch(decode_generic_kernel<float>, grid, smem, smax, s, a);
-    return launch(decode_generic_kernel<__nv_bfloat16>, grid, smem, smax, s, a);
+    if (d->act_dtype == RGLRU_F32) return launch(decode_generic_kernel<float>, grid, smem, s, a);
+    return launch(decode_generic_kernel<__nv_bfloat16>, grid, smem, s, a);
 }
 
 }  // namespace rglru

