@@ -11,14 +11,16 @@
 //     held by a running CTA;
 //   * warp roles: an x producer (TMA: x tile with a 3-token halo, and the ticket), a y producer
 //     (TMA: y tile, issued once the previous out store of that stage has left shared memory),
-//     8 conv warps (causal width-4 depthwise conv in fp32, written as the bf16 B operand in the
+//     4 conv warps (causal width-4 depthwise conv in fp32, written as the bf16 B operand in the
 //     128-byte swizzled K-major layout), 1 MMA thread (gates^T[128 ch x 64 tok] = W^T . xc^T for
 //     both gates, K = 256 in 16 steps, fp32 accumulators in TMEM), and 2 epilogue groups of 4
 //     warps, group g owning TMEM stage g, so one group's look-back wait overlaps the other
 //     group's math;
 //   * transposed orientation: a TMEM lane is an output channel and the 64 columns are tokens,
 //     so an epilogue thread owns one channel and runs the diagonal scan along its registers
-//     (no shuffles);
+//     (no shuffles); its first pass leaves the running (prod a, local h) of every token in
+//     TMEM, so once the carry C is known the second pass is h_t = P_t C + h_t^loc, with no
+//     serial chain; token pairs use the packed fp32x2 FMA of sm_100;
 //   * chunks of one sequence handled by different CTAs chain through a look-back in the spirit
 //     of Merrill & Garland ("Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016):
 //     after its first pass a chunk publishes its aggregate (prod a, local h) per channel; its
@@ -55,18 +57,18 @@ using namespace sm100;
 constexpr int DH = 256;                 // head dim (K of the gate contraction)
 constexpr int HALF = 128;               // output channels per CTA (= TMEM lanes = MMA M)
 constexpr int L = 64;                   // tokens per chunk (= MMA N)
-constexpr int LH = L / 2;               // tokens per conv warp
 constexpr int XROWS = L + kHist;        // x tile rows incl. the 3-token halo
 constexpr int KSTEPS = DH / 16;         // MMA K steps
 constexpr int STAGES = 2;
 constexpr int SLOTS = 8;                // ring of item ids, indexed by iteration
 constexpr int kSub = 8;                 // tokens per TMEM load in the epilogue
 
-// warp roles: 0-7 conv (K block = warp % 4, token half = warp / 4), 8-15 epilogue (TMEM lane
-// quarter = warp % 4, group = stage = (warp - 8) / 4), 16 x producer, 17 y producer, 18 MMA.
-constexpr int kConvWarps = 8, kEpiWarps = 8, kEpiGroup = 4;
-constexpr int kWarpEpi0 = 8, kWarpProdX = 16, kWarpProdY = 17, kWarpMma = 18;
-constexpr int kThreads = 19 * 32;
+// warp roles: 0-3 conv (K block = warp), 4-11 epilogue (TMEM lane quarter = warp % 4, group =
+// stage = (warp - 4) / 4), 12 x producer (x tiles and tickets), 13 y producer, 14 MMA.  The two
+// producers spin on different barriers, so they live in different warps.
+constexpr int kConvWarps = 4, kEpiWarps = 8, kEpiGroup = 4;
+constexpr int kWarpEpi0 = 4, kWarpProdX = 12, kWarpProdY = 13, kWarpMma = 14;
+constexpr int kThreads = 15 * 32;
 
 constexpr uint32_t X_BYTES = XROWS * DH * 2;      // 34304
 constexpr uint32_t Y_BYTES = L * HALF * 2;        // 16384
@@ -250,6 +252,40 @@ __device__ __forceinline__ void decay_beta(float l, bool small_range, float& a, 
     beta = v > 0.0f ? v * rsqrt_approx(v) : 0.0f;
 }
 
+// Packed helpers (two tokens per instruction on the fp32x2 pipe of sm_100).
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// Fast path of gates + decay + normalised input for a channel with |c log sigma(Lambda)| <= 1/8,
+// two tokens at a time.  With s = 1 + e^{-(g_a + b_a)}: sqrt(r) = rsqrt(s) and r = sqrt(r)^2 (so
+// one ex2 and one rsqrt give both); l = c_lab r; a = 1 + expm1(l) from the Taylor series of
+// expm1 (terms l^k / k!); sqrt(1 - a^2) = sqrt(-2 l) sqrt(expm1(2l) / 2l) = K sqrt(r) Q(l) with
+// K = sqrt(-2 c_lab) and Q(l) = sqrt(expm1(2l) / 2l) from its Taylor series in 2l,
+// 1 + x/4 + 5x^2/96 + x^3/128 + 79x^4/92160 (relative error < 1e-7 for |2l| <= 1/4).
+__device__ __forceinline__ void gates_pair(float2 ga, float2 gx, float nbl, float c_lab, float K,
+                                           float bxh, float2 xc, float2& a, float2& u) {
+    const float2 z = fma2(ga, f2(-1.4426950408889634f), f2(nbl));
+    const float2 s = add2(make_float2(ex2_approx(z.x), ex2_approx(z.y)), f2(1.0f));
+    const float2 rs = make_float2(rsqrt_approx(s.x), rsqrt_approx(s.y));
+    const float2 l = mul2(mul2(rs, rs), f2(c_lab));
+    float2 p = fma2(l, f2(1.0f / 720.0f), f2(1.0f / 120.0f));
+    p = fma2(l, p, f2(1.0f / 24.0f));
+    p = fma2(l, p, f2(1.0f / 6.0f));
+    p = fma2(l, p, f2(0.5f));
+    p = fma2(l, p, f2(1.0f));
+    a = fma2(l, p, f2(1.0f));
+    float2 q = fma2(l, f2(79.0f / 5760.0f), f2(1.0f / 16.0f));
+    q = fma2(l, q, f2(5.0f / 24.0f));
+    q = fma2(l, q, f2(0.5f));
+    q = fma2(l, q, f2(1.0f));
+    const float2 beta = mul2(mul2(rs, q), f2(K));
+    const float2 zi = fma2(gx, f2(0.5f), f2(bxh));
+    const float2 ig = fma2(make_float2(tanh_approx(zi.x), tanh_approx(zi.y)), f2(0.5f), f2(0.5f));
+    u = mul2(mul2(beta, ig), xc);
+}
+
 // GeLU(v) = v Phi(v).  Exact form: Phi from erf of Abramowitz & Stegun 7.1.28,
 // erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 for x >= 0 (|error| <= 3e-7), one reciprocal.
 // Tanh form: 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))).
@@ -271,6 +307,24 @@ __device__ __forceinline__ float gelu_fast(float v, int tanh_form) {
     p = p * p;                                        // (1 + ...)^16
     const float half_erfc = 0.5f * rcp_approx(p);     // (1 - erf(x)) / 2
     return v * (v >= 0.0f ? 1.0f - half_erfc : half_erfc);
+}
+
+// GeLU of two values at once (packed fp32x2 for the polynomial part).
+__device__ __forceinline__ float2 gelu_pair(float2 v, int tanh_form) {
+    if (tanh_form) return make_float2(gelu_fast(v.x, 1), gelu_fast(v.y, 1));
+    const float2 x = mul2(make_float2(fabsf(v.x), fabsf(v.y)), f2(0.70710678118654752f));
+    float2 p = fma2(x, f2(0.0000430638f), f2(0.0002765672f));
+    p = fma2(x, p, f2(0.0001520143f));
+    p = fma2(x, p, f2(0.0092705272f));
+    p = fma2(x, p, f2(0.0422820123f));
+    p = fma2(x, p, f2(0.0705230784f));
+    p = fma2(x, p, f2(1.0f));
+    p = mul2(p, p);
+    p = mul2(p, p);
+    p = mul2(p, p);
+    p = mul2(p, p);
+    const float2 e = mul2(make_float2(rcp_approx(p.x), rcp_approx(p.y)), f2(0.5f));
+    return make_float2(v.x * (v.x >= 0.0f ? 1.0f - e.x : e.x), v.y * (v.y >= 0.0f ? 1.0f - e.y : e.y));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -328,7 +382,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     // with coalesced 16-byte loads: gate a at byte 0, gate x at byte 65536 (B and x tiles are
     // still unused)
     if (warp < kConvWarps + kEpiWarps) {
-        const int tid = threadIdx.x;                       // 0..511
+        const int tid = threadIdx.x;                       // 0..383
         for (int e = tid; e < 2 * DH * (HALF / 8); e += (kConvWarps + kEpiWarps) * 32) {
             const int g = e / (DH * (HALF / 8)), r = e % (DH * (HALF / 8));
             const int i = r / (HALF / 8), o8 = r % (HALF / 8);
@@ -366,8 +420,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     __syncthreads();   // the staging area is free again before any TMA load lands in it
 
     if (warp == kWarpProdX) {
-        // ================================ x producer (and tickets) ============================
         if (lane == 0) {
+            // ============================ x producer (and tickets) ============================
             int issued[STAGES] = {0, 0};
             for (int n = 0;; ++n) {
                 const int st = n & 1;
@@ -399,8 +453,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 }
         }
     } else if (warp == kWarpProdY) {
-        // ================================ y producer ==========================================
         if (lane == 0) {
+            // ============================ y producer ==========================================
             int issued[STAGES] = {0, 0};
             for (int n = 0;; ++n) {
                 const int st = n & 1;
@@ -471,17 +525,14 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         }
     } else if (warp < kConvWarps) {
         // ================================ conv warps ==========================================
-        const int kb = warp & 3, th = warp >> 2;          // K block, token half
+        const int kb = warp;                              // K block of the B tile
         const int p = kb * 32 + lane;                     // channel pair 2p, 2p+1 of the head
         const int chg = head * DH + 2 * p;                // global channel of the pair
-        float w0[kConvWidth], w1[kConvWidth];
+        float2 w[kConvWidth];
 #pragma unroll
-        for (int k = 0; k < kConvWidth; ++k) {
-            w0[k] = a.conv_w[(size_t)k * W + chg];
-            w1[k] = a.conv_w[(size_t)k * W + chg + 1];
-        }
-        const float cb0 = a.conv_b ? a.conv_b[chg] : 0.f;
-        const float cb1 = a.conv_b ? a.conv_b[chg + 1] : 0.f;
+        for (int k = 0; k < kConvWidth; ++k)
+            w[k] = make_float2(a.conv_w[(size_t)k * W + chg], a.conv_w[(size_t)k * W + chg + 1]);
+        const float2 cb = make_float2(a.conv_b ? a.conv_b[chg] : 0.f, a.conv_b ? a.conv_b[chg + 1] : 0.f);
         const bool own_tail = (p >> 6) == half;          // this CTA writes these tail channels
         for (int n = 0;; ++n) {
             const int st = n & 1;
@@ -496,49 +547,61 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             }
             const int b = k / a.NC, c = k % a.NC, t0 = c * L;
             const int nt = min(L, a.T - t0);
-            const int tb = th * LH;                        // first token of this warp's half
-            const int ts = t0 + tb;                        // its sequence position
             const uint8_t* rst = a.reset ? a.reset + (size_t)b * a.T : nullptr;
             const uint8_t* xt = smem + OFF_X + st * X_BYTES + 4 * p;
             uint8_t* bt = smem + OFF_B + st * B_BYTES;
-            float h0a, h1a, h2a, h0b, h1b, h2b;          // window x_{t-3}, x_{t-2}, x_{t-1}
-            if (ts == 0) {
+            auto xrow = [&](int r) {                      // x tile row r = token t0 - 3 + r
+                const uint32_t v = *reinterpret_cast<const uint32_t*>(xt + r * DH * 2);
+                return make_float2(bf16lo(v), bf16hi(v));
+            };
+            float2 h0, h1, h2;                            // window x_{t-3}, x_{t-2}, x_{t-1}
+            if (c == 0) {
                 if (a.tail_state) {
                     const __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
-                    uint32_t v0 = *reinterpret_cast<const uint32_t*>(tl);
-                    uint32_t v1 = *reinterpret_cast<const uint32_t*>(tl + W);
-                    uint32_t v2 = *reinterpret_cast<const uint32_t*>(tl + 2 * W);
-                    h0a = bf16lo(v0); h0b = bf16hi(v0);
-                    h1a = bf16lo(v1); h1b = bf16hi(v1);
-                    h2a = bf16lo(v2); h2b = bf16hi(v2);
+                    const uint32_t v0 = *reinterpret_cast<const uint32_t*>(tl);
+                    const uint32_t v1 = *reinterpret_cast<const uint32_t*>(tl + W);
+                    const uint32_t v2 = *reinterpret_cast<const uint32_t*>(tl + 2 * W);
+                    h0 = make_float2(bf16lo(v0), bf16hi(v0));
+                    h1 = make_float2(bf16lo(v1), bf16hi(v1));
+                    h2 = make_float2(bf16lo(v2), bf16hi(v2));
                 } else {
-                    h0a = h1a = h2a = h0b = h1b = h2b = 0.f;
+                    h0 = h1 = h2 = make_float2(0.f, 0.f);
                 }
             } else {
-                uint32_t v0 = *reinterpret_cast<const uint32_t*>(xt + (tb + 0) * DH * 2);
-                uint32_t v1 = *reinterpret_cast<const uint32_t*>(xt + (tb + 1) * DH * 2);
-                uint32_t v2 = *reinterpret_cast<const uint32_t*>(xt + (tb + 2) * DH * 2);
-                h0a = bf16lo(v0); h0b = bf16hi(v0);
-                h1a = bf16lo(v1); h1b = bf16hi(v1);
-                h2a = bf16lo(v2); h2b = bf16hi(v2);
-                if (rst && ts < a.T) {
-                    if (rst[ts - 1]) { h0a = h0b = h1a = h1b = 0.f; }
-                    if (rst[ts - 2]) { h0a = h0b = 0.f; }
+                h0 = xrow(0);
+                h1 = xrow(1);
+                h2 = xrow(2);
+                if (rst) {
+                    if (rst[t0 - 1]) h0 = h1 = make_float2(0.f, 0.f);
+                    if (rst[t0 - 2]) h0 = make_float2(0.f, 0.f);
                 }
             }
-            float ta0 = 0.f, ta1 = 0.f, ta2 = 0.f, tb0 = 0.f, tb1 = 0.f, tb2 = 0.f;   // final window
+            float2 f0 = h0, f1 = h1, f2v = h2;            // final window (the tail of the row)
+            if (!rst && nt == L) {
+                // fast path: a full chunk without segment resets
 #pragma unroll 8
-            for (int j = 0; j < LH; ++j) {
-                const int t = tb + j;
-                const uint32_t v = *reinterpret_cast<const uint32_t*>(xt + (t + kHist) * DH * 2);
-                const float xa = bf16lo(v), xb = bf16hi(v);
-                if (rst && t < nt && rst[t0 + t]) { h0a = h1a = h2a = h0b = h1b = h2b = 0.f; }
-                float ya = fmaf(w0[3], xa, fmaf(w0[2], h2a, fmaf(w0[1], h1a, fmaf(w0[0], h0a, cb0))));
-                float yb = fmaf(w1[3], xb, fmaf(w1[2], h2b, fmaf(w1[1], h1b, fmaf(w1[0], h0b, cb1))));
-                *reinterpret_cast<uint32_t*>(bt + b_tile_offset(t, 2 * p)) = pack_bf16x2(ya, yb);
-                h0a = h1a; h1a = h2a; h2a = xa;
-                h0b = h1b; h1b = h2b; h2b = xb;
-                if (t == nt - 1) { ta0 = h0a; ta1 = h1a; ta2 = h2a; tb0 = h0b; tb1 = h1b; tb2 = h2b; }
+                for (int t = 0; t < L; ++t) {
+                    const float2 xv = xrow(t + kHist);
+                    float2 y = fma2(w[0], h0, cb);
+                    y = fma2(w[1], h1, y);
+                    y = fma2(w[2], h2, y);
+                    y = fma2(w[3], xv, y);
+                    *reinterpret_cast<uint32_t*>(bt + b_tile_offset(t, 2 * p)) = pack_bf16x2(y.x, y.y);
+                    h0 = h1; h1 = h2; h2 = xv;
+                }
+                f0 = h0; f1 = h1; f2v = h2;
+            } else {
+                for (int t = 0; t < L; ++t) {
+                    const float2 xv = xrow(t + kHist);
+                    if (rst && t < nt && rst[t0 + t]) h0 = h1 = h2 = make_float2(0.f, 0.f);
+                    float2 y = fma2(w[0], h0, cb);
+                    y = fma2(w[1], h1, y);
+                    y = fma2(w[2], h2, y);
+                    y = fma2(w[3], xv, y);
+                    *reinterpret_cast<uint32_t*>(bt + b_tile_offset(t, 2 * p)) = pack_bf16x2(y.x, y.y);
+                    h0 = h1; h1 = h2; h2 = xv;
+                    if (t == nt - 1) { f0 = h0; f1 = h1; f2v = h2; }
+                }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -547,14 +610,14 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 mbar_arrive(bars.b_full[st]);
             }
             // final conv history of the sequence, once its first chunk has read the old one
-            if (a.tail_state && c == a.NC - 1 && own_tail && nt - 1 >= tb && nt - 1 < tb + LH) {
+            if (a.tail_state && c == a.NC - 1 && own_tail) {
                 bool ok = true;
                 if (c > 0) ok = wait_flag(a.lb_flags + (lb_base + (size_t)b * a.NC) * 4, FLAG_AGG, wc, 8) != 0;
                 if (ok) {
                     __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
-                    *reinterpret_cast<uint32_t*>(tl) = pack_bf16x2(ta0, tb0);
-                    *reinterpret_cast<uint32_t*>(tl + W) = pack_bf16x2(ta1, tb1);
-                    *reinterpret_cast<uint32_t*>(tl + 2 * W) = pack_bf16x2(ta2, tb2);
+                    *reinterpret_cast<uint32_t*>(tl) = pack_bf16x2(f0.x, f0.y);
+                    *reinterpret_cast<uint32_t*>(tl + W) = pack_bf16x2(f1.x, f1.y);
+                    *reinterpret_cast<uint32_t*>(tl + 2 * W) = pack_bf16x2(f2v.x, f2v.y);
                 }
             }
         }
@@ -572,6 +635,9 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         const bool small_range = c_lab >= -0.125f;
         const float ba = a.b_a ? a.b_a[ch] : 0.f;
         const float bx = a.b_x ? a.b_x[ch] : 0.f;
+        const float nbl = -ba * 1.4426950408889634f;   // fast path constants
+        const float bxh = 0.5f * bx;
+        const float Kb = sqrtf(fmaxf(-2.0f * c_lab, 0.0f));
         const int tanh_form = a.gelu_tanh;
         const bool withhold_hook = (a.flags & RGLRU_FLAG_TEST_WITHHOLD) && group == 0;
         const uint8_t* bt = smem + OFF_B + st * B_BYTES;
@@ -591,34 +657,74 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             const bool withhold = withhold_hook && k == 0;
             unsigned* myflag = a.lb_flags + (lb_base + k) * 4 + q;
 
-            // ---- pass 1: gates, decay and normalised input of the chunk -> TMEM (a, u)
+            // ---- pass 1: gates, decay and normalised input; TMEM keeps the running product of
+            //      the decays P_t and the running local state H_t (from zero) of every token
             float aggA = 1.f, aggH = 0.f;
-#pragma unroll 1
-            for (int j0 = 0; j0 < L; j0 += kSub) {
-                float ga[kSub], gx[kSub];
-                tmem_ld8(dcol + j0, ga);
-                tmem_ld8(dcol + L + j0, gx);
+            const bool fast = !rst && nt == L && __all_sync(0xffffffffu, small_range);
+            if (fast) {
+                float ga[kSub], gx[kSub], gan[kSub], gxn[kSub];
+                tmem_ld8(dcol, ga);
+                tmem_ld8(dcol + L, gx);
                 tmem_wait_ld();
-                uint32_t ra[kSub], ru[kSub];
+#pragma unroll 1
+                for (int j0 = 0; j0 < L; j0 += kSub) {
+                    if (j0 + kSub < L) {                    // next sub-block in flight meanwhile
+                        tmem_ld8(dcol + j0 + kSub, gan);
+                        tmem_ld8(dcol + L + j0 + kSub, gxn);
+                    }
+                    uint32_t ra[kSub], ru[kSub];
 #pragma unroll
-                for (int j = 0; j < kSub; ++j) {
-                    const int t = j0 + j;
-                    const float xc = __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(
-                                                         bt + b_tile_offset(t, chl)) << 16);
-                    const float r = sigmoid_fast(ga[j] + ba);
-                    float at, beta;
-                    decay_beta(c_lab * r, small_range, at, beta);
-                    const float ig = sigmoid_tanh(gx[j] + bx);
-                    float u = beta * (ig * xc);
-                    if (rst && t < nt && rst[t]) at = 0.f;                // h_{t-1} := 0
-                    if (t >= nt) { at = 1.f; u = 0.f; }                   // padding: identity
-                    aggH = fmaf(at, aggH, u);
-                    aggA *= at;
-                    ra[j] = __float_as_uint(at);
-                    ru[j] = __float_as_uint(u);
+                    for (int j = 0; j < kSub; j += 2) {
+                        const int t = j0 + j;
+                        const float2 xc = make_float2(
+                            __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(bt + b_tile_offset(t, chl)) << 16),
+                            __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(bt + b_tile_offset(t + 1, chl)) << 16));
+                        float2 at, u;
+                        gates_pair(make_float2(ga[j], ga[j + 1]), make_float2(gx[j], gx[j + 1]), nbl, c_lab, Kb,
+                                   bxh, xc, at, u);
+                        aggH = fmaf(at.x, aggH, u.x);
+                        aggA *= at.x;
+                        ra[j] = __float_as_uint(aggA);
+                        ru[j] = __float_as_uint(aggH);
+                        aggH = fmaf(at.y, aggH, u.y);
+                        aggA *= at.y;
+                        ra[j + 1] = __float_as_uint(aggA);
+                        ru[j + 1] = __float_as_uint(aggH);
+                    }
+                    tmem_st8(dcol + j0, ra);
+                    tmem_st8(dcol + L + j0, ru);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < kSub; ++j) { ga[j] = gan[j]; gx[j] = gxn[j]; }
                 }
-                tmem_st8(dcol + j0, ra);
-                tmem_st8(dcol + L + j0, ru);
+            } else {
+#pragma unroll 1
+                for (int j0 = 0; j0 < L; j0 += kSub) {
+                    float ga[kSub], gx[kSub];
+                    tmem_ld8(dcol + j0, ga);
+                    tmem_ld8(dcol + L + j0, gx);
+                    tmem_wait_ld();
+                    uint32_t ra[kSub], ru[kSub];
+#pragma unroll
+                    for (int j = 0; j < kSub; ++j) {
+                        const int t = j0 + j;
+                        const float xc = __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(
+                                                             bt + b_tile_offset(t, chl)) << 16);
+                        const float r = sigmoid_fast(ga[j] + ba);
+                        float at, beta;
+                        decay_beta(c_lab * r, small_range, at, beta);
+                        const float ig = sigmoid_tanh(gx[j] + bx);
+                        float u = beta * (ig * xc);
+                        if (rst && t < nt && rst[t]) at = 0.f;                // h_{t-1} := 0
+                        if (t >= nt) { at = 1.f; u = 0.f; }                   // padding: identity
+                        aggH = fmaf(at, aggH, u);
+                        aggA *= at;
+                        ra[j] = __float_as_uint(aggA);
+                        ru[j] = __float_as_uint(aggH);
+                    }
+                    tmem_st8(dcol + j0, ra);
+                    tmem_st8(dcol + L + j0, ru);
+                }
             }
             // the B tile (xc) is no longer read by this warp
             __syncwarp();
@@ -690,24 +796,34 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 if (okw) a.h_state[(size_t)b * W + ch] = incl;
             }
 
-            // ---- pass 2: replay the scan from TMEM, merge with GeLU(y)
+            // ---- pass 2: h_t = P_t C + H_t (no serial chain), merged with GeLU(y_t)
             if (!wait_bar(bars.y_full[st], ph, wc, 16)) break;
             tmem_wait_st();
-            float h = carry;
-#pragma unroll 1
-            for (int j0 = 0; j0 < L; j0 += kSub) {
-                float av[kSub], uv[kSub];
-                tmem_ld8(dcol + j0, av);
-                tmem_ld8(dcol + L + j0, uv);
+            {
+                float pv[kSub], hv[kSub], pn[kSub], hn[kSub];
+                tmem_ld8(dcol, pv);
+                tmem_ld8(dcol + L, hv);
                 tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < kSub; ++j) {
-                    const int t = j0 + j;
-                    h = fmaf(av[j], h, uv[j]);
-                    if (t < nt) {
-                        __nv_bfloat16* yp = reinterpret_cast<__nv_bfloat16*>(yt + t * HALF * 2);
-                        *yp = __float2bfloat16_rn(h * gelu_fast(__bfloat162float(*yp), tanh_form));
+#pragma unroll 1
+                for (int j0 = 0; j0 < L; j0 += kSub) {
+                    if (j0 + kSub < L) {
+                        tmem_ld8(dcol + j0 + kSub, pn);
+                        tmem_ld8(dcol + L + j0 + kSub, hn);
                     }
+#pragma unroll
+                    for (int j = 0; j < kSub; j += 2) {
+                        const int t = j0 + j;
+                        const float2 hh = fma2(make_float2(pv[j], pv[j + 1]), f2(carry), make_float2(hv[j], hv[j + 1]));
+                        __nv_bfloat16* y0 = reinterpret_cast<__nv_bfloat16*>(yt + t * HALF * 2);
+                        __nv_bfloat16* y1 = reinterpret_cast<__nv_bfloat16*>(yt + (t + 1) * HALF * 2);
+                        const float2 g = gelu_pair(make_float2(__bfloat162float(*y0), __bfloat162float(*y1)), tanh_form);
+                        const float2 o = mul2(hh, g);
+                        if (t < nt) *y0 = __float2bfloat16_rn(o.x);
+                        if (t + 1 < nt) *y1 = __float2bfloat16_rn(o.y);
+                    }
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < kSub; ++j) { pv[j] = pn[j]; hv[j] = hn[j]; }
                 }
             }
             // TMEM accumulators of this stage are free again
