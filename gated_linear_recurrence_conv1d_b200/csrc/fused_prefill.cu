@@ -148,8 +148,8 @@ struct WaitCtx {
 __device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, WaitCtx w, unsigned where) {
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255) == 0) {
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;   // sleeps up to 100 us
+        {
             if (*w.abort) return false;
             if (*(volatile unsigned*)&w.status->code != 0) {
                 *w.abort = 1;
@@ -175,10 +175,10 @@ __device__ __noinline__ unsigned wait_flag(const unsigned* f, unsigned want, Wai
     if (v >= want) return v;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        __nanosleep(20);
+        __nanosleep(128);
         v = ld_acquire_gpu(f);
         if (v >= want) return v;
-        if ((i & 63) == 0) {
+        if ((i & 15) == 0) {
             if (*w.abort || *(volatile unsigned*)&w.status->code != 0) {
                 *w.abort = 1;
                 return 0;
@@ -447,7 +447,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 if (issued[st]) {
                     const int n = issued[st] - 1;
                     const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait(bars.x_full[st], (n >> 1) & 1) &&
+                    while (!mbar_try_wait_sleep(bars.x_full[st], (n >> 1) & 1, 100000u) &&
                            globaltimer_ns() - t0 < a.timeout_ns) {
                     }
                 }
@@ -479,7 +479,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 if (issued[st]) {
                     const int n = issued[st] - 1;
                     const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait(bars.y_full[st], (n >> 1) & 1) &&
+                    while (!mbar_try_wait_sleep(bars.y_full[st], (n >> 1) & 1, 100000u) &&
                            globaltimer_ns() - t0 < a.timeout_ns) {
                     }
                 }
@@ -520,7 +520,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             // every MMA this thread issued has finished before TMEM is released
             mma_commit(bars.mma_done);
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(bars.mma_done, 0) && globaltimer_ns() - t0 < a.timeout_ns) {
+            while (!mbar_try_wait_sleep(bars.mma_done, 0, 100000u) && globaltimer_ns() - t0 < a.timeout_ns) {
             }
         }
     } else if (warp < kConvWarps) {
@@ -755,8 +755,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     bool okl = mine ? ld_acquire_gpu(fl) >= FLAG_AGG : true;
                     if (lane == 0) okl = okl && ld_acquire_gpu(fa) >= FLAG_INCL;
                     if (__all_sync(0xffffffffu, okl)) { ready = true; break; }
-                    __nanosleep(20);
-                    if ((it & 63) == 63) {
+                    __nanosleep(128);
+                    if ((it & 15) == 15) {
                         int give_up = 0;
                         if (lane == 0) {
                             if (*abort || *(volatile unsigned*)&a.status->code != 0) give_up = 1;
