@@ -180,3 +180,49 @@ def tail_from_act(tail0: np.ndarray) -> np.ndarray:
     if tail0.dtype == np.uint16:
         return np.ascontiguousarray((tail0.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
     return np.ascontiguousarray(tail0, dtype=np.float64)
+
+
+def prefill_units(params: dict, x: np.ndarray, y: np.ndarray, heads: int, units: Sequence,
+                  reset: Optional[np.ndarray] = None, h0: Optional[np.ndarray] = None,
+                  tail0: Optional[np.ndarray] = None, c: float = 8.0, gelu_tanh: int = 0,
+                  workers: int = 0):
+    """Prefill of selected (b, head) sequences only, without materialising [B, T, W] outputs.
+
+    Returns {(b, head): (out [T, dh], h [dh], tail [3, dh])}, fp64.  Sequences run in parallel
+    threads (the C call releases the GIL); each one is the plain sequential definition.
+    """
+    from concurrent.futures import ThreadPoolExecutor
+    lib = _load()
+    B, T, W = x.shape
+    dh = W // heads
+    _, dt = _act(x[:1, :1])
+    es = 4 if dt == F32 else 2
+    w_a, _ = _act(params["w_a"])
+    w_x, _ = _act(params["w_x"])
+    conv_w = _f32(params["conv_w"])
+    conv_b, b_a, b_x, lam = (_f32(params.get(k)) for k in ("conv_b", "b_a", "b_x", "lam"))
+    base = lambda arr, off, size: ctypes.c_void_p(arr.ctypes.data + off * size)  # noqa: E731
+
+    def one(unit):
+        b, hd = unit
+        ch0 = hd * dh
+        xs, _ = _act(x[b, :, ch0:ch0 + dh])
+        ys, _ = _act(y[b, :, ch0:ch0 + dh])
+        h = np.zeros(dh) if h0 is None else np.array(h0[b, ch0:ch0 + dh], dtype=np.float64)
+        tail = (np.zeros((HIST, dh)) if tail0 is None
+                else np.ascontiguousarray(tail_from_act(tail0[b][:, ch0:ch0 + dh])))
+        out = np.zeros((T, dh))
+        rst = None if reset is None else np.ascontiguousarray(reset[b], dtype=np.uint8)
+        rc = lib.rglru_oracle_prefill_unit(
+            T, dh, c, gelu_tanh, dt, base(conv_w, ch0, 4), W,
+            None if conv_b is None else base(conv_b, ch0, 4),
+            base(w_a, hd * dh * dh, es), base(w_x, hd * dh * dh, es), dt,
+            None if b_a is None else base(b_a, ch0, 4), None if b_x is None else base(b_x, ch0, 4),
+            base(lam, ch0, 4), _p(xs), _p(ys), dh, _p(rst), _p(h), _p(tail), dh, _p(out), dh, None)
+        if rc != 0:
+            raise RuntimeError("oracle prefill_unit failed")
+        return (b, hd), (out, h, tail)
+
+    n = workers or min(len(units), max(1, os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        return dict(ex.map(one, [tuple(u) for u in units]))

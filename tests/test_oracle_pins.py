@@ -392,3 +392,24 @@ def test_oracle_regression_golden():
         _, _, out, h, _ = make_golden.make_case(case)
         np.testing.assert_array_equal(out.ravel(), np.array(case["out"]))
         np.testing.assert_array_equal(h.ravel(), np.array(case["h"]))
+
+
+def test_prefill_units_matches_full_batch():
+    """The per-sequence entry point computes exactly what the batched one does."""
+    rng = np.random.default_rng(12)
+    B, T, H, dh = 3, 30, 3, 8
+    W = H * dh
+    p = _params(W, H, dh, rng, dtype="bf16")
+    x = inputs.f32_to_bf16_bits(rng.standard_normal((B, T, W)).astype(np.float32))
+    y = inputs.f32_to_bf16_bits(rng.standard_normal((B, T, W)).astype(np.float32))
+    reset = (rng.random((B, T)) < 0.1).astype(np.uint8)
+    h0 = rng.standard_normal((B, W))
+    tail0 = inputs.f32_to_bf16_bits(rng.standard_normal((B, 3, W)).astype(np.float32))
+    out, hT, tT = oracle.prefill(p, x, y, H, reset=reset, h0=h0, tail0=tail0)
+    units = [(0, 2), (2, 0), (1, 1)]
+    got = oracle.prefill_units(p, x, y, H, units, reset=reset, h0=h0, tail0=tail0)
+    for (b, hd), (o, h, t) in got.items():
+        sl = slice(hd * dh, (hd + 1) * dh)
+        np.testing.assert_array_equal(o, out[b, :, sl])
+        np.testing.assert_array_equal(h, hT[b, sl])
+        np.testing.assert_array_equal(t, tT[b, :, sl])
