@@ -29,7 +29,11 @@ STATUS_NAMES = {0: "RGLRU_OK", 1: "RGLRU_ERR_INVALID_ARG", 2: "RGLRU_ERR_UNSUPPO
 
 EXPORTED = ("rglru_state_init", "rglru_prefill_workspace_size", "rglru_block_prefill",
             "rglru_decode_workspace_size", "rglru_block_decode", "rglru_read_device_status",
-            "rglru_status_string", "rglru_abi_version", "rglru_prefill_plan", "rglru_decode_plan")
+            "rglru_status_string", "rglru_abi_version", "rglru_prefill_plan", "rglru_decode_plan",
+            "rglru_block_prefill_noalloc")
+
+# Bytes of the static device scratch behind rglru_block_prefill_noalloc.
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class RglruError(RuntimeError):
@@ -83,6 +87,8 @@ def load(build_if_missing: bool = True):
     lib.rglru_decode_workspace_size.restype = S
     lib.rglru_block_prefill.argtypes = [PD, PP, V, V, V, PS, V, V, S, V]
     lib.rglru_block_prefill.restype = I
+    lib.rglru_block_prefill_noalloc.argtypes = [PD, PP, V, V, V, PS, V, V, V]
+    lib.rglru_block_prefill_noalloc.restype = I
     lib.rglru_block_decode.argtypes = [PD, PP, V, V, V, PS, V, V, S, V]
     lib.rglru_block_decode.restype = I
     lib.rglru_read_device_status.argtypes = [V, S, V]
@@ -165,6 +171,21 @@ def block_prefill(dims: Dims, params: Params, x: torch.Tensor, y: torch.Tensor,
                                     _ptr(reset), ctypes.byref(st) if st is not None else None,
                                     _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
     _check(rc, "rglru_block_prefill")
+
+
+def block_prefill_noalloc(dims: Dims, params: Params, x: torch.Tensor, y: torch.Tensor,
+                          out: torch.Tensor, reset: Optional[torch.Tensor] = None,
+                          h: Optional[torch.Tensor] = None, conv_tail: Optional[torch.Tensor] = None,
+                          status_out: Optional[torch.Tensor] = None, stream=None):
+    """rglru_block_prefill without a workspace: the library's static device scratch is used
+    (for callers that cannot allocate device memory).  status_out: optional 16-byte device
+    buffer that receives the device status word after the kernel."""
+    st = State(_ptr(h), _ptr(conv_tail)) if h is not None else None
+    rc = load().rglru_block_prefill_noalloc(ctypes.byref(dims), ctypes.byref(params), _ptr(x),
+                                            _ptr(y), _ptr(reset),
+                                            ctypes.byref(st) if st is not None else None,
+                                            _ptr(out), _ptr(status_out), _stream(stream))
+    _check(rc, "rglru_block_prefill_noalloc")
 
 
 def block_decode(dims: Dims, params: Params, x: torch.Tensor, y: torch.Tensor, out: torch.Tensor,

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "rglru.h"
@@ -67,6 +69,35 @@ rglru_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return RGLRU_OK;
     cudaGetLastError();   // clear a sticky launch-configuration error for the caller
     return RGLRU_ERR_CUDA;
+}
+
+// Scratch of rglru_block_prefill_noalloc: a fixed area in the library's device image, for
+// callers that cannot allocate device memory.  In host code `g_noalloc_scratch` names a host
+// shadow, not device memory, so kernels only ever receive the address that
+// cudaGetSymbolAddress returns for the current device.
+__device__ __align__(256) unsigned char g_noalloc_scratch[RGLRU_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of the static scratch on the current device, looked up once per device
+// (with that device current) and cached.
+cudaError_t noalloc_scratch(void** addr) {
+    static std::mutex mu;
+    static void* cache[kMaxDevices] = {};
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cache[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        if (!p) return cudaErrorInvalidSymbol;
+        cache[dev] = p;
+    }
+    *addr = cache[dev];
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -143,6 +174,36 @@ rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_params* para
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return cuda_status(rglru::launch_decode_generic(dims, params, x, y, reset, state, out, s));
+}
+
+rglru_status rglru_block_prefill_noalloc(const rglru_dims* dims, const rglru_params* params,
+                                         const void* x, const void* y, const uint8_t* reset,
+                                         rglru_state* state, void* out, void* status_out,
+                                         void* stream) {
+    rglru_status st = check_dims(dims, true);
+    if (st != RGLRU_OK) return st;
+    if ((st = check_params(params)) != RGLRU_OK) return st;
+    if ((st = check_io(x, y, out)) != RGLRU_OK) return st;
+    if (state && (st = check_state(state)) != RGLRU_OK) return st;
+    if (status_out && !aligned(status_out, 16)) return RGLRU_ERR_INVALID_ARG;
+    const size_t need = rglru_prefill_workspace_size(dims);
+    if (need == 0 || need > RGLRU_NOALLOC_SCRATCH_BYTES) return RGLRU_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the area keeps the previous call's contents: the status word must start at zero (the
+    // kernels clear their own tickets and flags)
+    e = cudaMemsetAsync(scratch, 0, sizeof(rglru::DeviceStatus), s);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (rglru::fused_prefill_supported(dims))
+        e = rglru::launch_fused_prefill(dims, params, x, y, reset, state, out, scratch,
+                                        RGLRU_NOALLOC_SCRATCH_BYTES, s);
+    else
+        e = rglru::launch_prefill_generic(dims, params, x, y, reset, state, out, s);
+    if (e == cudaSuccess && status_out)
+        e = cudaMemcpyAsync(status_out, scratch, sizeof(rglru::DeviceStatus), cudaMemcpyDeviceToDevice, s);
+    return cuda_status(e);
 }
 
 rglru_status rglru_prefill_plan(const rglru_dims* dims, int* kernel, int* launches) {

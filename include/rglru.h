@@ -147,6 +147,39 @@ RGLRU_API rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_pa
                                 rglru_state* state, void* out,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Prefill for callers that cannot allocate device memory.  The pages have no counterpart:
+ * this is a deployment variant of rglru_block_prefill, not a step of the method.
+ *
+ * Some callers cannot call cudaMalloc at all -- an engine whose device memory is one pool
+ * carved up before serving starts, a plugin inside a host that owns every allocation, code
+ * that runs where an allocation would synchronise the device.  They cannot provide the
+ * workspace rglru_block_prefill asks for.  This entry point computes exactly what
+ * rglru_block_prefill computes (same kernels, same arguments minus the workspace) and
+ * takes its scratch from a fixed area that the library reserves statically on the device:
+ *   - size RGLRU_NOALLOC_SCRATCH_BYTES; a problem whose rglru_prefill_workspace_size(dims)
+ *     exceeds it is rejected with RGLRU_ERR_WORKSPACE before anything is enqueued;
+ *   - the area is part of the library's device image: it stays reserved on every device that
+ *     has loaded it (with CUDA's default lazy loading: from this entry point's first call on
+ *     that device) until the process exits;
+ *   - the first call on each device looks up the area's device address (with that device
+ *     current), so make that first call before any stream capture;
+ *   - all calls share the one area and it keeps the previous call's contents; each call
+ *     clears what must start at zero (its status word and the kernel's tickets and flags);
+ *     two calls that overlap on the GPU (different streams, or concurrent host threads) race
+ *     on it and give undefined results, so serialise them.
+ * status_out: NULL, or a 16-byte, 16-byte aligned device buffer owned by the caller; after
+ * the kernel the device status word (code, where, info0, info1 as 32-bit words) is copied
+ * into it in stream order, so that a device-side TIMEOUT / DEVICE condition can be read
+ * (rglru_read_device_status decodes it when the buffer is 256-byte aligned).
+ * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ * Errors: as rglru_block_prefill (INVALID_ARG, UNSUPPORTED, CUDA), and WORKSPACE when the
+ * problem does not fit the static area. */
+#define RGLRU_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+RGLRU_API rglru_status rglru_block_prefill_noalloc(const rglru_dims* dims,
+                                 const rglru_params* params, const void* x, const void* y,
+                                 const uint8_t* reset, rglru_state* state, void* out,
+                                 void* status_out, void* stream);
+
 /* How a call with `dims` runs: *kernel receives RGLRU_KERNEL_GENERIC (CUDA-core kernels) or
  * RGLRU_KERNEL_TENSOR (tcgen05 / TMEM kernels), *launches the number of kernel launches one
  * call enqueues.  The choice depends on dims only (the library targets sm_100a alone).
