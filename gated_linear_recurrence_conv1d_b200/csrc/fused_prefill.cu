@@ -3,32 +3,41 @@
 // One kernel does the whole block (conv -> gates -> decay -> scan -> GeLU merge -> state):
 //
 //   * a persistent CTA owns one (head, 128-channel half) "group" for its whole life; its
-//     block-diagonal gate weights W_a[h][:, half], W_x[h][:, half] are written once into
-//     tensor memory (TMEM) and used as the A operand of tcgen05.mma (TS form), so shared
-//     memory only holds streamed tiles;
+//     block-diagonal gate weights W_a[h][:, half], W_x[h][:, half], pre-scaled by 1/2 (exact
+//     in bf16), are written once into tensor memory (TMEM) and used as the A operand of
+//     tcgen05.mma (TS form), so shared memory only holds streamed tiles;
 //   * work items are (batch row, 64-token chunk) of the group, handed out by a per-group
 //     atomic ticket so every CTA of a group stays busy and an item's predecessor is always
 //     held by a running CTA;
 //   * warp roles: an x producer (TMA: x tile with a 3-token halo, and the ticket), a y producer
 //     (TMA: y tile, issued once the previous out store of that stage has left shared memory),
-//     4 conv warps (causal width-4 depthwise conv in fp32, written as the bf16 B operand in the
-//     128-byte swizzled K-major layout), 1 MMA thread (gates^T[128 ch x 64 tok] = W^T . xc^T for
-//     both gates, K = 256 in 16 steps, fp32 accumulators in TMEM), and 2 epilogue groups of 4
-//     warps, group g owning TMEM stage g, so one group's look-back wait overlaps the other
-//     group's math;
+//     4 conv warps (one 16-token quarter of the chunk each; a lane convolves 8 channels with
+//     16-byte shared-memory loads and writes them as the bf16 B operand in the 128-byte
+//     swizzled K-major layout), 1 MMA thread (D = W^T/2 . xc^T for both gates, K = 256 in 16
+//     steps, accumulated onto the gate biases that the epilogue pre-loads into TMEM), and 2
+//     epilogue groups of 4 warps, group g owning TMEM stage g;
 //   * transposed orientation: a TMEM lane is an output channel and the 64 columns are tokens,
 //     so an epilogue thread owns one channel and runs the diagonal scan along its registers
 //     (no shuffles); its first pass leaves the running (prod a, local h) of every token in
-//     TMEM, so once the carry C is known the second pass is h_t = P_t C + h_t^loc, with no
-//     serial chain; token pairs use the packed fp32x2 FMA of sm_100;
+//     TMEM, so once the carry C is known the second pass is h_t = P_t C + h_t^loc;
 //   * chunks of one sequence handled by different CTAs chain through a look-back in the spirit
 //     of Merrill & Garland ("Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016):
 //     after its first pass a chunk publishes its aggregate (prod a, local h) per channel; its
 //     carry is the inclusive state of an anchor chunk (every 32nd chunk of the row) followed by
 //     the aggregates of the chunks in between, applied in a fixed order so the result does not
-//     depend on timing; it then publishes its own inclusive state and replays the scan from
-//     TMEM with the true carry.  Every wait is bounded by %globaltimer; on expiry the kernel
-//     latches RGLRU_ERR_TIMEOUT in the workspace status word and drains.
+//     depend on timing.  Every wait is bounded by %globaltimer; on expiry the kernel latches
+//     RGLRU_ERR_TIMEOUT in the workspace status word and drains.
+//
+// Element-wise arithmetic (one transcendental per gate, one square root, one for GeLU):
+//   D_a = (g_a + b_a) / 2, D_x = (g_x + b_x) / 2 come out of the MMA;
+//   r_t = (1 + tanh D_a) / 2 and l_t = c r_t log sigma(Lambda) = hK (1 + tanh D_a) with
+//   hK = c log sigma(Lambda) / 2;  E = expm1(l_t) = l(1 + l/2 + l^2/6) (|l| <= 1/8: the
+//   truncation, summed over the ~1/|l| tokens a decay acts on, stays below 1e-4), a_t = 1 + E,
+//   sqrt(1 - a_t^2) / 2 = sqrt(E (-E/4 - 1/2)) (no cancellation near a_t = 1);
+//   i_t x_t sqrt(1 - a^2) = w (1 + tanh D_x) with w = x_t sqrt(1 - a^2) / 2;
+//   GeLU(y) = y (1 + tanh(y (k1 + k3 y^2))) / 2, k1 / k3 fitted to the exact y Phi(y)
+//   (|error in Phi| <= 1.5e-4; the tanh form of the flag uses k1 = sqrt(2/pi), k3 = 0.044715 k1).
+// Channels with |c log sigma(Lambda)| > 1/8, resets and a ragged last chunk take a general path.
 //
 // Arithmetic follows "Griffin Guide: RecurrentGemma, RG-LRU & Hybrid Attention": recurrence /
 // input gates, a_t = a^(c r_t) in log space, h_t = a_t h_{t-1} + sqrt(1 - a_t^2)(i_t x_t)
@@ -61,11 +70,11 @@ constexpr int XROWS = L + kHist;        // x tile rows incl. the 3-token halo
 constexpr int KSTEPS = DH / 16;         // MMA K steps
 constexpr int STAGES = 2;
 constexpr int SLOTS = 8;                // ring of item ids, indexed by iteration
-constexpr int kSub = 8;                 // tokens per TMEM load in the epilogue
+constexpr int kBlk = 8;                 // tokens per TMEM load block in the epilogue
+constexpr int kConvTok = L / 4;         // tokens per conv warp
 
-// warp roles: 0-3 conv (K block = warp), 4-11 epilogue (TMEM lane quarter = warp % 4, group =
-// stage = (warp - 4) / 4), 12 x producer (x tiles and tickets), 13 y producer, 14 MMA.  The two
-// producers spin on different barriers, so they live in different warps.
+// warp roles: 0-3 conv (token quarter = warp), 4-11 epilogue (TMEM lane quarter = warp % 4,
+// group = stage = (warp - 4) / 4), 12 x producer (x tiles and tickets), 13 y producer, 14 MMA.
 constexpr int kConvWarps = 4, kEpiWarps = 8, kEpiGroup = 4;
 constexpr int kWarpEpi0 = 4, kWarpProdX = 12, kWarpProdY = 13, kWarpMma = 14;
 constexpr int kThreads = 15 * 32;
@@ -85,8 +94,8 @@ constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;               // slots, TMEM b
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;          // + slack for 1024 alignment
 static_assert(2 * HALF * DH * 2 <= OFF_Y, "weight staging reuses the B and x tiles");
 
-// TMEM columns: [0,128) A = W_a^T (bf16 pairs), [128,256) A = W_x^T, then per stage
-// 128 columns: gate a accumulators [0,64) and gate x accumulators [64,128).
+// TMEM columns: [0,128) A = W_a^T / 2 (bf16 pairs), [128,256) A = W_x^T / 2, then per stage
+// 128 columns: D_a [0,64) and D_x [64,128); the first pass overwrites them with P and H.
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_A = 0, TM_D = 256;
 
@@ -147,19 +156,17 @@ struct WaitCtx {
 
 __device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, WaitCtx w, unsigned where) {
     const uint64_t t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
+    for (;;) {
         if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;   // sleeps up to 100 us
-        {
-            if (*w.abort) return false;
-            if (*(volatile unsigned*)&w.status->code != 0) {
-                *w.abort = 1;
-                return false;
-            }
-            if (globaltimer_ns() - t0 > w.timeout_ns) {
-                latch_status(w.status, RGLRU_ERR_TIMEOUT, where, blockIdx.x, parity);
-                *w.abort = 1;
-                return false;
-            }
+        if (*w.abort) return false;
+        if (*(volatile unsigned*)&w.status->code != 0) {
+            *w.abort = 1;
+            return false;
+        }
+        if (globaltimer_ns() - t0 > w.timeout_ns) {
+            latch_status(w.status, RGLRU_ERR_TIMEOUT, where, blockIdx.x, parity);
+            *w.abort = 1;
+            return false;
         }
     }
 }
@@ -205,126 +212,99 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&p);
 }
-
-__device__ __forceinline__ float rcp_approx(float x) {
+__device__ __forceinline__ float sqrt_approx(float x) {
     float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
-}
-__device__ __forceinline__ float rsqrt_approx(float x) {
-    float r;
-    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
 }
 
-// sigma(z) = 1 / (1 + 2^(-z log2 e)) with the ex2 / rcp approximations: relative error of a
-// few ulp over the whole range (the recurrence gate needs it: sqrt(1 - a^2) ~ sqrt(r) for
-// small r).
-__device__ __forceinline__ float sigmoid_fast(float z) {
-    return rcp_approx(1.0f + ex2_approx(-1.4426950408889634f * z));
-}
-// sigma(z) = (1 + tanh(z / 2)) / 2: absolute error ~2.5e-4, enough for the input gate, whose
-// error enters h only additively through i_t x_t.
-__device__ __forceinline__ float sigmoid_tanh(float z) {
-    return fmaf(0.5f, tanh_approx(0.5f * z), 0.5f);
-}
-
-// Decay a = e^l and sqrt(1 - a^2) for l = c r log sigma(Lambda) <= 0.  When the channel's
-// |c log sigma(Lambda)| <= 1/8 (so |l| <= 1/8): em = expm1(l) from its Taylor series (terms
-// l^k / k!, truncation below 1e-8 relative), a = 1 + em, 1 - a^2 = -em (2 + em) without
-// cancellation.  Otherwise a = 2^(l log2 e) and 1 - a^2 directly, switching to the series when
-// |l| < 1/8.
-__device__ __forceinline__ void decay_beta(float l, bool small_range, float& a, float& beta) {
-    float v;
-    if (small_range || l > -0.125f) {
-        float p = fmaf(l, 1.0f / 720.0f, 1.0f / 120.0f);
-        p = fmaf(l, p, 1.0f / 24.0f);
-        p = fmaf(l, p, 1.0f / 6.0f);
-        p = fmaf(l, p, 0.5f);
-        p = fmaf(l, p, 1.0f);
-        const float em = l * p;
-        a = 1.0f + em;
-        v = -em * (2.0f + em);
-    } else {
-        a = ex2_approx(l * 1.4426950408889634f);
-        v = fmaf(-a, a, 1.0f);
-    }
-    beta = v > 0.0f ? v * rsqrt_approx(v) : 0.0f;
-}
-
-// Packed helpers (two tokens per instruction on the fp32x2 pipe of sm_100).
+// Packed helpers (two tokens per instruction on the fp32x2 path of sm_100).
 __device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 tanh2(float2 v) { return make_float2(tanh_approx(v.x), tanh_approx(v.y)); }
+__device__ __forceinline__ float2 sqrt2(float2 v) { return make_float2(sqrt_approx(v.x), sqrt_approx(v.y)); }
 
-// Fast path of gates + decay + normalised input for a channel with |c log sigma(Lambda)| <= 1/8,
-// two tokens at a time.  With s = 1 + e^{-(g_a + b_a)}: sqrt(r) = rsqrt(s) and r = sqrt(r)^2 (so
-// one ex2 and one rsqrt give both); l = c_lab r; a = 1 + expm1(l) from the Taylor series of
-// expm1 (terms l^k / k!); sqrt(1 - a^2) = sqrt(-2 l) sqrt(expm1(2l) / 2l) = K sqrt(r) Q(l) with
-// K = sqrt(-2 c_lab) and Q(l) = sqrt(expm1(2l) / 2l) from its Taylor series in 2l,
-// 1 + x/4 + 5x^2/96 + x^3/128 + 79x^4/92160 (relative error < 1e-7 for |2l| <= 1/4).
-__device__ __forceinline__ void gates_pair(float2 ga, float2 gx, float nbl, float c_lab, float K,
-                                           float bxh, float2 xc, float2& a, float2& u) {
-    const float2 z = fma2(ga, f2(-1.4426950408889634f), f2(nbl));
-    const float2 s = add2(make_float2(ex2_approx(z.x), ex2_approx(z.y)), f2(1.0f));
-    const float2 rs = make_float2(rsqrt_approx(s.x), rsqrt_approx(s.y));
-    const float2 l = mul2(mul2(rs, rs), f2(c_lab));
-    float2 p = fma2(l, f2(1.0f / 720.0f), f2(1.0f / 120.0f));
-    p = fma2(l, p, f2(1.0f / 24.0f));
-    p = fma2(l, p, f2(1.0f / 6.0f));
-    p = fma2(l, p, f2(0.5f));
+// TMEM block load / store of kBlk consecutive columns (32 lanes x 32 bits)
+__device__ __forceinline__ void tmem_ldb(uint32_t taddr, float (&v)[kBlk]) { tmem_ld8(taddr, v); }
+__device__ __forceinline__ void tmem_stbf(uint32_t taddr, const float (&v)[kBlk]) { tmem_st8f(taddr, v); }
+
+// Fast path of gates + decay + normalised input for two tokens of a channel with
+// |c log sigma(Lambda)| <= 1/8 (so |l| <= 1/8).  In: D_a, D_x (pre-scaled gate
+// pre-activations), xc (the bf16-rounded conv output).  Out: a_t and u_t = sqrt(1-a^2) i x.
+__device__ __forceinline__ void gates_pair(float2 da, float2 dx, float2 hk, float2 xc, float2& a, float2& u) {
+    const float2 ta = tanh2(da);
+    const float2 l = fma2(ta, hk, hk);                                  // c r log sigma(Lambda)
+    float2 p = fma2(l, f2(1.0f / 6.0f), f2(0.5f));
     p = fma2(l, p, f2(1.0f));
-    a = fma2(l, p, f2(1.0f));
-    float2 q = fma2(l, f2(79.0f / 5760.0f), f2(1.0f / 16.0f));
-    q = fma2(l, q, f2(5.0f / 24.0f));
-    q = fma2(l, q, f2(0.5f));
-    q = fma2(l, q, f2(1.0f));
-    const float2 beta = mul2(mul2(rs, q), f2(K));
-    const float2 zi = fma2(gx, f2(0.5f), f2(bxh));
-    const float2 ig = fma2(make_float2(tanh_approx(zi.x), tanh_approx(zi.y)), f2(0.5f), f2(0.5f));
-    u = mul2(mul2(beta, ig), xc);
+    const float2 e = mul2(l, p);                                        // expm1(l)
+    a = add2(e, f2(1.0f));
+    const float2 q = fma2(e, f2(-0.25f), f2(-0.5f));
+    const float2 bh = sqrt2(mul2(e, q));                                // sqrt(1 - a^2) / 2
+    const float2 ti = tanh2(dx);
+    const float2 w = mul2(bh, xc);
+    u = fma2(w, ti, w);                                                 // sqrt(1-a^2) i x
 }
 
-// GeLU(v) = v Phi(v).  Exact form: Phi from erf of Abramowitz & Stegun 7.1.28,
-// erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 for x >= 0 (|error| <= 3e-7), one reciprocal.
-// Tanh form: 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))).
-__device__ __forceinline__ float gelu_fast(float v, int tanh_form) {
-    if (tanh_form) {
-        const float k = 0.79788456080286535588f;
-        return 0.5f * v * (1.0f + tanh_approx(k * fmaf(0.044715f * v, v * v, v)));
+// General path of one token: any |c log sigma(Lambda)|.
+__device__ __forceinline__ void gates_one(float da, float dx, float hk, float xc, float& a, float& u) {
+    const float l = fmaf(tanh_approx(da), hk, hk);
+    float e;
+    if (l > -0.125f) {
+        float p = fmaf(l, 1.0f / 24.0f, 1.0f / 6.0f);
+        p = fmaf(l, p, 0.5f);
+        p = fmaf(l, p, 1.0f);
+        e = l * p;
+    } else {
+        e = ex2_approx(l * 1.4426950408889634f) - 1.0f;
     }
-    const float x = fabsf(v) * 0.70710678118654752f;
-    float p = fmaf(x, 0.0000430638f, 0.0002765672f);
-    p = fmaf(x, p, 0.0001520143f);
-    p = fmaf(x, p, 0.0092705272f);
-    p = fmaf(x, p, 0.0422820123f);
-    p = fmaf(x, p, 0.0705230784f);
-    p = fmaf(x, p, 1.0f);
-    p = p * p;
-    p = p * p;
-    p = p * p;
-    p = p * p;                                        // (1 + ...)^16
-    const float half_erfc = 0.5f * rcp_approx(p);     // (1 - erf(x)) / 2
-    return v * (v >= 0.0f ? 1.0f - half_erfc : half_erfc);
+    a = 1.0f + e;
+    const float bh = sqrt_approx(e * fmaf(e, -0.25f, -0.5f));
+    const float w = bh * xc;
+    u = fmaf(w, tanh_approx(dx), w);
 }
 
-// GeLU of two values at once (packed fp32x2 for the polynomial part).
-__device__ __forceinline__ float2 gelu_pair(float2 v, int tanh_form) {
-    if (tanh_form) return make_float2(gelu_fast(v.x, 1), gelu_fast(v.y, 1));
-    const float2 x = mul2(make_float2(fabsf(v.x), fabsf(v.y)), f2(0.70710678118654752f));
-    float2 p = fma2(x, f2(0.0000430638f), f2(0.0002765672f));
-    p = fma2(x, p, f2(0.0001520143f));
-    p = fma2(x, p, f2(0.0092705272f));
-    p = fma2(x, p, f2(0.0422820123f));
-    p = fma2(x, p, f2(0.0705230784f));
-    p = fma2(x, p, f2(1.0f));
-    p = mul2(p, p);
-    p = mul2(p, p);
-    p = mul2(p, p);
-    p = mul2(p, p);
-    const float2 e = mul2(make_float2(rcp_approx(p.x), rcp_approx(p.y)), f2(0.5f));
-    return make_float2(v.x * (v.x >= 0.0f ? 1.0f - e.x : e.x), v.y * (v.y >= 0.0f ? 1.0f - e.y : e.y));
+// out = h * GeLU(y) for two tokens, GeLU(y) = (y/2)(1 + tanh(w(y))), w = (y/2)(K1 + K3 (y/2)^2).
+__device__ __forceinline__ float2 merge_pair(float2 h, float2 y, float k1, float k3) {
+    const float2 hy = mul2(y, f2(0.5f));
+    const float2 s = mul2(hy, hy);
+    const float2 w = mul2(hy, fma2(s, f2(k3), f2(k1)));
+    const float2 t = tanh2(w);
+    const float2 m = mul2(h, hy);
+    return fma2(m, t, m);
+}
+
+// Bit j of the result = reset[t0 + j] != 0 for the 64 tokens of a chunk (0 past the end).
+__device__ __forceinline__ uint64_t chunk_reset_mask(const uint8_t* row, int t0, int T, int lane) {
+    const bool r0 = t0 + lane < T && row[t0 + lane] != 0;
+    const bool r1 = t0 + 32 + lane < T && row[t0 + 32 + lane] != 0;
+    const uint32_t lo = __ballot_sync(0xffffffffu, r0);
+    const uint32_t hi = __ballot_sync(0xffffffffu, r1);
+    return (uint64_t)lo | ((uint64_t)hi << 32);
+}
+
+// Conv of one token for a lane's 8 channels: y = cb + w0 h0 + w1 h1 + w2 h2 + w3 xv, as bf16.
+struct Vec8 {
+    float2 v[4];
+};
+__device__ __forceinline__ Vec8 unpack8(uint4 r) {
+    Vec8 o;
+    o.v[0] = make_float2(bf16lo(r.x), bf16hi(r.x));
+    o.v[1] = make_float2(bf16lo(r.y), bf16hi(r.y));
+    o.v[2] = make_float2(bf16lo(r.z), bf16hi(r.z));
+    o.v[3] = make_float2(bf16lo(r.w), bf16hi(r.w));
+    return o;
+}
+__device__ __forceinline__ uint4 pack8(const Vec8& h) {
+    return make_uint4(pack_bf16x2(h.v[0].x, h.v[0].y), pack_bf16x2(h.v[1].x, h.v[1].y),
+                      pack_bf16x2(h.v[2].x, h.v[2].y), pack_bf16x2(h.v[3].x, h.v[3].y));
+}
+__device__ __forceinline__ Vec8 zero8() {
+    Vec8 o;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o.v[i] = make_float2(0.f, 0.f);
+    return o;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -349,6 +329,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     const int head = group >> 1, half = group & 1;
     const int W = a.H * DH;
     const size_t lb_base = (size_t)group * a.items;
+    const bool bias_in_acc = a.b_a != nullptr || a.b_x != nullptr;
 
     // ---- set-up ------------------------------------------------------------------------------
     if (threadIdx.x == 0) {
@@ -378,17 +359,20 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         prefetch_tensormap(&map_y);
         prefetch_tensormap(&map_out);
     }
-    // stage this CTA's gate weights W_g[head][i][half*128 + o] (o contiguous) in shared memory
-    // with coalesced 16-byte loads: gate a at byte 0, gate x at byte 65536 (B and x tiles are
-    // still unused)
+    // stage this CTA's gate weights W_g[head][i][half*128 + o] / 2 (o contiguous) in shared
+    // memory with coalesced 16-byte loads: gate a at byte 0, gate x at byte 65536 (B and x
+    // tiles are still unused); halving a bf16 is exact
     if (warp < kConvWarps + kEpiWarps) {
         const int tid = threadIdx.x;                       // 0..383
         for (int e = tid; e < 2 * DH * (HALF / 8); e += (kConvWarps + kEpiWarps) * 32) {
             const int g = e / (DH * (HALF / 8)), r = e % (DH * (HALF / 8));
             const int i = r / (HALF / 8), o8 = r % (HALF / 8);
             const __nv_bfloat16* src = (g ? a.w_x : a.w_a) + ((size_t)head * DH + i) * DH + half * HALF + o8 * 8;
-            *reinterpret_cast<uint4*>(smem + g * (HALF * DH * 2) + (i * HALF + o8 * 8) * 2) =
-                __ldg(reinterpret_cast<const uint4*>(src));
+            uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
+            uint32_t* vv = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) vv[k] = pack_bf16x2(0.5f * bf16lo(vv[k]), 0.5f * bf16hi(vv[k]));
+            *reinterpret_cast<uint4*>(smem + g * (HALF * DH * 2) + (i * HALF + o8 * 8) * 2) = v;
         }
     }
     tc_fence_before();
@@ -399,7 +383,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
 
     if (warp >= kWarpEpi0 && warp < kWarpEpi0 + kEpiWarps) {
         // weights -> TMEM A operand: lane m, column j holds (W[2j][m], W[2j+1][m]); group 0 of
-        // each lane quarter writes gate a, group 1 gate x
+        // each lane quarter writes gate a, group 1 gate x.  Then each group pre-loads the gate
+        // biases of its accumulator stage.
         const int q = warp & 3, g = (warp - kWarpEpi0) >> 2, m = q * 32 + lane;
         const unsigned short* ws = reinterpret_cast<const unsigned short*>(smem + g * (HALF * DH * 2)) + m;
 #pragma unroll 1
@@ -411,6 +396,20 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 r[j] = (uint32_t)ws[i * HALF] | ((uint32_t)ws[(i + 1) * HALF] << 16);
             }
             tmem_st16(tmem + ((uint32_t)(q * 32) << 16) + TM_A + g * 128 + j0, r);
+        }
+        if (bias_in_acc) {
+            const int ch = head * DH + half * HALF + m;
+            const uint32_t ba = __float_as_uint(a.b_a ? 0.5f * a.b_a[ch] : 0.f);
+            const uint32_t bx = __float_as_uint(a.b_x ? 0.5f * a.b_x[ch] : 0.f);
+            uint32_t ra[16], rx[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) { ra[j] = ba; rx[j] = bx; }
+            const uint32_t d = tmem + ((uint32_t)(q * 32) << 16) + TM_D + g * 128;
+#pragma unroll
+            for (int j0 = 0; j0 < L; j0 += 16) {
+                tmem_st16(d + j0, ra);
+                tmem_st16(d + L + j0, rx);
+            }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -511,7 +510,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks) {
                         const uint64_t bd = desc_k_sw128(bt + (ks >> 2) * KBLK_BYTES + (ks & 3) * 32);
-                        mma_ts(d, tmem + TM_A + g * 128 + ks * 8, bd, idesc, ks > 0 ? 1u : 0u);
+                        mma_ts(d, tmem + TM_A + g * 128 + ks * 8, bd, idesc, (bias_in_acc || ks > 0) ? 1u : 0u);
                     }
                 }
                 mma_commit(bars.acc_full[st]);
@@ -525,15 +524,24 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         }
     } else if (warp < kConvWarps) {
         // ================================ conv warps ==========================================
-        const int kb = warp;                              // K block of the B tile
-        const int p = kb * 32 + lane;                     // channel pair 2p, 2p+1 of the head
-        const int chg = head * DH + 2 * p;                // global channel of the pair
-        float2 w[kConvWidth];
+        // warp w convolves tokens [16w, 16w + 16) of the chunk; lane l channels 8l .. 8l+7 of the
+        // head (K block l / 8, 16-byte chunk l % 8 of the B tile's 128-byte rows)
+        const int j0 = warp * kConvTok;
+        const int cl = lane * 8;                          // channel within the head
+        const int chg = head * DH + cl;                   // global channel
+        float2 w[kConvWidth][4];
 #pragma unroll
         for (int k = 0; k < kConvWidth; ++k)
-            w[k] = make_float2(a.conv_w[(size_t)k * W + chg], a.conv_w[(size_t)k * W + chg + 1]);
-        const float2 cb = make_float2(a.conv_b ? a.conv_b[chg] : 0.f, a.conv_b ? a.conv_b[chg + 1] : 0.f);
-        const bool own_tail = (p >> 6) == half;          // this CTA writes these tail channels
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                w[k][i] = make_float2(a.conv_w[(size_t)k * W + chg + 2 * i], a.conv_w[(size_t)k * W + chg + 2 * i + 1]);
+        float2 cb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            cb[i] = a.conv_b ? make_float2(a.conv_b[chg + 2 * i], a.conv_b[chg + 2 * i + 1]) : make_float2(0.f, 0.f);
+        const bool own_tail = (lane >> 4) == half;       // this CTA writes these tail channels
+        const uint32_t kb_off = (uint32_t)(lane >> 3) * KBLK_BYTES;
+        const uint32_t cchunk = lane & 7;
         for (int n = 0;; ++n) {
             const int st = n & 1;
             const uint32_t ph = (n >> 1) & 1;
@@ -547,61 +555,54 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             }
             const int b = k / a.NC, c = k % a.NC, t0 = c * L;
             const int nt = min(L, a.T - t0);
-            const uint8_t* rst = a.reset ? a.reset + (size_t)b * a.T : nullptr;
-            const uint8_t* xt = smem + OFF_X + st * X_BYTES + 4 * p;
-            uint8_t* bt = smem + OFF_B + st * B_BYTES;
+            const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
+            const uint64_t rmask = rrow ? chunk_reset_mask(rrow, t0, a.T, lane) : 0ull;
+            const uint8_t* xt = smem + OFF_X + st * X_BYTES + cl * 2;
+            uint8_t* bt = smem + OFF_B + st * B_BYTES + kb_off;
             auto xrow = [&](int r) {                      // x tile row r = token t0 - 3 + r
-                const uint32_t v = *reinterpret_cast<const uint32_t*>(xt + r * DH * 2);
-                return make_float2(bf16lo(v), bf16hi(v));
+                return unpack8(*reinterpret_cast<const uint4*>(xt + r * DH * 2));
             };
-            float2 h0, h1, h2;                            // window x_{t-3}, x_{t-2}, x_{t-1}
-            if (c == 0) {
+            Vec8 h0, h1, h2;                              // window x_{t-3}, x_{t-2}, x_{t-1}
+            if (c == 0 && j0 == 0) {
                 if (a.tail_state) {
                     const __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
-                    const uint32_t v0 = *reinterpret_cast<const uint32_t*>(tl);
-                    const uint32_t v1 = *reinterpret_cast<const uint32_t*>(tl + W);
-                    const uint32_t v2 = *reinterpret_cast<const uint32_t*>(tl + 2 * W);
-                    h0 = make_float2(bf16lo(v0), bf16hi(v0));
-                    h1 = make_float2(bf16lo(v1), bf16hi(v1));
-                    h2 = make_float2(bf16lo(v2), bf16hi(v2));
+                    h0 = unpack8(*reinterpret_cast<const uint4*>(tl));
+                    h1 = unpack8(*reinterpret_cast<const uint4*>(tl + W));
+                    h2 = unpack8(*reinterpret_cast<const uint4*>(tl + 2 * W));
                 } else {
-                    h0 = h1 = h2 = make_float2(0.f, 0.f);
+                    h0 = h1 = h2 = zero8();
                 }
             } else {
-                h0 = xrow(0);
-                h1 = xrow(1);
-                h2 = xrow(2);
-                if (rst) {
-                    if (rst[t0 - 1]) h0 = h1 = make_float2(0.f, 0.f);
-                    if (rst[t0 - 2]) h0 = make_float2(0.f, 0.f);
+                h0 = xrow(j0);
+                h1 = xrow(j0 + 1);
+                h2 = xrow(j0 + 2);
+                if (rrow) {
+                    // a segment that starts at token j0-1 (j0-2) empties the older history
+                    const int p1 = t0 + j0 - 1, p2 = t0 + j0 - 2;
+                    if (p1 < a.T && rrow[p1]) h0 = h1 = zero8();
+                    if (p2 >= 0 && p2 < a.T && rrow[p2]) h0 = zero8();
                 }
             }
-            float2 f0 = h0, f1 = h1, f2v = h2;            // final window (the tail of the row)
-            if (!rst && nt == L) {
-                // fast path: a full chunk without segment resets
-#pragma unroll 8
-                for (int t = 0; t < L; ++t) {
-                    const float2 xv = xrow(t + kHist);
-                    float2 y = fma2(w[0], h0, cb);
-                    y = fma2(w[1], h1, y);
-                    y = fma2(w[2], h2, y);
-                    y = fma2(w[3], xv, y);
-                    *reinterpret_cast<uint32_t*>(bt + b_tile_offset(t, 2 * p)) = pack_bf16x2(y.x, y.y);
-                    h0 = h1; h1 = h2; h2 = xv;
+            uint4 fw[3];                                  // final window (the tail of the row), bf16
+            const bool has_last = nt - 1 >= j0 && nt - 1 < j0 + kConvTok;
+#pragma unroll 4
+            for (int jj = 0; jj < kConvTok; ++jj) {
+                const int j = j0 + jj;
+                const Vec8 xv = xrow(j + kHist);
+                if ((rmask >> j) & 1ull) h0 = h1 = h2 = zero8();
+                uint4 o;
+                uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float2 y = fma2(w[0][i], h0.v[i], cb[i]);
+                    y = fma2(w[1][i], h1.v[i], y);
+                    y = fma2(w[2][i], h2.v[i], y);
+                    y = fma2(w[3][i], xv.v[i], y);
+                    op[i] = pack_bf16x2(y.x, y.y);
                 }
-                f0 = h0; f1 = h1; f2v = h2;
-            } else {
-                for (int t = 0; t < L; ++t) {
-                    const float2 xv = xrow(t + kHist);
-                    if (rst && t < nt && rst[t0 + t]) h0 = h1 = h2 = make_float2(0.f, 0.f);
-                    float2 y = fma2(w[0], h0, cb);
-                    y = fma2(w[1], h1, y);
-                    y = fma2(w[2], h2, y);
-                    y = fma2(w[3], xv, y);
-                    *reinterpret_cast<uint32_t*>(bt + b_tile_offset(t, 2 * p)) = pack_bf16x2(y.x, y.y);
-                    h0 = h1; h1 = h2; h2 = xv;
-                    if (t == nt - 1) { f0 = h0; f1 = h1; f2v = h2; }
-                }
+                *reinterpret_cast<uint4*>(bt + (j >> 3) * 1024 + (j & 7) * 128 + ((cchunk ^ (j & 7)) << 4)) = o;
+                h0 = h1; h1 = h2; h2 = xv;
+                if (has_last && j == nt - 1) { fw[0] = pack8(h0); fw[1] = pack8(h1); fw[2] = pack8(h2); }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -610,14 +611,24 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 mbar_arrive(bars.b_full[st]);
             }
             // final conv history of the sequence, once its first chunk has read the old one
-            if (a.tail_state && c == a.NC - 1 && own_tail) {
-                bool ok = true;
-                if (c > 0) ok = wait_flag(a.lb_flags + (lb_base + (size_t)b * a.NC) * 4, FLAG_AGG, wc, 8) != 0;
-                if (ok) {
+            if (a.tail_state && c == a.NC - 1 && has_last) {
+                bool ok;
+                if (c > 0) {
+                    unsigned f = 0;
+                    if (lane == 0) f = wait_flag(a.lb_flags + (lb_base + (size_t)b * a.NC) * 4, FLAG_AGG, wc, 8);
+                    ok = __shfl_sync(0xffffffffu, f, 0) != 0;
+                } else {
+                    // a row of one chunk: warp 0 read the old history in this very item; once
+                    // every conv warp has arrived on b_full, that read is done
+                    ok = wait_bar(bars.b_full[st], ph, wc, 18);
+                }
+                if (ok && own_tail) {
                     __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
-                    *reinterpret_cast<uint32_t*>(tl) = pack_bf16x2(f0.x, f0.y);
-                    *reinterpret_cast<uint32_t*>(tl + W) = pack_bf16x2(f1.x, f1.y);
-                    *reinterpret_cast<uint32_t*>(tl + 2 * W) = pack_bf16x2(f2v.x, f2v.y);
+#pragma unroll
+                    for (int r = 0; r < 3; ++r) {
+                        const uint4 o = fw[r];
+                        *reinterpret_cast<uint4*>(tl + (size_t)r * W) = o;
+                    }
                 }
             }
         }
@@ -630,19 +641,26 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         const int chl = half * HALF + m;                 // channel within the head
         const int ch = head * DH + chl;                  // global channel
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        const float lab = log_sigmoid_acc(a.lambda[ch]);
-        const float c_lab = a.c * lab;                   // log a_t = c_lab * r_t
-        const bool small_range = c_lab >= -0.125f;
-        const float ba = a.b_a ? a.b_a[ch] : 0.f;
-        const float bx = a.b_x ? a.b_x[ch] : 0.f;
-        const float nbl = -ba * 1.4426950408889634f;   // fast path constants
-        const float bxh = 0.5f * bx;
-        const float Kb = sqrtf(fmaxf(-2.0f * c_lab, 0.0f));
+        const float hk = 0.5f * a.c * log_sigmoid_acc(a.lambda[ch]);   // l_t = hk (1 + tanh D_a)
+        const bool small_range = hk >= -0.0625f;
+        const float2 hk2 = f2(hk);
         const int tanh_form = a.gelu_tanh;
+        // GeLU(y) = (y/2)(1 + tanh((y/2)(K1 + K3 (y/2)^2)))
+        const float gk1 = tanh_form ? 2.0f * 0.79788456080286535588f : 2.0f * 0.79879267f;
+        const float gk3 = tanh_form ? 8.0f * 0.044715f * 0.79788456080286535588f : 8.0f * 0.03528805f;
+        const uint32_t ba_bits = __float_as_uint(a.b_a ? 0.5f * a.b_a[ch] : 0.f);
+        const uint32_t bx_bits = __float_as_uint(a.b_x ? 0.5f * a.b_x[ch] : 0.f);
         const bool withhold_hook = (a.flags & RGLRU_FLAG_TEST_WITHHOLD) && group == 0;
         const uint8_t* bt = smem + OFF_B + st * B_BYTES;
         uint8_t* yt = smem + OFF_Y + st * Y_BYTES + 2 * m;
         const uint32_t dcol = tmem + lane_off + TM_D + st * 128;
+        // B-tile byte offsets of this channel for tokens 0..7 (token t: boff[t & 7] + (t >> 3) * 1024)
+        uint32_t boff[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) boff[r] = b_tile_offset(r, chl);
+        auto xc_at = [&](int t) {
+            return __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(bt + boff[t & 7] + (t >> 3) * 1024) << 16);
+        };
 
         for (int n = eg;; n += 2) {
             const uint32_t ph = (n >> 1) & 1;
@@ -652,7 +670,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             tc_fence_after();
             const int b = k / a.NC, c = k % a.NC, t0 = c * L;
             const int nt = min(L, a.T - t0);
-            const uint8_t* rst = a.reset ? a.reset + (size_t)b * a.T + t0 : nullptr;
+            const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
+            const uint64_t rmask = rrow ? chunk_reset_mask(rrow, t0, a.T, lane) : 0ull;
             const size_t kb_item = lb_base + (size_t)b * a.NC;       // first chunk of this row
             const bool withhold = withhold_hook && k == 0;
             unsigned* myflag = a.lb_flags + (lb_base + k) * 4 + q;
@@ -660,70 +679,63 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             // ---- pass 1: gates, decay and normalised input; TMEM keeps the running product of
             //      the decays P_t and the running local state H_t (from zero) of every token
             float aggA = 1.f, aggH = 0.f;
-            const bool fast = !rst && nt == L && __all_sync(0xffffffffu, small_range);
+            const bool fast = nt == L && __all_sync(0xffffffffu, small_range);
             if (fast) {
-                float ga[kSub], gx[kSub], gan[kSub], gxn[kSub];
-                tmem_ld8(dcol, ga);
-                tmem_ld8(dcol + L, gx);
+                float da[kBlk], dx[kBlk], dan[kBlk], dxn[kBlk];
+                tmem_ldb(dcol, da);
+                tmem_ldb(dcol + L, dx);
                 tmem_wait_ld();
 #pragma unroll 1
-                for (int j0 = 0; j0 < L; j0 += kSub) {
-                    if (j0 + kSub < L) {                    // next sub-block in flight meanwhile
-                        tmem_ld8(dcol + j0 + kSub, gan);
-                        tmem_ld8(dcol + L + j0 + kSub, gxn);
+                for (int j0 = 0; j0 < L; j0 += kBlk) {
+                    if (j0 + kBlk < L) {                    // next block in flight meanwhile
+                        tmem_ldb(dcol + j0 + kBlk, dan);
+                        tmem_ldb(dcol + L + j0 + kBlk, dxn);
                     }
-                    uint32_t ra[kSub], ru[kSub];
 #pragma unroll
-                    for (int j = 0; j < kSub; j += 2) {
-                        const int t = j0 + j;
-                        const float2 xc = make_float2(
-                            __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(bt + b_tile_offset(t, chl)) << 16),
-                            __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(bt + b_tile_offset(t + 1, chl)) << 16));
+                    for (int j = 0; j < kBlk; j += 2) {
                         float2 at, u;
-                        gates_pair(make_float2(ga[j], ga[j + 1]), make_float2(gx[j], gx[j + 1]), nbl, c_lab, Kb,
-                                   bxh, xc, at, u);
+                        gates_pair(make_float2(da[j], da[j + 1]), make_float2(dx[j], dx[j + 1]), hk2,
+                                   make_float2(xc_at(j0 + j), xc_at(j0 + j + 1)), at, u);
+                        if (rmask) {                                     // h_{t-1} := 0 at a reset
+                            if ((rmask >> (j0 + j)) & 1ull) at.x = 0.f;
+                            if ((rmask >> (j0 + j + 1)) & 1ull) at.y = 0.f;
+                        }
                         aggH = fmaf(at.x, aggH, u.x);
                         aggA *= at.x;
-                        ra[j] = __float_as_uint(aggA);
-                        ru[j] = __float_as_uint(aggH);
+                        da[j] = aggA;
+                        dx[j] = aggH;
                         aggH = fmaf(at.y, aggH, u.y);
                         aggA *= at.y;
-                        ra[j + 1] = __float_as_uint(aggA);
-                        ru[j + 1] = __float_as_uint(aggH);
+                        da[j + 1] = aggA;
+                        dx[j + 1] = aggH;
                     }
-                    tmem_st8(dcol + j0, ra);
-                    tmem_st8(dcol + L + j0, ru);
+                    tmem_stbf(dcol + j0, da);
+                    tmem_stbf(dcol + L + j0, dx);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < kSub; ++j) { ga[j] = gan[j]; gx[j] = gxn[j]; }
+                    for (int j = 0; j < kBlk; ++j) { da[j] = dan[j]; dx[j] = dxn[j]; }
                 }
             } else {
 #pragma unroll 1
-                for (int j0 = 0; j0 < L; j0 += kSub) {
-                    float ga[kSub], gx[kSub];
-                    tmem_ld8(dcol + j0, ga);
-                    tmem_ld8(dcol + L + j0, gx);
+                for (int j0 = 0; j0 < L; j0 += kBlk) {
+                    float da[kBlk], dx[kBlk];
+                    tmem_ldb(dcol + j0, da);
+                    tmem_ldb(dcol + L + j0, dx);
                     tmem_wait_ld();
-                    uint32_t ra[kSub], ru[kSub];
 #pragma unroll
-                    for (int j = 0; j < kSub; ++j) {
+                    for (int j = 0; j < kBlk; ++j) {
                         const int t = j0 + j;
-                        const float xc = __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(
-                                                             bt + b_tile_offset(t, chl)) << 16);
-                        const float r = sigmoid_fast(ga[j] + ba);
-                        float at, beta;
-                        decay_beta(c_lab * r, small_range, at, beta);
-                        const float ig = sigmoid_tanh(gx[j] + bx);
-                        float u = beta * (ig * xc);
-                        if (rst && t < nt && rst[t]) at = 0.f;                // h_{t-1} := 0
-                        if (t >= nt) { at = 1.f; u = 0.f; }                   // padding: identity
+                        float at, u;
+                        gates_one(da[j], dx[j], hk, xc_at(t), at, u);
+                        if ((rmask >> t) & 1ull) at = 0.f;                 // h_{t-1} := 0
+                        if (t >= nt) { at = 1.f; u = 0.f; }                // padding: identity
                         aggH = fmaf(at, aggH, u);
                         aggA *= at;
-                        ra[j] = __float_as_uint(aggA);
-                        ru[j] = __float_as_uint(aggH);
+                        da[j] = aggA;
+                        dx[j] = aggH;
                     }
-                    tmem_st8(dcol + j0, ra);
-                    tmem_st8(dcol + L + j0, ru);
+                    tmem_stbf(dcol + j0, da);
+                    tmem_stbf(dcol + L + j0, dx);
                 }
             }
             // the B tile (xc) is no longer read by this warp
@@ -755,7 +767,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     bool okl = mine ? ld_acquire_gpu(fl) >= FLAG_AGG : true;
                     if (lane == 0) okl = okl && ld_acquire_gpu(fa) >= FLAG_INCL;
                     if (__all_sync(0xffffffffu, okl)) { ready = true; break; }
-                    __nanosleep(128);
+                    __nanosleep(64);
                     if ((it & 15) == 15) {
                         int give_up = 0;
                         if (lane == 0) {
@@ -800,33 +812,46 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             if (!wait_bar(bars.y_full[st], ph, wc, 16)) break;
             tmem_wait_st();
             {
-                float pv[kSub], hv[kSub], pn[kSub], hn[kSub];
-                tmem_ld8(dcol, pv);
-                tmem_ld8(dcol + L, hv);
+                const float2 cv = f2(carry);
+                float pv[kBlk], hv[kBlk], pn[kBlk], hn[kBlk];
+                tmem_ldb(dcol, pv);
+                tmem_ldb(dcol + L, hv);
                 tmem_wait_ld();
 #pragma unroll 1
-                for (int j0 = 0; j0 < L; j0 += kSub) {
-                    if (j0 + kSub < L) {
-                        tmem_ld8(dcol + j0 + kSub, pn);
-                        tmem_ld8(dcol + L + j0 + kSub, hn);
+                for (int j0 = 0; j0 < L; j0 += kBlk) {
+                    if (j0 + kBlk < L) {
+                        tmem_ldb(dcol + j0 + kBlk, pn);
+                        tmem_ldb(dcol + L + j0 + kBlk, hn);
                     }
 #pragma unroll
-                    for (int j = 0; j < kSub; j += 2) {
+                    for (int j = 0; j < kBlk; j += 2) {
                         const int t = j0 + j;
-                        const float2 hh = fma2(make_float2(pv[j], pv[j + 1]), f2(carry), make_float2(hv[j], hv[j + 1]));
-                        __nv_bfloat16* y0 = reinterpret_cast<__nv_bfloat16*>(yt + t * HALF * 2);
-                        __nv_bfloat16* y1 = reinterpret_cast<__nv_bfloat16*>(yt + (t + 1) * HALF * 2);
-                        const float2 g = gelu_pair(make_float2(__bfloat162float(*y0), __bfloat162float(*y1)), tanh_form);
-                        const float2 o = mul2(hh, g);
-                        if (t < nt) *y0 = __float2bfloat16_rn(o.x);
-                        if (t + 1 < nt) *y1 = __float2bfloat16_rn(o.y);
+                        unsigned short* y0 = reinterpret_cast<unsigned short*>(yt + t * HALF * 2);
+                        unsigned short* y1 = reinterpret_cast<unsigned short*>(yt + (t + 1) * HALF * 2);
+                        const float2 yv = make_float2(__uint_as_float((uint32_t)*y0 << 16), __uint_as_float((uint32_t)*y1 << 16));
+                        const float2 hh = fma2(make_float2(pv[j], pv[j + 1]), cv, make_float2(hv[j], hv[j + 1]));
+                        const float2 o = merge_pair(hh, yv, gk1, gk3);
+                        const uint32_t ob = pack_bf16x2(o.x, o.y);
+                        *y0 = (unsigned short)(ob & 0xFFFFu);
+                        *y1 = (unsigned short)(ob >> 16);
                     }
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < kSub; ++j) { pv[j] = pn[j]; hv[j] = hn[j]; }
+                    for (int j = 0; j < kBlk; ++j) { pv[j] = pn[j]; hv[j] = hn[j]; }
                 }
             }
-            // TMEM accumulators of this stage are free again
+            // re-arm the accumulator stage with the gate biases, then hand it back to the MMA
+            if (bias_in_acc) {
+                uint32_t ra[16], rx[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) { ra[j] = ba_bits; rx[j] = bx_bits; }
+#pragma unroll
+                for (int j0 = 0; j0 < L; j0 += 16) {
+                    tmem_st16(dcol + j0, ra);
+                    tmem_st16(dcol + L + j0, rx);
+                }
+                tmem_wait_st();
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.acc_empty[st]);
@@ -942,9 +967,9 @@ cudaError_t launch_fused_prefill(const rglru_dims* d, const rglru_params* p, con
         !make_map_3d(&my, y, W, d->seq_len, d->batch, HALF, L) ||
         !make_map_3d(&mo, out, W, d->seq_len, d->batch, HALF, L))
         return cudaErrorInvalidValue;
-    static cudaError_t attr = cudaFuncSetAttribute(fused_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)SMEM_BYTES);
-    if (attr != cudaSuccess) return attr;
+    // per call (a cheap attribute write): the setting belongs to the current device
+    e = cudaFuncSetAttribute(fused_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
 
     uint8_t* w = static_cast<uint8_t*>(ws);
     Args a;

@@ -102,3 +102,38 @@ def test_withheld_carry_times_out_and_context_survives():
     assert status == binding.RGLRU_OK
     ref, _, _ = oracle.prefill(prob.params, prob.x, prob.y, 1)
     assert_close(to_np(out), ref, "bf16", "after timeout")
+
+
+def test_fused_nonzero_biases_resets_and_state():
+    """Gate biases (folded into the tensor-memory accumulators), a conv bias, resets and a
+    carried state together, against the oracle and the portable kernels."""
+    wl = BASE["packed_bf16"].scaled(batch=2, seq_len=700, heads=2, doc_len=(30, 400),
+                                    random_state=True)
+    prob = inputs.make_problem(wl, seed=21)
+    rng = np.random.default_rng(21)
+    W = wl.width
+    for k in ("b_a", "b_x", "conv_b"):
+        prob.params[k] = (0.7 * rng.standard_normal(W)).astype(np.float32)
+    gp = GpuProblem(prob)
+    out, h, tail, status = gp.prefill()
+    assert status == binding.RGLRU_OK
+    ref, ref_h, ref_tail = oracle.prefill(prob.params, prob.x, prob.y, wl.heads, reset=prob.reset,
+                                          h0=prob.h0, tail0=prob.tail0)
+    assert_close(to_np(out), ref, "bf16", "biased out")
+    assert_close(to_np(h), ref_h, "bf16", "biased h")
+    np.testing.assert_array_equal(to_np(tail), ref_tail)
+
+
+def test_fused_closed_recurrence_gate_freezes_state():
+    """b_a = -1e4 makes r_t = 0, so a_t = 1 and sqrt(1 - a_t^2) = 0: the carried state passes
+    through every token unchanged and out_t = h_0 GeLU(y_t)."""
+    wl = BASE["rg2b_bf16"].scaled(batch=2, seq_len=200, heads=2, random_state=True)
+    prob = inputs.make_problem(wl, seed=22)
+    prob.params["b_a"] = np.full(wl.width, -1e4, np.float32)
+    gp = GpuProblem(prob)
+    out, h, _, status = gp.prefill()
+    assert status == binding.RGLRU_OK
+    ref, ref_h, _ = oracle.prefill(prob.params, prob.x, prob.y, wl.heads, h0=prob.h0, tail0=prob.tail0)
+    np.testing.assert_array_equal(ref_h, prob.h0.astype(np.float64))     # the oracle's freeze
+    assert_close(to_np(out), ref, "bf16", "frozen out")
+    assert rel_err(to_np(h), ref_h) <= 1e-6
