@@ -140,6 +140,7 @@ size_t rglru_prefill_workspace_size(const rglru_dims* dims) {
 
 size_t rglru_decode_workspace_size(const rglru_dims* dims) {
     if (check_dims(dims, false) != RGLRU_OK) return 0;
+    if (rglru::fused_decode_supported(dims)) return rglru::fused_decode_workspace(dims);
     return kStatusBytes;
 }
 
@@ -173,6 +174,10 @@ rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_params* para
     if ((st = check_workspace(workspace, workspace_bytes, rglru_decode_workspace_size(dims))) != RGLRU_OK)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the tensor-core step reads and writes h with 16-byte vectors
+    if (rglru::fused_decode_supported(dims) && aligned(state->h, 16))
+        return cuda_status(rglru::launch_fused_decode(dims, params, x, y, reset, state, out, workspace,
+                                                      workspace_bytes, s));
     return cuda_status(rglru::launch_decode_generic(dims, params, x, y, reset, state, out, s));
 }
 
@@ -220,8 +225,9 @@ rglru_status rglru_decode_plan(const rglru_dims* dims, int* kernel, int* launche
     rglru_status st = check_dims(dims, false);
     if (st != RGLRU_OK) return st;
     if (!kernel || !launches) return RGLRU_ERR_INVALID_ARG;
-    *kernel = RGLRU_KERNEL_GENERIC;
-    *launches = 1;
+    const bool tc = rglru::fused_decode_supported(dims);
+    *kernel = tc ? RGLRU_KERNEL_TENSOR : RGLRU_KERNEL_GENERIC;
+    *launches = tc ? rglru::fused_decode_launches(dims) : 1;
     return RGLRU_OK;
 }
 

@@ -7,7 +7,26 @@
 
 #include "rglru.h"
 
+#include <mutex>
+
 namespace rglru {
+
+// Sets a kernel's dynamic shared-memory limit once per device (the attribute belongs to the
+// current device; doing it on the first call keeps it out of any later stream capture).
+template <typename Kernel>
+cudaError_t set_smem_once(Kernel k, int bytes) {
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[dev] = true;
+    return e;
+}
 
 constexpr int kConvWidth = 4;
 constexpr int kHist = kConvWidth - 1;

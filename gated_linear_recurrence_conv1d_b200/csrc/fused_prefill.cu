@@ -65,23 +65,23 @@ using namespace sm100;
 
 constexpr int DH = 256;                 // head dim (K of the gate contraction)
 constexpr int HALF = 128;               // output channels per CTA (= TMEM lanes = MMA M)
-constexpr int L = 64;                   // tokens per chunk (= MMA N)
+constexpr int L = 32;                   // tokens per chunk (= MMA N)
 constexpr int XROWS = L + kHist;        // x tile rows incl. the 3-token halo
 constexpr int KSTEPS = DH / 16;         // MMA K steps
-constexpr int STAGES = 2;
-constexpr int SLOTS = 8;                // ring of item ids, indexed by iteration
+constexpr int STAGES = 4;               // x / B / y tiles and TMEM accumulator slots
+constexpr int SLOTS = 16;               // ring of item ids, indexed by iteration (> the producers' lag)
 constexpr int kBlk = 8;                 // tokens per TMEM load block in the epilogue
-constexpr int kConvTok = L / 4;         // tokens per conv warp
+constexpr int kConvTok = L;             // tokens per conv warp
 
-// warp roles: 0-3 conv (token quarter = warp), 4-11 epilogue (TMEM lane quarter = warp % 4,
-// group = stage = (warp - 4) / 4), 12 x producer (x tiles and tickets), 13 y producer, 14 MMA.
-constexpr int kConvWarps = 4, kEpiWarps = 8, kEpiGroup = 4;
-constexpr int kWarpEpi0 = 4, kWarpProdX = 12, kWarpProdY = 13, kWarpMma = 14;
-constexpr int kThreads = 15 * 32;
+// warp roles: 0-1 conv (channel half = warp), 2-17 epilogue (TMEM lane quarter = warp % 4,
+// group = stage = (warp - 2) / 4), 18 x producer (x tiles and tickets), 19 y producer, 20 MMA.
+constexpr int kConvWarps = 2, kEpiGroups = STAGES, kEpiGroup = 4, kEpiWarps = kEpiGroups * kEpiGroup;
+constexpr int kWarpEpi0 = 2, kWarpProdX = 18, kWarpProdY = 19, kWarpMma = 20;
+constexpr int kThreads = 21 * 32;
 
-constexpr uint32_t X_BYTES = XROWS * DH * 2;      // 34304
-constexpr uint32_t Y_BYTES = L * HALF * 2;        // 16384
-constexpr uint32_t B_BYTES = L * DH * 2;          // 32768 (4 K-blocks of L x 128 B)
+constexpr uint32_t X_BYTES = XROWS * DH * 2;      // 17920
+constexpr uint32_t Y_BYTES = L * HALF * 2;        // 8192
+constexpr uint32_t B_BYTES = L * DH * 2;          // 16384 (4 K-blocks of L x 128 B)
 constexpr uint32_t KBLK_BYTES = L * 128;          // one 64-wide K block
 
 // shared memory map (offsets from a 1024-aligned base)
@@ -89,15 +89,19 @@ constexpr uint32_t OFF_B = 0;                                   // STAGES x B_BY
 constexpr uint32_t OFF_X = OFF_B + STAGES * B_BYTES;            // STAGES x X_BYTES
 constexpr uint32_t OFF_Y = OFF_X + STAGES * X_BYTES;            // STAGES x Y_BYTES
 constexpr uint32_t OFF_BAR = OFF_Y + STAGES * Y_BYTES;
-constexpr int NBAR = 9 * STAGES + 2;
-constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;               // slots, TMEM base, abort flag
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 64 + 1024;          // + slack for 1024 alignment
+constexpr int NBAR = 11 * STAGES + 2;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;               // item-id ring
+constexpr uint32_t OFF_TMEMP = OFF_MISC + SLOTS * 4;            // TMEM base address
+constexpr uint32_t OFF_ABORT = OFF_TMEMP + 16;                  // abort flag
+constexpr uint32_t SMEM_BYTES = OFF_ABORT + 16 + 1024;         // + slack for 1024 alignment
 static_assert(2 * HALF * DH * 2 <= OFF_Y, "weight staging reuses the B and x tiles");
 
 // TMEM columns: [0,128) A = W_a^T / 2 (bf16 pairs), [128,256) A = W_x^T / 2, then per stage
-// 128 columns: D_a [0,64) and D_x [64,128); the first pass overwrites them with P and H.
+// 2L = 64 columns: D_a [0,L) and D_x [L,2L); the first pass overwrites them with P and H.
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_A = 0, TM_D = 256;
+constexpr uint32_t TM_A = 0, TM_D = 256, TM_SLOT = 2 * L;
+static_assert(TM_D + STAGES * TM_SLOT <= TMEM_COLS, "TMEM budget");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 constexpr unsigned FLAG_AGG = 1, FLAG_INCL = 2;
 constexpr int LBW = 32;                 // look-back block: anchors every LBW chunks
@@ -129,7 +133,8 @@ struct Args {
 
 struct Bars {
     uint32_t x_full[STAGES], x_empty[STAGES], y_full[STAGES], y_empty[STAGES], b_full[STAGES],
-        b_empty[STAGES], acc_full[STAGES], acc_empty[STAGES], out_ready[STAGES], w_ready, mma_done;
+        b_empty[STAGES], acc_full[STAGES], acc_empty[STAGES], out_ready[STAGES], slot_full[STAGES],
+        slot_free[STAGES], w_ready, mma_done;
 };
 
 __device__ __forceinline__ Bars make_bars(uint32_t base) {
@@ -139,7 +144,7 @@ __device__ __forceinline__ Bars make_bars(uint32_t base) {
     for (int s = 0; s < STAGES; ++s) {
         b.x_full[s] = next(); b.x_empty[s] = next(); b.y_full[s] = next(); b.y_empty[s] = next();
         b.b_full[s] = next(); b.b_empty[s] = next(); b.acc_full[s] = next(); b.acc_empty[s] = next();
-        b.out_ready[s] = next();
+        b.out_ready[s] = next(); b.slot_full[s] = next(); b.slot_free[s] = next();
     }
     b.w_ready = next();
     b.mma_done = next();
@@ -174,6 +179,12 @@ __device__ __noinline__ bool wait_bar_slow(uint32_t bar, uint32_t parity, WaitCt
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, WaitCtx w, unsigned where) {
     if (mbar_try_wait(bar, parity)) return true;
     return wait_bar_slow(bar, parity, w, where);
+}
+
+// The same wait for a warp whose lanes then run warp-collective instructions: every lane waits,
+// and the outcome is made uniform, so that the warp never splits on a timeout.
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, WaitCtx w, unsigned where) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, w, where));
 }
 
 // Bounded wait for a look-back flag to reach at least `want`; returns the flag (0 on failure).
@@ -275,35 +286,33 @@ __device__ __forceinline__ float2 merge_pair(float2 h, float2 y, float k1, float
     return fma2(m, t, m);
 }
 
-// Bit j of the result = reset[t0 + j] != 0 for the 64 tokens of a chunk (0 past the end).
+// Bit j of the result = reset[t0 + j] != 0 for the L tokens of a chunk (0 past the end).
 __device__ __forceinline__ uint64_t chunk_reset_mask(const uint8_t* row, int t0, int T, int lane) {
-    const bool r0 = t0 + lane < T && row[t0 + lane] != 0;
-    const bool r1 = t0 + 32 + lane < T && row[t0 + 32 + lane] != 0;
-    const uint32_t lo = __ballot_sync(0xffffffffu, r0);
-    const uint32_t hi = __ballot_sync(0xffffffffu, r1);
-    return (uint64_t)lo | ((uint64_t)hi << 32);
+    uint64_t m = 0;
+#pragma unroll
+    for (int h = 0; h < L; h += 32) {
+        const bool r = t0 + h + lane < T && row[t0 + h + lane] != 0;
+        m |= (uint64_t)__ballot_sync(0xffffffffu, r) << h;
+    }
+    return m;
 }
 
-// Conv of one token for a lane's 8 channels: y = cb + w0 h0 + w1 h1 + w2 h2 + w3 xv, as bf16.
-struct Vec8 {
-    float2 v[4];
+// A lane's 4 channels of one token (conv window entries), fp32.
+struct Vec4 {
+    float2 v[2];
 };
-__device__ __forceinline__ Vec8 unpack8(uint4 r) {
-    Vec8 o;
+__device__ __forceinline__ Vec4 unpack4(uint2 r) {
+    Vec4 o;
     o.v[0] = make_float2(bf16lo(r.x), bf16hi(r.x));
     o.v[1] = make_float2(bf16lo(r.y), bf16hi(r.y));
-    o.v[2] = make_float2(bf16lo(r.z), bf16hi(r.z));
-    o.v[3] = make_float2(bf16lo(r.w), bf16hi(r.w));
     return o;
 }
-__device__ __forceinline__ uint4 pack8(const Vec8& h) {
-    return make_uint4(pack_bf16x2(h.v[0].x, h.v[0].y), pack_bf16x2(h.v[1].x, h.v[1].y),
-                      pack_bf16x2(h.v[2].x, h.v[2].y), pack_bf16x2(h.v[3].x, h.v[3].y));
+__device__ __forceinline__ uint2 pack4(const Vec4& h) {
+    return make_uint2(pack_bf16x2(h.v[0].x, h.v[0].y), pack_bf16x2(h.v[1].x, h.v[1].y));
 }
-__device__ __forceinline__ Vec8 zero8() {
-    Vec8 o;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o.v[i] = make_float2(0.f, 0.f);
+__device__ __forceinline__ Vec4 zero4() {
+    Vec4 o;
+    o.v[0] = o.v[1] = make_float2(0.f, 0.f);
     return o;
 }
 
@@ -315,8 +324,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     const uint32_t sbase = smem_u32(smem);
     const Bars bars = make_bars(sbase + OFF_BAR);
     volatile int* slot = reinterpret_cast<volatile int*>(smem + OFF_MISC);        // [SLOTS]
-    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 32);
-    volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 48);
+    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEMP);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -343,6 +352,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             mbar_init(bars.acc_full[s], 1);
             mbar_init(bars.acc_empty[s], kEpiGroup);
             mbar_init(bars.out_ready[s], kEpiGroup);
+            mbar_init(bars.slot_full[s], 1);
+            mbar_init(bars.slot_free[s], 1);
         }
         mbar_init(bars.w_ready, kEpiWarps);
         mbar_init(bars.mma_done, 1);
@@ -386,9 +397,9 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         // each lane quarter writes gate a, group 1 gate x.  Then each group pre-loads the gate
         // biases of its accumulator stage.
         const int q = warp & 3, g = (warp - kWarpEpi0) >> 2, m = q * 32 + lane;
-        const unsigned short* ws = reinterpret_cast<const unsigned short*>(smem + g * (HALF * DH * 2)) + m;
+        const unsigned short* ws = reinterpret_cast<const unsigned short*>(smem + (g & 1) * (HALF * DH * 2)) + m;
 #pragma unroll 1
-        for (int j0 = 0; j0 < DH / 2; j0 += 16) {
+        for (int j0 = 0; j0 < (g < 2 ? DH / 2 : 0); j0 += 16) {
             uint32_t r[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
@@ -404,7 +415,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             uint32_t ra[16], rx[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) { ra[j] = ba; rx[j] = bx; }
-            const uint32_t d = tmem + ((uint32_t)(q * 32) << 16) + TM_D + g * 128;
+            const uint32_t d = tmem + ((uint32_t)(q * 32) << 16) + TM_D + g * TM_SLOT;
 #pragma unroll
             for (int j0 = 0; j0 < L; j0 += 16) {
                 tmem_st16(d + j0, ra);
@@ -421,20 +432,24 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     if (warp == kWarpProdX) {
         if (lane == 0) {
             // ============================ x producer (and tickets) ============================
-            int issued[STAGES] = {0, 0};
+            int issued[STAGES] = {};
             for (int n = 0;; ++n) {
-                const int st = n & 1;
-                const uint32_t ph = (n >> 1) & 1;
+                const int st = n % STAGES;
+                const uint32_t ph = (n / STAGES) & 1;
                 if (!wait_bar(bars.x_empty[st], ph ^ 1, wc, 1)) break;
+                // the y producer has taken the id of iteration n - STAGES: it never lags further
+                if (!wait_bar(bars.slot_free[st], ph ^ 1, wc, 19)) break;
                 int k = (int)atomicAdd(&a.counters[group], 1u);
                 if (k >= a.items) {
-                    slot[n & (SLOTS - 1)] = -1;            // terminal item for the stage-n group
-                    slot[(n + 1) & (SLOTS - 1)] = -1;      // ... and for the other group
+                    // terminal item for the stage-n group and for the next STAGES-1 groups
+                    for (int i = 0; i < STAGES; ++i) slot[(n + i) & (SLOTS - 1)] = -1;
+                    mbar_arrive(bars.slot_full[st]);
                     mbar_arrive(bars.x_full[st]);
                     issued[st] = 0;   // that phase completing implies the earlier load landed
                     break;
                 }
                 slot[n & (SLOTS - 1)] = k;
+                mbar_arrive(bars.slot_full[st]);
                 const int b = k / a.NC, c = k % a.NC;
                 mbar_arrive_expect_tx(bars.x_full[st], X_BYTES);
                 tma_load_3d(sbase + OFF_X + st * X_BYTES, &map_x, head * DH, c * L - kHist, b,
@@ -446,7 +461,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 if (issued[st]) {
                     const int n = issued[st] - 1;
                     const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait_sleep(bars.x_full[st], (n >> 1) & 1, 100000u) &&
+                    while (!mbar_try_wait_sleep(bars.x_full[st], (n / STAGES) & 1, 100000u) &&
                            globaltimer_ns() - t0 < a.timeout_ns) {
                     }
                 }
@@ -454,20 +469,15 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     } else if (warp == kWarpProdY) {
         if (lane == 0) {
             // ============================ y producer ==========================================
-            int issued[STAGES] = {0, 0};
+            int issued[STAGES] = {};
             for (int n = 0;; ++n) {
-                const int st = n & 1;
-                const uint32_t ph = (n >> 1) & 1;
-                // b_full (the conv warps arrive after reading item n's slot, which the x producer
-                // wrote before x_full) orders the slot read for this thread too
-                if (!wait_bar(bars.b_full[st], ph, wc, 15)) break;
+                const int st = n % STAGES;
+                const uint32_t ph = (n / STAGES) & 1;
+                if (!wait_bar(bars.slot_full[st], ph, wc, 15)) break;
                 const int k = slot[n & (SLOTS - 1)];
+                mbar_arrive(bars.slot_free[st]);
+                if (k < 0) break;
                 if (!wait_bar(bars.y_empty[st], ph ^ 1, wc, 2)) break;
-                if (k < 0) {
-                    mbar_arrive(bars.y_full[st]);
-                    issued[st] = 0;
-                    break;
-                }
                 const int b = k / a.NC, c = k % a.NC;
                 mbar_arrive_expect_tx(bars.y_full[st], Y_BYTES);
                 tma_load_3d(sbase + OFF_Y + st * Y_BYTES, &map_y, head * DH + half * HALF, c * L, b,
@@ -478,7 +488,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 if (issued[st]) {
                     const int n = issued[st] - 1;
                     const uint64_t t0 = globaltimer_ns();
-                    while (!mbar_try_wait_sleep(bars.y_full[st], (n >> 1) & 1, 100000u) &&
+                    while (!mbar_try_wait_sleep(bars.y_full[st], (n / STAGES) & 1, 100000u) &&
                            globaltimer_ns() - t0 < a.timeout_ns) {
                     }
                 }
@@ -490,23 +500,26 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             bool ok = wait_bar(bars.w_ready, 0, wc, 3);
             tc_fence_after();
             for (int n = 0; ok; ++n) {
-                const int st = n & 1;
-                const uint32_t ph = (n >> 1) & 1;
+                const int st = n % STAGES;
+                const uint32_t ph = (n / STAGES) & 1;
                 if (!wait_bar(bars.b_full[st], ph, wc, 4)) break;
                 if (!wait_bar(bars.acc_empty[st], ph ^ 1, wc, 5)) break;
                 if (slot[n & (SLOTS - 1)] < 0) {
-                    // hand the terminal item to both epilogue groups: group st now, group st^1
-                    // once it has released its previous item (so that no phase is skipped)
+                    // hand the terminal item to every epilogue group: group st now, each other
+                    // group once it has released its previous item (so that no phase is skipped)
                     mbar_arrive(bars.acc_full[st]);
-                    const uint32_t ph1 = ((n + 1) >> 1) & 1;
-                    if (wait_bar(bars.acc_empty[st ^ 1], ph1 ^ 1, wc, 17)) mbar_arrive(bars.acc_full[st ^ 1]);
+                    for (int i = 1; i < STAGES; ++i) {
+                        const int s2 = (n + i) % STAGES;
+                        const uint32_t ph2 = ((n + i) / STAGES) & 1;
+                        if (wait_bar(bars.acc_empty[s2], ph2 ^ 1, wc, 17)) mbar_arrive(bars.acc_full[s2]);
+                    }
                     break;
                 }
                 tc_fence_after();
                 const uint32_t bt = sbase + OFF_B + st * B_BYTES;
 #pragma unroll 1
                 for (int g = 0; g < 2; ++g) {
-                    const uint32_t d = tmem + TM_D + st * 128 + g * L;
+                    const uint32_t d = tmem + TM_D + st * TM_SLOT + g * L;
 #pragma unroll
                     for (int ks = 0; ks < KSTEPS; ++ks) {
                         const uint64_t bd = desc_k_sw128(bt + (ks >> 2) * KBLK_BYTES + (ks & 3) * 32);
@@ -524,29 +537,32 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         }
     } else if (warp < kConvWarps) {
         // ================================ conv warps ==========================================
-        // warp w convolves tokens [16w, 16w + 16) of the chunk; lane l channels 8l .. 8l+7 of the
-        // head (K block l / 8, 16-byte chunk l % 8 of the B tile's 128-byte rows)
-        const int j0 = warp * kConvTok;
-        const int cl = lane * 8;                          // channel within the head
+        // warp w convolves channels [128 w, +128) of the head for every token of the chunk;
+        // lane l 4 channels (8 bytes of a B-tile row)
+        const int chh = warp;
+        const int j0 = 0;
+        const int cl = chh * HALF + lane * 4;             // channel within the head
         const int chg = head * DH + cl;                   // global channel
-        float2 w[kConvWidth][4];
+        float2 w[kConvWidth][2];
 #pragma unroll
         for (int k = 0; k < kConvWidth; ++k)
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 2; ++i)
                 w[k][i] = make_float2(a.conv_w[(size_t)k * W + chg + 2 * i], a.conv_w[(size_t)k * W + chg + 2 * i + 1]);
-        float2 cb[4];
+        float2 cb[2];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 2; ++i)
             cb[i] = a.conv_b ? make_float2(a.conv_b[chg + 2 * i], a.conv_b[chg + 2 * i + 1]) : make_float2(0.f, 0.f);
-        const bool own_tail = (lane >> 4) == half;       // this CTA writes these tail channels
-        const uint32_t kb_off = (uint32_t)(lane >> 3) * KBLK_BYTES;
-        const uint32_t cchunk = lane & 7;
+        const bool own_tail = chh == half;               // this CTA writes these tail channels
+        // B-tile byte offset of (token t, channel cl): kb * KBLK + (t / 8) * 1024 + (t % 8) * 128
+        //   + ((chunk ^ (t % 8)) * 16) + sub, chunk / sub = 16-byte chunk / byte within it
+        const uint32_t kb_off = (uint32_t)(cl >> 6) * KBLK_BYTES + ((cl & 7) * 2);
+        const uint32_t cchunk = (cl & 63) >> 3;
         for (int n = 0;; ++n) {
-            const int st = n & 1;
-            const uint32_t ph = (n >> 1) & 1;
-            if (!wait_bar(bars.x_full[st], ph, wc, 6)) break;
-            if (!wait_bar(bars.b_empty[st], ph ^ 1, wc, 7)) break;
+            const int st = n % STAGES;
+            const uint32_t ph = (n / STAGES) & 1;
+            if (!wait_bar_warp(bars.x_full[st], ph, wc, 6)) break;
+            if (!wait_bar_warp(bars.b_empty[st], ph ^ 1, wc, 7)) break;
             const int k = slot[n & (SLOTS - 1)];
             if (k < 0) {
                 __syncwarp();
@@ -560,17 +576,17 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             const uint8_t* xt = smem + OFF_X + st * X_BYTES + cl * 2;
             uint8_t* bt = smem + OFF_B + st * B_BYTES + kb_off;
             auto xrow = [&](int r) {                      // x tile row r = token t0 - 3 + r
-                return unpack8(*reinterpret_cast<const uint4*>(xt + r * DH * 2));
+                return unpack4(*reinterpret_cast<const uint2*>(xt + r * DH * 2));
             };
-            Vec8 h0, h1, h2;                              // window x_{t-3}, x_{t-2}, x_{t-1}
+            Vec4 h0, h1, h2;                              // window x_{t-3}, x_{t-2}, x_{t-1}
             if (c == 0 && j0 == 0) {
                 if (a.tail_state) {
                     const __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
-                    h0 = unpack8(*reinterpret_cast<const uint4*>(tl));
-                    h1 = unpack8(*reinterpret_cast<const uint4*>(tl + W));
-                    h2 = unpack8(*reinterpret_cast<const uint4*>(tl + 2 * W));
+                    h0 = unpack4(*reinterpret_cast<const uint2*>(tl));
+                    h1 = unpack4(*reinterpret_cast<const uint2*>(tl + W));
+                    h2 = unpack4(*reinterpret_cast<const uint2*>(tl + 2 * W));
                 } else {
-                    h0 = h1 = h2 = zero8();
+                    h0 = h1 = h2 = zero4();
                 }
             } else {
                 h0 = xrow(j0);
@@ -579,30 +595,31 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 if (rrow) {
                     // a segment that starts at token j0-1 (j0-2) empties the older history
                     const int p1 = t0 + j0 - 1, p2 = t0 + j0 - 2;
-                    if (p1 < a.T && rrow[p1]) h0 = h1 = zero8();
-                    if (p2 >= 0 && p2 < a.T && rrow[p2]) h0 = zero8();
+                    if (p1 < a.T && rrow[p1]) h0 = h1 = zero4();
+                    if (p2 >= 0 && p2 < a.T && rrow[p2]) h0 = zero4();
                 }
             }
-            uint4 fw[3];                                  // final window (the tail of the row), bf16
+            uint2 fw[3];                                  // final window (the tail of the row), bf16
             const bool has_last = nt - 1 >= j0 && nt - 1 < j0 + kConvTok;
 #pragma unroll 4
             for (int jj = 0; jj < kConvTok; ++jj) {
                 const int j = j0 + jj;
-                const Vec8 xv = xrow(j + kHist);
-                if ((rmask >> j) & 1ull) h0 = h1 = h2 = zero8();
-                uint4 o;
-                uint32_t* op = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float2 y = fma2(w[0][i], h0.v[i], cb[i]);
-                    y = fma2(w[1][i], h1.v[i], y);
-                    y = fma2(w[2][i], h2.v[i], y);
-                    y = fma2(w[3][i], xv.v[i], y);
-                    op[i] = pack_bf16x2(y.x, y.y);
-                }
-                *reinterpret_cast<uint4*>(bt + (j >> 3) * 1024 + (j & 7) * 128 + ((cchunk ^ (j & 7)) << 4)) = o;
+                const Vec4 xv = xrow(j + kHist);
+                if ((rmask >> j) & 1ull) h0 = h1 = h2 = zero4();
+                uint2 o;
+                float2 y = fma2(w[0][0], h0.v[0], cb[0]);
+                y = fma2(w[1][0], h1.v[0], y);
+                y = fma2(w[2][0], h2.v[0], y);
+                y = fma2(w[3][0], xv.v[0], y);
+                o.x = pack_bf16x2(y.x, y.y);
+                y = fma2(w[0][1], h0.v[1], cb[1]);
+                y = fma2(w[1][1], h1.v[1], y);
+                y = fma2(w[2][1], h2.v[1], y);
+                y = fma2(w[3][1], xv.v[1], y);
+                o.y = pack_bf16x2(y.x, y.y);
+                *reinterpret_cast<uint2*>(bt + (j >> 3) * 1024 + (j & 7) * 128 + ((cchunk ^ (j & 7)) << 4)) = o;
                 h0 = h1; h1 = h2; h2 = xv;
-                if (has_last && j == nt - 1) { fw[0] = pack8(h0); fw[1] = pack8(h1); fw[2] = pack8(h2); }
+                if (has_last && j == nt - 1) { fw[0] = pack4(h0); fw[1] = pack4(h1); fw[2] = pack4(h2); }
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -618,17 +635,14 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     if (lane == 0) f = wait_flag(a.lb_flags + (lb_base + (size_t)b * a.NC) * 4, FLAG_AGG, wc, 8);
                     ok = __shfl_sync(0xffffffffu, f, 0) != 0;
                 } else {
-                    // a row of one chunk: warp 0 read the old history in this very item; once
-                    // every conv warp has arrived on b_full, that read is done
-                    ok = wait_bar(bars.b_full[st], ph, wc, 18);
+                    // a row of one chunk: the old history was read in this very item (by this
+                    // warp, which owns these channels); b_full has completed once it is read
+                    ok = wait_bar_warp(bars.b_full[st], ph, wc, 18);
                 }
                 if (ok && own_tail) {
                     __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
 #pragma unroll
-                    for (int r = 0; r < 3; ++r) {
-                        const uint4 o = fw[r];
-                        *reinterpret_cast<uint4*>(tl + (size_t)r * W) = o;
-                    }
+                    for (int r = 0; r < 3; ++r) *reinterpret_cast<uint2*>(tl + (size_t)r * W) = fw[r];
                 }
             }
         }
@@ -653,7 +667,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         const bool withhold_hook = (a.flags & RGLRU_FLAG_TEST_WITHHOLD) && group == 0;
         const uint8_t* bt = smem + OFF_B + st * B_BYTES;
         uint8_t* yt = smem + OFF_Y + st * Y_BYTES + 2 * m;
-        const uint32_t dcol = tmem + lane_off + TM_D + st * 128;
+        const uint32_t dcol = tmem + lane_off + TM_D + st * TM_SLOT;
         // B-tile byte offsets of this channel for tokens 0..7 (token t: boff[t & 7] + (t >> 3) * 1024)
         uint32_t boff[8];
 #pragma unroll
@@ -662,9 +676,9 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             return __uint_as_float((uint32_t)*reinterpret_cast<const unsigned short*>(bt + boff[t & 7] + (t >> 3) * 1024) << 16);
         };
 
-        for (int n = eg;; n += 2) {
-            const uint32_t ph = (n >> 1) & 1;
-            if (!wait_bar(bars.acc_full[st], ph, wc, 9)) break;
+        for (int n = eg;; n += STAGES) {
+            const uint32_t ph = (n / STAGES) & 1;
+            if (!wait_bar_warp(bars.acc_full[st], ph, wc, 9)) break;
             const int k = slot[n & (SLOTS - 1)];
             if (k < 0) break;
             tc_fence_after();
@@ -681,16 +695,12 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             float aggA = 1.f, aggH = 0.f;
             const bool fast = nt == L && __all_sync(0xffffffffu, small_range);
             if (fast) {
-                float da[kBlk], dx[kBlk], dan[kBlk], dxn[kBlk];
-                tmem_ldb(dcol, da);
-                tmem_ldb(dcol + L, dx);
-                tmem_wait_ld();
 #pragma unroll 1
                 for (int j0 = 0; j0 < L; j0 += kBlk) {
-                    if (j0 + kBlk < L) {                    // next block in flight meanwhile
-                        tmem_ldb(dcol + j0 + kBlk, dan);
-                        tmem_ldb(dcol + L + j0 + kBlk, dxn);
-                    }
+                    float da[kBlk], dx[kBlk];
+                    tmem_ldb(dcol + j0, da);
+                    tmem_ldb(dcol + L + j0, dx);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < kBlk; j += 2) {
                         float2 at, u;
@@ -711,9 +721,6 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     }
                     tmem_stbf(dcol + j0, da);
                     tmem_stbf(dcol + L + j0, dx);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < kBlk; ++j) { da[j] = dan[j]; dx[j] = dxn[j]; }
                 }
             } else {
 #pragma unroll 1
@@ -809,20 +816,16 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             }
 
             // ---- pass 2: h_t = P_t C + H_t (no serial chain), merged with GeLU(y_t)
-            if (!wait_bar(bars.y_full[st], ph, wc, 16)) break;
+            if (!wait_bar_warp(bars.y_full[st], ph, wc, 16)) break;
             tmem_wait_st();
             {
                 const float2 cv = f2(carry);
-                float pv[kBlk], hv[kBlk], pn[kBlk], hn[kBlk];
-                tmem_ldb(dcol, pv);
-                tmem_ldb(dcol + L, hv);
-                tmem_wait_ld();
 #pragma unroll 1
                 for (int j0 = 0; j0 < L; j0 += kBlk) {
-                    if (j0 + kBlk < L) {
-                        tmem_ldb(dcol + j0 + kBlk, pn);
-                        tmem_ldb(dcol + L + j0 + kBlk, hn);
-                    }
+                    float pv[kBlk], hv[kBlk];
+                    tmem_ldb(dcol + j0, pv);
+                    tmem_ldb(dcol + L + j0, hv);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < kBlk; j += 2) {
                         const int t = j0 + j;
@@ -835,9 +838,6 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                         *y0 = (unsigned short)(ob & 0xFFFFu);
                         *y1 = (unsigned short)(ob >> 16);
                     }
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < kBlk; ++j) { pv[j] = pn[j]; hv[j] = hn[j]; }
                 }
             }
             // re-arm the accumulator stage with the gate biases, then hand it back to the MMA
@@ -869,6 +869,9 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 mbar_arrive(bars.y_empty[st]);
             }
         }
+        // no tensor-memory access of this warp may still be in flight when TMEM is released
+        tmem_wait_st();
+        tmem_wait_ld();
         if (q == 0 && lane == 0) bulk_wait0();
     }
 
@@ -909,6 +912,21 @@ bool make_map_3d(CUtensorMap* m, const void* base, int W, int T, int B, int box_
     cuuint32_t estr[3] = {1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map [outer][inner] of bf16 with a row pitch of row_bytes, box inner x outer, 128-byte
+// swizzle (box_inner * 2 must be 128), out-of-range elements read as zero.
+bool make_map_2d_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                       uint32_t box_inner, uint32_t box_outer) {
+    EncodeTiledFn f = encode_fn();
+    if (!f || box_inner * 2 != 128) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -967,8 +985,7 @@ cudaError_t launch_fused_prefill(const rglru_dims* d, const rglru_params* p, con
         !make_map_3d(&my, y, W, d->seq_len, d->batch, HALF, L) ||
         !make_map_3d(&mo, out, W, d->seq_len, d->batch, HALF, L))
         return cudaErrorInvalidValue;
-    // per call (a cheap attribute write): the setting belongs to the current device
-    e = cudaFuncSetAttribute(fused_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    e = set_smem_once(fused_prefill_kernel, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
 
     uint8_t* w = static_cast<uint8_t*>(ws);

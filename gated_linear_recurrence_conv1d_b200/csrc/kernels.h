@@ -24,4 +24,13 @@ cudaError_t launch_fused_prefill(const rglru_dims* d, const rglru_params* p, con
                                  const uint8_t* reset, rglru_state* st, void* out, void* ws, size_t ws_bytes,
                                  cudaStream_t s);
 
+// Tensor-core decode step (bf16, head_dim 256): conv + history shift, then tcgen05 gates and
+// the state update.  Needs the workspace fused_decode_workspace() (status word + conv scratch).
+bool fused_decode_supported(const rglru_dims* d);
+size_t fused_decode_workspace(const rglru_dims* d);
+int fused_decode_launches(const rglru_dims* d);
+cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, const void* x, const void* y,
+                                const uint8_t* reset, rglru_state* st, void* out, void* ws, size_t ws_bytes,
+                                cudaStream_t s);
+
 }  // namespace rglru

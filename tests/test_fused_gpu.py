@@ -137,3 +137,45 @@ def test_fused_closed_recurrence_gate_freezes_state():
     np.testing.assert_array_equal(ref_h, prob.h0.astype(np.float64))     # the oracle's freeze
     assert_close(to_np(out), ref, "bf16", "frozen out")
     assert rel_err(to_np(h), ref_h) <= 1e-6
+
+
+def test_plan_uses_tensor_cores_for_decode_bf16_dh256():
+    d = binding.make_dims(256, 1, 10, 256, binding.RGLRU_BF16)
+    kind, launches = binding.decode_plan(d)
+    assert kind == 1 and launches == 2
+    assert binding.decode_workspace_size(d) >= 256 + 256 * 2560 * 2
+    d.flags = binding.FLAG_GENERIC
+    assert binding.decode_plan(d)[0] == 0
+
+
+@pytest.mark.parametrize("B", [1, 77, 130, 256])
+def test_tensor_decode_matches_oracle_and_generic(B):
+    """Row tiles of 128 with a ragged last tile; biases and resets; against the oracle and the
+    portable kernel over a few steps."""
+    wl = BASE["decode_bf16"].scaled(batch=B, heads=2, decode_steps=4)
+    prob = inputs.make_problem(wl, seed=30 + B)
+    rng = np.random.default_rng(B)
+    for k in ("b_a", "b_x", "conv_b"):
+        prob.params[k] = (0.5 * rng.standard_normal(wl.width)).astype(np.float32)
+    outs = {}
+    for flags in (0, binding.FLAG_GENERIC):
+        gp = GpuProblem(prob, flags=flags)
+        h, tail = gp.new_state(B)
+        dims = gp.block.dims(B, 1)
+        ws = binding.alloc_workspace(binding.decode_workspace_size(dims))
+        h_ref = prob.h0.astype(np.float64).copy()
+        t_ref = oracle.tail_from_act(prob.tail0).copy()
+        res = []
+        for s in range(4):
+            rst_np = (np.arange(B) % 5 == s).astype(np.uint8)
+            out = torch.empty_like(gp.x[s])
+            binding.block_decode(dims, gp.block.params, gp.x[s], gp.y[s], out, h, tail, ws,
+                                 reset=binding.to_device(rst_np))
+            ref = oracle.decode(prob.params, prob.x[s], prob.y[s], wl.heads, h_ref, t_ref, reset=rst_np)
+            assert_close(to_np(out), ref, "bf16", f"decode step {s} flags {flags}")
+            np.testing.assert_array_equal(to_np(tail), t_ref)
+            res.append(to_np(out))
+        assert binding.read_device_status(ws) == binding.RGLRU_OK
+        assert_close(to_np(h), h_ref, "bf16", "decode h")
+        outs[flags] = np.stack(res)
+    assert rel_err(outs[0], outs[binding.FLAG_GENERIC]) <= 1e-2
