@@ -53,6 +53,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -71,13 +72,14 @@ constexpr int KSTEPS = DH / 16;         // MMA K steps
 constexpr int STAGES = 4;               // x / B / y tiles and TMEM accumulator slots
 constexpr int SLOTS = 16;               // ring of item ids, indexed by iteration (> the producers' lag)
 constexpr int kBlk = 8;                 // tokens per TMEM load block in the epilogue
-constexpr int kConvTok = L;             // tokens per conv warp
+constexpr int kConvTok = L / 2;         // tokens per conv warp
 
-// warp roles: 0-1 conv (channel half = warp), 2-17 epilogue (TMEM lane quarter = warp % 4,
-// group = stage = (warp - 2) / 4), 18 x producer (x tiles and tickets), 19 y producer, 20 MMA.
-constexpr int kConvWarps = 2, kEpiGroups = STAGES, kEpiGroup = 4, kEpiWarps = kEpiGroups * kEpiGroup;
-constexpr int kWarpEpi0 = 2, kWarpProdX = 18, kWarpProdY = 19, kWarpMma = 20;
-constexpr int kThreads = 21 * 32;
+// warp roles: 0-3 conv (channel half = warp % 2, token half = warp / 2), 4-19 epilogue (TMEM
+// lane quarter = warp % 4, group = stage = (warp - 4) / 4), 20 x producer (x tiles and
+// tickets), 21 y producer, 22 MMA.
+constexpr int kConvWarps = 4, kEpiGroups = STAGES, kEpiGroup = 4, kEpiWarps = kEpiGroups * kEpiGroup;
+constexpr int kWarpEpi0 = 4, kWarpProdX = 20, kWarpProdY = 21, kWarpMma = 22;
+constexpr int kThreads = 23 * 32;
 
 constexpr uint32_t X_BYTES = XROWS * DH * 2;      // 17920
 constexpr uint32_t Y_BYTES = L * HALF * 2;        // 8192
@@ -316,6 +318,35 @@ __device__ __forceinline__ Vec4 zero4() {
     return o;
 }
 
+// The conv of one warp's kConvTok tokens (j0 + jj, jj < kConvTok) for a lane's 4 channels, written
+// as bf16 into the B tile.  RST: the chunk has segment starts (bit jj of rm: token j0 + jj starts
+// one, so the history before it is dropped); LAST: the row's last token (jlast, relative to j0)
+// is in this range and the window after it is kept in fw (the conv history of the row).
+template <bool RST, bool LAST>
+__device__ __forceinline__ void conv_tokens(const uint8_t* xtw, uint8_t* btw, uint32_t cchunk, uint32_t rm, int jlast,
+                                            const float2 (&w)[kConvWidth][2], const float2 (&cb)[2], Vec4& h0, Vec4& h1,
+                                            Vec4& h2, uint2 (&fw)[3]) {
+#pragma unroll
+    for (int jj = 0; jj < kConvTok; ++jj) {
+        const Vec4 xv = unpack4(*reinterpret_cast<const uint2*>(xtw + (jj + kHist) * DH * 2));
+        if (RST && ((rm >> jj) & 1u)) h0 = h1 = h2 = zero4();
+        uint2 o;
+        float2 y = fma2(w[0][0], h0.v[0], cb[0]);
+        y = fma2(w[1][0], h1.v[0], y);
+        y = fma2(w[2][0], h2.v[0], y);
+        y = fma2(w[3][0], xv.v[0], y);
+        o.x = pack_bf16x2(y.x, y.y);
+        y = fma2(w[0][1], h0.v[1], cb[1]);
+        y = fma2(w[1][1], h1.v[1], y);
+        y = fma2(w[2][1], h2.v[1], y);
+        y = fma2(w[3][1], xv.v[1], y);
+        o.y = pack_bf16x2(y.x, y.y);
+        *reinterpret_cast<uint2*>(btw + (jj >> 3) * 1024 + (jj & 7) * 128 + ((cchunk ^ (jj & 7)) << 4)) = o;
+        h0 = h1; h1 = h2; h2 = xv;
+        if (LAST && jj == jlast) { fw[0] = pack4(h0); fw[1] = pack4(h1); fw[2] = pack4(h2); }
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_y,
                      const __grid_constant__ CUtensorMap map_out, const Args a) {
@@ -516,15 +547,15 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     break;
                 }
                 tc_fence_after();
-                const uint32_t bt = sbase + OFF_B + st * B_BYTES;
-#pragma unroll 1
-                for (int g = 0; g < 2; ++g) {
-                    const uint32_t d = tmem + TM_D + st * TM_SLOT + g * L;
+                // descriptor of K step ks = the stage's base descriptor + the step's byte offset / 16
+                const uint64_t bd0 = desc_k_sw128(sbase + OFF_B + st * B_BYTES);
+                const uint32_t d0 = tmem + TM_D + st * TM_SLOT;
 #pragma unroll
-                    for (int ks = 0; ks < KSTEPS; ++ks) {
-                        const uint64_t bd = desc_k_sw128(bt + (ks >> 2) * KBLK_BYTES + (ks & 3) * 32);
-                        mma_ts(d, tmem + TM_A + g * 128 + ks * 8, bd, idesc, (bias_in_acc || ks > 0) ? 1u : 0u);
-                    }
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    const uint64_t bd = bd0 + (uint64_t)((((ks >> 2) * KBLK_BYTES) + (ks & 3) * 32) >> 4);
+                    const uint32_t acc = (bias_in_acc || ks > 0) ? 1u : 0u;
+                    mma_ts(d0, tmem + TM_A + ks * 8, bd, idesc, acc);
+                    mma_ts(d0 + L, tmem + TM_A + 128 + ks * 8, bd, idesc, acc);
                 }
                 mma_commit(bars.acc_full[st]);
                 mma_commit(bars.b_empty[st]);
@@ -537,10 +568,10 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         }
     } else if (warp < kConvWarps) {
         // ================================ conv warps ==========================================
-        // warp w convolves channels [128 w, +128) of the head for every token of the chunk;
-        // lane l 4 channels (8 bytes of a B-tile row)
-        const int chh = warp;
-        const int j0 = 0;
+        // warp w convolves channels [128 (w % 2), +128) of the head for the tokens
+        // [16 (w / 2), +16) of the chunk; lane l 4 channels (8 bytes of a B-tile row)
+        const int chh = warp & 1;
+        const int j0 = (warp >> 1) * kConvTok;
         const int cl = chh * HALF + lane * 4;             // channel within the head
         const int chg = head * DH + cl;                   // global channel
         float2 w[kConvWidth][2];
@@ -601,25 +632,16 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             }
             uint2 fw[3];                                  // final window (the tail of the row), bf16
             const bool has_last = nt - 1 >= j0 && nt - 1 < j0 + kConvTok;
-#pragma unroll 4
-            for (int jj = 0; jj < kConvTok; ++jj) {
-                const int j = j0 + jj;
-                const Vec4 xv = xrow(j + kHist);
-                if ((rmask >> j) & 1ull) h0 = h1 = h2 = zero4();
-                uint2 o;
-                float2 y = fma2(w[0][0], h0.v[0], cb[0]);
-                y = fma2(w[1][0], h1.v[0], y);
-                y = fma2(w[2][0], h2.v[0], y);
-                y = fma2(w[3][0], xv.v[0], y);
-                o.x = pack_bf16x2(y.x, y.y);
-                y = fma2(w[0][1], h0.v[1], cb[1]);
-                y = fma2(w[1][1], h1.v[1], y);
-                y = fma2(w[2][1], h2.v[1], y);
-                y = fma2(w[3][1], xv.v[1], y);
-                o.y = pack_bf16x2(y.x, y.y);
-                *reinterpret_cast<uint2*>(bt + (j >> 3) * 1024 + (j & 7) * 128 + ((cchunk ^ (j & 7)) << 4)) = o;
-                h0 = h1; h1 = h2; h2 = xv;
-                if (has_last && j == nt - 1) { fw[0] = pack4(h0); fw[1] = pack4(h1); fw[2] = pack4(h2); }
+            const uint32_t rm = (uint32_t)(rmask >> j0);
+            const uint8_t* xtw = xt + j0 * DH * 2;
+            uint8_t* btw = bt + (j0 >> 3) * 1024;
+            const int jlast = nt - 1 - j0;
+            if (rm == 0) {
+                if (has_last) conv_tokens<false, true>(xtw, btw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
+                else conv_tokens<false, false>(xtw, btw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
+            } else {
+                if (has_last) conv_tokens<true, true>(xtw, btw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
+                else conv_tokens<true, false>(xtw, btw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -635,8 +657,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     if (lane == 0) f = wait_flag(a.lb_flags + (lb_base + (size_t)b * a.NC) * 4, FLAG_AGG, wc, 8);
                     ok = __shfl_sync(0xffffffffu, f, 0) != 0;
                 } else {
-                    // a row of one chunk: the old history was read in this very item (by this
-                    // warp, which owns these channels); b_full has completed once it is read
+                    // a row of one chunk: the warps of the first token half read the old history
+                    // in this very item; once every conv warp has arrived on b_full, it is read
                     ok = wait_bar_warp(bars.b_full[st], ph, wc, 18);
                 }
                 if (ok && own_tail) {
@@ -694,7 +716,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             //      the decays P_t and the running local state H_t (from zero) of every token
             float aggA = 1.f, aggH = 0.f;
             const bool fast = nt == L && __all_sync(0xffffffffu, small_range);
-            if (fast) {
+            // RST: the chunk has segment starts (a separate copy, so chunks without any pay nothing)
+            auto pass1_fast = [&](auto rst) {
 #pragma unroll 1
                 for (int j0 = 0; j0 < L; j0 += kBlk) {
                     float da[kBlk], dx[kBlk];
@@ -706,7 +729,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                         float2 at, u;
                         gates_pair(make_float2(da[j], da[j + 1]), make_float2(dx[j], dx[j + 1]), hk2,
                                    make_float2(xc_at(j0 + j), xc_at(j0 + j + 1)), at, u);
-                        if (rmask) {                                     // h_{t-1} := 0 at a reset
+                        if constexpr (decltype(rst)::value) {             // h_{t-1} := 0 at a reset
                             if ((rmask >> (j0 + j)) & 1ull) at.x = 0.f;
                             if ((rmask >> (j0 + j + 1)) & 1ull) at.y = 0.f;
                         }
@@ -722,6 +745,10 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     tmem_stbf(dcol + j0, da);
                     tmem_stbf(dcol + L + j0, dx);
                 }
+            };
+            if (fast) {
+                if (rmask) pass1_fast(std::true_type{});
+                else pass1_fast(std::false_type{});
             } else {
 #pragma unroll 1
                 for (int j0 = 0; j0 < L; j0 += kBlk) {
@@ -749,8 +776,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.b_empty[st]);
             if (c > 0 && !withhold) {                    // chunk aggregate, as early as possible
+                // every lane's store is ordered before lane 0's release by the warp barrier
                 a.lb_agg[(lb_base + k) * HALF + m] = make_float2(aggA, aggH);
-                __threadfence();
                 __syncwarp();
                 if (lane == 0) st_release_gpu(myflag, FLAG_AGG);
             }
@@ -789,18 +816,26 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     }
                 }
                 if (ready) {
+                    // the loads of a batch are independent (one L2 round trip per batch); the
+                    // combine stays in chunk order; padding entries are the identity (1, 0)
                     float hc = __ldcg(a.lb_incl + (kb_item + anc) * HALF + m);
-                    for (int i = 0; i < nagg; ++i) {
-                        const float2 g = __ldcg(a.lb_agg + (kb_item + anc + 1 + i) * HALF + m);
-                        hc = fmaf(g.x, hc, g.y);
+                    const float2* ag = a.lb_agg + (kb_item + anc + 1) * HALF + m;
+                    constexpr int kBatch = 8;
+#pragma unroll 1
+                    for (int i0 = 0; i0 < nagg; i0 += kBatch) {
+                        float2 g[kBatch];
+#pragma unroll
+                        for (int i = 0; i < kBatch; ++i)
+                            g[i] = i0 + i < nagg ? __ldcg(ag + (size_t)(i0 + i) * HALF) : make_float2(1.f, 0.f);
+#pragma unroll
+                        for (int i = 0; i < kBatch; ++i) hc = fmaf(g[i].x, hc, g[i].y);
                     }
                     carry = hc;
                 }
             }
             const float incl = fmaf(aggA, carry, aggH);             // state after the chunk
-            if (!withhold) {
+            if (c % LBW == 0 && !withhold) {             // only anchors' inclusive states are read
                 a.lb_incl[(lb_base + k) * HALF + m] = incl;
-                __threadfence();
                 __syncwarp();
                 if (lane == 0) st_release_gpu(myflag, FLAG_INCL);
             }
