@@ -76,10 +76,11 @@ constexpr int kConvTok = L / 2;         // tokens per conv warp
 
 // warp roles: 0-3 conv (channel half = warp % 2, token half = warp / 2), 4-19 epilogue (TMEM
 // lane quarter = warp % 4, group = stage = (warp - 4) / 4), 20 x producer (x tiles and
-// tickets), 21 y producer, 22 MMA.
+// tickets), 21 y producer, 22-23 MMA issuers (even / odd items: one thread issues the tensor
+// core instructions of an item, and one alone cannot keep up).
 constexpr int kConvWarps = 4, kEpiGroups = STAGES, kEpiGroup = 4, kEpiWarps = kEpiGroups * kEpiGroup;
-constexpr int kWarpEpi0 = 4, kWarpProdX = 20, kWarpProdY = 21, kWarpMma = 22;
-constexpr int kThreads = 23 * 32;
+constexpr int kWarpEpi0 = 4, kWarpProdX = 20, kWarpProdY = 21, kWarpMma = 22, kMmaWarps = 2;
+constexpr int kThreads = 24 * 32;
 
 constexpr uint32_t X_BYTES = XROWS * DH * 2;      // 17920
 constexpr uint32_t Y_BYTES = L * HALF * 2;        // 8192
@@ -387,7 +388,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             mbar_init(bars.slot_free[s], 1);
         }
         mbar_init(bars.w_ready, kEpiWarps);
-        mbar_init(bars.mma_done, 1);
+        mbar_init(bars.mma_done, kMmaWarps);
         *abort = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -524,22 +525,25 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     }
                 }
         }
-    } else if (warp == kWarpMma) {
-        // ================================ MMA issuer ===========================================
+    } else if (warp >= kWarpMma && warp < kWarpMma + kMmaWarps) {
+        // ================================ MMA issuers ==========================================
+        // issuer i takes the items n = i (mod kMmaWarps); at the end of the work each one hands
+        // the terminal item to the epilogue groups of its own next iterations
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(HALF, L);
             bool ok = wait_bar(bars.w_ready, 0, wc, 3);
             tc_fence_after();
-            for (int n = 0; ok; ++n) {
+            for (int n = warp - kWarpMma; ok; n += kMmaWarps) {
                 const int st = n % STAGES;
                 const uint32_t ph = (n / STAGES) & 1;
                 if (!wait_bar(bars.b_full[st], ph, wc, 4)) break;
                 if (!wait_bar(bars.acc_empty[st], ph ^ 1, wc, 5)) break;
                 if (slot[n & (SLOTS - 1)] < 0) {
-                    // hand the terminal item to every epilogue group: group st now, each other
-                    // group once it has released its previous item (so that no phase is skipped)
+                    // hand the terminal item to the groups of iterations n, n + kMmaWarps, ...:
+                    // group st now, each other one once it has released its previous item (so
+                    // that no phase is skipped)
                     mbar_arrive(bars.acc_full[st]);
-                    for (int i = 1; i < STAGES; ++i) {
+                    for (int i = kMmaWarps; i < STAGES; i += kMmaWarps) {
                         const int s2 = (n + i) % STAGES;
                         const uint32_t ph2 = ((n + i) / STAGES) & 1;
                         if (wait_bar(bars.acc_empty[s2], ph2 ^ 1, wc, 17)) mbar_arrive(bars.acc_full[s2]);
@@ -596,8 +600,10 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             if (!wait_bar_warp(bars.b_empty[st], ph ^ 1, wc, 7)) break;
             const int k = slot[n & (SLOTS - 1)];
             if (k < 0) {
+                // every MMA issuer meets the end of the work at its own next iteration
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bars.b_full[st]);
+                if (lane == 0)
+                    for (int i = 0; i < kMmaWarps; ++i) mbar_arrive(bars.b_full[(n + i) % STAGES]);
                 break;
             }
             const int b = k / a.NC, c = k % a.NC, t0 = c * L;
