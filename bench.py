@@ -374,6 +374,8 @@ def bench_decode(args, dev):
     from gated_linear_recurrence_conv1d_b200 import binding
 
     wl = inputs.WORKLOADS[DECODE_WORKLOAD]
+    if args.decode_steps > 0:
+        wl = wl.scaled(decode_steps=args.decode_steps)
     steps = wl.decode_steps
     prob = inputs.make_problem(wl, seed=0)
     block = binding.RGLRUBlock(prob.params, wl.heads, wl.head_dim, wl.dtype, dev)
@@ -438,12 +440,20 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode workload (prints its JSON object)")
+    ap.add_argument("--decode-steps", type=int, default=0,
+                    help="decode steps per graph replay (default: the workload's 1024)")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.decode_only:
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device())
+        print(json.dumps(bench_decode(args, dev)))
     else:
         run_ours(args)
 

@@ -174,8 +174,9 @@ rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_params* para
     if ((st = check_workspace(workspace, workspace_bytes, rglru_decode_workspace_size(dims))) != RGLRU_OK)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the tensor-core step reads and writes h with 16-byte vectors
-    if (rglru::fused_decode_supported(dims) && aligned(state->h, 16))
+    // the tensor-core step reads h and the conv parameters with 16-byte vectors
+    if (rglru::fused_decode_supported(dims) && aligned(state->h, 16) && aligned(params->conv_w, 16) &&
+        (!params->conv_b || aligned(params->conv_b, 16)))
         return cuda_status(rglru::launch_fused_decode(dims, params, x, y, reset, state, out, workspace,
                                                       workspace_bytes, s));
     return cuda_status(rglru::launch_decode_generic(dims, params, x, y, reset, state, out, s));

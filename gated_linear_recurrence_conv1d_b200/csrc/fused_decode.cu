@@ -141,6 +141,24 @@ conv_shift_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* tail, cons
         t1 = *reinterpret_cast<const uint4*>(tl + W);
         t2 = *reinterpret_cast<const uint4*>(tl + 2 * W);
     }
+    // taps k = 0..3 (oldest .. current) and the bias of these 8 channels, 16-byte loads
+    float wk[kConvWidth][8], bias[8];
+#pragma unroll
+    for (int k = 0; k < kConvWidth; ++k) {
+        const float4 w0 = *reinterpret_cast<const float4*>(conv_w + (size_t)k * W + c8);
+        const float4 w1 = *reinterpret_cast<const float4*>(conv_w + (size_t)k * W + c8 + 4);
+        wk[k][0] = w0.x; wk[k][1] = w0.y; wk[k][2] = w0.z; wk[k][3] = w0.w;
+        wk[k][4] = w1.x; wk[k][5] = w1.y; wk[k][6] = w1.z; wk[k][7] = w1.w;
+    }
+    if (conv_b) {
+        const float4 b0 = *reinterpret_cast<const float4*>(conv_b + c8);
+        const float4 b1 = *reinterpret_cast<const float4*>(conv_b + c8 + 4);
+        bias[0] = b0.x; bias[1] = b0.y; bias[2] = b0.z; bias[3] = b0.w;
+        bias[4] = b1.x; bias[5] = b1.y; bias[6] = b1.z; bias[7] = b1.w;
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) bias[e] = 0.f;
+    }
     const uint32_t* px = reinterpret_cast<const uint32_t*>(&xv);
     const uint32_t* p0 = reinterpret_cast<const uint32_t*>(&t0);
     const uint32_t* p1 = reinterpret_cast<const uint32_t*>(&t1);
@@ -149,20 +167,18 @@ conv_shift_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* tail, cons
     uint32_t* po = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int ch = c8 + 2 * i;
         float r[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
+            const int c = 2 * i + e;
             const float v0 = e ? bf16hi(p0[i]) : bf16lo(p0[i]);
             const float v1 = e ? bf16hi(p1[i]) : bf16lo(p1[i]);
             const float v2 = e ? bf16hi(p2[i]) : bf16lo(p2[i]);
             const float v3 = e ? bf16hi(px[i]) : bf16lo(px[i]);
-            float acc = conv_b ? conv_b[ch + e] : 0.f;
-            acc = fmaf(conv_w[ch + e], v0, acc);
-            acc = fmaf(conv_w[(size_t)W + ch + e], v1, acc);
-            acc = fmaf(conv_w[(size_t)2 * W + ch + e], v2, acc);
-            acc = fmaf(conv_w[(size_t)3 * W + ch + e], v3, acc);
-            r[e] = acc;
+            float acc = fmaf(wk[0][c], v0, bias[c]);
+            acc = fmaf(wk[1][c], v1, acc);
+            acc = fmaf(wk[2][c], v2, acc);
+            r[e] = fmaf(wk[3][c], v3, acc);
         }
         po[i] = pack_bf16x2(r[0], r[1]);
     }
@@ -257,90 +273,81 @@ decode_gates_kernel(const __grid_constant__ CUtensorMap map_xc, const __grid_con
         const bool valid = b < a.B;
         const float gk1 = a.gelu_tanh ? 2.0f * 0.79788456080286535588f : 2.0f * 0.79879267f;
         const float gk3 = a.gelu_tanh ? 8.0f * 0.044715f * 0.79788456080286535588f : 8.0f * 0.03528805f;
+        // this row's state and y while the tensor cores run (rows past the batch read nothing)
+        const bool rst = valid && a.reset && a.reset[b];
+        const size_t off = (size_t)(valid ? b : 0) * W + ch0 + cg * 32;
+        float* hp = a.h + off;
+        const __nv_bfloat16* yp = a.y + off;
+        __nv_bfloat16* op = a.out + off;
+        float4 hq[8];
+        uint4 yq[4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            hq[i] = (valid && !rst) ? *reinterpret_cast<const float4*>(hp + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) yq[i] = valid ? *reinterpret_cast<const uint4*>(yp + 8 * i) : make_uint4(0, 0, 0, 0);
         // uniform across the warp: the TMEM loads below are warp-collective
         const bool ok = __all_sync(0xffffffffu, wait_bounded(bar_acc, 0, a, abort, 2));
         tc_fence_after();
         const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + cg * 32;
-        float ga[32], gx[32];
-        {
-            float t[16];
-            tmem_ld16(taddr, t);
+        const int cbase = nt * NT + cg * 32;              // channel within the head
 #pragma unroll
-            for (int j = 0; j < 16; ++j) ga[j] = t[j];
-            tmem_ld16(taddr + 16, t);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) ga[16 + j] = t[j];
-            tmem_ld16(taddr + NT, t);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) gx[j] = t[j];
-            tmem_ld16(taddr + NT + 16, t);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) gx[16 + j] = t[j];
+        for (int v = 0; v < 4; ++v) {                     // 8 channels per step
+            float ga[8], gx[8];
+            tmem_ld8(taddr + v * 8, ga);
+            tmem_ld8(taddr + NT + v * 8, gx);
             tmem_wait_ld();
-        }
-        if (ok && valid) {
-            const bool rst = a.reset && a.reset[b];
-            const size_t off = (size_t)b * W + ch0 + cg * 32;
-            float* hp = a.h + off;
-            const __nv_bfloat16* yp = a.y + off;
-            __nv_bfloat16* op = a.out + off;
-            // conv output of this row: 16-byte chunks of the swizzled A tile
-            const int cbase = nt * NT + cg * 32;          // channel within the head
+            if (!(ok && valid)) continue;
+            // conv output of this row: a 16-byte chunk of the swizzled A tile
+            const int cl = cbase + v * 8;
+            const uint32_t aoff = (uint32_t)(cl >> 6) * A_KBLK + (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128 +
+                                  ((uint32_t)(((cl & 63) >> 3) ^ (r & 7)) << 4);
+            const uint4 xq = *reinterpret_cast<const uint4*>(smem + OFF_A + aoff);
+            float hv[8];
+            const float4 h0 = hq[2 * v], h1 = hq[2 * v + 1];
+            hv[0] = h0.x; hv[1] = h0.y; hv[2] = h0.z; hv[3] = h0.w;
+            hv[4] = h1.x; hv[5] = h1.y; hv[6] = h1.z; hv[7] = h1.w;
+            const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xq);
+            const uint32_t* yw = reinterpret_cast<const uint32_t*>(&yq[v]);
+            uint32_t ow[4];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {                 // 8 channels per step
-                const int cl = cbase + v * 8;
-                const uint32_t aoff = (uint32_t)(cl >> 6) * A_KBLK + (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128 +
-                                      ((uint32_t)(((cl & 63) >> 3) ^ (r & 7)) << 4);
-                const uint4 xq = *reinterpret_cast<const uint4*>(smem + OFF_A + aoff);
-                const uint4 yq = *reinterpret_cast<const uint4*>(yp + v * 8);
-                float4 h0 = make_float4(0.f, 0.f, 0.f, 0.f), h1 = h0;
-                if (!rst) {
-                    h0 = *reinterpret_cast<const float4*>(hp + v * 8);
-                    h1 = *reinterpret_cast<const float4*>(hp + v * 8 + 4);
-                }
-                float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-                const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xq);
-                const uint32_t* yw = reinterpret_cast<const uint32_t*>(&yq);
-                uint32_t ow[4];
+            for (int e2 = 0; e2 < 4; ++e2) {
+                float o[2];
 #pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    float o[2];
-#pragma unroll
-                    for (int e1 = 0; e1 < 2; ++e1) {
-                        const int e = 2 * e2 + e1;
-                        const int jc = cg * 32 + v * 8 + e;   // column within the tile
-                        const float xcv = e1 ? bf16hi(xw[e2]) : bf16lo(xw[e2]);
-                        const float yv = e1 ? bf16hi(yw[e2]) : bf16lo(yw[e2]);
-                        const float hk = s_hk[jc];
-                        const float da = fmaf(ga[v * 8 + e], 0.5f, s_ba[jc]);
-                        const float dx = fmaf(gx[v * 8 + e], 0.5f, s_bx[jc]);
-                        const float l = fmaf(tanh_approx(da), hk, hk);
-                        float em;
-                        if (l > -0.125f) {
-                            float pp = fmaf(l, 1.0f / 24.0f, 1.0f / 6.0f);
-                            pp = fmaf(l, pp, 0.5f);
-                            pp = fmaf(l, pp, 1.0f);
-                            em = l * pp;
-                        } else {
-                            em = ex2_approx(l * 1.4426950408889634f) - 1.0f;
-                        }
-                        const float at = 1.0f + em;
-                        const float bh = sqrt_approx(em * fmaf(em, -0.25f, -0.5f));
-                        const float w = bh * xcv;
-                        const float u = fmaf(w, tanh_approx(dx), w);
-                        const float hn = fmaf(at, hv[e], u);
-                        hv[e] = hn;
-                        const float hy = 0.5f * yv;
-                        const float t = tanh_approx(hy * fmaf(hy * hy, gk3, gk1));
-                        const float m = hn * hy;
-                        o[e1] = fmaf(m, t, m);
+                for (int e1 = 0; e1 < 2; ++e1) {
+                    const int e = 2 * e2 + e1;
+                    const int jc = cg * 32 + v * 8 + e;   // column within the tile
+                    const float xcv = e1 ? bf16hi(xw[e2]) : bf16lo(xw[e2]);
+                    const float yv = e1 ? bf16hi(yw[e2]) : bf16lo(yw[e2]);
+                    const float hk = s_hk[jc];
+                    const float da = fmaf(ga[e], 0.5f, s_ba[jc]);
+                    const float dx = fmaf(gx[e], 0.5f, s_bx[jc]);
+                    const float l = fmaf(tanh_approx(da), hk, hk);
+                    float em;
+                    if (l > -0.125f) {
+                        float pp = fmaf(l, 1.0f / 24.0f, 1.0f / 6.0f);
+                        pp = fmaf(l, pp, 0.5f);
+                        pp = fmaf(l, pp, 1.0f);
+                        em = l * pp;
+                    } else {
+                        em = ex2_approx(l * 1.4426950408889634f) - 1.0f;
                     }
-                    ow[e2] = pack_bf16x2(o[0], o[1]);
+                    const float at = 1.0f + em;
+                    const float bh = sqrt_approx(em * fmaf(em, -0.25f, -0.5f));
+                    const float w = bh * xcv;
+                    const float u = fmaf(w, tanh_approx(dx), w);
+                    const float hn = fmaf(at, hv[e], u);
+                    hv[e] = hn;
+                    const float hy = 0.5f * yv;
+                    const float t = tanh_approx(hy * fmaf(hy * hy, gk3, gk1));
+                    const float m = hn * hy;
+                    o[e1] = fmaf(m, t, m);
                 }
-                *reinterpret_cast<float4*>(hp + v * 8) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-                *reinterpret_cast<float4*>(hp + v * 8 + 4) = make_float4(hv[4], hv[5], hv[6], hv[7]);
-                *reinterpret_cast<uint4*>(op + v * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                ow[e2] = pack_bf16x2(o[0], o[1]);
             }
+            *reinterpret_cast<float4*>(hp + v * 8) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<float4*>(hp + v * 8 + 4) = make_float4(hv[4], hv[5], hv[6], hv[7]);
+            *reinterpret_cast<uint4*>(op + v * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         }
     }
     tc_fence_before();
