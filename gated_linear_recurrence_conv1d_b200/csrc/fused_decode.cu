@@ -128,6 +128,9 @@ __device__ bool wait_bounded(uint32_t bar, uint32_t parity, const Args& a, volat
 __global__ void __launch_bounds__(256)
 conv_shift_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* tail, const float* __restrict__ conv_w,
                   const float* __restrict__ conv_b, const uint8_t* __restrict__ reset, __nv_bfloat16* xc, int B, int W) {
+    // the gate kernel that follows may start its set-up now: it waits for this grid before it
+    // reads the conv output
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int groups = W / 8;
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= (long long)B * groups) return;
@@ -238,10 +241,14 @@ decode_gates_kernel(const __grid_constant__ CUtensorMap map_xc, const __grid_con
             prefetch_tensormap(&map_wx);
             mbar_arrive_expect_tx(bar_full, A_BYTES + 2 * B_BYTES);
             for (int kb = 0; kb < DH / 64; ++kb) {
-                tma_load_2d(sbase + OFF_A + kb * A_KBLK, &map_xc, head * DH + kb * 64, mt * MT, bar_full);
                 tma_load_2d(sbase + OFF_BA + kb * 8192, &map_wa, nt * NT, head * DH + kb * 64, bar_full);
                 tma_load_2d(sbase + OFF_BX + kb * 8192, &map_wx, nt * NT, head * DH + kb * 64, bar_full);
             }
+            // the conv output is written by the preceding conv kernel (a no-op without a
+            // programmatic launch dependency)
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            for (int kb = 0; kb < DH / 64; ++kb)
+                tma_load_2d(sbase + OFF_A + kb * A_KBLK, &map_xc, head * DH + kb * 64, mt * MT, bar_full);
             // never leave the CTA with a bulk copy still writing its shared memory
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait_sleep(bar_full, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
@@ -407,8 +414,20 @@ cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, cons
     a.h = st->h;
     a.out = static_cast<__nv_bfloat16*>(out);
     a.status = reinterpret_cast<DeviceStatus*>(ws);
-    const int grid = H * a.mtiles * (DH / NT);
-    decode_gates_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(mxc, mwa, mwx, a);
+    // programmatic dependent launch: this kernel's set-up (barriers, TMEM, constants, weight
+    // tiles, state prefetch) overlaps the conv kernel; it waits for it before loading the conv
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(H * a.mtiles * (DH / NT)));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_gates_kernel, mxc, mwa, mwx, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
