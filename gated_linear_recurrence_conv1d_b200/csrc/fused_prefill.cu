@@ -6,17 +6,19 @@
 //     block-diagonal gate weights W_a[h][:, half], W_x[h][:, half], pre-scaled by 1/2 (exact
 //     in bf16), are written once into tensor memory (TMEM) and used as the A operand of
 //     tcgen05.mma (TS form), so shared memory only holds streamed tiles;
-//   * work items are (batch row, 64-token chunk) of the group, handed out by a per-group
-//     atomic ticket so every CTA of a group stays busy and an item's predecessor is always
-//     held by a running CTA;
+//   * work items are (batch row, 32-token chunk) of the group, handed out by a per-group
+//     atomic ticket so every CTA of a group stays busy and an item's predecessors are always
+//     held by running CTAs; 4 stages of shared-memory tiles and of TMEM accumulators are in
+//     flight per CTA;
 //   * warp roles: an x producer (TMA: x tile with a 3-token halo, and the ticket), a y producer
-//     (TMA: y tile, issued once the previous out store of that stage has left shared memory),
-//     4 conv warps (one 16-token quarter of the chunk each; a lane convolves 8 channels with
-//     16-byte shared-memory loads and writes them as the bf16 B operand in the 128-byte
-//     swizzled K-major layout), 1 MMA thread (D = W^T/2 . xc^T for both gates, K = 256 in 16
-//     steps, accumulated onto the gate biases that the epilogue pre-loads into TMEM), and 2
-//     epilogue groups of 4 warps, group g owning TMEM stage g;
-//   * transposed orientation: a TMEM lane is an output channel and the 64 columns are tokens,
+//     (TMA: y tile, paced by a slot handshake with the x producer and by the out store of the
+//     stage's previous item), 8 conv warps (a channel half and a quarter of the chunk's tokens
+//     each; a lane convolves 4 channels with 8-byte shared-memory loads and writes them as the
+//     bf16 B operand in the 128-byte swizzled K-major layout), 2 MMA issuer threads (even / odd
+//     items; D = W^T/2 . xc^T for both gates, K = 256 in 16 steps, accumulated onto the gate
+//     biases that the epilogue pre-loads into TMEM), and 4 epilogue groups of 4 warps, group g
+//     owning TMEM stage g;
+//   * transposed orientation: a TMEM lane is an output channel and the 32 columns are tokens,
 //     so an epilogue thread owns one channel and runs the diagonal scan along its registers
 //     (no shuffles); its first pass leaves the running (prod a, local h) of every token in
 //     TMEM, so once the carry C is known the second pass is h_t = P_t C + h_t^loc;
@@ -72,15 +74,15 @@ constexpr int KSTEPS = DH / 16;         // MMA K steps
 constexpr int STAGES = 4;               // x / B / y tiles and TMEM accumulator slots
 constexpr int SLOTS = 16;               // ring of item ids, indexed by iteration (> the producers' lag)
 constexpr int kBlk = 8;                 // tokens per TMEM load block in the epilogue
-constexpr int kConvTok = L / 2;         // tokens per conv warp
+constexpr int kConvTok = L / 4;         // tokens per conv warp
 
-// warp roles: 0-3 conv (channel half = warp % 2, token half = warp / 2), 4-19 epilogue (TMEM
-// lane quarter = warp % 4, group = stage = (warp - 4) / 4), 20 x producer (x tiles and
-// tickets), 21 y producer, 22-23 MMA issuers (even / odd items: one thread issues the tensor
+// warp roles: 0-7 conv (channel half = warp % 2, token quarter = warp / 2), 8-23 epilogue (TMEM
+// lane quarter = warp % 4, group = stage = (warp - 8) / 4), 24 x producer (x tiles and
+// tickets), 25 y producer, 26-27 MMA issuers (even / odd items: one thread issues the tensor
 // core instructions of an item, and one alone cannot keep up).
-constexpr int kConvWarps = 4, kEpiGroups = STAGES, kEpiGroup = 4, kEpiWarps = kEpiGroups * kEpiGroup;
-constexpr int kWarpEpi0 = 4, kWarpProdX = 20, kWarpProdY = 21, kWarpMma = 22, kMmaWarps = 2;
-constexpr int kThreads = 24 * 32;
+constexpr int kConvWarps = 8, kEpiGroups = STAGES, kEpiGroup = 4, kEpiWarps = kEpiGroups * kEpiGroup;
+constexpr int kWarpEpi0 = 8, kWarpProdX = 24, kWarpProdY = 25, kWarpMma = 26, kMmaWarps = 2;
+constexpr int kThreads = 28 * 32;
 
 constexpr uint32_t X_BYTES = XROWS * DH * 2;      // 17920
 constexpr uint32_t Y_BYTES = L * HALF * 2;        // 8192
@@ -573,7 +575,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     } else if (warp < kConvWarps) {
         // ================================ conv warps ==========================================
         // warp w convolves channels [128 (w % 2), +128) of the head for the tokens
-        // [16 (w / 2), +16) of the chunk; lane l 4 channels (8 bytes of a B-tile row)
+        // [8 (w / 2), +8) of the chunk; lane l 4 channels (8 bytes of a B-tile row)
         const int chh = warp & 1;
         const int j0 = (warp >> 1) * kConvTok;
         const int cl = chh * HALF + lane * 4;             // channel within the head
