@@ -17,6 +17,7 @@ import torch
 from . import build as _build
 
 RGLRU_OK = 0
+RGLRU_ERR_CUDA = 4
 RGLRU_ERR_TIMEOUT = 5
 RGLRU_ERR_DEVICE = 6
 RGLRU_F32, RGLRU_BF16 = 0, 1
@@ -30,16 +31,16 @@ STATUS_NAMES = {0: "RGLRU_OK", 1: "RGLRU_ERR_INVALID_ARG", 2: "RGLRU_ERR_UNSUPPO
 EXPORTED = ("rglru_state_init", "rglru_prefill_workspace_size", "rglru_block_prefill",
             "rglru_decode_workspace_size", "rglru_block_decode", "rglru_read_device_status",
             "rglru_status_string", "rglru_abi_version", "rglru_prefill_plan", "rglru_decode_plan",
-            "rglru_block_prefill_noalloc")
+            "rglru_block_prefill_noalloc", "rglru_last_cuda_error")
 
 # Bytes of the static device scratch behind rglru_block_prefill_noalloc.
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class RglruError(RuntimeError):
-    def __init__(self, status: int, where: str):
+    def __init__(self, status: int, where: str, detail: str = ""):
         self.status = status
-        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}{detail}")
 
 
 class Dims(ctypes.Structure):
@@ -100,6 +101,8 @@ def load(build_if_missing: bool = True):
     lib.rglru_prefill_plan.restype = I
     lib.rglru_decode_plan.argtypes = [PD, PI, PI]
     lib.rglru_decode_plan.restype = I
+    lib.rglru_last_cuda_error.argtypes = [ctypes.POINTER(ctypes.c_char_p)]
+    lib.rglru_last_cuda_error.restype = I
     lib.rglru_abi_version.argtypes = []
     lib.rglru_abi_version.restype = I
     _lib = lib
@@ -138,9 +141,20 @@ def make_params(p: dict) -> Params:
     return Params(*(_ptr(p.get(k)) for k in ("conv_w", "conv_b", "w_a", "w_x", "b_a", "b_x", "lam")))
 
 
+def last_cuda_error() -> tuple:
+    """(cudaError_t value, its name) behind this thread's most recent RGLRU_ERR_CUDA."""
+    name = ctypes.c_char_p()
+    code = load().rglru_last_cuda_error(ctypes.byref(name))
+    return code, (name.value or b"").decode()
+
+
 def _check(status: int, where: str):
     if status != RGLRU_OK:
-        raise RglruError(status, where)
+        detail = ""
+        if status == RGLRU_ERR_CUDA:
+            code, name = last_cuda_error()
+            detail = f" ({name}, {code})"
+        raise RglruError(status, where, detail)
 
 
 def prefill_workspace_size(dims: Dims) -> int:

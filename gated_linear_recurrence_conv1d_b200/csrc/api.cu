@@ -65,8 +65,12 @@ rglru_status check_workspace(void* ws, size_t bytes, size_t need) {
     return RGLRU_OK;
 }
 
+// CUDA error behind the calling thread's most recent RGLRU_ERR_CUDA
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
 rglru_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return RGLRU_OK;
+    t_last_cuda_error = e;
     cudaGetLastError();   // clear a sticky launch-configuration error for the caller
     return RGLRU_ERR_CUDA;
 }
@@ -174,9 +178,8 @@ rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_params* para
     if ((st = check_workspace(workspace, workspace_bytes, rglru_decode_workspace_size(dims))) != RGLRU_OK)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the tensor-core step reads h and the conv parameters with 16-byte vectors
-    if (rglru::fused_decode_supported(dims) && aligned(state->h, 16) && aligned(params->conv_w, 16) &&
-        (!params->conv_b || aligned(params->conv_b, 16)))
+    // the tensor-core step reads and writes h with 16-byte vectors
+    if (rglru::fused_decode_supported(dims) && aligned(state->h, 16))
         return cuda_status(rglru::launch_fused_decode(dims, params, x, y, reset, state, out, workspace,
                                                       workspace_bytes, s));
     return cuda_status(rglru::launch_decode_generic(dims, params, x, y, reset, state, out, s));
@@ -248,3 +251,8 @@ rglru_status rglru_read_device_status(void* workspace, size_t workspace_bytes, v
 }
 
 }  // extern "C"
+
+int rglru_last_cuda_error(const char** name) {
+    if (name) *name = cudaGetErrorName(t_last_cuda_error);
+    return (int)t_last_cuda_error;
+}

@@ -3,18 +3,24 @@
 // A decode step updates every batch row by one token.  There is no recurrence across tokens
 // inside a call, so the batch is the parallel dimension and the gate contraction is a plain
 // GEMM per head: D[row, o] = sum_i xc[row, i] W[h][i][o] with M = rows, N = output channels,
-// K = 256 input channels.  Two launches:
+// K = 256 input channels.  One launch; a cluster of 4 CTAs per (head, 128-row tile), CTA r
+// owning the 64 channels [64 r, 64 r + 64) of the head:
 //
-//   1. conv_shift_kernel: per (row, 8 channels) the width-4 causal conv over the carried
-//      history and the new input, written as bf16 into workspace scratch (it is the tensor-core
-//      operand), and the history shifted in place (oldest out, x in).  A row with reset[b] set
-//      starts from an empty history.
-//   2. decode_gates_kernel: a CTA per (head, 128-row tile, 64-channel tile).  TMA brings the
-//      128 x 256 conv tile (K-major, 128-byte swizzle) and the 256 x 64 slices of W_a, W_x
-//      (as stored: output channel contiguous, i.e. MN-major for the MMA) into shared memory;
-//      one thread issues tcgen05.mma (M = 128, N = 64, K = 256 per gate) into TMEM; 8 epilogue
-//      warps (thread = row, 32 channels each) read the accumulators, apply the gates, update
-//      the fp32 state h in place and write out = h * GeLU(y) with 16-byte vector accesses.
+//   * conv: CTA r convolves its own 64 channels for the 128 rows (the width-4 causal conv over
+//     the carried history and the new input), shifts their history in place (oldest out, x in;
+//     a row with reset[b] set starts from an empty history), and writes the bf16 result as
+//     K-block r of its 128 x 256 MMA operand tile (K-major, 128-byte swizzle); one thread then
+//     copies that 16 KB block into the same place of the three sibling CTAs' tiles through
+//     distributed shared memory (bulk copies that complete on the siblings' mbarrier), so every
+//     channel is convolved once and only by the CTA that owns its history;
+//   * gates: TMA brings the 256 x 64 slices W_a[h][:, 64 r], W_x[h][:, 64 r] (as stored: output
+//     channel contiguous, i.e. MN-major for the MMA) side by side, one N = 128 operand; one
+//     thread issues tcgen05.mma (M = 128, N = 128, K = 16 each) into TMEM, K block by K block as
+//     the blocks become ready (its own first);
+//   * update: TMA also brings the h (fp32) and y tiles of the CTA into shared memory; 16 warps
+//     (thread = row, 16 channels each) compute GeLU(y) while the MMAs run, then read the
+//     accumulators, apply the gates and write h and out back into the shared tiles, which TMA
+//     stores (rows past the batch are clipped by the tensor maps).
 //
 // The element-wise arithmetic is that of the prefill kernel (fused_prefill.cu): one tanh per
 // gate, expm1 of the log-decay by its series near zero, sqrt(1 - a^2) without cancellation,
@@ -38,6 +44,8 @@ namespace rglru {
 namespace tc {
 bool make_map_2d_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                        uint32_t box_inner, uint32_t box_outer);
+bool make_map_2d_sw128_elem(CUtensorMap* m, const void* base, uint32_t elem_bytes, uint64_t inner, uint64_t outer,
+                            uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 }
 
 namespace dec {
@@ -48,23 +56,37 @@ constexpr int DH = 256;
 constexpr int MT = 128;                 // rows per CTA (MMA M, TMEM lanes)
 constexpr int NT = 64;                  // output channels per CTA (MMA N)
 constexpr int KSTEPS = DH / 16;
-constexpr int kWarpMma = 8, kWarpTma = 9;     // warps 0-7: epilogue (4 lane quarters x 2 channel halves)
-constexpr int kThreads = 10 * 32;
+constexpr int kEpiWarps = 16;                 // 4 lane quarters x 4 quarters of the tile's channels
+constexpr int kWarpMma = kEpiWarps, kWarpTma = kEpiWarps + 1;
+constexpr int kThreads = (kEpiWarps + 2) * 32;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kEpiCh = NT / (kEpiWarps / 4);  // channels per update thread (16)
+constexpr int kConvUnits = MT * (NT / 8) / kEpiThreads;  // (row, 8 channels) conv units per thread (2)
 
 constexpr uint32_t A_BYTES = MT * DH * 2;            // 65536: 4 K-blocks of 128 rows x 128 B
 constexpr uint32_t A_KBLK = MT * 128;                // 16384
 constexpr uint32_t B_BYTES = DH * NT * 2;            // 32768 per gate: 256 K-rows x 128 B
+constexpr uint32_t H_BOX = MT * 128;                 // h tile: 2 boxes of 128 rows x 32 fp32
+constexpr uint32_t Y_BYTES = MT * NT * 2;            // y tile (then out): 128 rows x 64 bf16
 constexpr uint32_t OFF_A = 0;
 constexpr uint32_t OFF_BA = OFF_A + A_BYTES;
-constexpr uint32_t OFF_BX = OFF_BA + B_BYTES;
-constexpr uint32_t OFF_CONST = OFF_BX + B_BYTES;     // hk, b_a / 2, b_x / 2 per channel: 3 x 64 fp32
-constexpr uint32_t OFF_BAR = OFF_CONST + 3 * NT * 4;
-constexpr uint32_t OFF_MISC = OFF_BAR + 32;
+constexpr uint32_t OFF_BX = OFF_BA + B_BYTES;        // right after W_a: one N = 128 operand
+constexpr uint32_t OFF_H = OFF_BX + B_BYTES;
+constexpr uint32_t OFF_Y = OFF_H + 2 * H_BOX;
+constexpr uint32_t OFF_CONST = OFF_Y + Y_BYTES;      // hk, b_a / 2, b_x / 2 per channel: 3 x 64 fp32
+constexpr uint32_t OFF_CONV = OFF_CONST + 3 * NT * 4; // conv taps [4][64] and bias [64], fp32
+constexpr uint32_t OFF_BAR = OFF_CONV + 5 * NT * 4;
+constexpr uint32_t OFF_MISC = OFF_BAR + 64;
+constexpr int kClusterSize = DH / NT;                 // CTAs of a (head, row tile)
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 32 + 1024;
 constexpr uint32_t TMEM_COLS = 128;                  // D_a [0,64), D_x [64,128)
 
 struct Args {
     int B, H, mtiles;
+    const __nv_bfloat16* x;
+    __nv_bfloat16* tail;
+    const float* conv_w;
+    const float* conv_b;
     float c;
     int gelu_tanh;
     unsigned long long timeout_ns;
@@ -72,9 +94,6 @@ struct Args {
     const float* b_x;
     const float* lambda;
     const uint8_t* reset;
-    const __nv_bfloat16* y;
-    float* h;
-    __nv_bfloat16* out;
     DeviceStatus* status;
 };
 
@@ -92,8 +111,9 @@ __device__ __forceinline__ float sqrt_approx(float x) {
 
 // Shared-memory matrix descriptor for an MN-major operand in the 128-byte swizzle layout: rows
 // of 128 B (64 bf16 along N) for consecutive K, 8-row atoms of 1024 B stacked along K at the
-// stride byte offset (1024 B); the leading byte offset (between 64-wide N atoms) is unused for
-// N = 64.  Same bit fields as desc_k_sw128.
+// stride byte offset (1024 B); the leading byte offset is the distance between 64-wide N atoms,
+// here from the W_a slice to the W_x slice, so that one N = 128 operand covers both gates.
+// Same bit fields as desc_k_sw128.
 __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr) {
     uint64_t d = 0;
     d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
@@ -124,198 +144,297 @@ __device__ bool wait_bounded(uint32_t bar, uint32_t parity, const Args& a, volat
     }
 }
 
-// ---------------------------------------------------------------- 1. conv + history shift --
-__global__ void __launch_bounds__(256)
-conv_shift_kernel(const __nv_bfloat16* __restrict__ x, __nv_bfloat16* tail, const float* __restrict__ conv_w,
-                  const float* __restrict__ conv_b, const uint8_t* __restrict__ reset, __nv_bfloat16* xc, int B, int W) {
-    // the gate kernel that follows may start its set-up now: it waits for this grid before it
-    // reads the conv output
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int groups = W / 8;
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (long long)B * groups) return;
-    const int b = (int)(idx / groups), c8 = (int)(idx % groups) * 8;
-    const size_t row = (size_t)b * W + c8;
-    __nv_bfloat16* tl = tail + (size_t)b * kHist * W + c8;
-    const uint4 xv = *reinterpret_cast<const uint4*>(x + row);
-    uint4 t0 = make_uint4(0, 0, 0, 0), t1 = t0, t2 = t0;
-    if (!(reset && reset[b])) {
-        t0 = *reinterpret_cast<const uint4*>(tl);
-        t1 = *reinterpret_cast<const uint4*>(tl + W);
-        t2 = *reinterpret_cast<const uint4*>(tl + 2 * W);
-    }
-    // taps k = 0..3 (oldest .. current) and the bias of these 8 channels, 16-byte loads
-    float wk[kConvWidth][8], bias[8];
-#pragma unroll
-    for (int k = 0; k < kConvWidth; ++k) {
-        const float4 w0 = *reinterpret_cast<const float4*>(conv_w + (size_t)k * W + c8);
-        const float4 w1 = *reinterpret_cast<const float4*>(conv_w + (size_t)k * W + c8 + 4);
-        wk[k][0] = w0.x; wk[k][1] = w0.y; wk[k][2] = w0.z; wk[k][3] = w0.w;
-        wk[k][4] = w1.x; wk[k][5] = w1.y; wk[k][6] = w1.z; wk[k][7] = w1.w;
-    }
-    if (conv_b) {
-        const float4 b0 = *reinterpret_cast<const float4*>(conv_b + c8);
-        const float4 b1 = *reinterpret_cast<const float4*>(conv_b + c8 + 4);
-        bias[0] = b0.x; bias[1] = b0.y; bias[2] = b0.z; bias[3] = b0.w;
-        bias[4] = b1.x; bias[5] = b1.y; bias[6] = b1.z; bias[7] = b1.w;
-    } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) bias[e] = 0.f;
-    }
-    const uint32_t* px = reinterpret_cast<const uint32_t*>(&xv);
-    const uint32_t* p0 = reinterpret_cast<const uint32_t*>(&t0);
-    const uint32_t* p1 = reinterpret_cast<const uint32_t*>(&t1);
-    const uint32_t* p2 = reinterpret_cast<const uint32_t*>(&t2);
-    uint4 o;
-    uint32_t* po = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float r[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int c = 2 * i + e;
-            const float v0 = e ? bf16hi(p0[i]) : bf16lo(p0[i]);
-            const float v1 = e ? bf16hi(p1[i]) : bf16lo(p1[i]);
-            const float v2 = e ? bf16hi(p2[i]) : bf16lo(p2[i]);
-            const float v3 = e ? bf16hi(px[i]) : bf16lo(px[i]);
-            float acc = fmaf(wk[0][c], v0, bias[c]);
-            acc = fmaf(wk[1][c], v1, acc);
-            acc = fmaf(wk[2][c], v2, acc);
-            r[e] = fmaf(wk[3][c], v3, acc);
-        }
-        po[i] = pack_bf16x2(r[0], r[1]);
-    }
-    *reinterpret_cast<uint4*>(xc + row) = o;
-    *reinterpret_cast<uint4*>(tl) = t1;
-    *reinterpret_cast<uint4*>(tl + W) = t2;
-    *reinterpret_cast<uint4*>(tl + 2 * W) = xv;
+// ---------------------------------------------------------------- cluster helpers -----------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of this CTA's shared address `a` in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+// copy `bytes` of this CTA's shared memory to another CTA's shared memory; completes on that
+// CTA's mbarrier (its transaction count)
+__device__ __forceinline__ void dsmem_copy(uint32_t dst_cluster, uint32_t src, uint32_t bytes, uint32_t bar_cluster) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst_cluster),
+                 "r"(src), "r"(bytes), "r"(bar_cluster)
+                 : "memory");
 }
 
-// ---------------------------------------------------------------- 2. gates + state update --
 __global__ void __launch_bounds__(kThreads, 1)
-decode_gates_kernel(const __grid_constant__ CUtensorMap map_xc, const __grid_constant__ CUtensorMap map_wa,
-                    const __grid_constant__ CUtensorMap map_wx, const Args a) {
+decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_constant__ CUtensorMap map_wx,
+                    const __grid_constant__ CUtensorMap map_h, const __grid_constant__ CUtensorMap map_y,
+                    const __grid_constant__ CUtensorMap map_out, const Args a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar_full = sbase + OFF_BAR, bar_acc = sbase + OFF_BAR + 8;
+    const uint32_t bar_w = sbase + OFF_BAR, bar_acc = sbase + OFF_BAR + 16;
+    const uint32_t bar_hy = sbase + OFF_BAR + 24;     // h and y tiles
+    // K block j of the operand tile: convolved here (j = rank) or copied in by CTA j
+    auto bar_k = [&](int j) { return sbase + OFF_BAR + 32 + 8 * (uint32_t)j; };
     volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 16);
     float* s_hk = reinterpret_cast<float*>(smem + OFF_CONST);
     float* s_ba = s_hk + NT;
     float* s_bx = s_ba + NT;
+    float* s_cw = reinterpret_cast<float*>(smem + OFF_CONV);   // [4][64]
+    float* s_cb = s_cw + 4 * NT;                                 // [64]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // CTA -> (head, row tile, channel tile); channel tiles of a head are adjacent
-    const int nt = blockIdx.x % (DH / NT);
-    const int mt = (blockIdx.x / (DH / NT)) % a.mtiles;
-    const int head = blockIdx.x / ((DH / NT) * a.mtiles);
+    // cluster = (head, row tile); rank = channel tile (blockIdx.x = (head * mtiles + mt) * 4 + rank)
+    const int nt = (int)cluster_ctarank();
+    const int mt = (blockIdx.x / kClusterSize) % a.mtiles;
+    const int head = blockIdx.x / (kClusterSize * a.mtiles);
     const int W = a.H * DH;
     const int ch0 = head * DH + nt * NT;                  // first global channel of the tile
 
+    // let the next step's CTAs start their set-up; they read nothing of ours before their wait
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
-        mbar_init(bar_full, 1);
+        mbar_init(bar_w, 1);
         mbar_init(bar_acc, 1);
+        mbar_init(bar_hy, 1);
+        for (int j = 0; j < kClusterSize; ++j) mbar_init(bar_k(j), 1);
         *abort = 0;
         fence_barrier_init();
-    }
-    if (threadIdx.x < NT) {
-        const int ch = ch0 + threadIdx.x;
-        s_hk[threadIdx.x] = 0.5f * a.c * log_sigmoid_acc(a.lambda[ch]);
-        s_ba[threadIdx.x] = a.b_a ? 0.5f * a.b_a[ch] : 0.f;
-        s_bx[threadIdx.x] = a.b_x ? 0.5f * a.b_x[ch] : 0.f;
+        for (int j = 0; j < kClusterSize; ++j)
+            if (j != nt) mbar_arrive_expect_tx(bar_k(j), A_KBLK);   // completed by CTA j's copy
     }
     if (warp == kWarpMma) {
         tmem_alloc(smem_u32((const void*)tmem_base_s), TMEM_COLS);
         tmem_relinquish();
     }
+    if (warp == kWarpTma && lane == 0) {
+        prefetch_tensormap(&map_wa);
+        prefetch_tensormap(&map_wx);
+        prefetch_tensormap(&map_h);
+        prefetch_tensormap(&map_y);
+        prefetch_tensormap(&map_out);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_s;
+    // every CTA of the cluster has initialised its barriers before any copy targets them
+    cluster_sync();
+    // everything above overlaps the previous kernel of the stream; global memory only from here
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == kWarpTma) {
         if (lane == 0) {
-            prefetch_tensormap(&map_xc);
-            prefetch_tensormap(&map_wa);
-            prefetch_tensormap(&map_wx);
-            mbar_arrive_expect_tx(bar_full, A_BYTES + 2 * B_BYTES);
+            mbar_arrive_expect_tx(bar_w, 2 * B_BYTES);
             for (int kb = 0; kb < DH / 64; ++kb) {
-                tma_load_2d(sbase + OFF_BA + kb * 8192, &map_wa, nt * NT, head * DH + kb * 64, bar_full);
-                tma_load_2d(sbase + OFF_BX + kb * 8192, &map_wx, nt * NT, head * DH + kb * 64, bar_full);
+                tma_load_2d(sbase + OFF_BA + kb * 8192, &map_wa, nt * NT, head * DH + kb * 64, bar_w);
+                tma_load_2d(sbase + OFF_BX + kb * 8192, &map_wx, nt * NT, head * DH + kb * 64, bar_w);
             }
-            // the conv output is written by the preceding conv kernel (a no-op without a
-            // programmatic launch dependency)
-            asm volatile("griddepcontrol.wait;" ::: "memory");
-            for (int kb = 0; kb < DH / 64; ++kb)
-                tma_load_2d(sbase + OFF_A + kb * A_KBLK, &map_xc, head * DH + kb * 64, mt * MT, bar_full);
-            // never leave the CTA with a bulk copy still writing its shared memory
+            // this tile's state and y (rows past the batch read as zeros)
+            mbar_arrive_expect_tx(bar_hy, 2 * H_BOX + Y_BYTES);
+            tma_load_2d(sbase + OFF_H, &map_h, ch0, mt * MT, bar_hy);
+            tma_load_2d(sbase + OFF_H + H_BOX, &map_h, ch0 + 32, mt * MT, bar_hy);
+            tma_load_2d(sbase + OFF_Y, &map_y, ch0, mt * MT, bar_hy);
+            // never leave the CTA with a bulk copy still writing its shared memory (the weight
+            // tiles, or a sibling's conv block, whose completion also ends the sibling's reads)
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait_sleep(bar_full, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
+            while (!mbar_try_wait_sleep(bar_w, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+            for (int j = 0; j < kClusterSize; ++j)
+                while (!mbar_try_wait_sleep(bar_k(j), 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
+                }
+            while (!mbar_try_wait_sleep(bar_hy, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
             }
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32_bmn(MT, NT);
-            if (wait_bounded(bar_full, 0, a, abort, 1)) {
+            const uint32_t idesc = idesc_bf16_f32_bmn(MT, 2 * NT);   // D_a | D_x
+            // K blocks in the order they become ready: this CTA's own first, then the siblings'
+            bool ok = wait_bounded(bar_w, 0, a, abort, 1);
+            uint32_t accum = 0;
+            for (int i = 0; i < kClusterSize && ok; ++i) {
+                const int j = (nt + i) % kClusterSize;
+                ok = wait_bounded(bar_k(j), 0, a, abort, 3);
+                if (!ok) break;
                 tc_fence_after();
-#pragma unroll 1
-                for (int g = 0; g < 2; ++g) {
-                    const uint32_t bsm = sbase + (g ? OFF_BX : OFF_BA);
 #pragma unroll
-                    for (int ks = 0; ks < KSTEPS; ++ks) {
-                        const uint64_t ad = desc_k_sw128(sbase + OFF_A + (ks >> 2) * A_KBLK + (ks & 3) * 32);
-                        const uint64_t bd = desc_mn_sw128(bsm + ks * 16 * 128);
-                        mma_ss(tmem + g * NT, ad, bd, idesc, ks > 0 ? 1u : 0u);
-                    }
+                for (int kk = 0; kk < KSTEPS / kClusterSize; ++kk) {
+                    const int ks = j * 4 + kk;
+                    const uint64_t ad = desc_k_sw128(sbase + OFF_A + j * A_KBLK + kk * 32);
+                    const uint64_t bd = desc_mn_sw128(sbase + OFF_BA + ks * 16 * 128);
+                    mma_ss(tmem, ad, bd, idesc, accum);
+                    accum = 1;
                 }
             }
-            mma_commit(bar_acc);     // also when the load failed: the epilogue must not wait forever
+            mma_commit(bar_acc);     // also when a wait failed: the epilogue must not wait forever
         }
     } else {
-        // ================================ epilogue ============================================
-        const int q = warp & 3, cg = warp >> 2;           // lane quarter, 32-channel half of the tile
+        // ================================ loads ================================================
+        // The per-channel constants (threads < 64, staged in shared memory), then the conv inputs of
+        // this thread's units (row rl = 64 k + tid / 8, channels 8 (tid % 8) .. +7 of the tile),
+        // issued together so their latencies overlap.
+        if (threadIdx.x < NT) {
+            const int ch = ch0 + threadIdx.x;
+            const float lam = a.lambda[ch];
+            const float ba = a.b_a ? a.b_a[ch] : 0.f;
+            const float bx = a.b_x ? a.b_x[ch] : 0.f;
+            const float cb0 = a.conv_b ? a.conv_b[ch] : 0.f;
+#pragma unroll
+            for (int k = 0; k < kConvWidth; ++k) s_cw[k * NT + threadIdx.x] = a.conv_w[(size_t)k * W + ch];
+            s_cb[threadIdx.x] = cb0;
+            s_hk[threadIdx.x] = 0.5f * a.c * log_sigmoid_acc(lam);
+            s_ba[threadIdx.x] = 0.5f * ba;
+            s_bx[threadIdx.x] = 0.5f * bx;
+        }
+        const int g8 = threadIdx.x & 7;
+        uint4 xv[kConvUnits], t0[kConvUnits], t1[kConvUnits], t2[kConvUnits];
+#pragma unroll
+        for (int k = 0; k < kConvUnits; ++k) {
+            const int rl = k * (kEpiThreads / 8) + (threadIdx.x >> 3);
+            const int bk = mt * MT + rl;
+            const int bs = bk < a.B ? bk : 0;                 // rows past the batch: any valid row
+            const __nv_bfloat16* tl = a.tail + (size_t)bs * kHist * W + ch0 + g8 * 8;
+            xv[k] = *reinterpret_cast<const uint4*>(a.x + (size_t)bs * W + ch0 + g8 * 8);
+            t0[k] = *reinterpret_cast<const uint4*>(tl);
+            t1[k] = *reinterpret_cast<const uint4*>(tl + W);
+            t2[k] = *reinterpret_cast<const uint4*>(tl + 2 * W);
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+
+        // ================================ conv of this CTA's channels ==========================
+        {
+            const uint32_t kblk = sbase + OFF_A + nt * A_KBLK;
+            float cw[4][8], cb[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+#pragma unroll
+                for (int k = 0; k < kConvWidth; ++k) cw[k][j] = s_cw[k * NT + g8 * 8 + j];
+                cb[j] = s_cb[g8 * 8 + j];
+            }
+#pragma unroll
+            for (int k = 0; k < kConvUnits; ++k) {
+                const int rl = k * (kEpiThreads / 8) + (threadIdx.x >> 3);
+                const int bk = mt * MT + rl;
+                uint4 o = make_uint4(0, 0, 0, 0);
+                if (bk < a.B) {
+                    if (a.reset && a.reset[bk]) {             // an empty history
+                        t0[k] = make_uint4(0, 0, 0, 0);
+                        t1[k] = t0[k];
+                        t2[k] = t0[k];
+                    }
+                    const uint32_t* px = reinterpret_cast<const uint32_t*>(&xv[k]);
+                    const uint32_t* p0 = reinterpret_cast<const uint32_t*>(&t0[k]);
+                    const uint32_t* p1 = reinterpret_cast<const uint32_t*>(&t1[k]);
+                    const uint32_t* p2 = reinterpret_cast<const uint32_t*>(&t2[k]);
+                    uint32_t* po = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float rr[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 2 * i + e;
+                            const float v0 = e ? bf16hi(p0[i]) : bf16lo(p0[i]);
+                            const float v1 = e ? bf16hi(p1[i]) : bf16lo(p1[i]);
+                            const float v2 = e ? bf16hi(p2[i]) : bf16lo(p2[i]);
+                            const float v3 = e ? bf16hi(px[i]) : bf16lo(px[i]);
+                            float acc = fmaf(cw[0][j], v0, cb[j]);
+                            acc = fmaf(cw[1][j], v1, acc);
+                            acc = fmaf(cw[2][j], v2, acc);
+                            rr[e] = fmaf(cw[3][j], v3, acc);
+                        }
+                        po[i] = pack_bf16x2(rr[0], rr[1]);
+                    }
+                }
+                // element (row rl, channels 8 g8 .. +7) of the 128-byte swizzled K block
+                const uint32_t so = (uint32_t)(rl >> 3) * 1024 + (uint32_t)(rl & 7) * 128 + ((uint32_t)(g8 ^ (rl & 7)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(kblk + so), "r"(o.x), "r"(o.y), "r"(o.z),
+                             "r"(o.w)
+                             : "memory");
+            }
+            // the block is complete: make it visible to the tensor core and the bulk copies, then
+            // hand it to this CTA's MMA and to the three siblings
+            fence_proxy_async_smem();
+            asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+            if (threadIdx.x == 0) {
+                mbar_arrive(bar_k(nt));
+                for (int rk = 1; rk < kClusterSize; ++rk) {
+                    const uint32_t peer = (uint32_t)((nt + rk) % kClusterSize);
+                    dsmem_copy(map_to_rank(kblk, peer), kblk, A_KBLK, map_to_rank(bar_k(nt), peer));
+                }
+            }
+            // history: oldest out, x in (after the hand-off, so that no fence waits for these)
+#pragma unroll
+            for (int k = 0; k < kConvUnits; ++k) {
+                const int bk = mt * MT + k * (kEpiThreads / 8) + (threadIdx.x >> 3);
+                if (bk < a.B) {
+                    __nv_bfloat16* tl = a.tail + (size_t)bk * kHist * W + ch0 + g8 * 8;
+                    *reinterpret_cast<uint4*>(tl) = t1[k];
+                    *reinterpret_cast<uint4*>(tl + W) = t2[k];
+                    *reinterpret_cast<uint4*>(tl + 2 * W) = xv[k];
+                }
+            }
+        }
+
+        // ================================ update ===============================================
+        // thread = row r of the tile, channels [16 cg, 16 cg + 16) of its 64; h, y and the conv
+        // output are read from (and h, out written back to) the swizzled shared tiles
+        const int q = warp & 3, cg = warp >> 2;           // lane quarter, channel quarter of the tile
         const int r = q * 32 + lane;                      // row within the tile
         const int b = mt * MT + r;
-        const bool valid = b < a.B;
+        const bool rst = b < a.B && a.reset && a.reset[b];
         const float gk1 = a.gelu_tanh ? 2.0f * 0.79788456080286535588f : 2.0f * 0.79879267f;
         const float gk3 = a.gelu_tanh ? 8.0f * 0.044715f * 0.79788456080286535588f : 8.0f * 0.03528805f;
-        // this row's state and y while the tensor cores run (rows past the batch read nothing)
-        const bool rst = valid && a.reset && a.reset[b];
-        const size_t off = (size_t)(valid ? b : 0) * W + ch0 + cg * 32;
-        float* hp = a.h + off;
-        const __nv_bfloat16* yp = a.y + off;
-        __nv_bfloat16* op = a.out + off;
-        float4 hq[8];
-        uint4 yq[4];
+        const uint32_t sw = (uint32_t)(r & 7);
+        // GeLU(y) while the siblings' blocks arrive and the tensor cores run
+        const bool ok_hy = __all_sync(0xffffffffu, wait_bounded(bar_hy, 0, a, abort, 4));
+        float gg[kEpiCh];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            hq[i] = (valid && !rst) ? *reinterpret_cast<const float4*>(hp + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int v = 0; v < kEpiCh / 8; ++v) {
+            const uint4 yq = *reinterpret_cast<const uint4*>(smem + OFF_Y + (uint32_t)r * 128 +
+                                                             ((((uint32_t)(cg * 2 + v)) ^ sw) << 4));
+            const uint32_t* yw = reinterpret_cast<const uint32_t*>(&yq);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) yq[i] = valid ? *reinterpret_cast<const uint4*>(yp + 8 * i) : make_uint4(0, 0, 0, 0);
+            for (int e = 0; e < 8; ++e) {
+                const float hy = 0.5f * ((e & 1) ? bf16hi(yw[e >> 1]) : bf16lo(yw[e >> 1]));
+                const float t = tanh_approx(hy * fmaf(hy * hy, gk3, gk1));
+                gg[v * 8 + e] = fmaf(hy, t, hy);          // y Phi(y) in the tanh form
+            }
+        }
         // uniform across the warp: the TMEM loads below are warp-collective
-        const bool ok = __all_sync(0xffffffffu, wait_bounded(bar_acc, 0, a, abort, 2));
+        const bool ok = __all_sync(0xffffffffu, ok_hy && wait_bounded(bar_acc, 0, a, abort, 2));
         tc_fence_after();
-        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + cg * 32;
-        const int cbase = nt * NT + cg * 32;              // channel within the head
+        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + cg * kEpiCh;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {                     // 8 channels per step
+        for (int v = 0; v < kEpiCh / 8; ++v) {            // 8 channels per step
             float ga[8], gx[8];
             tmem_ld8(taddr + v * 8, ga);
             tmem_ld8(taddr + NT + v * 8, gx);
             tmem_wait_ld();
-            if (!(ok && valid)) continue;
-            // conv output of this row: a 16-byte chunk of the swizzled A tile
-            const int cl = cbase + v * 8;
-            const uint32_t aoff = (uint32_t)(cl >> 6) * A_KBLK + (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128 +
-                                  ((uint32_t)(((cl & 63) >> 3) ^ (r & 7)) << 4);
-            const uint4 xq = *reinterpret_cast<const uint4*>(smem + OFF_A + aoff);
+            if (!ok) continue;
+            const int c8 = cg * 2 + v;                    // 8-channel chunk of the tile
+            // conv output: chunk c8 of row r in this CTA's K block
+            const uint32_t xo = OFF_A + nt * A_KBLK + (uint32_t)(r >> 3) * 1024 + sw * 128 + (((uint32_t)c8 ^ sw) << 4);
+            // h: 4-channel chunks 2 c8 and 2 c8 + 1, in the 32-channel box c8 / 4
+            const uint32_t hrow = OFF_H + (uint32_t)(c8 >> 2) * H_BOX + (uint32_t)r * 128;
+            const uint32_t ho0 = hrow + ((((uint32_t)(2 * c8) & 7) ^ sw) << 4);
+            const uint32_t ho1 = hrow + ((((uint32_t)(2 * c8 + 1) & 7) ^ sw) << 4);
+            // out, in the place of y
+            const uint32_t yo = OFF_Y + (uint32_t)r * 128 + (((uint32_t)c8 ^ sw) << 4);
+            const uint4 xq = *reinterpret_cast<const uint4*>(smem + xo);
+            float4 h0 = *reinterpret_cast<const float4*>(smem + ho0);
+            float4 h1 = *reinterpret_cast<const float4*>(smem + ho1);
+            if (rst) {                                    // the state restarts from zero
+                h0 = make_float4(0.f, 0.f, 0.f, 0.f);
+                h1 = h0;
+            }
             float hv[8];
-            const float4 h0 = hq[2 * v], h1 = hq[2 * v + 1];
             hv[0] = h0.x; hv[1] = h0.y; hv[2] = h0.z; hv[3] = h0.w;
             hv[4] = h1.x; hv[5] = h1.y; hv[6] = h1.z; hv[7] = h1.w;
             const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xq);
-            const uint32_t* yw = reinterpret_cast<const uint32_t*>(&yq[v]);
             uint32_t ow[4];
 #pragma unroll
             for (int e2 = 0; e2 < 4; ++e2) {
@@ -323,9 +442,8 @@ decode_gates_kernel(const __grid_constant__ CUtensorMap map_xc, const __grid_con
 #pragma unroll
                 for (int e1 = 0; e1 < 2; ++e1) {
                     const int e = 2 * e2 + e1;
-                    const int jc = cg * 32 + v * 8 + e;   // column within the tile
+                    const int jc = c8 * 8 + e;            // column within the tile
                     const float xcv = e1 ? bf16hi(xw[e2]) : bf16lo(xw[e2]);
-                    const float yv = e1 ? bf16hi(yw[e2]) : bf16lo(yw[e2]);
                     const float hk = s_hk[jc];
                     const float da = fmaf(ga[e], 0.5f, s_ba[jc]);
                     const float dx = fmaf(gx[e], 0.5f, s_bx[jc]);
@@ -345,16 +463,23 @@ decode_gates_kernel(const __grid_constant__ CUtensorMap map_xc, const __grid_con
                     const float u = fmaf(w, tanh_approx(dx), w);
                     const float hn = fmaf(at, hv[e], u);
                     hv[e] = hn;
-                    const float hy = 0.5f * yv;
-                    const float t = tanh_approx(hy * fmaf(hy * hy, gk3, gk1));
-                    const float m = hn * hy;
-                    o[e1] = fmaf(m, t, m);
+                    o[e1] = hn * gg[v * 8 + e];
                 }
                 ow[e2] = pack_bf16x2(o[0], o[1]);
             }
-            *reinterpret_cast<float4*>(hp + v * 8) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-            *reinterpret_cast<float4*>(hp + v * 8 + 4) = make_float4(hv[4], hv[5], hv[6], hv[7]);
-            *reinterpret_cast<uint4*>(op + v * 8) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+            *reinterpret_cast<float4*>(smem + ho0) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<float4*>(smem + ho1) = make_float4(hv[4], hv[5], hv[6], hv[7]);
+            *reinterpret_cast<uint4*>(smem + yo) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        }
+        // the tiles are complete: store h and out (rows past the batch are clipped by the maps)
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+        if (threadIdx.x == 0 && !*abort) {
+            tma_store_2d(&map_h, sbase + OFF_H, ch0, mt * MT);
+            tma_store_2d(&map_h, sbase + OFF_H + H_BOX, ch0 + 32, mt * MT);
+            tma_store_2d(&map_out, sbase + OFF_Y, ch0, mt * MT);
+            bulk_commit();
+            bulk_wait_read0();                            // the shared tiles stay until read
         }
     }
     tc_fence_before();
@@ -363,6 +488,8 @@ decode_gates_kernel(const __grid_constant__ CUtensorMap map_xc, const __grid_con
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
+    // no CTA leaves while a sibling's copy may still read its shared memory or write into it
+    cluster_sync();
 }
 
 }  // namespace dec
@@ -372,13 +499,13 @@ bool fused_decode_supported(const rglru_dims* d) {
 }
 
 size_t fused_decode_workspace(const rglru_dims* d) {
-    const size_t W = (size_t)d->heads * d->head_dim;
-    return 256 + (((size_t)d->batch * W * 2 + 255) & ~size_t(255));
+    (void)d;
+    return 256;   // the status word
 }
 
 int fused_decode_launches(const rglru_dims* d) {
     (void)d;
-    return 2;
+    return 1;
 }
 
 cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, const void* x, const void* y,
@@ -386,47 +513,42 @@ cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, cons
                                 cudaStream_t s) {
     using namespace dec;
     if (fused_decode_workspace(d) > ws_bytes) return cudaErrorInvalidValue;
-    const int B = d->batch, H = d->heads, W = H * DH;
-    __nv_bfloat16* xc = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + 256);
-    {
-        const long long n = (long long)B * (W / 8);
-        const int threads = 256;
-        const long long blocks = (n + threads - 1) / threads;
-        conv_shift_kernel<<<(unsigned)blocks, threads, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                                               static_cast<__nv_bfloat16*>(st->conv_tail), p->conv_w,
-                                                               p->conv_b, reset, xc, B, W);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    CUtensorMap mxc, mwa, mwx;
-    if (!tc::make_map_2d_sw128(&mxc, xc, W, B, (uint64_t)W * 2, 64, MT) ||
-        !tc::make_map_2d_sw128(&mwa, p->w_a, DH, (uint64_t)H * DH, DH * 2, NT, 64) ||
-        !tc::make_map_2d_sw128(&mwx, p->w_x, DH, (uint64_t)H * DH, DH * 2, NT, 64))
+    const int B = d->batch, H = d->heads;
+    const uint64_t W = (uint64_t)H * DH;
+    CUtensorMap mwa, mwx, mh, my, mo;
+    if (!tc::make_map_2d_sw128(&mwa, p->w_a, DH, W, DH * 2, NT, 64) ||
+        !tc::make_map_2d_sw128(&mwx, p->w_x, DH, W, DH * 2, NT, 64) ||
+        !tc::make_map_2d_sw128_elem(&mh, st->h, 4, W, (uint64_t)B, W * 4, 32, MT) ||
+        !tc::make_map_2d_sw128_elem(&my, y, 2, W, (uint64_t)B, W * 2, NT, MT) ||
+        !tc::make_map_2d_sw128_elem(&mo, out, 2, W, (uint64_t)B, W * 2, NT, MT))
         return cudaErrorInvalidValue;
-    cudaError_t e = set_smem_once(decode_gates_kernel, (int)SMEM_BYTES);
+    cudaError_t e = set_smem_once(decode_fused_kernel, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     Args a;
     a.B = B; a.H = H; a.mtiles = (B + MT - 1) / MT;
+    a.x = static_cast<const __nv_bfloat16*>(x);
+    a.tail = static_cast<__nv_bfloat16*>(st->conv_tail);
+    a.conv_w = p->conv_w; a.conv_b = p->conv_b;
     a.c = d->c; a.gelu_tanh = d->gelu_tanh;
     a.timeout_ns = 1000000000ull;
     a.b_a = p->b_a; a.b_x = p->b_x; a.lambda = p->lambda; a.reset = reset;
-    a.y = static_cast<const __nv_bfloat16*>(y);
-    a.h = st->h;
-    a.out = static_cast<__nv_bfloat16*>(out);
     a.status = reinterpret_cast<DeviceStatus*>(ws);
-    // programmatic dependent launch: this kernel's set-up (barriers, TMEM, constants, weight
-    // tiles, state prefetch) overlaps the conv kernel; it waits for it before loading the conv
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(H * a.mtiles * (DH / NT)));
+    cfg.gridDim = dim3((unsigned)(H * a.mtiles * kClusterSize));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClusterSize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    // the set-up of this step may overlap the tail of the stream's previous kernel
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_gates_kernel, mxc, mwa, mwx, a);
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, mwa, mwx, mh, my, mo, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

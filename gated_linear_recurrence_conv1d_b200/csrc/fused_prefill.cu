@@ -960,17 +960,24 @@ bool make_map_3d(CUtensorMap* m, const void* base, int W, int T, int B, int box_
 
 // 2-D map [outer][inner] of bf16 with a row pitch of row_bytes, box inner x outer, 128-byte
 // swizzle (box_inner * 2 must be 128), out-of-range elements read as zero.
-bool make_map_2d_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                       uint32_t box_inner, uint32_t box_outer) {
+// 2-D map (inner x outer elements of bf16 or fp32, rows row_bytes apart) whose box rows are
+// exactly 128 bytes, loaded and stored in the 128-byte swizzle
+bool make_map_2d_sw128_elem(CUtensorMap* m, const void* base, uint32_t elem_bytes, uint64_t inner, uint64_t outer,
+                            uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
     EncodeTiledFn f = encode_fn();
-    if (!f || box_inner * 2 != 128) return false;
+    if (!f || (elem_bytes != 2 && elem_bytes != 4) || box_inner * elem_bytes != 128) return false;
     cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
     cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    const CUtensorMapDataType t = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    return f(m, t, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool make_map_2d_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                       uint32_t box_inner, uint32_t box_outer) {
+    return make_map_2d_sw128_elem(m, base, 2, inner, outer, row_bytes, box_inner, box_outer);
 }
 
 struct Plan {

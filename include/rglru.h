@@ -197,6 +197,11 @@ RGLRU_API rglru_status rglru_read_device_status(void* workspace, size_t workspac
 /* Static, human-readable name of a status code. */
 RGLRU_API const char* rglru_status_string(rglru_status status);
 
+/* The CUDA runtime error (cudaError_t value) behind the calling host thread's most recent
+ * RGLRU_ERR_CUDA, 0 if it has had none; *name (when name is not NULL) receives the runtime's
+ * static name of that error.  Diagnostic only: it does not clear the value. */
+RGLRU_API int rglru_last_cuda_error(const char** name);
+
 /* RGLRU_ABI_VERSION of the built library. */
 RGLRU_API int rglru_abi_version(void);
 

@@ -37,6 +37,21 @@ def test_status_strings():
     assert lib.rglru_status_string(99).decode() == "RGLRU_ERR_UNKNOWN"
 
 
+def test_last_cuda_error_starts_clear():
+    """A host thread that has had no failed CUDA call reads back cudaSuccess."""
+    import threading
+    got = []
+    t = threading.Thread(target=lambda: got.append(binding.last_cuda_error()))
+    t.start()
+    t.join()
+    assert got == [(0, "cudaSuccess")]
+
+
+def test_cuda_status_error_carries_the_runtime_error_name():
+    with pytest.raises(binding.RglruError, match=r"RGLRU_ERR_CUDA \(cudaSuccess, 0\)"):
+        binding._check(binding.RGLRU_ERR_CUDA, "probe")
+
+
 def _dims(**kw):
     d = dict(batch=2, seq_len=16, heads=2, head_dim=64, act_dtype=binding.RGLRU_BF16)
     d.update(kw)
