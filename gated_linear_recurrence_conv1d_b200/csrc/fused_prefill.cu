@@ -25,9 +25,11 @@
 //   * chunks of one sequence handled by different CTAs chain through a look-back in the spirit
 //     of Merrill & Garland ("Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016):
 //     after its first pass a chunk publishes its aggregate (prod a, local h) per channel; its
-//     carry is the inclusive state of an anchor chunk (every 32nd chunk of the row) followed by
+//     carry is the inclusive state of an anchor chunk (every 8th chunk of the row) followed by
 //     the aggregates of the chunks in between, applied in a fixed order so the result does not
-//     depend on timing.  Every wait is bounded by %globaltimer; on expiry the kernel latches
+//     depend on timing.  Each published value is one 64-bit word that shows whether it has been
+//     written, so a reader polls the data itself: one round of independent loads per attempt,
+//     no separate flag.  Every wait is bounded by %globaltimer; on expiry the kernel latches
 //     RGLRU_ERR_TIMEOUT in the workspace status word and drains.
 //
 // Element-wise arithmetic (one transcendental per gate, one square root, one for GeLU):
@@ -109,7 +111,11 @@ static_assert(TM_D + STAGES * TM_SLOT <= TMEM_COLS, "TMEM budget");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 constexpr unsigned FLAG_AGG = 1, FLAG_INCL = 2;
-constexpr int LBW = 32;                 // look-back block: anchors every LBW chunks
+constexpr int LBW = 8;                  // look-back block: anchors every LBW chunks
+// A published look-back word is 64 bits, written by one relaxed store, and says itself whether it
+// has been written (the workspace starts zeroed): an aggregate is (prod a with its sign bit set,
+// local h) -- prod a is never negative -- and an anchor's inclusive state is (h, -1).
+constexpr uint32_t kReadyBit = 0x80000000u;
 
 struct Args {
     int B, T, H, NC, items;          // items = B * NC per group
@@ -132,8 +138,9 @@ struct Args {
     DeviceStatus* status;
     unsigned* counters;              // [groups] tickets
     unsigned* lb_flags;              // [groups][items][4]
-    float2* lb_agg;                  // [groups][items][128]
-    float* lb_incl;                  // [groups][items][128]
+    int NA;                          // anchors per row: ceil(NC / LBW)
+    uint64_t* lb_agg;                // [groups][items][128] aggregate words
+    uint64_t* lb_incl;               // [groups][B * NA][128] anchor inclusive-state words
 };
 
 struct Bars {
@@ -372,6 +379,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     const int head = group >> 1, half = group & 1;
     const int W = a.H * DH;
     const size_t lb_base = (size_t)group * a.items;
+    const size_t lb_base_a = (size_t)group * a.B * a.NA;     // anchors of the group
     const bool bias_in_acc = a.b_a != nullptr || a.b_x != nullptr;
 
     // ---- set-up ------------------------------------------------------------------------------
@@ -783,12 +791,9 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             // the B tile (xc) is no longer read by this warp
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.b_empty[st]);
-            if (c > 0 && !withhold) {                    // chunk aggregate, as early as possible
-                // every lane's store is ordered before lane 0's release by the warp barrier
-                a.lb_agg[(lb_base + k) * HALF + m] = make_float2(aggA, aggH);
-                __syncwarp();
-                if (lane == 0) st_release_gpu(myflag, FLAG_AGG);
-            }
+            if (c > 0 && !withhold)                      // chunk aggregate, as early as possible
+                st_relaxed_gpu_u64(a.lb_agg + (lb_base + k) * HALF + m,
+                                   ((uint64_t)__float_as_uint(aggH) << 32) | (__float_as_uint(aggA) | kReadyBit));
 
             // ---- carry: initial state for the first chunk, else the look-back
             float carry = 0.f;
@@ -799,16 +804,30 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 // nearest earlier chunk whose index is a multiple of LBW; carry = the anchor's
                 // inclusive state, then the aggregates of the chunks in between, in order
                 const int anc = ((c - 1) / LBW) * LBW;
-                const int nagg = c - 1 - anc;                       // < LBW <= 32
-                const unsigned* fa = a.lb_flags + (kb_item + anc) * 4 + q;
-                const bool mine = lane < nagg;
-                const unsigned* fl = fa + (size_t)(lane + 1) * 4;
+                const int nagg = c - 1 - anc;                       // < LBW
+                const uint64_t* wi = a.lb_incl + (lb_base_a + (size_t)b * a.NA + anc / LBW) * HALF + m;
+                const uint64_t* wa = a.lb_agg + (kb_item + anc + 1) * HALF + m;
                 const uint64_t tw = globaltimer_ns();
-                bool ready = false;
                 for (uint32_t it = 0;; ++it) {
-                    bool okl = mine ? ld_acquire_gpu(fl) >= FLAG_AGG : true;
-                    if (lane == 0) okl = okl && ld_acquire_gpu(fa) >= FLAG_INCL;
-                    if (__all_sync(0xffffffffu, okl)) { ready = true; break; }
+                    // every word of this channel's look-back in one batch of independent loads;
+                    // the combine stays in chunk order, padding entries are the identity (1, 0)
+                    uint64_t g[LBW];
+                    g[0] = ld_relaxed_gpu_u64(wi);
+#pragma unroll
+                    for (int i = 1; i < LBW; ++i)
+                        g[i] = i <= nagg ? ld_relaxed_gpu_u64(wa + (size_t)(i - 1) * HALF)
+                                         : (uint64_t)(__float_as_uint(1.0f) | kReadyBit);
+                    bool okl = (uint32_t)(g[0] >> 32) & kReadyBit;
+#pragma unroll
+                    for (int i = 1; i < LBW; ++i) okl = okl && ((uint32_t)g[i] & kReadyBit);
+                    if (__all_sync(0xffffffffu, okl)) {
+                        float hc = __uint_as_float((uint32_t)g[0]);
+#pragma unroll
+                        for (int i = 1; i < LBW; ++i)
+                            hc = fmaf(__uint_as_float((uint32_t)g[i] & ~kReadyBit), hc, __uint_as_float((uint32_t)(g[i] >> 32)));
+                        carry = hc;
+                        break;
+                    }
                     __nanosleep(64);
                     if ((it & 15) == 15) {
                         int give_up = 0;
@@ -823,29 +842,17 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                         if (__shfl_sync(0xffffffffu, give_up, 0)) break;
                     }
                 }
-                if (ready) {
-                    // the loads of a batch are independent (one L2 round trip per batch); the
-                    // combine stays in chunk order; padding entries are the identity (1, 0)
-                    float hc = __ldcg(a.lb_incl + (kb_item + anc) * HALF + m);
-                    const float2* ag = a.lb_agg + (kb_item + anc + 1) * HALF + m;
-                    constexpr int kBatch = 8;
-#pragma unroll 1
-                    for (int i0 = 0; i0 < nagg; i0 += kBatch) {
-                        float2 g[kBatch];
-#pragma unroll
-                        for (int i = 0; i < kBatch; ++i)
-                            g[i] = i0 + i < nagg ? __ldcg(ag + (size_t)(i0 + i) * HALF) : make_float2(1.f, 0.f);
-#pragma unroll
-                        for (int i = 0; i < kBatch; ++i) hc = fmaf(g[i].x, hc, g[i].y);
-                    }
-                    carry = hc;
-                }
             }
             const float incl = fmaf(aggA, carry, aggH);             // state after the chunk
             if (c % LBW == 0 && !withhold) {             // only anchors' inclusive states are read
-                a.lb_incl[(lb_base + k) * HALF + m] = incl;
-                __syncwarp();
-                if (lane == 0) st_release_gpu(myflag, FLAG_INCL);
+                st_relaxed_gpu_u64(a.lb_incl + (lb_base_a + (size_t)b * a.NA + c / LBW) * HALF + m,
+                                   ((uint64_t)0xBF800000u << 32) | __float_as_uint(incl));
+                if (c == 0) {
+                    // the row's first chunk has read the old state and history: the flag that the
+                    // writers of the final state and history wait for
+                    __syncwarp();
+                    if (lane == 0) st_release_gpu(myflag, FLAG_INCL);
+                }
             }
             // final state of the row, once its first chunk has read the old one
             if (a.h_state && c == a.NC - 1) {
@@ -982,6 +989,7 @@ bool make_map_2d_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_
 
 struct Plan {
     int NC, items, groups, ctas, base, extra;
+    int NA;
     size_t off_counters, off_flags, off_agg, off_incl, total;
 };
 
@@ -997,8 +1005,9 @@ Plan make_plan(const rglru_dims* d, int sms) {
     p.off_counters = 256;
     p.off_flags = up(p.off_counters + (size_t)p.groups * 4);
     p.off_agg = up(p.off_flags + (size_t)p.groups * p.items * 16);
+    p.NA = (p.NC + LBW - 1) / LBW;
     p.off_incl = up(p.off_agg + (size_t)p.groups * p.items * HALF * 8);
-    p.total = up(p.off_incl + (size_t)p.groups * p.items * HALF * 4);
+    p.total = up(p.off_incl + (size_t)p.groups * d->batch * p.NA * HALF * 8);
     return p;
 }
 
@@ -1052,9 +1061,11 @@ cudaError_t launch_fused_prefill(const rglru_dims* d, const rglru_params* p, con
     a.status = reinterpret_cast<DeviceStatus*>(w);
     a.counters = reinterpret_cast<unsigned*>(w + pl.off_counters);
     a.lb_flags = reinterpret_cast<unsigned*>(w + pl.off_flags);
-    a.lb_agg = reinterpret_cast<float2*>(w + pl.off_agg);
-    a.lb_incl = reinterpret_cast<float*>(w + pl.off_incl);
-    const size_t clear = pl.off_agg - pl.off_counters;      // tickets and look-back flags
+    a.NA = pl.NA;
+    a.lb_agg = reinterpret_cast<uint64_t*>(w + pl.off_agg);
+    a.lb_incl = reinterpret_cast<uint64_t*>(w + pl.off_incl);
+    // tickets, flags and look-back words all start at zero ("not written")
+    const size_t clear = pl.total - pl.off_counters;
     e = cudaMemsetAsync(w + pl.off_counters, 0, clear, s);
     if (e != cudaSuccess) return e;
     fused_prefill_kernel<<<pl.ctas, kThreads, SMEM_BYTES, s>>>(mx, my, mo, a);
