@@ -15,9 +15,9 @@
 //     stage's previous item), 8 conv warps (a channel half and a quarter of the chunk's tokens
 //     each; a lane convolves 4 channels with 8-byte shared-memory loads and writes them as the
 //     bf16 B operand in the 128-byte swizzled K-major layout), 2 MMA issuer threads (even / odd
-//     items; D = W^T/2 . xc^T for both gates, K = 256 in 16 steps, accumulated onto the gate
-//     biases that the epilogue pre-loads into TMEM), and 4 epilogue groups of 4 warps, group g
-//     owning TMEM stage g;
+//     items; D = W^T/2 . xc^T for both gates, K = 256 in 16 steps; the epilogue adds the halved
+//     gate biases, so a stage needs no re-arming between items), and 4 epilogue groups of 4
+//     warps, group g owning TMEM stage g;
 //   * transposed orientation: a TMEM lane is an output channel and the 32 columns are tokens,
 //     so an epilogue thread owns one channel and runs the diagonal scan along its registers
 //     (no shuffles); its first pass leaves the running (prod a, local h) of every token in
@@ -25,7 +25,7 @@
 //   * chunks of one sequence handled by different CTAs chain through a look-back in the spirit
 //     of Merrill & Garland ("Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016):
 //     after its first pass a chunk publishes its aggregate (prod a, local h) per channel; its
-//     carry is the inclusive state of an anchor chunk (every 8th chunk of the row) followed by
+//     carry is the inclusive state of an anchor chunk (every 4th chunk of the row) followed by
 //     the aggregates of the chunks in between, applied in a fixed order so the result does not
 //     depend on timing.  Each published value is one 64-bit word that shows whether it has been
 //     written, so a reader polls the data itself: one round of independent loads per attempt,
@@ -33,7 +33,7 @@
 //     RGLRU_ERR_TIMEOUT in the workspace status word and drains.
 //
 // Element-wise arithmetic (one transcendental per gate, one square root, one for GeLU):
-//   D_a = (g_a + b_a) / 2, D_x = (g_x + b_x) / 2 come out of the MMA;
+//   D_a = (g_a + b_a) / 2, D_x = (g_x + b_x) / 2 (the MMA gives g / 2, the epilogue adds b / 2);
 //   r_t = (1 + tanh D_a) / 2 and l_t = c r_t log sigma(Lambda) = hK (1 + tanh D_a) with
 //   hK = c log sigma(Lambda) / 2;  E = expm1(l_t) = l(1 + l/2 + l^2/6) (|l| <= 1/8: the
 //   truncation, summed over the ~1/|l| tokens a decay acts on, stays below 1e-4), a_t = 1 + E,
@@ -111,7 +111,7 @@ static_assert(TM_D + STAGES * TM_SLOT <= TMEM_COLS, "TMEM budget");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 constexpr unsigned FLAG_AGG = 1, FLAG_INCL = 2;
-constexpr int LBW = 8;                  // look-back block: anchors every LBW chunks
+constexpr int LBW = 4;                  // look-back block: anchors every LBW chunks
 // A published look-back word is 64 bits, written by one relaxed store, and says itself whether it
 // has been written (the workspace starts zeroed): an aggregate is (prod a with its sign bit set,
 // local h) -- prod a is never negative -- and an anchor's inclusive state is (h, -1).
@@ -380,7 +380,6 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
     const int W = a.H * DH;
     const size_t lb_base = (size_t)group * a.items;
     const size_t lb_base_a = (size_t)group * a.B * a.NA;     // anchors of the group
-    const bool bias_in_acc = a.b_a != nullptr || a.b_x != nullptr;
 
     // ---- set-up ------------------------------------------------------------------------------
     if (threadIdx.x == 0) {
@@ -436,8 +435,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
 
     if (warp >= kWarpEpi0 && warp < kWarpEpi0 + kEpiWarps) {
         // weights -> TMEM A operand: lane m, column j holds (W[2j][m], W[2j+1][m]); group 0 of
-        // each lane quarter writes gate a, group 1 gate x.  Then each group pre-loads the gate
-        // biases of its accumulator stage.
+        // each lane quarter writes gate a, group 1 gate x.
         const int q = warp & 3, g = (warp - kWarpEpi0) >> 2, m = q * 32 + lane;
         const unsigned short* ws = reinterpret_cast<const unsigned short*>(smem + (g & 1) * (HALF * DH * 2)) + m;
 #pragma unroll 1
@@ -449,20 +447,6 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 r[j] = (uint32_t)ws[i * HALF] | ((uint32_t)ws[(i + 1) * HALF] << 16);
             }
             tmem_st16(tmem + ((uint32_t)(q * 32) << 16) + TM_A + g * 128 + j0, r);
-        }
-        if (bias_in_acc) {
-            const int ch = head * DH + half * HALF + m;
-            const uint32_t ba = __float_as_uint(a.b_a ? 0.5f * a.b_a[ch] : 0.f);
-            const uint32_t bx = __float_as_uint(a.b_x ? 0.5f * a.b_x[ch] : 0.f);
-            uint32_t ra[16], rx[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) { ra[j] = ba; rx[j] = bx; }
-            const uint32_t d = tmem + ((uint32_t)(q * 32) << 16) + TM_D + g * TM_SLOT;
-#pragma unroll
-            for (int j0 = 0; j0 < L; j0 += 16) {
-                tmem_st16(d + j0, ra);
-                tmem_st16(d + L + j0, rx);
-            }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -567,7 +551,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
                     const uint64_t bd = bd0 + (uint64_t)((((ks >> 2) * KBLK_BYTES) + (ks & 3) * 32) >> 4);
-                    const uint32_t acc = (bias_in_acc || ks > 0) ? 1u : 0u;
+                    const uint32_t acc = ks > 0 ? 1u : 0u;
                     mma_ts(d0, tmem + TM_A + ks * 8, bd, idesc, acc);
                     mma_ts(d0 + L, tmem + TM_A + 128 + ks * 8, bd, idesc, acc);
                 }
@@ -700,8 +684,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
         // GeLU(y) = (y/2)(1 + tanh((y/2)(K1 + K3 (y/2)^2)))
         const float gk1 = tanh_form ? 2.0f * 0.79788456080286535588f : 2.0f * 0.79879267f;
         const float gk3 = tanh_form ? 8.0f * 0.044715f * 0.79788456080286535588f : 8.0f * 0.03528805f;
-        const uint32_t ba_bits = __float_as_uint(a.b_a ? 0.5f * a.b_a[ch] : 0.f);
-        const uint32_t bx_bits = __float_as_uint(a.b_x ? 0.5f * a.b_x[ch] : 0.f);
+        const float2 ba2 = f2(a.b_a ? 0.5f * a.b_a[ch] : 0.f);     // gate biases, halved
+        const float2 bx2 = f2(a.b_x ? 0.5f * a.b_x[ch] : 0.f);
         const bool withhold_hook = (a.flags & RGLRU_FLAG_TEST_WITHHOLD) && group == 0;
         const uint8_t* bt = smem + OFF_B + st * B_BYTES;
         uint8_t* yt = smem + OFF_Y + st * Y_BYTES + 2 * m;
@@ -743,7 +727,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
 #pragma unroll
                     for (int j = 0; j < kBlk; j += 2) {
                         float2 at, u;
-                        gates_pair(make_float2(da[j], da[j + 1]), make_float2(dx[j], dx[j + 1]), hk2,
+                        gates_pair(add2(make_float2(da[j], da[j + 1]), ba2), add2(make_float2(dx[j], dx[j + 1]), bx2), hk2,
                                    make_float2(xc_at(j0 + j), xc_at(j0 + j + 1)), at, u);
                         if constexpr (decltype(rst)::value) {             // h_{t-1} := 0 at a reset
                             if ((rmask >> (j0 + j)) & 1ull) at.x = 0.f;
@@ -776,7 +760,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     for (int j = 0; j < kBlk; ++j) {
                         const int t = j0 + j;
                         float at, u;
-                        gates_one(da[j], dx[j], hk, xc_at(t), at, u);
+                        gates_one(da[j] + ba2.x, dx[j] + bx2.x, hk, xc_at(t), at, u);
                         if ((rmask >> t) & 1ull) at = 0.f;                 // h_{t-1} := 0
                         if (t >= nt) { at = 1.f; u = 0.f; }                // padding: identity
                         aggH = fmaf(at, aggH, u);
@@ -890,18 +874,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                     }
                 }
             }
-            // re-arm the accumulator stage with the gate biases, then hand it back to the MMA
-            if (bias_in_acc) {
-                uint32_t ra[16], rx[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) { ra[j] = ba_bits; rx[j] = bx_bits; }
-#pragma unroll
-                for (int j0 = 0; j0 < L; j0 += 16) {
-                    tmem_st16(dcol + j0, ra);
-                    tmem_st16(dcol + L + j0, rx);
-                }
-                tmem_wait_st();
-            }
+            // hand the accumulator stage back to the MMA
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.acc_empty[st]);
