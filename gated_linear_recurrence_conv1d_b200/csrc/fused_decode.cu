@@ -89,6 +89,7 @@ struct Args {
     const float* conv_b;
     float c;
     int gelu_tanh;
+    int withhold;                     // test hook: CTA 0 keeps its conv block from its siblings
     unsigned long long timeout_ns;
     const float* b_a;
     const float* b_x;
@@ -361,7 +362,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
             asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
             if (threadIdx.x == 0) {
                 mbar_arrive(bar_k(nt));
-                for (int rk = 1; rk < kClusterSize; ++rk) {
+                for (int rk = 1; rk < kClusterSize && !(a.withhold && blockIdx.x == 0); ++rk) {
                     const uint32_t peer = (uint32_t)((nt + rk) % kClusterSize);
                     dsmem_copy(map_to_rank(kblk, peer), kblk, A_KBLK, map_to_rank(bar_k(nt), peer));
                 }
@@ -530,7 +531,8 @@ cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, cons
     a.tail = static_cast<__nv_bfloat16*>(st->conv_tail);
     a.conv_w = p->conv_w; a.conv_b = p->conv_b;
     a.c = d->c; a.gelu_tanh = d->gelu_tanh;
-    a.timeout_ns = 1000000000ull;
+    a.withhold = (d->flags & RGLRU_FLAG_TEST_WITHHOLD) != 0;
+    a.timeout_ns = a.withhold ? 2000000ull : 1000000000ull;
     a.b_a = p->b_a; a.b_x = p->b_x; a.lambda = p->lambda; a.reset = reset;
     a.status = reinterpret_cast<DeviceStatus*>(ws);
     cudaLaunchConfig_t cfg = {};

@@ -79,8 +79,9 @@ typedef enum {
 
 /* Problem description.  `flags` is 0 in normal use; bit RGLRU_FLAG_GENERIC forces the
  * portable (non-tensor-core) kernels, bit RGLRU_FLAG_TEST_WITHHOLD makes the fused prefill
- * kernel withhold the carry of its first time chunk so that its successors' bounded waits
- * expire (a test hook for the timeout path; results are then undefined). */
+ * kernel withhold the carry of its first time chunk, and the tensor-core decode step's first
+ * CTA withhold its conv block from the other CTAs of its cluster, so that their bounded waits
+ * expire after 2 ms (a test hook for the timeout path; outputs and state are then undefined). */
 typedef struct {
     int batch;        /* B */
     int seq_len;      /* T (prefill); ignored by decode */

@@ -179,3 +179,33 @@ def test_tensor_decode_matches_oracle_and_generic(B):
         assert_close(to_np(h), h_ref, "bf16", "decode h")
         outs[flags] = np.stack(res)
     assert rel_err(outs[0], outs[binding.FLAG_GENERIC]) <= 1e-2
+
+
+def test_tensor_decode_withheld_block_times_out_and_context_survives():
+    """Test hook: the decode step's first CTA keeps its conv block from the other CTAs of its
+    cluster, so their bounded waits expire; the call must report RGLRU_ERR_TIMEOUT and return,
+    and the same context must then run a correct decode step."""
+    B = 130
+    wl = BASE["decode_bf16"].scaled(batch=B, heads=2, decode_steps=1)
+    prob = inputs.make_problem(wl, seed=44)
+    bad = GpuProblem(prob, flags=binding.FLAG_TEST_WITHHOLD)
+    h, tail = bad.new_state(B)
+    dims = bad.block.dims(B, 1)
+    assert binding.decode_plan(dims) == (1, 1)
+    ws = binding.alloc_workspace(binding.decode_workspace_size(dims))
+    out = torch.empty_like(bad.x[0])
+    binding.block_decode(dims, bad.block.params, bad.x[0], bad.y[0], out, h, tail, ws)
+    assert binding.read_device_status(ws) == binding.RGLRU_ERR_TIMEOUT
+
+    gp = GpuProblem(prob)
+    h, tail = gp.new_state(B)
+    dims = gp.block.dims(B, 1)
+    binding.block_decode(dims, gp.block.params, gp.x[0], gp.y[0], out, h, tail, ws)
+    assert binding.read_device_status(ws) == binding.RGLRU_OK
+    h_ref = prob.h0.astype(np.float64).copy()
+    t_ref = oracle.tail_from_act(prob.tail0).copy()
+    ref = oracle.decode(prob.params, prob.x[0], prob.y[0], wl.heads, h_ref, t_ref)
+    assert_close(to_np(out), ref, "bf16", "decode after timeout")
+    assert_close(to_np(h), h_ref, "bf16", "decode h after timeout")
+    np.testing.assert_array_equal(to_np(tail), t_ref)
+
