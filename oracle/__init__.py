@@ -49,6 +49,8 @@ def load_library(path: str):
     lib.rglru_oracle_prefill.restype = I
     lib.rglru_oracle_prefill.argtypes = [I, I, I, I, D, I, I, P, P, P, P, P, P, P,
                                          P, P, P, P, P, P, P, I, I]
+    lib.rglru_oracle_backward.restype = I
+    lib.rglru_oracle_backward.argtypes = [I, I, I, I, D, I, I] + [P] * 26
     lib.rglru_oracle_decode.restype = I
     lib.rglru_oracle_decode.argtypes = [I, I, I, D, I, I, P, P, P, P, P, P, P,
                                         P, P, P, P, P, P, I]
@@ -226,3 +228,45 @@ def prefill_units(params: dict, x: np.ndarray, y: np.ndarray, heads: int, units:
     n = workers or min(len(units), max(1, os.cpu_count() or 1))
     with ThreadPoolExecutor(max_workers=n) as ex:
         return dict(ex.map(one, [tuple(u) for u in units]))
+
+
+def backward(params: dict, x: np.ndarray, y: np.ndarray, heads: int, dout: np.ndarray,
+             reset: Optional[np.ndarray] = None, h0: Optional[np.ndarray] = None,
+             tail0: Optional[np.ndarray] = None, dh_final: Optional[np.ndarray] = None,
+             dtail_final: Optional[np.ndarray] = None, c: float = 8.0, gelu_tanh: int = 0) -> dict:
+    """Exact fp64 gradients of L = <dout, out> + <dh_final, h_T> + <dtail_final, tail_T> for the
+    prefill of x, y [B, T, W] from the state (h0, tail0) (zero when None).
+
+    Returns a dict of fp64 arrays: dx, dy [B, T, W]; dh0 [B, W]; dtail0 [B, 3, W];
+    dconv_w [4, W]; dconv_b, db_a, db_x, dlam [W]; dw_a, dw_x [H, dh, dh].
+    """
+    lib = _load()
+    x, dt = _act(x)
+    y, _ = _act(y)
+    dout, dtd = _act(dout)
+    assert dtd == dt and dout.shape == x.shape
+    B, T, W = x.shape
+    dh = W // heads
+    w_a, _ = _act(params["w_a"])
+    w_x, _ = _act(params["w_x"])
+    conv_w, conv_b = _f32(params["conv_w"]), _f32(params.get("conv_b"))
+    b_a, b_x, lam = _f32(params.get("b_a")), _f32(params.get("b_x")), _f32(params["lam"])
+    f64 = lambda a: None if a is None else np.ascontiguousarray(a, dtype=np.float64)  # noqa: E731
+    h0 = f64(h0)
+    tail0 = None if tail0 is None else tail_from_act(tail0)
+    dh_final, dtail_final = f64(dh_final), f64(dtail_final)
+    rst = None if reset is None else np.ascontiguousarray(reset, dtype=np.uint8)
+    g = {"dx": np.zeros((B, T, W)), "dy": np.zeros((B, T, W)), "dh0": np.zeros((B, W)),
+         "dtail0": np.zeros((B, HIST, W)), "dconv_w": np.zeros((4, W)), "dconv_b": np.zeros(W),
+         "dw_a": np.zeros((heads, dh, dh)), "dw_x": np.zeros((heads, dh, dh)),
+         "db_a": np.zeros(W), "db_x": np.zeros(W), "dlam": np.zeros(W)}
+    rc = lib.rglru_oracle_backward(
+        B, T, heads, dh, c, gelu_tanh, dt, _p(conv_w), _p(conv_b), _p(w_a), _p(w_x), _p(b_a),
+        _p(b_x), _p(lam), _p(x), _p(y), _p(rst), _p(h0), _p(tail0), _p(dout), _p(dh_final),
+        _p(dtail_final), _p(g["dx"]), _p(g["dy"]), _p(g["dh0"]), _p(g["dtail0"]),
+        _p(g["dconv_w"]), _p(g["dconv_b"]), _p(g["dw_a"]), _p(g["dw_x"]), _p(g["db_a"]),
+        _p(g["db_x"]), _p(g["dlam"]))
+    if rc != 0:
+        raise RuntimeError("oracle backward failed")
+    return g
+

@@ -13,6 +13,7 @@ import tempfile
 import pytest
 
 import oracle
+from tests import test_backward_oracle as bwd_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "rglru_oracle.c")
@@ -42,6 +43,57 @@ PIN_TESTS = [
     pins.test_packed_rows_equal_separate_documents,
     pins.test_reset_cuts_all_dependence_on_the_past,
 ]
+
+
+# Mistakes in the backward pass, each of which the backward pins must catch.
+BACKWARD_MUTANTS = {
+    "bwd_reset_keeps_gradient": ("g[o] = (reset && reset[t]) ? 0.0 : a * g[o];", "g[o] = a * g[o];"),
+    "bwd_beta_term_sign": ("double q = dl_da * a * r - dl_dbeta * a * a * r_over_beta;",
+                           "double q = dl_da * a * r + dl_dbeta * a * a * r_over_beta;"),
+    "bwd_dropped_direct_input_path": ("dxc[e] = g[o] * beta * ig;", "dxc[e] = 0.0;"),
+    "bwd_gelu_density_dropped": ("return 0.5 * erfc(-v / sqrt(2.0)) + v * exp(-0.5 * v * v) / sqrt(2.0 * pi);",
+                                 "return 0.5 * erfc(-v / sqrt(2.0));"),
+    "bwd_weight_grad_transposed": ("dw_a[(long)i * dh + o] += xct[i] * dga[o];",
+                                   "dw_a[(long)o * dh + i] += xct[i] * dga[o];"),
+    "bwd_conv_scatter_wrong_tap": ("if (src >= 0) dx[(long)src * ld + j] += (double)conv_w[k * conv_ld + j] * d;",
+                                   "if (src >= 0) dx[(long)src * ld + j] += (double)conv_w[(3 - k) * conv_ld + j] * d;"),
+}
+
+BACKWARD_PIN_TESTS = [
+    bwd_pins.test_backward_matches_finite_differences,
+    bwd_pins.test_backward_frozen_state_closed_form,
+    bwd_pins.test_backward_reset_at_the_first_token_cuts_the_initial_state,
+    lambda: bwd_pins.test_gelu_derivative_matches_a_difference_quotient(0.7, 0),
+]
+
+
+def _build_mutant(old, new, tmp):
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation anchor not found exactly once"
+    path = os.path.join(tmp, "mutant.c")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    lib_path = os.path.join(tmp, "libmutant.so")
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-ffp-contract=off", "-fopenmp", "-fPIC",
+                           "-shared", "-o", lib_path, path, "-lm"])
+    return lib_path
+
+
+@pytest.mark.parametrize("name", sorted(BACKWARD_MUTANTS))
+def test_backward_pins_catch_planted_mistake(name, monkeypatch):
+    old, new = BACKWARD_MUTANTS[name]
+    tmp = tempfile.mkdtemp(prefix="oracle_mutant_")
+    try:
+        monkeypatch.setattr(oracle, "_lib", oracle.load_library(_build_mutant(old, new, tmp)))
+        caught = 0
+        for pin in BACKWARD_PIN_TESTS:
+            try:
+                pin()
+            except AssertionError:
+                caught += 1
+        assert caught >= 1, f"no backward pin caught the planted mistake {name}"
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
