@@ -31,7 +31,12 @@ STATUS_NAMES = {0: "RGLRU_OK", 1: "RGLRU_ERR_INVALID_ARG", 2: "RGLRU_ERR_UNSUPPO
 EXPORTED = ("rglru_state_init", "rglru_prefill_workspace_size", "rglru_block_prefill",
             "rglru_decode_workspace_size", "rglru_block_decode", "rglru_read_device_status",
             "rglru_status_string", "rglru_abi_version", "rglru_prefill_plan", "rglru_decode_plan",
-            "rglru_block_prefill_noalloc", "rglru_last_cuda_error")
+            "rglru_block_prefill_noalloc", "rglru_last_cuda_error", "rglru_backward_workspace_size",
+            "rglru_block_backward")
+
+# Fields of rglru_grads, in order (fp32 device tensors).
+GRAD_FIELDS = ("dx", "dy", "dh0", "dtail0", "dconv_w", "dconv_b", "dw_a", "dw_x", "db_a", "db_x",
+               "dlambda")
 
 # Bytes of the static device scratch behind rglru_block_prefill_noalloc.
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -57,6 +62,10 @@ class Params(ctypes.Structure):
 
 class State(ctypes.Structure):
     _fields_ = [("h", ctypes.c_void_p), ("conv_tail", ctypes.c_void_p)]
+
+
+class Grads(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in GRAD_FIELDS]
 
 
 _lib = None
@@ -101,6 +110,11 @@ def load(build_if_missing: bool = True):
     lib.rglru_prefill_plan.restype = I
     lib.rglru_decode_plan.argtypes = [PD, PI, PI]
     lib.rglru_decode_plan.restype = I
+    PG = ctypes.POINTER(Grads)
+    lib.rglru_backward_workspace_size.argtypes = [PD]
+    lib.rglru_backward_workspace_size.restype = S
+    lib.rglru_block_backward.argtypes = [PD, PP, V, V, V, PS, V, V, V, PG, V, S, V]
+    lib.rglru_block_backward.restype = I
     lib.rglru_last_cuda_error.argtypes = [ctypes.POINTER(ctypes.c_char_p)]
     lib.rglru_last_cuda_error.restype = I
     lib.rglru_abi_version.argtypes = []
@@ -210,6 +224,26 @@ def block_decode(dims: Dims, params: Params, x: torch.Tensor, y: torch.Tensor, o
                                    _ptr(reset), ctypes.byref(st), _ptr(out), _ptr(workspace),
                                    workspace.numel(), _stream(stream))
     _check(rc, "rglru_block_decode")
+
+
+def backward_workspace_size(dims: Dims) -> int:
+    return load().rglru_backward_workspace_size(ctypes.byref(dims))
+
+
+def block_backward(dims: Dims, params: Params, x: torch.Tensor, y: torch.Tensor,
+                   dout: torch.Tensor, grads: dict, workspace: torch.Tensor,
+                   reset: Optional[torch.Tensor] = None, h0: Optional[torch.Tensor] = None,
+                   tail0: Optional[torch.Tensor] = None, dh_final: Optional[torch.Tensor] = None,
+                   dtail_final: Optional[torch.Tensor] = None, stream=None):
+    """rglru_block_backward: writes the gradients into the fp32 tensors of ``grads`` (keys of
+    GRAD_FIELDS; dh0 / dtail0 may be absent)."""
+    st = State(_ptr(h0), _ptr(tail0)) if h0 is not None else None
+    g = Grads(*(_ptr(grads.get(k)) for k in GRAD_FIELDS))
+    rc = load().rglru_block_backward(ctypes.byref(dims), ctypes.byref(params), _ptr(x), _ptr(y),
+                                     _ptr(reset), ctypes.byref(st) if st is not None else None,
+                                     _ptr(dout), _ptr(dh_final), _ptr(dtail_final), ctypes.byref(g),
+                                     _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "rglru_block_backward")
 
 
 def _plan(fn, dims: Dims):

@@ -185,6 +185,39 @@ rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_params* para
     return cuda_status(rglru::launch_decode_generic(dims, params, x, y, reset, state, out, s));
 }
 
+size_t rglru_backward_workspace_size(const rglru_dims* dims) {
+    if (check_dims(dims, true) != RGLRU_OK) return 0;
+    return rglru::backward_workspace(dims);
+}
+
+rglru_status rglru_block_backward(const rglru_dims* dims, const rglru_params* params,
+                                  const void* x, const void* y, const uint8_t* reset,
+                                  const rglru_state* state0, const void* dout,
+                                  const float* dh_final, const float* dtail_final,
+                                  const rglru_grads* grads, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    rglru_status st = check_dims(dims, true);
+    if (st != RGLRU_OK) return st;
+    if ((st = check_params(params)) != RGLRU_OK) return st;
+    if (!x || !y || !dout || !aligned(x, 16) || !aligned(y, 16) || !aligned(dout, 16)) return RGLRU_ERR_INVALID_ARG;
+    if (state0 && (st = check_state(state0)) != RGLRU_OK) return st;
+    if ((dh_final && !aligned(dh_final, 4)) || (dtail_final && !aligned(dtail_final, 4))) return RGLRU_ERR_INVALID_ARG;
+    if (!grads || !grads->dx || !grads->dy || !grads->dconv_w || !grads->dconv_b || !grads->dw_a ||
+        !grads->dw_x || !grads->db_a || !grads->db_x || !grads->dlambda)
+        return RGLRU_ERR_INVALID_ARG;
+    const void* outs[] = {grads->dx, grads->dy, grads->dh0, grads->dtail0, grads->dconv_w, grads->dconv_b,
+                          grads->dw_a, grads->dw_x, grads->db_a, grads->db_x, grads->dlambda};
+    for (const void* o : outs) {
+        if (o && !aligned(o, 4)) return RGLRU_ERR_INVALID_ARG;
+        if (o && (o == x || o == y || o == dout)) return RGLRU_ERR_INVALID_ARG;
+    }
+    if ((st = check_workspace(workspace, workspace_bytes, rglru_backward_workspace_size(dims))) != RGLRU_OK)
+        return st;
+    return cuda_status(rglru::launch_backward(dims, params, x, y, reset, state0, dout, dh_final, dtail_final,
+                                              grads, workspace, workspace_bytes,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 rglru_status rglru_block_prefill_noalloc(const rglru_dims* dims, const rglru_params* params,
                                          const void* x, const void* y, const uint8_t* reset,
                                          rglru_state* state, void* out, void* status_out,

@@ -24,13 +24,22 @@ cudaError_t launch_fused_prefill(const rglru_dims* d, const rglru_params* p, con
                                  const uint8_t* reset, rglru_state* st, void* out, void* ws, size_t ws_bytes,
                                  cudaStream_t s);
 
-// Tensor-core decode step (bf16, head_dim 256): conv + history shift, then tcgen05 gates and
-// the state update.  Needs the workspace fused_decode_workspace() (status word + conv scratch).
+// Tensor-core decode step (bf16, head_dim 256): one launch of 4-CTA clusters (conv + history
+// shift per channel quarter, conv blocks shared over distributed shared memory, tcgen05 gates,
+// the state update).  Needs the workspace fused_decode_workspace() (the status word).
 bool fused_decode_supported(const rglru_dims* d);
 size_t fused_decode_workspace(const rglru_dims* d);
 int fused_decode_launches(const rglru_dims* d);
 cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, const void* x, const void* y,
                                 const uint8_t* reset, rglru_state* st, void* out, void* ws, size_t ws_bytes,
                                 cudaStream_t s);
+
+// Backward pass of the prefill (CUDA cores, fp32, any supported shape): four launches.
+size_t backward_workspace(const rglru_dims* d);
+int backward_launches(const rglru_dims* d);
+cudaError_t launch_backward(const rglru_dims* d, const rglru_params* p, const void* x, const void* y,
+                            const uint8_t* reset, const rglru_state* st0, const void* dout,
+                            const float* dh_final, const float* dtail_final, const rglru_grads* grads,
+                            void* ws, size_t ws_bytes, cudaStream_t s);
 
 }  // namespace rglru

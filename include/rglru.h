@@ -112,6 +112,24 @@ typedef struct {
     void* conv_tail;   /* [B, 3, W] act dtype */
 } rglru_state;
 
+/* Gradients written by rglru_block_backward (device pointers, fp32, overwritten).  dx, dy:
+ * [B, T, W]; dh0: [B, W] and dtail0: [B, 3, W] (the initial state's gradient; either may be
+ * NULL when not wanted); dconv_w [4, W]; dconv_b, db_a, db_x, dlambda [W]; dw_a, dw_x
+ * [H, dh, dh] in the layout of w_a, w_x.  Gradients of absent biases are still written. */
+typedef struct {
+    float* dx;
+    float* dy;
+    float* dh0;
+    float* dtail0;
+    float* dconv_w;
+    float* dconv_b;
+    float* dw_a;
+    float* dw_x;
+    float* db_a;
+    float* db_x;
+    float* dlambda;
+} rglru_grads;
+
 /* Zero-fills state->h and state->conv_tail (the listing's "no prev_state" start).
  * Enqueued on `stream`.  Errors: INVALID_ARG (NULL/misaligned), CUDA. */
 RGLRU_API rglru_status rglru_state_init(const rglru_dims* dims, rglru_state* state, void* stream);
@@ -180,6 +198,29 @@ RGLRU_API rglru_status rglru_block_prefill_noalloc(const rglru_dims* dims,
                                  const rglru_params* params, const void* x, const void* y,
                                  const uint8_t* reset, rglru_state* state, void* out,
                                  void* status_out, void* stream);
+
+/* Bytes of device workspace rglru_block_backward needs (0 on invalid dims): the status word,
+ * four fp32 [B, T, W] arrays of per-token forward terms and eight fp32 [B, W] partial sums. */
+RGLRU_API size_t rglru_backward_workspace_size(const rglru_dims* dims);
+
+/* Backward pass of the prefill (the pages give the forward only; this is its chain rule,
+ * training being the pages' other use of the block): with out, h_{T-1} and the final conv
+ * history tail_T those of rglru_block_prefill(dims, params, x, y, reset, state0 copy), writes
+ * the gradients of
+ *     L = <dout, out> + <dh_final, h_{T-1}> + <dtail_final, tail_T>
+ * with respect to x, y, every parameter and the initial state into *grads.
+ *   x, y, dout [B, T, W] act dtype; reset [B, T] or NULL, as for the prefill.
+ *   state0: the state the forward started from, or NULL for zero (not modified).
+ *   dh_final [B, W], dtail_final [B, 3, W] fp32, or NULL for zero.
+ * CUDA cores, fp32 arithmetic; the forward is recomputed, so only its inputs are needed.
+ * Outputs must not alias inputs.  Errors as for rglru_block_prefill (host side, nothing
+ * launched on error). */
+RGLRU_API rglru_status rglru_block_backward(const rglru_dims* dims, const rglru_params* params,
+                                            const void* x, const void* y, const uint8_t* reset,
+                                            const rglru_state* state0, const void* dout,
+                                            const float* dh_final, const float* dtail_final,
+                                            const rglru_grads* grads, void* workspace,
+                                            size_t workspace_bytes, void* stream);
 
 /* How a call with `dims` runs: *kernel receives RGLRU_KERNEL_GENERIC (CUDA-core kernels) or
  * RGLRU_KERNEL_TENSOR (tcgen05 / TMEM kernels), *launches the number of kernel launches one
