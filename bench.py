@@ -307,6 +307,11 @@ def run_ours(args):
     if not args.no_decode:
         decode = bench_decode(args, dev)
 
+    # ---- backward pass of the same prefill workload (portable kernels) ----
+    backward = None
+    if not args.no_backward:
+        backward = bench_backward(args, dev)
+
     # ---- CPU oracle on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -339,6 +344,7 @@ def run_ours(args):
         "gpu_launches": args.steps * launches_per_prefill(dims),
         "clocks": clk,
         "decode": decode,
+        "backward": backward,
     }
     print(json.dumps(line), flush=True)
 
@@ -476,6 +482,50 @@ def bench_decode(args, dev):
             "gpu_launches": steps * binding.decode_launches(dims)}
 
 
+def bench_backward(args, dev, steps=3, warmup=1):
+    """rglru_block_backward on the prefill workload (zero initial state, random dout)."""
+    import torch
+    from gated_linear_recurrence_conv1d_b200 import binding
+
+    wl = inputs.WORKLOADS[args.workload]
+    prob = inputs.make_problem(wl, seed=0)
+    block = binding.RGLRUBlock(prob.params, wl.heads, wl.head_dim, wl.dtype, dev)
+    x = binding.to_device(prob.x, dev)
+    y = binding.to_device(prob.y, dev)
+    rng = np.random.default_rng(1)
+    dout = binding.to_device(inputs.make_activation(wl, rng, wl.batch, wl.seq_len), dev)
+    B, T, W, H, dh = wl.batch, wl.seq_len, wl.width, wl.heads, wl.head_dim
+    reset = None if prob.reset is None else binding.to_device(prob.reset, dev)
+    dims = block.dims(B, T)
+    ws = binding.alloc_workspace(binding.backward_workspace_size(dims), dev)
+    shapes = {"dx": (B, T, W), "dy": (B, T, W), "dh0": (B, W), "dtail0": (B, 3, W),
+              "dconv_w": (4, W), "dconv_b": (W,), "dw_a": (H, dh, dh), "dw_x": (H, dh, dh),
+              "db_a": (W,), "db_x": (W,), "dlambda": (W,)}
+    grads = {k: torch.empty(v, device=dev, dtype=torch.float32) for k, v in shapes.items()}
+    s = torch.cuda.Stream(device=dev)
+    for _ in range(warmup):
+        binding.block_backward(dims, block.params, x, y, dout, grads, ws, reset=reset, stream=s)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        binding.block_backward(dims, block.params, x, y, dout, grads, ws, reset=reset, stream=s)
+    e1.record(s)
+    torch.cuda.synchronize()
+    if binding.read_device_status(ws) != binding.RGLRU_OK:
+        raise RuntimeError("backward: device status not OK")
+    ms = e0.elapsed_time(e1) / steps
+    # algorithmic bytes: x, y, dout read (act dtype), dx, dy written (fp32), weights both ways
+    es = x.element_size()
+    alg = B * T * W * (3 * es + 8) + 2 * H * dh * dh * (es + 4)
+    peak, _ = measured_peaks()
+    return {"workload": wl.name, "value": B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": steps, "kernels": "portable CUDA-core kernels, fp32 arithmetic",
+            "effective_gbs": alg / (ms * 1e-3) / 1e9, "effective_frac": alg / (ms * 1e-3) / 1e9 / peak,
+            "gpu_launches": steps * binding.backward_launches(dims)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -492,6 +542,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=0,
                     help="decode steps per graph replay (default: the workload's 1024)")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

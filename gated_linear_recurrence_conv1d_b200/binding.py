@@ -32,7 +32,7 @@ EXPORTED = ("rglru_state_init", "rglru_prefill_workspace_size", "rglru_block_pre
             "rglru_decode_workspace_size", "rglru_block_decode", "rglru_read_device_status",
             "rglru_status_string", "rglru_abi_version", "rglru_prefill_plan", "rglru_decode_plan",
             "rglru_block_prefill_noalloc", "rglru_last_cuda_error", "rglru_backward_workspace_size",
-            "rglru_block_backward")
+            "rglru_block_backward", "rglru_backward_plan")
 
 # Fields of rglru_grads, in order (fp32 device tensors).
 GRAD_FIELDS = ("dx", "dy", "dh0", "dtail0", "dconv_w", "dconv_b", "dw_a", "dw_x", "db_a", "db_x",
@@ -110,6 +110,8 @@ def load(build_if_missing: bool = True):
     lib.rglru_prefill_plan.restype = I
     lib.rglru_decode_plan.argtypes = [PD, PI, PI]
     lib.rglru_decode_plan.restype = I
+    lib.rglru_backward_plan.argtypes = [PD, PI, PI]
+    lib.rglru_backward_plan.restype = I
     PG = ctypes.POINTER(Grads)
     lib.rglru_backward_workspace_size.argtypes = [PD]
     lib.rglru_backward_workspace_size.restype = S
@@ -267,6 +269,14 @@ def prefill_launches(dims: Dims) -> int:
 
 def decode_launches(dims: Dims) -> int:
     return decode_plan(dims)[1]
+
+
+def backward_plan(dims: Dims):
+    return _plan(load().rglru_backward_plan, dims)
+
+
+def backward_launches(dims: Dims) -> int:
+    return backward_plan(dims)[1]
 
 
 def read_device_status(workspace: torch.Tensor, stream=None) -> int:

@@ -268,6 +268,15 @@ rglru_status rglru_decode_plan(const rglru_dims* dims, int* kernel, int* launche
     return RGLRU_OK;
 }
 
+rglru_status rglru_backward_plan(const rglru_dims* dims, int* kernel, int* launches) {
+    rglru_status st = check_dims(dims, true);
+    if (st != RGLRU_OK) return st;
+    if (!kernel || !launches) return RGLRU_ERR_INVALID_ARG;
+    *kernel = RGLRU_KERNEL_GENERIC;
+    *launches = rglru::backward_launches(dims);
+    return RGLRU_OK;
+}
+
 rglru_status rglru_read_device_status(void* workspace, size_t workspace_bytes, void* stream) {
     if (!workspace || workspace_bytes < sizeof(rglru::DeviceStatus) || !aligned(workspace, 256))
         return RGLRU_ERR_INVALID_ARG;

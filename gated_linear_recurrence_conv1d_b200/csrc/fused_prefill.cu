@@ -649,18 +649,20 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 mbar_arrive(bars.x_empty[st]);
                 mbar_arrive(bars.b_full[st]);
             }
-            // final conv history of the sequence, once its first chunk has read the old one
+            // final conv history of the sequence.  The old one is read by the conv of the row's
+            // first chunk in BOTH channel-half groups of the head (each convolves all 256 input
+            // channels), so it is overwritten only once both of those chunks have published
+            // their state (which follows their conv); this one included when the row has one
+            // chunk.
             if (a.tail_state && c == a.NC - 1 && has_last) {
-                bool ok;
-                if (c > 0) {
-                    unsigned f = 0;
-                    if (lane == 0) f = wait_flag(a.lb_flags + (lb_base + (size_t)b * a.NC) * 4, FLAG_AGG, wc, 8);
-                    ok = __shfl_sync(0xffffffffu, f, 0) != 0;
-                } else {
-                    // a row of one chunk: the warps of the first token half read the old history
-                    // in this very item; once every conv warp has arrived on b_full, it is read
-                    ok = wait_bar_warp(bars.b_full[st], ph, wc, 18);
+                unsigned f = 0;
+                if (lane == 0) {
+                    f = wait_flag(a.lb_flags + (lb_base + (size_t)b * a.NC) * 4, FLAG_AGG, wc, 8);
+                    if (f)
+                        f = wait_flag(a.lb_flags + ((size_t)(group ^ 1) * a.items + (size_t)b * a.NC) * 4,
+                                      FLAG_AGG, wc, 18);
                 }
+                const bool ok = __shfl_sync(0xffffffffu, f, 0) != 0;
                 if (ok && own_tail) {
                     __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
 #pragma unroll

@@ -230,6 +230,7 @@ RGLRU_API rglru_status rglru_block_backward(const rglru_dims* dims, const rglru_
 #define RGLRU_KERNEL_TENSOR 1
 RGLRU_API rglru_status rglru_prefill_plan(const rglru_dims* dims, int* kernel, int* launches);
 RGLRU_API rglru_status rglru_decode_plan(const rglru_dims* dims, int* kernel, int* launches);
+RGLRU_API rglru_status rglru_backward_plan(const rglru_dims* dims, int* kernel, int* launches);
 
 /* Synchronises `stream`, reads and clears the device status word at the start of
  * `workspace`, and returns RGLRU_OK, RGLRU_ERR_TIMEOUT or RGLRU_ERR_DEVICE (or

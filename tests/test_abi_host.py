@@ -126,3 +126,34 @@ def test_read_status_rejects_bad_workspace():
     lib = binding.load()
     assert lib.rglru_read_device_status(None, 256, None) == 1
     assert lib.rglru_read_device_status(ctypes.c_void_p(FAKE + 4), 256, None) == 1
+
+
+def _backward(d, grads=None, x=FAKE, dout=FAKE + 0x300, ws=FAKE, ws_bytes=1 << 30):
+    lib = binding.load()
+    p = _params()
+    if grads is None:
+        grads = binding.Grads(*(ctypes.c_void_p(FAKE + 0x1000 * (i + 1)) for i in range(len(binding.GRAD_FIELDS))))
+    g = ctypes.byref(grads) if grads is not False else None
+    return lib.rglru_block_backward(ctypes.byref(d), ctypes.byref(p), ctypes.c_void_p(x) if x else None,
+                                    ctypes.c_void_p(FAKE + 0x100), None, None,
+                                    ctypes.c_void_p(dout) if dout else None, None, None, g,
+                                    ctypes.c_void_p(ws) if ws else None, ws_bytes, None)
+
+
+def test_backward_rejects_bad_arguments():
+    d = _dims()
+    assert binding.backward_workspace_size(d) > 4 * 2 * 16 * 128 * 4
+    assert binding.backward_workspace_size(_dims(seq_len=0)) == 0
+    assert binding.backward_plan(d) == (0, 4)
+    assert _backward(_dims(head_dim=24)) == 2
+    assert _backward(d, x=None) == 1
+    assert _backward(d, dout=None) == 1
+    assert _backward(d, dout=FAKE + 2) == 1                  # misaligned
+    assert _backward(d, grads=False) == 1                     # no output struct
+    fields = [ctypes.c_void_p(FAKE + 0x1000 * (i + 1)) for i in range(len(binding.GRAD_FIELDS))]
+    fields[0] = None                                          # dx is required
+    assert _backward(d, grads=binding.Grads(*fields)) == 1
+    fields[0] = ctypes.c_void_p(FAKE)                         # dx aliases x
+    assert _backward(d, grads=binding.Grads(*fields)) == 1
+    assert _backward(d, ws=None) == 3
+    assert _backward(d, ws_bytes=64) == 3
