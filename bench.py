@@ -310,7 +310,10 @@ def run_ours(args):
     # ---- backward pass of the same prefill workload (portable kernels) ----
     backward = None
     if not args.no_backward:
-        backward = bench_backward(args, dev)
+        try:
+            backward = bench_backward(args, dev)
+        except Exception as exc:  # the prefill line above is the contract; report, do not lose it
+            backward = {"error": f"{type(exc).__name__}: {exc}"}
 
     # ---- CPU oracle on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
