@@ -190,6 +190,28 @@ def oracle_prefill_rate(prob: inputs.Problem, target_s: float = 15.0, threads: i
     return done / dt, desc, cores, dt
 
 
+def oracle_backward_rate(prob: inputs.Problem, target_s: float = 3.0):
+    """Times the fp64 oracle's backward (sequential, one core) on one row with all its heads,
+    the leading tokens, sized to about target_s.  Returns (tokens/s, description, cores, s)."""
+    import oracle
+    wl = prob.wl
+    rng = np.random.default_rng(1)
+
+    def run(tokens):
+        x, y = prob.x[:1, :tokens], prob.y[:1, :tokens]
+        dout = inputs.make_activation(wl, rng, 1, tokens)
+        reset = None if prob.reset is None else prob.reset[:1, :tokens]
+        t0 = time.perf_counter()
+        oracle.backward(prob.params, x, y, wl.heads, dout, reset=reset, gelu_tanh=wl.gelu_tanh)
+        return time.perf_counter() - t0
+
+    per_token = max(run(min(8, wl.seq_len)) / min(8, wl.seq_len), 1e-7)
+    tokens = int(min(wl.seq_len, max(8, target_s / per_token)))
+    dt = run(tokens)
+    desc = f"1 row x first {tokens} tokens x all {wl.heads} heads of {wl.name}, one pass"
+    return tokens / dt, desc, 1, dt
+
+
 def run_reference(args):
     rank, world, _ = env_rank()
     if rank != 0:
@@ -523,10 +545,15 @@ def bench_backward(args, dev, steps=3, warmup=1):
     es = x.element_size()
     alg = B * T * W * (3 * es + 8) + 2 * H * dh * dh * (es + 4)
     peak, _ = measured_peaks()
-    return {"workload": wl.name, "value": B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+    line = {"workload": wl.name, "value": B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "steps": steps, "kernels": "portable CUDA-core kernels, fp32 arithmetic",
             "effective_gbs": alg / (ms * 1e-3) / 1e9, "effective_frac": alg / (ms * 1e-3) / 1e9 / peak,
             "gpu_launches": steps * binding.backward_launches(dims)}
+    if not args.no_cpu:
+        rate, desc, cores, secs = oracle_backward_rate(prob, target_s=min(3.0, args.cpu_seconds))
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": round(secs, 2)}
+    return line
 
 
 def main():

@@ -65,3 +65,13 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
 
     bench.run_reference(Args())
     assert capsys.readouterr().out == ""
+
+
+def test_oracle_backward_rate_on_a_small_sample():
+    """The CPU baseline beside the backward measurement: a bounded oracle sample."""
+    from gated_linear_recurrence_conv1d_b200 import inputs
+    wl = inputs.WORKLOADS["tiny_f32"].scaled(seq_len=40)
+    prob = inputs.make_problem(wl, seed=0)
+    rate, desc, cores, secs = bench.oracle_backward_rate(prob, target_s=0.05)
+    assert rate > 0 and cores == 1 and secs > 0
+    assert "tiny_f32" in desc
