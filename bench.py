@@ -343,6 +343,13 @@ def run_ours(args):
         rate, desc, cores, secs = oracle_prefill_rate(prob, target_s=args.cpu_seconds)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc,
                "seconds": round(secs, 2)}
+        # the same oracle on one core, on this workload and on the tiny fp32 one
+        single = {}
+        for name, pr in ((wl.name, prob),
+                         ("tiny_f32", inputs.make_problem(inputs.WORKLOADS["tiny_f32"], seed=0))):
+            r1, d1, _, s1 = oracle_prefill_rate(pr, target_s=min(3.0, args.cpu_seconds), threads=1)
+            single[name] = {"value": r1, "unit": "tokens/s", "sample": d1, "seconds": round(s1, 2)}
+        cpu["single_thread"] = single
 
     if world > 1:
         dist.barrier()
