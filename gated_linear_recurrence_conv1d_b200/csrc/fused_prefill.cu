@@ -135,6 +135,7 @@ struct Args {
     const uint8_t* reset;
     float* h_state;                  // nullptr: zero initial state, no write-back
     __nv_bfloat16* tail_state;
+    const __nv_bfloat16* tail_old;   // the conv history as the call found it (a copy), or nullptr
     DeviceStatus* status;
     unsigned* counters;              // [groups] tickets
     unsigned* lb_flags;              // [groups][items][4]
@@ -611,8 +612,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             };
             Vec4 h0, h1, h2;                              // window x_{t-3}, x_{t-2}, x_{t-1}
             if (c == 0 && j0 == 0) {
-                if (a.tail_state) {
-                    const __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
+                if (a.tail_old) {
+                    const __nv_bfloat16* tl = a.tail_old + (size_t)b * kHist * W + chg;
                     h0 = unpack4(*reinterpret_cast<const uint2*>(tl));
                     h1 = unpack4(*reinterpret_cast<const uint2*>(tl + W));
                     h2 = unpack4(*reinterpret_cast<const uint2*>(tl + 2 * W));
@@ -649,25 +650,14 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 mbar_arrive(bars.x_empty[st]);
                 mbar_arrive(bars.b_full[st]);
             }
-            // final conv history of the sequence.  The old one is read by the conv of the row's
-            // first chunk in BOTH channel-half groups of the head (each convolves all 256 input
-            // channels), so it is overwritten only once both of those chunks have published
-            // their state (which follows their conv); this one included when the row has one
-            // chunk.
-            if (a.tail_state && c == a.NC - 1 && has_last) {
-                unsigned f = 0;
-                if (lane == 0) {
-                    f = wait_flag(a.lb_flags + (lb_base + (size_t)b * a.NC) * 4, FLAG_AGG, wc, 8);
-                    if (f)
-                        f = wait_flag(a.lb_flags + ((size_t)(group ^ 1) * a.items + (size_t)b * a.NC) * 4,
-                                      FLAG_AGG, wc, 18);
-                }
-                const bool ok = __shfl_sync(0xffffffffu, f, 0) != 0;
-                if (ok && own_tail) {
-                    __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
+            // final conv history of the sequence.  Both channel-half groups of the head read the
+            // old history (each convolves all 256 input channels), from the copy taken before the
+            // launch, so the state buffer is only written, by the group that owns the channels,
+            // as soon as the row's last token is convolved: no CTA waits for another here.
+            if (a.tail_state && c == a.NC - 1 && has_last && own_tail) {
+                __nv_bfloat16* tl = a.tail_state + (size_t)b * kHist * W + chg;
 #pragma unroll
-                    for (int r = 0; r < 3; ++r) *reinterpret_cast<uint2*>(tl + (size_t)r * W) = fw[r];
-                }
+                for (int r = 0; r < 3; ++r) *reinterpret_cast<uint2*>(tl + (size_t)r * W) = fw[r];
             }
         }
     } else if (warp < kWarpEpi0 + kEpiWarps) {
@@ -965,7 +955,7 @@ bool make_map_2d_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_
 struct Plan {
     int NC, items, groups, ctas, base, extra;
     int NA;
-    size_t off_counters, off_flags, off_agg, off_incl, total;
+    size_t off_counters, off_flags, off_agg, off_incl, off_tail, total;
 };
 
 Plan make_plan(const rglru_dims* d, int sms) {
@@ -982,7 +972,8 @@ Plan make_plan(const rglru_dims* d, int sms) {
     p.off_agg = up(p.off_flags + (size_t)p.groups * p.items * 16);
     p.NA = (p.NC + LBW - 1) / LBW;
     p.off_incl = up(p.off_agg + (size_t)p.groups * p.items * HALF * 8);
-    p.total = up(p.off_incl + (size_t)p.groups * d->batch * p.NA * HALF * 8);
+    p.off_tail = up(p.off_incl + (size_t)p.groups * d->batch * p.NA * HALF * 8);
+    p.total = up(p.off_tail + (size_t)d->batch * kHist * d->heads * DH * sizeof(__nv_bfloat16));
     return p;
 }
 
@@ -998,7 +989,8 @@ size_t fused_prefill_workspace(const rglru_dims* d) { return tc::make_plan(d, 10
 
 int fused_prefill_launches(const rglru_dims* d) {
     (void)d;
-    return 2;   // one memset of the tickets / look-back flags, one kernel
+    return 2;   // one memset of the tickets / look-back words, one kernel (plus a copy of the
+                // conv history when a state is given: not a kernel)
 }
 
 cudaError_t launch_fused_prefill(const rglru_dims* d, const rglru_params* p, const void* x, const void* y,
@@ -1040,9 +1032,17 @@ cudaError_t launch_fused_prefill(const rglru_dims* d, const rglru_params* p, con
     a.lb_agg = reinterpret_cast<uint64_t*>(w + pl.off_agg);
     a.lb_incl = reinterpret_cast<uint64_t*>(w + pl.off_incl);
     // tickets, flags and look-back words all start at zero ("not written")
-    const size_t clear = pl.total - pl.off_counters;
+    const size_t clear = pl.off_tail - pl.off_counters;
     e = cudaMemsetAsync(w + pl.off_counters, 0, clear, s);
     if (e != cudaSuccess) return e;
+    // the conv history as this call finds it: the kernel reads the copy and writes the state
+    a.tail_old = nullptr;
+    if (a.tail_state) {
+        const size_t tail_bytes = (size_t)d->batch * kHist * W * sizeof(__nv_bfloat16);
+        e = cudaMemcpyAsync(w + pl.off_tail, a.tail_state, tail_bytes, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return e;
+        a.tail_old = reinterpret_cast<const __nv_bfloat16*>(w + pl.off_tail);
+    }
     fused_prefill_kernel<<<pl.ctas, kThreads, SMEM_BYTES, s>>>(mx, my, mo, a);
     return cudaGetLastError();
 }
