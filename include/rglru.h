@@ -222,9 +222,11 @@ RGLRU_API rglru_status rglru_block_backward(const rglru_dims* dims, const rglru_
                                             const rglru_grads* grads, void* workspace,
                                             size_t workspace_bytes, void* stream);
 
-/* How a call with `dims` runs: *kernel receives RGLRU_KERNEL_GENERIC (CUDA-core kernels) or
- * RGLRU_KERNEL_TENSOR (tcgen05 / TMEM kernels), *launches the number of kernel launches one
- * call enqueues.  The choice depends on dims only (the library targets sm_100a alone).
+/* How a call with `dims` runs (rglru_block_prefill, rglru_block_decode, rglru_block_backward):
+ * *kernel receives RGLRU_KERNEL_GENERIC (CUDA-core kernels) or RGLRU_KERNEL_TENSOR (tcgen05 /
+ * TMEM kernels), *launches the number of operations one call enqueues (the tensor-core prefill
+ * counts its workspace memset with its kernel; its copy of a given conv history is not
+ * counted).  The choice depends on dims only (the library targets sm_100a alone).
  * Errors: INVALID_ARG / UNSUPPORTED exactly as the corresponding call would return them. */
 #define RGLRU_KERNEL_GENERIC 0
 #define RGLRU_KERNEL_TENSOR 1
