@@ -120,6 +120,27 @@ def test_backward_reset_at_the_first_token_cuts_the_initial_state():
     assert not np.any(g["dh0"]) and not np.any(g["dtail0"])
 
 
+def test_gelu_tanh_derivative_matches_torch_autograd():
+    """The backward's tanh-GeLU derivative against torch autograd of torch's own fp64
+    gelu(approximate="tanh"): one token per channel, out = h_0 GeLU(y), so
+    dy / (dout h_0) = GeLU'(y) for 16 values of y across [-6, 6]."""
+    import torch
+    vs = np.linspace(-6.0, 6.0, 16).astype(np.float32)
+    t = torch.tensor(vs.astype(np.float64), requires_grad=True)
+    torch.nn.functional.gelu(t, approximate="tanh").sum().backward()
+    ref = t.grad.numpy()
+    p = dict(conv_w=np.zeros((4, 16), np.float32), conv_b=np.ones(16, np.float32),
+             w_a=np.zeros((1, 16, 16), np.float32), w_x=np.zeros((1, 16, 16), np.float32),
+             b_a=np.zeros(16, np.float32), b_x=np.full(16, 40.0, np.float32), lam=np.full(16, 2.0, np.float32))
+    x = np.zeros((1, 1, 16), np.float32)
+    y = vs.reshape(1, 1, 16)
+    dout = np.ones((1, 1, 16), np.float32)
+    _, h_after, _ = oracle.prefill(p, x, y, 1, gelu_tanh=1)
+    g = oracle.backward(p, x, y, 1, dout, gelu_tanh=1)
+    got = g["dy"][0, 0] / h_after[0]
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14)
+
+
 @pytest.mark.parametrize("v", [-6.0, -1.5, -0.3, 0.0, 0.7, 2.5, 9.0])
 @pytest.mark.parametrize("tanh_form", [0, 1])
 def test_gelu_derivative_matches_a_difference_quotient(v, tanh_form):

@@ -29,10 +29,14 @@ MUTANTS = {
     "gate_bias_swapped": ("ga[o] = b_a ? (double)b_a[o] : 0.0;", "ga[o] = b_x ? (double)b_x[o] : 0.0;"),
     "input_gate_from_recurrence_weights": ("gx[o] += xi * widen(w_x, (long)i * dh + o, w_dtype);", "gx[o] += xi * widen(w_a, (long)i * dh + o, w_dtype);"),
     "gelu_tanh_by_default": ("    return 0.5 * v * erfc(-v / sqrt(2.0));", "    return 0.5 * v * (1.0 + tanh(0.7978845608028654 * (v + 0.044715 * v * v * v)));"),
+    # constants of the tanh form perturbed within 1e-3 of the exact GeLU
+    "gelu_tanh_constants": ("        return 0.5 * v * (1.0 + tanh(k * (v + 0.044715 * v * v * v)));",
+                            "        return 0.5 * v * (1.0 + tanh(0.8 * (v + 0.0447 * v * v * v)));"),
 }
 
 PIN_TESTS = [
     pins.test_gelu_spot_values,
+    pins.test_gelu_tanh_form_matches_torch,
     pins.test_closed_form_geometric_sum,
     pins.test_freeze_when_recurrence_gate_is_zero,
     pins.test_decay_strictly_inside_unit_interval,
@@ -57,10 +61,12 @@ BACKWARD_MUTANTS = {
                                    "dw_a[(long)o * dh + i] += xct[i] * dga[o];"),
     "bwd_conv_scatter_wrong_tap": ("if (src >= 0) dx[(long)src * ld + j] += (double)conv_w[k * conv_ld + j] * d;",
                                    "if (src >= 0) dx[(long)src * ld + j] += (double)conv_w[(3 - k) * conv_ld + j] * d;"),
+    "bwd_gelu_tanh_chain_factor": ("k * (1.0 + 3.0 * 0.044715 * v * v);", "k * (1.0 + 0.044715 * v * v);"),
 }
 
 BACKWARD_PIN_TESTS = [
     bwd_pins.test_backward_matches_finite_differences,
+    bwd_pins.test_gelu_tanh_derivative_matches_torch_autograd,
     bwd_pins.test_backward_frozen_state_closed_form,
     bwd_pins.test_backward_reset_at_the_first_token_cuts_the_initial_state,
     lambda: bwd_pins.test_gelu_derivative_matches_a_difference_quotient(0.7, 0),

@@ -68,6 +68,17 @@ def test_gelu_spot_values():
         assert oracle.gelu(v) == pytest.approx(_gelu_ref(v), rel=1e-13, abs=1e-300)
 
 
+def test_gelu_tanh_form_matches_torch():
+    """The tanh variant against an independent implementation of the same formula: torch's
+    fp64 gelu(approximate="tanh") at 121 points across [-8, 8] (both sides evaluate
+    0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))), so they agree to rounding)."""
+    import torch
+    vs = np.concatenate([np.linspace(-8, 8, 113), [-1e-3, 1e-3, -0.5, 0.5, 3.0, -3.0, 1e-8, 20.0]])
+    ref = torch.nn.functional.gelu(torch.tensor(vs, dtype=torch.float64), approximate="tanh").numpy()
+    for v, r in zip(vs, ref):
+        assert oracle.gelu(v, 1) == pytest.approx(r, rel=1e-13, abs=1e-300), v
+
+
 def test_gelu_tanh_form_properties():
     # odd-symmetric part: g(v) - g(-v) = v for both forms (1 + s(v), s odd)
     for v in np.linspace(-5, 5, 41):
