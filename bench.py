@@ -1,14 +1,19 @@
 #!/usr/bin/env python
-"""Benchmark of the RG-LRU recurrent block on B200: prefill tokens/s and HBM roofline.
+"""Benchmark of the RG-LRU recurrent block on B200: prefill / decode tokens/s and HBM roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one full-sequence prefill (conv -> gates -> scan -> GeLU merge, state written back)
-of the RecurrentGemma-2B-shaped workload: batch 8 x 2048 tokens, LRU width 2560 = 10 heads x
-256, bf16 activations and gate weights, fp32 state; synthetic seeded inputs (no dataset, no
-trained weights).  Inputs stay resident in HBM; one step moves 252 MB, more than the 126 MB L2,
-so consecutive steps do not hit in L2.  The same JSON line also reports the single-token
-decode workload (batch 256, width 2560, 1024 steps replayed from one CUDA graph).
+A step is one full-sequence prefill (conv -> gates -> scan -> GeLU merge, state read and
+written back) through the C ABI.  The headline workload is the packed variable-length
+prefill: batch 16 x 8192 tokens, LRU width 6144 = 24 heads x 256, documents of 64..4096
+tokens packed per row with a segment-reset mask, bf16 activations and gate weights, fp32
+state; synthetic seeded inputs (no dataset, no trained weights).  Inputs stay resident in HBM;
+one step moves 4.8 GB, far more than the 126 MB L2.  The same JSON line carries one entry per
+workload under "configs": the tiny fp32 check (L2 flushed between launches), the
+RecurrentGemma-2B-shaped batch (B8 T2048, 10 x 256), the long-context row (B1 T65536,
+16 x 256), the packed headline, and the single-token decode (batch 256, width 2560, 1024 steps
+replayed from one CUDA graph); each with tokens/s, time per launch, algorithmic bytes, the
+roofline fraction and the fp64 oracle timed on the host cores on a bounded sample.
 
 N > 1 (torchrun): every rank runs its own replica of the workload on its own GPU (the block
 shards over batch rows and heads with no exchange), the timed region is bracketed by a
@@ -21,6 +26,7 @@ workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import gc
 import hashlib
 import json
 import os
@@ -37,15 +43,17 @@ sys.path.insert(0, ROOT)
 
 from gated_linear_recurrence_conv1d_b200 import inputs  # noqa: E402
 
-WORKLOAD = "rg2b_bf16"
+WORKLOAD = "packed_bf16"                 # the headline: the largest single-GPU workload
+PREFILL_WORKLOADS = ("tiny_f32", "rg2b_bf16", "long_bf16", "packed_bf16")
 DECODE_WORKLOAD = "decode_bf16"
-METRIC = "RG-LRU block prefill tokens/s (RecurrentGemma-2B-shaped, bf16, fp32 state)"
+METRIC = "RG-LRU block tokens/s (prefill, decode) and achieved HBM GB/s"
+# seconds of GPU time each non-headline prefill workload is timed for
+CONFIG_SECONDS = 1.0
 
 # DRAM bytes per launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum) for a
 # given kernel source; keyed by the sha256 of that source so a changed kernel reports null.
 NCU_TRAFFIC = {
-    # rg2b_bf16 step with state, one launch: 179.69 MB read + 88.97 MB written
-    ("fused_prefill.cu", "e7f5915d5d3c3389"): 268657152,
+    # (kernel source, its sha256 prefix, workload): bytes per launch
 }
 
 
@@ -220,8 +228,10 @@ def run_reference(args):
     prob = inputs.make_problem(wl, seed=0)
     vals = []
     desc, cores = "", 0
+    # each step a bounded sample, so that the whole run stays within about two minutes
+    step_s = min(args.ref_step_s, 120.0 / (args.warmup + args.steps))
     for i in range(args.warmup + args.steps):
-        rate, desc, cores, _ = oracle_prefill_rate(prob, target_s=args.ref_step_s)
+        rate, desc, cores, _ = oracle_prefill_rate(prob, target_s=step_s)
         if i >= args.warmup:
             vals.append(rate)
     value = float(statistics.median(vals))
@@ -230,8 +240,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * wl.batch * wl.seq_len / value, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seq_len,
-                   "heads": wl.heads, "head_dim": wl.head_dim, "width": wl.width},
+        "config": workload_config(wl, world=1),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -239,7 +248,108 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def workload_config(wl: inputs.Workload, world: int) -> dict:
+    moved = algorithmic_bytes(wl, wl.batch * wl.seq_len)
+    cfg = {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seq_len, "heads": wl.heads,
+           "head_dim": wl.head_dim, "width": wl.width, "act_dtype": wl.dtype,
+           "state": "fp32, read and written back",
+           "parallelism": f"replicas x{world}"}
+    if wl.doc_len is not None:
+        cfg["documents"] = f"lengths U{{{wl.doc_len[0]}..{wl.doc_len[1]}}} packed per row, reset mask"
+    cfg["l2"] = (f"inputs larger than L2 ({moved / 1e6:.0f} MB moved per step > 126 MB L2)"
+                 if moved > 126e6 else "L2 flushed (256 MB write) between timed launches")
+    return cfg
+
+
 # ------------------------------------------------------------------ GPU path --------------
+
+class PrefillRig:
+    """One prefill workload resident on the device, run through the C ABI."""
+
+    def __init__(self, binding, wl: inputs.Workload, dev):
+        import torch
+        self.binding, self.wl, self.dev = binding, wl, dev
+        self.prob = inputs.make_problem(wl, seed=0)
+        self.block = binding.RGLRUBlock(self.prob.params, wl.heads, wl.head_dim, wl.dtype, dev)
+        self.x = binding.to_device(self.prob.x, dev)
+        self.y = binding.to_device(self.prob.y, dev)
+        self.reset = None if self.prob.reset is None else binding.to_device(self.prob.reset, dev)
+        self.out = torch.empty_like(self.x)
+        B, W = wl.batch, wl.width
+        self.h = torch.zeros(B, W, device=dev)
+        self.tail = torch.zeros(B, 3, W, device=dev, dtype=self.x.dtype)
+        self.dims = self.block.dims(B, wl.seq_len)
+        self.ws = binding.alloc_workspace(binding.prefill_workspace_size(self.dims), dev)
+
+    def step(self, stream=None):
+        self.binding.block_prefill(self.dims, self.block.params, self.x, self.y, self.out, self.ws,
+                                   reset=self.reset, h=self.h, conv_tail=self.tail, stream=stream)
+
+    def check_status(self, when: str):
+        if self.binding.read_device_status(self.ws) != self.binding.RGLRU_OK:
+            raise RuntimeError(f"{self.wl.name}: device status not OK {when}")
+
+
+def time_prefill(rig: PrefillRig, steps: int, warmup: int, flush_l2: bool, dev, dist=None,
+                 world: int = 1, clocks_gpu=None):
+    """Times `steps` launches of the prefill on the current stream with CUDA events: per-launch
+    events around each call and one pair around the whole loop (between barrier + synchronize
+    on both sides).  With flush_l2 a 256 MB buffer is written between launches, outside the
+    per-launch events.  Returns (total_ms, per-launch ms list, clock summary)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev) if flush_l2 else None
+    for _ in range(max(3, warmup)):
+        rig.step()
+    torch.cuda.synchronize()
+    rig.check_status("after warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(clocks_gpu if clocks_gpu is not None else dev.index) as clocks:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(steps):
+            if flush is not None:
+                flush.fill_(float(i))
+            evs[i][0].record(stream)
+            rig.step()
+            evs[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    rig.check_status("after the timed region")
+    per = [a.elapsed_time(b) for a, b in evs]
+    total = sum(per) if flush_l2 else t0.elapsed_time(t1)
+    return max_over_ranks(total, dist, dev), per, clocks.summary()
+
+
+def prefill_entry(rig: PrefillRig, total_ms: float, per_ms, steps: int, world: int, clk) -> dict:
+    wl = rig.wl
+    B, T = wl.batch, wl.seq_len
+    peak, peak_kind = measured_peaks()
+    alg = algorithmic_bytes(wl, B * T, with_state=True)
+    launch_ms = statistics.mean(per_ms)
+    achieved = alg / (launch_ms / 1e3) / 1e9
+    kernel, launches = rig.binding.prefill_plan(rig.dims)
+    return {"workload": wl.name, "batch": B, "seq_len": T, "heads": wl.heads,
+            "head_dim": wl.head_dim, "act_dtype": wl.dtype, "steps": steps,
+            "value": job_throughput(B * T, world, steps, total_ms), "unit": "tokens/s",
+            "ms_per_launch": launch_ms, "ms_per_launch_median": statistics.median(per_ms),
+            "algorithmic_bytes_per_launch": alg, "achieved_gbs": achieved,
+            "roofline_frac": achieved / peak, "peak_gbs": peak, "peak_kind": peak_kind,
+            "frac_of_8TBs": achieved / 8000.0,
+            "kernel": "tensor" if kernel == 1 else "generic", "launches_per_step": launches,
+            "l2": workload_config(wl, world)["l2"], "clocks": clk}
+
+
+def steps_for(ms_per_launch: float, seconds: float, lo: int = 5, hi: int = 2000) -> int:
+    return int(min(hi, max(lo, seconds * 1000.0 / max(ms_per_launch, 1e-3))))
+
 
 def run_ours(args):
     import torch
@@ -252,84 +362,75 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     dev = torch.device("cuda", torch.cuda.current_device())
-    lib = binding.load()
-    del lib
+    binding.load()
+    dd = dist if world > 1 else None
+    clocks_gpu = dev.index if world == 1 else local
+    cpu_on = rank == 0 and world == 1 and not args.no_cpu
 
-    wl = inputs.WORKLOADS[args.workload]
-    prob = inputs.make_problem(wl, seed=0)
-    block = binding.RGLRUBlock(prob.params, wl.heads, wl.head_dim, wl.dtype, dev)
-    x = binding.to_device(prob.x, dev)
-    y = binding.to_device(prob.y, dev)
-    reset = None if prob.reset is None else binding.to_device(prob.reset, dev)
-    out = torch.empty_like(x)
+    # ---- the headline workload: K timed steps ----
+    head = PrefillRig(binding, inputs.WORKLOADS[args.workload], dev)
+    wl = head.wl
     B, T, W = wl.batch, wl.seq_len, wl.width
-    h = torch.zeros(B, W, device=dev)
-    tail = torch.zeros(B, 3, W, device=dev, dtype=x.dtype)
-    dims = block.dims(B, T)
-    ws = binding.alloc_workspace(binding.prefill_workspace_size(dims), dev)
-    stream = torch.cuda.current_stream()
-
-    def step():
-        binding.block_prefill(dims, block.params, x, y, out, ws, reset=reset, h=h, conv_tail=tail)
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    torch.cuda.synchronize()
-    if binding.read_device_status(ws) != binding.RGLRU_OK:
-        raise RuntimeError("device status not OK after warm-up")
-
-    # ---- timed region: K prefill steps, per-launch CUDA events on the launching stream ----
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(dev.index if world == 1 else local) as clocks:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        for i in range(args.steps):
-            evs[i][0].record(stream)
-            step()
-            evs[i][1].record(stream)
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    total_ms = t_start.elapsed_time(t_end)
-    launch_ms = [a.elapsed_time(b) for a, b in evs]
-    status = binding.read_device_status(ws)
-    if status != binding.RGLRU_OK:
-        raise RuntimeError(f"device status {status} after the timed region")
-
-    total_ms = max_over_ranks(total_ms, dist if world > 1 else None, dev)
-    tokens_per_rank = B * T
-    value = job_throughput(tokens_per_rank, world, args.steps, total_ms)
-
-    # ---- roofline of the prefill kernel ----
+    total_ms, per_ms, clk = time_prefill(head, args.steps, args.warmup, flush_l2=False, dev=dev,
+                                         dist=dd, world=world, clocks_gpu=clocks_gpu)
+    value = job_throughput(B * T, world, args.steps, total_ms)
+    head_entry = prefill_entry(head, total_ms, per_ms, args.steps, world, clk)
     peak, peak_kind = measured_peaks()
-    alg = algorithmic_bytes(wl, B * T, with_state=True)
-    avg_launch_s = statistics.mean(launch_ms) / 1000.0
-    achieved = alg / avg_launch_s / 1e9
     src = os.path.join(ROOT, "gated_linear_recurrence_conv1d_b200", "csrc", "fused_prefill.cu")
-    if not os.path.exists(src):
-        src = os.path.join(ROOT, "gated_linear_recurrence_conv1d_b200", "csrc", "generic.cu")
-    traffic = NCU_TRAFFIC.get((os.path.basename(src), _sha(src)))
+    traffic = NCU_TRAFFIC.get((os.path.basename(src), _sha(src), wl.name))
+    roofline = {"bound": "hbm", "achieved": head_entry["achieved_gbs"], "peak": peak, "unit": "GB/s",
+                "frac": head_entry["roofline_frac"], "traffic": traffic, "peak_kind": peak_kind,
+                "algorithmic_bytes_per_launch": head_entry["algorithmic_bytes_per_launch"],
+                "frac_of_8TBs": head_entry["frac_of_8TBs"], "kernel_source": os.path.basename(src),
+                "workload": wl.name}
 
     # ---- end to end through the C ABI with pinned host buffers ----
     e2e_steps = max(3, min(args.steps, args.e2e_steps))
-    e2e_ms = e2e_pipelined(binding, block, x, y, h, tail, reset, B, T, e2e_steps, dev, dist if world > 1 else None)
-    e2e_value = job_throughput(tokens_per_rank, world, e2e_steps, e2e_ms)
-    es = x.element_size()
-    h2d = 2 * B * T * W * es
+    e2e_ms = e2e_pipelined(binding, head.block, head.x, head.y, head.h, head.tail, head.reset, B, T,
+                           e2e_steps, dev, dd)
+    e2e_value = job_throughput(B * T, world, e2e_steps, e2e_ms)
+    es = head.x.element_size()
+    h2d = 2 * B * T * W * es + (0 if head.reset is None else B * T)
     d2h = B * T * W * es
+    gpu_launches = args.steps * binding.prefill_launches(head.dims)
+
+    cpu = None
+    if cpu_on:
+        rate, desc, cores, secs = oracle_prefill_rate(head.prob, target_s=args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc,
+               "seconds": round(secs, 2)}
+        head_entry["cpu_baseline"] = cpu
+    configs = {wl.name: head_entry}
+    del head
+    gc.collect()
+    torch.cuda.empty_cache()
+
+    # ---- every other prefill workload, timed for about CONFIG_SECONDS each ----
+    if not args.headline_only:
+        for name in PREFILL_WORKLOADS:
+            if name == wl.name:
+                continue
+            rig = PrefillRig(binding, inputs.WORKLOADS[name], dev)
+            flush = algorithmic_bytes(rig.wl, rig.wl.batch * rig.wl.seq_len) <= 126e6
+            # a short probe sizes the timed run (same launch configuration)
+            _, probe, _ = time_prefill(rig, 3, 3, flush, dev, dd, world, clocks_gpu)
+            n = steps_for(statistics.mean(probe), CONFIG_SECONDS)
+            tot, per, ck = time_prefill(rig, n, 3, flush, dev, dd, world, clocks_gpu)
+            entry = prefill_entry(rig, tot, per, n, world, ck)
+            if cpu_on:
+                r, d, c, sec = oracle_prefill_rate(rig.prob, target_s=args.config_cpu_seconds)
+                entry["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": c, "kind": "oracle",
+                                         "sample": d, "seconds": round(sec, 2)}
+            configs[name] = entry
+            del rig
+            gc.collect()
+            torch.cuda.empty_cache()
 
     # ---- decode workload: 1024 single-token steps replayed from one CUDA graph ----
-    decode = None
     if not args.no_decode:
-        decode = bench_decode(args, dev)
+        configs[DECODE_WORKLOAD] = bench_decode(args, dev, cpu_on)
 
-    # ---- backward pass of the same prefill workload (portable kernels) ----
+    # ---- backward pass of the RecurrentGemma-2B-shaped prefill ----
     backward = None
     if not args.no_backward:
         try:
@@ -337,53 +438,22 @@ def run_ours(args):
         except Exception as exc:  # the prefill line above is the contract; report, do not lose it
             backward = {"error": f"{type(exc).__name__}: {exc}"}
 
-    # ---- CPU oracle on a bounded sample (rank 0, N = 1 only) ----
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
-        rate, desc, cores, secs = oracle_prefill_rate(prob, target_s=args.cpu_seconds)
-        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": desc,
-               "seconds": round(secs, 2)}
-        # the same oracle on one core, on this workload and on the tiny fp32 one
-        single = {}
-        for name, pr in ((wl.name, prob),
-                         ("tiny_f32", inputs.make_problem(inputs.WORKLOADS["tiny_f32"], seed=0))):
-            r1, d1, _, s1 = oracle_prefill_rate(pr, target_s=min(3.0, args.cpu_seconds), threads=1)
-            single[name] = {"value": r1, "unit": "tokens/s", "sample": d1, "seconds": round(s1, 2)}
-        cpu["single_thread"] = single
-
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
-    clk = clocks.summary()
+    cfg = workload_config(wl, world)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": wl.name, "batch": B, "seq_len": T, "heads": wl.heads,
-                   "head_dim": wl.head_dim, "width": W, "state": "fp32, read and written back",
-                   "l2": "inputs larger than L2 (252 MB moved per step > 126 MB L2)",
-                   "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": alg,
-                     "frac_of_8TBs": achieved / 8000.0, "kernel_source": os.path.basename(src)},
-        "cpu_baseline": cpu,
+        "data": "synthetic", "config": cfg, "roofline": roofline, "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * launches_per_prefill(dims),
-        "clocks": clk,
-        "decode": decode,
-        "backward": backward,
+        "gpu_launches": gpu_launches, "clocks": clk, "configs": configs, "backward": backward,
     }
     print(json.dumps(line), flush=True)
-
-
-def launches_per_prefill(dims) -> int:
-    from gated_linear_recurrence_conv1d_b200 import binding
-    return binding.prefill_launches(dims)
 
 
 def e2e_pipelined(binding, block, x, y, h, tail, reset, B, T, steps, dev, dist=None, groups=4):
@@ -454,7 +524,28 @@ def e2e_pipelined(binding, block, x, y, h, tail, reset, B, T, steps, dev, dist=N
     return max_over_ranks(ms, dist, dev)
 
 
-def bench_decode(args, dev):
+def oracle_decode_rate(prob: inputs.Problem, target_s: float = 3.0):
+    """Times the fp64 oracle's decode on the host cores: successive single-token steps of the
+    decode workload from its initial state, for about target_s.  Returns (tokens/s, description,
+    cores, seconds)."""
+    import oracle
+    wl = prob.wl
+    cores = len(os.sched_getaffinity(0))
+    h = prob.h0.astype(np.float64).copy()
+    tail = oracle.tail_from_act(prob.tail0).copy()
+    done = 0
+    t0 = time.perf_counter()
+    while done < wl.decode_steps:
+        oracle.decode(prob.params, prob.x[done], prob.y[done], wl.heads, h, tail, threads=cores)
+        done += 1
+        if time.perf_counter() - t0 >= target_s:
+            break
+    dt = time.perf_counter() - t0
+    desc = f"first {done} of {wl.decode_steps} steps x batch {wl.batch} x all {wl.heads} heads of {wl.name}"
+    return wl.batch * done / dt, desc, cores, dt
+
+
+def bench_decode(args, dev, cpu_on: bool = False):
     import torch
     from gated_linear_recurrence_conv1d_b200 import binding
 
@@ -505,13 +596,19 @@ def bench_decode(args, dev):
     peak, _ = measured_peaks()
     bps = decode_bytes_per_step(wl)
     del g
-    return {"workload": wl.name, "batch": wl.batch, "width": wl.width, "steps": steps,
+    entry = {"workload": wl.name, "batch": wl.batch, "width": wl.width, "steps": steps,
             "value": tok_s, "unit": "tokens/s", "us_per_step": us_step,
             "effective_gbs": bps / (us_step * 1e-6) / 1e9,
             "effective_frac": bps / (us_step * 1e-6) / 1e9 / peak,
             "note": "state (h, conv_tail) and gate weights stay L2-resident across steps; "
                     "GB/s is algorithmic bytes over time (effective bandwidth)",
-            "gpu_launches": steps * binding.decode_launches(dims)}
+            "gpu_launches": steps * binding.decode_launches(dims),
+            "roofline_frac": bps / (us_step * 1e-6) / 1e9 / peak}
+    if cpu_on:
+        r, d, c, sec = oracle_decode_rate(prob, target_s=min(3.0, args.config_cpu_seconds))
+        entry["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": c, "kind": "oracle", "sample": d,
+                                 "seconds": round(sec, 2)}
+    return entry
 
 
 def bench_backward(args, dev, steps=3, warmup=1):
@@ -519,7 +616,7 @@ def bench_backward(args, dev, steps=3, warmup=1):
     import torch
     from gated_linear_recurrence_conv1d_b200 import binding
 
-    wl = inputs.WORKLOADS[args.workload]
+    wl = inputs.WORKLOADS["rg2b_bf16"]
     prob = inputs.make_problem(wl, seed=0)
     block = binding.RGLRUBlock(prob.params, wl.heads, wl.head_dim, wl.dtype, dev)
     x = binding.to_device(prob.x, dev)
@@ -566,13 +663,18 @@ def bench_backward(args, dev, steps=3, warmup=1):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(inputs.WORKLOADS))
-    ap.add_argument("--e2e-steps", type=int, default=50)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="oracle seconds on the headline workload")
+    ap.add_argument("--config-cpu-seconds", type=float, default=4.0,
+                    help="oracle seconds on each other workload")
     ap.add_argument("--ref-step-s", type=float, default=4.0)
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the headline workload (no per-workload entries)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode workload (prints its JSON object)")

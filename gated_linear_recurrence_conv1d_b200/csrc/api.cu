@@ -83,22 +83,53 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[RGLRU_NOALLOC_SCRATCH_
 
 constexpr int kMaxDevices = 64;
 
-// Device address of the static scratch on the current device, looked up once per device
-// (with that device current) and cached.
+// Unique id of the calling thread's current context (cuCtxGetId, reached through the runtime's
+// driver entry point so that the library needs no link against libcuda).  0 when unavailable.
+unsigned long long current_context_id() {
+    typedef int (*GetCurrentFn)(void**);
+    typedef int (*GetIdFn)(void*, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    void* ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+    return id;
+}
+
+// Device address of the static scratch in the calling thread's current context, looked up with
+// cudaGetSymbolAddress the first time a device is used and again whenever that device's
+// context has changed since (a cudaDeviceReset destroys the primary context, the module is
+// loaded anew in the next one and the area moves); cached per device with the context's
+// unique id.  Without a context id the address is looked up on every call.
 cudaError_t noalloc_scratch(void** addr) {
     static std::mutex mu;
     static void* cache[kMaxDevices] = {};
+    static unsigned long long cache_ctx[kMaxDevices] = {};
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const unsigned long long ctx = current_context_id();   // 0 before the context exists
     std::lock_guard<std::mutex> lock(mu);
-    if (!cache[dev]) {
+    if (!cache[dev] || ctx == 0 || cache_ctx[dev] != ctx) {
         void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);     // creates the context if needed
         if (e != cudaSuccess) return e;
         if (!p) return cudaErrorInvalidSymbol;
         cache[dev] = p;
+        cache_ctx[dev] = current_context_id();
     }
     *addr = cache[dev];
     return cudaSuccess;

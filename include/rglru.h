@@ -181,7 +181,10 @@ RGLRU_API rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_pa
  *     has loaded it (with CUDA's default lazy loading: from this entry point's first call on
  *     that device) until the process exits;
  *   - the first call on each device looks up the area's device address (with that device
- *     current), so make that first call before any stream capture;
+ *     current), so make that first call before any stream capture; the lookup is repeated
+ *     when the device's context has changed since (after a cudaDeviceReset the area is
+ *     reloaded at another address), so the first call after such a reset must also come
+ *     before any capture;
  *   - all calls share the one area and it keeps the previous call's contents; each call
  *     clears what must start at zero (its status word and the kernel's tickets and flags);
  *     two calls that overlap on the GPU (different streams, or concurrent host threads) race
@@ -190,6 +193,8 @@ RGLRU_API rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_pa
  * the kernel the device status word (code, where, info0, info1 as 32-bit words) is copied
  * into it in stream order, so that a device-side TIMEOUT / DEVICE condition can be read
  * (rglru_read_device_status decodes it when the buffer is 256-byte aligned).
+ * Besides what rglru_prefill_plan counts for rglru_block_prefill, each call enqueues one
+ * more memset (its status word) and, when status_out is given, one device-to-device copy.
  * Nothing here calls cudaMalloc, cudaFree or any allocating routine.
  * Errors: as rglru_block_prefill (INVALID_ARG, UNSUPPORTED, CUDA), and WORKSPACE when the
  * problem does not fit the static area. */

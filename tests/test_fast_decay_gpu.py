@@ -1,0 +1,75 @@
+"""Fast-decaying channels on the tensor-core kernels.
+
+The default workloads draw Lambda so that a^c lies in [0.9, 0.999] (the pages'
+initialisation, "Griffin Guide: RecurrentGemma, RG-LRU & Hybrid Attention", "1. Formulation
+of the RG-LRU Gating Mechanism"), which keeps |c log sigma(Lambda)| below 1/8: the range where
+the kernels evaluate expm1 of the log-decay by its series.  Trained layers also have channels
+that decay fast.  Here a^c is drawn from [1e-4, 0.999] and every 16th channel gets
+Lambda in [-3, -0.5] (sigma(Lambda) < 1/2), so that the kernels' other branch (the exponential
+itself) runs on full 32-token chunks, on a ragged last chunk, across resets and from a carried
+state, in the prefill and in the decode step, against the oracle on the same bytes.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_linear_recurrence_conv1d_b200 import binding, inputs
+from tests.gpu_util import GpuProblem, assert_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+BASE = inputs.WORKLOADS
+
+
+def _fast_decay(prob, seed):
+    rng = np.random.default_rng(seed)
+    lam = prob.params["lam"].copy()
+    idx = np.arange(0, lam.size, 16)
+    lam[idx] = rng.uniform(-3.0, -0.5, idx.size).astype(np.float32)
+    prob.params["lam"] = lam
+    sig = 1.0 / (1.0 + np.exp(-lam.astype(np.float64)))
+    c_log = 8.0 * np.log(sig)
+    assert (c_log < -0.125).mean() > 0.3 and (lam < 0).sum() >= idx.size   # both branches present
+    return prob
+
+
+@pytest.mark.parametrize("T,resets", [(32 * 5, False), (32 * 5 + 7, True), (1000, True)])
+def test_prefill_fast_decay_channels(T, resets):
+    kw = dict(batch=2, seq_len=T, heads=2, random_state=True, lam_lo=1e-4, lam_hi=0.999)
+    wl = (BASE["packed_bf16"].scaled(doc_len=(5, 120), **kw) if resets
+          else BASE["rg2b_bf16"].scaled(**kw))
+    prob = _fast_decay(inputs.make_problem(wl, seed=T), seed=T)
+    gp = GpuProblem(prob)
+    assert binding.prefill_plan(gp.block.dims(2, T))[0] == 1       # the tensor-core kernel
+    out, h, tail, status = gp.prefill()
+    assert status == binding.RGLRU_OK
+    ref, ref_h, ref_tail = oracle.prefill(prob.params, prob.x, prob.y, wl.heads, reset=prob.reset,
+                                          h0=prob.h0, tail0=prob.tail0)
+    assert_close(to_np(out), ref, "bf16", "fast-decay prefill out")
+    assert_close(to_np(h), ref_h, "bf16", "fast-decay prefill h")
+    np.testing.assert_array_equal(to_np(tail), ref_tail)
+
+
+def test_decode_fast_decay_channels():
+    B, steps = 130, 5
+    wl = BASE["decode_bf16"].scaled(batch=B, heads=2, decode_steps=steps, lam_lo=1e-4, lam_hi=0.999)
+    prob = _fast_decay(inputs.make_problem(wl, seed=51), seed=51)
+    gp = GpuProblem(prob)
+    h, tail = gp.new_state(B)
+    dims = gp.block.dims(B, 1)
+    assert binding.decode_plan(dims)[0] == 1
+    ws = binding.alloc_workspace(binding.decode_workspace_size(dims))
+    h_ref = prob.h0.astype(np.float64).copy()
+    t_ref = oracle.tail_from_act(prob.tail0).copy()
+    for s in range(steps):
+        rst_np = (np.arange(B) % 4 == s % 4).astype(np.uint8)
+        out = torch.empty_like(gp.x[s])
+        binding.block_decode(dims, gp.block.params, gp.x[s], gp.y[s], out, h, tail, ws,
+                             reset=binding.to_device(rst_np))
+        ref = oracle.decode(prob.params, prob.x[s], prob.y[s], wl.heads, h_ref, t_ref, reset=rst_np)
+        assert_close(to_np(out), ref, "bf16", f"fast-decay decode step {s}")
+        np.testing.assert_array_equal(to_np(tail), t_ref)
+    assert binding.read_device_status(ws) == binding.RGLRU_OK
+    assert_close(to_np(h), h_ref, "bf16", "fast-decay decode h")
