@@ -23,7 +23,7 @@ _SRC = os.path.join(_HERE, "rglru_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "librglru_oracle.so")
 _lib = None
 
-F32, BF16 = 0, 1
+F32, BF16, F64 = 0, 1, 2
 HIST = 3  # conv width 4 -> 3 past inputs
 
 
@@ -117,6 +117,67 @@ def prefill(params: dict, x: np.ndarray, y: np.ndarray, heads: int,
     if rc != 0:
         raise RuntimeError("oracle prefill failed")
     return out, h, tail
+
+
+def layer(params: dict, proj: dict, u: np.ndarray, heads: int, reset: Optional[np.ndarray] = None,
+          h0: Optional[np.ndarray] = None, tail0: Optional[np.ndarray] = None, c: float = 8.0,
+          gelu_tanh: int = 0, units: Optional[Sequence] = None):
+    """The block with its projections ("Griffin Guide: RecurrentGemma, RG-LRU & Hybrid
+    Attention", listing RecurrentBlock.forward: proj_in_1 / proj_in_2 before the branches,
+    proj_out after the merge; RecurrentGemma's linear_x / linear_y / linear_out):
+
+        x = u W_in_x,  y = u W_in_y,  z = block(x, y),  out = z W_out
+
+    all in fp64 from the exact input values (u [B, T, D] and the weights w_in_x, w_in_y [D, W],
+    w_out [W, D] of ``proj`` in the act dtype); the block is this oracle's prefill of x, y as
+    fp64 inputs.  Returns (out [B, T, D], h [B, W], tail [B, 3, W], z [B, T, W]), fp64.
+    ``units`` = list of (b, head) sequences to run (the others leave z at 0)."""
+    lib = _load()
+    u64 = as_f64(u)
+    wx, wy, wo = as_f64(proj["w_in_x"]), as_f64(proj["w_in_y"]), as_f64(proj["w_out"])
+    B, T, D = u64.shape
+    W = wx.shape[1]
+    dh = W // heads
+    x = np.ascontiguousarray(np.matmul(u64, wx))
+    y = np.ascontiguousarray(np.matmul(u64, wy))
+    w_a, dtw = _act(params["w_a"])
+    w_x, _ = _act(params["w_x"])
+    wes = 4 if dtw == F32 else 2
+    conv_w = _f32(params["conv_w"])
+    conv_b, b_a, b_x, lam = (_f32(params.get(k)) for k in ("conv_b", "b_a", "b_x", "lam"))
+    h = np.zeros((B, W)) if h0 is None else np.array(h0, dtype=np.float64, copy=True)
+    tail = np.zeros((B, HIST, W)) if tail0 is None else tail_from_act(tail0).copy()
+    z = np.zeros((B, T, W))
+    base = lambda arr, off, size: ctypes.c_void_p(arr.ctypes.data + off * size)  # noqa: E731
+    todo = units if units is not None else [(b, hd) for b in range(B) for hd in range(heads)]
+    for b, hd in todo:
+        ch0 = hd * dh
+        hb = np.ascontiguousarray(h[b, ch0:ch0 + dh])
+        tb = np.ascontiguousarray(tail[b][:, ch0:ch0 + dh])
+        zb = np.zeros((T, dh))
+        rst = None if reset is None else np.ascontiguousarray(reset[b], dtype=np.uint8)
+        rc = lib.rglru_oracle_prefill_unit(
+            T, dh, c, gelu_tanh, F64, base(conv_w, ch0, 4), W,
+            None if conv_b is None else base(conv_b, ch0, 4),
+            base(w_a, hd * dh * dh, wes), base(w_x, hd * dh * dh, wes), dtw,
+            None if b_a is None else base(b_a, ch0, 4), None if b_x is None else base(b_x, ch0, 4),
+            base(lam, ch0, 4), base(x, b * T * W + ch0, 8), base(y, b * T * W + ch0, 8), W,
+            _p(rst), _p(hb), _p(tb), dh, _p(zb), dh, None)
+        if rc != 0:
+            raise RuntimeError("oracle layer: prefill_unit failed")
+        z[b, :, ch0:ch0 + dh] = zb
+        h[b, ch0:ch0 + dh] = hb
+        tail[b][:, ch0:ch0 + dh] = tb
+    out = np.matmul(z, wo)
+    return out, h, tail, z
+
+
+def as_f64(a: np.ndarray) -> np.ndarray:
+    """Exact fp64 copy of an act-dtype array (bf16 bits widened)."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray((a.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    return np.ascontiguousarray(a, dtype=np.float64)
 
 
 def prefill_unit_decay(params: dict, x: np.ndarray, y: np.ndarray, heads: int, b: int, head: int,

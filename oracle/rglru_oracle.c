@@ -57,9 +57,12 @@
 #define ORACLE_CONV_WIDTH 4   /* [C]: "small temporal kernel width of k = 4" */
 #define ORACLE_HIST (ORACLE_CONV_WIDTH - 1)
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_F64 = 2 };
 
+/* Exact fp64 value of element idx: fp32, bf16 bits, or (for the layer oracle, whose projections
+ * produce fp64 activations) fp64 as is. */
 static double widen(const void* p, long idx, int dtype) {
+    if (dtype == ORACLE_F64) return ((const double*)p)[idx];
     if (dtype == ORACLE_F32) return (double)((const float*)p)[idx];
     uint32_t bits = ((uint32_t)((const uint16_t*)p)[idx]) << 16;
     float f;
