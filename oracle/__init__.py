@@ -119,9 +119,17 @@ def prefill(params: dict, x: np.ndarray, y: np.ndarray, heads: int,
     return out, h, tail
 
 
+def round_bf16(a: np.ndarray) -> np.ndarray:
+    """fp64 -> the nearest bf16 value (ties to even), returned as fp64: 8 significant bits by
+    frexp / rint, exact for the normal range (no detour through fp32, so no double rounding)."""
+    a = np.asarray(a, dtype=np.float64)
+    m, e = np.frexp(a)                       # a = m 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+
+
 def layer(params: dict, proj: dict, u: np.ndarray, heads: int, reset: Optional[np.ndarray] = None,
           h0: Optional[np.ndarray] = None, tail0: Optional[np.ndarray] = None, c: float = 8.0,
-          gelu_tanh: int = 0, units: Optional[Sequence] = None):
+          gelu_tanh: int = 0, units: Optional[Sequence] = None, act_interface: bool = False):
     """The block with its projections ("Griffin Guide: RecurrentGemma, RG-LRU & Hybrid
     Attention", listing RecurrentBlock.forward: proj_in_1 / proj_in_2 before the branches,
     proj_out after the merge; RecurrentGemma's linear_x / linear_y / linear_out):
@@ -131,7 +139,12 @@ def layer(params: dict, proj: dict, u: np.ndarray, heads: int, reset: Optional[n
     all in fp64 from the exact input values (u [B, T, D] and the weights w_in_x, w_in_y [D, W],
     w_out [W, D] of ``proj`` in the act dtype); the block is this oracle's prefill of x, y as
     fp64 inputs.  Returns (out [B, T, D], h [B, W], tail [B, 3, W], z [B, T, W]), fp64.
-    ``units`` = list of (b, head) sequences to run (the others leave z at 0)."""
+    ``units`` = list of (b, head) sequences to run (the others leave z at 0).
+
+    act_interface: the three steps meet at the block's interface, whose activations are bf16
+    tensors (the block takes x and y and returns z in the activation dtype): x, y and z are
+    rounded to bf16 (nearest, ties to even) where they cross it, everything else stays fp64.
+    The conv history the block keeps is then the bf16 x it was given."""
     lib = _load()
     u64 = as_f64(u)
     wx, wy, wo = as_f64(proj["w_in_x"]), as_f64(proj["w_in_y"]), as_f64(proj["w_out"])
@@ -140,6 +153,8 @@ def layer(params: dict, proj: dict, u: np.ndarray, heads: int, reset: Optional[n
     dh = W // heads
     x = np.ascontiguousarray(np.matmul(u64, wx))
     y = np.ascontiguousarray(np.matmul(u64, wy))
+    if act_interface:
+        x, y = np.ascontiguousarray(round_bf16(x)), np.ascontiguousarray(round_bf16(y))
     w_a, dtw = _act(params["w_a"])
     w_x, _ = _act(params["w_x"])
     wes = 4 if dtw == F32 else 2
@@ -168,7 +183,7 @@ def layer(params: dict, proj: dict, u: np.ndarray, heads: int, reset: Optional[n
         z[b, :, ch0:ch0 + dh] = zb
         h[b, ch0:ch0 + dh] = hb
         tail[b][:, ch0:ch0 + dh] = tb
-    out = np.matmul(z, wo)
+    out = np.matmul(round_bf16(z) if act_interface else z, wo)
     return out, h, tail, z
 
 

@@ -11,6 +11,7 @@ a planted transposition is caught.
 import os
 
 import numpy as np
+import torch
 import pytest
 
 import oracle
@@ -87,3 +88,15 @@ def test_transposed_projection_is_caught():
     ns["_lib"] = oracle._load()
     with pytest.raises(AssertionError):
         _check_layer(ns["layer"], 32)
+
+
+def test_round_bf16_is_nearest_even_bf16():
+    """The layer oracle's interface rounding: torch's fp32 -> bf16 conversion (round to nearest
+    even) on fp32-representable values over 12 decades, and the ties at 1 + 2^-8 (to 1) and
+    1 + 3 2^-8 (to 1 + 2^-6)."""
+    rng = np.random.default_rng(0)
+    a = (rng.standard_normal(100000) * 10.0 ** rng.uniform(-6, 6, 100000)).astype(np.float32)
+    want = torch.from_numpy(a).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(oracle.round_bf16(a.astype(np.float64)), want)
+    ties = oracle.round_bf16(np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8)]))
+    np.testing.assert_array_equal(ties, [1.0, 1 + 2.0 ** -6, -1.0])
