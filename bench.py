@@ -438,6 +438,16 @@ def run_ours(args):
         except Exception as exc:  # the prefill line above is the contract; report, do not lose it
             backward = {"error": f"{type(exc).__name__}: {exc}"}
 
+    extras = {}
+    if not args.no_extras:
+        for name, fn in (("layer", bench_layer), ("mqa", bench_mqa)):
+            try:
+                extras[name] = fn(args, dev)
+            except Exception as exc:  # the headline line is the contract; report, do not lose it
+                extras[name] = {"error": f"{type(exc).__name__}: {exc}"}
+            gc.collect()
+            torch.cuda.empty_cache()
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -452,6 +462,7 @@ def run_ours(args):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": gpu_launches, "clocks": clk, "configs": configs, "backward": backward,
+        "layer": extras.get("layer"), "mqa": extras.get("mqa"),
     }
     print(json.dumps(line), flush=True)
 
@@ -596,14 +607,45 @@ def bench_decode(args, dev, cpu_on: bool = False):
     peak, _ = measured_peaks()
     bps = decode_bytes_per_step(wl)
     del g
+    single = {"value": tok_s, "unit": "tokens/s", "us_per_step": us_step,
+              "effective_gbs": bps / (us_step * 1e-6) / 1e9,
+              "effective_frac": bps / (us_step * 1e-6) / 1e9 / peak,
+              "note": "one rglru_block_decode launch per step, 1024 steps replayed from one CUDA "
+                      "graph; state (h, conv_tail) and gate weights stay L2-resident across steps; "
+                      "GB/s is algorithmic bytes (26 B per row-channel per step) over time",
+              "gpu_launches": steps * binding.decode_launches(dims)}
+
+    # the same steps in one persistent launch (rglru_block_decode_steps): the state stays on chip
+    wss = binding.alloc_workspace(binding.decode_steps_workspace_size(dims, steps), dev)
+    ptimes = []
+    for rep in range(4):
+        h.copy_(h0)
+        tail.copy_(t0)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        binding.block_decode_steps(dims, block.params, xs, ys, outs, h, tail, wss, stream=s)
+        e1.record(s)
+        torch.cuda.synchronize()
+        if rep > 0:
+            ptimes.append(e0.elapsed_time(e1))
+    if binding.read_device_status(wss) != binding.RGLRU_OK:
+        raise RuntimeError("persistent decode: device status not OK")
+    pms = statistics.median(ptimes)
+    pus = 1000.0 * pms / steps
+    W = wl.width
+    # algorithmic bytes of the whole launch: x, y, out per step; the state read and written
+    # once; gate weights and parameters once
+    p_alg = steps * wl.batch * W * 6 + wl.batch * W * (8 + 12) + 2 * wl.heads * 256 * 256 * 2 + 8 * W * 4
+    p_gbs = p_alg / (pms * 1e-3) / 1e9
+    kind, launches = binding.decode_steps_plan(dims, steps)
     entry = {"workload": wl.name, "batch": wl.batch, "width": wl.width, "steps": steps,
-            "value": tok_s, "unit": "tokens/s", "us_per_step": us_step,
-            "effective_gbs": bps / (us_step * 1e-6) / 1e9,
-            "effective_frac": bps / (us_step * 1e-6) / 1e9 / peak,
-            "note": "state (h, conv_tail) and gate weights stay L2-resident across steps; "
-                    "GB/s is algorithmic bytes over time (effective bandwidth)",
-            "gpu_launches": steps * binding.decode_launches(dims),
-            "roofline_frac": bps / (us_step * 1e-6) / 1e9 / peak}
+             "value": wl.batch * steps / (pms / 1000.0), "unit": "tokens/s", "us_per_step": pus,
+             "path": "rglru_block_decode_steps: all steps in one persistent launch",
+             "algorithmic_bytes_per_launch": p_alg, "achieved_gbs": p_gbs, "roofline_frac": p_gbs / peak,
+             "peak_gbs": peak, "kernel": "tensor" if kind == 1 else "generic",
+             "gpu_launches": launches, "single_step": single}
     if cpu_on:
         r, d, c, sec = oracle_decode_rate(prob, target_s=min(3.0, args.config_cpu_seconds))
         entry["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": c, "kind": "oracle", "sample": d,
@@ -650,7 +692,8 @@ def bench_backward(args, dev, steps=3, warmup=1):
     alg = B * T * W * (3 * es + 8) + 2 * H * dh * dh * (es + 4)
     peak, _ = measured_peaks()
     line = {"workload": wl.name, "value": B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
-            "steps": steps, "kernels": "portable CUDA-core kernels, fp32 arithmetic",
+            "steps": steps,
+            "kernels": "tensor-core path" if binding.backward_plan(dims)[0] == 1 else "portable kernels",
             "effective_gbs": alg / (ms * 1e-3) / 1e9, "effective_frac": alg / (ms * 1e-3) / 1e9 / peak,
             "gpu_launches": steps * binding.backward_launches(dims)}
     if not args.no_cpu:
@@ -658,6 +701,136 @@ def bench_backward(args, dev, steps=3, warmup=1):
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                 "sample": desc, "seconds": round(secs, 2)}
     return line
+
+
+def bench_layer(args, dev, steps=10):
+    """rglru_layer_forward on the RecurrentGemma-2B-shaped batch with model width 2560: the three
+    projections (tensor-core GEMMs) around the block, against the same computation with torch
+    matmuls (cuBLAS) around rglru_block_prefill."""
+    import torch
+    from gated_linear_recurrence_conv1d_b200 import binding
+
+    wl = inputs.WORKLOADS["rg2b_bf16"]
+    D = 2560
+    prob = inputs.make_problem(wl, seed=0)
+    rng = np.random.default_rng(2)
+    B, T, W = wl.batch, wl.seq_len, wl.width
+    block = binding.RGLRUBlock(prob.params, wl.heads, wl.head_dim, wl.dtype, dev)
+    u = torch.randn(B, T, D, device=dev).to(torch.bfloat16)
+    wx = (torch.randn(D, W, device=dev) / D ** 0.5).to(torch.bfloat16)
+    wy = (torch.randn(D, W, device=dev) / D ** 0.5).to(torch.bfloat16)
+    wo = (torch.randn(W, D, device=dev) / W ** 0.5).to(torch.bfloat16)
+    del rng
+    pj = binding.make_projections(D, wx, wy, wo)
+    dims = block.dims(B, T)
+    ws = binding.alloc_workspace(binding.layer_workspace_size(dims), dev)
+    out = torch.empty(B, T, D, dtype=torch.bfloat16, device=dev)
+    h = torch.zeros(B, W, device=dev)
+    tail = torch.zeros(B, 3, W, dtype=torch.bfloat16, device=dev)
+
+    def ours():
+        binding.layer_forward(dims, block.params, pj, u, out, ws, h=h, conv_tail=tail)
+
+    wsb = binding.alloc_workspace(binding.prefill_workspace_size(dims), dev)
+    z = torch.empty(B, T, W, dtype=torch.bfloat16, device=dev)
+
+    def composed():
+        x = torch.matmul(u, wx)
+        y = torch.matmul(u, wy)
+        binding.block_prefill(dims, block.params, x, y, z, wsb, h=h, conv_tail=tail)
+        torch.matmul(z, wo)
+
+    def timeit(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    ms = timeit(ours)
+    if binding.read_device_status(ws) != binding.RGLRU_OK:
+        raise RuntimeError("layer: device status not OK")
+    ms_c = timeit(composed)
+    flops = 2.0 * B * T * D * W * 3
+    return {"workload": "rg2b_bf16 with model width 2560", "batch": B, "seq_len": T, "model_dim": D,
+            "value": B * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "projection_tflops": flops / (ms * 1e-3) / 1e12,
+            "torch_matmuls_around_block": {"value": B * T / (ms_c * 1e-3), "unit": "tokens/s", "ms_per_step": ms_c},
+            "gpu_launches": steps * binding.layer_plan(dims, pj)[1]}
+
+
+def bench_mqa(args, dev, steps=10, dsteps=32):
+    """Local sliding-window MQA, RecurrentGemma-2B-shaped: 10 query heads x 256 over one key /
+    value head, window 2048; prefill of batch 8 x 2048 tokens and decode of batch 256 against
+    full rings."""
+    import torch
+    from gated_linear_recurrence_conv1d_b200 import binding
+
+    B, T, H, d, w = 8, 2048, 10, 256, 2048
+    q = torch.randn(B, T, H, d, device=dev).to(torch.bfloat16)
+    k = torch.randn(B, T, d, device=dev).to(torch.bfloat16)
+    v = torch.randn(B, T, d, device=dev).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    dims = binding.make_mqa_dims(B, T, H, d, w)
+    ws = binding.alloc_workspace(binding.mqa_workspace_size(dims), dev)
+    for _ in range(3):
+        binding.mqa_prefill(dims, q, k, v, out, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        binding.mqa_prefill(dims, q, k, v, out, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    if binding.read_device_status(ws) != binding.RGLRU_OK:
+        raise RuntimeError("mqa prefill: device status not OK")
+    ms = e0.elapsed_time(e1) / steps
+    # score and weighted-sum flops over the causal window (every query sees min(t + 1, w) keys)
+    keys = sum(min(t + 1, w) for t in range(T))
+    flops = 4.0 * B * H * d * keys
+    peak_tf = measured_tensor_peak()
+    pre = {"workload": f"B{B} T{T} {H} query heads x {d}, window {w}", "value": B * T / (ms * 1e-3),
+           "unit": "tokens/s", "ms_per_step": ms, "tflops": flops / (ms * 1e-3) / 1e12,
+           "tensor_frac": flops / (ms * 1e-3) / 1e12 / peak_tf, "tensor_peak_tflops": peak_tf}
+    Bd = 256
+    cache = torch.randn(Bd, 2, w, d, device=dev).to(torch.bfloat16)
+    ddims = binding.make_mqa_dims(Bd, 1, H, d, w)
+    wsd = binding.alloc_workspace(binding.mqa_workspace_size(ddims, decode=True), dev)
+    qd = torch.randn(dsteps, Bd, H, d, device=dev).to(torch.bfloat16)
+    kd = torch.randn(dsteps, Bd, d, device=dev).to(torch.bfloat16)
+    vd = torch.randn(dsteps, Bd, d, device=dev).to(torch.bfloat16)
+    od = torch.empty(Bd, H, d, dtype=torch.bfloat16, device=dev)
+    pos = [torch.full((Bd,), 4096 + s, dtype=torch.int32, device=dev) for s in range(dsteps)]
+    for s in range(3):
+        binding.mqa_decode(ddims, qd[s], kd[s], vd[s], pos[s], cache, od, wsd)
+    torch.cuda.synchronize()
+    e0.record()
+    for s in range(dsteps):
+        binding.mqa_decode(ddims, qd[s], kd[s], vd[s], pos[s], cache, od, wsd)
+    e1.record()
+    torch.cuda.synchronize()
+    if binding.read_device_status(wsd) != binding.RGLRU_OK:
+        raise RuntimeError("mqa decode: device status not OK")
+    us = 1000.0 * e0.elapsed_time(e1) / dsteps
+    bytes_step = Bd * 2 * w * d * 2 + Bd * (H + 2) * d * 2 * 2
+    peak, _ = measured_peaks()
+    dec = {"workload": f"B{Bd} {H} query heads x {d}, full rings of {w}", "value": Bd / (us * 1e-6),
+           "unit": "tokens/s", "us_per_step": us, "achieved_gbs": bytes_step / (us * 1e-6) / 1e9,
+           "roofline_frac": bytes_step / (us * 1e-6) / 1e9 / peak}
+    return {"prefill": pre, "decode": dec}
+
+
+def measured_tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def main():
@@ -682,6 +855,7 @@ def main():
                     help="decode steps per graph replay (default: the workload's 1024)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the layer and MQA entries")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

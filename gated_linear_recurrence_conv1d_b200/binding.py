@@ -32,7 +32,10 @@ EXPORTED = ("rglru_state_init", "rglru_prefill_workspace_size", "rglru_block_pre
             "rglru_decode_workspace_size", "rglru_block_decode", "rglru_read_device_status",
             "rglru_status_string", "rglru_abi_version", "rglru_prefill_plan", "rglru_decode_plan",
             "rglru_block_prefill_noalloc", "rglru_last_cuda_error", "rglru_backward_workspace_size",
-            "rglru_block_backward", "rglru_backward_plan")
+            "rglru_block_backward", "rglru_backward_plan", "rglru_decode_steps_workspace_size",
+            "rglru_block_decode_steps", "rglru_decode_steps_plan", "rglru_layer_workspace_size",
+            "rglru_layer_forward", "rglru_layer_plan", "rglru_mqa_workspace_size", "rglru_mqa_prefill",
+            "rglru_mqa_decode")
 
 # Fields of rglru_grads, in order (fp32 device tensors).
 GRAD_FIELDS = ("dx", "dy", "dh0", "dtail0", "dconv_w", "dconv_b", "dw_a", "dw_x", "db_a", "db_x",
@@ -62,6 +65,17 @@ class Params(ctypes.Structure):
 
 class State(ctypes.Structure):
     _fields_ = [("h", ctypes.c_void_p), ("conv_tail", ctypes.c_void_p)]
+
+
+class Projections(ctypes.Structure):
+    _fields_ = [("model_dim", ctypes.c_int), ("w_in_x", ctypes.c_void_p), ("w_in_y", ctypes.c_void_p),
+                ("w_out", ctypes.c_void_p)]
+
+
+class MqaDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("seq_len", ctypes.c_int), ("q_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("window", ctypes.c_int), ("scale", ctypes.c_float),
+                ("rope_base", ctypes.c_float)]
 
 
 class Grads(ctypes.Structure):
@@ -117,6 +131,26 @@ def load(build_if_missing: bool = True):
     lib.rglru_backward_workspace_size.restype = S
     lib.rglru_block_backward.argtypes = [PD, PP, V, V, V, PS, V, V, V, PG, V, S, V]
     lib.rglru_block_backward.restype = I
+    lib.rglru_decode_steps_workspace_size.argtypes = [PD, I]
+    lib.rglru_decode_steps_workspace_size.restype = S
+    lib.rglru_block_decode_steps.argtypes = [PD, PP, V, V, V, I, PS, V, V, S, V]
+    lib.rglru_block_decode_steps.restype = I
+    lib.rglru_decode_steps_plan.argtypes = [PD, I, PI, PI]
+    lib.rglru_decode_steps_plan.restype = I
+    PJ = ctypes.POINTER(Projections)
+    lib.rglru_layer_workspace_size.argtypes = [PD]
+    lib.rglru_layer_workspace_size.restype = S
+    lib.rglru_layer_forward.argtypes = [PD, PP, PJ, V, V, PS, V, V, S, V]
+    lib.rglru_layer_forward.restype = I
+    lib.rglru_layer_plan.argtypes = [PD, PJ, PI, PI]
+    lib.rglru_layer_plan.restype = I
+    PM = ctypes.POINTER(MqaDims)
+    lib.rglru_mqa_workspace_size.argtypes = [PM, I]
+    lib.rglru_mqa_workspace_size.restype = S
+    lib.rglru_mqa_prefill.argtypes = [PM, V, V, V, I, V, V, V, S, V]
+    lib.rglru_mqa_prefill.restype = I
+    lib.rglru_mqa_decode.argtypes = [PM, V, V, V, V, V, V, V, S, V]
+    lib.rglru_mqa_decode.restype = I
     lib.rglru_last_cuda_error.argtypes = [ctypes.POINTER(ctypes.c_char_p)]
     lib.rglru_last_cuda_error.restype = I
     lib.rglru_abi_version.argtypes = []
@@ -226,6 +260,82 @@ def block_decode(dims: Dims, params: Params, x: torch.Tensor, y: torch.Tensor, o
                                    _ptr(reset), ctypes.byref(st), _ptr(out), _ptr(workspace),
                                    workspace.numel(), _stream(stream))
     _check(rc, "rglru_block_decode")
+
+
+def decode_steps_workspace_size(dims: Dims, steps: int) -> int:
+    return load().rglru_decode_steps_workspace_size(ctypes.byref(dims), int(steps))
+
+
+def block_decode_steps(dims: Dims, params: Params, x: torch.Tensor, y: torch.Tensor, out: torch.Tensor,
+                       h: torch.Tensor, conv_tail: torch.Tensor, workspace: torch.Tensor,
+                       reset: Optional[torch.Tensor] = None, stream=None):
+    """rglru_block_decode_steps: x, y, out [steps, B, W]; reset [steps, B] uint8 or None."""
+    steps = x.shape[0]
+    st = State(_ptr(h), _ptr(conv_tail))
+    rc = load().rglru_block_decode_steps(ctypes.byref(dims), ctypes.byref(params), _ptr(x), _ptr(y),
+                                         _ptr(reset), int(steps), ctypes.byref(st), _ptr(out),
+                                         _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "rglru_block_decode_steps")
+
+
+def decode_steps_plan(dims: Dims, steps: int):
+    k, n = ctypes.c_int(), ctypes.c_int()
+    fn = load().rglru_decode_steps_plan
+    _check(fn(ctypes.byref(dims), int(steps), ctypes.byref(k), ctypes.byref(n)), "rglru_decode_steps_plan")
+    return k.value, n.value
+
+
+def make_projections(model_dim: int, w_in_x: torch.Tensor, w_in_y: torch.Tensor, w_out: torch.Tensor) -> Projections:
+    """w_in_x, w_in_y [D, W] and w_out [W, D] device tensors in the act dtype."""
+    return Projections(int(model_dim), _ptr(w_in_x), _ptr(w_in_y), _ptr(w_out))
+
+
+def layer_workspace_size(dims: Dims) -> int:
+    return load().rglru_layer_workspace_size(ctypes.byref(dims))
+
+
+def layer_forward(dims: Dims, params: Params, proj: Projections, u: torch.Tensor, out: torch.Tensor,
+                  workspace: torch.Tensor, reset: Optional[torch.Tensor] = None,
+                  h: Optional[torch.Tensor] = None, conv_tail: Optional[torch.Tensor] = None, stream=None):
+    """rglru_layer_forward: u, out [B, T, D]."""
+    st = State(_ptr(h), _ptr(conv_tail)) if h is not None else None
+    rc = load().rglru_layer_forward(ctypes.byref(dims), ctypes.byref(params), ctypes.byref(proj), _ptr(u),
+                                    _ptr(reset), ctypes.byref(st) if st is not None else None, _ptr(out),
+                                    _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "rglru_layer_forward")
+
+
+def layer_plan(dims: Dims, proj: Projections):
+    k, n = ctypes.c_int(), ctypes.c_int()
+    _check(load().rglru_layer_plan(ctypes.byref(dims), ctypes.byref(proj), ctypes.byref(k), ctypes.byref(n)),
+           "rglru_layer_plan")
+    return k.value, n.value
+
+
+def make_mqa_dims(batch: int, seq_len: int, q_heads: int, head_dim: int, window: int, scale: Optional[float] = None,
+                  rope_base: float = 10000.0) -> MqaDims:
+    return MqaDims(batch, seq_len, q_heads, head_dim, window,
+                   (head_dim ** -0.5) if scale is None else scale, rope_base)
+
+
+def mqa_workspace_size(dims: MqaDims, decode: bool = False) -> int:
+    return load().rglru_mqa_workspace_size(ctypes.byref(dims), int(decode))
+
+
+def mqa_prefill(dims: MqaDims, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                workspace: torch.Tensor, pos0: int = 0, cache: Optional[torch.Tensor] = None, stream=None):
+    """rglru_mqa_prefill: q [B, T, H, d], k, v [B, T, d] -> out [B, T, H, d]."""
+    rc = load().rglru_mqa_prefill(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), int(pos0), _ptr(out), _ptr(cache),
+                                  _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "rglru_mqa_prefill")
+
+
+def mqa_decode(dims: MqaDims, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor,
+               cache: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor, stream=None):
+    """rglru_mqa_decode: q [B, H, d], k, v [B, d], pos [B] int32 (device) -> out [B, H, d]."""
+    rc = load().rglru_mqa_decode(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(pos), _ptr(cache), _ptr(out),
+                                 _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "rglru_mqa_decode")
 
 
 def backward_workspace_size(dims: Dims) -> int:

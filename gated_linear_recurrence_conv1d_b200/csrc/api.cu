@@ -11,6 +11,62 @@
 #include "kernels.h"
 #include "rglru.h"
 
+namespace rglru {
+
+// Unique id of the calling thread's current context (cuCtxGetId, reached through the runtime's
+// driver entry point so that the library needs no link against libcuda).  0 when unavailable.
+unsigned long long current_context_id() {
+    typedef int (*GetCurrentFn)(void**);
+    typedef int (*GetIdFn)(void*, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    void* ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
+    return id;
+}
+
+
+cudaError_t set_smem_limit(const void* kernel, int bytes) {
+    struct Entry {
+        const void* fn;
+        unsigned long long ctx;
+        int bytes;
+    };
+    static std::mutex mu;
+    static Entry done[256];
+    static int n = 0;
+    const unsigned long long ctx = current_context_id();
+    std::lock_guard<std::mutex> lock(mu);
+    if (ctx != 0)
+        for (int i = 0; i < n; ++i)
+            if (done[i].fn == kernel && done[i].ctx == ctx && done[i].bytes == bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess || ctx == 0) return e;
+    int slot = -1;
+    for (int i = 0; i < n && slot < 0; ++i)
+        if (done[i].fn == kernel) slot = i;          // a kernel keeps one entry: its latest context
+    if (slot < 0) slot = n < 256 ? n++ : 255;
+    done[slot] = Entry{kernel, ctx, bytes};
+    return cudaSuccess;
+}
+
+}  // namespace rglru
+
+using rglru::current_context_id;
+
 namespace {
 
 constexpr size_t kStatusBytes = 256;   // status word area at the start of every workspace
@@ -82,31 +138,6 @@ rglru_status cuda_status(cudaError_t e) {
 __device__ __align__(256) unsigned char g_noalloc_scratch[RGLRU_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-
-// Unique id of the calling thread's current context (cuCtxGetId, reached through the runtime's
-// driver entry point so that the library needs no link against libcuda).  0 when unavailable.
-unsigned long long current_context_id() {
-    typedef int (*GetCurrentFn)(void**);
-    typedef int (*GetIdFn)(void*, unsigned long long*);
-    static GetCurrentFn get_current = nullptr;
-    static GetIdFn get_id = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_current = reinterpret_cast<GetCurrentFn>(p);
-        p = nullptr;
-        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_id = reinterpret_cast<GetIdFn>(p);
-    });
-    void* ctx = nullptr;
-    unsigned long long id = 0;
-    if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx || get_id(ctx, &id) != 0) return 0;
-    return id;
-}
 
 // Device address of the static scratch in the calling thread's current context, looked up with
 // cudaGetSymbolAddress the first time a device is used and again whenever that device's
@@ -216,8 +247,132 @@ rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_params* para
     return cuda_status(rglru::launch_decode_generic(dims, params, x, y, reset, state, out, s));
 }
 
+size_t rglru_decode_steps_workspace_size(const rglru_dims* dims, int steps) {
+    if (check_dims(dims, false) != RGLRU_OK || steps <= 0) return 0;
+    return kStatusBytes;
+}
+
+rglru_status rglru_block_decode_steps(const rglru_dims* dims, const rglru_params* params, const void* x,
+                                      const void* y, const uint8_t* reset, int steps, rglru_state* state,
+                                      void* out, void* workspace, size_t workspace_bytes, void* stream) {
+    rglru_status st = check_dims(dims, false);
+    if (st != RGLRU_OK) return st;
+    if (steps <= 0) return RGLRU_ERR_INVALID_ARG;
+    if ((long long)steps * dims->batch * dims->heads * dims->head_dim > (1LL << 40)) return RGLRU_ERR_UNSUPPORTED;
+    if ((st = check_params(params)) != RGLRU_OK) return st;
+    if ((st = check_io(x, y, out)) != RGLRU_OK) return st;
+    if ((st = check_state(state)) != RGLRU_OK) return st;
+    if ((st = check_workspace(workspace, workspace_bytes, rglru_decode_steps_workspace_size(dims, steps))) != RGLRU_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the persistent kernel keeps h in registers and moves it with 16-byte vectors
+    if (rglru::fused_decode_steps_supported(dims) && aligned(state->h, 16))
+        return cuda_status(rglru::launch_fused_decode_steps(dims, params, x, y, reset, steps, state, out, workspace,
+                                                            workspace_bytes, s));
+    // other shapes: one portable step after another, in stream order
+    const size_t step_elems = (size_t)dims->batch * dims->heads * dims->head_dim;
+    const size_t es = act_size(dims->act_dtype);
+    for (int k = 0; k < steps; ++k) {
+        const size_t off = (size_t)k * step_elems * es;
+        cudaError_t e = rglru::launch_decode_generic(
+            dims, params, static_cast<const char*>(x) + off, static_cast<const char*>(y) + off,
+            reset ? reset + (size_t)k * dims->batch : nullptr, state, static_cast<char*>(out) + off, s);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    return RGLRU_OK;
+}
+
+rglru_status rglru_decode_steps_plan(const rglru_dims* dims, int steps, int* kernel, int* launches) {
+    rglru_status st = check_dims(dims, false);
+    if (st != RGLRU_OK) return st;
+    if (steps <= 0 || !kernel || !launches) return RGLRU_ERR_INVALID_ARG;
+    const bool tc = rglru::fused_decode_steps_supported(dims);
+    *kernel = tc ? RGLRU_KERNEL_TENSOR : RGLRU_KERNEL_GENERIC;
+    *launches = tc ? 1 : steps;
+    return RGLRU_OK;
+}
+
+size_t rglru_layer_workspace_size(const rglru_dims* dims) {
+    if (check_dims(dims, true) != RGLRU_OK) return 0;
+    return rglru::layer_workspace(dims);
+}
+
+rglru_status rglru_layer_forward(const rglru_dims* dims, const rglru_params* params, const rglru_projections* proj,
+                                 const void* u, const uint8_t* reset, rglru_state* state, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    rglru_status st = check_dims(dims, true);
+    if (st != RGLRU_OK) return st;
+    if ((st = check_params(params)) != RGLRU_OK) return st;
+    if (!proj || !proj->w_in_x || !proj->w_in_y || !proj->w_out) return RGLRU_ERR_INVALID_ARG;
+    if (!aligned(proj->w_in_x, 16) || !aligned(proj->w_in_y, 16) || !aligned(proj->w_out, 16))
+        return RGLRU_ERR_INVALID_ARG;
+    if (proj->model_dim <= 0) return RGLRU_ERR_INVALID_ARG;
+    if (!u || !out || !aligned(u, 16) || !aligned(out, 16) || u == out) return RGLRU_ERR_INVALID_ARG;
+    if (state && (st = check_state(state)) != RGLRU_OK) return st;
+    if (!rglru::layer_supported(dims, proj->model_dim)) return RGLRU_ERR_UNSUPPORTED;
+    if ((long long)dims->batch * dims->seq_len * proj->model_dim > (1LL << 40)) return RGLRU_ERR_UNSUPPORTED;
+    if ((st = check_workspace(workspace, workspace_bytes, rglru_layer_workspace_size(dims))) != RGLRU_OK) return st;
+    return cuda_status(rglru::launch_layer(dims, params, proj->model_dim, proj->w_in_x, proj->w_in_y, proj->w_out, u,
+                                           reset, state, out, workspace, workspace_bytes,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+rglru_status rglru_layer_plan(const rglru_dims* dims, const rglru_projections* proj, int* kernel, int* launches) {
+    rglru_status st = check_dims(dims, true);
+    if (st != RGLRU_OK) return st;
+    if (!proj || !kernel || !launches) return RGLRU_ERR_INVALID_ARG;
+    if (!rglru::layer_supported(dims, proj->model_dim)) return RGLRU_ERR_UNSUPPORTED;
+    *kernel = RGLRU_KERNEL_TENSOR;
+    *launches = rglru::layer_launches(dims);
+    return RGLRU_OK;
+}
+
+static rglru_status check_mqa(const rglru_mqa_dims* d, bool decode) {
+    if (!d || d->batch <= 0 || d->q_heads <= 0 || d->head_dim <= 0 || d->window <= 0) return RGLRU_ERR_INVALID_ARG;
+    if (!decode && d->seq_len <= 0) return RGLRU_ERR_INVALID_ARG;
+    if (!(d->scale == d->scale) || !(d->rope_base > 0.0f)) return RGLRU_ERR_INVALID_ARG;
+    if (!rglru::mqa_supported(d)) return RGLRU_ERR_UNSUPPORTED;
+    if (!decode && (long long)d->batch * d->seq_len * d->q_heads * d->head_dim > (1LL << 40)) return RGLRU_ERR_UNSUPPORTED;
+    if (d->batch > (1 << 16) || (!decode && d->seq_len > (1 << 30))) return RGLRU_ERR_UNSUPPORTED;
+    return RGLRU_OK;
+}
+
+size_t rglru_mqa_workspace_size(const rglru_mqa_dims* dims, int decode) {
+    if (check_mqa(dims, decode != 0) != RGLRU_OK) return 0;
+    return rglru::mqa_workspace(dims, decode != 0);
+}
+
+rglru_status rglru_mqa_prefill(const rglru_mqa_dims* dims, const void* q, const void* k, const void* v, int pos0,
+                               void* out, void* cache, void* workspace, size_t workspace_bytes, void* stream) {
+    rglru_status st = check_mqa(dims, false);
+    if (st != RGLRU_OK) return st;
+    if (!q || !k || !v || !out || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+        return RGLRU_ERR_INVALID_ARG;
+    if (out == q || out == k || out == v || pos0 < 0) return RGLRU_ERR_INVALID_ARG;
+    if (cache && !aligned(cache, 16)) return RGLRU_ERR_INVALID_ARG;
+    if ((st = check_workspace(workspace, workspace_bytes, rglru_mqa_workspace_size(dims, 0))) != RGLRU_OK) return st;
+    return cuda_status(rglru::launch_mqa_prefill(dims, q, k, v, pos0, out, cache, workspace, workspace_bytes,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+rglru_status rglru_mqa_decode(const rglru_mqa_dims* dims, const void* q, const void* k, const void* v,
+                              const int* pos, void* cache, void* out, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    rglru_status st = check_mqa(dims, true);
+    if (st != RGLRU_OK) return st;
+    if (!q || !k || !v || !out || !pos || !cache) return RGLRU_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(cache, 16) ||
+        !aligned(pos, 4))
+        return RGLRU_ERR_INVALID_ARG;
+    if (out == q || out == k || out == v) return RGLRU_ERR_INVALID_ARG;
+    if ((st = check_workspace(workspace, workspace_bytes, rglru_mqa_workspace_size(dims, 1))) != RGLRU_OK) return st;
+    return cuda_status(rglru::launch_mqa_decode(dims, q, k, v, pos, cache, out, workspace, workspace_bytes,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
 size_t rglru_backward_workspace_size(const rglru_dims* dims) {
     if (check_dims(dims, true) != RGLRU_OK) return 0;
+    if (rglru::backward_tc_supported(dims)) return rglru::backward_tc_workspace(dims);
     return rglru::backward_workspace(dims);
 }
 
@@ -244,6 +399,10 @@ rglru_status rglru_block_backward(const rglru_dims* dims, const rglru_params* pa
     }
     if ((st = check_workspace(workspace, workspace_bytes, rglru_backward_workspace_size(dims))) != RGLRU_OK)
         return st;
+    if (rglru::backward_tc_supported(dims))
+        return cuda_status(rglru::launch_backward_tc(dims, params, x, y, reset, state0, dout, dh_final, dtail_final,
+                                                     grads, workspace, workspace_bytes,
+                                                     static_cast<cudaStream_t>(stream)));
     return cuda_status(rglru::launch_backward(dims, params, x, y, reset, state0, dout, dh_final, dtail_final,
                                               grads, workspace, workspace_bytes,
                                               static_cast<cudaStream_t>(stream)));
@@ -303,8 +462,9 @@ rglru_status rglru_backward_plan(const rglru_dims* dims, int* kernel, int* launc
     rglru_status st = check_dims(dims, true);
     if (st != RGLRU_OK) return st;
     if (!kernel || !launches) return RGLRU_ERR_INVALID_ARG;
-    *kernel = RGLRU_KERNEL_GENERIC;
-    *launches = rglru::backward_launches(dims);
+    const bool tc = rglru::backward_tc_supported(dims);
+    *kernel = tc ? RGLRU_KERNEL_TENSOR : RGLRU_KERNEL_GENERIC;
+    *launches = tc ? rglru::backward_tc_launches(dims) : rglru::backward_launches(dims);
     return RGLRU_OK;
 }
 

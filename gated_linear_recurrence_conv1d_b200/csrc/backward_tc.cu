@@ -1,0 +1,419 @@
+// backward_tc.cu -- gradients of the RG-LRU block for bf16 activations, head_dim 256, with the
+// dense contractions on the tensor cores (sm_100a).
+//
+// The gradients are those of backward.cu (the chain rule through the forward the pages define,
+// "Griffin Guide: RecurrentGemma, RG-LRU & Hybrid Attention": "1. Formulation of the RG-LRU
+// Gating Mechanism", "2. The Role of Square-Root Variance Normalization", "1. Temporal Filtering
+// via Separable 1D Convolutions", "2. Non-Linear Multiplicative Gating with GeLU", "3.
+// Block-Diagonal Sharding ..."), computed in six launches:
+//
+//   1. the tensor-core prefill in its save mode (fused_prefill.cu) runs the forward again and
+//      keeps, per token-channel, the complete gate pre-activations ga, gx (fp32), h_{t-1} as the
+//      update used it (fp32) and the conv output as a bf16 pair hi + lo (x = hi + lo to 2^-16);
+//      its gate contraction runs on both bf16 parts of the conv output, so the pre-activations
+//      are those of the fp32 conv output;
+//   2. bwd_scan_kernel: one thread per (row, channel) walks the tokens backwards carrying
+//      g = dL/dh_t:  g_t = dout_t GeLU(y_t) + a_{t+1} g_{t+1} (0 across a reset); it writes
+//      dy, the direct part of dL/dxc (g beta i) and dL/dga, dL/dgx as bf16 hi / lo pairs, and
+//      per-row partial sums of dLambda, db_a, db_x;
+//   3. dL/dxc += dga W_a^T + dgx W_x^T: a tensor-core GEMM per head over the B T tokens with the
+//      hi and lo parts of dga and dgx as four K ranges (gemm.cu);
+//   4. bwd_convT_kernel: the conv's transpose in parallel over (row, 64-token block, channel):
+//      dx_s gathers w_k dxc_{s+3-k} over the windows that read x_s, the initial history gets the
+//      taps that read it, the final history's gradient goes to the inputs it copied; partial
+//      sums of dconv_w, dconv_b per block;
+//   5. dW[h] = sum over tokens of xc^T dg for both gates: tensor-core GEMMs with the hi / lo
+//      parts (xc_hi dg_hi + xc_hi dg_lo + xc_lo dg_hi), K cut into slices whose partial sums
+//      are kept apart;
+//   6. bwdtc_reduce_kernel: every partial sum in a fixed order.
+// No atomics: the gradients are bitwise repeatable.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rglru {
+
+namespace {
+
+constexpr int DH = 256;
+constexpr int kTB = 64;          // tokens per conv-transpose block
+constexpr int kSplits = 4;       // K slices of the weight-gradient GEMMs
+constexpr int kScanThreads = 128;
+
+struct Layout {
+    size_t ga, gx, hprev, dxc, xc_hi, xc_lo, dga_hi, dga_lo, dgx_hi, dgx_lo;
+    size_t part_scan, part_conv, dw, fwd, total;
+    int ntb;
+};
+
+Layout layout(const rglru_dims* d) {
+    auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
+    const size_t W = (size_t)d->heads * d->head_dim;
+    const size_t n = (size_t)d->batch * d->seq_len * W;
+    Layout l;
+    l.ntb = (d->seq_len + kTB - 1) / kTB;
+    size_t o = 256;
+    l.ga = o;      o = up(o + n * 4);
+    l.gx = o;      o = up(o + n * 4);
+    l.hprev = o;   o = up(o + n * 4);
+    l.dxc = o;     o = up(o + n * 4);
+    l.xc_hi = o;   o = up(o + n * 2);
+    l.xc_lo = o;   o = up(o + n * 2);
+    l.dga_hi = o;  o = up(o + n * 2);
+    l.dga_lo = o;  o = up(o + n * 2);
+    l.dgx_hi = o;  o = up(o + n * 2);
+    l.dgx_lo = o;  o = up(o + n * 2);
+    l.part_scan = o; o = up(o + 3 * (size_t)d->batch * W * 4);
+    l.part_conv = o; o = up(o + 5 * (size_t)d->batch * l.ntb * W * 4);
+    l.dw = o;      o = up(o + 2 * (size_t)kSplits * d->heads * DH * DH * 4);
+    l.fwd = o;     o = up(o + fused_prefill_workspace(d));
+    l.total = o;
+    return l;
+}
+
+__device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+// d/dv [v Phi(v)] = Phi(v) + v phi(v); the tanh form's derivative for the flag
+__device__ __forceinline__ float gelu_grad(float v, int tanh_form) {
+    if (tanh_form) {
+        const float k = 0.79788456080286535588f;
+        const float th = tanhf(k * (v + 0.044715f * v * v * v));
+        return 0.5f * (1.0f + th) + 0.5f * v * (1.0f - th * th) * k * (1.0f + 3.0f * 0.044715f * v * v);
+    }
+    return 0.5f * erfcf(-v * 0.70710678118654752440f) + v * expf(-0.5f * v * v) * 0.39894228040143267794f;
+}
+
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bfloat16* lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    *hi = h;
+    *lo = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+struct ScanArgs {
+    int B, T, W;
+    float c;
+    int gelu_tanh;
+    const float* lambda;
+    const __nv_bfloat16* y;
+    const __nv_bfloat16* dout;
+    const uint8_t* reset;
+    const float* dh_final;
+    const float* ga;
+    const float* gx;
+    const float* hprev;
+    const __nv_bfloat16* xc_hi;
+    const __nv_bfloat16* xc_lo;
+    float* dy;
+    float* dxc;
+    __nv_bfloat16* dga_hi;
+    __nv_bfloat16* dga_lo;
+    __nv_bfloat16* dgx_hi;
+    __nv_bfloat16* dgx_lo;
+    float* dh0;
+    float* part;          // [3][B][W]: dLambda, db_a, db_x
+};
+
+// ---------------------------------------------------------------- 2. the reverse scan -------
+// Thread = (row b, channel ch); the inputs of a block of kPF tokens are loaded together before
+// the block is walked, so that their latencies overlap.
+constexpr int kPF = 8;
+__global__ void __launch_bounds__(kScanThreads) bwd_scan_kernel(ScanArgs a) {
+    const int ch = blockIdx.x * kScanThreads + threadIdx.x, b = blockIdx.y;
+    if (ch >= a.W) return;
+    const float kappa = a.c * log_sigmoid_acc(a.lambda[ch]);
+    const float c_sneg = a.c * sigmoid_acc(-a.lambda[ch]);
+    float g = a.dh_final ? a.dh_final[(size_t)b * a.W + ch] : 0.f;
+    float s_lam = 0.f, s_ba = 0.f, s_bx = 0.f;
+    const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
+    for (int tb = ((a.T - 1) / kPF) * kPF; tb >= 0; tb -= kPF) {
+        const int n = min(kPF, a.T - tb);
+        float vga[kPF], vgx[kPF], vhp[kPF], vxc[kPF], vy[kPF], vdz[kPF];
+        bool rs[kPF];
+#pragma unroll
+        for (int j = 0; j < kPF; ++j) {
+            if (j < n) {
+                const size_t e = ((size_t)b * a.T + tb + j) * a.W + ch;
+                vga[j] = a.ga[e];
+                vgx[j] = a.gx[e];
+                vhp[j] = a.hprev[e];
+                vxc[j] = bf(a.xc_hi + e) + bf(a.xc_lo + e);
+                vy[j] = bf(a.y + e);
+                vdz[j] = bf(a.dout + e);
+                rs[j] = rrow && rrow[tb + j];
+            }
+        }
+#pragma unroll
+        for (int j = kPF - 1; j >= 0; --j) {
+            if (j >= n) continue;
+            const size_t e = ((size_t)b * a.T + tb + j) * a.W + ch;
+            const float r = sigmoid_acc(vga[j]), ig = sigmoid_acc(vgx[j]);
+            float at, beta;
+            decay_and_beta_acc(kappa, r, &at, &beta);
+            const float xcv = vxc[j], hp = vhp[j];
+            const float h = fmaf(at, hp, beta * (ig * xcv));
+            g = fmaf(vdz[j], gelu_acc(vy[j], a.gelu_tanh), g);
+            a.dy[e] = vdz[j] * h * gelu_grad(vy[j], a.gelu_tanh);
+            const float dl_da = g * hp, dl_dbeta = g * ig * xcv, dl_di = g * beta * xcv;
+            const float r_over_beta = beta > 0.f ? r / beta : 0.f;
+            const float q = dl_da * at * r - dl_dbeta * at * at * r_over_beta;
+            const float dga = kappa * (1.0f - r) * q;
+            const float dgx = dl_di * ig * (1.0f - ig);
+            s_lam = fmaf(c_sneg, q, s_lam);
+            s_ba += dga;
+            s_bx += dgx;
+            split_bf16(dga, a.dga_hi + e, a.dga_lo + e);
+            split_bf16(dgx, a.dgx_hi + e, a.dgx_lo + e);
+            a.dxc[e] = g * beta * ig;
+            g = rs[j] ? 0.f : at * g;
+        }
+    }
+    if (a.dh0) a.dh0[(size_t)b * a.W + ch] = g;
+    const size_t pb = (size_t)a.B * a.W;
+    float* p = a.part + (size_t)b * a.W + ch;
+    p[0 * pb] = s_lam;
+    p[1 * pb] = s_ba;
+    p[2 * pb] = s_bx;
+}
+
+// ---------------------------------------------------------------- 4. the conv's transpose ---
+struct ConvTArgs {
+    int B, T, W, ntb;
+    const float* conv_w;
+    const __nv_bfloat16* x;
+    const __nv_bfloat16* tail0;       // [B][3][W] or nullptr
+    const uint8_t* reset;
+    const float* dtail_final;         // [B][3][W] or nullptr
+    const float* dxc;
+    float* dx;
+    float* dtail0;                    // [B][3][W] or nullptr
+    float* part;                      // [5][B * ntb][W]: dconv_w[4], dconv_b
+};
+
+// True when the window of token t reads position s (s in [t-3, t]): no reset in (s, t].
+__device__ __forceinline__ bool window_reads(const uint8_t* rrow, int s, int t) {
+    if (!rrow) return true;
+    for (int p = (s + 1 > 0 ? s + 1 : 0); p <= t; ++p)
+        if (rrow[p]) return false;
+    return true;
+}
+
+__global__ void __launch_bounds__(128) bwd_convT_kernel(ConvTArgs a) {
+    const int ch = blockIdx.x * 128 + threadIdx.x, tb = blockIdx.y, b = blockIdx.z;
+    if (ch >= a.W) return;
+    const int t0 = tb * kTB, t1 = min(a.T, t0 + kTB);
+    const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
+    float cw[kConvWidth];
+#pragma unroll
+    for (int k = 0; k < kConvWidth; ++k) cw[k] = a.conv_w[(size_t)k * a.W + ch];
+    auto xval = [&](int s) -> float {                       // x_s, the initial history for s < 0
+        if (s >= 0) return bf(a.x + ((size_t)b * a.T + s) * a.W + ch);
+        return a.tail0 ? bf(a.tail0 + ((size_t)b * kHist + (kHist + s)) * a.W + ch) : 0.f;
+    };
+    auto dxcv = [&](int t) -> float { return a.dxc[((size_t)b * a.T + t) * a.W + ch]; };
+    // parameter gradients over the block's tokens
+    float s_cw[kConvWidth] = {0.f, 0.f, 0.f, 0.f}, s_cb = 0.f;
+    for (int t = t0; t < t1; ++t) {
+        const float d = dxcv(t);
+        s_cb += d;
+#pragma unroll
+        for (int k = 0; k < kConvWidth; ++k) {
+            const int s = t - kHist + k;
+            if (window_reads(rrow, s, t)) s_cw[k] = fmaf(d, xval(s), s_cw[k]);
+        }
+    }
+    const size_t pb = (size_t)a.B * a.ntb * a.W, pi = ((size_t)b * a.ntb + tb) * a.W + ch;
+#pragma unroll
+    for (int k = 0; k < kConvWidth; ++k) a.part[k * pb + pi] = s_cw[k];
+    a.part[4 * pb + pi] = s_cb;
+    // dx of the block's positions (and the initial history, from the first block)
+    for (int s = (tb == 0 ? -kHist : t0); s < t1; ++s) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < kConvWidth; ++k) {
+            const int t = s + kHist - k;                     // the token whose tap k reads s
+            if (t >= 0 && t < a.T && window_reads(rrow, s, t)) acc = fmaf(cw[k], dxcv(t), acc);
+        }
+        if (a.dtail_final && s >= a.T - kHist && window_reads(rrow, s, a.T - 1))
+            acc += a.dtail_final[((size_t)b * kHist + (s - (a.T - kHist))) * a.W + ch];
+        if (s >= 0) a.dx[((size_t)b * a.T + s) * a.W + ch] = acc;
+        else if (a.dtail0) a.dtail0[((size_t)b * kHist + (kHist + s)) * a.W + ch] = acc;
+    }
+}
+
+// ---------------------------------------------------------------- 6. fixed-order sums -------
+struct ReduceArgs {
+    int B, ntb, W, H;
+    const float* part_scan;
+    const float* part_conv;
+    const float* dw;                  // [2][kSplits][H][256][256]
+    rglru_grads g;
+};
+
+__global__ void bwdtc_reduce_vec_kernel(ReduceArgs a) {
+    const int ch = blockIdx.x * blockDim.x + threadIdx.x;
+    if (ch >= a.W) return;
+    const size_t ps = (size_t)a.B * a.W;
+    float s[3] = {0.f, 0.f, 0.f};
+    for (int b = 0; b < a.B; ++b)
+#pragma unroll
+        for (int k = 0; k < 3; ++k) s[k] += a.part_scan[k * ps + (size_t)b * a.W + ch];
+    a.g.dlambda[ch] = s[0];
+    a.g.db_a[ch] = s[1];
+    a.g.db_x[ch] = s[2];
+    const size_t pc = (size_t)a.B * a.ntb * a.W;
+    float c[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < a.B * a.ntb; ++i)
+#pragma unroll
+        for (int k = 0; k < 5; ++k) c[k] += a.part_conv[k * pc + (size_t)i * a.W + ch];
+#pragma unroll
+    for (int k = 0; k < kConvWidth; ++k) a.g.dconv_w[(size_t)k * a.W + ch] = c[k];
+    a.g.dconv_b[ch] = c[4];
+}
+
+__global__ void bwdtc_reduce_w_kernel(ReduceArgs a) {
+    const size_t n = (size_t)a.H * DH * DH;
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+#pragma unroll
+    for (int gate = 0; gate < 2; ++gate) {
+        float s = 0.f;
+        for (int sp = 0; sp < kSplits; ++sp) s += a.dw[((size_t)gate * kSplits + sp) * n + i];
+        (gate ? a.g.dw_x : a.g.dw_a)[i] = s;
+    }
+}
+
+GemmPair pair_tokens_x_weights(const __nv_bfloat16* dg, const __nv_bfloat16* w, long long tokens, int H, int W) {
+    // A (m = token, k = output channel o of head h): dg[token][h * 256 + o], K-major
+    // B (n = input channel i, k = o): W[h][i][o], K-major (rows h * 256 + i)
+    GemmPair p{};
+    p.a = dg; p.a_rows = tokens; p.a_cols = W; p.a_ld = W;
+    p.a_kmajor = 1; p.a_boff_row = 0; p.a_boff_col = 0; p.a_bstep_row = 0; p.a_bstep_col = DH;
+    p.b = w; p.b_rows = (long long)H * DH; p.b_cols = DH; p.b_ld = DH;
+    p.b_kmajor = 1; p.b_boff_row = 0; p.b_boff_col = 0; p.b_bstep_row = DH; p.b_bstep_col = 0;
+    p.K = DH;
+    return p;
+}
+
+GemmPair pair_xc_dg(const __nv_bfloat16* xc, const __nv_bfloat16* dg, long long tokens, int W) {
+    // A (m = input channel i, k = token): xc[token][h * 256 + i], M-major
+    // B (n = output channel o, k = token): dg[token][h * 256 + o], N-major
+    GemmPair p{};
+    p.a = xc; p.a_rows = tokens; p.a_cols = W; p.a_ld = W;
+    p.a_kmajor = 0; p.a_boff_row = 0; p.a_boff_col = 0; p.a_bstep_row = 0; p.a_bstep_col = DH;
+    p.b = dg; p.b_rows = tokens; p.b_cols = W; p.b_ld = W;
+    p.b_kmajor = 0; p.b_boff_row = 0; p.b_boff_col = 0; p.b_bstep_row = 0; p.b_bstep_col = DH;
+    p.K = (int)((tokens + 63) / 64 * 64);   // rows past the tokens read as zeros
+    return p;
+}
+
+}  // namespace
+
+bool backward_tc_supported(const rglru_dims* d) {
+    return d->act_dtype == RGLRU_BF16 && d->head_dim == DH && !(d->flags & RGLRU_FLAG_GENERIC);
+}
+
+size_t backward_tc_workspace(const rglru_dims* d) { return layout(d).total; }
+
+int backward_tc_launches(const rglru_dims* d) {
+    (void)d;
+    return 9;   // prefill (memset + kernel), scan, GEMM, conv transpose, 2 GEMMs, 2 reductions
+}
+
+cudaError_t launch_backward_tc(const rglru_dims* d, const rglru_params* p, const void* x, const void* y,
+                               const uint8_t* reset, const rglru_state* st0, const void* dout,
+                               const float* dh_final, const float* dtail_final, const rglru_grads* grads,
+                               void* ws, size_t ws_bytes, cudaStream_t s) {
+    const Layout l = layout(d);
+    if (l.total > ws_bytes) return cudaErrorInvalidValue;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    DeviceStatus* status = reinterpret_cast<DeviceStatus*>(w);
+    const int B = d->batch, T = d->seq_len, H = d->heads, W = H * DH;
+    const long long tokens = (long long)B * T;
+    auto f32 = [&](size_t o) { return reinterpret_cast<float*>(w + o); };
+    auto b16 = [&](size_t o) { return reinterpret_cast<__nv_bfloat16*>(w + o); };
+
+    // 1. the forward again, keeping what the gradients need
+    PrefillSave sv{};
+    sv.ga = f32(l.ga); sv.gx = f32(l.gx); sv.hprev = f32(l.hprev);
+    sv.xc_hi = b16(l.xc_hi); sv.xc_lo = b16(l.xc_lo);
+    rglru_state st_copy{};
+    rglru_state* stp = nullptr;
+    if (st0) {   // the save mode reads the initial state and writes nothing back
+        st_copy = *st0;
+        stp = &st_copy;
+    }
+    cudaError_t e = launch_fused_prefill_save(d, p, x, reset, stp, &sv, w + l.fwd, ws_bytes - l.fwd, status, s);
+    if (e != cudaSuccess) return e;
+
+    // 2. the reverse scan
+    ScanArgs sa{};
+    sa.B = B; sa.T = T; sa.W = W; sa.c = d->c; sa.gelu_tanh = d->gelu_tanh;
+    sa.lambda = p->lambda; sa.y = static_cast<const __nv_bfloat16*>(y);
+    sa.dout = static_cast<const __nv_bfloat16*>(dout); sa.reset = reset; sa.dh_final = dh_final;
+    sa.ga = f32(l.ga); sa.gx = f32(l.gx); sa.hprev = f32(l.hprev);
+    sa.xc_hi = b16(l.xc_hi); sa.xc_lo = b16(l.xc_lo);
+    sa.dy = grads->dy; sa.dxc = f32(l.dxc);
+    sa.dga_hi = b16(l.dga_hi); sa.dga_lo = b16(l.dga_lo); sa.dgx_hi = b16(l.dgx_hi); sa.dgx_lo = b16(l.dgx_lo);
+    sa.dh0 = grads->dh0; sa.part = f32(l.part_scan);
+    bwd_scan_kernel<<<dim3((W + kScanThreads - 1) / kScanThreads, B), kScanThreads, 0, s>>>(sa);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    // 3. dL/dxc += dga W_a^T + dgx W_x^T (hi and lo parts of dga, dgx), in place
+    const __nv_bfloat16* wa = static_cast<const __nv_bfloat16*>(p->w_a);
+    const __nv_bfloat16* wx = static_cast<const __nv_bfloat16*>(p->w_x);
+    GemmOperands gx{};
+    gx.M = (int)tokens; gx.N = DH; gx.batch = H; gx.splits = 1; gx.npairs = 4;
+    gx.p[0] = pair_tokens_x_weights(b16(l.dga_hi), wa, tokens, H, W);
+    gx.p[1] = pair_tokens_x_weights(b16(l.dga_lo), wa, tokens, H, W);
+    gx.p[2] = pair_tokens_x_weights(b16(l.dgx_hi), wx, tokens, H, W);
+    gx.p[3] = pair_tokens_x_weights(b16(l.dgx_lo), wx, tokens, H, W);
+    gx.C = f32(l.dxc); gx.c_ld = W; gx.c_bstride = DH; gx.c_split = 0;
+    gx.Cadd = f32(l.dxc); gx.add_ld = W; gx.add_bstride = DH;
+    gx.status = status;
+    e = launch_gemm(gx, s);
+    if (e != cudaSuccess) return e;
+
+    // 4. the conv's transpose
+    ConvTArgs ca{};
+    ca.B = B; ca.T = T; ca.W = W; ca.ntb = l.ntb;
+    ca.conv_w = p->conv_w; ca.x = static_cast<const __nv_bfloat16*>(x);
+    ca.tail0 = st0 ? static_cast<const __nv_bfloat16*>(st0->conv_tail) : nullptr;
+    ca.reset = reset; ca.dtail_final = dtail_final; ca.dxc = f32(l.dxc);
+    ca.dx = grads->dx; ca.dtail0 = grads->dtail0; ca.part = f32(l.part_conv);
+    bwd_convT_kernel<<<dim3((W + 127) / 128, l.ntb, B), 128, 0, s>>>(ca);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    // 5. dW = xc^T dg per head and gate, K (the tokens) cut into kSplits slices
+    for (int gate = 0; gate < 2; ++gate) {
+        GemmOperands gw{};
+        gw.M = DH; gw.N = DH; gw.batch = H; gw.splits = kSplits; gw.npairs = 3;
+        const __nv_bfloat16* hi = b16(gate ? l.dgx_hi : l.dga_hi);
+        const __nv_bfloat16* lo = b16(gate ? l.dgx_lo : l.dga_lo);
+        gw.p[0] = pair_xc_dg(b16(l.xc_hi), hi, tokens, W);
+        gw.p[1] = pair_xc_dg(b16(l.xc_hi), lo, tokens, W);
+        gw.p[2] = pair_xc_dg(b16(l.xc_lo), hi, tokens, W);
+        gw.C = f32(l.dw) + (size_t)gate * kSplits * H * DH * DH;
+        gw.c_ld = DH; gw.c_bstride = (long long)DH * DH; gw.c_split = (long long)H * DH * DH;
+        gw.Cadd = nullptr;
+        gw.status = status;
+        e = launch_gemm(gw, s);
+        if (e != cudaSuccess) return e;
+    }
+
+    // 6. every partial sum, in a fixed order
+    ReduceArgs ra{};
+    ra.B = B; ra.ntb = l.ntb; ra.W = W; ra.H = H;
+    ra.part_scan = f32(l.part_scan); ra.part_conv = f32(l.part_conv); ra.dw = f32(l.dw);
+    ra.g = *grads;
+    bwdtc_reduce_vec_kernel<<<(W + 255) / 256, 256, 0, s>>>(ra);
+    const size_t nw = (size_t)H * DH * DH;
+    bwdtc_reduce_w_kernel<<<(unsigned)((nw + 255) / 256), 256, 0, s>>>(ra);
+    return cudaGetLastError();
+}
+
+}  // namespace rglru

@@ -11,21 +11,17 @@
 
 namespace rglru {
 
-// Sets a kernel's dynamic shared-memory limit once per device (the attribute belongs to the
-// current device; doing it on the first call keeps it out of any later stream capture).
+// Unique id of the calling thread's current CUDA context (0 when unavailable).
+unsigned long long current_context_id();
+
+// Sets a kernel's dynamic shared-memory limit once per kernel and context (the attribute belongs
+// to the kernel in the current context; doing it on the first call keeps it out of any later
+// stream capture, and a new context -- after a cudaDeviceReset -- gets it again).
+cudaError_t set_smem_limit(const void* kernel, int bytes);
+
 template <typename Kernel>
 cudaError_t set_smem_once(Kernel k, int bytes) {
-    static std::mutex mu;
-    static bool done[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    std::lock_guard<std::mutex> lock(mu);
-    if (done[dev]) return cudaSuccess;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) done[dev] = true;
-    return e;
+    return set_smem_limit(reinterpret_cast<const void*>(k), bytes);
 }
 
 constexpr int kConvWidth = 4;

@@ -8,49 +8,48 @@
 //
 //   * conv: CTA r convolves its own 64 channels for the 128 rows (the width-4 causal conv over
 //     the carried history and the new input), shifts their history in place (oldest out, x in;
-//     a row with reset[b] set starts from an empty history), and writes the bf16 result as
-//     K-block r of its 128 x 256 MMA operand tile (K-major, 128-byte swizzle); one thread then
+//     a row with reset[b] set starts from an empty history), keeps the fp32 result for the
+//     state update, and writes it rounded to fp16 as K-block r of its 128 x 256 MMA operand
+//     tile (K-major, 128-byte swizzle); one thread then
 //     copies that 16 KB block into the same place of the three sibling CTAs' tiles through
 //     distributed shared memory (bulk copies that complete on the siblings' mbarrier), so every
 //     channel is convolved once and only by the CTA that owns its history;
 //   * gates: TMA brings the 256 x 64 slices W_a[h][:, 64 r], W_x[h][:, 64 r] (as stored: output
-//     channel contiguous, i.e. MN-major for the MMA) side by side, one N = 128 operand; one
-//     thread issues tcgen05.mma (M = 128, N = 128, K = 16 each) into TMEM, K block by K block as
-//     the blocks become ready (its own first);
+//     channel contiguous, i.e. MN-major for the MMA) side by side, one N = 128 operand, which
+//     the update threads convert to fp16 in place once it has landed (exact for 2^-14 <= |w| <
+//     65504); an elected lane of the MMA warp issues tcgen05.mma (M = 128, N = 128, K = 16
+//     each, fp16 operands, fp32 accumulation) into TMEM, K block by K block as the blocks
+//     become ready (its own first);
 //   * update: TMA also brings the h (fp32) and y tiles of the CTA into shared memory; 16 warps
 //     (thread = row, 16 channels each) compute GeLU(y) while the MMAs run, then read the
 //     accumulators, apply the gates and write h and out back into the shared tiles, which TMA
 //     stores (rows past the batch are clipped by the tensor maps).
 //
-// The element-wise arithmetic is that of the prefill kernel (fused_prefill.cu): one tanh per
-// gate, expm1 of the log-decay by its series near zero, sqrt(1 - a^2) without cancellation,
-// GeLU in its tanh form fitted to y Phi(y).  Sources ("Griffin Guide: RecurrentGemma, RG-LRU &
+// The element-wise arithmetic is rglru_math.cuh's (shared with the prefill): gates by ex2 and a
+// reciprocal, expm1 of the log-decay by its series near zero, sqrt(1 - a^2) i_t by one rsqrt,
+// GeLU by a fitted tail polynomial and one ex2.  Sources ("Griffin Guide: RecurrentGemma, RG-LRU &
 // Hybrid Attention"): "1. Formulation of the RG-LRU Gating Mechanism", "2. The Role of
 // Square-Root Variance Normalization", "1. Temporal Filtering via Separable 1D Convolutions",
 // "2. Non-Linear Multiplicative Gating with GeLU", "3. Block-Diagonal Sharding for
 // Zero-Communication Tensor Parallelism", and the listing's RGLRU.step.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "rglru_math.cuh"
 #include "sm100.cuh"
+#include "tma_maps.h"
 
 namespace rglru {
-
-// shared with fused_prefill.cu (host side)
-namespace tc {
-bool make_map_2d_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                       uint32_t box_inner, uint32_t box_outer);
-bool make_map_2d_sw128_elem(CUtensorMap* m, const void* base, uint32_t elem_bytes, uint64_t inner, uint64_t outer,
-                            uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
-}
 
 namespace dec {
 
 using namespace sm100;
+using namespace fm;
 
 constexpr int DH = 256;
 constexpr int MT = 128;                 // rows per CTA (MMA M, TMEM lanes)
@@ -61,28 +60,30 @@ constexpr int kWarpMma = kEpiWarps, kWarpTma = kEpiWarps + 1;
 constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kEpiCh = NT / (kEpiWarps / 4);  // channels per update thread (16)
-constexpr int kConvUnits = MT * (NT / 8) / kEpiThreads;  // (row, 8 channels) conv units per thread (2)
 
 constexpr uint32_t A_BYTES = MT * DH * 2;            // 65536: 4 K-blocks of 128 rows x 128 B
 constexpr uint32_t A_KBLK = MT * 128;                // 16384
 constexpr uint32_t B_BYTES = DH * NT * 2;            // 32768 per gate: 256 K-rows x 128 B
-constexpr uint32_t H_BOX = MT * 128;                 // h tile: 2 boxes of 128 rows x 32 fp32
 constexpr uint32_t Y_BYTES = MT * NT * 2;            // y tile (then out): 128 rows x 64 bf16
-constexpr uint32_t OFF_A = 0;
-constexpr uint32_t OFF_BA = OFF_A + A_BYTES;
+constexpr uint32_t OFF_A = 0;                        // conv output, fp16 hi part
+constexpr uint32_t OFF_ALO = OFF_A + A_BYTES;        // and lo part (xc - hi)
+constexpr uint32_t OFF_BA = OFF_ALO + A_BYTES;
 constexpr uint32_t OFF_BX = OFF_BA + B_BYTES;        // right after W_a: one N = 128 operand
-constexpr uint32_t OFF_H = OFF_BX + B_BYTES;
-constexpr uint32_t OFF_Y = OFF_H + 2 * H_BOX;
-constexpr uint32_t OFF_CONST = OFF_Y + Y_BYTES;      // hk, b_a / 2, b_x / 2 per channel: 3 x 64 fp32
+constexpr uint32_t OFF_Y = OFF_BX + B_BYTES;
+constexpr uint32_t OFF_CONST = OFF_Y + Y_BYTES;      // K, -b_a log2 e, -b_x log2 e per channel: 3 x 64 fp32
 constexpr uint32_t OFF_CONV = OFF_CONST + 3 * NT * 4; // conv taps [4][64] and bias [64], fp32
 constexpr uint32_t OFF_BAR = OFF_CONV + 5 * NT * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + 64;
 constexpr int kClusterSize = DH / NT;                 // CTAs of a (head, row tile)
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 32 + 1024;
-constexpr uint32_t TMEM_COLS = 128;                  // D_a [0,64), D_x [64,128)
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// TMEM: D_a [0,64), D_x [64,128), the fp32 conv output [128,192) (lane = row)
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TM_XC = 2 * NT;
 
 struct Args {
     int B, H, mtiles;
+    float* h;                         // [B][W] state, read and written in place
     const __nv_bfloat16* x;
     __nv_bfloat16* tail;
     const float* conv_w;
@@ -104,10 +105,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&p);
 }
-__device__ __forceinline__ float sqrt_approx(float x) {
-    float r;
-    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-    return r;
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 p = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&p);
 }
 
 // Shared-memory matrix descriptor for an MN-major operand in the 128-byte swizzle layout: rows
@@ -125,10 +125,9 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr) {
     return d;
 }
 
-// Instruction descriptor: fp32 accumulator, bf16 A (K-major) and B (MN-major), M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+// Instruction descriptor: fp32 accumulator, fp16 A (K-major) and B (MN-major), M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
+    return (1u << 4) | (1u << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 __device__ bool wait_bounded(uint32_t bar, uint32_t parity, const Args& a, volatile int* abort, unsigned where) {
@@ -145,46 +144,23 @@ __device__ bool wait_bounded(uint32_t bar, uint32_t parity, const Args& a, volat
     }
 }
 
-// ---------------------------------------------------------------- cluster helpers -----------
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// shared::cluster address of this CTA's shared address `a` in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t a, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
-    return r;
-}
-// copy `bytes` of this CTA's shared memory to another CTA's shared memory; completes on that
-// CTA's mbarrier (its transaction count)
-__device__ __forceinline__ void dsmem_copy(uint32_t dst_cluster, uint32_t src, uint32_t bytes, uint32_t bar_cluster) {
-    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     dst_cluster),
-                 "r"(src), "r"(bytes), "r"(bar_cluster)
-                 : "memory");
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_constant__ CUtensorMap map_wx,
-                    const __grid_constant__ CUtensorMap map_h, const __grid_constant__ CUtensorMap map_y,
-                    const __grid_constant__ CUtensorMap map_out, const Args a) {
+                    const __grid_constant__ CUtensorMap map_y, const __grid_constant__ CUtensorMap map_out,
+                    const Args a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_w = sbase + OFF_BAR, bar_acc = sbase + OFF_BAR + 16;
-    const uint32_t bar_hy = sbase + OFF_BAR + 24;     // h and y tiles
+    const uint32_t bar_wc = sbase + OFF_BAR + 8;      // the weight tile is in fp16
+    const uint32_t bar_y = sbase + OFF_BAR + 24;      // y tile
     // K block j of the operand tile: convolved here (j = rank) or copied in by CTA j
     auto bar_k = [&](int j) { return sbase + OFF_BAR + 32 + 8 * (uint32_t)j; };
     volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
     volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 16);
-    float* s_hk = reinterpret_cast<float*>(smem + OFF_CONST);
-    float* s_ba = s_hk + NT;
-    float* s_bx = s_ba + NT;
+    float* s_K = reinterpret_cast<float*>(smem + OFF_CONST);
+    float* s_nba = s_K + NT;
+    float* s_nbx = s_nba + NT;
     float* s_cw = reinterpret_cast<float*>(smem + OFF_CONV);   // [4][64]
     float* s_cb = s_cw + 4 * NT;                                 // [64]
 
@@ -200,13 +176,14 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         mbar_init(bar_w, 1);
+        mbar_init(bar_wc, 1);
         mbar_init(bar_acc, 1);
-        mbar_init(bar_hy, 1);
+        mbar_init(bar_y, 1);
         for (int j = 0; j < kClusterSize; ++j) mbar_init(bar_k(j), 1);
         *abort = 0;
         fence_barrier_init();
         for (int j = 0; j < kClusterSize; ++j)
-            if (j != nt) mbar_arrive_expect_tx(bar_k(j), A_KBLK);   // completed by CTA j's copy
+            if (j != nt) mbar_arrive_expect_tx(bar_k(j), 2 * A_KBLK);   // completed by CTA j's copies
     }
     if (warp == kWarpMma) {
         tmem_alloc(smem_u32((const void*)tmem_base_s), TMEM_COLS);
@@ -215,7 +192,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
     if (warp == kWarpTma && lane == 0) {
         prefetch_tensormap(&map_wa);
         prefetch_tensormap(&map_wx);
-        prefetch_tensormap(&map_h);
         prefetch_tensormap(&map_y);
         prefetch_tensormap(&map_out);
     }
@@ -235,11 +211,9 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
                 tma_load_2d(sbase + OFF_BA + kb * 8192, &map_wa, nt * NT, head * DH + kb * 64, bar_w);
                 tma_load_2d(sbase + OFF_BX + kb * 8192, &map_wx, nt * NT, head * DH + kb * 64, bar_w);
             }
-            // this tile's state and y (rows past the batch read as zeros)
-            mbar_arrive_expect_tx(bar_hy, 2 * H_BOX + Y_BYTES);
-            tma_load_2d(sbase + OFF_H, &map_h, ch0, mt * MT, bar_hy);
-            tma_load_2d(sbase + OFF_H + H_BOX, &map_h, ch0 + 32, mt * MT, bar_hy);
-            tma_load_2d(sbase + OFF_Y, &map_y, ch0, mt * MT, bar_hy);
+            // this tile's y (rows past the batch read as zeros)
+            mbar_arrive_expect_tx(bar_y, Y_BYTES);
+            tma_load_2d(sbase + OFF_Y, &map_y, ch0, mt * MT, bar_y);
             // never leave the CTA with a bulk copy still writing its shared memory (the weight
             // tiles, or a sibling's conv block, whose completion also ends the sibling's reads)
             const uint64_t t0 = globaltimer_ns();
@@ -248,37 +222,51 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
             for (int j = 0; j < kClusterSize; ++j)
                 while (!mbar_try_wait_sleep(bar_k(j), 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
                 }
-            while (!mbar_try_wait_sleep(bar_hy, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
+            while (!mbar_try_wait_sleep(bar_y, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
             }
         }
     } else if (warp == kWarpMma) {
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16_f32_bmn(MT, 2 * NT);   // D_a | D_x
-            // K blocks in the order they become ready: this CTA's own first, then the siblings'
-            bool ok = wait_bounded(bar_w, 0, a, abort, 1);
-            uint32_t accum = 0;
-            for (int i = 0; i < kClusterSize && ok; ++i) {
-                const int j = (nt + i) % kClusterSize;
-                ok = wait_bounded(bar_k(j), 0, a, abort, 3);
-                if (!ok) break;
-                tc_fence_after();
+        // the whole warp follows the waits; one elected lane issues (warp-uniform operands)
+        const uint32_t idesc = idesc_f16_f32_bmn(MT, 2 * NT);   // D_a | D_x
+        const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+        // K blocks in the order they become ready: this CTA's own first, then the siblings'
+        bool ok = __all_sync(0xffffffffu, wait_bounded(bar_wc, 0, a, abort, 1));
+        uint32_t accum = 0;
+        for (int i = 0; i < kClusterSize && ok; ++i) {
+            const int j = (nt + i) % kClusterSize;
+            ok = __all_sync(0xffffffffu, wait_bounded(bar_k(j), 0, a, abort, 3));
+            if (!ok) break;
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < KSTEPS / kClusterSize; ++kk) {
-                    const int ks = j * 4 + kk;
-                    const uint64_t ad = desc_k_sw128(sbase + OFF_A + j * A_KBLK + kk * 32);
-                    const uint64_t bd = desc_mn_sw128(sbase + OFF_BA + ks * 16 * 128);
-                    mma_ss(tmem, ad, bd, idesc, accum);
-                    accum = 1;
-                }
+                for (int part = 0; part < 2; ++part)          // the conv output's hi and lo parts
+#pragma unroll
+                    for (int kk = 0; kk < KSTEPS / kClusterSize; ++kk) {
+                        const int ks = j * 4 + kk;
+                        const uint64_t ad = desc_k_sw128(sbase + (part ? OFF_ALO : OFF_A) + j * A_KBLK + kk * 32);
+                        const uint64_t bd = desc_mn_sw128(sbase + OFF_BA + ks * 16 * 128);
+                        mma_ss(tm, ad, bd, idesc, (accum | (uint32_t)kk | (uint32_t)part) ? 1u : 0u);
+                    }
             }
-            mma_commit(bar_acc);     // also when a wait failed: the epilogue must not wait forever
+            __syncwarp();
+            accum = 1;
         }
+        if (elect_one()) mma_commit(bar_acc);     // also when a wait failed: the update must not wait forever
+        __syncwarp();
     } else {
-        // ================================ loads ================================================
-        // The per-channel constants (threads < 64, staged in shared memory), then the conv inputs of
-        // this thread's units (row rl = 64 k + tid / 8, channels 8 (tid % 8) .. +7 of the tile),
-        // issued together so their latencies overlap.
-        if (threadIdx.x < NT) {
+        // ================================ update threads =======================================
+        // thread = row r of the tile (= TMEM lane r), channels [16 cg, 16 cg + 16) of its 64: it
+        // convolves them, keeps their fp32 conv output in its TMEM lane, and later updates them
+        const int q = warp & 3, cg = warp >> 2;           // lane quarter, channel quarter of the tile
+        const int r = q * 32 + lane;                      // row within the tile
+        const int b = mt * MT + r;
+        const bool live = b < a.B;
+        const int bs = live ? b : 0;                      // rows past the batch: any valid row
+        const uint32_t sw = (uint32_t)(r & 7);
+        const int cbase = ch0 + cg * kEpiCh;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const uint32_t xcol = tmem + lane_off + TM_XC + cg * kEpiCh;
+        if (threadIdx.x < NT) {                           // per-channel constants
             const int ch = ch0 + threadIdx.x;
             const float lam = a.lambda[ch];
             const float ba = a.b_a ? a.b_a[ch] : 0.f;
@@ -287,111 +275,126 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
 #pragma unroll
             for (int k = 0; k < kConvWidth; ++k) s_cw[k * NT + threadIdx.x] = a.conv_w[(size_t)k * W + ch];
             s_cb[threadIdx.x] = cb0;
-            s_hk[threadIdx.x] = 0.5f * a.c * log_sigmoid_acc(lam);
-            s_ba[threadIdx.x] = 0.5f * ba;
-            s_bx[threadIdx.x] = 0.5f * bx;
+            s_K[threadIdx.x] = a.c * log_sigmoid_acc(lam);
+            s_nba[threadIdx.x] = -ba * kLog2e;
+            s_nbx[threadIdx.x] = -bx * kLog2e;
         }
-        const int g8 = threadIdx.x & 7;
-        uint4 xv[kConvUnits], t0[kConvUnits], t1[kConvUnits], t2[kConvUnits];
+        // the conv's inputs (x and the three past inputs) and the state, issued together
+        uint4 xv[2], t0[2], t1[2], t2[2];
+        const __nv_bfloat16* tl = a.tail + (size_t)bs * kHist * W + cbase;
 #pragma unroll
-        for (int k = 0; k < kConvUnits; ++k) {
-            const int rl = k * (kEpiThreads / 8) + (threadIdx.x >> 3);
-            const int bk = mt * MT + rl;
-            const int bs = bk < a.B ? bk : 0;                 // rows past the batch: any valid row
-            const __nv_bfloat16* tl = a.tail + (size_t)bs * kHist * W + ch0 + g8 * 8;
-            xv[k] = *reinterpret_cast<const uint4*>(a.x + (size_t)bs * W + ch0 + g8 * 8);
-            t0[k] = *reinterpret_cast<const uint4*>(tl);
-            t1[k] = *reinterpret_cast<const uint4*>(tl + W);
-            t2[k] = *reinterpret_cast<const uint4*>(tl + 2 * W);
+        for (int v = 0; v < 2; ++v) {
+            xv[v] = *reinterpret_cast<const uint4*>(a.x + (size_t)bs * W + cbase + 8 * v);
+            t0[v] = *reinterpret_cast<const uint4*>(tl + 8 * v);
+            t1[v] = *reinterpret_cast<const uint4*>(tl + W + 8 * v);
+            t2[v] = *reinterpret_cast<const uint4*>(tl + 2 * W + 8 * v);
         }
+        float hv[kEpiCh];
+        {
+            const float4* hp = reinterpret_cast<const float4*>(a.h + (size_t)bs * W + cbase);
+#pragma unroll
+            for (int i = 0; i < kEpiCh / 4; ++i) {
+                const float4 v = hp[i];
+                hv[4 * i] = v.x; hv[4 * i + 1] = v.y; hv[4 * i + 2] = v.z; hv[4 * i + 3] = v.w;
+            }
+        }
+        const bool rst = live && a.reset && a.reset[b];
         asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
 
         // ================================ conv of this CTA's channels ==========================
         {
-            const uint32_t kblk = sbase + OFF_A + nt * A_KBLK;
-            float cw[4][8], cb[8];
+            if (rst) {                                    // an empty history
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-#pragma unroll
-                for (int k = 0; k < kConvWidth; ++k) cw[k][j] = s_cw[k * NT + g8 * 8 + j];
-                cb[j] = s_cb[g8 * 8 + j];
+                for (int v = 0; v < 2; ++v) t0[v] = t1[v] = t2[v] = make_uint4(0, 0, 0, 0);
             }
+            const float* cwp = s_cw + cg * kEpiCh;
+            const float* cbp = s_cb + cg * kEpiCh;
 #pragma unroll
-            for (int k = 0; k < kConvUnits; ++k) {
-                const int rl = k * (kEpiThreads / 8) + (threadIdx.x >> 3);
-                const int bk = mt * MT + rl;
-                uint4 o = make_uint4(0, 0, 0, 0);
-                if (bk < a.B) {
-                    if (a.reset && a.reset[bk]) {             // an empty history
-                        t0[k] = make_uint4(0, 0, 0, 0);
-                        t1[k] = t0[k];
-                        t2[k] = t0[k];
+            for (int v = 0; v < 2; ++v) {
+                const uint32_t* px = reinterpret_cast<const uint32_t*>(&xv[v]);
+                const uint32_t* p0 = reinterpret_cast<const uint32_t*>(&t0[v]);
+                const uint32_t* p1 = reinterpret_cast<const uint32_t*>(&t1[v]);
+                const uint32_t* p2 = reinterpret_cast<const uint32_t*>(&t2[v]);
+                uint32_t ohi[4], olo[4], xo[8];
+#pragma unroll
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    float rr[2];
+#pragma unroll
+                    for (int e1 = 0; e1 < 2; ++e1) {
+                        const int j = v * 8 + 2 * e2 + e1;
+                        const float v0 = e1 ? bf16hi(p0[e2]) : bf16lo(p0[e2]);
+                        const float v1 = e1 ? bf16hi(p1[e2]) : bf16lo(p1[e2]);
+                        const float v2 = e1 ? bf16hi(p2[e2]) : bf16lo(p2[e2]);
+                        const float v3 = e1 ? bf16hi(px[e2]) : bf16lo(px[e2]);
+                        float acc = fmaf(cwp[j], v0, cbp[j]);
+                        acc = fmaf(cwp[NT + j], v1, acc);
+                        acc = fmaf(cwp[2 * NT + j], v2, acc);
+                        acc = fmaf(cwp[3 * NT + j], v3, acc);
+                        rr[e1] = acc;
+                        xo[2 * e2 + e1] = __float_as_uint(acc);
                     }
-                    const uint32_t* px = reinterpret_cast<const uint32_t*>(&xv[k]);
-                    const uint32_t* p0 = reinterpret_cast<const uint32_t*>(&t0[k]);
-                    const uint32_t* p1 = reinterpret_cast<const uint32_t*>(&t1[k]);
-                    const uint32_t* p2 = reinterpret_cast<const uint32_t*>(&t2[k]);
-                    uint32_t* po = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        float rr[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int j = 2 * i + e;
-                            const float v0 = e ? bf16hi(p0[i]) : bf16lo(p0[i]);
-                            const float v1 = e ? bf16hi(p1[i]) : bf16lo(p1[i]);
-                            const float v2 = e ? bf16hi(p2[i]) : bf16lo(p2[i]);
-                            const float v3 = e ? bf16hi(px[i]) : bf16lo(px[i]);
-                            float acc = fmaf(cw[0][j], v0, cb[j]);
-                            acc = fmaf(cw[1][j], v1, acc);
-                            acc = fmaf(cw[2][j], v2, acc);
-                            rr[e] = fmaf(cw[3][j], v3, acc);
-                        }
-                        po[i] = pack_bf16x2(rr[0], rr[1]);
-                    }
+                    ohi[e2] = pack_f16x2(rr[0], rr[1]);
+                    olo[e2] = pack_f16x2(rr[0] - __half2float(__ushort_as_half((unsigned short)(ohi[e2] & 0xFFFFu))),
+                                         rr[1] - __half2float(__ushort_as_half((unsigned short)(ohi[e2] >> 16))));
                 }
-                // element (row rl, channels 8 g8 .. +7) of the 128-byte swizzled K block
-                const uint32_t so = (uint32_t)(rl >> 3) * 1024 + (uint32_t)(rl & 7) * 128 + ((uint32_t)(g8 ^ (rl & 7)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(kblk + so), "r"(o.x), "r"(o.y), "r"(o.z),
-                             "r"(o.w)
-                             : "memory");
+                // row r, 16-byte chunk (2 cg + v) of this CTA's K block (128-byte swizzle)
+                const uint32_t so = nt * A_KBLK + (uint32_t)(r >> 3) * 1024 + sw * 128 + ((((uint32_t)(cg * 2 + v)) ^ sw) << 4);
+                *reinterpret_cast<uint4*>(smem + OFF_A + so) = make_uint4(ohi[0], ohi[1], ohi[2], ohi[3]);
+                *reinterpret_cast<uint4*>(smem + OFF_ALO + so) = make_uint4(olo[0], olo[1], olo[2], olo[3]);
+                tmem_st8(xcol + v * 8, xo);
             }
-            // the block is complete: make it visible to the tensor core and the bulk copies, then
-            // hand it to this CTA's MMA and to the three siblings
+            tmem_wait_st();
+            // the blocks are complete: make them visible to the tensor core and the bulk copies,
+            // then hand them to this CTA's MMA and to the three siblings
             fence_proxy_async_smem();
             asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
             if (threadIdx.x == 0) {
                 mbar_arrive(bar_k(nt));
                 for (int rk = 1; rk < kClusterSize && !(a.withhold && blockIdx.x == 0); ++rk) {
                     const uint32_t peer = (uint32_t)((nt + rk) % kClusterSize);
-                    dsmem_copy(map_to_rank(kblk, peer), kblk, A_KBLK, map_to_rank(bar_k(nt), peer));
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+                        const uint32_t blk = sbase + (part ? OFF_ALO : OFF_A) + nt * A_KBLK;
+                        dsmem_copy(map_to_rank(blk, peer), blk, A_KBLK, map_to_rank(bar_k(nt), peer));
+                    }
                 }
             }
             // history: oldest out, x in (after the hand-off, so that no fence waits for these)
+            if (live) {
+                __nv_bfloat16* tw = a.tail + (size_t)b * kHist * W + cbase;
 #pragma unroll
-            for (int k = 0; k < kConvUnits; ++k) {
-                const int bk = mt * MT + k * (kEpiThreads / 8) + (threadIdx.x >> 3);
-                if (bk < a.B) {
-                    __nv_bfloat16* tl = a.tail + (size_t)bk * kHist * W + ch0 + g8 * 8;
-                    *reinterpret_cast<uint4*>(tl) = t1[k];
-                    *reinterpret_cast<uint4*>(tl + W) = t2[k];
-                    *reinterpret_cast<uint4*>(tl + 2 * W) = xv[k];
+                for (int v = 0; v < 2; ++v) {
+                    *reinterpret_cast<uint4*>(tw + 8 * v) = t1[v];
+                    *reinterpret_cast<uint4*>(tw + W + 8 * v) = t2[v];
+                    *reinterpret_cast<uint4*>(tw + 2 * W + 8 * v) = xv[v];
                 }
             }
         }
 
+        // ================================ weights to fp16 ======================================
+        // in place, 16 bytes a step; the tile's layout does not matter to an element-wise pass
+        {
+            const bool okw = wait_bounded(bar_w, 0, a, abort, 5);
+            if (okw) {
+                uint4* wt = reinterpret_cast<uint4*>(smem + OFF_BA);
+#pragma unroll 4
+                for (int i = threadIdx.x; i < (int)(2 * B_BYTES / 16); i += kEpiThreads) {
+                    uint4 v = wt[i];
+                    v.x = pack_f16x2(bf16lo(v.x), bf16hi(v.x));
+                    v.y = pack_f16x2(bf16lo(v.y), bf16hi(v.y));
+                    v.z = pack_f16x2(bf16lo(v.z), bf16hi(v.z));
+                    v.w = pack_f16x2(bf16lo(v.w), bf16hi(v.w));
+                    wt[i] = v;
+                }
+            }
+            fence_proxy_async_smem();
+            asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+            if (threadIdx.x == 0) mbar_arrive(bar_wc);   // also after a failed wait: the MMA warp drains
+        }
+
         // ================================ update ===============================================
-        // thread = row r of the tile, channels [16 cg, 16 cg + 16) of its 64; h, y and the conv
-        // output are read from (and h, out written back to) the swizzled shared tiles
-        const int q = warp & 3, cg = warp >> 2;           // lane quarter, channel quarter of the tile
-        const int r = q * 32 + lane;                      // row within the tile
-        const int b = mt * MT + r;
-        const bool rst = b < a.B && a.reset && a.reset[b];
-        const float gk1 = a.gelu_tanh ? 2.0f * 0.79788456080286535588f : 2.0f * 0.79879267f;
-        const float gk3 = a.gelu_tanh ? 8.0f * 0.044715f * 0.79788456080286535588f : 8.0f * 0.03528805f;
-        const uint32_t sw = (uint32_t)(r & 7);
         // GeLU(y) while the siblings' blocks arrive and the tensor cores run
-        const bool ok_hy = __all_sync(0xffffffffu, wait_bounded(bar_hy, 0, a, abort, 4));
+        const bool ok_y = __all_sync(0xffffffffu, wait_bounded(bar_y, 0, a, abort, 4));
         float gg[kEpiCh];
 #pragma unroll
         for (int v = 0; v < kEpiCh / 8; ++v) {
@@ -399,43 +402,27 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
                                                              ((((uint32_t)(cg * 2 + v)) ^ sw) << 4));
             const uint32_t* yw = reinterpret_cast<const uint32_t*>(&yq);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float hy = 0.5f * ((e & 1) ? bf16hi(yw[e >> 1]) : bf16lo(yw[e >> 1]));
-                const float t = tanh_approx(hy * fmaf(hy * hy, gk3, gk1));
-                gg[v * 8 + e] = fmaf(hy, t, hy);          // y Phi(y) in the tanh form
-            }
+            for (int e = 0; e < 8; ++e)
+                gg[v * 8 + e] = gelu1((e & 1) ? bf16hi(yw[e >> 1]) : bf16lo(yw[e >> 1]), a.gelu_tanh);
+        }
+        if (rst) {                                        // the state restarts from zero
+#pragma unroll
+            for (int i = 0; i < kEpiCh; ++i) hv[i] = 0.f;
         }
         // uniform across the warp: the TMEM loads below are warp-collective
-        const bool ok = __all_sync(0xffffffffu, ok_hy && wait_bounded(bar_acc, 0, a, abort, 2));
+        const bool ok = __all_sync(0xffffffffu, ok_y && wait_bounded(bar_acc, 0, a, abort, 2));
         tc_fence_after();
-        const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + cg * kEpiCh;
+        const uint32_t taddr = tmem + lane_off + cg * kEpiCh;
 #pragma unroll
         for (int v = 0; v < kEpiCh / 8; ++v) {            // 8 channels per step
-            float ga[8], gx[8];
+            float ga[8], gx[8], xc[8];
             tmem_ld8(taddr + v * 8, ga);
             tmem_ld8(taddr + NT + v * 8, gx);
+            tmem_ld8(xcol + v * 8, xc);
             tmem_wait_ld();
             if (!ok) continue;
             const int c8 = cg * 2 + v;                    // 8-channel chunk of the tile
-            // conv output: chunk c8 of row r in this CTA's K block
-            const uint32_t xo = OFF_A + nt * A_KBLK + (uint32_t)(r >> 3) * 1024 + sw * 128 + (((uint32_t)c8 ^ sw) << 4);
-            // h: 4-channel chunks 2 c8 and 2 c8 + 1, in the 32-channel box c8 / 4
-            const uint32_t hrow = OFF_H + (uint32_t)(c8 >> 2) * H_BOX + (uint32_t)r * 128;
-            const uint32_t ho0 = hrow + ((((uint32_t)(2 * c8) & 7) ^ sw) << 4);
-            const uint32_t ho1 = hrow + ((((uint32_t)(2 * c8 + 1) & 7) ^ sw) << 4);
-            // out, in the place of y
-            const uint32_t yo = OFF_Y + (uint32_t)r * 128 + (((uint32_t)c8 ^ sw) << 4);
-            const uint4 xq = *reinterpret_cast<const uint4*>(smem + xo);
-            float4 h0 = *reinterpret_cast<const float4*>(smem + ho0);
-            float4 h1 = *reinterpret_cast<const float4*>(smem + ho1);
-            if (rst) {                                    // the state restarts from zero
-                h0 = make_float4(0.f, 0.f, 0.f, 0.f);
-                h1 = h0;
-            }
-            float hv[8];
-            hv[0] = h0.x; hv[1] = h0.y; hv[2] = h0.z; hv[3] = h0.w;
-            hv[4] = h1.x; hv[5] = h1.y; hv[6] = h1.z; hv[7] = h1.w;
-            const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xq);
+            const uint32_t yo = OFF_Y + (uint32_t)r * 128 + (((uint32_t)c8 ^ sw) << 4);   // out, in the place of y
             uint32_t ow[4];
 #pragma unroll
             for (int e2 = 0; e2 < 4; ++e2) {
@@ -444,43 +431,30 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
                 for (int e1 = 0; e1 < 2; ++e1) {
                     const int e = 2 * e2 + e1;
                     const int jc = c8 * 8 + e;            // column within the tile
-                    const float xcv = e1 ? bf16hi(xw[e2]) : bf16lo(xw[e2]);
-                    const float hk = s_hk[jc];
-                    const float da = fmaf(ga[e], 0.5f, s_ba[jc]);
-                    const float dx = fmaf(gx[e], 0.5f, s_bx[jc]);
-                    const float l = fmaf(tanh_approx(da), hk, hk);
-                    float em;
-                    if (l > -0.125f) {
-                        float pp = fmaf(l, 1.0f / 24.0f, 1.0f / 6.0f);
-                        pp = fmaf(l, pp, 0.5f);
-                        pp = fmaf(l, pp, 1.0f);
-                        em = l * pp;
-                    } else {
-                        em = ex2_approx(l * 1.4426950408889634f) - 1.0f;
-                    }
-                    const float at = 1.0f + em;
-                    const float bh = sqrt_approx(em * fmaf(em, -0.25f, -0.5f));
-                    const float w = bh * xcv;
-                    const float u = fmaf(w, tanh_approx(dx), w);
-                    const float hn = fmaf(at, hv[e], u);
-                    hv[e] = hn;
+                    float at, u;
+                    gates1<false>(ga[e], gx[e], s_nba[jc], s_nbx[jc], s_K[jc], xc[e], at, u);
+                    const float hn = fmaf(at, hv[v * 8 + e], u);
+                    hv[v * 8 + e] = hn;
                     o[e1] = hn * gg[v * 8 + e];
                 }
                 ow[e2] = pack_bf16x2(o[0], o[1]);
             }
-            *reinterpret_cast<float4*>(smem + ho0) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-            *reinterpret_cast<float4*>(smem + ho1) = make_float4(hv[4], hv[5], hv[6], hv[7]);
             *reinterpret_cast<uint4*>(smem + yo) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         }
-        // the tiles are complete: store h and out (rows past the batch are clipped by the maps)
+        // the state, straight from registers (only rows of the batch)
+        if (ok && live) {
+            float4* hp = reinterpret_cast<float4*>(a.h + (size_t)b * W + cbase);
+#pragma unroll
+            for (int i = 0; i < kEpiCh / 4; ++i)
+                hp[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+        }
+        // the out tile is complete: store it (rows past the batch are clipped by the map)
         fence_proxy_async_smem();
         asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
         if (threadIdx.x == 0 && !*abort) {
-            tma_store_2d(&map_h, sbase + OFF_H, ch0, mt * MT);
-            tma_store_2d(&map_h, sbase + OFF_H + H_BOX, ch0 + 32, mt * MT);
             tma_store_2d(&map_out, sbase + OFF_Y, ch0, mt * MT);
             bulk_commit();
-            bulk_wait_read0();                            // the shared tiles stay until read
+            bulk_wait_read0();                            // the shared tile stays until read
         }
     }
     tc_fence_before();
@@ -516,10 +490,9 @@ cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, cons
     if (fused_decode_workspace(d) > ws_bytes) return cudaErrorInvalidValue;
     const int B = d->batch, H = d->heads;
     const uint64_t W = (uint64_t)H * DH;
-    CUtensorMap mwa, mwx, mh, my, mo;
+    CUtensorMap mwa, mwx, my, mo;
     if (!tc::make_map_2d_sw128(&mwa, p->w_a, DH, W, DH * 2, NT, 64) ||
         !tc::make_map_2d_sw128(&mwx, p->w_x, DH, W, DH * 2, NT, 64) ||
-        !tc::make_map_2d_sw128_elem(&mh, st->h, 4, W, (uint64_t)B, W * 4, 32, MT) ||
         !tc::make_map_2d_sw128_elem(&my, y, 2, W, (uint64_t)B, W * 2, NT, MT) ||
         !tc::make_map_2d_sw128_elem(&mo, out, 2, W, (uint64_t)B, W * 2, NT, MT))
         return cudaErrorInvalidValue;
@@ -527,6 +500,7 @@ cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, cons
     if (e != cudaSuccess) return e;
     Args a;
     a.B = B; a.H = H; a.mtiles = (B + MT - 1) / MT;
+    a.h = st->h;
     a.x = static_cast<const __nv_bfloat16*>(x);
     a.tail = static_cast<__nv_bfloat16*>(st->conv_tail);
     a.conv_w = p->conv_w; a.conv_b = p->conv_b;
@@ -550,7 +524,7 @@ cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, cons
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, mwa, mwx, mh, my, mo, a);
+    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, mwa, mwx, my, mo, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -1,0 +1,414 @@
+// gemm.cu -- batched bf16 GEMM on the 5th-generation tensor cores (sm_100a) for the dense
+// contractions around the recurrence: the transposed gate contraction and the weight gradient
+// of the backward pass.
+//
+//   C[b][m][n] (fp32) = sum over the operand pairs p of sum_k A_p[b][m][k] B_p[b][k][n]
+//                       (+ Cadd[b][m][n]),  for m < M, n < N;
+// with up to four operand pairs (K ranges accumulated into one C: both gates, or the hi and lo
+// bf16 parts of an fp32 operand) and an
+// optional split of K into `splits` slices whose partial sums go to separate C slices (a
+// reduction in fixed order follows, so results are bitwise repeatable).
+//
+//   * A is [M x K] "K-major" (k contiguous: element (m, k) at a_row[m] + k) or "M-major" (m
+//     contiguous: element (m, k) at k * ld + m); B likewise N x K, "K-major" or "N-major".  The
+//     operands are read by TMA in 128-byte swizzled tiles straight from the caller's tensors
+//     (2-D maps; the batch index adds a fixed row or column offset);
+//   * a persistent CTA per SM walks output tiles of 128 x 128 (batch, m-tile, n-tile, k-slice);
+//     one warp loads K blocks of 64 through a 4-stage ring, one thread issues tcgen05.mma
+//     (M = 128, N = 128, K = 16 per instruction) into one of two TMEM accumulators, and 4
+//     epilogue warps (thread = row of the tile) read the other accumulator, add Cadd and store.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+#include "tma_maps.h"
+
+namespace rglru {
+namespace gm {
+
+using namespace sm100;
+
+constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int STAGES = 4;
+constexpr uint32_t TILE_A = BM * BK * 2;           // 16384
+constexpr uint32_t TILE_B = BN * BK * 2;           // 16384
+constexpr uint32_t STAGE_BYTES = TILE_A + TILE_B;
+constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
+constexpr int kEpiWarps = 4, kWarpTma = 4, kWarpMma = 5;
+constexpr int kThreads = 6 * 32;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int kMaxPairs = 4;
+
+struct Pair {
+    int K;               // K of this pair (a multiple of 64)
+    int a_kmajor;        // 1: A (m, k) at row m, column k of its map; 0: row k, column m
+    int b_kmajor;        // 1: B (n, k) at row n, column k;             0: row k, column n
+    int a_boff_row, a_boff_col, a_bstep_row, a_bstep_col;   // A's map coordinates: boff + b * bstep
+    int b_boff_row, b_boff_col, b_bstep_row, b_bstep_col;
+};
+
+struct Args {
+    int M, N, batch, splits, npairs;
+    int mt, nt;          // tiles along M and N
+    Pair p[kMaxPairs];
+    float* C;            // C[split][b][m][n] at C + split * c_split + b * c_bstride + m * c_ld + n
+    long long c_ld, c_bstride, c_split;
+    const float* Cadd;   // same indexing without the split, or nullptr (only with splits == 1)
+    long long add_ld, add_bstride;
+    __nv_bfloat16* C16;  // if set: C is written here as bf16 (round to nearest even) instead
+    DeviceStatus* status;
+    unsigned long long timeout_ns;
+};
+
+// K blocks of one output tile: the blocks of pair 0, then those of pair 1, ..., cut into
+// `splits` equal slices (the last may be shorter)
+struct KPlan {
+    int total, per;      // blocks in all, blocks per slice
+};
+__host__ __device__ inline KPlan kplan(const Args& a) {
+    KPlan k;
+    k.total = 0;
+    for (int i = 0; i < a.npairs; ++i) k.total += a.p[i].K / BK;
+    k.per = (k.total + a.splits - 1) / a.splits;
+    return k;
+}
+// the pair of K block kb and the block's index within that pair
+__device__ __forceinline__ int pair_of(const Args& a, int kb, int& local) {
+    int i = 0;
+    while (i + 1 < a.npairs && kb >= a.p[i].K / BK) {
+        kb -= a.p[i].K / BK;
+        ++i;
+    }
+    local = kb;
+    return i;
+}
+
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, const Args& a, volatile int* abort, unsigned where) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (*abort) return false;
+        if (*(volatile unsigned*)&a.status->code != 0) {
+            *abort = 1;
+            return false;
+        }
+        if (globaltimer_ns() - t0 > a.timeout_ns) {
+            latch_status(a.status, RGLRU_ERR_TIMEOUT, where, blockIdx.x, parity);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool wait_b(uint32_t bar, uint32_t parity, const Args& a, volatile int* abort, unsigned where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_slow(bar, parity, a, abort, where);
+}
+
+// Shared-memory descriptors (128-byte swizzle) of a 128-row, 64-wide tile: K-major (rows of
+// 128 B = 64 K, 8-row atoms 1024 B apart) or MN-major (two 64-wide MN atoms of 64 K-rows each,
+// 8192 B apart; 8-row K groups 1024 B apart)
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+    d |= (uint64_t)(8192 >> 4) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+// instruction descriptor: fp32 accumulator, bf16 A and B, their majorness, M x N
+__device__ __forceinline__ uint32_t idesc(int a_mn, int b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUtensorMap mb0,
+            const __grid_constant__ CUtensorMap ma1, const __grid_constant__ CUtensorMap mb1,
+            const __grid_constant__ CUtensorMap ma2, const __grid_constant__ CUtensorMap mb2,
+            const __grid_constant__ CUtensorMap ma3, const __grid_constant__ CUtensorMap mb3, const Args a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + OFF_BAR;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto acc_full = [&](int i) { return bar0 + 8u * (2 * STAGES + i); };
+    auto acc_empty = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 + i); };
+    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 8 * (2 * STAGES + 5));
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_BAR + 8 * (2 * STAGES + 5) + 16);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(acc_full(i), 1);
+            mbar_init(acc_empty(i), kEpiWarps);
+        }
+        mbar_init(acc_empty(0) + 8u * 2, 1);                  // mma_done
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32((const void*)tmem_base_s), TMEM_COLS);
+        tmem_relinquish();
+    }
+    const CUtensorMap* mas[kMaxPairs] = {&ma0, &ma1, &ma2, &ma3};
+    const CUtensorMap* mbs[kMaxPairs] = {&mb0, &mb1, &mb2, &mb3};
+    if (warp == kWarpTma && lane == 0) {
+        for (int i = 0; i < a.npairs; ++i) {
+            prefetch_tensormap(mas[i]);
+            prefetch_tensormap(mbs[i]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_s;
+    const KPlan kp = kplan(a);
+    const int ntiles = a.batch * a.mt * a.nt * a.splits;
+
+    auto tile_of = [&](int t, int& b, int& m0, int& n0, int& sp) {
+        sp = t % a.splits;
+        t /= a.splits;
+        const int ni = t % a.nt;
+        t /= a.nt;
+        const int mi = t % a.mt;
+        b = t / a.mt;
+        m0 = mi * BM;
+        n0 = ni * BN;
+    };
+
+    if (warp == kWarpTma) {
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                int b, m0, n0, sp;
+                tile_of(t, b, m0, n0, sp);
+                const int k_beg = sp * kp.per, k_end = min(kp.total, k_beg + kp.per);
+                for (int kb = k_beg; kb < k_end; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (!wait_b(empty(s), ((it / STAGES) & 1) ^ 1, a, abort, 1)) {
+                        ok = false;
+                        break;
+                    }
+                    int local;
+                    const int pi = pair_of(a, kb, local);
+                    const Pair& p = a.p[pi];
+                    const int k0 = local * BK;
+                    const CUtensorMap* ma = mas[pi];
+                    const CUtensorMap* mb = mbs[pi];
+                    const uint32_t sa = sbase + s * STAGE_BYTES, sb = sa + TILE_A;
+                    const int ar = p.a_boff_row + b * p.a_bstep_row, ac = p.a_boff_col + b * p.a_bstep_col;
+                    const int br = p.b_boff_row + b * p.b_bstep_row, bc = p.b_boff_col + b * p.b_bstep_col;
+                    mbar_arrive_expect_tx(full(s), STAGE_BYTES);
+                    if (p.a_kmajor) {
+                        tma_load_2d(sa, ma, ac + k0, ar + m0, full(s));
+                    } else {
+                        tma_load_2d(sa, ma, ac + m0, ar + k0, full(s));
+                        tma_load_2d(sa + 8192, ma, ac + m0 + 64, ar + k0, full(s));
+                    }
+                    if (p.b_kmajor) {
+                        tma_load_2d(sb, mb, bc + k0, br + n0, full(s));
+                    } else {
+                        tma_load_2d(sb, mb, bc + n0, br + k0, full(s));
+                        tma_load_2d(sb + 8192, mb, bc + n0 + 64, br + k0, full(s));
+                    }
+                }
+            }
+            // never leave the CTA with a bulk copy still writing its shared memory
+            const uint64_t t0 = globaltimer_ns();
+            for (int i = it - STAGES; i < it; ++i)
+                if (i >= 0)
+                    while (!mbar_try_wait_sleep(full(i % STAGES), (i / STAGES) & 1, 20000u) &&
+                           globaltimer_ns() - t0 < a.timeout_ns) {
+                    }
+        }
+    } else if (warp == kWarpMma) {
+        // the whole warp follows the waits (warp-uniform control flow); one elected lane issues,
+        // so that the descriptors stay uniform and consecutive MMAs issue back to back
+        const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+        int it = 0, tc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tc) {
+            int b, m0, n0, sp;
+            tile_of(t, b, m0, n0, sp);
+            const int k_beg = sp * kp.per, k_end = min(kp.total, k_beg + kp.per);
+            const int ai = tc & 1;
+            if (!__all_sync(0xffffffffu, wait_b(acc_empty(ai), ((tc >> 1) & 1) ^ 1, a, abort, 2))) break;
+            tc_fence_after();
+            const uint32_t d = tm + ai * BN;
+            for (int kb = k_beg; kb < k_end; ++kb, ++it) {
+                const int s = it % STAGES;
+                if (!__all_sync(0xffffffffu, wait_b(full(s), (it / STAGES) & 1, a, abort, 3))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                int local;
+                const Pair& p = a.p[pair_of(a, kb, local)];
+                const uint32_t id = idesc(p.a_kmajor ? 0 : 1, p.b_kmajor ? 0 : 1);
+                const uint32_t sa = sbase + s * STAGE_BYTES, sb = sa + TILE_A;
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        // K step kk: 32 bytes along a K-major row, or 16 K-rows (2048 B) of an
+                        // MN-major tile
+                        const uint64_t ad = p.a_kmajor ? desc_k_sw128(sa + kk * 32) : desc_mn_sw128(sa + kk * 2048);
+                        const uint64_t bd = p.b_kmajor ? desc_k_sw128(sb + kk * 32) : desc_mn_sw128(sb + kk * 2048);
+                        mma_ss(d, ad, bd, id, (kb > k_beg || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(empty(s));
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (elect_one()) mma_commit(acc_full(ai));
+            __syncwarp();
+        }
+        // every MMA of this warp has finished before TMEM is released
+        if (elect_one()) mma_commit(acc_empty(0) + 8u * 2);     // the mma_done barrier after acc_empty[1]
+        __syncwarp();
+        if (lane == 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait_sleep(acc_empty(0) + 8u * 2, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+        }
+        __syncwarp();
+    } else {
+        // ================================ epilogue: thread = row of the tile ==================
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        int tc = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+            int b, m0, n0, sp;
+            tile_of(t, b, m0, n0, sp);
+            const int ai = tc & 1;
+            if (!__all_sync(0xffffffffu, wait_b(acc_full(ai), (tc >> 1) & 1, a, abort, 4))) break;
+            tc_fence_after();
+            const int m = m0 + r;
+            // a K slice without blocks (more slices than K blocks) contributes zeros: its
+            // accumulator was never written
+            const bool no_k = sp * kp.per >= kp.total;
+            const long long coff = sp * a.c_split + b * a.c_bstride + (long long)m * a.c_ld + n0;
+            float* crow = a.C + coff;
+            __nv_bfloat16* crow16 = a.C16 ? a.C16 + coff : nullptr;
+            const float* arow = a.Cadd ? a.Cadd + b * a.add_bstride + (long long)m * a.add_ld + n0 : nullptr;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                float v[16];
+                if (no_k) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                } else {
+                    tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + ai * BN + c0, v);
+                    tmem_wait_ld();
+                }
+                if (m < a.M && crow16) {
+                    const int nn = a.N - (n0 + c0);
+                    if (nn >= 16) {
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            __nv_bfloat162 p2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+                            pk[j] = *reinterpret_cast<uint32_t*>(&p2);
+                        }
+                        *reinterpret_cast<uint4*>(crow16 + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        *reinterpret_cast<uint4*>(crow16 + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    } else {
+                        for (int j = 0; j < nn; ++j) crow16[c0 + j] = __float2bfloat16_rn(v[j]);
+                    }
+                } else if (m < a.M) {
+                    const int nn = a.N - (n0 + c0);
+                    if (nn >= 16) {
+#pragma unroll
+                        for (int j = 0; j < 16; j += 4) {
+                            float4 o = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                            if (arow) {
+                                const float4 ad = *reinterpret_cast<const float4*>(arow + c0 + j);
+                                o.x += ad.x; o.y += ad.y; o.z += ad.z; o.w += ad.w;
+                            }
+                            *reinterpret_cast<float4*>(crow + c0 + j) = o;
+                        }
+                    } else {
+                        for (int j = 0; j < nn; ++j) crow[c0 + j] = v[j] + (arow ? arow[c0 + j] : 0.f);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty(ai));
+        }
+        tmem_wait_ld();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// one 2-D bf16 map over a [rows x cols] row-major tensor (row pitch ld elements), box 64 x box_rows
+bool map_2d(CUtensorMap* m, const void* base, long long rows, long long cols, long long ld, int box_rows) {
+    return tc::make_map_2d_sw128(m, base, (uint64_t)cols, (uint64_t)rows, (uint64_t)ld * 2, 64, (uint32_t)box_rows);
+}
+
+}  // namespace gm
+
+size_t gemm_smem_bytes() { return gm::SMEM_BYTES; }
+
+// See kernels.h for the operand description.
+cudaError_t launch_gemm(const GemmOperands& g, cudaStream_t s) {
+    using namespace gm;
+    if (g.npairs < 1 || g.npairs > kMaxPairs || g.M <= 0 || g.N <= 0 || g.batch <= 0 || g.splits <= 0) return cudaErrorInvalidValue;
+    if (g.N % 16 != 0 || (g.splits > 1 && g.Cadd)) return cudaErrorInvalidValue;
+    CUtensorMap maps[2 * kMaxPairs];
+    Args a{};
+    a.M = g.M; a.N = g.N; a.batch = g.batch; a.splits = g.splits; a.npairs = g.npairs;
+    a.mt = (g.M + BM - 1) / BM; a.nt = (g.N + BN - 1) / BN;
+    for (int i = 0; i < kMaxPairs; ++i) {
+        const GemmPair& gp = g.p[i < g.npairs ? i : 0];
+        if (gp.K <= 0 || gp.K % BK != 0) return cudaErrorInvalidValue;
+        // a K-major operand's tile is 128 rows of 64 K; an MN-major one 64 K-rows of 2 x 64
+        if (!map_2d(&maps[2 * i], gp.a, gp.a_rows, gp.a_cols, gp.a_ld, gp.a_kmajor ? BM : BK) ||
+            !map_2d(&maps[2 * i + 1], gp.b, gp.b_rows, gp.b_cols, gp.b_ld, gp.b_kmajor ? BN : BK))
+            return cudaErrorInvalidValue;
+        a.p[i].K = gp.K;
+        a.p[i].a_kmajor = gp.a_kmajor; a.p[i].b_kmajor = gp.b_kmajor;
+        a.p[i].a_boff_row = gp.a_boff_row; a.p[i].a_boff_col = gp.a_boff_col;
+        a.p[i].a_bstep_row = gp.a_bstep_row; a.p[i].a_bstep_col = gp.a_bstep_col;
+        a.p[i].b_boff_row = gp.b_boff_row; a.p[i].b_boff_col = gp.b_boff_col;
+        a.p[i].b_bstep_row = gp.b_bstep_row; a.p[i].b_bstep_col = gp.b_bstep_col;
+    }
+    a.C = g.C; a.c_ld = g.c_ld; a.c_bstride = g.c_bstride; a.c_split = g.c_split;
+    a.Cadd = g.Cadd; a.add_ld = g.add_ld; a.add_bstride = g.add_bstride;
+    a.C16 = g.C16;
+    if (a.C16 && (a.Cadd || g.splits > 1 || g.c_ld % 8 != 0)) return cudaErrorInvalidValue;
+    a.status = g.status;
+    a.timeout_ns = 1000000000ull;
+    cudaError_t e = set_smem_once(gemm_kernel, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int ntiles = a.batch * a.mt * a.nt * a.splits;
+    const int grid = ntiles < sms ? ntiles : sms;
+    gemm_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6],
+                                                   maps[7], a);
+    return cudaGetLastError();
+}
+
+}  // namespace rglru

@@ -1,0 +1,690 @@
+// mqa.cu -- Griffin's local sliding-window multi-query attention on sm_100a (bf16, head_dim 256).
+//
+// "Griffin Guide: RecurrentGemma, RG-LRU & Hybrid Attention", "2. Local Sliding-Window
+// Multi-Query Attention (MQA)" and "3. Bounding the Key-Value Cache Footprint"; the "Griffin"
+// notes, "Local Attention Path":  H query heads share one key head and one value head; token t
+// attends to N(t) = {i : t - w < i <= t}:  y_t = sum_{i in N(t)} softmax_i(s q_t . k_i) v_i, with
+// rotary position embeddings on queries and keys; decoding keeps the last w keys / values in a
+// ring buffer (slot = position mod w).  RoPE turns the pairs (j, j + d/2) by p base^(-2j/d).
+//
+//   * mqa_rope_kernel: rotates q and k (angles in fp64, reduced mod 2 pi, then fp32 sine and
+//     cosine) into bf16 copies; copies the last w rotated keys and values into the ring cache;
+//   * mqa_prefill_kernel: one CTA per (row, head, 128 queries), in the manner of
+//     FlashAttention: the query tile sits in TMEM as the A operand (TS form); per 64-key tile of
+//     the window, S = Q K^T (tcgen05.mma, M = 128, N = 64, K = 256) goes to one of two TMEM
+//     buffers; 4 softmax warps (thread = query) mask the window, take exp2 against a running
+//     reference maximum that moves only when the maximum grows by more than 2^8 (then the
+//     accumulator is rescaled), write P in bf16 to shared memory; O += P V (M = 128, N = 256,
+//     K = 64) accumulates in TMEM; the S of the next tile overlaps the softmax of this one;
+//   * mqa_decode_kernel: one token per row against the ring: CTAs split the window, each keeps
+//     (max, sum, sum of p v) per head over its part (CUDA cores: the step is bound by the cache
+//     read); mqa_merge_kernel combines the parts.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+#include "tma_maps.h"
+
+namespace rglru {
+namespace mq {
+
+using namespace sm100;
+
+constexpr int D = 256;                 // head dim (the tensor-core path)
+constexpr int BQ = 128;                // queries per CTA (MMA M)
+constexpr int BKV = 64;                // keys per tile (MMA N of S, K of P V)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- rotary embedding ----------
+struct RopeArgs {
+    int B, T, H, w, pos0;
+    float base;
+    const __nv_bfloat16* q;            // [B, T, H, d]
+    const __nv_bfloat16* k;            // [B, T, d]
+    const __nv_bfloat16* v;            // [B, T, d]
+    __nv_bfloat16* q_rot;
+    __nv_bfloat16* k_rot;
+    __nv_bfloat16* cache;              // [B][2][w][d] or nullptr
+};
+
+__device__ __forceinline__ void rot_pair(float x1, float x2, double ang, float& o1, float& o2) {
+    const double two_pi = 6.283185307179586476925286766559;
+    double r = fmod(ang, two_pi);
+    float s, c;
+    sincosf((float)r, &s, &c);
+    o1 = x1 * c - x2 * s;
+    o2 = x2 * c + x1 * s;
+}
+
+// thread = (row b, token t, j < d/2) over the H query heads and the key
+__global__ void mqa_rope_kernel(RopeArgs a) {
+    const int j = threadIdx.x;                       // 0 .. d/2 - 1
+    const int t = blockIdx.x, b = blockIdx.y;
+    const int p = a.pos0 + t;
+    const double ang = (double)p * pow((double)a.base, -2.0 * j / D);
+    const size_t qrow = ((size_t)b * a.T + t) * a.H * D;
+    for (int h = 0; h < a.H; ++h) {
+        const size_t e = qrow + (size_t)h * D;
+        float o1, o2;
+        rot_pair(__bfloat162float(a.q[e + j]), __bfloat162float(a.q[e + j + D / 2]), ang, o1, o2);
+        a.q_rot[e + j] = __float2bfloat16_rn(o1);
+        a.q_rot[e + j + D / 2] = __float2bfloat16_rn(o2);
+    }
+    const size_t ke = ((size_t)b * a.T + t) * D;
+    float o1, o2;
+    rot_pair(__bfloat162float(a.k[ke + j]), __bfloat162float(a.k[ke + j + D / 2]), ang, o1, o2);
+    const __nv_bfloat16 r1 = __float2bfloat16_rn(o1), r2 = __float2bfloat16_rn(o2);
+    a.k_rot[ke + j] = r1;
+    a.k_rot[ke + j + D / 2] = r2;
+    if (a.cache && t >= a.T - a.w) {                 // the last w positions stay for decoding
+        const int slot = p % a.w;
+        __nv_bfloat16* ck = a.cache + ((size_t)b * 2 * a.w + slot) * D;
+        __nv_bfloat16* cv = a.cache + ((size_t)b * 2 * a.w + a.w + slot) * D;
+        ck[j] = r1;
+        ck[j + D / 2] = r2;
+        cv[j] = a.v[ke + j];
+        cv[j + D / 2] = a.v[ke + j + D / 2];
+    }
+}
+
+// one decode token per row at position pos[b]: q_rot [B, H, d]; the rotated key and the value
+// go into ring slot pos mod w
+struct RopeDecArgs {
+    int B, H, w;
+    float base;
+    const int* pos;
+    const __nv_bfloat16* q;            // [B, H, d]
+    const __nv_bfloat16* k;            // [B, d]
+    const __nv_bfloat16* v;
+    __nv_bfloat16* q_rot;
+    __nv_bfloat16* cache;              // [B][2][w][d]
+};
+
+__global__ void mqa_rope_decode_kernel(RopeDecArgs a) {
+    const int j = threadIdx.x, b = blockIdx.x;
+    const int p = a.pos[b];
+    const double ang = (double)p * pow((double)a.base, -2.0 * j / D);
+    for (int h = 0; h < a.H; ++h) {
+        const size_t e = ((size_t)b * a.H + h) * D;
+        float o1, o2;
+        rot_pair(__bfloat162float(a.q[e + j]), __bfloat162float(a.q[e + j + D / 2]), ang, o1, o2);
+        a.q_rot[e + j] = __float2bfloat16_rn(o1);
+        a.q_rot[e + j + D / 2] = __float2bfloat16_rn(o2);
+    }
+    float o1, o2;
+    rot_pair(__bfloat162float(a.k[(size_t)b * D + j]), __bfloat162float(a.k[(size_t)b * D + j + D / 2]), ang, o1, o2);
+    const int slot = p % a.w;
+    __nv_bfloat16* ck = a.cache + ((size_t)b * 2 * a.w + slot) * D;
+    __nv_bfloat16* cv = a.cache + ((size_t)b * 2 * a.w + a.w + slot) * D;
+    ck[j] = __float2bfloat16_rn(o1);
+    ck[j + D / 2] = __float2bfloat16_rn(o2);
+    cv[j] = a.v[(size_t)b * D + j];
+    cv[j + D / 2] = a.v[(size_t)b * D + j + D / 2];
+}
+
+// ---------------------------------------------------------------- prefill attention ---------
+struct PrefArgs {
+    int B, T, H, w;
+    float scale_log2;                  // score scale * log2(e)
+    __nv_bfloat16* out;                // [B, T, H, d]
+    DeviceStatus* status;
+    unsigned long long timeout_ns;
+};
+
+constexpr uint32_t Q_BYTES = BQ * D * 2;             // 65536, row-major staging of the query tile
+constexpr uint32_t KT_BYTES = BKV * D * 2;           // 32768: 4 K-blocks of [64 keys x 128 B]
+constexpr uint32_t VT_BYTES = BKV * D * 2;           // 32768: 4 atoms of [64 keys x 64 d] (MN-major)
+constexpr uint32_t P_BYTES = BQ * BKV * 2;           // 16384: [128 queries x 64 keys], 128B swizzle
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;          // 2 stages
+constexpr uint32_t OFF_V = OFF_K + 2 * KT_BYTES;     // 2 stages
+constexpr uint32_t OFF_P = OFF_V + 2 * VT_BYTES;
+constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// TMEM: [0,128) Q (A operand, bf16 pairs), [128,256) S double buffer, [256,512) O (fp32)
+constexpr uint32_t TM_Q = 0, TM_S = 128, TM_O = 256;
+constexpr int kSmWarps = 4, kWarpTma = 4, kWarpMma = 5, kThreads = 6 * 32;
+
+struct Bars {
+    uint32_t base;
+    __device__ __forceinline__ uint32_t q_full() const { return base; }
+    __device__ __forceinline__ uint32_t q_tmem() const { return base + 8; }
+    __device__ __forceinline__ uint32_t k_full(int i) const { return base + 16 + 8u * i; }
+    __device__ __forceinline__ uint32_t k_empty(int i) const { return base + 32 + 8u * i; }
+    __device__ __forceinline__ uint32_t v_full(int i) const { return base + 48 + 8u * i; }
+    __device__ __forceinline__ uint32_t v_empty(int i) const { return base + 64 + 8u * i; }
+    __device__ __forceinline__ uint32_t s_full(int i) const { return base + 80 + 8u * i; }
+    __device__ __forceinline__ uint32_t s_free(int i) const { return base + 96 + 8u * i; }
+    __device__ __forceinline__ uint32_t p_full() const { return base + 112; }
+    __device__ __forceinline__ uint32_t o_done() const { return base + 120; }   // a P V finished
+    __device__ __forceinline__ uint32_t mma_done() const { return base + 128; }
+};
+
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, const PrefArgs& a, volatile int* abort, unsigned where) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (*abort) return false;
+        if (*(volatile unsigned*)&a.status->code != 0) {
+            *abort = 1;
+            return false;
+        }
+        if (globaltimer_ns() - t0 > a.timeout_ns) {
+            latch_status(a.status, RGLRU_ERR_TIMEOUT, where, blockIdx.x, parity);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool wait_b(uint32_t bar, uint32_t parity, const PrefArgs& a, volatile int* abort, unsigned where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_slow(bar, parity, a, abort, where);
+}
+
+// MN-major (128-byte swizzle) descriptor of the V tile: 4 atoms of 64 d-columns, 8192 B apart
+__device__ __forceinline__ uint64_t desc_v(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+    d |= (uint64_t)(8192 >> 4) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+__device__ __forceinline__ uint32_t idesc_mk(int n, int b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(BQ >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                   const __grid_constant__ CUtensorMap map_v, const PrefArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const Bars bars{sbase + OFF_BAR};
+    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 144);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_BAR + 160);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // blockIdx.x = query tile, y = head, z = row
+    const int t0 = blockIdx.x * BQ, h = blockIdx.y, b = blockIdx.z;
+    const int q_last = min(a.T, t0 + BQ) - 1;
+    const int k_lo = max(0, t0 - a.w + 1);                // first key any query of the tile sees
+    const int j0 = k_lo / BKV, j1 = q_last / BKV;         // key tiles [j0, j1]
+    const int ntiles = j1 - j0 + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bars.q_full(), 1);
+        mbar_init(bars.q_tmem(), kSmWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bars.k_full(i), 1);
+            mbar_init(bars.k_empty(i), 1);
+            mbar_init(bars.v_full(i), 1);
+            mbar_init(bars.v_empty(i), 1);
+            mbar_init(bars.s_full(i), 1);
+            mbar_init(bars.s_free(i), kSmWarps);
+        }
+        mbar_init(bars.p_full(), kSmWarps);
+        mbar_init(bars.o_done(), 1);
+        mbar_init(bars.mma_done(), 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == kWarpMma) {
+        tmem_alloc(smem_u32((const void*)tmem_base_s), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_s;
+
+    if (warp == kWarpTma) {
+        if (lane == 0) {
+            // query tile: rows (b, t0 .. t0 + 127, head h) of the [B T H, d] rotated queries
+            mbar_arrive_expect_tx(bars.q_full(), Q_BYTES);
+            for (int kb = 0; kb < D / 64; ++kb)
+                tma_load_3d(sbase + OFF_Q + kb * (BQ * 128), &map_q, kb * 64, h, b * a.T + t0, bars.q_full());
+            for (int j = 0; j < ntiles; ++j) {
+                const int s = j & 1;
+                const int key0 = (j0 + j) * BKV;
+                if (!wait_b(bars.k_empty(s), ((j >> 1) & 1) ^ 1, a, abort, 1)) break;
+                mbar_arrive_expect_tx(bars.k_full(s), KT_BYTES);
+                for (int kb = 0; kb < D / 64; ++kb)
+                    tma_load_2d(sbase + OFF_K + s * KT_BYTES + kb * (BKV * 128), &map_k, kb * 64, b * a.T + key0,
+                                bars.k_full(s));
+                if (!wait_b(bars.v_empty(s), ((j >> 1) & 1) ^ 1, a, abort, 2)) break;
+                mbar_arrive_expect_tx(bars.v_full(s), VT_BYTES);
+                for (int dn = 0; dn < D / 64; ++dn)
+                    tma_load_2d(sbase + OFF_V + s * VT_BYTES + dn * 8192, &map_v, dn * 64, b * a.T + key0,
+                                bars.v_full(s));
+            }
+            // no bulk copy may still be writing shared memory at the exit
+            const uint64_t tt = globaltimer_ns();
+            for (int j = ntiles - 2; j < ntiles; ++j)
+                if (j >= 0)
+                    while (!(mbar_try_wait(bars.k_full(j & 1), (j >> 1) & 1) &&
+                             mbar_try_wait(bars.v_full(j & 1), (j >> 1) & 1)) &&
+                           globaltimer_ns() - tt < a.timeout_ns) {
+                    }
+            while (!mbar_try_wait(bars.q_full(), 0) && globaltimer_ns() - tt < a.timeout_ns) {
+            }
+        }
+    } else if (warp == kWarpMma) {
+        // the whole warp follows the waits; one elected lane issues (warp-uniform operands)
+        const uint32_t id_s = idesc_mk(BKV, 0), id_o = idesc_mk(D, 1);
+        const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+        auto wait_w = [&](uint32_t bar, uint32_t par, unsigned where) {
+            return __all_sync(0xffffffffu, wait_b(bar, par, a, abort, where));
+        };
+        bool ok = wait_w(bars.q_tmem(), 0, 3);
+        tc_fence_after();
+        for (int j = 0; ok && j <= ntiles; ++j) {
+            if (j < ntiles) {                                // S_j = Q K_j^T
+                const int s = j & 1;
+                if (!wait_w(bars.k_full(s), (j >> 1) & 1, 4)) break;
+                if (!wait_w(bars.s_free(s), ((j >> 1) & 1) ^ 1, 5)) break;
+                tc_fence_after();
+                const uint32_t ds = tm + TM_S + s * BKV;
+                if (elect_one()) {
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint64_t bd = desc_k_sw128(sbase + OFF_K + s * KT_BYTES + (ks >> 2) * (BKV * 128) + (ks & 3) * 32);
+                        mma_ts(ds, tm + TM_Q + ks * 8, bd, id_s, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bars.s_full(s));
+                    mma_commit(bars.k_empty(s));
+                }
+                __syncwarp();
+            }
+            if (j >= 1) {                                    // O += P_{j-1} V_{j-1}
+                const int jj = j - 1, s = jj & 1;
+                if (!wait_w(bars.p_full(), jj & 1, 6)) break;
+                if (!wait_w(bars.v_full(s), (jj >> 1) & 1, 7)) break;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int ks = 0; ks < BKV / 16; ++ks) {
+                        const uint64_t ad = desc_k_sw128(sbase + OFF_P + ks * 32);
+                        const uint64_t bd = desc_v(sbase + OFF_V + s * VT_BYTES + ks * 2048);
+                        mma_ss(tm + TM_O, ad, bd, id_o, (jj > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bars.o_done());
+                    mma_commit(bars.v_empty(s));
+                }
+                __syncwarp();
+            }
+        }
+        // every MMA of this warp has finished before TMEM is released
+        if (elect_one()) mma_commit(bars.mma_done());
+        __syncwarp();
+        if (lane == 0) {
+            const uint64_t tt = globaltimer_ns();
+            while (!mbar_try_wait_sleep(bars.mma_done(), 0, 20000u) && globaltimer_ns() - tt < a.timeout_ns) {
+            }
+        }
+        __syncwarp();
+    } else {
+        // ================================ softmax warps: thread = query row ==================
+        const int q = warp, r = q * 32 + lane;
+        const int t = t0 + r;
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        // the query tile: shared memory (K-major rows of 128 B per 64-wide block) -> TMEM A
+        bool ok = __all_sync(0xffffffffu, wait_b(bars.q_full(), 0, a, abort, 8));
+        if (ok) {
+#pragma unroll 1
+            for (int kb = 0; kb < D / 64; ++kb) {
+                // row r of block kb: 128 bytes, 16-byte chunks swizzled by (r & 7)
+                uint32_t rr[32];
+                const uint8_t* row = smem + OFF_Q + kb * (BQ * 128) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ (r & 7)) << 4));
+                    rr[4 * c] = v.x; rr[4 * c + 1] = v.y; rr[4 * c + 2] = v.z; rr[4 * c + 3] = v.w;
+                }
+                uint32_t lo[16], hi[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) { lo[i] = rr[i]; hi[i] = rr[16 + i]; }
+                tmem_st16(tmem + lane_off + TM_Q + kb * 32, lo);
+                tmem_st16(tmem + lane_off + TM_Q + kb * 32 + 16, hi);
+            }
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.q_tmem());
+
+        float m_ref = -INFINITY, l = 0.f;                     // log2-domain reference max, sum
+        const int lo_key = max(0, t - a.w + 1);
+        int pv_issued = 0;                                    // P V products handed to the MMA
+        for (int j = 0; ok && j < ntiles; ++j) {
+            const int s = j & 1;
+            ok = __all_sync(0xffffffffu, wait_b(bars.s_full(s), (j >> 1) & 1, a, abort, 9));
+            if (!ok) break;
+            tc_fence_after();
+            const int key0 = (j0 + j) * BKV;
+            float sv[BKV];
+#pragma unroll
+            for (int c = 0; c < BKV; c += 16) {
+                float tmp[16];
+                tmem_ld16(tmem + lane_off + TM_S + s * BKV + c, tmp);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sv[c + i] = tmp[i];
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.s_free(s));
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < BKV; ++i) {
+                const int key = key0 + i;
+                const bool in = t < a.T && key >= lo_key && key <= t;
+                sv[i] = in ? sv[i] * a.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, sv[i]);
+            }
+            // the reference maximum moves (and the accumulator is rescaled) only when the
+            // tile's maximum passes it by more than 8 (a factor 256 in P)
+            const bool move = mx > m_ref + 8.0f;
+            const bool any_move = __any_sync(0xffffffffu, move);
+            const float m_new = move ? mx : m_ref;
+            // P of the previous tile must be consumed (and O complete) before P and O change
+            if (pv_issued > 0) {
+                ok = __all_sync(0xffffffffu, wait_b(bars.o_done(), (pv_issued - 1) & 1, a, abort, 10));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            if (any_move && pv_issued > 0) {
+                const float f = (move && m_ref != -INFINITY) ? exp2f(m_ref - m_new) : 1.0f;
+#pragma unroll 1
+                for (int c = 0; c < D; c += 16) {
+                    float o[16];
+                    tmem_ld16(tmem + lane_off + TM_O + c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o[i] *= f;
+                    tmem_st16f(tmem + lane_off + TM_O + c, o);
+                }
+                tmem_wait_st();
+                l *= f;
+            }
+            m_ref = m_new;
+            // P in bf16: row r, 64 keys = 128 bytes, 16-byte chunks swizzled by (r & 7)
+            uint8_t* prow = smem + OFF_P + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float p[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    p[i] = (m_ref == -INFINITY) ? 0.f : exp2f(sv[8 * c + i] - m_ref);
+                    l += p[i];
+                }
+                uint4 pk;
+                __nv_bfloat162 t0v = __floats2bfloat162_rn(p[0], p[1]), t1v = __floats2bfloat162_rn(p[2], p[3]);
+                __nv_bfloat162 t2v = __floats2bfloat162_rn(p[4], p[5]), t3v = __floats2bfloat162_rn(p[6], p[7]);
+                pk.x = *reinterpret_cast<uint32_t*>(&t0v); pk.y = *reinterpret_cast<uint32_t*>(&t1v);
+                pk.z = *reinterpret_cast<uint32_t*>(&t2v); pk.w = *reinterpret_cast<uint32_t*>(&t3v);
+                *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = pk;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.p_full());
+            ++pv_issued;
+        }
+        // the last P V, then out = O / l
+        if (ok && pv_issued > 0)
+            ok = __all_sync(0xffffffffu, wait_b(bars.o_done(), (pv_issued - 1) & 1, a, abort, 11));
+        if (ok) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.0f / l : 0.f;
+            __nv_bfloat16* orow = a.out + (((size_t)b * a.T + t) * a.H + h) * D;
+#pragma unroll 1
+            for (int c = 0; c < D; c += 16) {
+                float o[16];
+                tmem_ld16(tmem + lane_off + TM_O + c, o);
+                tmem_wait_ld();
+                if (t < a.T) {
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        __nv_bfloat162 p2 = __floats2bfloat162_rn(o[2 * i] * inv, o[2 * i + 1] * inv);
+                        pk[i] = *reinterpret_cast<uint32_t*>(&p2);
+                    }
+                    *reinterpret_cast<uint4*>(orow + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4*>(orow + c + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+        }
+        tmem_wait_ld();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWarpMma) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- decode ---------------------
+constexpr int kDecThreads = D;         // thread = one of the d columns
+constexpr int kDecKeys = 32;           // keys per tile
+constexpr int kMaxH = 16;
+
+struct DecArgs {
+    int B, H, w, nsplit, per;          // keys per split
+    float scale;
+    const __nv_bfloat16* q_rot;        // [B, H, d]
+    const int* pos;                    // [B]
+    const __nv_bfloat16* cache;        // [B][2][w][d]
+    float* part_m;                     // [B][nsplit][H]
+    float* part_l;
+    float* part_o;                     // [B][nsplit][H][d]
+};
+
+__global__ void __launch_bounds__(kDecThreads) mqa_decode_kernel(DecArgs a) {
+    __shared__ float qs[kMaxH][D];
+    __shared__ __nv_bfloat16 ks[kDecKeys][D + 8];     // padded rows: no bank conflicts
+    __shared__ float ps[kMaxH][kDecKeys];
+    __shared__ float mcur[kMaxH], lcur[kMaxH], fscale[kMaxH];
+    const int sp = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    const int pos = a.pos[b];
+    const int lo = max(0, pos - a.w + 1);
+    const int n = pos - lo + 1;                        // keys in the window
+    const int s0 = sp * a.per, s1 = min(n, s0 + a.per);
+    for (int h = 0; h < a.H; ++h) qs[h][tid] = __bfloat162float(a.q_rot[((size_t)b * a.H + h) * D + tid]);
+    if (tid < a.H) {
+        mcur[tid] = -INFINITY;
+        lcur[tid] = 0.f;
+    }
+    float o[kMaxH];
+#pragma unroll
+    for (int h = 0; h < kMaxH; ++h) o[h] = 0.f;
+    const __nv_bfloat16* kc = a.cache + (size_t)b * 2 * a.w * D;
+    const __nv_bfloat16* vc = kc + (size_t)a.w * D;
+    __syncthreads();
+    for (int i0 = s0; i0 < s1; i0 += kDecKeys) {
+        const int cnt = min(kDecKeys, s1 - i0);
+        // the tile's keys into shared memory (coalesced: a warp reads whole rows)
+        for (int e = tid; e < cnt * (D / 8); e += kDecThreads) {
+            const int i = e / (D / 8), c8 = e % (D / 8);
+            const int slot = (lo + i0 + i) % a.w;
+            *reinterpret_cast<uint4*>(&ks[i][c8 * 8]) = *reinterpret_cast<const uint4*>(kc + (size_t)slot * D + c8 * 8);
+        }
+        __syncthreads();
+        // scores: thread = (head, key) pairs
+        for (int e = tid; e < a.H * cnt; e += kDecThreads) {
+            const int h = e / cnt, i = e % cnt;
+            float acc = 0.f;
+#pragma unroll 8
+            for (int dd = 0; dd < D; ++dd) acc = fmaf(qs[h][dd], __bfloat162float(ks[i][dd]), acc);
+            ps[h][i] = acc * a.scale;
+        }
+        __syncthreads();
+        if (tid < a.H) {                               // running max / sum of head tid
+            const int h = tid;
+            float mx = mcur[h];
+            for (int i = 0; i < cnt; ++i) mx = fmaxf(mx, ps[h][i]);
+            const float f = mcur[h] == -INFINITY ? 0.f : expf(mcur[h] - mx);
+            float l = lcur[h] * f;
+            for (int i = 0; i < cnt; ++i) {
+                const float p = expf(ps[h][i] - mx);
+                ps[h][i] = p;
+                l += p;
+            }
+            mcur[h] = mx;
+            lcur[h] = l;
+            fscale[h] = f;
+        }
+        __syncthreads();
+        // o[h][tid] = o f + sum_i p v[i][tid]
+#pragma unroll
+        for (int h = 0; h < kMaxH; ++h)
+            if (h < a.H) o[h] *= fscale[h];
+        for (int i = 0; i < cnt; ++i) {
+            const int slot = (lo + i0 + i) % a.w;
+            const float vv = __bfloat162float(vc[(size_t)slot * D + tid]);
+#pragma unroll
+            for (int h = 0; h < kMaxH; ++h)
+                if (h < a.H) o[h] = fmaf(ps[h][i], vv, o[h]);
+        }
+        __syncthreads();
+    }
+    const size_t pb = ((size_t)b * a.nsplit + sp) * a.H;
+    if (tid < a.H) {
+        a.part_m[pb + tid] = mcur[tid];
+        a.part_l[pb + tid] = lcur[tid];
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxH; ++h)
+        if (h < a.H) a.part_o[(pb + h) * D + tid] = o[h];
+}
+
+struct MergeArgs {
+    int B, H, nsplit;
+    const float* part_m;
+    const float* part_l;
+    const float* part_o;
+    __nv_bfloat16* out;                // [B, H, d]
+};
+
+__global__ void __launch_bounds__(D) mqa_merge_kernel(MergeArgs a) {
+    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    float mx = -INFINITY;
+    for (int s = 0; s < a.nsplit; ++s) mx = fmaxf(mx, a.part_m[((size_t)b * a.nsplit + s) * a.H + h]);
+    float l = 0.f, o = 0.f;
+    for (int s = 0; s < a.nsplit; ++s) {
+        const size_t pb = ((size_t)b * a.nsplit + s) * a.H + h;
+        const float m = a.part_m[pb];
+        if (m == -INFINITY) continue;
+        const float f = expf(m - mx);
+        l += a.part_l[pb] * f;
+        o += a.part_o[pb * D + tid] * f;
+    }
+    a.out[((size_t)b * a.H + h) * D + tid] = __float2bfloat16_rn(l > 0.f ? o / l : 0.f);
+}
+
+}  // namespace mq
+
+// --------------------------------------------------------------------------- host side ------
+
+bool mqa_supported(const rglru_mqa_dims* d) {
+    return d->head_dim == mq::D && d->q_heads >= 1 && d->q_heads <= mq::kMaxH && d->window >= 1;
+}
+
+namespace {
+struct MqaLayout {
+    size_t q_rot, k_rot, part_m, part_l, part_o, total;
+    int nsplit, per;
+};
+MqaLayout mqa_layout(const rglru_mqa_dims* d, bool decode) {
+    auto up = [](size_t v) { return (v + 255) & ~size_t(255); };
+    MqaLayout l{};
+    const size_t T = decode ? 1 : (size_t)d->seq_len;
+    size_t o = 256;
+    l.q_rot = o; o = up(o + (size_t)d->batch * T * d->q_heads * mq::D * 2);
+    l.k_rot = o; o = up(o + (size_t)d->batch * T * mq::D * 2);
+    l.per = 256;
+    l.nsplit = (d->window + l.per - 1) / l.per;
+    l.part_m = o; o = up(o + (size_t)d->batch * l.nsplit * d->q_heads * 4);
+    l.part_l = o; o = up(o + (size_t)d->batch * l.nsplit * d->q_heads * 4);
+    l.part_o = o; o = up(o + (size_t)d->batch * l.nsplit * d->q_heads * mq::D * 4);
+    l.total = o;
+    return l;
+}
+}  // namespace
+
+size_t mqa_workspace(const rglru_mqa_dims* d, bool decode) { return mqa_layout(d, decode).total; }
+
+cudaError_t launch_mqa_prefill(const rglru_mqa_dims* d, const void* q, const void* k, const void* v, int pos0,
+                               void* out, void* cache, void* ws, size_t ws_bytes, cudaStream_t s) {
+    using namespace mq;
+    const MqaLayout l = mqa_layout(d, false);
+    if (l.total > ws_bytes) return cudaErrorInvalidValue;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    const int B = d->batch, T = d->seq_len, H = d->q_heads;
+    RopeArgs ra{};
+    ra.B = B; ra.T = T; ra.H = H; ra.w = d->window; ra.pos0 = pos0; ra.base = d->rope_base;
+    ra.q = static_cast<const __nv_bfloat16*>(q); ra.k = static_cast<const __nv_bfloat16*>(k);
+    ra.v = static_cast<const __nv_bfloat16*>(v);
+    ra.q_rot = reinterpret_cast<__nv_bfloat16*>(w + l.q_rot);
+    ra.k_rot = reinterpret_cast<__nv_bfloat16*>(w + l.k_rot);
+    ra.cache = static_cast<__nv_bfloat16*>(cache);
+    mqa_rope_kernel<<<dim3(T, B), D / 2, 0, s>>>(ra);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // tensor maps: queries as a 3-D [B T rows][H][d] tensor (box 64 x 1 head x 128 rows),
+    // keys and values as 2-D [B T rows][d] (box 64 x 64 rows), all in the 128-byte swizzle
+    CUtensorMap mqm, mkm, mvm;
+    if (!tc::make_map_3d_box_sw128(&mqm, ra.q_rot, D, (uint64_t)H, (uint64_t)B * T, 64, 1, BQ) ||
+        !tc::make_map_2d_sw128(&mkm, ra.k_rot, D, (uint64_t)B * T, D * 2, 64, BKV) ||
+        !tc::make_map_2d_sw128(&mvm, v, D, (uint64_t)B * T, D * 2, 64, BKV))
+        return cudaErrorInvalidValue;
+    e = set_smem_once(mqa_prefill_kernel, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    PrefArgs pa{};
+    pa.B = B; pa.T = T; pa.H = H; pa.w = d->window;
+    pa.scale_log2 = d->scale * kLog2e;
+    pa.out = static_cast<__nv_bfloat16*>(out);
+    pa.status = reinterpret_cast<DeviceStatus*>(w);
+    pa.timeout_ns = 1000000000ull;
+    mqa_prefill_kernel<<<dim3((T + BQ - 1) / BQ, H, B), kThreads, SMEM_BYTES, s>>>(mqm, mkm, mvm, pa);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mqa_decode(const rglru_mqa_dims* d, const void* q, const void* k, const void* v, const int* pos,
+                              void* cache, void* out, void* ws, size_t ws_bytes, cudaStream_t s) {
+    using namespace mq;
+    const MqaLayout l = mqa_layout(d, true);
+    if (l.total > ws_bytes) return cudaErrorInvalidValue;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    const int B = d->batch, H = d->q_heads;
+    RopeDecArgs ra{};
+    ra.B = B; ra.H = H; ra.w = d->window; ra.base = d->rope_base; ra.pos = pos;
+    ra.q = static_cast<const __nv_bfloat16*>(q); ra.k = static_cast<const __nv_bfloat16*>(k);
+    ra.v = static_cast<const __nv_bfloat16*>(v);
+    ra.q_rot = reinterpret_cast<__nv_bfloat16*>(w + l.q_rot);
+    ra.cache = static_cast<__nv_bfloat16*>(cache);
+    mqa_rope_decode_kernel<<<B, D / 2, 0, s>>>(ra);
+    DecArgs da{};
+    da.B = B; da.H = H; da.w = d->window; da.nsplit = l.nsplit; da.per = l.per; da.scale = d->scale;
+    da.q_rot = ra.q_rot; da.pos = pos; da.cache = ra.cache;
+    da.part_m = reinterpret_cast<float*>(w + l.part_m);
+    da.part_l = reinterpret_cast<float*>(w + l.part_l);
+    da.part_o = reinterpret_cast<float*>(w + l.part_o);
+    mqa_decode_kernel<<<dim3(l.nsplit, B), kDecThreads, 0, s>>>(da);
+    MergeArgs ma{};
+    ma.B = B; ma.H = H; ma.nsplit = l.nsplit;
+    ma.part_m = da.part_m; ma.part_l = da.part_l; ma.part_o = da.part_o;
+    ma.out = static_cast<__nv_bfloat16*>(out);
+    mqa_merge_kernel<<<dim3(H, B), D, 0, s>>>(ma);
+    return cudaGetLastError();
+}
+
+}  // namespace rglru

@@ -166,6 +166,104 @@ RGLRU_API rglru_status rglru_block_decode(const rglru_dims* dims, const rglru_pa
                                 rglru_state* state, void* out,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Persistent multi-step decode: `steps` successive single-token decode steps of every row in one
+ * call (RGLRU.step of the listing, plus the conv, applied steps times), for a batch of decode
+ * slots under continuous batching.
+ *   x, y, out  [steps, B, W] act dtype: the token of step s for row b at [s][b][:]
+ *   reset      [steps, B] uint8 or NULL: reset[s][b] != 0 empties row b's state (h and the conv
+ *              history) before step s, so a slot can take a new sequence at any step
+ *   state      required, in/out: the state before step 0, overwritten with the state after the
+ *              last step
+ * Results equal `steps` calls of rglru_block_decode in order (up to the rounding of the
+ * arithmetic).  The tensor-core path (bf16, head_dim 256, state->h 16-byte aligned) is one
+ * launch that keeps the state of every row on chip from the first step to the last, so only x,
+ * y and out move per step; other shapes run the portable step kernel once per step.
+ * Workspace: rglru_decode_steps_workspace_size bytes (the status word).  Errors as for
+ * rglru_block_decode, and INVALID_ARG when steps <= 0. */
+RGLRU_API size_t rglru_decode_steps_workspace_size(const rglru_dims* dims, int steps);
+RGLRU_API rglru_status rglru_block_decode_steps(const rglru_dims* dims, const rglru_params* params,
+                                                const void* x, const void* y, const uint8_t* reset,
+                                                int steps, rglru_state* state, void* out,
+                                                void* workspace, size_t workspace_bytes, void* stream);
+/* How rglru_block_decode_steps runs for `dims` and `steps`: *kernel as for the other plans,
+ * *launches = 1 on the tensor-core path, `steps` otherwise. */
+RGLRU_API rglru_status rglru_decode_steps_plan(const rglru_dims* dims, int steps, int* kernel, int* launches);
+
+/* The projections on either side of the block (the listing's RecurrentBlock.forward:
+ * proj_in_1 / proj_in_2 / proj_out; linear_x / linear_y / linear_out in RecurrentGemma):
+ *   model_dim  D, a multiple of 64
+ *   w_in_x     [D, W] act dtype: x = u @ w_in_x    (the conv / RG-LRU branch)
+ *   w_in_y     [D, W] act dtype: y = u @ w_in_y    (the GeLU branch)
+ *   w_out      [W, D] act dtype: out = z @ w_out   (z = h * GeLU(y), the block's output) */
+typedef struct {
+    int model_dim;
+    const void* w_in_x;
+    const void* w_in_y;
+    const void* w_out;
+} rglru_projections;
+
+/* Bytes of device workspace rglru_layer_forward needs for `dims` (0 on invalid dims): the
+ * block's prefill workspace and the x, y, z activations [B, T, W] in the act dtype. */
+RGLRU_API size_t rglru_layer_workspace_size(const rglru_dims* dims);
+
+/* The recurrent block with its projections, for a whole sequence:
+ *   u [B, T, D] act dtype  ->  out [B, T, D] act dtype
+ *   x = u w_in_x, y = u w_in_y, z = rglru_block_prefill(x, y, reset, state), out = z w_out.
+ * The projections run on the tensor cores with fp32 accumulation and bf16 results; x, y and z
+ * live in the workspace.  reset / state as for rglru_block_prefill.  Supported: bf16, head_dim
+ * 256, model_dim a multiple of 64 (else UNSUPPORTED).  Errors as for rglru_block_prefill; the
+ * device status word is the workspace's first 16 bytes. */
+RGLRU_API rglru_status rglru_layer_forward(const rglru_dims* dims, const rglru_params* params,
+                                           const rglru_projections* proj, const void* u,
+                                           const uint8_t* reset, rglru_state* state, void* out,
+                                           void* workspace, size_t workspace_bytes, void* stream);
+/* *kernel = RGLRU_KERNEL_TENSOR and *launches = the operations one rglru_layer_forward call
+ * enqueues (three projection GEMMs and the block's), or UNSUPPORTED. */
+RGLRU_API rglru_status rglru_layer_plan(const rglru_dims* dims, const rglru_projections* proj, int* kernel,
+                                        int* launches);
+
+/* ---- Griffin's second temporal-mixing block: local sliding-window multi-query attention ----
+ * ("Griffin Guide: RecurrentGemma, RG-LRU & Hybrid Attention", "2. Local Sliding-Window
+ * Multi-Query Attention (MQA)" and "3. Bounding the Key-Value Cache Footprint"; "Griffin"
+ * notes, "Local Attention Path").  q_heads query heads share one key and one value head; token
+ * t attends to the positions N(t) = {i : t - window < i <= t} of its own sequence:
+ *     y_t = sum_{i in N(t)} softmax_i(scale * q_t . k_i) v_i,
+ * with rotary position embeddings on q and k: the pairs (j, j + head_dim/2) of position p turn
+ * by p * rope_base^(-2j / head_dim).  All tensors bf16, row-major; head_dim 256, 1 <= q_heads
+ * <= 16, window >= 1 (else UNSUPPORTED).  Device pointers owned by the caller, work on `stream`.
+ * The ring cache of a row holds, for position p, its rotated key in slot p mod window and its
+ * value in the same slot of the value half: [B][2][window][head_dim]. */
+typedef struct {
+    int batch;        /* B */
+    int seq_len;      /* T (prefill); ignored by decode */
+    int q_heads;      /* H */
+    int head_dim;     /* d, 256 */
+    int window;       /* w */
+    float scale;      /* score scale, e.g. 1 / sqrt(head_dim) */
+    float rope_base;  /* e.g. 10000 */
+} rglru_mqa_dims;
+
+/* Workspace bytes of rglru_mqa_prefill (decode = 0) or rglru_mqa_decode (decode = 1); 0 on
+ * invalid dims.  256-byte aligned, first 16 bytes: the device status word. */
+RGLRU_API size_t rglru_mqa_workspace_size(const rglru_mqa_dims* dims, int decode);
+
+/* Prefill: q [B, T, H, d], k, v [B, T, d] at positions pos0 .. pos0 + T - 1 -> out
+ * [B, T, H, d].  The window is restricted to the T tokens given.  cache: NULL, or the ring
+ * cache [B][2][w][d], which receives the last min(T, w) rotated keys and values.  The score
+ * contraction and the weighted sum run on the tensor cores (bf16 operands, fp32 accumulation).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+RGLRU_API rglru_status rglru_mqa_prefill(const rglru_mqa_dims* dims, const void* q, const void* k,
+                                         const void* v, int pos0, void* out, void* cache,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* One decode token per row: q [B, H, d], k, v [B, d] at position pos[b] (a device int32 array
+ * [B]); the rotated key and the value are written into slot pos[b] mod w of the row's ring, then
+ * the token attends to the positions max(0, pos - w + 1) .. pos, all of which must have been
+ * written by earlier prefill or decode calls.  out [B, H, d].  Errors as rglru_mqa_prefill. */
+RGLRU_API rglru_status rglru_mqa_decode(const rglru_mqa_dims* dims, const void* q, const void* k,
+                                        const void* v, const int* pos, void* cache, void* out,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Prefill for callers that cannot allocate device memory.  The pages have no counterpart:
  * this is a deployment variant of rglru_block_prefill, not a step of the method.
  *

@@ -5,13 +5,11 @@ fp64 oracle under the error metrics of the parity bar.
    1e-5 for fp32 inputs and 2e-2 for bf16 inputs with fp32 state.
 2. RMS relative error, rms(g - r) / rms(r), at most 2e-6 (fp32) / 5e-3 (bf16): it catches a
    bias spread over many elements that the max norm would let through.
-3. Element-wise guard, max_i |g_i - r_i| / max(|r_i|, 0.1 rms(r)): at most 1e-4 (fp32) /
-   0.5 (bf16).  It catches isolated misplaced or garbage elements (those score >= 1).  It is
-   not tighter because it amplifies an absolute error wherever h_t * GeLU(y_t) crosses zero:
-   an exact fp32 emulation of the block already scores 4e-5, and an exact emulation whose
-   only approximation is the bf16 rounding of the conv output that feeds the tensor-core gate
-   contraction scores 0.13 at 64 tokens and 0.2 at 1000 tokens (2.4e-3 RMS, 2.8e-3 max norm),
-   which is what the tensor-core prefill reproduces digit for digit.
+3. Element-wise error, max_i |g_i - r_i| / max(|r_i|, 0.1 rms(r)) (the denominator floored where
+   h_t * GeLU(y_t) crosses zero): at most 2e-2 for bf16, the same bar element by element.  For
+   fp32 it is 1e-4: there the floor amplifies plain rounding, and an exact fp32 emulation of
+   the block already scores 4e-5.  The bf16 kernels round only the tensor-core operand of the
+   gate contraction to bf16; the conv output entering the state update stays fp32.
 """
 
 from __future__ import annotations
@@ -23,7 +21,7 @@ from gated_linear_recurrence_conv1d_b200 import binding, inputs
 
 TOL = {"f32": 1e-5, "bf16": 2e-2}
 TOL_RMS = {"f32": 2e-6, "bf16": 5e-3}
-TOL_ELEMENTWISE = {"f32": 1e-4, "bf16": 0.5}
+TOL_ELEMENTWISE = {"f32": 1e-4, "bf16": 2e-2}
 
 
 def rel_err(g: np.ndarray, r: np.ndarray) -> float:

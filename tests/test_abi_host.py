@@ -122,6 +122,43 @@ def test_decode_requires_state():
     assert rc == 1
 
 
+def test_decode_steps_rejects_bad_arguments():
+    lib = binding.load()
+    d = _dims(seq_len=1)
+    p = _params()
+    st = binding.State(ctypes.c_void_p(FAKE + 0x1000), ctypes.c_void_p(FAKE + 0x2000))
+    args = lambda steps, state, ws_bytes: (ctypes.byref(d), ctypes.byref(p), ctypes.c_void_p(FAKE),  # noqa: E731
+                                           ctypes.c_void_p(FAKE + 0x100), None, steps, state,
+                                           ctypes.c_void_p(FAKE + 0x200), ctypes.c_void_p(FAKE), ws_bytes, None)
+    assert lib.rglru_block_decode_steps(*args(0, ctypes.byref(st), 1 << 20)) == 1      # no steps
+    assert lib.rglru_block_decode_steps(*args(-3, ctypes.byref(st), 1 << 20)) == 1
+    assert lib.rglru_block_decode_steps(*args(4, None, 1 << 20)) == 1                  # state required
+    assert lib.rglru_block_decode_steps(*args(4, ctypes.byref(st), 8)) == 3            # workspace too small
+    assert binding.decode_steps_workspace_size(d, 4) >= 16
+    assert binding.decode_steps_workspace_size(d, 0) == 0
+    k, n = ctypes.c_int(), ctypes.c_int()
+    assert lib.rglru_decode_steps_plan(ctypes.byref(d), 0, ctypes.byref(k), ctypes.byref(n)) == 1
+
+
+def test_mqa_rejects_bad_arguments():
+    lib = binding.load()
+    good = binding.make_mqa_dims(2, 64, 4, 256, 32)
+    assert binding.mqa_workspace_size(good) >= 256 and binding.mqa_workspace_size(good, decode=True) >= 256
+    for bad, code in ((binding.make_mqa_dims(2, 64, 4, 128, 32), 2),     # head_dim
+                      (binding.make_mqa_dims(2, 64, 17, 256, 32), 2),    # too many query heads
+                      (binding.make_mqa_dims(2, 64, 4, 256, 0), 1),      # window
+                      (binding.make_mqa_dims(0, 64, 4, 256, 8), 1)):     # batch
+        assert binding.mqa_workspace_size(bad) == 0
+        rc = lib.rglru_mqa_prefill(ctypes.byref(bad), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + 0x100),
+                                   ctypes.c_void_p(FAKE + 0x200), 0, ctypes.c_void_p(FAKE + 0x300), None,
+                                   ctypes.c_void_p(FAKE), 1 << 30, None)
+        assert rc == code
+    rc = lib.rglru_mqa_decode(ctypes.byref(good), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + 0x100),
+                              ctypes.c_void_p(FAKE + 0x200), None, ctypes.c_void_p(FAKE + 0x400),
+                              ctypes.c_void_p(FAKE + 0x300), ctypes.c_void_p(FAKE), 1 << 30, None)
+    assert rc == 1                                                       # positions required
+
+
 def test_read_status_rejects_bad_workspace():
     lib = binding.load()
     assert lib.rglru_read_device_status(None, 256, None) == 1

@@ -1,8 +1,9 @@
 """Backward pass on the GPU against the fp64 oracle's gradients (every output of
 rglru_block_backward, element by element).
 
-The GPU computes in fp32 from the exact input values (bf16 inputs are widened, nothing inside
-is rounded to bf16), so one bar serves both activation dtypes.  It is ten times the forward's
+The portable kernels compute in fp32 from the exact input values.  The tensor-core path (bf16,
+head_dim 256) runs its dense contractions on bf16 operands split into hi + lo parts (fp32 to
+about 2^-16), so the same bar serves it and both activation dtypes.  It is ten times the forward's
 fp32 bar: the backward chains about three times as many roundings per element (the forward
 again, the reverse recurrence, two transposed contractions) and its parameter gradients are
 sums over all B T tokens; a wrong term, sign, index or reset gives errors of order one.
@@ -72,7 +73,8 @@ def _compare(grads, ref, label):
 
 @pytest.mark.parametrize("B,T,H,dh,dtype,tanh", [
     (2, 70, 2, 64, "f32", 0),      # two full tiles and a ragged one
-    (2, 100, 2, 256, "bf16", 0),   # the tensor-core shape, through the portable backward
+    (2, 100, 2, 256, "bf16", 0),   # the tensor-core backward: chunks, a ragged one, resets
+    (3, 257, 2, 256, "bf16", 1),   # tanh GeLU, more rows than chunks of the dW slices
     (3, 2, 3, 16, "f32", 0),       # shorter than the conv history
     (1, 45, 2, 48, "f32", 1),      # a head width that does not divide the CTA
 ])
@@ -88,6 +90,16 @@ def test_backward_without_state_or_final_gradients():
     wl = inputs.WORKLOADS["tiny_f32"].scaled(batch=2, seq_len=40, heads=2, head_dim=32)
     grads, ref = _run(wl, seed=3, with_state=False, with_final=False, biases=False)
     _compare(grads, ref, "zero state")
+
+
+def test_tensor_backward_agrees_with_portable_and_repeats_bitwise():
+    wl = inputs.WORKLOADS["packed_bf16"].scaled(batch=2, seq_len=96, heads=2, doc_len=(10, 60))
+    assert binding.backward_plan(binding.make_dims(2, 96, 2, 256, binding.RGLRU_BF16))[0] == 1
+    a, ref = _run(wl, seed=21)
+    _compare(a, ref, "tensor backward")
+    b, _ = _run(wl, seed=21)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
 
 
 def test_backward_bitwise_repeatable():

