@@ -92,7 +92,7 @@ constexpr int kSlots = 4;               // TMEM accumulator slots (item n uses s
 constexpr uint32_t KBLK_BYTES = L * 128;               // one 64-channel K block of the B tile
 constexpr uint32_t B_BYTES = 4 * KBLK_BYTES;           // [32 tokens x 256 channels] bf16, 128B swizzle
 constexpr uint32_t X_BYTES = XROWS * DH * 2;           // 17920: [35 tokens x 256 channels] bf16
-constexpr uint32_t X_STRIDE = 18432;
+constexpr uint32_t X_STRIDE = X_BYTES;
 constexpr uint32_t XC_BYTES = L * HALF * 4;            // [32 tokens x 128 channels] fp32 conv output
 constexpr uint32_t Y_BYTES = L * HALF * 2;             // [32 tokens x 128 channels] bf16, y then out
 
@@ -102,7 +102,8 @@ constexpr uint32_t OFF_BLO = OFF_B + G * B_BYTES;      // bf16 lo parts
 constexpr uint32_t OFF_X = OFF_BLO + G * B_BYTES;
 constexpr uint32_t OFF_XC = OFF_X + G * X_STRIDE;
 constexpr uint32_t OFF_Y = OFF_XC + G * XC_BYTES;
-constexpr uint32_t OFF_BAR = OFF_Y + G * Y_BYTES;
+constexpr uint32_t OFF_CW = OFF_Y + G * Y_BYTES;       // conv taps [4][256] and bias [256] of the head, fp32
+constexpr uint32_t OFF_BAR = OFF_CW + 5 * DH * 4;
 constexpr int kBarsPerStage = 6;
 constexpr int NBAR = kBarsPerStage * G + kSlots + RING + 2;
 constexpr uint32_t OFF_SLOT = (OFF_BAR + NBAR * 8 + 15) & ~15u;   // slot[RING]
@@ -111,6 +112,7 @@ constexpr uint32_t OFF_ABORT = OFF_TMEMP + 16;
 constexpr uint32_t SMEM_BYTES = OFF_ABORT + 16 + 1024;           // + slack for 1024 alignment
 static_assert(OFF_BLO % 1024 == 0 && B_BYTES % 1024 == 0, "swizzled MMA operands");
 static_assert(OFF_X % 128 == 0 && X_STRIDE % 128 == 0 && OFF_Y % 128 == 0, "TMA destinations");
+static_assert(OFF_CW % 16 == 0, "16-byte loads of the conv taps");
 static_assert(2 * HALF * DH * 2 <= OFF_BAR, "weight staging reuses the stage tiles");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -515,6 +517,12 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(src));
             *reinterpret_cast<uint4*>(smem + g * (HALF * DH * 2) + (i * HALF + o8 * 8) * 2) = v;
         }
+        // the conv taps and bias of the head's 256 channels (the conv of every item reads them)
+        float* cw = reinterpret_cast<float*>(smem + OFF_CW);
+        for (int e = tid; e < 5 * DH; e += kEpiWarps * 32) {
+            const int k = e / DH, c = e % DH;
+            cw[e] = k < kConvWidth ? a.conv_w[(size_t)k * W + head * DH + c] : (a.conv_b ? a.conv_b[head * DH + c] : 0.f);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -674,19 +682,25 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             const uint32_t rm = rmask >> j0;
             const int jlast = nt - 1 - j0;
 #pragma unroll 1
-            for (int p4 = 0; p4 < 2; ++p4) {              // channels cl + 4 p4 .. + 3
+            for (int pp = 0; pp < 2; ++pp) {
+                // channels cl + 4 p4 .. + 3; lanes of odd K blocks take the halves the other way
+                // round, so that lanes 8 apart never meet in a bank
+                const int p4 = pp ^ ((lane >> 3) & 1);
                 const int chg = head * DH + cl + 4 * p4;  // global channel
                 float2 w[kConvWidth][2];
+                const float* cwp = reinterpret_cast<const float*>(smem + OFF_CW) + cl + 4 * p4;
 #pragma unroll
-                for (int k2 = 0; k2 < kConvWidth; ++k2)
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        w[k2][i] = make_float2(a.conv_w[(size_t)k2 * W + chg + 2 * i],
-                                               a.conv_w[(size_t)k2 * W + chg + 2 * i + 1]);
+                for (int k2 = 0; k2 < kConvWidth; ++k2) {
+                    const float4 v = *reinterpret_cast<const float4*>(cwp + k2 * DH);
+                    w[k2][0] = make_float2(v.x, v.y);
+                    w[k2][1] = make_float2(v.z, v.w);
+                }
                 float2 cb[2];
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-                    cb[i] = a.conv_b ? make_float2(a.conv_b[chg + 2 * i], a.conv_b[chg + 2 * i + 1]) : make_float2(0.f, 0.f);
+                {
+                    const float4 v = *reinterpret_cast<const float4*>(cwp + kConvWidth * DH);
+                    cb[0] = make_float2(v.x, v.y);
+                    cb[1] = make_float2(v.z, v.w);
+                }
                 const uint8_t* xt = smem + OFF_X + st * X_STRIDE + lane * 16 + 8 * p4;
                 auto xrow = [&](int r) {                  // x tile row r = token t0 - 3 + r
                     return unpack4(*reinterpret_cast<const uint2*>(xt + r * DH * 2));
