@@ -6,24 +6,24 @@
 // K = 256 input channels.  One launch; a cluster of 4 CTAs per (head, 128-row tile), CTA r
 // owning the 64 channels [64 r, 64 r + 64) of the head:
 //
-//   * conv: CTA r convolves its own 64 channels for the 128 rows (the width-4 causal conv over
-//     the carried history and the new input), shifts their history in place (oldest out, x in;
-//     a row with reset[b] set starts from an empty history), keeps the fp32 result for the
-//     state update, and writes it rounded to fp16 as K-block r of its 128 x 256 MMA operand
-//     tile (K-major, 128-byte swizzle); one thread then
-//     copies that 16 KB block into the same place of the three sibling CTAs' tiles through
-//     distributed shared memory (bulk copies that complete on the siblings' mbarrier), so every
-//     channel is convolved once and only by the CTA that owns its history;
-//   * gates: TMA brings the 256 x 64 slices W_a[h][:, 64 r], W_x[h][:, 64 r] (as stored: output
-//     channel contiguous, i.e. MN-major for the MMA) side by side, one N = 128 operand, which
-//     the update threads convert to fp16 in place once it has landed (exact for 2^-14 <= |w| <
-//     65504); an elected lane of the MMA warp issues tcgen05.mma (M = 128, N = 128, K = 16
-//     each, fp16 operands, fp32 accumulation) into TMEM, K block by K block as the blocks
-//     become ready (its own first);
-//   * update: TMA also brings the h (fp32) and y tiles of the CTA into shared memory; 16 warps
-//     (thread = row, 16 channels each) compute GeLU(y) while the MMAs run, then read the
-//     accumulators, apply the gates and write h and out back into the shared tiles, which TMA
-//     stores (rows past the batch are clipped by the tensor maps).
+//   * conv: update thread (row, 16 channels) convolves its channels of CTA r's 64 (the width-4
+//     causal conv over the carried history and the new input), shifts their history in place
+//     (oldest out, x in; a row with reset[b] set starts from an empty history), keeps the fp32
+//     result in its TMEM lane for the state update, and writes it as a bf16 pair -- hi = the
+//     fp32 value truncated, lo = the remainder rounded, hi + lo = the value to 2^-16 -- into
+//     K-block r of the CTA's two 128 x 256 operand tiles (K-major, 128-byte swizzle); one thread
+//     then copies the two 16 KB blocks into the same place of the three sibling CTAs' tiles
+//     through distributed shared memory (bulk copies that complete on the siblings' mbarrier),
+//     so every channel is convolved once and only by the CTA that owns its history;
+//   * gates: TMA brings the 256 x 64 slices W_a[h][:, 64 r], W_x[h][:, 64 r] (bf16 as stored:
+//     output channel contiguous, i.e. MN-major for the MMA) side by side, one N = 128 operand;
+//     an elected lane of the MMA warp issues tcgen05.mma (M = 128, N = 128, K = 16 each, bf16
+//     operands, fp32 accumulation) on both parts of the conv output into TMEM, K block by K
+//     block as the blocks become ready (its own first);
+//   * update: TMA brings the y tile of the CTA; the update threads compute GeLU(y) while the
+//     MMAs run, read their h from global memory, then the accumulators, apply the gates and
+//     write h back and out into the shared tile, which TMA stores (rows past the batch are
+//     clipped by the tensor map).
 //
 // The element-wise arithmetic is rglru_math.cuh's (shared with the prefill): gates by ex2 and a
 // reciprocal, expm1 of the log-decay by its series near zero, sqrt(1 - a^2) i_t by one rsqrt,
@@ -34,7 +34,6 @@
 // Zero-Communication Tensor Parallelism", and the listing's RGLRU.step.
 #include <cuda.h>
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -65,7 +64,7 @@ constexpr uint32_t A_BYTES = MT * DH * 2;            // 65536: 4 K-blocks of 128
 constexpr uint32_t A_KBLK = MT * 128;                // 16384
 constexpr uint32_t B_BYTES = DH * NT * 2;            // 32768 per gate: 256 K-rows x 128 B
 constexpr uint32_t Y_BYTES = MT * NT * 2;            // y tile (then out): 128 rows x 64 bf16
-constexpr uint32_t OFF_A = 0;                        // conv output, fp16 hi part
+constexpr uint32_t OFF_A = 0;                        // conv output, bf16 hi part
 constexpr uint32_t OFF_ALO = OFF_A + A_BYTES;        // and lo part (xc - hi)
 constexpr uint32_t OFF_BA = OFF_ALO + A_BYTES;
 constexpr uint32_t OFF_BX = OFF_BA + B_BYTES;        // right after W_a: one N = 128 operand
@@ -105,9 +104,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&p);
 }
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-    __half2 p = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&p);
+// bf16 hi part (truncation) of two fp32 values, packed; the remainder v - hi is exact in fp32
+__device__ __forceinline__ uint32_t trunc_bf16x2(float lo, float hi) {
+    return __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
 }
 
 // Shared-memory matrix descriptor for an MN-major operand in the 128-byte swizzle layout: rows
@@ -125,9 +124,9 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr) {
     return d;
 }
 
-// Instruction descriptor: fp32 accumulator, fp16 A (K-major) and B (MN-major), M x N.
-__host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
-    return (1u << 4) | (1u << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// Instruction descriptor: fp32 accumulator, bf16 A (K-major) and B (MN-major), M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 __device__ bool wait_bounded(uint32_t bar, uint32_t parity, const Args& a, volatile int* abort, unsigned where) {
@@ -152,7 +151,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_w = sbase + OFF_BAR, bar_acc = sbase + OFF_BAR + 16;
-    const uint32_t bar_wc = sbase + OFF_BAR + 8;      // the weight tile is in fp16
     const uint32_t bar_y = sbase + OFF_BAR + 24;      // y tile
     // K block j of the operand tile: convolved here (j = rank) or copied in by CTA j
     auto bar_k = [&](int j) { return sbase + OFF_BAR + 32 + 8 * (uint32_t)j; };
@@ -176,7 +174,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         mbar_init(bar_w, 1);
-        mbar_init(bar_wc, 1);
         mbar_init(bar_acc, 1);
         mbar_init(bar_y, 1);
         for (int j = 0; j < kClusterSize; ++j) mbar_init(bar_k(j), 1);
@@ -227,10 +224,10 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
         }
     } else if (warp == kWarpMma) {
         // the whole warp follows the waits; one elected lane issues (warp-uniform operands)
-        const uint32_t idesc = idesc_f16_f32_bmn(MT, 2 * NT);   // D_a | D_x
+        const uint32_t idesc = idesc_bf16_f32_bmn(MT, 2 * NT);   // D_a | D_x
         const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
         // K blocks in the order they become ready: this CTA's own first, then the siblings'
-        bool ok = __all_sync(0xffffffffu, wait_bounded(bar_wc, 0, a, abort, 1));
+        bool ok = __all_sync(0xffffffffu, wait_bounded(bar_w, 0, a, abort, 1));
         uint32_t accum = 0;
         for (int i = 0; i < kClusterSize && ok; ++i) {
             const int j = (nt + i) % kClusterSize;
@@ -333,9 +330,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
                         rr[e1] = acc;
                         xo[2 * e2 + e1] = __float_as_uint(acc);
                     }
-                    ohi[e2] = pack_f16x2(rr[0], rr[1]);
-                    olo[e2] = pack_f16x2(rr[0] - __half2float(__ushort_as_half((unsigned short)(ohi[e2] & 0xFFFFu))),
-                                         rr[1] - __half2float(__ushort_as_half((unsigned short)(ohi[e2] >> 16))));
+                    ohi[e2] = trunc_bf16x2(rr[0], rr[1]);
+                    olo[e2] = pack_bf16x2(rr[0] - bf16lo(ohi[e2]), rr[1] - bf16hi(ohi[e2]));
                 }
                 // row r, 16-byte chunk (2 cg + v) of this CTA's K block (128-byte swizzle)
                 const uint32_t so = nt * A_KBLK + (uint32_t)(r >> 3) * 1024 + sw * 128 + ((((uint32_t)(cg * 2 + v)) ^ sw) << 4);
@@ -369,27 +365,6 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
                     *reinterpret_cast<uint4*>(tw + 2 * W + 8 * v) = xv[v];
                 }
             }
-        }
-
-        // ================================ weights to fp16 ======================================
-        // in place, 16 bytes a step; the tile's layout does not matter to an element-wise pass
-        {
-            const bool okw = wait_bounded(bar_w, 0, a, abort, 5);
-            if (okw) {
-                uint4* wt = reinterpret_cast<uint4*>(smem + OFF_BA);
-#pragma unroll 4
-                for (int i = threadIdx.x; i < (int)(2 * B_BYTES / 16); i += kEpiThreads) {
-                    uint4 v = wt[i];
-                    v.x = pack_f16x2(bf16lo(v.x), bf16hi(v.x));
-                    v.y = pack_f16x2(bf16lo(v.y), bf16hi(v.y));
-                    v.z = pack_f16x2(bf16lo(v.z), bf16hi(v.z));
-                    v.w = pack_f16x2(bf16lo(v.w), bf16hi(v.w));
-                    wt[i] = v;
-                }
-            }
-            fence_proxy_async_smem();
-            asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-            if (threadIdx.x == 0) mbar_arrive(bar_wc);   // also after a failed wait: the MMA warp drains
         }
 
         // ================================ update ===============================================
