@@ -16,9 +16,9 @@
 //     reference maximum that moves only when the maximum grows by more than 2^8 (then the
 //     accumulator is rescaled), write P in bf16 to shared memory; O += P V (M = 128, N = 256,
 //     K = 64) accumulates in TMEM; the S of the next tile overlaps the softmax of this one;
-//   * mqa_decode_kernel: one token per row against the ring: CTAs split the window, each keeps
-//     (max, sum, sum of p v) per head over its part (CUDA cores: the step is bound by the cache
-//     read); mqa_merge_kernel combines the parts.
+//   * mqa_decode_kernel: one token per row against the ring: CTAs split the ring's slots, each
+//     keeps (max, sum, sum of p v) per head over its part (CUDA cores: the step is bound by
+//     reading the cache, not by its arithmetic); mqa_merge_kernel combines the parts.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -473,12 +473,24 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 }
 
 // ---------------------------------------------------------------- decode ---------------------
-constexpr int kDecThreads = D;         // thread = one of the d columns
-constexpr int kDecKeys = 32;           // keys per tile
+// One token per row against its ring.  The window is a set: softmax over it does not depend on
+// the order of its keys, and the ring holds exactly the window -- slots [0, n), n = min(pos + 1,
+// w) (slot = position mod w, keys cached after their rotation) -- so a CTA walks the slots of its
+// split in slot order.  CTA = (split of kDecPer slots, row); 256 threads:
+//   * scores: lane = slot; a lane streams its key row (16-byte loads) and accumulates q_h . k
+//     for every head with packed fp32x2 FMAs, the rotated queries read from shared memory as
+//     broadcasts;
+//   * softmax of the split per head (warp shuffles): its maximum m_h, sum l_h, weights in shared
+//     memory;
+//   * thread = (pair of value columns, half of the split's slots): sum of p v over its slots,
+//     halves added through shared memory; (m, l, o) per head go to the merge.
+// The step moves the whole ring (2 w d bf16 per row): it is bound by HBM, not by arithmetic.
+constexpr int kDecThreads = D;
+constexpr int kDecPer = 256;           // slots per split
 constexpr int kMaxH = 16;
 
 struct DecArgs {
-    int B, H, w, nsplit, per;          // keys per split
+    int B, H, w, nsplit;
     float scale;
     const __nv_bfloat16* q_rot;        // [B, H, d]
     const int* pos;                    // [B]
@@ -488,82 +500,135 @@ struct DecArgs {
     float* part_o;                     // [B][nsplit][H][d]
 };
 
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
+template <int HM>
 __global__ void __launch_bounds__(kDecThreads) mqa_decode_kernel(DecArgs a) {
-    __shared__ float qs[kMaxH][D];
-    __shared__ __nv_bfloat16 ks[kDecKeys][D + 8];     // padded rows: no bank conflicts
-    __shared__ float ps[kMaxH][kDecKeys];
-    __shared__ float mcur[kMaxH], lcur[kMaxH], fscale[kMaxH];
+    __shared__ __align__(16) float qs[HM][D];
+    __shared__ __align__(16) float ps[HM][kDecPer];
+    __shared__ float mh[HM], lh[HM];
     const int sp = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-    const int pos = a.pos[b];
-    const int lo = max(0, pos - a.w + 1);
-    const int n = pos - lo + 1;                        // keys in the window
-    const int s0 = sp * a.per, s1 = min(n, s0 + a.per);
-    for (int h = 0; h < a.H; ++h) qs[h][tid] = __bfloat162float(a.q_rot[((size_t)b * a.H + h) * D + tid]);
-    if (tid < a.H) {
-        mcur[tid] = -INFINITY;
-        lcur[tid] = 0.f;
-    }
-    float o[kMaxH];
-#pragma unroll
-    for (int h = 0; h < kMaxH; ++h) o[h] = 0.f;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int H = a.H;
+    const int n = min(a.pos[b] + 1, a.w);               // slots in the window
+    const int s0 = sp * kDecPer, cnt = max(0, min(n, s0 + kDecPer) - s0);
+    for (int e = tid; e < H * D; e += kDecThreads)
+        qs[e / D][e % D] = __bfloat162float(a.q_rot[(size_t)b * H * D + e]);
+    __syncthreads();
     const __nv_bfloat16* kc = a.cache + (size_t)b * 2 * a.w * D;
     const __nv_bfloat16* vc = kc + (size_t)a.w * D;
-    __syncthreads();
-    for (int i0 = s0; i0 < s1; i0 += kDecKeys) {
-        const int cnt = min(kDecKeys, s1 - i0);
-        // the tile's keys into shared memory (coalesced: a warp reads whole rows)
-        for (int e = tid; e < cnt * (D / 8); e += kDecThreads) {
-            const int i = e / (D / 8), c8 = e % (D / 8);
-            const int slot = (lo + i0 + i) % a.w;
-            *reinterpret_cast<uint4*>(&ks[i][c8 * 8]) = *reinterpret_cast<const uint4*>(kc + (size_t)slot * D + c8 * 8);
-        }
-        __syncthreads();
-        // scores: thread = (head, key) pairs
-        for (int e = tid; e < a.H * cnt; e += kDecThreads) {
-            const int h = e / cnt, i = e % cnt;
-            float acc = 0.f;
-#pragma unroll 8
-            for (int dd = 0; dd < D; ++dd) acc = fmaf(qs[h][dd], __bfloat162float(ks[i][dd]), acc);
-            ps[h][i] = acc * a.scale;
-        }
-        __syncthreads();
-        if (tid < a.H) {                               // running max / sum of head tid
-            const int h = tid;
-            float mx = mcur[h];
-            for (int i = 0; i < cnt; ++i) mx = fmaxf(mx, ps[h][i]);
-            const float f = mcur[h] == -INFINITY ? 0.f : expf(mcur[h] - mx);
-            float l = lcur[h] * f;
-            for (int i = 0; i < cnt; ++i) {
-                const float p = expf(ps[h][i] - mx);
-                ps[h][i] = p;
-                l += p;
+
+    // ---- scores: lane = slot s0 + 32 warp + lane
+#pragma unroll 1
+    for (int i0 = 32 * warp; i0 < kDecPer; i0 += 32 * (kDecThreads / 32)) {
+        const int i = i0 + lane;
+        float2 acc[HM];
+#pragma unroll
+        for (int h = 0; h < HM; ++h) acc[h] = make_float2(0.f, 0.f);
+        if (i < cnt) {
+            const uint4* kr = reinterpret_cast<const uint4*>(kc + (size_t)(s0 + i) * D);
+#pragma unroll 4
+            for (int c = 0; c < D / 8; ++c) {
+                const uint4 kv = __ldg(kr + c);
+                const float2 k0 = bf2_to_f2(kv.x), k1 = bf2_to_f2(kv.y), k2 = bf2_to_f2(kv.z), k3 = bf2_to_f2(kv.w);
+#pragma unroll
+                for (int h = 0; h < HM; ++h) {
+                    if (h < H) {
+                        const float4 qa = *reinterpret_cast<const float4*>(&qs[h][8 * c]);
+                        const float4 qb = *reinterpret_cast<const float4*>(&qs[h][8 * c + 4]);
+                        float2 t = acc[h];
+                        t = __ffma2_rn(make_float2(qa.x, qa.y), k0, t);
+                        t = __ffma2_rn(make_float2(qa.z, qa.w), k1, t);
+                        t = __ffma2_rn(make_float2(qb.x, qb.y), k2, t);
+                        t = __ffma2_rn(make_float2(qb.z, qb.w), k3, t);
+                        acc[h] = t;
+                    }
+                }
             }
-            mcur[h] = mx;
-            lcur[h] = l;
-            fscale[h] = f;
         }
-        __syncthreads();
-        // o[h][tid] = o f + sum_i p v[i][tid]
 #pragma unroll
-        for (int h = 0; h < kMaxH; ++h)
-            if (h < a.H) o[h] *= fscale[h];
-        for (int i = 0; i < cnt; ++i) {
-            const int slot = (lo + i0 + i) % a.w;
-            const float vv = __bfloat162float(vc[(size_t)slot * D + tid]);
+        for (int h = 0; h < HM; ++h)
+            if (h < H) ps[h][i] = i < cnt ? (acc[h].x + acc[h].y) * a.scale : -INFINITY;
+    }
+    __syncthreads();
+
+    // ---- softmax of the split, one warp per head
+    for (int h = warp; h < H; h += kDecThreads / 32) {
+        float v[kDecPer / 32];
+        float mx = -INFINITY;
 #pragma unroll
-            for (int h = 0; h < kMaxH; ++h)
-                if (h < a.H) o[h] = fmaf(ps[h][i], vv, o[h]);
+        for (int j = 0; j < kDecPer / 32; ++j) {
+            v[j] = ps[h][lane + 32 * j];
+            mx = fmaxf(mx, v[j]);
         }
-        __syncthreads();
-    }
-    const size_t pb = ((size_t)b * a.nsplit + sp) * a.H;
-    if (tid < a.H) {
-        a.part_m[pb + tid] = mcur[tid];
-        a.part_l[pb + tid] = lcur[tid];
-    }
 #pragma unroll
-    for (int h = 0; h < kMaxH; ++h)
-        if (h < a.H) a.part_o[(pb + h) * D + tid] = o[h];
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float l = 0.f;
+#pragma unroll
+        for (int j = 0; j < kDecPer / 32; ++j) {
+            const float p = mx == -INFINITY ? 0.f : expf(v[j] - mx);
+            ps[h][lane + 32 * j] = p;
+            l += p;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) {
+            mh[h] = mx;
+            lh[h] = l;
+        }
+    }
+    __syncthreads();
+
+    // ---- o = sum_i p_i v_i: thread = (columns 2 dp, 2 dp + 1; half kh of the slots)
+    const int dp = tid & (D / 2 - 1), kh = tid / (D / 2);
+    const int half = ((cnt + 7) / 8) * 4;                // slots per half, a multiple of 4
+    const int i_beg = kh * half, i_end = min(cnt, i_beg + half);
+    float2 o[HM];
+#pragma unroll
+    for (int h = 0; h < HM; ++h) o[h] = make_float2(0.f, 0.f);
+#pragma unroll 1
+    for (int i = i_beg; i < i_end; i += 4) {
+        float2 vv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            vv[j] = i + j < i_end ? bf2_to_f2(__ldg(reinterpret_cast<const uint32_t*>(vc + (size_t)(s0 + i + j) * D) + dp))
+                                  : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < HM; ++h) {
+            if (h < H) {
+                const float4 p4 = *reinterpret_cast<const float4*>(&ps[h][i]);   // past cnt: 0 or unused
+                float2 t = o[h];
+                t = __ffma2_rn(make_float2(p4.x, p4.x), vv[0], t);
+                t = __ffma2_rn(make_float2(p4.y, p4.y), vv[1], t);
+                t = __ffma2_rn(make_float2(p4.z, p4.z), vv[2], t);
+                t = __ffma2_rn(make_float2(p4.w, p4.w), vv[3], t);
+                o[h] = t;
+            }
+        }
+    }
+    __syncthreads();                                     // the scores are read: reuse qs for the halves
+    float2* red = reinterpret_cast<float2*>(&qs[0][0]);  // [H][D / 2]
+    if (kh == 1) {
+#pragma unroll
+        for (int h = 0; h < HM; ++h)
+            if (h < H) red[h * (D / 2) + dp] = o[h];
+    }
+    __syncthreads();
+    const size_t pb = ((size_t)b * a.nsplit + sp) * H;
+    if (kh == 0) {
+#pragma unroll
+        for (int h = 0; h < HM; ++h)
+            if (h < H) {
+                const float2 r = red[h * (D / 2) + dp];
+                reinterpret_cast<float2*>(a.part_o + (pb + h) * D)[dp] = make_float2(o[h].x + r.x, o[h].y + r.y);
+            }
+    }
+    if (tid < H) {
+        a.part_m[pb + tid] = mh[tid];
+        a.part_l[pb + tid] = lh[tid];
+    }
 }
 
 struct MergeArgs {
@@ -610,7 +675,7 @@ MqaLayout mqa_layout(const rglru_mqa_dims* d, bool decode) {
     size_t o = 256;
     l.q_rot = o; o = up(o + (size_t)d->batch * T * d->q_heads * mq::D * 2);
     l.k_rot = o; o = up(o + (size_t)d->batch * T * mq::D * 2);
-    l.per = 256;
+    l.per = mq::kDecPer;
     l.nsplit = (d->window + l.per - 1) / l.per;
     l.part_m = o; o = up(o + (size_t)d->batch * l.nsplit * d->q_heads * 4);
     l.part_l = o; o = up(o + (size_t)d->batch * l.nsplit * d->q_heads * 4);
@@ -673,12 +738,15 @@ cudaError_t launch_mqa_decode(const rglru_mqa_dims* d, const void* q, const void
     ra.cache = static_cast<__nv_bfloat16*>(cache);
     mqa_rope_decode_kernel<<<B, D / 2, 0, s>>>(ra);
     DecArgs da{};
-    da.B = B; da.H = H; da.w = d->window; da.nsplit = l.nsplit; da.per = l.per; da.scale = d->scale;
+    da.B = B; da.H = H; da.w = d->window; da.nsplit = l.nsplit; da.scale = d->scale;
     da.q_rot = ra.q_rot; da.pos = pos; da.cache = ra.cache;
     da.part_m = reinterpret_cast<float*>(w + l.part_m);
     da.part_l = reinterpret_cast<float*>(w + l.part_l);
     da.part_o = reinterpret_cast<float*>(w + l.part_o);
-    mqa_decode_kernel<<<dim3(l.nsplit, B), kDecThreads, 0, s>>>(da);
+    const dim3 grid(l.nsplit, B);
+    if (H <= 4) mqa_decode_kernel<4><<<grid, kDecThreads, 0, s>>>(da);
+    else if (H <= 8) mqa_decode_kernel<8><<<grid, kDecThreads, 0, s>>>(da);
+    else mqa_decode_kernel<16><<<grid, kDecThreads, 0, s>>>(da);
     MergeArgs ma{};
     ma.B = B; ma.H = H; ma.nsplit = l.nsplit;
     ma.part_m = da.part_m; ma.part_l = da.part_l; ma.part_o = da.part_o;

@@ -54,10 +54,15 @@ def test_mqa_prefill_matches_oracle(B, T, H, w):
     assert_attention_close(to_np(out), ref, pav, f"mqa prefill B{B} T{T} H{H} w{w}")
 
 
-def test_mqa_decode_continues_the_prefill_through_the_ring():
-    """Prefill 150 tokens with the cache, then 40 decode steps (rows at different positions);
-    each step against the oracle's ring-buffer decode."""
-    B, T0, H, w, steps = 2, 150, 4, 64, 40
+@pytest.mark.parametrize("T0,H,w,steps", [
+    (150, 4, 64, 40),      # a full ring that wraps many times
+    (300, 10, 600, 6),     # a ring not yet full, window cut into splits (one of them empty)
+    (700, 3, 600, 4),      # a full ring of several splits, the last one ragged
+])
+def test_mqa_decode_continues_the_prefill_through_the_ring(T0, H, w, steps):
+    """Prefill T0 tokens with the cache, then decode steps; each step against the oracle's
+    ring-buffer decode."""
+    B = 2
     rng = np.random.default_rng(7)
     q, k, v = _bf16(rng, (B, T0, H, D)), _bf16(rng, (B, T0, D)), _bf16(rng, (B, T0, D))
     dims = binding.make_mqa_dims(B, T0, H, D, w)
