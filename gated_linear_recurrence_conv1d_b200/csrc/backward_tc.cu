@@ -5,17 +5,22 @@
 // "Griffin Guide: RecurrentGemma, RG-LRU & Hybrid Attention": "1. Formulation of the RG-LRU
 // Gating Mechanism", "2. The Role of Square-Root Variance Normalization", "1. Temporal Filtering
 // via Separable 1D Convolutions", "2. Non-Linear Multiplicative Gating with GeLU", "3.
-// Block-Diagonal Sharding ..."), computed in six launches:
+// Block-Diagonal Sharding ..."), computed in these steps:
 //
 //   1. the tensor-core prefill in its save mode (fused_prefill.cu) runs the forward again and
 //      keeps, per token-channel, the complete gate pre-activations ga, gx (fp32), h_{t-1} as the
 //      update used it (fp32) and the conv output as a bf16 pair hi + lo (x = hi + lo to 2^-16);
 //      its gate contraction runs on both bf16 parts of the conv output, so the pre-activations
 //      are those of the fp32 conv output;
-//   2. bwd_scan_kernel: one thread per (row, channel) walks the tokens backwards carrying
-//      g = dL/dh_t:  g_t = dout_t GeLU(y_t) + a_{t+1} g_{t+1} (0 across a reset); it writes
-//      dy, the direct part of dL/dxc (g beta i) and dL/dga, dL/dgx as bf16 hi / lo pairs, and
-//      per-row partial sums of dLambda, db_a, db_x;
+//   2. the reverse scan of g = dL/dh_t:  g_t = dout_t GeLU(y_t) + a_{t+1} g_{t+1} (0 across a
+//      reset), a first-order linear recurrence run backwards, cut into chunks of kChunk tokens:
+//      bwd_scan_agg_kernel gives each (row, chunk, channel) its map c -> P c + Q from the carry
+//      entering the chunk's last token to the one leaving its first (P the product of the a_t,
+//      Q the chunk's own contribution); bwd_scan_carry_kernel chains the maps of a row from the
+//      last chunk to the first (dh_final in, dL/dh_{-1} out); bwd_scan_out_kernel walks every
+//      chunk again from its carry and writes dy, the direct part of dL/dxc (g beta i) and
+//      dL/dga, dL/dgx as bf16 hi / lo pairs, and per-(row, chunk) partial sums of dLambda, db_a,
+//      db_x;
 //   3. dL/dxc += dga W_a^T + dgx W_x^T: a tensor-core GEMM per head over the B T tokens with the
 //      hi and lo parts of dga and dgx as four K ranges (gemm.cu);
 //   4. bwd_convT_kernel: the conv's transpose in parallel over (row, 64-token block, channel):
@@ -27,12 +32,15 @@
 //      are kept apart;
 //   6. bwdtc_reduce_kernel: every partial sum in a fixed order.
 // No atomics: the gradients are bitwise repeatable.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "rglru_math.cuh"
 
 namespace rglru {
 
@@ -40,13 +48,14 @@ namespace {
 
 constexpr int DH = 256;
 constexpr int kTB = 64;          // tokens per conv-transpose block
-constexpr int kSplits = 4;       // K slices of the weight-gradient GEMMs
+constexpr int kMaxSplits = 16;   // K slices of the weight-gradient GEMMs, at most
 constexpr int kScanThreads = 128;
+constexpr int kChunk = 64;       // tokens per chunk of the reverse scan
 
 struct Layout {
     size_t ga, gx, hprev, dxc, xc_hi, xc_lo, dga_hi, dga_lo, dgx_hi, dgx_lo;
-    size_t part_scan, part_conv, dw, fwd, total;
-    int ntb;
+    size_t agg, part_scan, part_conv, dw, fwd, total;
+    int ntb, nch;
 };
 
 Layout layout(const rglru_dims* d) {
@@ -55,6 +64,7 @@ Layout layout(const rglru_dims* d) {
     const size_t n = (size_t)d->batch * d->seq_len * W;
     Layout l;
     l.ntb = (d->seq_len + kTB - 1) / kTB;
+    l.nch = (d->seq_len + kChunk - 1) / kChunk;
     size_t o = 256;
     l.ga = o;      o = up(o + n * 4);
     l.gx = o;      o = up(o + n * 4);
@@ -66,9 +76,10 @@ Layout layout(const rglru_dims* d) {
     l.dga_lo = o;  o = up(o + n * 2);
     l.dgx_hi = o;  o = up(o + n * 2);
     l.dgx_lo = o;  o = up(o + n * 2);
-    l.part_scan = o; o = up(o + 3 * (size_t)d->batch * W * 4);
+    l.agg = o;     o = up(o + 2 * (size_t)d->batch * l.nch * W * 4);
+    l.part_scan = o; o = up(o + 3 * (size_t)d->batch * l.nch * W * 4);
     l.part_conv = o; o = up(o + 5 * (size_t)d->batch * l.ntb * W * 4);
-    l.dw = o;      o = up(o + 2 * (size_t)kSplits * d->heads * DH * DH * 4);
+    l.dw = o;      o = up(o + 2 * (size_t)kMaxSplits * d->heads * DH * DH * 4);
     l.fwd = o;     o = up(o + fused_prefill_workspace(d));
     l.total = o;
     return l;
@@ -86,6 +97,33 @@ __device__ __forceinline__ float gelu_grad(float v, int tanh_form) {
     return 0.5f * erfcf(-v * 0.70710678118654752440f) + v * expf(-0.5f * v * v) * 0.39894228040143267794f;
 }
 
+// The per-token arithmetic of the reverse scan, with hardware exp2 / reciprocal (relative
+// errors near 2^-22) where CUDA's accurate functions would cost several times the instructions:
+//   sigma(z) = 1 / (1 + 2^(-z log2 e));
+//   a = 1 + E, E = expm1(c r log sigma(Lambda)) by its series to l^5 for l >= -1/8 (no
+//   cancellation as a -> 1, where the reverse recurrence carries errors of a over ~1 / (1 - a)
+//   tokens), else 2^(l log2 e) - 1; beta = sqrt(1 - a^2) = sqrt(-E (2 + E));
+//   GeLU and its derivative from one erfc: Phi(v) = erfc(-v / sqrt 2) / 2, GeLU = v Phi,
+//   GeLU' = Phi + v phi(v) (the tanh form keeps tanhf).
+__device__ __forceinline__ float sig_fast(float z) { return fm::rcpf(1.0f + fm::ex2f(-z * fm::kLog2e)); }
+
+__device__ __forceinline__ void decay_beta_fast(float kappa, float r, float& at, float& beta) {
+    const float E = fm::expm1_any(kappa * r);
+    at = 1.0f + E;
+    beta = sqrtf(-E * (2.0f + E));
+}
+
+__device__ __forceinline__ void gelu_and_grad(float v, int tanh_form, float& g, float& gp) {
+    if (tanh_form) {
+        g = gelu_acc(v, 1);
+        gp = gelu_grad(v, 1);
+        return;
+    }
+    const float phi_c = 0.5f * erfcf(-v * 0.70710678118654752440f);
+    g = v * phi_c;
+    gp = fmaf(v * fm::ex2f((v * v) * (-0.5f * fm::kLog2e)), 0.39894228040143267794f, phi_c);
+}
+
 __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bfloat16* lo) {
     const __nv_bfloat16 h = __float2bfloat16_rn(v);
     *hi = h;
@@ -93,7 +131,7 @@ __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bflo
 }
 
 struct ScanArgs {
-    int B, T, W;
+    int B, T, W, nch;
     float c;
     int gelu_tanh;
     const float* lambda;
@@ -113,51 +151,128 @@ struct ScanArgs {
     __nv_bfloat16* dgx_hi;
     __nv_bfloat16* dgx_lo;
     float* dh0;
-    float* part;          // [3][B][W]: dLambda, db_a, db_x
+    float* agg;           // [2][B][nch][W]: P, Q of each chunk, then Q replaced by the carry into it
+    float* part;          // [3][B][nch][W]: dLambda, db_a, db_x
 };
 
 // ---------------------------------------------------------------- 2. the reverse scan -------
-// Thread = (row b, channel ch); the inputs of a block of kPF tokens are loaded together before
-// the block is walked, so that their latencies overlap.
+// Thread = (row b, chunk k, channel ch); the inputs of a block of kPF tokens are loaded together
+// before the block is walked, so that their latencies overlap.
 constexpr int kPF = 8;
-__global__ void __launch_bounds__(kScanThreads) bwd_scan_kernel(ScanArgs a) {
+
+// a'_t: the factor that carries g from token t to t - 1 (a_t, or 0 where t starts a segment)
+__device__ __forceinline__ float carry_factor(float kappa, float ga, bool rs) {
+    const float at = 1.0f + fm::expm1_any(kappa * sig_fast(ga));
+    return rs ? 0.f : at;
+}
+
+// P = prod a'_t and Q = the carry leaving the chunk's first token when none enters its last
+__global__ void __launch_bounds__(kScanThreads) bwd_scan_agg_kernel(ScanArgs a) {
+    const int ch = blockIdx.x * kScanThreads + threadIdx.x, k = blockIdx.y, b = blockIdx.z;
+    if (ch >= a.W) return;
+    const float kappa = a.c * log_sigmoid_acc(a.lambda[ch]);
+    const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
+    const int t0 = k * kChunk, t1 = min(a.T, t0 + kChunk);
+    float P = 1.f, g = 0.f;
+    for (int tb = t1 - kPF; tb > t0 - kPF; tb -= kPF) {
+        float vga[kPF], vy[kPF], vdz[kPF];
+        bool rs[kPF];
+#pragma unroll
+        for (int j = 0; j < kPF; ++j) {
+            const int t = tb + j;
+            if (t >= t0) {
+                const size_t e = ((size_t)b * a.T + t) * a.W + ch;
+                vga[j] = a.ga[e];
+                vy[j] = bf(a.y + e);
+                vdz[j] = bf(a.dout + e);
+                rs[j] = rrow && rrow[t];
+            }
+        }
+#pragma unroll
+        for (int j = kPF - 1; j >= 0; --j) {
+            if (tb + j < t0) continue;
+            float gl, gp;
+            gelu_and_grad(vy[j], a.gelu_tanh, gl, gp);
+            g = fmaf(vdz[j], gl, g);
+            const float f = carry_factor(kappa, vga[j], rs[j]);
+            g *= f;
+            P *= f;
+        }
+    }
+    const size_t pb = (size_t)a.B * a.nch * a.W, pi = ((size_t)b * a.nch + k) * a.W + ch;
+    a.agg[pi] = P;
+    a.agg[pb + pi] = g;
+}
+
+// per (row, channel): the carries into every chunk, from the last chunk to the first
+__global__ void __launch_bounds__(kScanThreads) bwd_scan_carry_kernel(ScanArgs a) {
     const int ch = blockIdx.x * kScanThreads + threadIdx.x, b = blockIdx.y;
+    if (ch >= a.W) return;
+    const size_t pb = (size_t)a.B * a.nch * a.W;
+    float c = a.dh_final ? a.dh_final[(size_t)b * a.W + ch] : 0.f;
+    for (int kb = a.nch - kPF; kb > -kPF; kb -= kPF) {
+        float vp[kPF], vq[kPF];
+#pragma unroll
+        for (int j = 0; j < kPF; ++j) {
+            if (kb + j >= 0) {
+                const size_t pi = ((size_t)b * a.nch + kb + j) * a.W + ch;
+                vp[j] = a.agg[pi];
+                vq[j] = a.agg[pb + pi];
+            }
+        }
+#pragma unroll
+        for (int j = kPF - 1; j >= 0; --j) {
+            if (kb + j < 0) continue;
+            a.agg[pb + ((size_t)b * a.nch + kb + j) * a.W + ch] = c;
+            c = fmaf(vp[j], c, vq[j]);
+        }
+    }
+    if (a.dh0) a.dh0[(size_t)b * a.W + ch] = c;
+}
+
+// every output of a chunk, from the carry into its last token
+__global__ void __launch_bounds__(kScanThreads) bwd_scan_out_kernel(ScanArgs a) {
+    const int ch = blockIdx.x * kScanThreads + threadIdx.x, k = blockIdx.y, b = blockIdx.z;
     if (ch >= a.W) return;
     const float kappa = a.c * log_sigmoid_acc(a.lambda[ch]);
     const float c_sneg = a.c * sigmoid_acc(-a.lambda[ch]);
-    float g = a.dh_final ? a.dh_final[(size_t)b * a.W + ch] : 0.f;
+    const size_t pb = (size_t)a.B * a.nch * a.W, pi = ((size_t)b * a.nch + k) * a.W + ch;
+    float g = a.agg[pb + pi];
     float s_lam = 0.f, s_ba = 0.f, s_bx = 0.f;
     const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
-    for (int tb = ((a.T - 1) / kPF) * kPF; tb >= 0; tb -= kPF) {
-        const int n = min(kPF, a.T - tb);
+    const int t0 = k * kChunk, t1 = min(a.T, t0 + kChunk);
+    for (int tb = t1 - kPF; tb > t0 - kPF; tb -= kPF) {
         float vga[kPF], vgx[kPF], vhp[kPF], vxc[kPF], vy[kPF], vdz[kPF];
         bool rs[kPF];
 #pragma unroll
         for (int j = 0; j < kPF; ++j) {
-            if (j < n) {
-                const size_t e = ((size_t)b * a.T + tb + j) * a.W + ch;
+            const int t = tb + j;
+            if (t >= t0) {
+                const size_t e = ((size_t)b * a.T + t) * a.W + ch;
                 vga[j] = a.ga[e];
                 vgx[j] = a.gx[e];
                 vhp[j] = a.hprev[e];
                 vxc[j] = bf(a.xc_hi + e) + bf(a.xc_lo + e);
                 vy[j] = bf(a.y + e);
                 vdz[j] = bf(a.dout + e);
-                rs[j] = rrow && rrow[tb + j];
+                rs[j] = rrow && rrow[t];
             }
         }
 #pragma unroll
         for (int j = kPF - 1; j >= 0; --j) {
-            if (j >= n) continue;
+            if (tb + j < t0) continue;
             const size_t e = ((size_t)b * a.T + tb + j) * a.W + ch;
-            const float r = sigmoid_acc(vga[j]), ig = sigmoid_acc(vgx[j]);
+            const float r = sig_fast(vga[j]), ig = sig_fast(vgx[j]);
             float at, beta;
-            decay_and_beta_acc(kappa, r, &at, &beta);
+            decay_beta_fast(kappa, r, at, beta);
             const float xcv = vxc[j], hp = vhp[j];
             const float h = fmaf(at, hp, beta * (ig * xcv));
-            g = fmaf(vdz[j], gelu_acc(vy[j], a.gelu_tanh), g);
-            a.dy[e] = vdz[j] * h * gelu_grad(vy[j], a.gelu_tanh);
+            float gl, gp;
+            gelu_and_grad(vy[j], a.gelu_tanh, gl, gp);
+            g = fmaf(vdz[j], gl, g);
+            a.dy[e] = vdz[j] * h * gp;
             const float dl_da = g * hp, dl_dbeta = g * ig * xcv, dl_di = g * beta * xcv;
-            const float r_over_beta = beta > 0.f ? r / beta : 0.f;
+            const float r_over_beta = beta > 0.f ? r * fm::rcpf(beta) : 0.f;
             const float q = dl_da * at * r - dl_dbeta * at * at * r_over_beta;
             const float dga = kappa * (1.0f - r) * q;
             const float dgx = dl_di * ig * (1.0f - ig);
@@ -170,15 +285,12 @@ __global__ void __launch_bounds__(kScanThreads) bwd_scan_kernel(ScanArgs a) {
             g = rs[j] ? 0.f : at * g;
         }
     }
-    if (a.dh0) a.dh0[(size_t)b * a.W + ch] = g;
-    const size_t pb = (size_t)a.B * a.W;
-    float* p = a.part + (size_t)b * a.W + ch;
-    p[0 * pb] = s_lam;
-    p[1 * pb] = s_ba;
-    p[2 * pb] = s_bx;
+    const size_t ps = (size_t)a.B * a.nch * a.W;
+    a.part[pi] = s_lam;
+    a.part[ps + pi] = s_ba;
+    a.part[2 * ps + pi] = s_bx;
 }
 
-// ---------------------------------------------------------------- 4. the conv's transpose ---
 struct ConvTArgs {
     int B, T, W, ntb;
     const float* conv_w;
@@ -200,77 +312,108 @@ __device__ __forceinline__ bool window_reads(const uint8_t* rrow, int s, int t) 
     return true;
 }
 
+// Thread = (row b, block of kTB positions, channel ch); one walk over the block's positions s
+// with the last three x and the next three dxc in registers: the parameter gradients of token
+// t = s (the taps that read x_{s-3..s}) and dx_s (the taps of the tokens s..s+3 that read x_s).
+// A window reads position s for token t when no segment starts in (s, t]: L below is the last
+// segment start at or before the current token.
 __global__ void __launch_bounds__(128) bwd_convT_kernel(ConvTArgs a) {
     const int ch = blockIdx.x * 128 + threadIdx.x, tb = blockIdx.y, b = blockIdx.z;
     if (ch >= a.W) return;
     const int t0 = tb * kTB, t1 = min(a.T, t0 + kTB);
     const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
+    const size_t rowe = (size_t)b * a.T * a.W + ch;        // element (b, 0, ch)
     float cw[kConvWidth];
 #pragma unroll
     for (int k = 0; k < kConvWidth; ++k) cw[k] = a.conv_w[(size_t)k * a.W + ch];
     auto xval = [&](int s) -> float {                       // x_s, the initial history for s < 0
-        if (s >= 0) return bf(a.x + ((size_t)b * a.T + s) * a.W + ch);
+        if (s >= 0) return bf(a.x + rowe + (size_t)s * a.W);
         return a.tail0 ? bf(a.tail0 + ((size_t)b * kHist + (kHist + s)) * a.W + ch) : 0.f;
     };
-    auto dxcv = [&](int t) -> float { return a.dxc[((size_t)b * a.T + t) * a.W + ch]; };
-    // parameter gradients over the block's tokens
+    auto dxcv = [&](int t) -> float { return t >= 0 && t < a.T ? a.dxc[rowe + (size_t)t * a.W] : 0.f; };
+    auto rs = [&](int p) -> bool { return rrow && p >= 0 && p < a.T && rrow[p] != 0; };
+
+    int L = -kHist - 1;                                     // no segment start within reach
+    for (int p = max(0, t0 - kHist); p < t0; ++p)
+        if (rs(p)) L = p;
+    float xa = xval(t0 - 3), xb = xval(t0 - 2), xcc = xval(t0 - 1);   // x_{t-3}, x_{t-2}, x_{t-1}
     float s_cw[kConvWidth] = {0.f, 0.f, 0.f, 0.f}, s_cb = 0.f;
-    for (int t = t0; t < t1; ++t) {
-        const float d = dxcv(t);
-        s_cb += d;
-#pragma unroll
-        for (int k = 0; k < kConvWidth; ++k) {
-            const int s = t - kHist + k;
-            if (window_reads(rrow, s, t)) s_cw[k] = fmaf(d, xval(s), s_cw[k]);
+    const int sb = tb == 0 ? -kHist : t0;                   // the first block also owns the history
+    float d0 = dxcv(sb), d1 = dxcv(sb + 1), d2 = dxcv(sb + 2);
+    bool q0 = rs(sb), q1 = rs(sb + 1), q2 = rs(sb + 2);
+    for (int s = sb; s < t1; ++s) {
+        const float d3 = dxcv(s + 3);
+        const bool q3 = rs(s + 3);
+        if (s >= t0) {                                      // token t = s: its four taps
+            const float xs = bf(a.x + rowe + (size_t)s * a.W);
+            if (q0) L = s;
+            s_cb += d0;
+            if (s - 3 >= L) s_cw[0] = fmaf(d0, xa, s_cw[0]);
+            if (s - 2 >= L) s_cw[1] = fmaf(d0, xb, s_cw[1]);
+            if (s - 1 >= L) s_cw[2] = fmaf(d0, xcc, s_cw[2]);
+            s_cw[3] = fmaf(d0, xs, s_cw[3]);
+            xa = xb; xb = xcc; xcc = xs;
         }
+        // dx_s: tap k of token s + 3 - k, while no segment starts in (s, s + 3 - k]
+        const bool ok1 = !q1, ok2 = ok1 && !q2, ok3 = ok2 && !q3;
+        float acc = 0.f;
+        if (ok3 && s + 3 >= 0 && s + 3 < a.T) acc = fmaf(cw[0], d3, acc);
+        if (ok2 && s + 2 >= 0 && s + 2 < a.T) acc = fmaf(cw[1], d2, acc);
+        if (ok1 && s + 1 >= 0 && s + 1 < a.T) acc = fmaf(cw[2], d1, acc);
+        if (s >= 0) acc = fmaf(cw[3], d0, acc);
+        if (a.dtail_final && s >= a.T - kHist && window_reads(rrow, s, a.T - 1))
+            acc += a.dtail_final[((size_t)b * kHist + (s - (a.T - kHist))) * a.W + ch];
+        if (s >= 0) a.dx[rowe + (size_t)s * a.W] = acc;
+        else if (a.dtail0) a.dtail0[((size_t)b * kHist + (kHist + s)) * a.W + ch] = acc;
+        d0 = d1; d1 = d2; d2 = d3;
+        q0 = q1; q1 = q2; q2 = q3;
     }
     const size_t pb = (size_t)a.B * a.ntb * a.W, pi = ((size_t)b * a.ntb + tb) * a.W + ch;
 #pragma unroll
     for (int k = 0; k < kConvWidth; ++k) a.part[k * pb + pi] = s_cw[k];
     a.part[4 * pb + pi] = s_cb;
-    // dx of the block's positions (and the initial history, from the first block)
-    for (int s = (tb == 0 ? -kHist : t0); s < t1; ++s) {
-        float acc = 0.f;
-#pragma unroll
-        for (int k = 0; k < kConvWidth; ++k) {
-            const int t = s + kHist - k;                     // the token whose tap k reads s
-            if (t >= 0 && t < a.T && window_reads(rrow, s, t)) acc = fmaf(cw[k], dxcv(t), acc);
-        }
-        if (a.dtail_final && s >= a.T - kHist && window_reads(rrow, s, a.T - 1))
-            acc += a.dtail_final[((size_t)b * kHist + (s - (a.T - kHist))) * a.W + ch];
-        if (s >= 0) a.dx[((size_t)b * a.T + s) * a.W + ch] = acc;
-        else if (a.dtail0) a.dtail0[((size_t)b * kHist + (kHist + s)) * a.W + ch] = acc;
-    }
 }
 
 // ---------------------------------------------------------------- 6. fixed-order sums -------
 struct ReduceArgs {
-    int B, ntb, W, H;
+    int B, ntb, nch, W, H, splits;
     const float* part_scan;
     const float* part_conv;
-    const float* dw;                  // [2][kSplits][H][256][256]
+    const float* dw;                  // [2][splits][H][256][256]
     rglru_grads g;
 };
 
-__global__ void bwdtc_reduce_vec_kernel(ReduceArgs a) {
-    const int ch = blockIdx.x * blockDim.x + threadIdx.x;
-    if (ch >= a.W) return;
-    const size_t ps = (size_t)a.B * a.W;
-    float s[3] = {0.f, 0.f, 0.f};
-    for (int b = 0; b < a.B; ++b)
+// Block = 32 channels x kRedGroups row groups: group g sums the partial rows i = g (mod
+// kRedGroups) in order, then the groups are added in order -- a fixed order, so the sums repeat
+// bitwise.
+constexpr int kRedGroups = 16;
+__global__ void __launch_bounds__(32 * kRedGroups) bwdtc_reduce_vec_kernel(ReduceArgs a) {
+    __shared__ float red[8][kRedGroups][33];
+    const int c = threadIdx.x, g = threadIdx.y;
+    const int ch = blockIdx.x * 32 + c;
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (ch < a.W) {
+        const size_t ps = (size_t)a.B * a.nch * a.W;
+        for (int i = g; i < a.B * a.nch; i += kRedGroups)
 #pragma unroll
-        for (int k = 0; k < 3; ++k) s[k] += a.part_scan[k * ps + (size_t)b * a.W + ch];
-    a.g.dlambda[ch] = s[0];
-    a.g.db_a[ch] = s[1];
-    a.g.db_x[ch] = s[2];
-    const size_t pc = (size_t)a.B * a.ntb * a.W;
-    float c[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int i = 0; i < a.B * a.ntb; ++i)
+            for (int k = 0; k < 3; ++k) s[k] += a.part_scan[k * ps + (size_t)i * a.W + ch];
+        const size_t pc = (size_t)a.B * a.ntb * a.W;
+        for (int i = g; i < a.B * a.ntb; i += kRedGroups)
 #pragma unroll
-        for (int k = 0; k < 5; ++k) c[k] += a.part_conv[k * pc + (size_t)i * a.W + ch];
+            for (int k = 0; k < 5; ++k) s[3 + k] += a.part_conv[k * pc + (size_t)i * a.W + ch];
+    }
 #pragma unroll
-    for (int k = 0; k < kConvWidth; ++k) a.g.dconv_w[(size_t)k * a.W + ch] = c[k];
-    a.g.dconv_b[ch] = c[4];
+    for (int k = 0; k < 8; ++k) red[k][g][c] = s[k];
+    __syncthreads();
+    if (g < 8 && ch < a.W) {
+        float t = 0.f;
+        for (int j = 0; j < kRedGroups; ++j) t += red[g][j][c];
+        if (g == 0) a.g.dlambda[ch] = t;
+        else if (g == 1) a.g.db_a[ch] = t;
+        else if (g == 2) a.g.db_x[ch] = t;
+        else if (g < 7) a.g.dconv_w[(size_t)(g - 3) * a.W + ch] = t;
+        else a.g.dconv_b[ch] = t;
+    }
 }
 
 __global__ void bwdtc_reduce_w_kernel(ReduceArgs a) {
@@ -280,7 +423,7 @@ __global__ void bwdtc_reduce_w_kernel(ReduceArgs a) {
 #pragma unroll
     for (int gate = 0; gate < 2; ++gate) {
         float s = 0.f;
-        for (int sp = 0; sp < kSplits; ++sp) s += a.dw[((size_t)gate * kSplits + sp) * n + i];
+        for (int sp = 0; sp < a.splits; ++sp) s += a.dw[((size_t)gate * a.splits + sp) * n + i];
         (gate ? a.g.dw_x : a.g.dw_a)[i] = s;
     }
 }
@@ -319,7 +462,7 @@ size_t backward_tc_workspace(const rglru_dims* d) { return layout(d).total; }
 
 int backward_tc_launches(const rglru_dims* d) {
     (void)d;
-    return 9;   // prefill (memset + kernel), scan, GEMM, conv transpose, 2 GEMMs, 2 reductions
+    return 11;  // prefill (memset + kernel), 3 scan kernels, GEMM, conv transpose, 2 GEMMs, 2 reductions
 }
 
 cudaError_t launch_backward_tc(const rglru_dims* d, const rglru_params* p, const void* x, const void* y,
@@ -350,15 +493,18 @@ cudaError_t launch_backward_tc(const rglru_dims* d, const rglru_params* p, const
 
     // 2. the reverse scan
     ScanArgs sa{};
-    sa.B = B; sa.T = T; sa.W = W; sa.c = d->c; sa.gelu_tanh = d->gelu_tanh;
+    sa.B = B; sa.T = T; sa.W = W; sa.nch = l.nch; sa.c = d->c; sa.gelu_tanh = d->gelu_tanh;
     sa.lambda = p->lambda; sa.y = static_cast<const __nv_bfloat16*>(y);
     sa.dout = static_cast<const __nv_bfloat16*>(dout); sa.reset = reset; sa.dh_final = dh_final;
     sa.ga = f32(l.ga); sa.gx = f32(l.gx); sa.hprev = f32(l.hprev);
     sa.xc_hi = b16(l.xc_hi); sa.xc_lo = b16(l.xc_lo);
     sa.dy = grads->dy; sa.dxc = f32(l.dxc);
     sa.dga_hi = b16(l.dga_hi); sa.dga_lo = b16(l.dga_lo); sa.dgx_hi = b16(l.dgx_hi); sa.dgx_lo = b16(l.dgx_lo);
-    sa.dh0 = grads->dh0; sa.part = f32(l.part_scan);
-    bwd_scan_kernel<<<dim3((W + kScanThreads - 1) / kScanThreads, B), kScanThreads, 0, s>>>(sa);
+    sa.dh0 = grads->dh0; sa.agg = f32(l.agg); sa.part = f32(l.part_scan);
+    const unsigned cblk = (unsigned)((W + kScanThreads - 1) / kScanThreads);
+    bwd_scan_agg_kernel<<<dim3(cblk, l.nch, B), kScanThreads, 0, s>>>(sa);
+    bwd_scan_carry_kernel<<<dim3(cblk, B), kScanThreads, 0, s>>>(sa);
+    bwd_scan_out_kernel<<<dim3(cblk, l.nch, B), kScanThreads, 0, s>>>(sa);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -388,16 +534,22 @@ cudaError_t launch_backward_tc(const rglru_dims* d, const rglru_params* p, const
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
-    // 5. dW = xc^T dg per head and gate, K (the tokens) cut into kSplits slices
+    // 5. dW = xc^T dg per head and gate, K (the tokens) cut into slices so that the tiles of
+    //    both gates' GEMM fill the SMs about once
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return cudaGetLastError();
+    const int wtiles = H * (DH / 128);                     // 128 x 256 output tiles per gate
+    const int splits = std::max(1, std::min(kMaxSplits, sms / wtiles));
     for (int gate = 0; gate < 2; ++gate) {
         GemmOperands gw{};
-        gw.M = DH; gw.N = DH; gw.batch = H; gw.splits = kSplits; gw.npairs = 3;
+        gw.M = DH; gw.N = DH; gw.batch = H; gw.splits = splits; gw.npairs = 3;
         const __nv_bfloat16* hi = b16(gate ? l.dgx_hi : l.dga_hi);
         const __nv_bfloat16* lo = b16(gate ? l.dgx_lo : l.dga_lo);
         gw.p[0] = pair_xc_dg(b16(l.xc_hi), hi, tokens, W);
         gw.p[1] = pair_xc_dg(b16(l.xc_hi), lo, tokens, W);
         gw.p[2] = pair_xc_dg(b16(l.xc_lo), hi, tokens, W);
-        gw.C = f32(l.dw) + (size_t)gate * kSplits * H * DH * DH;
+        gw.C = f32(l.dw) + (size_t)gate * splits * H * DH * DH;
         gw.c_ld = DH; gw.c_bstride = (long long)DH * DH; gw.c_split = (long long)H * DH * DH;
         gw.Cadd = nullptr;
         gw.status = status;
@@ -407,10 +559,10 @@ cudaError_t launch_backward_tc(const rglru_dims* d, const rglru_params* p, const
 
     // 6. every partial sum, in a fixed order
     ReduceArgs ra{};
-    ra.B = B; ra.ntb = l.ntb; ra.W = W; ra.H = H;
+    ra.B = B; ra.ntb = l.ntb; ra.nch = l.nch; ra.W = W; ra.H = H; ra.splits = splits;
     ra.part_scan = f32(l.part_scan); ra.part_conv = f32(l.part_conv); ra.dw = f32(l.dw);
     ra.g = *grads;
-    bwdtc_reduce_vec_kernel<<<(W + 255) / 256, 256, 0, s>>>(ra);
+    bwdtc_reduce_vec_kernel<<<(W + 31) / 32, dim3(32, kRedGroups), 0, s>>>(ra);
     const size_t nw = (size_t)H * DH * DH;
     bwdtc_reduce_w_kernel<<<(unsigned)((nw + 255) / 256), 256, 0, s>>>(ra);
     return cudaGetLastError();

@@ -13,10 +13,12 @@
 //     contiguous: element (m, k) at k * ld + m); B likewise N x K, "K-major" or "N-major".  The
 //     operands are read by TMA in 128-byte swizzled tiles straight from the caller's tensors
 //     (2-D maps; the batch index adds a fixed row or column offset);
-//   * a persistent CTA per SM walks output tiles of 128 x 128 (batch, m-tile, n-tile, k-slice);
-//     one warp loads K blocks of 64 through a 4-stage ring, one thread issues tcgen05.mma
-//     (M = 128, N = 128, K = 16 per instruction) into one of two TMEM accumulators, and 4
-//     epilogue warps (thread = row of the tile) read the other accumulator, add Cadd and store.
+//   * a persistent CTA per SM walks output tiles of 128 x 256 (batch, m-tile, n-tile, k-slice);
+//     one warp loads K blocks of 64 through a 4-stage ring (48 KB a stage), an elected lane of
+//     another issues tcgen05.mma (M = 128, N = 256, K = 16 per instruction) into one of two TMEM
+//     accumulators of 256 columns, and 4 epilogue warps (thread = row of the tile) read the
+//     other accumulator, add Cadd and store.  The wide tile halves the operand bytes per flop
+//     that L2 has to deliver to each SM, compared with a square 128 x 128 tile.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -34,10 +36,10 @@ namespace gm {
 
 using namespace sm100;
 
-constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int STAGES = 4;
 constexpr uint32_t TILE_A = BM * BK * 2;           // 16384
-constexpr uint32_t TILE_B = BN * BK * 2;           // 16384
+constexpr uint32_t TILE_B = BN * BK * 2;           // 32768
 constexpr uint32_t STAGE_BYTES = TILE_A + TILE_B;
 constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
@@ -111,8 +113,8 @@ __device__ __forceinline__ bool wait_b(uint32_t bar, uint32_t parity, const Args
     return wait_slow(bar, parity, a, abort, where);
 }
 
-// Shared-memory descriptors (128-byte swizzle) of a 128-row, 64-wide tile: K-major (rows of
-// 128 B = 64 K, 8-row atoms 1024 B apart) or MN-major (two 64-wide MN atoms of 64 K-rows each,
+// Shared-memory descriptors (128-byte swizzle) of a 128- or 256-row, 64-wide tile: K-major (rows
+// of 128 B = 64 K, 8-row atoms 1024 B apart) or MN-major (64-wide MN atoms of 64 K-rows each,
 // 8192 B apart; 8-row K groups 1024 B apart)
 __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr) {
     uint64_t d = 0;
@@ -222,8 +224,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
                     if (p.b_kmajor) {
                         tma_load_2d(sb, mb, bc + k0, br + n0, full(s));
                     } else {
-                        tma_load_2d(sb, mb, bc + n0, br + k0, full(s));
-                        tma_load_2d(sb + 8192, mb, bc + n0 + 64, br + k0, full(s));
+#pragma unroll
+                        for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, mb, bc + n0 + 64 * j, br + k0, full(s));
                     }
                 }
             }

@@ -86,6 +86,15 @@ def test_backward_matches_oracle(B, T, H, dh, dtype, tanh):
     _compare(grads, ref, f"B{B} T{T} H{H} dh{dh} {dtype}")
 
 
+def test_backward_long_carry_across_many_chunks():
+    """The tensor-core reverse scan cuts a row into chunks and chains their carries: rows of
+    1100 tokens (18 chunks, a ragged last one, more than one prefetch block of chunks) with
+    documents of several hundred tokens, so that g crosses many chunk boundaries."""
+    wl = inputs.WORKLOADS["packed_bf16"].scaled(batch=2, seq_len=1100, heads=1, doc_len=(300, 900))
+    grads, ref = _run(wl, seed=77)
+    _compare(grads, ref, "long carry")
+
+
 def test_backward_without_state_or_final_gradients():
     wl = inputs.WORKLOADS["tiny_f32"].scaled(batch=2, seq_len=40, heads=2, head_dim=32)
     grads, ref = _run(wl, seed=3, with_state=False, with_final=False, biases=False)
