@@ -341,32 +341,47 @@ __global__ void __launch_bounds__(128) bwd_convT_kernel(ConvTArgs a) {
     const int sb = tb == 0 ? -kHist : t0;                   // the first block also owns the history
     float d0 = dxcv(sb), d1 = dxcv(sb + 1), d2 = dxcv(sb + 2);
     bool q0 = rs(sb), q1 = rs(sb + 1), q2 = rs(sb + 2);
-    for (int s = sb; s < t1; ++s) {
-        const float d3 = dxcv(s + 3);
-        const bool q3 = rs(s + 3);
-        if (s >= t0) {                                      // token t = s: its four taps
-            const float xs = bf(a.x + rowe + (size_t)s * a.W);
-            if (q0) L = s;
-            s_cb += d0;
-            if (s - 3 >= L) s_cw[0] = fmaf(d0, xa, s_cw[0]);
-            if (s - 2 >= L) s_cw[1] = fmaf(d0, xb, s_cw[1]);
-            if (s - 1 >= L) s_cw[2] = fmaf(d0, xcc, s_cw[2]);
-            s_cw[3] = fmaf(d0, xs, s_cw[3]);
-            xa = xb; xb = xcc; xcc = xs;
+    // positions in batches of kPF: the batch's loads are issued together, ahead of its arithmetic
+    for (int s0 = sb; s0 < t1; s0 += kPF) {
+        float dn[kPF], xn[kPF];
+        bool qn[kPF];
+#pragma unroll
+        for (int j = 0; j < kPF; ++j) {
+            const int s = s0 + j;
+            dn[j] = dxcv(s + 3);
+            qn[j] = rs(s + 3);
+            xn[j] = s >= t0 && s < t1 ? bf(a.x + rowe + (size_t)s * a.W) : 0.f;
         }
-        // dx_s: tap k of token s + 3 - k, while no segment starts in (s, s + 3 - k]
-        const bool ok1 = !q1, ok2 = ok1 && !q2, ok3 = ok2 && !q3;
-        float acc = 0.f;
-        if (ok3 && s + 3 >= 0 && s + 3 < a.T) acc = fmaf(cw[0], d3, acc);
-        if (ok2 && s + 2 >= 0 && s + 2 < a.T) acc = fmaf(cw[1], d2, acc);
-        if (ok1 && s + 1 >= 0 && s + 1 < a.T) acc = fmaf(cw[2], d1, acc);
-        if (s >= 0) acc = fmaf(cw[3], d0, acc);
-        if (a.dtail_final && s >= a.T - kHist && window_reads(rrow, s, a.T - 1))
-            acc += a.dtail_final[((size_t)b * kHist + (s - (a.T - kHist))) * a.W + ch];
-        if (s >= 0) a.dx[rowe + (size_t)s * a.W] = acc;
-        else if (a.dtail0) a.dtail0[((size_t)b * kHist + (kHist + s)) * a.W + ch] = acc;
-        d0 = d1; d1 = d2; d2 = d3;
-        q0 = q1; q1 = q2; q2 = q3;
+#pragma unroll
+        for (int j = 0; j < kPF; ++j) {
+            const int s = s0 + j;
+            if (s >= t1) break;
+            const float d3 = dn[j];
+            const bool q3 = qn[j];
+            if (s >= t0) {                                  // token t = s: its four taps
+                const float xs = xn[j];
+                if (q0) L = s;
+                s_cb += d0;
+                if (s - 3 >= L) s_cw[0] = fmaf(d0, xa, s_cw[0]);
+                if (s - 2 >= L) s_cw[1] = fmaf(d0, xb, s_cw[1]);
+                if (s - 1 >= L) s_cw[2] = fmaf(d0, xcc, s_cw[2]);
+                s_cw[3] = fmaf(d0, xs, s_cw[3]);
+                xa = xb; xb = xcc; xcc = xs;
+            }
+            // dx_s: tap k of token s + 3 - k, while no segment starts in (s, s + 3 - k]
+            const bool ok1 = !q1, ok2 = ok1 && !q2, ok3 = ok2 && !q3;
+            float acc = 0.f;
+            if (ok3 && s + 3 >= 0 && s + 3 < a.T) acc = fmaf(cw[0], d3, acc);
+            if (ok2 && s + 2 >= 0 && s + 2 < a.T) acc = fmaf(cw[1], d2, acc);
+            if (ok1 && s + 1 >= 0 && s + 1 < a.T) acc = fmaf(cw[2], d1, acc);
+            if (s >= 0) acc = fmaf(cw[3], d0, acc);
+            if (a.dtail_final && s >= a.T - kHist && window_reads(rrow, s, a.T - 1))
+                acc += a.dtail_final[((size_t)b * kHist + (s - (a.T - kHist))) * a.W + ch];
+            if (s >= 0) a.dx[rowe + (size_t)s * a.W] = acc;
+            else if (a.dtail0) a.dtail0[((size_t)b * kHist + (kHist + s)) * a.W + ch] = acc;
+            d0 = d1; d1 = d2; d2 = d3;
+            q0 = q1; q1 = q2; q2 = q3;
+        }
     }
     const size_t pb = (size_t)a.B * a.ntb * a.W, pi = ((size_t)b * a.ntb + tb) * a.W + ch;
 #pragma unroll

@@ -68,11 +68,17 @@ constexpr uint32_t OFF_A = 0;                        // conv output, bf16 hi par
 constexpr uint32_t OFF_ALO = OFF_A + A_BYTES;        // and lo part (xc - hi)
 constexpr uint32_t OFF_BA = OFF_ALO + A_BYTES;
 constexpr uint32_t OFF_BX = OFF_BA + B_BYTES;        // right after W_a: one N = 128 operand
+// Before the weights arrive, their 64 KB hold the conv's inputs, staged by TMA in the 128-byte
+// swizzle: x [128 rows][64 channels] bf16 and the history [128 rows][3][64 channels] bf16.
+constexpr uint32_t X_ST_BYTES = MT * NT * 2;          // 16384
+constexpr uint32_t OFF_XST = OFF_BA;
+constexpr uint32_t OFF_TST = OFF_BA + X_ST_BYTES;     // 49152 bytes of history
+static_assert(X_ST_BYTES * (1 + kHist) == 2 * B_BYTES, "staging fills the weight tile");
 constexpr uint32_t OFF_Y = OFF_BX + B_BYTES;
 constexpr uint32_t OFF_CONST = OFF_Y + Y_BYTES;      // K, -b_a log2 e, -b_x log2 e per channel: 3 x 64 fp32
 constexpr uint32_t OFF_CONV = OFF_CONST + 3 * NT * 4; // conv taps [4][64] and bias [64], fp32
 constexpr uint32_t OFF_BAR = OFF_CONV + 5 * NT * 4;
-constexpr uint32_t OFF_MISC = OFF_BAR + 64;
+constexpr uint32_t OFF_MISC = OFF_BAR + 72;
 constexpr int kClusterSize = DH / NT;                 // CTAs of a (head, row tile)
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 32 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -143,15 +149,21 @@ __device__ bool wait_bounded(uint32_t bar, uint32_t parity, const Args& a, volat
     }
 }
 
+// 16-byte chunk c of line l of a tile in the 128-byte swizzle
+__device__ __forceinline__ uint32_t sw128(uint32_t l, uint32_t c) { return l * 128 + ((c ^ (l & 7)) << 4); }
+
 __global__ void __launch_bounds__(kThreads, 1)
 decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_constant__ CUtensorMap map_wx,
                     const __grid_constant__ CUtensorMap map_y, const __grid_constant__ CUtensorMap map_out,
-                    const Args a) {
+                    const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_tail,
+                    const __grid_constant__ CUtensorMap map_h, const Args a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_w = sbase + OFF_BAR, bar_acc = sbase + OFF_BAR + 16;
     const uint32_t bar_y = sbase + OFF_BAR + 24;      // y tile
+    const uint32_t bar_x = sbase + OFF_BAR + 8;       // the conv's staged inputs
+    const uint32_t bar_st = sbase + OFF_BAR + 64;     // the staging has been read: the weights may come
     // K block j of the operand tile: convolved here (j = rank) or copied in by CTA j
     auto bar_k = [&](int j) { return sbase + OFF_BAR + 32 + 8 * (uint32_t)j; };
     volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
@@ -174,6 +186,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         mbar_init(bar_w, 1);
+        mbar_init(bar_x, 1);
+        mbar_init(bar_st, 1);
         mbar_init(bar_acc, 1);
         mbar_init(bar_y, 1);
         for (int j = 0; j < kClusterSize; ++j) mbar_init(bar_k(j), 1);
@@ -191,6 +205,9 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
         prefetch_tensormap(&map_wx);
         prefetch_tensormap(&map_y);
         prefetch_tensormap(&map_out);
+        prefetch_tensormap(&map_x);
+        prefetch_tensormap(&map_tail);
+        prefetch_tensormap(&map_h);
     }
     tc_fence_before();
     __syncthreads();
@@ -203,18 +220,30 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
 
     if (warp == kWarpTma) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(bar_w, 2 * B_BYTES);
-            for (int kb = 0; kb < DH / 64; ++kb) {
-                tma_load_2d(sbase + OFF_BA + kb * 8192, &map_wa, nt * NT, head * DH + kb * 64, bar_w);
-                tma_load_2d(sbase + OFF_BX + kb * 8192, &map_wx, nt * NT, head * DH + kb * 64, bar_w);
-            }
-            // this tile's y (rows past the batch read as zeros)
+            // the conv's inputs of this tile (rows past the batch read as zeros), then its y
+            mbar_arrive_expect_tx(bar_x, (1 + kHist) * X_ST_BYTES);
+            tma_load_2d(sbase + OFF_XST, &map_x, ch0, mt * MT, bar_x);
+            tma_load_3d(sbase + OFF_TST, &map_tail, ch0, 0, mt * MT, bar_x);
             mbar_arrive_expect_tx(bar_y, Y_BYTES);
             tma_load_2d(sbase + OFF_Y, &map_y, ch0, mt * MT, bar_y);
-            // never leave the CTA with a bulk copy still writing its shared memory (the weight
-            // tiles, or a sibling's conv block, whose completion also ends the sibling's reads)
+            // the weights, into the staging area once the conv has read it
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait_sleep(bar_w, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
+            bool staged = false;
+            while (!(staged = mbar_try_wait_sleep(bar_st, 0, 20000u)) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+            if (staged) {
+                mbar_arrive_expect_tx(bar_w, 2 * B_BYTES);
+                for (int kb = 0; kb < DH / 64; ++kb) {
+                    tma_load_2d(sbase + OFF_BA + kb * 8192, &map_wa, nt * NT, head * DH + kb * 64, bar_w);
+                    tma_load_2d(sbase + OFF_BX + kb * 8192, &map_wx, nt * NT, head * DH + kb * 64, bar_w);
+                }
+            }
+            // never leave the CTA with a bulk copy still writing its shared memory (the staged
+            // inputs, the weight tiles, or a sibling's conv block, whose completion also ends the
+            // sibling's reads)
+            while (!mbar_try_wait_sleep(bar_x, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+            while (staged && !mbar_try_wait_sleep(bar_w, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
             }
             for (int j = 0; j < kClusterSize; ++j)
                 while (!mbar_try_wait_sleep(bar_k(j), 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
@@ -250,6 +279,14 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
         }
         if (elect_one()) mma_commit(bar_acc);     // also when a wait failed: the update must not wait forever
         __syncwarp();
+        // every MMA issued here has completed before TMEM can be released (bounded by time only,
+        // so that an aborted step still drains its tensor-core work)
+        if (lane == 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait_sleep(bar_acc, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+        }
+        __syncwarp();
     } else {
         // ================================ update threads =======================================
         // thread = row r of the tile (= TMEM lane r), channels [16 cg, 16 cg + 16) of its 64: it
@@ -264,46 +301,51 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
         const uint32_t xcol = tmem + lane_off + TM_XC + cg * kEpiCh;
         if (threadIdx.x < NT) {                           // per-channel constants
+            // every load first: a shared-memory store between two of them would order them
             const int ch = ch0 + threadIdx.x;
             const float lam = a.lambda[ch];
             const float ba = a.b_a ? a.b_a[ch] : 0.f;
             const float bx = a.b_x ? a.b_x[ch] : 0.f;
             const float cb0 = a.conv_b ? a.conv_b[ch] : 0.f;
+            float cwv[kConvWidth];
 #pragma unroll
-            for (int k = 0; k < kConvWidth; ++k) s_cw[k * NT + threadIdx.x] = a.conv_w[(size_t)k * W + ch];
+            for (int k = 0; k < kConvWidth; ++k) cwv[k] = a.conv_w[(size_t)k * W + ch];
+#pragma unroll
+            for (int k = 0; k < kConvWidth; ++k) s_cw[k * NT + threadIdx.x] = cwv[k];
             s_cb[threadIdx.x] = cb0;
             s_K[threadIdx.x] = a.c * log_sigmoid_acc(lam);
             s_nba[threadIdx.x] = -ba * kLog2e;
             s_nbx[threadIdx.x] = -bx * kLog2e;
         }
-        // the conv's inputs (x and the three past inputs) and the state, issued together
+        const bool rst = live && a.reset && a.reset[b];
+        // the conv's inputs from the staged tiles: x and the three past inputs of this thread's
+        // row and 16 channels (16-byte chunks 2 cg, 2 cg + 1 of their 128-byte lines)
+        const bool ok_x = wait_bounded(bar_x, 0, a, abort, 6);
         uint4 xv[2], t0[2], t1[2], t2[2];
-        const __nv_bfloat16* tl = a.tail + (size_t)bs * kHist * W + cbase;
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
-            xv[v] = *reinterpret_cast<const uint4*>(a.x + (size_t)bs * W + cbase + 8 * v);
-            t0[v] = *reinterpret_cast<const uint4*>(tl + 8 * v);
-            t1[v] = *reinterpret_cast<const uint4*>(tl + W + 8 * v);
-            t2[v] = *reinterpret_cast<const uint4*>(tl + 2 * W + 8 * v);
+            const uint32_t c = (uint32_t)(2 * cg + v);
+            xv[v] = *reinterpret_cast<const uint4*>(smem + OFF_XST + sw128((uint32_t)r, c));
+            t0[v] = *reinterpret_cast<const uint4*>(smem + OFF_TST + sw128((uint32_t)(r * kHist + 0), c));
+            t1[v] = *reinterpret_cast<const uint4*>(smem + OFF_TST + sw128((uint32_t)(r * kHist + 1), c));
+            t2[v] = *reinterpret_cast<const uint4*>(smem + OFF_TST + sw128((uint32_t)(r * kHist + 2), c));
         }
-        float hv[kEpiCh];
-        {
-            const float4* hp = reinterpret_cast<const float4*>(a.h + (size_t)bs * W + cbase);
-#pragma unroll
-            for (int i = 0; i < kEpiCh / 4; ++i) {
-                const float4 v = hp[i];
-                hv[4 * i] = v.x; hv[4 * i + 1] = v.y; hv[4 * i + 2] = v.z; hv[4 * i + 3] = v.w;
-            }
-        }
-        const bool rst = live && a.reset && a.reset[b];
         asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+        if (rst) {                                        // an empty history
+#pragma unroll
+            for (int v = 0; v < 2; ++v) t0[v] = t1[v] = t2[v] = make_uint4(0, 0, 0, 0);
+        }
+        // the new history (oldest out, x in) over the staged one, stored by TMA after the conv
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+            const uint32_t c = (uint32_t)(2 * cg + v);
+            *reinterpret_cast<uint4*>(smem + OFF_TST + sw128((uint32_t)(r * kHist + 0), c)) = t1[v];
+            *reinterpret_cast<uint4*>(smem + OFF_TST + sw128((uint32_t)(r * kHist + 1), c)) = t2[v];
+            *reinterpret_cast<uint4*>(smem + OFF_TST + sw128((uint32_t)(r * kHist + 2), c)) = xv[v];
+        }
 
         // ================================ conv of this CTA's channels ==========================
         {
-            if (rst) {                                    // an empty history
-#pragma unroll
-                for (int v = 0; v < 2; ++v) t0[v] = t1[v] = t2[v] = make_uint4(0, 0, 0, 0);
-            }
             const float* cwp = s_cw + cg * kEpiCh;
             const float* cbp = s_cb + cg * kEpiCh;
 #pragma unroll
@@ -354,20 +396,28 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
                         dsmem_copy(map_to_rank(blk, peer), blk, A_KBLK, map_to_rank(bar_k(nt), peer));
                     }
                 }
-            }
-            // history: oldest out, x in (after the hand-off, so that no fence waits for these)
-            if (live) {
-                __nv_bfloat16* tw = a.tail + (size_t)b * kHist * W + cbase;
-#pragma unroll
-                for (int v = 0; v < 2; ++v) {
-                    *reinterpret_cast<uint4*>(tw + 8 * v) = t1[v];
-                    *reinterpret_cast<uint4*>(tw + W + 8 * v) = t2[v];
-                    *reinterpret_cast<uint4*>(tw + 2 * W + 8 * v) = xv[v];
+                // the new history of the tile's rows (rows past the batch are clipped); once the
+                // store has read the staging area, the weights may take its place
+                if (ok_x && !*abort) {
+                    tma_store_3d(&map_tail, sbase + OFF_TST, ch0, 0, mt * MT);
+                    bulk_commit();
+                    bulk_wait_read0();
                 }
+                mbar_arrive(bar_st);
             }
         }
 
         // ================================ update ===============================================
+        // the state of this thread's row and channels (its latency overlaps the exchange)
+        float hv[kEpiCh];
+        {
+            const float4* hp = reinterpret_cast<const float4*>(a.h + (size_t)bs * W + cbase);
+#pragma unroll
+            for (int i = 0; i < kEpiCh / 4; ++i) {
+                const float4 v = hp[i];
+                hv[4 * i] = v.x; hv[4 * i + 1] = v.y; hv[4 * i + 2] = v.z; hv[4 * i + 3] = v.w;
+            }
+        }
         // GeLU(y) while the siblings' blocks arrive and the tensor cores run
         const bool ok_y = __all_sync(0xffffffffu, wait_bounded(bar_y, 0, a, abort, 4));
         float gg[kEpiCh];
@@ -385,7 +435,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
             for (int i = 0; i < kEpiCh; ++i) hv[i] = 0.f;
         }
         // uniform across the warp: the TMEM loads below are warp-collective
-        const bool ok = __all_sync(0xffffffffu, ok_y && wait_bounded(bar_acc, 0, a, abort, 2));
+        const bool acc_ok = wait_bounded(bar_acc, 0, a, abort, 2);
+        const bool ok = __all_sync(0xffffffffu, ok_x && ok_y && acc_ok);
         tc_fence_after();
         const uint32_t taddr = tmem + lane_off + cg * kEpiCh;
 #pragma unroll
@@ -401,35 +452,39 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
             uint32_t ow[4];
 #pragma unroll
             for (int e2 = 0; e2 < 4; ++e2) {
-                float o[2];
-#pragma unroll
-                for (int e1 = 0; e1 < 2; ++e1) {
-                    const int e = 2 * e2 + e1;
-                    const int jc = c8 * 8 + e;            // column within the tile
-                    float at, u;
-                    gates1<false>(ga[e], gx[e], s_nba[jc], s_nbx[jc], s_K[jc], xc[e], at, u);
-                    const float hn = fmaf(at, hv[v * 8 + e], u);
-                    hv[v * 8 + e] = hn;
-                    o[e1] = hn * gg[v * 8 + e];
-                }
-                ow[e2] = pack_bf16x2(o[0], o[1]);
+                const int e = 2 * e2;
+                const int jc = c8 * 8 + e;                // column within the tile (even)
+                float2 at, u;
+                gates2<false>(make_float2(ga[e], ga[e + 1]), make_float2(gx[e], gx[e + 1]),
+                              *reinterpret_cast<const float2*>(s_nba + jc), *reinterpret_cast<const float2*>(s_nbx + jc),
+                              *reinterpret_cast<const float2*>(s_K + jc), make_float2(xc[e], xc[e + 1]), at, u);
+                const float2 hn = fma2(at, make_float2(hv[v * 8 + e], hv[v * 8 + e + 1]), u);
+                hv[v * 8 + e] = hn.x;
+                hv[v * 8 + e + 1] = hn.y;
+                const float2 o = mul2(hn, make_float2(gg[v * 8 + e], gg[v * 8 + e + 1]));
+                ow[e2] = pack_bf16x2(o.x, o.y);
             }
             *reinterpret_cast<uint4*>(smem + yo) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         }
-        // the state, straight from registers (only rows of the batch)
-        if (ok && live) {
-            float4* hp = reinterpret_cast<float4*>(a.h + (size_t)b * W + cbase);
+        // the state into the operand tile's space (the MMAs that read it are done): two boxes
+        // of [128 rows x 32 channels] fp32 in the 128-byte swizzle, box cg / 2, chunks
+        // 4 (cg % 2) .. 4 (cg % 2) + 3 of the row's line
 #pragma unroll
-            for (int i = 0; i < kEpiCh / 4; ++i)
-                hp[i] = make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
-        }
-        // the out tile is complete: store it (rows past the batch are clipped by the map)
+        for (int i = 0; i < kEpiCh / 4; ++i)
+            *reinterpret_cast<float4*>(smem + OFF_A + (uint32_t)(cg >> 1) * (MT * 128) +
+                                       sw128((uint32_t)r, (uint32_t)(4 * (cg & 1) + i))) =
+                make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+        // the out and state tiles are complete: store them (rows past the batch are clipped)
         fence_proxy_async_smem();
         asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-        if (threadIdx.x == 0 && !*abort) {
-            tma_store_2d(&map_out, sbase + OFF_Y, ch0, mt * MT);
-            bulk_commit();
-            bulk_wait_read0();                            // the shared tile stays until read
+        if (threadIdx.x == 0) {
+            if (!*abort) {                                // (every failed wait has set it)
+                tma_store_2d(&map_out, sbase + OFF_Y, ch0, mt * MT);
+                tma_store_2d(&map_h, sbase + OFF_A, ch0, mt * MT);
+                tma_store_2d(&map_h, sbase + OFF_A + MT * 128, ch0 + NT / 2, mt * MT);
+                bulk_commit();
+            }
+            bulk_wait0();                                 // every store of this CTA has completed
         }
     }
     tc_fence_before();
@@ -465,8 +520,11 @@ cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, cons
     if (fused_decode_workspace(d) > ws_bytes) return cudaErrorInvalidValue;
     const int B = d->batch, H = d->heads;
     const uint64_t W = (uint64_t)H * DH;
-    CUtensorMap mwa, mwx, my, mo;
-    if (!tc::make_map_2d_sw128(&mwa, p->w_a, DH, W, DH * 2, NT, 64) ||
+    CUtensorMap mwa, mwx, my, mo, mx, mt, mh;
+    if (!tc::make_map_2d_sw128(&mx, x, W, (uint64_t)B, W * 2, NT, MT) ||
+        !tc::make_map_2d_sw128_elem(&mh, st->h, 4, W, (uint64_t)B, W * 4, NT / 2, MT) ||
+        !tc::make_map_3d_box_sw128(&mt, st->conv_tail, W, kHist, (uint64_t)B, NT, kHist, MT) ||
+        !tc::make_map_2d_sw128(&mwa, p->w_a, DH, W, DH * 2, NT, 64) ||
         !tc::make_map_2d_sw128(&mwx, p->w_x, DH, W, DH * 2, NT, 64) ||
         !tc::make_map_2d_sw128_elem(&my, y, 2, W, (uint64_t)B, W * 2, NT, MT) ||
         !tc::make_map_2d_sw128_elem(&mo, out, 2, W, (uint64_t)B, W * 2, NT, MT))
@@ -499,7 +557,7 @@ cudaError_t launch_fused_decode(const rglru_dims* d, const rglru_params* p, cons
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, mwa, mwx, my, mo, a);
+    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, mwa, mwx, my, mo, mx, mt, mh, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

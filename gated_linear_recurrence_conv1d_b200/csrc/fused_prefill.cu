@@ -358,11 +358,12 @@ __device__ __forceinline__ void pass1(uint32_t dcol, const float* xcs, const Cha
     aggH = Hc;
 }
 
-// Save-mode first pass: the same with accurate fp32 math (CUDA's expf / sqrtf), writing the
-// complete gate pre-activations (with their biases) and the conv output (as a bf16 hi + lo pair)
-// of every token of the chunk to the save arrays (e0: element of token 0).
-__device__ __forceinline__ void pass1_save(uint32_t dcol, const float* xcs, float kappa, float ba, float bx, uint32_t rm,
-                                           int nt, const Args& a, size_t e0, int W, float& aggA, float& aggH) {
+// Save-mode first pass: the same arithmetic (any decay range), also writing the complete gate
+// pre-activations (with their biases) and the conv output (as a bf16 hi + lo pair) of every token
+// of the chunk to the save arrays (e0: element of token 0).
+__device__ __forceinline__ void pass1_save(uint32_t dcol, const float* xcs, const ChanK& ck, float ba, float bx,
+                                           uint32_t rm, int nt, const Args& a, size_t e0, int W, float& aggA,
+                                           float& aggH) {
     float A = 1.0f, Hc = 0.0f;
 #pragma unroll 1
     for (int t0 = 0; t0 < L; t0 += kBT) {
@@ -374,29 +375,30 @@ __device__ __forceinline__ void pass1_save(uint32_t dcol, const float* xcs, floa
         tmem_wait_ld();
         float av[kBT], uv[kBT];
 #pragma unroll
+        for (int i = 0; i < kBT; i += 2) {
+            float2 a2, u2;
+            gates2<false>(make_float2(da[i], da[i + 1]), make_float2(dx[i], dx[i + 1]), ck.nba, ck.nbx, ck.K,
+                          make_float2(xc[i], xc[i + 1]), a2, u2);
+            av[i] = a2.x; av[i + 1] = a2.y;
+            uv[i] = u2.x; uv[i + 1] = u2.y;
+        }
+#pragma unroll
         for (int i = 0; i < kBT; ++i) {
             const int t = t0 + i;
-            const float ga = da[i] + ba, gx = dx[i] + bx;
-            const float r = sigmoid_acc(ga), ig = sigmoid_acc(gx);
-            float at, beta;
-            decay_and_beta_acc(kappa, r, &at, &beta);
-            float u = beta * (ig * xc[i]);
-            if ((rm >> t) & 1u) at = 0.f;                     // h_{t-1} := 0 at a segment start
+            if ((rm >> t) & 1u) av[i] = 0.f;                  // h_{t-1} := 0 at a segment start
             if (t < nt) {
                 const size_t e = e0 + (size_t)t * W;
-                a.sv_ga[e] = ga;
-                a.sv_gx[e] = gx;
+                a.sv_ga[e] = da[i] + ba;
+                a.sv_gx[e] = dx[i] + bx;
                 const __nv_bfloat16 hi = __float2bfloat16_rn(xc[i]);
                 a.sv_xc_hi[e] = hi;
                 a.sv_xc_lo[e] = __float2bfloat16_rn(xc[i] - __bfloat162float(hi));
             } else {                                          // past the end: identity
-                at = 1.f;
-                u = 0.f;
+                av[i] = 1.f;
+                uv[i] = 0.f;
             }
-            av[i] = at;
-            uv[i] = u;
-            Hc = fmaf(at, Hc, u);
-            A *= at;
+            Hc = fmaf(av[i], Hc, uv[i]);
+            A *= av[i];
         }
         tmem_st8f(dcol + t0, av);
         tmem_st8f(dcol + L + t0, uv);
@@ -793,7 +795,7 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             float aggA, aggH;
             const size_t e0 = ((size_t)b * a.T + t0) * W + ch;
             if constexpr (SAVE) {
-                pass1_save(dcol, xcs, kappa, ba, bx, rmask, nt, a, e0, W, aggA, aggH);
+                pass1_save(dcol, xcs, ck, ba, bx, rmask, nt, a, e0, W, aggA, aggH);
             } else if (nt == L && warp_small) {
                 if (rmask) pass1<true, false>(dcol, xcs, ck, rmask, nt, aggA, aggH);
                 else pass1<false, false>(dcol, xcs, ck, rmask, nt, aggA, aggH);
