@@ -103,8 +103,8 @@ __device__ __forceinline__ float gelu_grad(float v, int tanh_form) {
 //   a = 1 + E, E = expm1(c r log sigma(Lambda)) by its series to l^5 for l >= -1/8 (no
 //   cancellation as a -> 1, where the reverse recurrence carries errors of a over ~1 / (1 - a)
 //   tokens), else 2^(l log2 e) - 1; beta = sqrt(1 - a^2) = sqrt(-E (2 + E));
-//   GeLU and its derivative from one erfc: Phi(v) = erfc(-v / sqrt 2) / 2, GeLU = v Phi,
-//   GeLU' = Phi + v phi(v) (the tanh form keeps tanhf).
+//   GeLU = v Phi and GeLU' = Phi + v phi(v) from one exp2 and a polynomial (below; the tanh
+//   form keeps tanhf).
 __device__ __forceinline__ float sig_fast(float z) { return fm::rcpf(1.0f + fm::ex2f(-z * fm::kLog2e)); }
 
 __device__ __forceinline__ void decay_beta_fast(float kappa, float r, float& at, float& beta) {
@@ -113,15 +113,53 @@ __device__ __forceinline__ void decay_beta_fast(float kappa, float r, float& at,
     beta = sqrtf(-E * (2.0f + E));
 }
 
+// Phi(v) to ~1e-7 without erfc: with s = |v| and e = exp(-v^2 / 2) (one exp2), the upper tail
+// Q(s) = e R(s), R a degree-14 polynomial in t = (s - 2.75) / 2.75 on s in [0, 5.5] (s clamped
+// there; beyond it Q < 2e-8), fitted by gelu_tail_fit.py --precise beside this file (max |Phi
+// error| 1.1e-7 in fp32); Phi(v) = 1 - Q for v >= 0, Q otherwise.
+constexpr float kPhiR0 = 1.307247281e-01f;
+constexpr float kPhiR1 = -1.084856018e-01f;
+constexpr float kPhiR2 = 8.409250528e-02f;
+constexpr float kPhiR3 = -6.148617715e-02f;
+constexpr float kPhiR4 = 4.272365198e-02f;
+constexpr float kPhiR5 = -2.843398601e-02f;
+constexpr float kPhiR6 = 1.814154349e-02f;
+constexpr float kPhiR7 = -1.083536446e-02f;
+constexpr float kPhiR8 = 6.395316683e-03f;
+constexpr float kPhiR9 = -4.469349980e-03f;
+constexpr float kPhiR10 = 2.545840805e-03f;
+constexpr float kPhiR11 = -3.012927773e-04f;
+constexpr float kPhiR12 = 1.266671024e-04f;
+constexpr float kPhiR13 = -8.168322383e-04f;
+constexpr float kPhiR14 = 4.210809420e-04f;
+
 __device__ __forceinline__ void gelu_and_grad(float v, int tanh_form, float& g, float& gp) {
     if (tanh_form) {
         g = gelu_acc(v, 1);
         gp = gelu_grad(v, 1);
         return;
     }
-    const float phi_c = 0.5f * erfcf(-v * 0.70710678118654752440f);
+    const float e = fm::ex2f((v * v) * (-0.5f * fm::kLog2e));
+    const float t = fmaf(fminf(fabsf(v), 5.5f), 1.0f / 2.75f, -1.0f);
+    float r = kPhiR14;
+    r = fmaf(r, t, kPhiR13);
+    r = fmaf(r, t, kPhiR12);
+    r = fmaf(r, t, kPhiR11);
+    r = fmaf(r, t, kPhiR10);
+    r = fmaf(r, t, kPhiR9);
+    r = fmaf(r, t, kPhiR8);
+    r = fmaf(r, t, kPhiR7);
+    r = fmaf(r, t, kPhiR6);
+    r = fmaf(r, t, kPhiR5);
+    r = fmaf(r, t, kPhiR4);
+    r = fmaf(r, t, kPhiR3);
+    r = fmaf(r, t, kPhiR2);
+    r = fmaf(r, t, kPhiR1);
+    r = fmaf(r, t, kPhiR0);
+    const float q = e * r;
+    const float phi_c = v >= 0.f ? 1.0f - q : q;
     g = v * phi_c;
-    gp = fmaf(v * fm::ex2f((v * v) * (-0.5f * fm::kLog2e)), 0.39894228040143267794f, phi_c);
+    gp = fmaf(v * e, 0.39894228040143267794f, phi_c);
 }
 
 __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bfloat16* lo) {
@@ -312,81 +350,99 @@ __device__ __forceinline__ bool window_reads(const uint8_t* rrow, int s, int t) 
     return true;
 }
 
-// Thread = (row b, block of kTB positions, channel ch); one walk over the block's positions s
-// with the last three x and the next three dxc in registers: the parameter gradients of token
-// t = s (the taps that read x_{s-3..s}) and dx_s (the taps of the tokens s..s+3 that read x_s).
-// A window reads position s for token t when no segment starts in (s, t]: L below is the last
-// segment start at or before the current token.
+// Thread = (row b, block of kTB positions, channel pair ch, ch + 1); one walk over the block's
+// positions s with the last three x and the next three dxc in registers: the parameter gradients
+// of token t = s (the taps that read x_{s-3..s}) and dx_s (the taps of the tokens s..s+3 that
+// read x_s).  A window reads position s for token t when no segment starts in (s, t]: L below is
+// the last segment start at or before the current token.  Every value is a channel pair.
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
 __global__ void __launch_bounds__(128) bwd_convT_kernel(ConvTArgs a) {
-    const int ch = blockIdx.x * 128 + threadIdx.x, tb = blockIdx.y, b = blockIdx.z;
+    const int ch = 2 * (blockIdx.x * 128 + threadIdx.x), tb = blockIdx.y, b = blockIdx.z;
     if (ch >= a.W) return;
-    const int t0 = tb * kTB, t1 = min(a.T, t0 + kTB);
-    const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
-    const size_t rowe = (size_t)b * a.T * a.W + ch;        // element (b, 0, ch)
-    float cw[kConvWidth];
+    const int T = a.T;
+    const int t0 = tb * kTB, t1 = min(T, t0 + kTB);
+    const long long W = a.W;
+    const uint8_t* rrow = a.reset ? a.reset + (size_t)b * T : nullptr;
+    const size_t rowe = (size_t)b * T * W + ch;             // element (b, 0, ch)
+    const __nv_bfloat162* xr = reinterpret_cast<const __nv_bfloat162*>(a.x + rowe);
+    const float2* dr = reinterpret_cast<const float2*>(a.dxc + rowe);
+    float* dxr = a.dx + rowe;                               // caller's buffer: 4-byte aligned only
+    const long long W2 = W / 2;                             // row pitch in channel pairs
+    float2 cw[kConvWidth];
 #pragma unroll
-    for (int k = 0; k < kConvWidth; ++k) cw[k] = a.conv_w[(size_t)k * a.W + ch];
-    auto xval = [&](int s) -> float {                       // x_s, the initial history for s < 0
-        if (s >= 0) return bf(a.x + rowe + (size_t)s * a.W);
-        return a.tail0 ? bf(a.tail0 + ((size_t)b * kHist + (kHist + s)) * a.W + ch) : 0.f;
+    for (int k = 0; k < kConvWidth; ++k) cw[k] = make_float2(a.conv_w[(size_t)k * W + ch], a.conv_w[(size_t)k * W + ch + 1]);
+    auto xval = [&](int s) -> float2 {                      // x_s, the initial history for s < 0
+        if (s >= 0) return __bfloat1622float2(xr[s * W2]);
+        if (!a.tail0) return make_float2(0.f, 0.f);
+        return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(a.tail0 + ((size_t)b * kHist + (kHist + s)) * W + ch));
     };
-    auto dxcv = [&](int t) -> float { return t >= 0 && t < a.T ? a.dxc[rowe + (size_t)t * a.W] : 0.f; };
-    auto rs = [&](int p) -> bool { return rrow && p >= 0 && p < a.T && rrow[p] != 0; };
+    auto dxcv = [&](int t) -> float2 { return t >= 0 && t < T ? dr[t * W2] : make_float2(0.f, 0.f); };
+    auto rs = [&](int p) -> bool { return rrow && p >= 0 && p < T && rrow[p] != 0; };
 
     int L = -kHist - 1;                                     // no segment start within reach
     for (int p = max(0, t0 - kHist); p < t0; ++p)
         if (rs(p)) L = p;
-    float xa = xval(t0 - 3), xb = xval(t0 - 2), xcc = xval(t0 - 1);   // x_{t-3}, x_{t-2}, x_{t-1}
-    float s_cw[kConvWidth] = {0.f, 0.f, 0.f, 0.f}, s_cb = 0.f;
+    float2 xa = xval(t0 - 3), xb = xval(t0 - 2), xcc = xval(t0 - 1);   // x_{t-3}, x_{t-2}, x_{t-1}
+    const float2 z2 = make_float2(0.f, 0.f);
+    float2 s_cw[kConvWidth] = {z2, z2, z2, z2}, s_cb = z2;
     const int sb = tb == 0 ? -kHist : t0;                   // the first block also owns the history
-    float d0 = dxcv(sb), d1 = dxcv(sb + 1), d2 = dxcv(sb + 2);
+    float2 d0 = dxcv(sb), d1 = dxcv(sb + 1), d2 = dxcv(sb + 2);
     bool q0 = rs(sb), q1 = rs(sb + 1), q2 = rs(sb + 2);
     // positions in batches of kPF: the batch's loads are issued together, ahead of its arithmetic
     for (int s0 = sb; s0 < t1; s0 += kPF) {
-        float dn[kPF], xn[kPF];
+        float2 dn[kPF], xn[kPF];
         bool qn[kPF];
 #pragma unroll
         for (int j = 0; j < kPF; ++j) {
             const int s = s0 + j;
             dn[j] = dxcv(s + 3);
             qn[j] = rs(s + 3);
-            xn[j] = s >= t0 && s < t1 ? bf(a.x + rowe + (size_t)s * a.W) : 0.f;
+            xn[j] = s >= t0 && s < t1 ? __bfloat1622float2(xr[s * W2]) : z2;
         }
 #pragma unroll
         for (int j = 0; j < kPF; ++j) {
             const int s = s0 + j;
             if (s >= t1) break;
-            const float d3 = dn[j];
+            const float2 d3 = dn[j];
             const bool q3 = qn[j];
             if (s >= t0) {                                  // token t = s: its four taps
-                const float xs = xn[j];
+                const float2 xs = xn[j];
                 if (q0) L = s;
-                s_cb += d0;
-                if (s - 3 >= L) s_cw[0] = fmaf(d0, xa, s_cw[0]);
-                if (s - 2 >= L) s_cw[1] = fmaf(d0, xb, s_cw[1]);
-                if (s - 1 >= L) s_cw[2] = fmaf(d0, xcc, s_cw[2]);
-                s_cw[3] = fmaf(d0, xs, s_cw[3]);
+                s_cb = make_float2(s_cb.x + d0.x, s_cb.y + d0.y);
+                if (s - 3 >= L) s_cw[0] = f2fma(d0, xa, s_cw[0]);
+                if (s - 2 >= L) s_cw[1] = f2fma(d0, xb, s_cw[1]);
+                if (s - 1 >= L) s_cw[2] = f2fma(d0, xcc, s_cw[2]);
+                s_cw[3] = f2fma(d0, xs, s_cw[3]);
                 xa = xb; xb = xcc; xcc = xs;
             }
             // dx_s: tap k of token s + 3 - k, while no segment starts in (s, s + 3 - k]
             const bool ok1 = !q1, ok2 = ok1 && !q2, ok3 = ok2 && !q3;
-            float acc = 0.f;
-            if (ok3 && s + 3 >= 0 && s + 3 < a.T) acc = fmaf(cw[0], d3, acc);
-            if (ok2 && s + 2 >= 0 && s + 2 < a.T) acc = fmaf(cw[1], d2, acc);
-            if (ok1 && s + 1 >= 0 && s + 1 < a.T) acc = fmaf(cw[2], d1, acc);
-            if (s >= 0) acc = fmaf(cw[3], d0, acc);
-            if (a.dtail_final && s >= a.T - kHist && window_reads(rrow, s, a.T - 1))
-                acc += a.dtail_final[((size_t)b * kHist + (s - (a.T - kHist))) * a.W + ch];
-            if (s >= 0) a.dx[rowe + (size_t)s * a.W] = acc;
-            else if (a.dtail0) a.dtail0[((size_t)b * kHist + (kHist + s)) * a.W + ch] = acc;
+            float2 acc = z2;
+            if (ok3 && s + 3 >= 0 && s + 3 < T) acc = f2fma(cw[0], d3, acc);
+            if (ok2 && s + 2 >= 0 && s + 2 < T) acc = f2fma(cw[1], d2, acc);
+            if (ok1 && s + 1 >= 0 && s + 1 < T) acc = f2fma(cw[2], d1, acc);
+            if (s >= 0) acc = f2fma(cw[3], d0, acc);
+            if (a.dtail_final && s >= T - kHist && window_reads(rrow, s, T - 1)) {
+                const float* df = a.dtail_final + ((size_t)b * kHist + (s - (T - kHist))) * W + ch;
+                acc = make_float2(acc.x + df[0], acc.y + df[1]);
+            }
+            if (s >= 0) {
+                dxr[s * W] = acc.x;
+                dxr[s * W + 1] = acc.y;
+            } else if (a.dtail0) {
+                float* dt = a.dtail0 + ((size_t)b * kHist + (kHist + s)) * W + ch;
+                dt[0] = acc.x;
+                dt[1] = acc.y;
+            }
             d0 = d1; d1 = d2; d2 = d3;
             q0 = q1; q1 = q2; q2 = q3;
         }
     }
-    const size_t pb = (size_t)a.B * a.ntb * a.W, pi = ((size_t)b * a.ntb + tb) * a.W + ch;
+    const size_t pb = (size_t)a.B * a.ntb * W, pi = ((size_t)b * a.ntb + tb) * W + ch;
 #pragma unroll
-    for (int k = 0; k < kConvWidth; ++k) a.part[k * pb + pi] = s_cw[k];
-    a.part[4 * pb + pi] = s_cb;
+    for (int k = 0; k < kConvWidth; ++k) *reinterpret_cast<float2*>(a.part + k * pb + pi) = s_cw[k];
+    *reinterpret_cast<float2*>(a.part + 4 * pb + pi) = s_cb;
 }
 
 // ---------------------------------------------------------------- 6. fixed-order sums -------
@@ -545,7 +601,7 @@ cudaError_t launch_backward_tc(const rglru_dims* d, const rglru_params* p, const
     ca.tail0 = st0 ? static_cast<const __nv_bfloat16*>(st0->conv_tail) : nullptr;
     ca.reset = reset; ca.dtail_final = dtail_final; ca.dxc = f32(l.dxc);
     ca.dx = grads->dx; ca.dtail0 = grads->dtail0; ca.part = f32(l.part_conv);
-    bwd_convT_kernel<<<dim3((W + 127) / 128, l.ntb, B), 128, 0, s>>>(ca);
+    bwd_convT_kernel<<<dim3((W + 255) / 256, l.ntb, B), 128, 0, s>>>(ca);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 

@@ -256,10 +256,11 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
         const uint32_t idesc = idesc_bf16_f32_bmn(MT, 2 * NT);   // D_a | D_x
         const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
         // K blocks in the order they become ready: this CTA's own first, then the siblings'
+        // (CTA j sends its block to j + 1, j + 2, j + 3 in turn, so CTA nt - 1's arrives first)
         bool ok = __all_sync(0xffffffffu, wait_bounded(bar_w, 0, a, abort, 1));
         uint32_t accum = 0;
         for (int i = 0; i < kClusterSize && ok; ++i) {
-            const int j = (nt + i) % kClusterSize;
+            const int j = (nt - i + kClusterSize) % kClusterSize;
             ok = __all_sync(0xffffffffu, wait_bounded(bar_k(j), 0, a, abort, 3));
             if (!ok) break;
             tc_fence_after();

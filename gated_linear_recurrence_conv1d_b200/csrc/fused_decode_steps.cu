@@ -328,7 +328,8 @@ decode_steps_kernel(const __grid_constant__ CUtensorMap map_wa, const __grid_con
             tc_fence_after();
             const uint32_t d = tm + bi * (2 * NT);
             for (int i = 0; i < kCluster && ok; ++i) {
-                const int j = (nt + i) % kCluster;           // own block first
+                // own block first, then in arrival order (CTA j sends to j + 1, j + 2, j + 3)
+                const int j = (nt - i + kCluster) % kCluster;
                 if (j != nt && !wait_wcl(bars.k(j), ph, a, abort, 6)) {
                     ok = false;
                     break;

@@ -1,6 +1,7 @@
-"""Fits the polynomial behind the kernels' erf-form GeLU and prints it as C constants.
+"""Fits the polynomials behind the kernels' erf-form GeLU and prints them as C constants.
 
-    python gated_linear_recurrence_conv1d_b200/csrc/gelu_tail_fit.py
+    python gated_linear_recurrence_conv1d_b200/csrc/gelu_tail_fit.py            (forward)
+    python gated_linear_recurrence_conv1d_b200/csrc/gelu_tail_fit.py --precise  (backward)
 
 GeLU(y) = y Phi(y) = max(y, 0) - s Q(s) with s = |y| and Q the upper tail of the standard normal
 distribution.  Q(s) = exp(-s^2 / 2) R(s), where R(s) = Q(s) exp(s^2 / 2) is smooth and slowly
@@ -36,8 +37,39 @@ def gelu_error(coef):
     return float(np.max(np.abs(approx - exact)))
 
 
+# The backward needs Phi itself (GeLU' = Phi + v phi) to about 1e-7: R of degree PDEG in the
+# centred variable t = (s - S_MAX / 2) / (S_MAX / 2), whose power-basis coefficients stay small,
+# so that fp32 Horner keeps the fit's accuracy.
+PDEG = 14
+
+
+def fit_precise():
+    s = np.linspace(0.0, S_MAX, 200001)
+    r = 0.5 * erfc(s / np.sqrt(2.0)) * np.exp(s * s / 2.0)
+    t = (s - S_MAX / 2) / (S_MAX / 2)
+    cheb = np.polynomial.chebyshev.Chebyshev.fit(t, r, PDEG, domain=[-1.0, 1.0])
+    return cheb.convert(kind=np.polynomial.Polynomial).coef.astype(np.float32)
+
+
+def phi_error(coef):
+    s = np.linspace(0.0, S_MAX, 200001)
+    t = ((s - S_MAX / 2) / (S_MAX / 2)).astype(np.float32)
+    acc = np.full_like(t, coef[-1])
+    for k in range(len(coef) - 2, -1, -1):
+        acc = (acc * t + coef[k]).astype(np.float32)
+    q = np.exp(-s * s / 2.0) * acc.astype(np.float64)
+    return float(np.max(np.abs(q - 0.5 * erfc(s / np.sqrt(2.0)))))
+
+
 if __name__ == "__main__":
-    c = fit()
-    print(f"// degree {DEG} on [0, {S_MAX}], max |GeLU error| {gelu_error(c):.2e}")
-    for k, v in enumerate(c):
-        print(f"constexpr float kGeluR{k} = {float(v):.9e}f;")
+    import sys
+    if "--precise" in sys.argv:
+        c = fit_precise()
+        print(f"// degree {PDEG} in t = (s - {S_MAX / 2}) / {S_MAX / 2}, max |Phi error| {phi_error(c):.2e} (fp32 Horner)")
+        for k, v in enumerate(c):
+            print(f"constexpr float kPhiR{k} = {float(v):.9e}f;")
+    else:
+        c = fit()
+        print(f"// degree {DEG} on [0, {S_MAX}], max |GeLU error| {gelu_error(c):.2e}")
+        for k, v in enumerate(c):
+            print(f"constexpr float kGeluR{k} = {float(v):.9e}f;")

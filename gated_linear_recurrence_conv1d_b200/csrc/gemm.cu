@@ -16,8 +16,8 @@
 //   * a persistent CTA per SM walks output tiles of 128 x 256 (batch, m-tile, n-tile, k-slice);
 //     one warp loads K blocks of 64 through a 4-stage ring (48 KB a stage), an elected lane of
 //     another issues tcgen05.mma (M = 128, N = 256, K = 16 per instruction) into one of two TMEM
-//     accumulators of 256 columns, and 4 epilogue warps (thread = row of the tile) read the
-//     other accumulator, add Cadd and store.  The wide tile halves the operand bytes per flop
+//     accumulators of 256 columns, and 8 epilogue warps (thread = row of the tile, two warps
+//     per row, 128 columns each) read the other accumulator, add Cadd and store.  The wide tile halves the operand bytes per flop
 //     that L2 has to deliver to each SM, compared with a square 128 x 128 tile.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -43,8 +43,8 @@ constexpr uint32_t TILE_B = BN * BK * 2;           // 32768
 constexpr uint32_t STAGE_BYTES = TILE_A + TILE_B;
 constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr int kEpiWarps = 4, kWarpTma = 4, kWarpMma = 5;
-constexpr int kThreads = 6 * 32;
+constexpr int kEpiWarps = 8, kWarpTma = 8, kWarpMma = 9;   // two epilogue warps per TMEM lane quadrant
+constexpr int kThreads = 10 * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int kMaxPairs = 4;
 
@@ -290,8 +290,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
         __syncwarp();
     } else {
         // ================================ epilogue: thread = row of the tile ==================
+        // warp w reads lane quadrant w % 4 (the TMEM lanes a warp may access) and the columns
+        // [128 (w / 4), 128 (w / 4) + 128) of the tile
         const int q = warp & 3;
         const int r = q * 32 + lane;
+        const int cb = (warp >> 2) * (BN / 2);
         int tc = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
             int b, m0, n0, sp;
@@ -308,7 +311,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
             __nv_bfloat16* crow16 = a.C16 ? a.C16 + coff : nullptr;
             const float* arow = a.Cadd ? a.Cadd + b * a.add_bstride + (long long)m * a.add_ld + n0 : nullptr;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 16) {
+            for (int c0 = cb; c0 < cb + BN / 2; c0 += 16) {
                 float v[16];
                 if (no_k) {
 #pragma unroll
