@@ -85,7 +85,6 @@ Layout layout(const rglru_dims* d) {
     return l;
 }
 
-__device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
 // d/dv [v Phi(v)] = Phi(v) + v phi(v); the tanh form's derivative for the flag
 __device__ __forceinline__ float gelu_grad(float v, int tanh_form) {
@@ -162,11 +161,6 @@ __device__ __forceinline__ void gelu_and_grad(float v, int tanh_form, float& g, 
     gp = fmaf(v * e, 0.39894228040143267794f, phi_c);
 }
 
-__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bfloat16* lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    *hi = h;
-    *lo = __float2bfloat16_rn(v - __bfloat162float(h));
-}
 
 struct ScanArgs {
     int B, T, W, nch;
@@ -204,42 +198,51 @@ __device__ __forceinline__ float carry_factor(float kappa, float ga, bool rs) {
     return rs ? 0.f : at;
 }
 
-// P = prod a'_t and Q = the carry leaving the chunk's first token when none enters its last
+// P = prod a'_t and Q = the carry leaving the chunk's first token when none enters its last.
+// Thread = (row b, chunk k, channel pair ch, ch + 1): paired loads halve the address arithmetic.
+__device__ __forceinline__ float2 bf2f(const __nv_bfloat16* p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+
 __global__ void __launch_bounds__(kScanThreads) bwd_scan_agg_kernel(ScanArgs a) {
-    const int ch = blockIdx.x * kScanThreads + threadIdx.x, k = blockIdx.y, b = blockIdx.z;
+    const int ch = 2 * (blockIdx.x * kScanThreads + threadIdx.x), k = blockIdx.y, b = blockIdx.z;
     if (ch >= a.W) return;
-    const float kappa = a.c * log_sigmoid_acc(a.lambda[ch]);
+    const float kap0 = a.c * log_sigmoid_acc(a.lambda[ch]), kap1 = a.c * log_sigmoid_acc(a.lambda[ch + 1]);
     const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
     const int t0 = k * kChunk, t1 = min(a.T, t0 + kChunk);
-    float P = 1.f, g = 0.f;
+    float P0 = 1.f, P1 = 1.f, g0 = 0.f, g1 = 0.f;
     for (int tb = t1 - kPF; tb > t0 - kPF; tb -= kPF) {
-        float vga[kPF], vy[kPF], vdz[kPF];
+        float2 vga[kPF], vy[kPF], vdz[kPF];
         bool rs[kPF];
+        const size_t eb = ((size_t)b * a.T + tb) * a.W + ch;
 #pragma unroll
         for (int j = 0; j < kPF; ++j) {
-            const int t = tb + j;
-            if (t >= t0) {
-                const size_t e = ((size_t)b * a.T + t) * a.W + ch;
-                vga[j] = a.ga[e];
-                vy[j] = bf(a.y + e);
-                vdz[j] = bf(a.dout + e);
-                rs[j] = rrow && rrow[t];
+            if (tb + j >= t0) {
+                const size_t e = eb + (size_t)j * a.W;
+                vga[j] = *reinterpret_cast<const float2*>(a.ga + e);
+                vy[j] = bf2f(a.y + e);
+                vdz[j] = bf2f(a.dout + e);
+                rs[j] = rrow && rrow[tb + j];
             }
         }
 #pragma unroll
         for (int j = kPF - 1; j >= 0; --j) {
             if (tb + j < t0) continue;
             float gl, gp;
-            gelu_and_grad(vy[j], a.gelu_tanh, gl, gp);
-            g = fmaf(vdz[j], gl, g);
-            const float f = carry_factor(kappa, vga[j], rs[j]);
-            g *= f;
-            P *= f;
+            gelu_and_grad(vy[j].x, a.gelu_tanh, gl, gp);
+            g0 = fmaf(vdz[j].x, gl, g0);
+            gelu_and_grad(vy[j].y, a.gelu_tanh, gl, gp);
+            g1 = fmaf(vdz[j].y, gl, g1);
+            const float f0 = carry_factor(kap0, vga[j].x, rs[j]), f1 = carry_factor(kap1, vga[j].y, rs[j]);
+            g0 *= f0;
+            g1 *= f1;
+            P0 *= f0;
+            P1 *= f1;
         }
     }
     const size_t pb = (size_t)a.B * a.nch * a.W, pi = ((size_t)b * a.nch + k) * a.W + ch;
-    a.agg[pi] = P;
-    a.agg[pb + pi] = g;
+    *reinterpret_cast<float2*>(a.agg + pi) = make_float2(P0, P1);
+    *reinterpret_cast<float2*>(a.agg + pb + pi) = make_float2(g0, g1);
 }
 
 // per (row, channel): the carries into every chunk, from the last chunk to the first
@@ -268,65 +271,103 @@ __global__ void __launch_bounds__(kScanThreads) bwd_scan_carry_kernel(ScanArgs a
     if (a.dh0) a.dh0[(size_t)b * a.W + ch] = c;
 }
 
-// every output of a chunk, from the carry into its last token
+// every output of a chunk, from the carry into its last token; thread = (row b, chunk k, channel
+// pair ch, ch + 1), kPF2 tokens a batch
+constexpr int kPF2 = 4;
+
+struct ScanOut1 {             // the results of one token-channel
+    float dy, dxc, dga, dgx, q;
+};
+__device__ __forceinline__ ScanOut1 scan_out_one(float kappa, float ga, float gx, float hp, float xcv, float yv,
+                                                 float dz, int tanh_form, float& g) {
+    const float r = sig_fast(ga), ig = sig_fast(gx);
+    float at, beta;
+    decay_beta_fast(kappa, r, at, beta);
+    const float h = fmaf(at, hp, beta * (ig * xcv));
+    float gl, gp;
+    gelu_and_grad(yv, tanh_form, gl, gp);
+    g = fmaf(dz, gl, g);
+    ScanOut1 o;
+    o.dy = dz * h * gp;
+    const float dl_da = g * hp, dl_dbeta = g * ig * xcv, dl_di = g * beta * xcv;
+    const float r_over_beta = beta > 0.f ? r * fm::rcpf(beta) : 0.f;
+    o.q = dl_da * at * r - dl_dbeta * at * at * r_over_beta;
+    o.dga = kappa * (1.0f - r) * o.q;
+    o.dgx = dl_di * ig * (1.0f - ig);
+    o.dxc = g * beta * ig;
+    g *= at;                                             // the carry to the previous token
+    return o;
+}
+
+// bf16 pair hi + lo of two fp32 values, each packed in one word
+__device__ __forceinline__ void split_bf16x2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+    const float2 hf = __bfloat1622float2(h);
+    __nv_bfloat162 l = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+    hi = *reinterpret_cast<uint32_t*>(&h);
+    lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
 __global__ void __launch_bounds__(kScanThreads) bwd_scan_out_kernel(ScanArgs a) {
-    const int ch = blockIdx.x * kScanThreads + threadIdx.x, k = blockIdx.y, b = blockIdx.z;
+    const int ch = 2 * (blockIdx.x * kScanThreads + threadIdx.x), k = blockIdx.y, b = blockIdx.z;
     if (ch >= a.W) return;
-    const float kappa = a.c * log_sigmoid_acc(a.lambda[ch]);
-    const float c_sneg = a.c * sigmoid_acc(-a.lambda[ch]);
+    const float kap0 = a.c * log_sigmoid_acc(a.lambda[ch]), kap1 = a.c * log_sigmoid_acc(a.lambda[ch + 1]);
+    const float cs0 = a.c * sigmoid_acc(-a.lambda[ch]), cs1 = a.c * sigmoid_acc(-a.lambda[ch + 1]);
     const size_t pb = (size_t)a.B * a.nch * a.W, pi = ((size_t)b * a.nch + k) * a.W + ch;
-    float g = a.agg[pb + pi];
-    float s_lam = 0.f, s_ba = 0.f, s_bx = 0.f;
+    const float2 gin = *reinterpret_cast<const float2*>(a.agg + pb + pi);
+    float g0 = gin.x, g1 = gin.y;
+    float2 s_lam = make_float2(0.f, 0.f), s_ba = s_lam, s_bx = s_lam;
     const uint8_t* rrow = a.reset ? a.reset + (size_t)b * a.T : nullptr;
     const int t0 = k * kChunk, t1 = min(a.T, t0 + kChunk);
-    for (int tb = t1 - kPF; tb > t0 - kPF; tb -= kPF) {
-        float vga[kPF], vgx[kPF], vhp[kPF], vxc[kPF], vy[kPF], vdz[kPF];
-        bool rs[kPF];
+    for (int tb = t1 - kPF2; tb > t0 - kPF2; tb -= kPF2) {
+        float2 vga[kPF2], vgx[kPF2], vhp[kPF2], vxh[kPF2], vxl[kPF2], vy[kPF2], vdz[kPF2];
+        bool rs[kPF2];
+        const size_t eb = ((size_t)b * a.T + tb) * a.W + ch;
 #pragma unroll
-        for (int j = 0; j < kPF; ++j) {
-            const int t = tb + j;
-            if (t >= t0) {
-                const size_t e = ((size_t)b * a.T + t) * a.W + ch;
-                vga[j] = a.ga[e];
-                vgx[j] = a.gx[e];
-                vhp[j] = a.hprev[e];
-                vxc[j] = bf(a.xc_hi + e) + bf(a.xc_lo + e);
-                vy[j] = bf(a.y + e);
-                vdz[j] = bf(a.dout + e);
-                rs[j] = rrow && rrow[t];
+        for (int j = 0; j < kPF2; ++j) {
+            if (tb + j >= t0) {
+                const size_t e = eb + (size_t)j * a.W;
+                vga[j] = *reinterpret_cast<const float2*>(a.ga + e);
+                vgx[j] = *reinterpret_cast<const float2*>(a.gx + e);
+                vhp[j] = *reinterpret_cast<const float2*>(a.hprev + e);
+                vxh[j] = bf2f(a.xc_hi + e);
+                vxl[j] = bf2f(a.xc_lo + e);
+                vy[j] = bf2f(a.y + e);
+                vdz[j] = bf2f(a.dout + e);
+                rs[j] = rrow && rrow[tb + j];
             }
         }
 #pragma unroll
-        for (int j = kPF - 1; j >= 0; --j) {
+        for (int j = kPF2 - 1; j >= 0; --j) {
             if (tb + j < t0) continue;
-            const size_t e = ((size_t)b * a.T + tb + j) * a.W + ch;
-            const float r = sig_fast(vga[j]), ig = sig_fast(vgx[j]);
-            float at, beta;
-            decay_beta_fast(kappa, r, at, beta);
-            const float xcv = vxc[j], hp = vhp[j];
-            const float h = fmaf(at, hp, beta * (ig * xcv));
-            float gl, gp;
-            gelu_and_grad(vy[j], a.gelu_tanh, gl, gp);
-            g = fmaf(vdz[j], gl, g);
-            a.dy[e] = vdz[j] * h * gp;
-            const float dl_da = g * hp, dl_dbeta = g * ig * xcv, dl_di = g * beta * xcv;
-            const float r_over_beta = beta > 0.f ? r * fm::rcpf(beta) : 0.f;
-            const float q = dl_da * at * r - dl_dbeta * at * at * r_over_beta;
-            const float dga = kappa * (1.0f - r) * q;
-            const float dgx = dl_di * ig * (1.0f - ig);
-            s_lam = fmaf(c_sneg, q, s_lam);
-            s_ba += dga;
-            s_bx += dgx;
-            split_bf16(dga, a.dga_hi + e, a.dga_lo + e);
-            split_bf16(dgx, a.dgx_hi + e, a.dgx_lo + e);
-            a.dxc[e] = g * beta * ig;
-            g = rs[j] ? 0.f : at * g;
+            const size_t e = eb + (size_t)j * a.W;
+            const ScanOut1 o0 = scan_out_one(kap0, vga[j].x, vgx[j].x, vhp[j].x, vxh[j].x + vxl[j].x, vy[j].x,
+                                             vdz[j].x, a.gelu_tanh, g0);
+            const ScanOut1 o1 = scan_out_one(kap1, vga[j].y, vgx[j].y, vhp[j].y, vxh[j].y + vxl[j].y, vy[j].y,
+                                             vdz[j].y, a.gelu_tanh, g1);
+            a.dy[e] = o0.dy;                             // caller's buffer: 4-byte aligned only
+            a.dy[e + 1] = o1.dy;
+            *reinterpret_cast<float2*>(a.dxc + e) = make_float2(o0.dxc, o1.dxc);
+            uint32_t hi, lo;
+            split_bf16x2(o0.dga, o1.dga, hi, lo);
+            *reinterpret_cast<uint32_t*>(a.dga_hi + e) = hi;
+            *reinterpret_cast<uint32_t*>(a.dga_lo + e) = lo;
+            split_bf16x2(o0.dgx, o1.dgx, hi, lo);
+            *reinterpret_cast<uint32_t*>(a.dgx_hi + e) = hi;
+            *reinterpret_cast<uint32_t*>(a.dgx_lo + e) = lo;
+            s_lam.x = fmaf(cs0, o0.q, s_lam.x);
+            s_lam.y = fmaf(cs1, o1.q, s_lam.y);
+            s_ba.x += o0.dga;
+            s_ba.y += o1.dga;
+            s_bx.x += o0.dgx;
+            s_bx.y += o1.dgx;
+            if (rs[j]) g0 = g1 = 0.f;                    // no carry across a segment start
         }
     }
     const size_t ps = (size_t)a.B * a.nch * a.W;
-    a.part[pi] = s_lam;
-    a.part[ps + pi] = s_ba;
-    a.part[2 * ps + pi] = s_bx;
+    *reinterpret_cast<float2*>(a.part + pi) = s_lam;
+    *reinterpret_cast<float2*>(a.part + ps + pi) = s_ba;
+    *reinterpret_cast<float2*>(a.part + 2 * ps + pi) = s_bx;
 }
 
 struct ConvTArgs {
@@ -573,9 +614,10 @@ cudaError_t launch_backward_tc(const rglru_dims* d, const rglru_params* p, const
     sa.dga_hi = b16(l.dga_hi); sa.dga_lo = b16(l.dga_lo); sa.dgx_hi = b16(l.dgx_hi); sa.dgx_lo = b16(l.dgx_lo);
     sa.dh0 = grads->dh0; sa.agg = f32(l.agg); sa.part = f32(l.part_scan);
     const unsigned cblk = (unsigned)((W + kScanThreads - 1) / kScanThreads);
-    bwd_scan_agg_kernel<<<dim3(cblk, l.nch, B), kScanThreads, 0, s>>>(sa);
+    const unsigned cblk2 = (unsigned)((W / 2 + kScanThreads - 1) / kScanThreads);   // channel pairs
+    bwd_scan_agg_kernel<<<dim3(cblk2, l.nch, B), kScanThreads, 0, s>>>(sa);
     bwd_scan_carry_kernel<<<dim3(cblk, B), kScanThreads, 0, s>>>(sa);
-    bwd_scan_out_kernel<<<dim3(cblk, l.nch, B), kScanThreads, 0, s>>>(sa);
+    bwd_scan_out_kernel<<<dim3(cblk2, l.nch, B), kScanThreads, 0, s>>>(sa);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
