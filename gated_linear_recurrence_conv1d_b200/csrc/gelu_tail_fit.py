@@ -38,22 +38,23 @@ def gelu_error(coef):
 
 
 # The backward needs Phi itself (GeLU' = Phi + v phi) to about 1e-7: R of degree PDEG in the
-# centred variable t = (s - S_MAX / 2) / (S_MAX / 2), whose power-basis coefficients stay small,
+# centred variable t = (s - P_SMAX / 2) / (P_SMAX / 2), whose power-basis coefficients stay small,
 # so that fp32 Horner keeps the fit's accuracy.
 PDEG = 14
+P_SMAX = 5.5
 
 
 def fit_precise():
-    s = np.linspace(0.0, S_MAX, 200001)
+    s = np.linspace(0.0, P_SMAX, 200001)
     r = 0.5 * erfc(s / np.sqrt(2.0)) * np.exp(s * s / 2.0)
-    t = (s - S_MAX / 2) / (S_MAX / 2)
+    t = (s - P_SMAX / 2) / (P_SMAX / 2)
     cheb = np.polynomial.chebyshev.Chebyshev.fit(t, r, PDEG, domain=[-1.0, 1.0])
     return cheb.convert(kind=np.polynomial.Polynomial).coef.astype(np.float32)
 
 
 def phi_error(coef):
-    s = np.linspace(0.0, S_MAX, 200001)
-    t = ((s - S_MAX / 2) / (S_MAX / 2)).astype(np.float32)
+    s = np.linspace(0.0, P_SMAX, 200001)
+    t = ((s - P_SMAX / 2) / (P_SMAX / 2)).astype(np.float32)
     acc = np.full_like(t, coef[-1])
     for k in range(len(coef) - 2, -1, -1):
         acc = (acc * t + coef[k]).astype(np.float32)
@@ -65,7 +66,7 @@ if __name__ == "__main__":
     import sys
     if "--precise" in sys.argv:
         c = fit_precise()
-        print(f"// degree {PDEG} in t = (s - {S_MAX / 2}) / {S_MAX / 2}, max |Phi error| {phi_error(c):.2e} (fp32 Horner)")
+        print(f"// degree {PDEG} in t = (s - {P_SMAX / 2}) / {P_SMAX / 2}, max |Phi error| {phi_error(c):.2e} (fp32 Horner)")
         for k, v in enumerate(c):
             print(f"constexpr float kPhiR{k} = {float(v):.9e}f;")
     else:
