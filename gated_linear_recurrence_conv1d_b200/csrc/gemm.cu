@@ -16,8 +16,10 @@
 //   * a persistent CTA per SM walks output tiles of 128 x 256 (batch, m-tile, n-tile, k-slice);
 //     one warp loads K blocks of 64 through a 4-stage ring (48 KB a stage), an elected lane of
 //     another issues tcgen05.mma (M = 128, N = 256, K = 16 per instruction) into one of two TMEM
-//     accumulators of 256 columns, and 8 epilogue warps (thread = row of the tile, two warps
-//     per row, 128 columns each) read the other accumulator, add Cadd and store.  The wide tile halves the operand bytes per flop
+//     accumulators of 256 columns, and 8 epilogue warps (two per TMEM lane quadrant, 128
+//     columns each) read the other accumulator 32 columns at a time and pass it through a
+//     swizzled shared-memory tile, so that Cadd is read and C written in whole 128-byte row
+//     segments.  The wide tile halves the operand bytes per flop
 //     that L2 has to deliver to each SM, compared with a square 128 x 128 tile.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -42,7 +44,13 @@ constexpr uint32_t TILE_A = BM * BK * 2;           // 16384
 constexpr uint32_t TILE_B = BN * BK * 2;           // 32768
 constexpr uint32_t STAGE_BYTES = TILE_A + TILE_B;
 constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
+// per epilogue warp, a [32 rows x 32 columns] fp32 staging tile (rows of 128 B, 16-byte chunks
+// XOR-swizzled by the row): the warp's accumulator rows go in row by row and come out as whole
+// 128-byte row segments, so that global loads and stores are coalesced
+constexpr uint32_t OFF_STG = OFF_BAR + 256;
+constexpr uint32_t STG_BYTES = 32 * 32 * 4;
+constexpr uint32_t SMEM_BYTES = OFF_STG + 8 * STG_BYTES + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 constexpr int kEpiWarps = 8, kWarpTma = 8, kWarpMma = 9;   // two epilogue warps per TMEM lane quadrant
 constexpr int kThreads = 10 * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -293,7 +301,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
         // warp w reads lane quadrant w % 4 (the TMEM lanes a warp may access) and the columns
         // [128 (w / 4), 128 (w / 4) + 128) of the tile
         const int q = warp & 3;
-        const int r = q * 32 + lane;
         const int cb = (warp >> 2) * (BN / 2);
         int tc = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
@@ -302,54 +309,55 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
             const int ai = tc & 1;
             if (!__all_sync(0xffffffffu, wait_b(acc_full(ai), (tc >> 1) & 1, a, abort, 4))) break;
             tc_fence_after();
-            const int m = m0 + r;
             // a K slice without blocks (more slices than K blocks) contributes zeros: its
             // accumulator was never written
             const bool no_k = sp * kp.per >= kp.total;
-            const long long coff = sp * a.c_split + b * a.c_bstride + (long long)m * a.c_ld + n0;
-            float* crow = a.C + coff;
-            __nv_bfloat16* crow16 = a.C16 ? a.C16 + coff : nullptr;
-            const float* arow = a.Cadd ? a.Cadd + b * a.add_bstride + (long long)m * a.add_ld + n0 : nullptr;
+            uint8_t* stg = smem + OFF_STG + (uint32_t)warp * STG_BYTES;
+            const long long tbase = sp * a.c_split + b * a.c_bstride;
+            const long long abase = b * a.add_bstride;
 #pragma unroll 1
-            for (int c0 = cb; c0 < cb + BN / 2; c0 += 16) {
-                float v[16];
+            for (int c0 = cb; c0 < cb + BN / 2; c0 += 32) {
+                float v0[16], v1[16];
                 if (no_k) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) v[j] = 0.f;
+                    for (int j = 0; j < 16; ++j) v0[j] = v1[j] = 0.f;
                 } else {
-                    tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + ai * BN + c0, v);
+                    const uint32_t ta = tmem + ((uint32_t)(q * 32) << 16) + ai * BN + c0;
+                    tmem_ld16(ta, v0);
+                    tmem_ld16(ta + 16, v1);
                     tmem_wait_ld();
                 }
-                if (m < a.M && crow16) {
-                    const int nn = a.N - (n0 + c0);
-                    if (nn >= 16) {
-                        uint32_t pk[8];
+                // row `lane` of the warp's 32 rows into the staging tile
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            __nv_bfloat162 p2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-                            pk[j] = *reinterpret_cast<uint32_t*>(&p2);
-                        }
-                        *reinterpret_cast<uint4*>(crow16 + c0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        *reinterpret_cast<uint4*>(crow16 + c0 + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    } else {
-                        for (int j = 0; j < nn; ++j) crow16[c0 + j] = __float2bfloat16_rn(v[j]);
-                    }
-                } else if (m < a.M) {
-                    const int nn = a.N - (n0 + c0);
-                    if (nn >= 16) {
+                for (int j = 0; j < 4; ++j) {
+                    *reinterpret_cast<float4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                        make_float4(v0[4 * j], v0[4 * j + 1], v0[4 * j + 2], v0[4 * j + 3]);
+                    *reinterpret_cast<float4*>(stg + lane * 128 + (((j + 4) ^ (lane & 7)) << 4)) =
+                        make_float4(v1[4 * j], v1[4 * j + 1], v1[4 * j + 2], v1[4 * j + 3]);
+                }
+                __syncwarp();
+                // out as 4 rows x 32 columns per step: lane = (row 4 i + lane / 8, 4 columns)
 #pragma unroll
-                        for (int j = 0; j < 16; j += 4) {
-                            float4 o = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-                            if (arow) {
-                                const float4 ad = *reinterpret_cast<const float4*>(arow + c0 + j);
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = 4 * i + (lane >> 3), cc = lane & 7;
+                    float4 o = *reinterpret_cast<const float4*>(stg + rr * 128 + ((cc ^ (rr & 7)) << 4));
+                    const int m = m0 + q * 32 + rr, n = n0 + c0 + 4 * cc;
+                    if (m < a.M && n < a.N) {                // N is a multiple of 16: n + 3 < N too
+                        const long long off = tbase + (long long)m * a.c_ld + n;
+                        if (a.C16) {
+                            __nv_bfloat162 p0 = __floats2bfloat162_rn(o.x, o.y), p1 = __floats2bfloat162_rn(o.z, o.w);
+                            *reinterpret_cast<uint2*>(a.C16 + off) =
+                                make_uint2(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1));
+                        } else {
+                            if (a.Cadd) {
+                                const float4 ad = *reinterpret_cast<const float4*>(a.Cadd + abase + (long long)m * a.add_ld + n);
                                 o.x += ad.x; o.y += ad.y; o.z += ad.z; o.w += ad.w;
                             }
-                            *reinterpret_cast<float4*>(crow + c0 + j) = o;
+                            *reinterpret_cast<float4*>(a.C + off) = o;
                         }
-                    } else {
-                        for (int j = 0; j < nn; ++j) crow[c0 + j] = v[j] + (arow ? arow[c0 + j] : 0.f);
                     }
                 }
+                __syncwarp();
             }
             tc_fence_before();
             __syncwarp();
