@@ -336,7 +336,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
                         make_float4(v1[4 * j], v1[4 * j + 1], v1[4 * j + 2], v1[4 * j + 3]);
                 }
                 __syncwarp();
-                // out as 4 rows x 32 columns per step: lane = (row 4 i + lane / 8, 4 columns)
+                // out as 4 rows x 32 columns per step: lane = (row 4 i + lane / 8, 4 columns); every
+                // Cadd load is issued before any store (C may be Cadd itself, accumulated in place)
+                float4 add[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int m = m0 + q * 32 + 4 * i + (lane >> 3), n = n0 + c0 + 4 * (lane & 7);
+                    add[i] = a.Cadd && m < a.M && n < a.N
+                                 ? *reinterpret_cast<const float4*>(a.Cadd + abase + (long long)m * a.add_ld + n)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int rr = 4 * i + (lane >> 3), cc = lane & 7;
@@ -349,10 +358,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
                             *reinterpret_cast<uint2*>(a.C16 + off) =
                                 make_uint2(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1));
                         } else {
-                            if (a.Cadd) {
-                                const float4 ad = *reinterpret_cast<const float4*>(a.Cadd + abase + (long long)m * a.add_ld + n);
-                                o.x += ad.x; o.y += ad.y; o.z += ad.z; o.w += ad.w;
-                            }
+                            o.x += add[i].x; o.y += add[i].y; o.z += add[i].z; o.w += add[i].w;
                             *reinterpret_cast<float4*>(a.C + off) = o;
                         }
                     }
