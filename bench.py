@@ -856,6 +856,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the layer and MQA entries")
+    ap.add_argument("--extras-only", action="store_true",
+                    help="time only the backward, layer and MQA entries (prints their JSON object)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -865,6 +867,11 @@ def main():
         import torch
         dev = torch.device("cuda", torch.cuda.current_device())
         print(json.dumps(bench_decode(args, dev)))
+    elif args.extras_only:
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device())
+        print(json.dumps({"backward": bench_backward(args, dev), "layer": bench_layer(args, dev),
+                          "mqa": bench_mqa(args, dev)}))
     else:
         run_ours(args)
 
