@@ -170,5 +170,46 @@ __device__ __forceinline__ float2 gelu_tanh2(float2 y) {
 }
 __device__ __forceinline__ float gelu1(float y, int tanh_form) { return tanh_form ? gelu_tanh1(y) : gelu_erf1(y); }
 
+// Phi(v) to ~1e-7 without erfc, for the gradients: with s = |v| and e = exp(-v^2 / 2) (one exp2,
+// returned too), the upper tail Q(s) = e R(s), R a degree-14 polynomial in t = (s - 2.75) / 2.75
+// on s in [0, 5.5] (s clamped there; beyond it Q < 2e-8), fitted by gelu_tail_fit.py --precise
+// beside this file (max |Phi error| 1.1e-7 in fp32); Phi(v) = 1 - Q for v >= 0, Q otherwise.
+constexpr float kPhiR0 = 1.307247281e-01f;
+constexpr float kPhiR1 = -1.084856018e-01f;
+constexpr float kPhiR2 = 8.409250528e-02f;
+constexpr float kPhiR3 = -6.148617715e-02f;
+constexpr float kPhiR4 = 4.272365198e-02f;
+constexpr float kPhiR5 = -2.843398601e-02f;
+constexpr float kPhiR6 = 1.814154349e-02f;
+constexpr float kPhiR7 = -1.083536446e-02f;
+constexpr float kPhiR8 = 6.395316683e-03f;
+constexpr float kPhiR9 = -4.469349980e-03f;
+constexpr float kPhiR10 = 2.545840805e-03f;
+constexpr float kPhiR11 = -3.012927773e-04f;
+constexpr float kPhiR12 = 1.266671024e-04f;
+constexpr float kPhiR13 = -8.168322383e-04f;
+constexpr float kPhiR14 = 4.210809420e-04f;
+__device__ __forceinline__ float phi_precise(float v, float& e) {
+    e = ex2f((v * v) * (-0.5f * kLog2e));
+    const float t = fmaf(fminf(fabsf(v), 5.5f), 1.0f / 2.75f, -1.0f);
+    float r = kPhiR14;
+    r = fmaf(r, t, kPhiR13);
+    r = fmaf(r, t, kPhiR12);
+    r = fmaf(r, t, kPhiR11);
+    r = fmaf(r, t, kPhiR10);
+    r = fmaf(r, t, kPhiR9);
+    r = fmaf(r, t, kPhiR8);
+    r = fmaf(r, t, kPhiR7);
+    r = fmaf(r, t, kPhiR6);
+    r = fmaf(r, t, kPhiR5);
+    r = fmaf(r, t, kPhiR4);
+    r = fmaf(r, t, kPhiR3);
+    r = fmaf(r, t, kPhiR2);
+    r = fmaf(r, t, kPhiR1);
+    r = fmaf(r, t, kPhiR0);
+    const float q = e * r;
+    return v >= 0.f ? 1.0f - q : q;
+}
+
 }  // namespace fm
 }  // namespace rglru
