@@ -16,9 +16,10 @@
 //     reference maximum that moves only when the maximum grows by more than 2^8 (then the
 //     accumulator is rescaled), write P in bf16 to shared memory; O += P V (M = 128, N = 256,
 //     K = 64) accumulates in TMEM; the S of the next tile overlaps the softmax of this one;
-//   * mqa_decode_kernel: one token per row against the ring: CTAs split the ring's slots, each
-//     keeps (max, sum, sum of p v) per head over its part (CUDA cores: the step is bound by
-//     reading the cache, not by its arithmetic); mqa_merge_kernel combines the parts.
+//   * mqa_decode_kernel: one token per row against the ring: CTAs split the ring's slots into
+//     parts of 128; per part S^T = K Q^T and O^T = V^T P^T run on the tensor cores (the H heads
+//     of a row form the MMA's N), the softmax of the part on 4 warps; each CTA leaves (max, sum,
+//     sum of p v) per head, and mqa_merge_kernel combines the parts.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -475,159 +476,285 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 // ---------------------------------------------------------------- decode ---------------------
 // One token per row against its ring.  The window is a set: softmax over it does not depend on
 // the order of its keys, and the ring holds exactly the window -- slots [0, n), n = min(pos + 1,
-// w) (slot = position mod w, keys cached after their rotation) -- so a CTA walks the slots of its
-// split in slot order.  CTA = (split of kDecPer slots, row); 256 threads:
-//   * scores: lane = slot; a lane streams its key row (16-byte loads) and accumulates q_h . k
-//     for every head with packed fp32x2 FMAs, the rotated queries read from shared memory as
-//     broadcasts;
-//   * softmax of the split per head (warp shuffles): its maximum m_h, sum l_h, weights in shared
-//     memory;
-//   * thread = (pair of value columns, half of the split's slots): sum of p v over its slots,
-//     halves added through shared memory; (m, l, o) per head go to the merge.
-// The step moves the whole ring (2 w d bf16 per row): it is bound by HBM, not by arithmetic.
-constexpr int kDecThreads = D;
-constexpr int kDecPer = 256;           // slots per split
-constexpr int kMaxH = 16;
+// w) (slot = position mod w, keys cached after their rotation) -- so a CTA takes a split of
+// kDecPer consecutive slots.  Per CTA, on the tensor cores:
+//   * TMA brings the split's keys [128 slots x 256 d] and the row's rotated queries [16 x 256]
+//     (heads past H read other data: their columns are never used) in the 128-byte swizzle;
+//   * S^T = K Q^T (M = 128 slots, N = 16 heads, K = 256): a TMEM lane is a slot;
+//   * meanwhile the values come into the keys' place once the MMAs have read them;
+//   * 4 warps (thread = slot) mask the slots past n, take per head the split's maximum and sum
+//     (shuffles, then across the warps) and write p = exp(s - m) in bf16 as the B operand of
+//     O^T = V^T P^T (M = 128 d-columns x 2, N = 16, K = 128 slots; V^T is the value tile read
+//     MN-major); value rows past n are zeroed first (an unfilled slot may hold anything);
+//   * the same warps read O^T (thread = d-column) and write (m, l, o) per head for the merge.
+// The step reads the ring once (2 w d bf16 per row): it is bound by HBM.
+constexpr int kDecPer = 128;           // slots per split (the MMA's M)
+constexpr int kMaxH = 16;              // heads (the MMA's N), padded
+constexpr uint32_t KV_BYTES = kDecPer * D * 2;        // 65536: 4 boxes of [128 slots x 64 d]
+constexpr uint32_t QD_BYTES = kMaxH * D * 2;          // 8192: 4 boxes of [16 heads x 64 d]
+constexpr uint32_t PD_BYTES = kMaxH * kDecPer * 2;    // 4096: 2 K blocks of [16 heads x 64 slots]
+constexpr uint32_t D_OFF_KV = 0;
+constexpr uint32_t D_OFF_Q = D_OFF_KV + KV_BYTES;
+constexpr uint32_t D_OFF_P = D_OFF_Q + QD_BYTES;
+constexpr uint32_t D_OFF_RED = D_OFF_P + PD_BYTES;   // [2][4 warps][16] fp32: maxima, then sums
+constexpr uint32_t D_OFF_BAR = D_OFF_RED + 2 * 4 * kMaxH * 4;
+constexpr uint32_t D_SMEM_BYTES = D_OFF_BAR + 128 + 1024;
+constexpr uint32_t D_TM_S = 0, D_TM_O = 32, D_TMEM_COLS = 64;
+constexpr int kDecThreads = 6 * 32;    // 4 softmax / epilogue warps, a TMA warp, an MMA warp
 
 struct DecArgs {
     int B, H, w, nsplit;
     float scale;
-    const __nv_bfloat16* q_rot;        // [B, H, d]
     const int* pos;                    // [B]
     const __nv_bfloat16* cache;        // [B][2][w][d]
     float* part_m;                     // [B][nsplit][H]
     float* part_l;
     float* part_o;                     // [B][nsplit][H][d]
+    DeviceStatus* status;
+    unsigned long long timeout_ns;
 };
 
-__device__ __forceinline__ float2 bf2_to_f2(uint32_t v) {
-    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+struct DBars {
+    uint32_t base;
+    __device__ __forceinline__ uint32_t kq_full() const { return base; }
+    __device__ __forceinline__ uint32_t s_full() const { return base + 8; }     // S^T done: keys read
+    __device__ __forceinline__ uint32_t v_full() const { return base + 16; }
+    __device__ __forceinline__ uint32_t p_full() const { return base + 24; }    // P written, V rows zeroed
+    __device__ __forceinline__ uint32_t o_full() const { return base + 32; }
+};
+
+__device__ __noinline__ bool dwait_slow(uint32_t bar, uint32_t parity, const DecArgs& a, volatile int* abort,
+                                        unsigned where) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (*abort) return false;
+        if (*(volatile unsigned*)&a.status->code != 0) {
+            *abort = 1;
+            return false;
+        }
+        if (globaltimer_ns() - t0 > a.timeout_ns) {
+            latch_status(a.status, RGLRU_ERR_TIMEOUT, where, blockIdx.x, parity);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool dwait(uint32_t bar, uint32_t parity, const DecArgs& a, volatile int* abort,
+                                      unsigned where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return dwait_slow(bar, parity, a, abort, where);
 }
 
-template <int HM>
-__global__ void __launch_bounds__(kDecThreads) mqa_decode_kernel(DecArgs a) {
-    __shared__ __align__(16) float qs[HM][D];
-    __shared__ __align__(16) float ps[HM][kDecPer];
-    __shared__ float mh[HM], lh[HM];
-    const int sp = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int H = a.H;
-    const int n = min(a.pos[b] + 1, a.w);               // slots in the window
+// MN-major (128-byte swizzle) descriptor of the value tile read as V^T: atoms of 64 d-columns,
+// each [128 slots x 128 B], 16384 B apart
+__device__ __forceinline__ uint64_t desc_vt(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+    d |= (uint64_t)(16384 >> 4) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+// fp32 accumulator, bf16 operands, A K-major (a_mn = 0) or MN-major (1), B K-major, M 128, N 16
+__device__ __forceinline__ uint32_t idesc_dec(int a_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)(kMaxH >> 3) << 17) |
+           ((uint32_t)(kDecPer >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(kDecThreads, 2)
+mqa_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
+                  const DecArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const DBars bars{sbase + D_OFF_BAR};
+    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + D_OFF_BAR + 64);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + D_OFF_BAR + 80);
+    float* red = reinterpret_cast<float*>(smem + D_OFF_RED);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int sp = blockIdx.x, b = blockIdx.y, H = a.H;
+    const int n = min(a.pos[b] + 1, a.w);                // slots in the window
     const int s0 = sp * kDecPer, cnt = max(0, min(n, s0 + kDecPer) - s0);
-    for (int e = tid; e < H * D; e += kDecThreads)
-        qs[e / D][e % D] = __bfloat162float(a.q_rot[(size_t)b * H * D + e]);
-    __syncthreads();
-    const __nv_bfloat16* kc = a.cache + (size_t)b * 2 * a.w * D;
-    const __nv_bfloat16* vc = kc + (size_t)a.w * D;
-
-    // ---- scores: lane = slot s0 + 32 warp + lane
-#pragma unroll 1
-    for (int i0 = 32 * warp; i0 < kDecPer; i0 += 32 * (kDecThreads / 32)) {
-        const int i = i0 + lane;
-        float2 acc[HM];
-#pragma unroll
-        for (int h = 0; h < HM; ++h) acc[h] = make_float2(0.f, 0.f);
-        if (i < cnt) {
-            const uint4* kr = reinterpret_cast<const uint4*>(kc + (size_t)(s0 + i) * D);
-#pragma unroll 4
-            for (int c = 0; c < D / 8; ++c) {
-                const uint4 kv = __ldg(kr + c);
-                const float2 k0 = bf2_to_f2(kv.x), k1 = bf2_to_f2(kv.y), k2 = bf2_to_f2(kv.z), k3 = bf2_to_f2(kv.w);
-#pragma unroll
-                for (int h = 0; h < HM; ++h) {
-                    if (h < H) {
-                        const float4 qa = *reinterpret_cast<const float4*>(&qs[h][8 * c]);
-                        const float4 qb = *reinterpret_cast<const float4*>(&qs[h][8 * c + 4]);
-                        float2 t = acc[h];
-                        t = __ffma2_rn(make_float2(qa.x, qa.y), k0, t);
-                        t = __ffma2_rn(make_float2(qa.z, qa.w), k1, t);
-                        t = __ffma2_rn(make_float2(qb.x, qb.y), k2, t);
-                        t = __ffma2_rn(make_float2(qb.z, qb.w), k3, t);
-                        acc[h] = t;
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int h = 0; h < HM; ++h)
-            if (h < H) ps[h][i] = i < cnt ? (acc[h].x + acc[h].y) * a.scale : -INFINITY;
-    }
-    __syncthreads();
-
-    // ---- softmax of the split, one warp per head
-    for (int h = warp; h < H; h += kDecThreads / 32) {
-        float v[kDecPer / 32];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < kDecPer / 32; ++j) {
-            v[j] = ps[h][lane + 32 * j];
-            mx = fmaxf(mx, v[j]);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        float l = 0.f;
-#pragma unroll
-        for (int j = 0; j < kDecPer / 32; ++j) {
-            const float p = mx == -INFINITY ? 0.f : expf(v[j] - mx);
-            ps[h][lane + 32 * j] = p;
-            l += p;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-        if (lane == 0) {
-            mh[h] = mx;
-            lh[h] = l;
-        }
-    }
-    __syncthreads();
-
-    // ---- o = sum_i p_i v_i: thread = (columns 2 dp, 2 dp + 1; half kh of the slots)
-    const int dp = tid & (D / 2 - 1), kh = tid / (D / 2);
-    const int half = ((cnt + 7) / 8) * 4;                // slots per half, a multiple of 4
-    const int i_beg = kh * half, i_end = min(cnt, i_beg + half);
-    float2 o[HM];
-#pragma unroll
-    for (int h = 0; h < HM; ++h) o[h] = make_float2(0.f, 0.f);
-#pragma unroll 1
-    for (int i = i_beg; i < i_end; i += 4) {
-        float2 vv[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            vv[j] = i + j < i_end ? bf2_to_f2(__ldg(reinterpret_cast<const uint32_t*>(vc + (size_t)(s0 + i + j) * D) + dp))
-                                  : make_float2(0.f, 0.f);
-#pragma unroll
-        for (int h = 0; h < HM; ++h) {
-            if (h < H) {
-                const float4 p4 = *reinterpret_cast<const float4*>(&ps[h][i]);   // past cnt: 0 or unused
-                float2 t = o[h];
-                t = __ffma2_rn(make_float2(p4.x, p4.x), vv[0], t);
-                t = __ffma2_rn(make_float2(p4.y, p4.y), vv[1], t);
-                t = __ffma2_rn(make_float2(p4.z, p4.z), vv[2], t);
-                t = __ffma2_rn(make_float2(p4.w, p4.w), vv[3], t);
-                o[h] = t;
-            }
-        }
-    }
-    __syncthreads();                                     // the scores are read: reuse qs for the halves
-    float2* red = reinterpret_cast<float2*>(&qs[0][0]);  // [H][D / 2]
-    if (kh == 1) {
-#pragma unroll
-        for (int h = 0; h < HM; ++h)
-            if (h < H) red[h * (D / 2) + dp] = o[h];
-    }
-    __syncthreads();
     const size_t pb = ((size_t)b * a.nsplit + sp) * H;
-    if (kh == 0) {
-#pragma unroll
-        for (int h = 0; h < HM; ++h)
-            if (h < H) {
-                const float2 r = red[h * (D / 2) + dp];
-                reinterpret_cast<float2*>(a.part_o + (pb + h) * D)[dp] = make_float2(o[h].x + r.x, o[h].y + r.y);
-            }
+    if (cnt == 0) {                                      // a split past the window: an empty part
+        for (int e = threadIdx.x; e < H * D; e += blockDim.x) a.part_o[pb * D + e] = 0.f;
+        if (threadIdx.x < H) {
+            a.part_m[pb + threadIdx.x] = -INFINITY;
+            a.part_l[pb + threadIdx.x] = 0.f;
+        }
+        return;
     }
-    if (tid < H) {
-        a.part_m[pb + tid] = mh[tid];
-        a.part_l[pb + tid] = lh[tid];
+    if (threadIdx.x == 0) {
+        mbar_init(bars.kq_full(), 1);
+        mbar_init(bars.s_full(), 1);
+        mbar_init(bars.v_full(), 1);
+        mbar_init(bars.p_full(), 4);
+        mbar_init(bars.o_full(), 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_u32((const void*)tmem_base_s), D_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_s;
+    const int krow = b * 2 * a.w + s0, vrow = krow + a.w;   // the split's first key / value row
+
+    if (warp == 4) {
+        // ============================ TMA: keys and queries, then values ========================
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bars.kq_full(), KV_BYTES + QD_BYTES);
+            for (int kb = 0; kb < D / 64; ++kb) {
+                tma_load_2d(sbase + D_OFF_KV + kb * (kDecPer * 128), &map_kv, kb * 64, krow, bars.kq_full());
+                tma_load_2d(sbase + D_OFF_Q + kb * (kMaxH * 128), &map_q, kb * 64, b * H, bars.kq_full());
+            }
+            const uint64_t t0 = globaltimer_ns();
+            bool ok = dwait(bars.s_full(), 0, a, abort, 1);      // the keys have been read
+            if (ok) {
+                mbar_arrive_expect_tx(bars.v_full(), KV_BYTES);
+                for (int kb = 0; kb < D / 64; ++kb)
+                    tma_load_2d(sbase + D_OFF_KV + kb * (kDecPer * 128), &map_kv, kb * 64, vrow, bars.v_full());
+            }
+            // no bulk copy may still be writing shared memory at the exit
+            while (!mbar_try_wait(bars.kq_full(), 0) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+            while (ok && !mbar_try_wait(bars.v_full(), 0) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+        }
+    } else if (warp == 5) {
+        // ============================ MMA: S^T = K Q^T, then O^T = V^T P^T ======================
+        const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+        auto wait_w = [&](uint32_t bar, uint32_t par, unsigned where) {
+            return __all_sync(0xffffffffu, dwait(bar, par, a, abort, where));
+        };
+        if (wait_w(bars.kq_full(), 0, 2)) {
+            tc_fence_after();
+            if (elect_one()) {
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t ad = desc_k_sw128(sbase + D_OFF_KV + (ks >> 2) * (kDecPer * 128) + (ks & 3) * 32);
+                    const uint64_t bd = desc_k_sw128(sbase + D_OFF_Q + (ks >> 2) * (kMaxH * 128) + (ks & 3) * 32);
+                    mma_ss(tm + D_TM_S, ad, bd, idesc_dec(0), ks > 0 ? 1u : 0u);
+                }
+                mma_commit(bars.s_full());
+            }
+            __syncwarp();
+            if (wait_w(bars.p_full(), 0, 3) && wait_w(bars.v_full(), 0, 4)) {
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)             // d-columns [128 hh, 128 hh + 128)
+#pragma unroll
+                        for (int kk = 0; kk < kDecPer / 16; ++kk) {
+                            const uint64_t ad = desc_vt(sbase + D_OFF_KV + (2 * hh) * (kDecPer * 128) + kk * 2048);
+                            const uint64_t bd = desc_k_sw128(sbase + D_OFF_P + (kk >> 2) * (kMaxH * 128) + (kk & 3) * 32);
+                            mma_ss(tm + D_TM_O + hh * kMaxH, ad, bd, idesc_dec(1), kk > 0 ? 1u : 0u);
+                        }
+                    mma_commit(bars.o_full());
+                }
+                __syncwarp();
+            } else if (elect_one()) {
+                mma_commit(bars.o_full());                   // the epilogue drains on a failed wait
+            }
+            __syncwarp();
+        } else if (elect_one()) {
+            mma_commit(bars.s_full());
+            mma_commit(bars.o_full());
+        }
+        __syncwarp();
+        // every MMA issued here has completed before TMEM is released
+        if (lane == 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(bars.o_full(), 0) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+        }
+        __syncwarp();
+    } else {
+        // ============================ softmax of the split, then the output ====================
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int i = warp * 32 + lane;                  // slot within the split (TMEM lane)
+        const bool valid = i < cnt;
+        const float sc = a.scale * 1.4426950408889634f;
+        const bool ok_s = __all_sync(0xffffffffu, dwait(bars.s_full(), 0, a, abort, 5));
+        float s[kMaxH];
+        tc_fence_after();
+        tmem_ld16(tmem + lane_off + D_TM_S, s);
+        tmem_wait_ld();
+        // per head: the split's maximum (in units of log2), across the lanes, then the warps
+#pragma unroll
+        for (int h = 0; h < kMaxH; ++h) {
+            float v = valid && h < H ? s[h] * sc : -INFINITY;
+            s[h] = v;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (lane == 0) red[warp * kMaxH + h] = v;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        float m[kMaxH];
+#pragma unroll
+        for (int h = 0; h < kMaxH; ++h)
+            m[h] = fmaxf(fmaxf(red[h], red[kMaxH + h]), fmaxf(red[2 * kMaxH + h], red[3 * kMaxH + h]));
+        // p = 2^(s - m) (0 past the window and for padded heads), in bf16 as the B operand
+        // [16 heads x 128 slots]: row h, slot i at K block i / 64, 16-byte chunk (i % 64) / 8
+        const uint32_t pcol = (uint32_t)(i >> 6) * (kMaxH * 128) + (uint32_t)(i & 7) * 2;
+        const uint32_t pch = (uint32_t)((i & 63) >> 3);
+#pragma unroll
+        for (int h = 0; h < kMaxH; ++h) {
+            const float p = s[h] == -INFINITY ? 0.f : exp2f(s[h] - m[h]);
+            const __nv_bfloat16 pb16 = __float2bfloat16_rn(p);
+            *reinterpret_cast<__nv_bfloat16*>(smem + D_OFF_P + pcol + (uint32_t)h * 128 + ((pch ^ (uint32_t)(h & 7)) << 4)) = pb16;
+            float v = p;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) red[4 * kMaxH + warp * kMaxH + h] = v;
+        }
+        // value rows of slots past the window: zero (the MMA multiplies them by p = 0)
+        const bool ok_v = __all_sync(0xffffffffu, ok_s && dwait(bars.v_full(), 0, a, abort, 6));
+        if (ok_v && !valid) {
+#pragma unroll
+            for (int kb = 0; kb < D / 64; ++kb)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(smem + D_OFF_KV + kb * (kDecPer * 128) + i * 128 + c * 16) =
+                        make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (lane == 0) mbar_arrive(bars.p_full());
+        if (threadIdx.x < H) {
+            const int h = threadIdx.x;
+            const float mh = fmaxf(fmaxf(red[h], red[kMaxH + h]), fmaxf(red[2 * kMaxH + h], red[3 * kMaxH + h]));
+            const float lh = red[4 * kMaxH + h] + red[5 * kMaxH + h] + red[6 * kMaxH + h] + red[7 * kMaxH + h];
+            a.part_m[pb + h] = mh == -INFINITY ? -INFINITY : mh * 0.69314718055994531f;   // natural units
+            a.part_l[pb + h] = lh;
+        }
+        // O^T: lanes = d-columns (two halves), columns = heads
+        const bool ok_o = __all_sync(0xffffffffu, dwait(bars.o_full(), 0, a, abort, 7));
+        float o0[kMaxH], o1[kMaxH];
+        tc_fence_after();
+        tmem_ld16(tmem + lane_off + D_TM_O, o0);
+        tmem_ld16(tmem + lane_off + D_TM_O + kMaxH, o1);
+        tmem_wait_ld();
+        if (ok_o && ok_v) {
+            const int dcol = warp * 32 + lane;
+#pragma unroll
+            for (int h = 0; h < kMaxH; ++h)
+                if (h < H) {
+                    a.part_o[(pb + h) * D + dcol] = o0[h];
+                    a.part_o[(pb + h) * D + 128 + dcol] = o1[h];
+                }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, D_TMEM_COLS);
     }
 }
 
@@ -737,16 +864,25 @@ cudaError_t launch_mqa_decode(const rglru_mqa_dims* d, const void* q, const void
     ra.q_rot = reinterpret_cast<__nv_bfloat16*>(w + l.q_rot);
     ra.cache = static_cast<__nv_bfloat16*>(cache);
     mqa_rope_decode_kernel<<<B, D / 2, 0, s>>>(ra);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // the rotated queries as a 2-D [B H rows][d] tensor (box 64 x 16 rows: a row's heads, padded
+    // with the next row's or with zeros), the ring as 2-D [B 2 w rows][d] (box 64 x 128 slots)
+    CUtensorMap mqm, mkv;
+    if (!tc::make_map_2d_sw128(&mqm, ra.q_rot, D, (uint64_t)B * H, D * 2, 64, kMaxH) ||
+        !tc::make_map_2d_sw128(&mkv, ra.cache, D, (uint64_t)B * 2 * d->window, D * 2, 64, kDecPer))
+        return cudaErrorInvalidValue;
+    e = set_smem_once(mqa_decode_kernel, (int)D_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     DecArgs da{};
     da.B = B; da.H = H; da.w = d->window; da.nsplit = l.nsplit; da.scale = d->scale;
-    da.q_rot = ra.q_rot; da.pos = pos; da.cache = ra.cache;
+    da.pos = pos; da.cache = ra.cache;
     da.part_m = reinterpret_cast<float*>(w + l.part_m);
     da.part_l = reinterpret_cast<float*>(w + l.part_l);
     da.part_o = reinterpret_cast<float*>(w + l.part_o);
-    const dim3 grid(l.nsplit, B);
-    if (H <= 4) mqa_decode_kernel<4><<<grid, kDecThreads, 0, s>>>(da);
-    else if (H <= 8) mqa_decode_kernel<8><<<grid, kDecThreads, 0, s>>>(da);
-    else mqa_decode_kernel<16><<<grid, kDecThreads, 0, s>>>(da);
+    da.status = reinterpret_cast<DeviceStatus*>(w);
+    da.timeout_ns = 1000000000ull;
+    mqa_decode_kernel<<<dim3(l.nsplit, B), kDecThreads, D_SMEM_BYTES, s>>>(mqm, mkv, da);
     MergeArgs ma{};
     ma.B = B; ma.H = H; ma.nsplit = l.nsplit;
     ma.part_m = da.part_m; ma.part_l = da.part_l; ma.part_o = da.part_o;

@@ -58,6 +58,7 @@ def test_mqa_prefill_matches_oracle(B, T, H, w):
     (150, 4, 64, 40),      # a full ring that wraps many times
     (300, 10, 600, 6),     # a ring not yet full, window cut into splits (one of them empty)
     (700, 3, 600, 4),      # a full ring of several splits, the last one ragged
+    (5, 16, 300, 3),       # a nearly empty ring (two empty splits), all 16 heads of the MMA's N
 ])
 def test_mqa_decode_continues_the_prefill_through_the_ring(T0, H, w, steps):
     """Prefill T0 tokens with the cache, then decode steps; each step against the oracle's
