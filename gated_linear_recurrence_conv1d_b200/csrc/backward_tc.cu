@@ -51,6 +51,11 @@ constexpr int kTB = 64;          // tokens per conv-transpose block
 constexpr int kMaxSplits = 16;   // K slices of the weight-gradient GEMMs, at most
 constexpr int kScanThreads = 128;
 constexpr int kChunk = 64;       // tokens per chunk of the reverse scan
+// Resident blocks per SM asked of the three streaming kernels (their register caps) and the
+// conv transpose's prefetch depth, set by measurement on B200 (rg2b_bf16): more resident warps
+// hide the scans' load latency better than deeper per-thread batches.
+constexpr int kAggMinBlocks = 12, kOutMinBlocks = 12, kConvTMinBlocks = 6;
+constexpr int kPFC = 8;          // positions a conv-transpose batch loads ahead
 
 struct Layout {
     size_t ga, gx, hprev, dxc, xc_hi, xc_lo, dga_hi, dga_lo, dgx_hi, dgx_lo;
@@ -154,7 +159,7 @@ struct ScanArgs {
 // ---------------------------------------------------------------- 2. the reverse scan -------
 // Thread = (row b, chunk k, channel ch); the inputs of a block of kPF tokens are loaded together
 // before the block is walked, so that their latencies overlap.
-constexpr int kPF = 8;
+constexpr int kPF = 4;
 
 // a'_t: the factor that carries g from token t to t - 1 (a_t, or 0 where t starts a segment)
 __device__ __forceinline__ float carry_factor(float kappa, float ga, bool rs) {
@@ -168,7 +173,7 @@ __device__ __forceinline__ float2 bf2f(const __nv_bfloat16* p) {
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
 }
 
-__global__ void __launch_bounds__(kScanThreads) bwd_scan_agg_kernel(ScanArgs a) {
+__global__ void __launch_bounds__(kScanThreads, kAggMinBlocks) bwd_scan_agg_kernel(ScanArgs a) {
     const int ch = 2 * (blockIdx.x * kScanThreads + threadIdx.x), k = blockIdx.y, b = blockIdx.z;
     if (ch >= a.W) return;
     const float kap0 = a.c * log_sigmoid_acc(a.lambda[ch]), kap1 = a.c * log_sigmoid_acc(a.lambda[ch + 1]);
@@ -237,7 +242,7 @@ __global__ void __launch_bounds__(kScanThreads) bwd_scan_carry_kernel(ScanArgs a
 
 // every output of a chunk, from the carry into its last token; thread = (row b, chunk k, channel
 // pair ch, ch + 1), kPF2 tokens a batch
-constexpr int kPF2 = 4;
+constexpr int kPF2 = 1;
 
 struct ScanOut1 {             // the results of one token-channel
     float dy, dxc, dga, dgx, q;
@@ -272,7 +277,7 @@ __device__ __forceinline__ void split_bf16x2(float v0, float v1, uint32_t& hi, u
     lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
-__global__ void __launch_bounds__(kScanThreads) bwd_scan_out_kernel(ScanArgs a) {
+__global__ void __launch_bounds__(kScanThreads, kOutMinBlocks) bwd_scan_out_kernel(ScanArgs a) {
     const int ch = 2 * (blockIdx.x * kScanThreads + threadIdx.x), k = blockIdx.y, b = blockIdx.z;
     if (ch >= a.W) return;
     const float kap0 = a.c * log_sigmoid_acc(a.lambda[ch]), kap1 = a.c * log_sigmoid_acc(a.lambda[ch + 1]);
@@ -362,7 +367,8 @@ __device__ __forceinline__ bool window_reads(const uint8_t* rrow, int s, int t) 
 // the last segment start at or before the current token.  Every value is a channel pair.
 __device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
-__global__ void __launch_bounds__(128) bwd_convT_kernel(ConvTArgs a) {
+
+__global__ void __launch_bounds__(128, kConvTMinBlocks) bwd_convT_kernel(ConvTArgs a) {
     const int ch = 2 * (blockIdx.x * 128 + threadIdx.x), tb = blockIdx.y, b = blockIdx.z;
     if (ch >= a.W) return;
     const int T = a.T;
@@ -394,19 +400,19 @@ __global__ void __launch_bounds__(128) bwd_convT_kernel(ConvTArgs a) {
     const int sb = tb == 0 ? -kHist : t0;                   // the first block also owns the history
     float2 d0 = dxcv(sb), d1 = dxcv(sb + 1), d2 = dxcv(sb + 2);
     bool q0 = rs(sb), q1 = rs(sb + 1), q2 = rs(sb + 2);
-    // positions in batches of kPF: the batch's loads are issued together, ahead of its arithmetic
-    for (int s0 = sb; s0 < t1; s0 += kPF) {
-        float2 dn[kPF], xn[kPF];
-        bool qn[kPF];
+    // positions in batches of kPFC: the batch's loads are issued together, ahead of its arithmetic
+    for (int s0 = sb; s0 < t1; s0 += kPFC) {
+        float2 dn[kPFC], xn[kPFC];
+        bool qn[kPFC];
 #pragma unroll
-        for (int j = 0; j < kPF; ++j) {
+        for (int j = 0; j < kPFC; ++j) {
             const int s = s0 + j;
             dn[j] = dxcv(s + 3);
             qn[j] = rs(s + 3);
             xn[j] = s >= t0 && s < t1 ? __bfloat1622float2(xr[s * W2]) : z2;
         }
 #pragma unroll
-        for (int j = 0; j < kPF; ++j) {
+        for (int j = 0; j < kPFC; ++j) {
             const int s = s0 + j;
             if (s >= t1) break;
             const float2 d3 = dn[j];

@@ -16,10 +16,13 @@
 //     reference maximum that moves only when the maximum grows by more than 2^8 (then the
 //     accumulator is rescaled), write P in bf16 to shared memory; O += P V (M = 128, N = 256,
 //     K = 64) accumulates in TMEM; the S of the next tile overlaps the softmax of this one;
-//   * mqa_decode_kernel: one token per row against the ring: CTAs split the ring's slots into
-//     parts of 128; per part S^T = K Q^T and O^T = V^T P^T run on the tensor cores (the H heads
-//     of a row form the MMA's N), the softmax of the part on 4 warps; each CTA leaves (max, sum,
-//     sum of p v) per head, and mqa_merge_kernel combines the parts.
+//   * mqa_decode_kernel: one token per row against the ring, persistent: the ring's slots are cut
+//     into tiles of 128 and a row's tiles into parts; per tile S^T = K Q^T and O^T = V^T P^T run
+//     on the tensor cores (the H heads of a row form the MMA's N) while the next tiles stream in
+//     by TMA, the softmax on 4 warps; each part leaves (max, sum, sum of p v) per head, and
+//     mqa_merge_kernel combines the parts.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -476,38 +479,45 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 // ---------------------------------------------------------------- decode ---------------------
 // One token per row against its ring.  The window is a set: softmax over it does not depend on
 // the order of its keys, and the ring holds exactly the window -- slots [0, n), n = min(pos + 1,
-// w) (slot = position mod w, keys cached after their rotation) -- so a CTA takes a split of
-// kDecPer consecutive slots.  Per CTA, on the tensor cores:
-//   * TMA brings the split's keys [128 slots x 256 d] and the row's rotated queries [16 x 256]
-//     (heads past H read other data: their columns are never used) in the 128-byte swizzle;
-//   * S^T = K Q^T (M = 128 slots, N = 16 heads, K = 256): a TMEM lane is a slot;
-//   * meanwhile the values come into the keys' place once the MMAs have read them;
-//   * 4 warps (thread = slot) mask the slots past n, take per head the split's maximum and sum
-//     (shuffles, then across the warps) and write p = exp(s - m) in bf16 as the B operand of
-//     O^T = V^T P^T (M = 128 d-columns x 2, N = 16, K = 128 slots; V^T is the value tile read
-//     MN-major); value rows past n are zeroed first (an unfilled slot may hold anything);
-//   * the same warps read O^T (thread = d-column) and write (m, l, o) per head for the merge.
+// w) (slot = position mod w, keys cached after their rotation) -- so the slots are cut into
+// tiles of 128 and the tiles of a row into parts ("items") of up to kTilesMax consecutive tiles.
+// A persistent CTA takes items blockIdx.x, + gridDim.x, ... and streams their tiles:
+//   * a TMA warp brings each tile's keys [128 slots x 256 d], then its values, into a ring of
+//     three 64 KB buffers (the row's rotated queries [16 x 256] come with an item's first keys;
+//     heads past H read other data, whose columns are never used), 128-byte swizzle;
+//   * an MMA warp issues S^T = K Q^T (M = 128 slots, N = 16 heads, K = 256: a TMEM lane is a
+//     slot) for tile i, then O^T = V^T P^T (M = 128 d-columns x 2, N = 16, K = 128 slots; V^T is
+//     the value tile read MN-major) for tile i - 1, so that the scores of the next tile overlap
+//     the softmax of this one; S and O^T are double-buffered in TMEM, P in shared memory;
+//   * 4 warps (thread = slot) mask the slots past n, take per head the tile's maximum and sum
+//     (shuffles, then across the warps), write p = 2^(s - m) in bf16 as the B operand of the
+//     value MMA (value rows past n are zeroed first: an unfilled slot may hold anything), then
+//     read tile i - 1's O^T (thread = d-column) and fold it into the item's running (max, sum,
+//     sum of p v) per head; an item's last tile writes them for the merge.
 // The step reads the ring once (2 w d bf16 per row): it is bound by HBM.
-constexpr int kDecPer = 128;           // slots per split (the MMA's M)
+constexpr int kTile = 128;             // slots per tile (the MMA's M)
 constexpr int kMaxH = 16;              // heads (the MMA's N), padded
-constexpr uint32_t KV_BYTES = kDecPer * D * 2;        // 65536: 4 boxes of [128 slots x 64 d]
+constexpr int kTilesMax = 4;           // tiles per item, at most
+constexpr int kNBuf = 3;               // 64 KB tile buffers
+constexpr uint32_t KV_BYTES = kTile * D * 2;          // 65536: 4 boxes of [128 slots x 64 d]
 constexpr uint32_t QD_BYTES = kMaxH * D * 2;          // 8192: 4 boxes of [16 heads x 64 d]
-constexpr uint32_t PD_BYTES = kMaxH * kDecPer * 2;    // 4096: 2 K blocks of [16 heads x 64 slots]
+constexpr uint32_t PD_BYTES = kMaxH * kTile * 2;      // 4096: 2 K blocks of [16 heads x 64 slots]
 constexpr uint32_t D_OFF_KV = 0;
-constexpr uint32_t D_OFF_Q = D_OFF_KV + KV_BYTES;
-constexpr uint32_t D_OFF_P = D_OFF_Q + QD_BYTES;
-constexpr uint32_t D_OFF_RED = D_OFF_P + PD_BYTES;   // [2][4 warps][16] fp32: maxima, then sums
+constexpr uint32_t D_OFF_Q = D_OFF_KV + kNBuf * KV_BYTES;   // 2 buffers (item parity)
+constexpr uint32_t D_OFF_P = D_OFF_Q + 2 * QD_BYTES;        // 2 buffers (tile parity)
+constexpr uint32_t D_OFF_RED = D_OFF_P + 2 * PD_BYTES;      // [2][4 warps][16] fp32: maxima, sums
 constexpr uint32_t D_OFF_BAR = D_OFF_RED + 2 * 4 * kMaxH * 4;
-constexpr uint32_t D_SMEM_BYTES = D_OFF_BAR + 128 + 1024;
-constexpr uint32_t D_TM_S = 0, D_TM_O = 32, D_TMEM_COLS = 64;
+constexpr uint32_t D_SMEM_BYTES = D_OFF_BAR + 256 + 1024;
+static_assert(D_SMEM_BYTES <= 232448, "shared memory budget");
+// TMEM: S^T [0, 32) (two buffers of 16 columns), O^T [32, 96) (two buffers of 2 x 16)
+constexpr uint32_t D_TM_S = 0, D_TM_O = 32, D_TMEM_COLS = 128;
 constexpr int kDecThreads = 6 * 32;    // 4 softmax / epilogue warps, a TMA warp, an MMA warp
 
 struct DecArgs {
-    int B, H, w, nsplit;
+    int B, H, w, nsplit, tiles;        // nsplit items per row of `tiles` tiles (the last ragged)
     float scale;
     const int* pos;                    // [B]
-    const __nv_bfloat16* cache;        // [B][2][w][d]
-    float* part_m;                     // [B][nsplit][H]
+    float* part_m;                     // [B][nsplit][H], natural-log units
     float* part_l;
     float* part_o;                     // [B][nsplit][H][d]
     DeviceStatus* status;
@@ -516,12 +526,29 @@ struct DecArgs {
 
 struct DBars {
     uint32_t base;
-    __device__ __forceinline__ uint32_t kq_full() const { return base; }
-    __device__ __forceinline__ uint32_t s_full() const { return base + 8; }     // S^T done: keys read
-    __device__ __forceinline__ uint32_t v_full() const { return base + 16; }
-    __device__ __forceinline__ uint32_t p_full() const { return base + 24; }    // P written, V rows zeroed
-    __device__ __forceinline__ uint32_t o_full() const { return base + 32; }
+    __device__ __forceinline__ uint32_t kv_full(int i) const { return base + 8u * i; }
+    __device__ __forceinline__ uint32_t kv_empty(int i) const { return base + 24u + 8u * i; }
+    __device__ __forceinline__ uint32_t s_full(int i) const { return base + 48u + 8u * i; }
+    __device__ __forceinline__ uint32_t p_full(int i) const { return base + 64u + 8u * i; }   // P written, V rows zeroed
+    __device__ __forceinline__ uint32_t o_full(int i) const { return base + 80u + 8u * i; }
+    __device__ __forceinline__ uint32_t o_empty(int i) const { return base + 96u + 8u * i; }  // O^T read
+    __device__ __forceinline__ uint32_t mma_done() const { return base + 112u; }
 };
+
+// An item of the stream: row b, its tiles [t0, t0 + nt) (slot 128 t0 first), cnt valid slots.
+struct DecItem {
+    int b, sp, s0, cnt, nt;
+};
+__device__ __forceinline__ DecItem dec_item(const DecArgs& a, int j) {
+    DecItem it;
+    it.b = j / a.nsplit;
+    it.sp = j % a.nsplit;
+    it.s0 = it.sp * a.tiles * kTile;
+    const int n = min(a.pos[it.b] + 1, a.w);
+    it.cnt = max(0, min(n, it.s0 + a.tiles * kTile) - it.s0);
+    it.nt = (it.cnt + kTile - 1) / kTile;
+    return it;
+}
 
 __device__ __noinline__ bool dwait_slow(uint32_t bar, uint32_t parity, const DecArgs& a, volatile int* abort,
                                         unsigned where) {
@@ -546,6 +573,20 @@ __device__ __forceinline__ bool dwait(uint32_t bar, uint32_t parity, const DecAr
     return dwait_slow(bar, parity, a, abort, where);
 }
 
+// Named barrier 1 over the 4 softmax warps, returning the AND of v over their threads.
+__device__ __forceinline__ bool bar_and_128(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "barrier.red.and.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v)
+        : "memory");
+    return r != 0;
+}
+
 // MN-major (128-byte swizzle) descriptor of the value tile read as V^T: atoms of 64 d-columns,
 // each [128 slots x 128 B], 16384 B apart
 __device__ __forceinline__ uint64_t desc_vt(uint32_t smem_addr) {
@@ -560,38 +601,33 @@ __device__ __forceinline__ uint64_t desc_vt(uint32_t smem_addr) {
 // fp32 accumulator, bf16 operands, A K-major (a_mn = 0) or MN-major (1), B K-major, M 128, N 16
 __device__ __forceinline__ uint32_t idesc_dec(int a_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)(kMaxH >> 3) << 17) |
-           ((uint32_t)(kDecPer >> 4) << 24);
+           ((uint32_t)(kTile >> 4) << 24);
 }
 
-__global__ void __launch_bounds__(kDecThreads, 2)
+__global__ void __launch_bounds__(kDecThreads, 1)
 mqa_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kv,
                   const DecArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const DBars bars{sbase + D_OFF_BAR};
-    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + D_OFF_BAR + 64);
-    volatile int* abort = reinterpret_cast<volatile int*>(smem + D_OFF_BAR + 80);
+    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + D_OFF_BAR + 128);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + D_OFF_BAR + 144);
     float* red = reinterpret_cast<float*>(smem + D_OFF_RED);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int sp = blockIdx.x, b = blockIdx.y, H = a.H;
-    const int n = min(a.pos[b] + 1, a.w);                // slots in the window
-    const int s0 = sp * kDecPer, cnt = max(0, min(n, s0 + kDecPer) - s0);
-    const size_t pb = ((size_t)b * a.nsplit + sp) * H;
-    if (cnt == 0) {                                      // a split past the window: an empty part
-        for (int e = threadIdx.x; e < H * D; e += blockDim.x) a.part_o[pb * D + e] = 0.f;
-        if (threadIdx.x < H) {
-            a.part_m[pb + threadIdx.x] = -INFINITY;
-            a.part_l[pb + threadIdx.x] = 0.f;
-        }
-        return;
-    }
+    const int H = a.H, nitems = a.B * a.nsplit;
     if (threadIdx.x == 0) {
-        mbar_init(bars.kq_full(), 1);
-        mbar_init(bars.s_full(), 1);
-        mbar_init(bars.v_full(), 1);
-        mbar_init(bars.p_full(), 4);
-        mbar_init(bars.o_full(), 1);
+        for (int i = 0; i < kNBuf; ++i) {
+            mbar_init(bars.kv_full(i), 1);
+            mbar_init(bars.kv_empty(i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bars.s_full(i), 1);
+            mbar_init(bars.p_full(i), 4);
+            mbar_init(bars.o_full(i), 1);
+            mbar_init(bars.o_empty(i), 4);
+        }
+        mbar_init(bars.mma_done(), 1);
         *abort = 0;
         fence_barrier_init();
     }
@@ -603,152 +639,263 @@ mqa_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_s;
-    const int krow = b * 2 * a.w + s0, vrow = krow + a.w;   // the split's first key / value row
 
     if (warp == 4) {
-        // ============================ TMA: keys and queries, then values ========================
+        // ============================ TMA: per tile its keys, then its values =================
         if (lane == 0) {
-            mbar_arrive_expect_tx(bars.kq_full(), KV_BYTES + QD_BYTES);
-            for (int kb = 0; kb < D / 64; ++kb) {
-                tma_load_2d(sbase + D_OFF_KV + kb * (kDecPer * 128), &map_kv, kb * 64, krow, bars.kq_full());
-                tma_load_2d(sbase + D_OFF_Q + kb * (kMaxH * 128), &map_q, kb * 64, b * H, bars.kq_full());
+            uint32_t L = 0;                                   // loads issued
+            bool ok = true;
+            for (int j = blockIdx.x; ok && j < nitems; j += gridDim.x) {
+                const DecItem it = dec_item(a, j);
+                const int krow0 = it.b * 2 * a.w + it.s0;
+                const int jl = (j - (int)blockIdx.x) / (int)gridDim.x;   // item number within this CTA
+                for (int ti = 0; ok && ti < it.nt; ++ti) {
+                    for (int kv = 0; ok && kv < 2; ++kv, ++L) {
+                        const int buf = (int)(L % kNBuf);
+                        const uint32_t use = L / kNBuf;
+                        if (use > 0 && !(ok = dwait(bars.kv_empty(buf), (use - 1) & 1, a, abort, 1))) break;
+                        const bool q = kv == 0 && ti == 0;
+                        mbar_arrive_expect_tx(bars.kv_full(buf), KV_BYTES + (q ? QD_BYTES : 0u));
+                        const int row = krow0 + ti * kTile + (kv ? a.w : 0);
+                        for (int kb = 0; kb < D / 64; ++kb)
+                            tma_load_2d(sbase + D_OFF_KV + buf * KV_BYTES + kb * (kTile * 128), &map_kv, kb * 64, row,
+                                        bars.kv_full(buf));
+                        if (q)
+                            for (int kb = 0; kb < D / 64; ++kb)
+                                tma_load_2d(sbase + D_OFF_Q + (jl & 1) * QD_BYTES + kb * (kMaxH * 128), &map_q, kb * 64,
+                                            it.b * H, bars.kv_full(buf));
+                    }
+                }
             }
+            // no bulk copy may still be writing shared memory at the exit: the last loads
+            // (up to kNBuf of them) have landed
             const uint64_t t0 = globaltimer_ns();
-            bool ok = dwait(bars.s_full(), 0, a, abort, 1);      // the keys have been read
-            if (ok) {
-                mbar_arrive_expect_tx(bars.v_full(), KV_BYTES);
-                for (int kb = 0; kb < D / 64; ++kb)
-                    tma_load_2d(sbase + D_OFF_KV + kb * (kDecPer * 128), &map_kv, kb * 64, vrow, bars.v_full());
-            }
-            // no bulk copy may still be writing shared memory at the exit
-            while (!mbar_try_wait(bars.kq_full(), 0) && globaltimer_ns() - t0 < a.timeout_ns) {
-            }
-            while (ok && !mbar_try_wait(bars.v_full(), 0) && globaltimer_ns() - t0 < a.timeout_ns) {
-            }
+            for (uint32_t l = L > kNBuf ? L - kNBuf : 0; l < L; ++l)
+                while (!mbar_try_wait(bars.kv_full(l % kNBuf), (l / kNBuf) & 1) &&
+                       globaltimer_ns() - t0 < a.timeout_ns) {
+                }
         }
     } else if (warp == 5) {
-        // ============================ MMA: S^T = K Q^T, then O^T = V^T P^T ======================
+        // ============================ MMA: S^T of tile i, then O^T of tile i - 1 ==============
         const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
         auto wait_w = [&](uint32_t bar, uint32_t par, unsigned where) {
             return __all_sync(0xffffffffu, dwait(bar, par, a, abort, where));
         };
-        if (wait_w(bars.kq_full(), 0, 2)) {
+        bool ok = true;
+        uint32_t i = 0;                                       // tiles whose S^T is issued
+        auto issue_pv = [&](uint32_t t) -> bool {             // O^T of tile t (V: load 2 t + 1)
+            const uint32_t lv = 2 * t + 1, buf = lv % kNBuf;
+            if (!wait_w(bars.p_full(t & 1), (t >> 1) & 1, 3)) return false;
+            if (!wait_w(bars.kv_full(buf), (lv / kNBuf) & 1, 4)) return false;
+            if (t >= 2 && !wait_w(bars.o_empty(t & 1), ((t >> 1) - 1) & 1, 5)) return false;
             tc_fence_after();
             if (elect_one()) {
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t ad = desc_k_sw128(sbase + D_OFF_KV + (ks >> 2) * (kDecPer * 128) + (ks & 3) * 32);
-                    const uint64_t bd = desc_k_sw128(sbase + D_OFF_Q + (ks >> 2) * (kMaxH * 128) + (ks & 3) * 32);
-                    mma_ss(tm + D_TM_S, ad, bd, idesc_dec(0), ks > 0 ? 1u : 0u);
-                }
-                mma_commit(bars.s_full());
+                for (int hh = 0; hh < 2; ++hh)                 // d-columns [128 hh, 128 hh + 128)
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk) {
+                        const uint64_t ad = desc_vt(sbase + D_OFF_KV + buf * KV_BYTES + (2 * hh) * (kTile * 128) + kk * 2048);
+                        const uint64_t bd = desc_k_sw128(sbase + D_OFF_P + (t & 1) * PD_BYTES + (kk >> 2) * (kMaxH * 128) +
+                                                         (kk & 3) * 32);
+                        mma_ss(tm + D_TM_O + (t & 1) * 32 + hh * kMaxH, ad, bd, idesc_dec(1), kk > 0 ? 1u : 0u);
+                    }
+                mma_commit(bars.o_full(t & 1));
+                mma_commit(bars.kv_empty(buf));
             }
             __syncwarp();
-            if (wait_w(bars.p_full(), 0, 3) && wait_w(bars.v_full(), 0, 4)) {
+            return true;
+        };
+        for (int j = blockIdx.x; ok && j < nitems; j += gridDim.x) {
+            const DecItem it = dec_item(a, j);
+            const int jl = (j - (int)blockIdx.x) / (int)gridDim.x;
+            for (int ti = 0; ok && ti < it.nt; ++ti, ++i) {
+                const uint32_t lk = 2 * i, buf = lk % kNBuf;
+                if (!(ok = wait_w(bars.kv_full(buf), (lk / kNBuf) & 1, 2))) break;
                 tc_fence_after();
                 if (elect_one()) {
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)             // d-columns [128 hh, 128 hh + 128)
-#pragma unroll
-                        for (int kk = 0; kk < kDecPer / 16; ++kk) {
-                            const uint64_t ad = desc_vt(sbase + D_OFF_KV + (2 * hh) * (kDecPer * 128) + kk * 2048);
-                            const uint64_t bd = desc_k_sw128(sbase + D_OFF_P + (kk >> 2) * (kMaxH * 128) + (kk & 3) * 32);
-                            mma_ss(tm + D_TM_O + hh * kMaxH, ad, bd, idesc_dec(1), kk > 0 ? 1u : 0u);
-                        }
-                    mma_commit(bars.o_full());
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint64_t ad = desc_k_sw128(sbase + D_OFF_KV + buf * KV_BYTES + (ks >> 2) * (kTile * 128) + (ks & 3) * 32);
+                        const uint64_t bd = desc_k_sw128(sbase + D_OFF_Q + (jl & 1) * QD_BYTES + (ks >> 2) * (kMaxH * 128) +
+                                                         (ks & 3) * 32);
+                        mma_ss(tm + D_TM_S + (i & 1) * kMaxH, ad, bd, idesc_dec(0), ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bars.s_full(i & 1));
+                    mma_commit(bars.kv_empty(buf));
                 }
                 __syncwarp();
-            } else if (elect_one()) {
-                mma_commit(bars.o_full());                   // the epilogue drains on a failed wait
+                if (i > 0) ok = issue_pv(i - 1);
             }
-            __syncwarp();
-        } else if (elect_one()) {
-            mma_commit(bars.s_full());
-            mma_commit(bars.o_full());
         }
+        if (ok && i > 0) ok = issue_pv(i - 1);
+        // every MMA issued here has completed before TMEM is released (also after a failed wait)
+        if (elect_one()) mma_commit(bars.mma_done());
         __syncwarp();
-        // every MMA issued here has completed before TMEM is released
         if (lane == 0) {
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(bars.o_full(), 0) && globaltimer_ns() - t0 < a.timeout_ns) {
+            while (!mbar_try_wait(bars.mma_done(), 0) && globaltimer_ns() - t0 < a.timeout_ns) {
             }
         }
         __syncwarp();
     } else {
-        // ============================ softmax of the split, then the output ====================
+        // ============================ softmax of tile i, then the output of tile i - 1 ========
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const int i = warp * 32 + lane;                  // slot within the split (TMEM lane)
-        const bool valid = i < cnt;
+        const int r = warp * 32 + lane;                  // slot within a tile (TMEM lane), then d-column
         const float sc = a.scale * 1.4426950408889634f;
-        const bool ok_s = __all_sync(0xffffffffu, dwait(bars.s_full(), 0, a, abort, 5));
-        float s[kMaxH];
-        tc_fence_after();
-        tmem_ld16(tmem + lane_off + D_TM_S, s);
-        tmem_wait_ld();
-        // per head: the split's maximum (in units of log2), across the lanes, then the warps
-#pragma unroll
-        for (int h = 0; h < kMaxH; ++h) {
-            float v = valid && h < H ? s[h] * sc : -INFINITY;
-            s[h] = v;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-            if (lane == 0) red[warp * kMaxH + h] = v;
+        // empty items (a part of the ring past the window): an empty part for the merge
+        for (int j = blockIdx.x; j < nitems; j += gridDim.x) {
+            const DecItem it = dec_item(a, j);
+            if (it.nt > 0) continue;
+            const size_t pb = ((size_t)it.b * a.nsplit + it.sp) * H;
+            for (int e = threadIdx.x; e < H * D; e += 128) a.part_o[pb * D + e] = 0.f;
+            if (threadIdx.x < H) {
+                a.part_m[pb + threadIdx.x] = -INFINITY;
+                a.part_l[pb + threadIdx.x] = 0.f;
+            }
         }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        float m[kMaxH];
+        float M[kMaxH], acc0[kMaxH], acc1[kMaxH], mt[kMaxH];   // item's running max, O; tile's max
+        float Lh = 0.f, lt = 0.f;                         // item's running sum, tile's (head r < H)
+        bool ok = true;
+        uint32_t i = 0;
+        int pend_b = -1, pend_sp = 0;                     // item of tile i - 1 and whether it ends it
+        bool pend_last = false, pend_first = false;
+        // fold tile t's O^T into the item's running values; write them at the item's end
+        auto epilogue = [&](uint32_t t) -> bool {
+            if (!__all_sync(0xffffffffu, dwait(bars.o_full(t & 1), (t >> 1) & 1, a, abort, 7))) return false;
+            tc_fence_after();
+            float o0[kMaxH], o1[kMaxH];
+            tmem_ld16(tmem + lane_off + D_TM_O + (t & 1) * 32, o0);
+            tmem_ld16(tmem + lane_off + D_TM_O + (t & 1) * 32 + kMaxH, o1);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.o_empty(t & 1));
+            if (pend_first) {
 #pragma unroll
-        for (int h = 0; h < kMaxH; ++h)
-            m[h] = fmaxf(fmaxf(red[h], red[kMaxH + h]), fmaxf(red[2 * kMaxH + h], red[3 * kMaxH + h]));
-        // p = 2^(s - m) (0 past the window and for padded heads), in bf16 as the B operand
-        // [16 heads x 128 slots]: row h, slot i at K block i / 64, 16-byte chunk (i % 64) / 8
-        const uint32_t pcol = (uint32_t)(i >> 6) * (kMaxH * 128) + (uint32_t)(i & 7) * 2;
-        const uint32_t pch = (uint32_t)((i & 63) >> 3);
-#pragma unroll
-        for (int h = 0; h < kMaxH; ++h) {
-            const float p = s[h] == -INFINITY ? 0.f : exp2f(s[h] - m[h]);
-            const __nv_bfloat16 pb16 = __float2bfloat16_rn(p);
-            *reinterpret_cast<__nv_bfloat16*>(smem + D_OFF_P + pcol + (uint32_t)h * 128 + ((pch ^ (uint32_t)(h & 7)) << 4)) = pb16;
-            float v = p;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) red[4 * kMaxH + warp * kMaxH + h] = v;
-        }
-        // value rows of slots past the window: zero (the MMA multiplies them by p = 0)
-        const bool ok_v = __all_sync(0xffffffffu, ok_s && dwait(bars.v_full(), 0, a, abort, 6));
-        if (ok_v && !valid) {
-#pragma unroll
-            for (int kb = 0; kb < D / 64; ++kb)
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4*>(smem + D_OFF_KV + kb * (kDecPer * 128) + i * 128 + c * 16) =
-                        make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (lane == 0) mbar_arrive(bars.p_full());
-        if (threadIdx.x < H) {
-            const int h = threadIdx.x;
-            const float mh = fmaxf(fmaxf(red[h], red[kMaxH + h]), fmaxf(red[2 * kMaxH + h], red[3 * kMaxH + h]));
-            const float lh = red[4 * kMaxH + h] + red[5 * kMaxH + h] + red[6 * kMaxH + h] + red[7 * kMaxH + h];
-            a.part_m[pb + h] = mh == -INFINITY ? -INFINITY : mh * 0.69314718055994531f;   // natural units
-            a.part_l[pb + h] = lh;
-        }
-        // O^T: lanes = d-columns (two halves), columns = heads
-        const bool ok_o = __all_sync(0xffffffffu, dwait(bars.o_full(), 0, a, abort, 7));
-        float o0[kMaxH], o1[kMaxH];
-        tc_fence_after();
-        tmem_ld16(tmem + lane_off + D_TM_O, o0);
-        tmem_ld16(tmem + lane_off + D_TM_O + kMaxH, o1);
-        tmem_wait_ld();
-        if (ok_o && ok_v) {
-            const int dcol = warp * 32 + lane;
-#pragma unroll
-            for (int h = 0; h < kMaxH; ++h)
-                if (h < H) {
-                    a.part_o[(pb + h) * D + dcol] = o0[h];
-                    a.part_o[(pb + h) * D + 128 + dcol] = o1[h];
+                for (int h = 0; h < kMaxH; ++h) {
+                    M[h] = mt[h];
+                    acc0[h] = o0[h];
+                    acc1[h] = o1[h];
                 }
+                Lh = lt;
+            } else {
+                float fo_l = 1.f, fn_l = 1.f;
+#pragma unroll
+                for (int h = 0; h < kMaxH; ++h) {
+                    const float mn = fmaxf(M[h], mt[h]);
+                    const float fo = mn == -INFINITY ? 0.f : exp2f(M[h] - mn);
+                    const float fn = mn == -INFINITY ? 0.f : exp2f(mt[h] - mn);
+                    acc0[h] = fmaf(acc0[h], fo, o0[h] * fn);
+                    acc1[h] = fmaf(acc1[h], fo, o1[h] * fn);
+                    M[h] = mn;
+                    if (h == r) {
+                        fo_l = fo;
+                        fn_l = fn;
+                    }
+                }
+                Lh = fmaf(Lh, fo_l, lt * fn_l);
+            }
+            if (pend_last) {
+                const size_t pb = ((size_t)pend_b * a.nsplit + pend_sp) * H;
+#pragma unroll
+                for (int h = 0; h < kMaxH; ++h)
+                    if (h < H) {
+                        a.part_o[(pb + h) * D + r] = acc0[h];
+                        a.part_o[(pb + h) * D + 128 + r] = acc1[h];
+                    }
+                if (r < H) {
+                    float mh = M[0];
+#pragma unroll
+                    for (int h = 1; h < kMaxH; ++h)
+                        if (h == r) mh = M[h];
+                    a.part_m[pb + r] = mh * 0.69314718055994531f;   // natural units
+                    a.part_l[pb + r] = Lh;
+                }
+            }
+            return true;
+        };
+        // The 4 warps meet at named barriers that also AND a flag across them, so that they leave
+        // the loop together when any wait failed (a warp that stayed would wait forever).
+        bool stop = false;                                // the same in all 4 warps
+        for (int j = blockIdx.x; !stop && j < nitems; j += gridDim.x) {
+            const DecItem it = dec_item(a, j);
+            for (int ti = 0; ti < it.nt; ++ti, ++i) {
+                const int cnt = min(kTile, it.cnt - ti * kTile);   // valid slots of the tile
+                const bool valid = r < cnt;
+                ok = ok && __all_sync(0xffffffffu, dwait(bars.s_full(i & 1), (i >> 1) & 1, a, abort, 6));
+                float s[kMaxH];
+                if (ok) {
+                    tc_fence_after();
+                    tmem_ld16(tmem + lane_off + D_TM_S + (i & 1) * kMaxH, s);
+                    tmem_wait_ld();
+                    // per head: the tile's maximum (in units of log2), across the lanes, then the warps
+#pragma unroll
+                    for (int h = 0; h < kMaxH; ++h) {
+                        float v = valid && h < H ? s[h] * sc : -INFINITY;
+                        s[h] = v;
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                        if (lane == 0) red[warp * kMaxH + h] = v;
+                    }
+                }
+                if (!bar_and_128(ok)) {
+                    stop = true;
+                    break;
+                }
+                float m[kMaxH];
+#pragma unroll
+                for (int h = 0; h < kMaxH; ++h)
+                    m[h] = fmaxf(fmaxf(red[h], red[kMaxH + h]), fmaxf(red[2 * kMaxH + h], red[3 * kMaxH + h]));
+                // p = 2^(s - m) (0 past the window and for padded heads), in bf16 as the B operand
+                // [16 heads x 128 slots]: row h, slot r at K block r / 64, 16-byte chunk (r % 64) / 8
+                uint8_t* pbuf = smem + D_OFF_P + (i & 1) * PD_BYTES;
+                const uint32_t pcol = (uint32_t)(r >> 6) * (kMaxH * 128) + (uint32_t)(r & 7) * 2;
+                const uint32_t pch = (uint32_t)((r & 63) >> 3);
+#pragma unroll
+                for (int h = 0; h < kMaxH; ++h) {
+                    const float p = s[h] == -INFINITY ? 0.f : exp2f(s[h] - m[h]);
+                    *reinterpret_cast<__nv_bfloat16*>(pbuf + pcol + (uint32_t)h * 128 + ((pch ^ (uint32_t)(h & 7)) << 4)) =
+                        __float2bfloat16_rn(p);
+                    float v = p;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                    if (lane == 0) red[4 * kMaxH + warp * kMaxH + h] = v;
+                }
+                // value rows of slots past the window (the item's last tile only): zero, once
+                // the values have landed (the MMA multiplies them by p = 0)
+                if (cnt < kTile) {
+                    const uint32_t lv = 2 * i + 1;
+                    ok = __all_sync(0xffffffffu, dwait(bars.kv_full(lv % kNBuf), (lv / kNBuf) & 1, a, abort, 8));
+                    if (ok && !valid) {
+                        uint8_t* vt = smem + D_OFF_KV + (lv % kNBuf) * KV_BYTES + r * 128;
+#pragma unroll
+                        for (int kb = 0; kb < D / 64; ++kb)
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                *reinterpret_cast<uint4*>(vt + kb * (kTile * 128) + c * 16) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                if (!bar_and_128(ok)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) mbar_arrive(bars.p_full(i & 1));
+                // the previous tile's output (a failed wait there reaches the next barrier as
+                // ok = false), then this tile's statistics take its place
+                if (i > 0) ok = epilogue(i - 1);
+#pragma unroll
+                for (int h = 0; h < kMaxH; ++h) mt[h] = m[h];
+                lt = 0.f;
+                if (r < H) lt = red[4 * kMaxH + r] + red[5 * kMaxH + r] + red[6 * kMaxH + r] + red[7 * kMaxH + r];
+                pend_b = it.b;
+                pend_sp = it.sp;
+                pend_first = ti == 0;
+                pend_last = ti == it.nt - 1;
+            }
         }
+        if (!stop && ok && i > 0) ok = epilogue(i - 1);
     }
     tc_fence_before();
     __syncthreads();
@@ -802,8 +949,8 @@ MqaLayout mqa_layout(const rglru_mqa_dims* d, bool decode) {
     size_t o = 256;
     l.q_rot = o; o = up(o + (size_t)d->batch * T * d->q_heads * mq::D * 2);
     l.k_rot = o; o = up(o + (size_t)d->batch * T * mq::D * 2);
-    l.per = mq::kDecPer;
-    l.nsplit = (d->window + l.per - 1) / l.per;
+    l.per = mq::kTile;
+    l.nsplit = (d->window + l.per - 1) / l.per;       // the most parts a row is cut into
     l.part_m = o; o = up(o + (size_t)d->batch * l.nsplit * d->q_heads * 4);
     l.part_l = o; o = up(o + (size_t)d->batch * l.nsplit * d->q_heads * 4);
     l.part_o = o; o = up(o + (size_t)d->batch * l.nsplit * d->q_heads * mq::D * 4);
@@ -870,21 +1017,31 @@ cudaError_t launch_mqa_decode(const rglru_mqa_dims* d, const void* q, const void
     // with the next row's or with zeros), the ring as 2-D [B 2 w rows][d] (box 64 x 128 slots)
     CUtensorMap mqm, mkv;
     if (!tc::make_map_2d_sw128(&mqm, ra.q_rot, D, (uint64_t)B * H, D * 2, 64, kMaxH) ||
-        !tc::make_map_2d_sw128(&mkv, ra.cache, D, (uint64_t)B * 2 * d->window, D * 2, 64, kDecPer))
+        !tc::make_map_2d_sw128(&mkv, ra.cache, D, (uint64_t)B * 2 * d->window, D * 2, 64, kTile))
         return cudaErrorInvalidValue;
     e = set_smem_once(mqa_decode_kernel, (int)D_SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    // tiles per item: up to kTilesMax while the items still give every SM about two
+    const int tiles_row = (d->window + kTile - 1) / kTile;
+    const int tpi = std::max(1, std::min(kTilesMax, (int)(((long long)B * tiles_row) / (2LL * sms))));
     DecArgs da{};
-    da.B = B; da.H = H; da.w = d->window; da.nsplit = l.nsplit; da.scale = d->scale;
-    da.pos = pos; da.cache = ra.cache;
+    da.B = B; da.H = H; da.w = d->window; da.tiles = tpi; da.nsplit = (tiles_row + tpi - 1) / tpi;
+    da.scale = d->scale;
+    da.pos = pos;
     da.part_m = reinterpret_cast<float*>(w + l.part_m);
     da.part_l = reinterpret_cast<float*>(w + l.part_l);
     da.part_o = reinterpret_cast<float*>(w + l.part_o);
     da.status = reinterpret_cast<DeviceStatus*>(w);
     da.timeout_ns = 1000000000ull;
-    mqa_decode_kernel<<<dim3(l.nsplit, B), kDecThreads, D_SMEM_BYTES, s>>>(mqm, mkv, da);
+    const int items = B * da.nsplit;
+    mqa_decode_kernel<<<std::min(items, sms), kDecThreads, D_SMEM_BYTES, s>>>(mqm, mkv, da);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     MergeArgs ma{};
-    ma.B = B; ma.H = H; ma.nsplit = l.nsplit;
+    ma.B = B; ma.H = H; ma.nsplit = da.nsplit;
     ma.part_m = da.part_m; ma.part_l = da.part_l; ma.part_o = da.part_o;
     ma.out = static_cast<__nv_bfloat16*>(out);
     mqa_merge_kernel<<<dim3(H, B), D, 0, s>>>(ma);

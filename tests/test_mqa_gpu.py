@@ -90,3 +90,32 @@ def test_mqa_decode_continues_the_prefill_through_the_ring(T0, H, w, steps):
         pav = np.stack([mqa.decode_step(arings[b], qd[b], kd[b], _abs_bits(vd[b]), int(pos[b])) for b in range(B)])
         assert_attention_close(to_np(od), ref, pav, f"mqa decode step {s}")
     assert binding.read_device_status(wsd) == binding.RGLRU_OK
+
+
+def test_mqa_decode_many_rows_multi_tile_parts():
+    """Enough rows that the decode cuts each ring of 2048 into parts of several 128-slot tiles
+    and a CTA streams several parts (running max / sum across tiles, queries of consecutive
+    rows in flight together).  The ring is filled with random bf16 data, so slots past a short
+    window hold values that must not leak; rows mix full rings (wrapped) and partial ones."""
+    B, H, w = 80, 10, 2048
+    rng = np.random.default_rng(11)
+    cache_np = _bf16(rng, (B, 2, w, D))
+    cache = binding.to_device(cache_np)
+    pos = np.array([3000 + 37 * b if b % 4 else (b * 97) % 1900 for b in range(B)], dtype=np.int32)
+    qd, kd, vd = _bf16(rng, (B, H, D)), _bf16(rng, (B, D)), _bf16(rng, (B, D))
+    ddims = binding.make_mqa_dims(B, 1, H, D, w)
+    wsd = binding.alloc_workspace(binding.mqa_workspace_size(ddims, decode=True))
+    od = torch.empty(B, H, D, dtype=torch.bfloat16, device="cuda")
+    td = lambda a: binding.to_device(a)  # noqa: E731
+    binding.mqa_decode(ddims, td(qd), td(kd), td(vd), td(pos), cache, od, wsd)
+    assert binding.read_device_status(wsd) == binding.RGLRU_OK
+    got = to_np(od)
+    kv = mqa._f64(cache_np)
+    for b in range(B):
+        ring, aring = mqa.RingCache(w, D), mqa.RingCache(w, D)
+        ring.k[:], ring.v[:] = kv[b, 0], kv[b, 1]
+        aring.k[:], aring.v[:] = kv[b, 0], np.abs(kv[b, 1])
+        ring.filled = aring.filled = int(pos[b])
+        ref = mqa.decode_step(ring, qd[b], kd[b], vd[b], int(pos[b]))
+        pav = mqa.decode_step(aring, qd[b], kd[b], _abs_bits(vd[b]), int(pos[b]))
+        assert_attention_close(got[b], ref, pav, f"mqa decode row {b} pos {pos[b]}")
