@@ -20,7 +20,8 @@
 //     into tiles of 128 and a row's tiles into parts; per tile S^T = K Q^T and O^T = V^T P^T run
 //     on the tensor cores (the H heads of a row form the MMA's N) while the next tiles stream in
 //     by TMA, the softmax on 4 warps; each part leaves (max, sum, sum of p v) per head, and
-//     mqa_merge_kernel combines the parts.
+//     mqa_merge_kernel combines the parts (the three kernels chained by programmatic dependent
+//     launch).
 #include <algorithm>
 
 #include <cuda.h>
@@ -42,6 +43,7 @@ using namespace sm100;
 constexpr int D = 256;                 // head dim (the tensor-core path)
 constexpr int BQ = 128;                // queries per CTA (MMA M)
 constexpr int BKV = 64;                // keys per tile (MMA N of S, K of P V)
+constexpr int kRopeMaxH = 16;          // query heads a row may have
 constexpr float kLog2e = 1.4426950408889634f;
 
 // ---------------------------------------------------------------- rotary embedding ----------
@@ -56,33 +58,38 @@ struct RopeArgs {
     __nv_bfloat16* cache;              // [B][2][w][d] or nullptr
 };
 
-__device__ __forceinline__ void rot_pair(float x1, float x2, double ang, float& o1, float& o2) {
+// sine and cosine of an angle given in fp64: reduced mod 2 pi in fp64, then fp32
+__device__ __forceinline__ void sincos_of(double ang, float& s, float& c) {
     const double two_pi = 6.283185307179586476925286766559;
-    double r = fmod(ang, two_pi);
-    float s, c;
-    sincosf((float)r, &s, &c);
-    o1 = x1 * c - x2 * s;
-    o2 = x2 * c + x1 * s;
+    sincosf((float)fmod(ang, two_pi), &s, &c);
 }
 
-// thread = (row b, token t, j < d/2) over the H query heads and the key
-__global__ void mqa_rope_kernel(RopeArgs a) {
+// thread = (row b, token t, j < d/2) over the H query heads and the key: the inputs first
+// (independent loads), then one angle, its sine and cosine for all of them
+__global__ void __launch_bounds__(D / 2) mqa_rope_kernel(RopeArgs a) {
     const int j = threadIdx.x;                       // 0 .. d/2 - 1
-    const int t = blockIdx.x, b = blockIdx.y;
+    const int t = blockIdx.x, b = blockIdx.y, H = a.H;
     const int p = a.pos0 + t;
-    const double ang = (double)p * pow((double)a.base, -2.0 * j / D);
-    const size_t qrow = ((size_t)b * a.T + t) * a.H * D;
-    for (int h = 0; h < a.H; ++h) {
-        const size_t e = qrow + (size_t)h * D;
-        float o1, o2;
-        rot_pair(__bfloat162float(a.q[e + j]), __bfloat162float(a.q[e + j + D / 2]), ang, o1, o2);
-        a.q_rot[e + j] = __float2bfloat16_rn(o1);
-        a.q_rot[e + j + D / 2] = __float2bfloat16_rn(o2);
-    }
+    const size_t qrow = ((size_t)b * a.T + t) * H * D;
     const size_t ke = ((size_t)b * a.T + t) * D;
-    float o1, o2;
-    rot_pair(__bfloat162float(a.k[ke + j]), __bfloat162float(a.k[ke + j + D / 2]), ang, o1, o2);
-    const __nv_bfloat16 r1 = __float2bfloat16_rn(o1), r2 = __float2bfloat16_rn(o2);
+    float x1[kRopeMaxH], x2[kRopeMaxH];
+#pragma unroll
+    for (int h = 0; h < kRopeMaxH; ++h)
+        if (h < H) {
+            x1[h] = __bfloat162float(__ldg(a.q + qrow + h * D + j));
+            x2[h] = __bfloat162float(__ldg(a.q + qrow + h * D + j + D / 2));
+        }
+    const float k1 = __bfloat162float(__ldg(a.k + ke + j)), k2 = __bfloat162float(__ldg(a.k + ke + j + D / 2));
+    const double ang = (double)p * pow((double)a.base, -2.0 * j / D);
+    float sn, cs;
+    sincos_of(ang, sn, cs);
+#pragma unroll
+    for (int h = 0; h < kRopeMaxH; ++h)
+        if (h < H) {
+            a.q_rot[qrow + h * D + j] = __float2bfloat16_rn(x1[h] * cs - x2[h] * sn);
+            a.q_rot[qrow + h * D + j + D / 2] = __float2bfloat16_rn(x2[h] * cs + x1[h] * sn);
+        }
+    const __nv_bfloat16 r1 = __float2bfloat16_rn(k1 * cs - k2 * sn), r2 = __float2bfloat16_rn(k2 * cs + k1 * sn);
     a.k_rot[ke + j] = r1;
     a.k_rot[ke + j + D / 2] = r2;
     if (a.cache && t >= a.T - a.w) {                 // the last w positions stay for decoding
@@ -109,26 +116,40 @@ struct RopeDecArgs {
     __nv_bfloat16* cache;              // [B][2][w][d]
 };
 
-__global__ void mqa_rope_decode_kernel(RopeDecArgs a) {
-    const int j = threadIdx.x, b = blockIdx.x;
-    const int p = a.pos[b];
+__global__ void __launch_bounds__(D / 2) mqa_rope_decode_kernel(RopeDecArgs a) {
+    // the attention kernel may start its set-up now; it waits for this grid before reading
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int j = threadIdx.x, b = blockIdx.x, H = a.H;
+    // every input of the thread first (independent loads), then one angle for all of them
+    const __nv_bfloat16* qb = a.q + (size_t)b * H * D;
+    float x1[kRopeMaxH], x2[kRopeMaxH];
+#pragma unroll
+    for (int h = 0; h < kRopeMaxH; ++h)
+        if (h < H) {
+            x1[h] = __bfloat162float(__ldg(qb + h * D + j));
+            x2[h] = __bfloat162float(__ldg(qb + h * D + j + D / 2));
+        }
+    const float k1 = __bfloat162float(__ldg(a.k + (size_t)b * D + j));
+    const float k2 = __bfloat162float(__ldg(a.k + (size_t)b * D + j + D / 2));
+    const __nv_bfloat16 v1 = __ldg(a.v + (size_t)b * D + j), v2 = __ldg(a.v + (size_t)b * D + j + D / 2);
+    const int p = __ldg(a.pos + b);
     const double ang = (double)p * pow((double)a.base, -2.0 * j / D);
-    for (int h = 0; h < a.H; ++h) {
-        const size_t e = ((size_t)b * a.H + h) * D;
-        float o1, o2;
-        rot_pair(__bfloat162float(a.q[e + j]), __bfloat162float(a.q[e + j + D / 2]), ang, o1, o2);
-        a.q_rot[e + j] = __float2bfloat16_rn(o1);
-        a.q_rot[e + j + D / 2] = __float2bfloat16_rn(o2);
-    }
-    float o1, o2;
-    rot_pair(__bfloat162float(a.k[(size_t)b * D + j]), __bfloat162float(a.k[(size_t)b * D + j + D / 2]), ang, o1, o2);
+    float sn, cs;
+    sincos_of(ang, sn, cs);
+    __nv_bfloat16* qr = a.q_rot + (size_t)b * H * D;
+#pragma unroll
+    for (int h = 0; h < kRopeMaxH; ++h)
+        if (h < H) {
+            qr[h * D + j] = __float2bfloat16_rn(x1[h] * cs - x2[h] * sn);
+            qr[h * D + j + D / 2] = __float2bfloat16_rn(x2[h] * cs + x1[h] * sn);
+        }
     const int slot = p % a.w;
     __nv_bfloat16* ck = a.cache + ((size_t)b * 2 * a.w + slot) * D;
     __nv_bfloat16* cv = a.cache + ((size_t)b * 2 * a.w + a.w + slot) * D;
-    ck[j] = __float2bfloat16_rn(o1);
-    ck[j + D / 2] = __float2bfloat16_rn(o2);
-    cv[j] = a.v[(size_t)b * D + j];
-    cv[j + D / 2] = a.v[(size_t)b * D + j + D / 2];
+    ck[j] = __float2bfloat16_rn(k1 * cs - k2 * sn);
+    ck[j + D / 2] = __float2bfloat16_rn(k2 * cs + k1 * sn);
+    cv[j] = v1;
+    cv[j + D / 2] = v2;
 }
 
 // ---------------------------------------------------------------- prefill attention ---------
@@ -497,6 +518,7 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
 // The step reads the ring once (2 w d bf16 per row): it is bound by HBM.
 constexpr int kTile = 128;             // slots per tile (the MMA's M)
 constexpr int kMaxH = 16;              // heads (the MMA's N), padded
+static_assert(kMaxH == kRopeMaxH, "one bound on the heads of a row");
 constexpr int kTilesMax = 4;           // tiles per item, at most
 constexpr int kNBuf = 3;               // 64 KB tile buffers
 constexpr uint32_t KV_BYTES = kTile * D * 2;          // 65536: 4 boxes of [128 slots x 64 d]
@@ -639,6 +661,8 @@ mqa_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_s;
+    // the rotated queries and the new ring slot come from the rotation kernel
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == 4) {
         // ============================ TMA: per tile its keys, then its values =================
@@ -897,6 +921,8 @@ mqa_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
         }
         if (!stop && ok && i > 0) ok = epilogue(i - 1);
     }
+    // the merge may be scheduled once every CTA is past its work (it waits for this grid)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     if (warp == 5) {
@@ -913,20 +939,32 @@ struct MergeArgs {
     __nv_bfloat16* out;                // [B, H, d]
 };
 
-__global__ void __launch_bounds__(D) mqa_merge_kernel(MergeArgs a) {
-    const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+// Block = (head, row), thread = 4 d-columns: few enough threads that all are resident at once,
+// each with its loads of the parts in flight together.
+constexpr int kMergeThreads = D / 4;
+__global__ void __launch_bounds__(kMergeThreads) mqa_merge_kernel(MergeArgs a) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // the parts of the attention kernel
+    const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
+    const size_t rb = (size_t)b * a.nsplit * a.H + h;   // part s of (b, h): rb + s H
     float mx = -INFINITY;
-    for (int s = 0; s < a.nsplit; ++s) mx = fmaxf(mx, a.part_m[((size_t)b * a.nsplit + s) * a.H + h]);
-    float l = 0.f, o = 0.f;
+    for (int s = 0; s < a.nsplit; ++s) mx = fmaxf(mx, a.part_m[rb + (size_t)s * a.H]);
+    float l = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s = 0; s < a.nsplit; ++s) {
-        const size_t pb = ((size_t)b * a.nsplit + s) * a.H + h;
-        const float m = a.part_m[pb];
+        const size_t ps = rb + (size_t)s * a.H;
+        const float m = a.part_m[ps];
         if (m == -INFINITY) continue;
         const float f = expf(m - mx);
-        l += a.part_l[pb] * f;
-        o += a.part_o[pb * D + tid] * f;
+        l = fmaf(a.part_l[ps], f, l);
+        const float4 v = reinterpret_cast<const float4*>(a.part_o + ps * D)[c];
+        o = make_float4(fmaf(v.x, f, o.x), fmaf(v.y, f, o.y), fmaf(v.z, f, o.z), fmaf(v.w, f, o.w));
     }
-    a.out[((size_t)b * a.H + h) * D + tid] = __float2bfloat16_rn(l > 0.f ? o / l : 0.f);
+    const float il = l > 0.f ? 1.0f / l : 0.f;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(o.x * il, o.y * il), hi = __floats2bfloat162_rn(o.z * il, o.w * il);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(a.out + ((size_t)b * a.H + h) * D + 4 * c) = pk;
 }
 
 }  // namespace mq
@@ -1036,16 +1074,31 @@ cudaError_t launch_mqa_decode(const rglru_mqa_dims* d, const void* q, const void
     da.part_o = reinterpret_cast<float*>(w + l.part_o);
     da.status = reinterpret_cast<DeviceStatus*>(w);
     da.timeout_ns = 1000000000ull;
-    const int items = B * da.nsplit;
-    mqa_decode_kernel<<<std::min(items, sms), kDecThreads, D_SMEM_BYTES, s>>>(mqm, mkv, da);
-    e = cudaGetLastError();
+    // the attention and merge kernels are programmatic dependents of the kernel before them:
+    // each one's launch and set-up overlap its predecessor's run
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min(B * da.nsplit, sms));
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = D_SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, mqa_decode_kernel, mqm, mkv, da);
     if (e != cudaSuccess) return e;
     MergeArgs ma{};
     ma.B = B; ma.H = H; ma.nsplit = da.nsplit;
     ma.part_m = da.part_m; ma.part_l = da.part_l; ma.part_o = da.part_o;
     ma.out = static_cast<__nv_bfloat16*>(out);
-    mqa_merge_kernel<<<dim3(H, B), D, 0, s>>>(ma);
-    return cudaGetLastError();
+    cudaLaunchConfig_t mcfg = {};
+    mcfg.gridDim = dim3(H, B);
+    mcfg.blockDim = dim3(kMergeThreads);
+    mcfg.stream = s;
+    mcfg.attrs = attr;
+    mcfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&mcfg, mqa_merge_kernel, ma);
 }
 
 }  // namespace rglru
