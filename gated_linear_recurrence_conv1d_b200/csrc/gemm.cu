@@ -66,6 +66,7 @@ struct Pair {
 
 struct Args {
     int M, N, batch, splits, npairs;
+    int interleave;      // every pair has the same K: their K blocks alternate
     int mt, nt;          // tiles along M and N
     Pair p[kMaxPairs];
     float* C;            // C[split][b][m][n] at C + split * c_split + b * c_bstride + m * c_ld + n
@@ -77,8 +78,11 @@ struct Args {
     unsigned long long timeout_ns;
 };
 
-// K blocks of one output tile: the blocks of pair 0, then those of pair 1, ..., cut into
-// `splits` equal slices (the last may be shorter)
+// K blocks of one output tile: when every pair has the same K, block kb is block kb / npairs of
+// pair kb % npairs (the pairs interleaved, so that an operand shared by two pairs -- the hi part
+// of xc against both parts of dg -- is read twice within a few blocks and the second read hits
+// L2); otherwise the blocks of pair 0, then those of pair 1, ...  Cut into `splits` equal slices
+// (the last may be shorter).
 struct KPlan {
     int total, per;      // blocks in all, blocks per slice
 };
@@ -91,6 +95,10 @@ __host__ __device__ inline KPlan kplan(const Args& a) {
 }
 // the pair of K block kb and the block's index within that pair
 __device__ __forceinline__ int pair_of(const Args& a, int kb, int& local) {
+    if (a.interleave) {
+        local = kb / a.npairs;
+        return kb % a.npairs;
+    }
     int i = 0;
     while (i + 1 < a.npairs && kb >= a.p[i].K / BK) {
         kb -= a.p[i].K / BK;
@@ -411,6 +419,9 @@ cudaError_t launch_gemm(const GemmOperands& g, cudaStream_t s) {
         a.p[i].b_boff_row = gp.b_boff_row; a.p[i].b_boff_col = gp.b_boff_col;
         a.p[i].b_bstep_row = gp.b_bstep_row; a.p[i].b_bstep_col = gp.b_bstep_col;
     }
+    a.interleave = 1;
+    for (int i = 1; i < g.npairs; ++i)
+        if (g.p[i].K != g.p[0].K) a.interleave = 0;
     a.C = g.C; a.c_ld = g.c_ld; a.c_bstride = g.c_bstride; a.c_split = g.c_split;
     a.Cadd = g.Cadd; a.add_ld = g.add_ld; a.add_bstride = g.add_bstride;
     a.C16 = g.C16;
