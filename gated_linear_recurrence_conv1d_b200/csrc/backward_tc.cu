@@ -622,8 +622,8 @@ cudaError_t launch_backward_tc(const rglru_dims* d, const rglru_params* p, const
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return cudaGetLastError();
-    const int wtiles = H * (DH / 128);                     // 128 x 256 output tiles per gate
-    const int splits = std::max(1, std::min(kMaxSplits, sms / wtiles));
+    const int wtiles = H;                                  // 256 x 256 output tiles (a CTA pair each) per gate
+    const int splits = std::max(1, std::min(kMaxSplits, (sms / 2) / wtiles));
     for (int gate = 0; gate < 2; ++gate) {
         GemmOperands gw{};
         gw.M = DH; gw.N = DH; gw.batch = H; gw.splits = splits; gw.npairs = 3;

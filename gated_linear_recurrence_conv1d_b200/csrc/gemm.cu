@@ -13,14 +13,18 @@
 //     contiguous: element (m, k) at k * ld + m); B likewise N x K, "K-major" or "N-major".  The
 //     operands are read by TMA in 128-byte swizzled tiles straight from the caller's tensors
 //     (2-D maps; the batch index adds a fixed row or column offset);
-//   * a persistent CTA per SM walks output tiles of 128 x 256 (batch, m-tile, n-tile, k-slice);
-//     one warp loads K blocks of 64 through a 4-stage ring (48 KB a stage), an elected lane of
-//     another issues tcgen05.mma (M = 128, N = 256, K = 16 per instruction) into one of two TMEM
-//     accumulators of 256 columns, and 8 epilogue warps (two per TMEM lane quadrant, 128
-//     columns each) read the other accumulator 32 columns at a time and pass it through a
-//     swizzled shared-memory tile, so that Cadd is read and C written in whole 128-byte row
-//     segments.  The wide tile halves the operand bytes per flop
-//     that L2 has to deliver to each SM, compared with a square 128 x 128 tile.
+//   * a persistent pair of CTAs (a 2-CTA cluster on neighbouring SMs) walks output tiles of
+//     256 x 256 (batch, m-tile, n-tile, k-slice) with tcgen05.mma.cta_group::2 (M = 256, N = 256,
+//     K = 16 per instruction): each CTA holds half of A (128 rows) and half of B (128 columns)
+//     of every 64-wide K block in a 6-stage ring (32 KB a stage), so a CTA moves 2/3 of the
+//     bytes a 128 x 256 tile would for the same flops and has more of them in flight; the
+//     leader CTA's MMA warp issues for both, its commits arrive on both CTAs' barriers, and
+//     its ring barriers count both CTAs' TMA bytes (the partner's loads complete on the
+//     leader's barrier).  Each CTA's accumulator half (its 128 rows x 256 columns, two TMEM
+//     buffers) is read by its 8 epilogue warps (two per TMEM lane quadrant, 128 columns each)
+//     32 columns at a time through a swizzled shared-memory tile, so that Cadd is read and C
+//     written in whole 128-byte row segments; they hand the buffer back to the leader.
+//   * no multicast loads: each CTA's TMA reads only its own halves.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -38,10 +42,11 @@ namespace gm {
 
 using namespace sm100;
 
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64;         // BM rows per CTA (256 per pair), BN columns
+constexpr int BNH = BN / 2;                        // B columns a CTA loads
+constexpr int STAGES = 6;
 constexpr uint32_t TILE_A = BM * BK * 2;           // 16384
-constexpr uint32_t TILE_B = BN * BK * 2;           // 32768
+constexpr uint32_t TILE_B = BNH * BK * 2;          // 16384
 constexpr uint32_t STAGE_BYTES = TILE_A + TILE_B;
 constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
 // per epilogue warp, a [32 rows x 32 columns] fp32 staging tile (rows of 128 B, 16-byte chunks
@@ -141,10 +146,73 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr) {
     d |= (uint64_t)2 << 61;
     return d;
 }
-// instruction descriptor: fp32 accumulator, bf16 A and B, their majorness, M x N
+// instruction descriptor: fp32 accumulator, bf16 A and B, their majorness, M (the pair's 256
+// rows) x N
 __device__ __forceinline__ uint32_t idesc(int a_mn, int b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-           ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+           ((uint32_t)(BN >> 3) << 17) | ((uint32_t)((2 * BM) >> 4) << 24);
+}
+
+// ---- the CTA pair: every tcgen05 instruction of this kernel is of cta_group::2
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D (both CTAs' TMEM) (+)= A (both CTAs' halves) * B (both CTAs' halves)^T
+__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t id,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(id), "r"(accumulate)
+        : "memory");
+}
+// arrive on the mbarrier at this shared address in both CTAs of the pair once every prior MMA
+// of this thread completes
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+}
+// a tile of this CTA's half into its own shared memory, its bytes counted on the leader's
+// barrier (a shared::cluster address)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+// waits on barriers that other CTAs of the pair arrive on (cluster-scope acquire)
+__device__ __noinline__ bool wait_slow_c(uint32_t bar, uint32_t parity, const Args& a, volatile int* abort,
+                                        unsigned where) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (it > 64) __nanosleep(200);
+        if (*abort) return false;
+        if (*(volatile unsigned*)&a.status->code != 0) {
+            *abort = 1;
+            return false;
+        }
+        if (globaltimer_ns() - t0 > a.timeout_ns) {
+            latch_status(a.status, RGLRU_ERR_TIMEOUT, where, blockIdx.x, parity);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool wait_c(uint32_t bar, uint32_t parity, const Args& a, volatile int* abort, unsigned where) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    return wait_slow_c(bar, parity, a, abort, where);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -160,26 +228,29 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
     auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto acc_full = [&](int i) { return bar0 + 8u * (2 * STAGES + i); };
     auto acc_empty = [&](int i) { return bar0 + 8u * (2 * STAGES + 2 + i); };
+    const uint32_t mma_done = bar0 + 8u * (2 * STAGES + 4);
     volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 8 * (2 * STAGES + 5));
     volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_BAR + 8 * (2 * STAGES + 5) + 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();             // 0: the leader, which issues the MMAs
+    const int pair = blockIdx.x >> 1, npair = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full(s), 1);
+            mbar_init(full(s), 1);                       // the leader's arrival + both CTAs' bytes
             mbar_init(empty(s), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(acc_full(i), 1);
-            mbar_init(acc_empty(i), kEpiWarps);
+            mbar_init(acc_empty(i), 2 * kEpiWarps);      // the epilogue warps of both CTAs
         }
-        mbar_init(acc_empty(0) + 8u * 2, 1);                  // mma_done
+        mbar_init(mma_done, 1);
         *abort = 0;
         fence_barrier_init();
     }
     if (warp == kWarpMma) {
-        tmem_alloc(smem_u32((const void*)tmem_base_s), TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32((const void*)tmem_base_s), TMEM_COLS);
+        tmem_relinquish_pair();
     }
     const CUtensorMap* mas[kMaxPairs] = {&ma0, &ma1, &ma2, &ma3};
     const CUtensorMap* mbs[kMaxPairs] = {&mb0, &mb1, &mb2, &mb3};
@@ -191,6 +262,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync();                                      // both CTAs' barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem = *tmem_base_s;
     const KPlan kp = kplan(a);
@@ -203,21 +275,24 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
         t /= a.nt;
         const int mi = t % a.mt;
         b = t / a.mt;
-        m0 = mi * BM;
+        m0 = mi * (2 * BM);
         n0 = ni * BN;
     };
 
     if (warp == kWarpTma) {
         if (lane == 0) {
+            // this CTA's halves: A rows [m0 + 128 rank, + 128), B columns [n0 + 128 rank, + 128);
+            // their bytes complete on the leader's full barrier, which the leader arms for both
+            const uint32_t rb = (uint32_t)rank * BM;
             int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            for (int t = pair; t < ntiles && ok; t += npair) {
                 int b, m0, n0, sp;
                 tile_of(t, b, m0, n0, sp);
                 const int k_beg = sp * kp.per, k_end = min(kp.total, k_beg + kp.per);
                 for (int kb = k_beg; kb < k_end; ++kb, ++it) {
                     const int s = it % STAGES;
-                    if (!wait_b(empty(s), ((it / STAGES) & 1) ^ 1, a, abort, 1)) {
+                    if (!wait_c(empty(s), ((it / STAGES) & 1) ^ 1, a, abort, 1)) {
                         ok = false;
                         break;
                     }
@@ -228,94 +303,101 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
                     const CUtensorMap* ma = mas[pi];
                     const CUtensorMap* mb = mbs[pi];
                     const uint32_t sa = sbase + s * STAGE_BYTES, sb = sa + TILE_A;
+                    const uint32_t fb = map_to_rank(full(s), 0);
                     const int ar = p.a_boff_row + b * p.a_bstep_row, ac = p.a_boff_col + b * p.a_bstep_col;
                     const int br = p.b_boff_row + b * p.b_bstep_row, bc = p.b_boff_col + b * p.b_bstep_col;
-                    mbar_arrive_expect_tx(full(s), STAGE_BYTES);
+                    if (rank == 0) mbar_arrive_expect_tx(full(s), 2 * STAGE_BYTES);
                     if (p.a_kmajor) {
-                        tma_load_2d(sa, ma, ac + k0, ar + m0, full(s));
+                        tma_load_2d_pair(sa, ma, ac + k0, ar + m0 + rb, fb);
                     } else {
-                        tma_load_2d(sa, ma, ac + m0, ar + k0, full(s));
-                        tma_load_2d(sa + 8192, ma, ac + m0 + 64, ar + k0, full(s));
+                        tma_load_2d_pair(sa, ma, ac + m0 + rb, ar + k0, fb);
+                        tma_load_2d_pair(sa + 8192, ma, ac + m0 + rb + 64, ar + k0, fb);
                     }
                     if (p.b_kmajor) {
-                        tma_load_2d(sb, mb, bc + k0, br + n0, full(s));
+                        tma_load_2d_pair(sb, mb, bc + k0, br + n0 + rb, fb);
                     } else {
-#pragma unroll
-                        for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, mb, bc + n0 + 64 * j, br + k0, full(s));
+                        tma_load_2d_pair(sb, mb, bc + n0 + rb, br + k0, fb);
+                        tma_load_2d_pair(sb + 8192, mb, bc + n0 + rb + 64, br + k0, fb);
                     }
                 }
             }
-            // never leave the CTA with a bulk copy still writing its shared memory
-            const uint64_t t0 = globaltimer_ns();
-            for (int i = it - STAGES; i < it; ++i)
-                if (i >= 0)
-                    while (!mbar_try_wait_sleep(full(i % STAGES), (i / STAGES) & 1, 20000u) &&
-                           globaltimer_ns() - t0 < a.timeout_ns) {
-                    }
+            // never leave the pair with a bulk copy still writing shared memory: the leader sees
+            // every load of both CTAs land on its barriers (the partner waits for it below)
+            if (rank == 0) {
+                const uint64_t t0 = globaltimer_ns();
+                for (int i = it - STAGES; i < it; ++i)
+                    if (i >= 0)
+                        while (!mbar_try_wait_cluster(full(i % STAGES), (i / STAGES) & 1) &&
+                               globaltimer_ns() - t0 < a.timeout_ns) {
+                        }
+            }
         }
     } else if (warp == kWarpMma) {
-        // the whole warp follows the waits (warp-uniform control flow); one elected lane issues,
-        // so that the descriptors stay uniform and consecutive MMAs issue back to back
+        // the leader's warp follows the waits (warp-uniform control flow); one elected lane
+        // issues for the pair.  The partner's warp only waits for the pair's last MMA.
         const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
-        int it = 0, tc = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++tc) {
-            int b, m0, n0, sp;
-            tile_of(t, b, m0, n0, sp);
-            const int k_beg = sp * kp.per, k_end = min(kp.total, k_beg + kp.per);
-            const int ai = tc & 1;
-            if (!__all_sync(0xffffffffu, wait_b(acc_empty(ai), ((tc >> 1) & 1) ^ 1, a, abort, 2))) break;
-            tc_fence_after();
-            const uint32_t d = tm + ai * BN;
-            for (int kb = k_beg; kb < k_end; ++kb, ++it) {
-                const int s = it % STAGES;
-                if (!__all_sync(0xffffffffu, wait_b(full(s), (it / STAGES) & 1, a, abort, 3))) {
-                    ok = false;
-                    break;
-                }
+        if (rank == 0) {
+            int it = 0, tc = 0;
+            bool ok = true;
+            for (int t = pair; t < ntiles && ok; t += npair, ++tc) {
+                int b, m0, n0, sp;
+                tile_of(t, b, m0, n0, sp);
+                const int k_beg = sp * kp.per, k_end = min(kp.total, k_beg + kp.per);
+                const int ai = tc & 1;
+                if (!__all_sync(0xffffffffu, wait_c(acc_empty(ai), ((tc >> 1) & 1) ^ 1, a, abort, 2))) break;
                 tc_fence_after();
-                int local;
-                const Pair& p = a.p[pair_of(a, kb, local)];
-                const uint32_t id = idesc(p.a_kmajor ? 0 : 1, p.b_kmajor ? 0 : 1);
-                const uint32_t sa = sbase + s * STAGE_BYTES, sb = sa + TILE_A;
-                if (elect_one()) {
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        // K step kk: 32 bytes along a K-major row, or 16 K-rows (2048 B) of an
-                        // MN-major tile
-                        const uint64_t ad = p.a_kmajor ? desc_k_sw128(sa + kk * 32) : desc_mn_sw128(sa + kk * 2048);
-                        const uint64_t bd = p.b_kmajor ? desc_k_sw128(sb + kk * 32) : desc_mn_sw128(sb + kk * 2048);
-                        mma_ss(d, ad, bd, id, (kb > k_beg || kk > 0) ? 1u : 0u);
+                const uint32_t d = tm + ai * BN;
+                for (int kb = k_beg; kb < k_end; ++kb, ++it) {
+                    const int s = it % STAGES;
+                    if (!__all_sync(0xffffffffu, wait_c(full(s), (it / STAGES) & 1, a, abort, 3))) {
+                        ok = false;
+                        break;
                     }
-                    mma_commit(empty(s));
+                    tc_fence_after();
+                    int local;
+                    const Pair& p = a.p[pair_of(a, kb, local)];
+                    const uint32_t id = idesc(p.a_kmajor ? 0 : 1, p.b_kmajor ? 0 : 1);
+                    const uint32_t sa = sbase + s * STAGE_BYTES, sb = sa + TILE_A;
+                    if (elect_one()) {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            // K step kk: 32 bytes along a K-major row, or 16 K-rows (2048 B) of an
+                            // MN-major tile; the same offsets address the partner's halves
+                            const uint64_t ad = p.a_kmajor ? desc_k_sw128(sa + kk * 32) : desc_mn_sw128(sa + kk * 2048);
+                            const uint64_t bd = p.b_kmajor ? desc_k_sw128(sb + kk * 32) : desc_mn_sw128(sb + kk * 2048);
+                            mma_ss_pair(d, ad, bd, id, (kb > k_beg || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit_pair(empty(s));
+                    }
+                    __syncwarp();
                 }
+                if (!ok) break;
+                if (elect_one()) mma_commit_pair(acc_full(ai));
                 __syncwarp();
             }
-            if (!ok) break;
-            if (elect_one()) mma_commit(acc_full(ai));
+            // every MMA has finished (in both CTAs' TMEM) before TMEM is released
+            if (elect_one()) mma_commit_pair(mma_done);
             __syncwarp();
         }
-        // every MMA of this warp has finished before TMEM is released
-        if (elect_one()) mma_commit(acc_empty(0) + 8u * 2);     // the mma_done barrier after acc_empty[1]
-        __syncwarp();
         if (lane == 0) {
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait_sleep(acc_empty(0) + 8u * 2, 0, 20000u) && globaltimer_ns() - t0 < a.timeout_ns) {
+            while (!mbar_try_wait_cluster(mma_done, 0) && globaltimer_ns() - t0 < a.timeout_ns) {
             }
         }
         __syncwarp();
     } else {
         // ================================ epilogue: thread = row of the tile ==================
         // warp w reads lane quadrant w % 4 (the TMEM lanes a warp may access) and the columns
-        // [128 (w / 4), 128 (w / 4) + 128) of the tile
+        // [128 (w / 4), 128 (w / 4) + 128) of this CTA's 128 rows of the tile
         const int q = warp & 3;
         const int cb = (warp >> 2) * (BN / 2);
         int tc = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tc) {
+        for (int t = pair; t < ntiles; t += npair, ++tc) {
             int b, m0, n0, sp;
             tile_of(t, b, m0, n0, sp);
+            m0 += (int)rank * BM;                        // this CTA's rows
             const int ai = tc & 1;
-            if (!__all_sync(0xffffffffu, wait_b(acc_full(ai), (tc >> 1) & 1, a, abort, 4))) break;
+            if (!__all_sync(0xffffffffu, wait_c(acc_full(ai), (tc >> 1) & 1, a, abort, 4))) break;
             tc_fence_after();
             // a K slice without blocks (more slices than K blocks) contributes zeros: its
             // accumulator was never written
@@ -375,15 +457,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty(ai));
+            if (lane == 0) mbar_arrive_cluster(map_to_rank(acc_empty(ai), 0));   // the leader's barrier
         }
         tmem_wait_ld();
     }
+    // no CTA of the pair leaves while the other may still reach its shared memory or TMEM
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == kWarpMma) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc_pair(tmem, TMEM_COLS);
     }
 }
 
@@ -404,13 +488,13 @@ cudaError_t launch_gemm(const GemmOperands& g, cudaStream_t s) {
     CUtensorMap maps[2 * kMaxPairs];
     Args a{};
     a.M = g.M; a.N = g.N; a.batch = g.batch; a.splits = g.splits; a.npairs = g.npairs;
-    a.mt = (g.M + BM - 1) / BM; a.nt = (g.N + BN - 1) / BN;
+    a.mt = (g.M + 2 * BM - 1) / (2 * BM); a.nt = (g.N + BN - 1) / BN;
     for (int i = 0; i < kMaxPairs; ++i) {
         const GemmPair& gp = g.p[i < g.npairs ? i : 0];
         if (gp.K <= 0 || gp.K % BK != 0) return cudaErrorInvalidValue;
-        // a K-major operand's tile is 128 rows of 64 K; an MN-major one 64 K-rows of 2 x 64
+        // a CTA's half of an operand tile: K-major, 128 rows of 64 K; MN-major, 64 K-rows of 2 x 64
         if (!map_2d(&maps[2 * i], gp.a, gp.a_rows, gp.a_cols, gp.a_ld, gp.a_kmajor ? BM : BK) ||
-            !map_2d(&maps[2 * i + 1], gp.b, gp.b_rows, gp.b_cols, gp.b_ld, gp.b_kmajor ? BN : BK))
+            !map_2d(&maps[2 * i + 1], gp.b, gp.b_rows, gp.b_cols, gp.b_ld, gp.b_kmajor ? BNH : BK))
             return cudaErrorInvalidValue;
         a.p[i].K = gp.K;
         a.p[i].a_kmajor = gp.a_kmajor; a.p[i].b_kmajor = gp.b_kmajor;
@@ -430,15 +514,38 @@ cudaError_t launch_gemm(const GemmOperands& g, cudaStream_t s) {
     a.timeout_ns = 1000000000ull;
     cudaError_t e = set_smem_once(gemm_kernel, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
+    // pairs of CTAs (2-CTA clusters), as many as can be resident at once, each walking tiles
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static std::mutex mu;
+    static int max_pairs[64] = {};
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    int pairs = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev >= 0 && dev < 64) pairs = max_pairs[dev];
+    }
+    if (pairs <= 0) {
+        cfg.gridDim = dim3(2);
+        if ((e = cudaOccupancyMaxActiveClusters(&pairs, gemm_kernel, &cfg)) != cudaSuccess) return e;
+        if (pairs <= 0) return cudaErrorLaunchOutOfResources;
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev >= 0 && dev < 64) max_pairs[dev] = pairs;
+    }
     const int ntiles = a.batch * a.mt * a.nt * a.splits;
-    const int grid = ntiles < sms ? ntiles : sms;
-    gemm_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6],
-                                                   maps[7], a);
-    return cudaGetLastError();
+    cfg.gridDim = dim3(2u * (unsigned)(ntiles < pairs ? ntiles : pairs));
+    return cudaLaunchKernelEx(&cfg, gemm_kernel, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6],
+                              maps[7], a);
 }
 
 }  // namespace rglru
