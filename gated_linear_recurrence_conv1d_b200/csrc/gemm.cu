@@ -252,12 +252,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
         tmem_alloc_pair(smem_u32((const void*)tmem_base_s), TMEM_COLS);
         tmem_relinquish_pair();
     }
-    const CUtensorMap* mas[kMaxPairs] = {&ma0, &ma1, &ma2, &ma3};
-    const CUtensorMap* mbs[kMaxPairs] = {&mb0, &mb1, &mb2, &mb3};
     if (warp == kWarpTma && lane == 0) {
-        for (int i = 0; i < a.npairs; ++i) {
-            prefetch_tensormap(mas[i]);
-            prefetch_tensormap(mbs[i]);
+        prefetch_tensormap(&ma0);
+        prefetch_tensormap(&mb0);
+        if (a.npairs > 1) {
+            prefetch_tensormap(&ma1);
+            prefetch_tensormap(&mb1);
+        }
+        if (a.npairs > 2) {
+            prefetch_tensormap(&ma2);
+            prefetch_tensormap(&mb2);
+        }
+        if (a.npairs > 3) {
+            prefetch_tensormap(&ma3);
+            prefetch_tensormap(&mb3);
         }
     }
     tc_fence_before();
@@ -279,53 +287,90 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
         n0 = ni * BN;
     };
 
+    // the operand pairs share their majorness (checked on the host): one instruction descriptor,
+    // and descriptor steps per K step of 16 -- 32 bytes along a K-major row, or 16 K-rows (2048
+    // bytes) of an MN-major tile, i.e. 2 or 128 in the descriptor's address field
+    const bool akm = a.p[0].a_kmajor != 0, bkm = a.p[0].b_kmajor != 0;
+    const uint32_t id = idesc(akm ? 0 : 1, bkm ? 0 : 1);
+    const uint64_t a_step = akm ? 2 : 128, b_step = bkm ? 2 : 128;
+    // (pair, block within the pair) of K block kb, then advanced one block at a time
+    auto advance = [&](int& pi, int& local) {
+        if (a.interleave) {
+            if (++pi == a.npairs) {
+                pi = 0;
+                ++local;
+            }
+        } else if (++local == a.p[pi].K / BK) {
+            local = 0;
+            ++pi;
+        }
+    };
+
     if (warp == kWarpTma) {
         if (lane == 0) {
             // this CTA's halves: A rows [m0 + 128 rank, + 128), B columns [n0 + 128 rank, + 128);
             // their bytes complete on the leader's full barrier, which the leader arms for both
-            const uint32_t rb = (uint32_t)rank * BM;
-            int it = 0;
+            const int rb = (int)rank * BM;
+            const uint32_t fb0 = map_to_rank(full(0), 0);
+            int s = 0;
+            uint32_t ph = 0;
+            int issued = 0;
             bool ok = true;
             for (int t = pair; t < ntiles && ok; t += npair) {
                 int b, m0, n0, sp;
                 tile_of(t, b, m0, n0, sp);
                 const int k_beg = sp * kp.per, k_end = min(kp.total, k_beg + kp.per);
-                for (int kb = k_beg; kb < k_end; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    if (!wait_c(empty(s), ((it / STAGES) & 1) ^ 1, a, abort, 1)) {
+                // the tile's operand coordinates per pair (selected by value: no indexed arrays)
+                int ar[kMaxPairs], ac[kMaxPairs], br[kMaxPairs], bc[kMaxPairs];
+#pragma unroll
+                for (int i = 0; i < kMaxPairs; ++i) {
+                    ar[i] = a.p[i].a_boff_row + b * a.p[i].a_bstep_row + (akm ? m0 + rb : 0);
+                    ac[i] = a.p[i].a_boff_col + b * a.p[i].a_bstep_col + (akm ? 0 : m0 + rb);
+                    br[i] = a.p[i].b_boff_row + b * a.p[i].b_bstep_row + (bkm ? n0 + rb : 0);
+                    bc[i] = a.p[i].b_boff_col + b * a.p[i].b_bstep_col + (bkm ? 0 : n0 + rb);
+                }
+                int pi = 0, local = 0;
+                if (k_beg < k_end) pi = pair_of(a, k_beg, local);
+                for (int kb = k_beg; kb < k_end; ++kb) {
+                    if (!wait_c(empty(s), ph ^ 1, a, abort, 1)) {
                         ok = false;
                         break;
                     }
-                    int local;
-                    const int pi = pair_of(a, kb, local);
-                    const Pair& p = a.p[pi];
                     const int k0 = local * BK;
-                    const CUtensorMap* ma = mas[pi];
-                    const CUtensorMap* mb = mbs[pi];
+                    const CUtensorMap* ma = pi == 0 ? &ma0 : pi == 1 ? &ma1 : pi == 2 ? &ma2 : &ma3;
+                    const CUtensorMap* mb = pi == 0 ? &mb0 : pi == 1 ? &mb1 : pi == 2 ? &mb2 : &mb3;
+                    const int arr = pi == 0 ? ar[0] : pi == 1 ? ar[1] : pi == 2 ? ar[2] : ar[3];
+                    const int acc_ = pi == 0 ? ac[0] : pi == 1 ? ac[1] : pi == 2 ? ac[2] : ac[3];
+                    const int brr = pi == 0 ? br[0] : pi == 1 ? br[1] : pi == 2 ? br[2] : br[3];
+                    const int bcc = pi == 0 ? bc[0] : pi == 1 ? bc[1] : pi == 2 ? bc[2] : bc[3];
                     const uint32_t sa = sbase + s * STAGE_BYTES, sb = sa + TILE_A;
-                    const uint32_t fb = map_to_rank(full(s), 0);
-                    const int ar = p.a_boff_row + b * p.a_bstep_row, ac = p.a_boff_col + b * p.a_bstep_col;
-                    const int br = p.b_boff_row + b * p.b_bstep_row, bc = p.b_boff_col + b * p.b_bstep_col;
+                    const uint32_t fb = fb0 + 8u * s;
                     if (rank == 0) mbar_arrive_expect_tx(full(s), 2 * STAGE_BYTES);
-                    if (p.a_kmajor) {
-                        tma_load_2d_pair(sa, ma, ac + k0, ar + m0 + rb, fb);
+                    if (akm) {
+                        tma_load_2d_pair(sa, ma, acc_ + k0, arr, fb);
                     } else {
-                        tma_load_2d_pair(sa, ma, ac + m0 + rb, ar + k0, fb);
-                        tma_load_2d_pair(sa + 8192, ma, ac + m0 + rb + 64, ar + k0, fb);
+                        tma_load_2d_pair(sa, ma, acc_, arr + k0, fb);
+                        tma_load_2d_pair(sa + 8192, ma, acc_ + 64, arr + k0, fb);
                     }
-                    if (p.b_kmajor) {
-                        tma_load_2d_pair(sb, mb, bc + k0, br + n0 + rb, fb);
+                    if (bkm) {
+                        tma_load_2d_pair(sb, mb, bcc + k0, brr, fb);
                     } else {
-                        tma_load_2d_pair(sb, mb, bc + n0 + rb, br + k0, fb);
-                        tma_load_2d_pair(sb + 8192, mb, bc + n0 + rb + 64, br + k0, fb);
+                        tma_load_2d_pair(sb, mb, bcc, brr + k0, fb);
+                        tma_load_2d_pair(sb + 8192, mb, bcc + 64, brr + k0, fb);
                     }
+                    ++issued;
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                    advance(pi, local);
                 }
             }
             // never leave the pair with a bulk copy still writing shared memory: the leader sees
             // every load of both CTAs land on its barriers (the partner waits for it below)
             if (rank == 0) {
                 const uint64_t t0 = globaltimer_ns();
-                for (int i = it - STAGES; i < it; ++i)
+                for (int i = issued - STAGES; i < issued; ++i)
                     if (i >= 0)
                         while (!mbar_try_wait_cluster(full(i % STAGES), (i / STAGES) & 1) &&
                                globaltimer_ns() - t0 < a.timeout_ns) {
@@ -337,8 +382,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
         // issues for the pair.  The partner's warp only waits for the pair's last MMA.
         const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
         if (rank == 0) {
-            int it = 0, tc = 0;
+            int s = 0, tc = 0;
+            uint32_t ph = 0;
             bool ok = true;
+            const uint64_t da0 = akm ? desc_k_sw128(sbase) : desc_mn_sw128(sbase);
+            const uint64_t db0 = bkm ? desc_k_sw128(sbase + TILE_A) : desc_mn_sw128(sbase + TILE_A);
             for (int t = pair; t < ntiles && ok; t += npair, ++tc) {
                 int b, m0, n0, sp;
                 tile_of(t, b, m0, n0, sp);
@@ -347,29 +395,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
                 if (!__all_sync(0xffffffffu, wait_c(acc_empty(ai), ((tc >> 1) & 1) ^ 1, a, abort, 2))) break;
                 tc_fence_after();
                 const uint32_t d = tm + ai * BN;
-                for (int kb = k_beg; kb < k_end; ++kb, ++it) {
-                    const int s = it % STAGES;
-                    if (!__all_sync(0xffffffffu, wait_c(full(s), (it / STAGES) & 1, a, abort, 3))) {
+                for (int kb = k_beg; kb < k_end; ++kb) {
+                    if (!__all_sync(0xffffffffu, wait_c(full(s), ph, a, abort, 3))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    int local;
-                    const Pair& p = a.p[pair_of(a, kb, local)];
-                    const uint32_t id = idesc(p.a_kmajor ? 0 : 1, p.b_kmajor ? 0 : 1);
-                    const uint32_t sa = sbase + s * STAGE_BYTES, sb = sa + TILE_A;
                     if (elect_one()) {
+                        // stage s's descriptors: the stage base's plus the stage offset / 16; the
+                        // same offsets address the partner's halves
+                        const uint64_t ad = da0 + (uint64_t)((s * STAGE_BYTES) >> 4);
+                        const uint64_t bd = db0 + (uint64_t)((s * STAGE_BYTES) >> 4);
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {
-                            // K step kk: 32 bytes along a K-major row, or 16 K-rows (2048 B) of an
-                            // MN-major tile; the same offsets address the partner's halves
-                            const uint64_t ad = p.a_kmajor ? desc_k_sw128(sa + kk * 32) : desc_mn_sw128(sa + kk * 2048);
-                            const uint64_t bd = p.b_kmajor ? desc_k_sw128(sb + kk * 32) : desc_mn_sw128(sb + kk * 2048);
-                            mma_ss_pair(d, ad, bd, id, (kb > k_beg || kk > 0) ? 1u : 0u);
-                        }
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            mma_ss_pair(d, ad + kk * a_step, bd + kk * b_step, id, (kb > k_beg || kk > 0) ? 1u : 0u);
                         mma_commit_pair(empty(s));
                     }
                     __syncwarp();
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
                 }
                 if (!ok) break;
                 if (elect_one()) mma_commit_pair(acc_full(ai));
@@ -504,8 +550,10 @@ cudaError_t launch_gemm(const GemmOperands& g, cudaStream_t s) {
         a.p[i].b_bstep_row = gp.b_bstep_row; a.p[i].b_bstep_col = gp.b_bstep_col;
     }
     a.interleave = 1;
-    for (int i = 1; i < g.npairs; ++i)
+    for (int i = 1; i < g.npairs; ++i) {
         if (g.p[i].K != g.p[0].K) a.interleave = 0;
+        if (g.p[i].a_kmajor != g.p[0].a_kmajor || g.p[i].b_kmajor != g.p[0].b_kmajor) return cudaErrorInvalidValue;
+    }
     a.C = g.C; a.c_ld = g.c_ld; a.c_bstride = g.c_bstride; a.c_split = g.c_split;
     a.Cadd = g.Cadd; a.add_ld = g.add_ld; a.add_bstride = g.add_bstride;
     a.C16 = g.C16;
