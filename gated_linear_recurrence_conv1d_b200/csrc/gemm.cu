@@ -215,6 +215,9 @@ __device__ __forceinline__ bool wait_c(uint32_t bar, uint32_t parity, const Args
     return wait_slow_c(bar, parity, a, abort, where);
 }
 
+// NP: the number of operand pairs (a compile-time constant, so that the producer's per-pair
+// selections fold away for a single pair)
+template <int NP>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUtensorMap mb0,
             const __grid_constant__ CUtensorMap ma1, const __grid_constant__ CUtensorMap mb1,
@@ -255,15 +258,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
     if (warp == kWarpTma && lane == 0) {
         prefetch_tensormap(&ma0);
         prefetch_tensormap(&mb0);
-        if (a.npairs > 1) {
+        if (NP > 1) {
             prefetch_tensormap(&ma1);
             prefetch_tensormap(&mb1);
         }
-        if (a.npairs > 2) {
+        if (NP > 2) {
             prefetch_tensormap(&ma2);
             prefetch_tensormap(&mb2);
         }
-        if (a.npairs > 3) {
+        if (NP > 3) {
             prefetch_tensormap(&ma3);
             prefetch_tensormap(&mb3);
         }
@@ -296,7 +299,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
     // (pair, block within the pair) of K block kb, then advanced one block at a time
     auto advance = [&](int& pi, int& local) {
         if (a.interleave) {
-            if (++pi == a.npairs) {
+            if (++pi == NP) {
                 pi = 0;
                 ++local;
             }
@@ -321,9 +324,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
                 tile_of(t, b, m0, n0, sp);
                 const int k_beg = sp * kp.per, k_end = min(kp.total, k_beg + kp.per);
                 // the tile's operand coordinates per pair (selected by value: no indexed arrays)
-                int ar[kMaxPairs], ac[kMaxPairs], br[kMaxPairs], bc[kMaxPairs];
+                int ar[NP], ac[NP], br[NP], bc[NP];
 #pragma unroll
-                for (int i = 0; i < kMaxPairs; ++i) {
+                for (int i = 0; i < NP; ++i) {
                     ar[i] = a.p[i].a_boff_row + b * a.p[i].a_bstep_row + (akm ? m0 + rb : 0);
                     ac[i] = a.p[i].a_boff_col + b * a.p[i].a_bstep_col + (akm ? 0 : m0 + rb);
                     br[i] = a.p[i].b_boff_row + b * a.p[i].b_bstep_row + (bkm ? n0 + rb : 0);
@@ -337,12 +340,19 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
                         break;
                     }
                     const int k0 = local * BK;
-                    const CUtensorMap* ma = pi == 0 ? &ma0 : pi == 1 ? &ma1 : pi == 2 ? &ma2 : &ma3;
-                    const CUtensorMap* mb = pi == 0 ? &mb0 : pi == 1 ? &mb1 : pi == 2 ? &mb2 : &mb3;
-                    const int arr = pi == 0 ? ar[0] : pi == 1 ? ar[1] : pi == 2 ? ar[2] : ar[3];
-                    const int acc_ = pi == 0 ? ac[0] : pi == 1 ? ac[1] : pi == 2 ? ac[2] : ac[3];
-                    const int brr = pi == 0 ? br[0] : pi == 1 ? br[1] : pi == 2 ? br[2] : br[3];
-                    const int bcc = pi == 0 ? bc[0] : pi == 1 ? bc[1] : pi == 2 ? bc[2] : bc[3];
+                    const CUtensorMap* ma = &ma0;
+                    const CUtensorMap* mb = &mb0;
+                    int arr = ar[0], acc_ = ac[0], brr = br[0], bcc = bc[0];
+#pragma unroll
+                    for (int i = 1; i < NP; ++i)
+                        if (pi == i) {
+                            ma = i == 1 ? &ma1 : i == 2 ? &ma2 : &ma3;
+                            mb = i == 1 ? &mb1 : i == 2 ? &mb2 : &mb3;
+                            arr = ar[i];
+                            acc_ = ac[i];
+                            brr = br[i];
+                            bcc = bc[i];
+                        }
                     const uint32_t sa = sbase + s * STAGE_BYTES, sb = sa + TILE_A;
                     const uint32_t fb = fb0 + 8u * s;
                     if (rank == 0) mbar_arrive_expect_tx(full(s), 2 * STAGE_BYTES);
@@ -560,7 +570,12 @@ cudaError_t launch_gemm(const GemmOperands& g, cudaStream_t s) {
     if (a.C16 && (a.Cadd || g.splits > 1 || g.c_ld % 8 != 0)) return cudaErrorInvalidValue;
     a.status = g.status;
     a.timeout_ns = 1000000000ull;
-    cudaError_t e = set_smem_once(gemm_kernel, (int)SMEM_BYTES);
+    void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                 CUtensorMap, Args) = g.npairs == 1   ? gemm_kernel<1>
+                                      : g.npairs == 2 ? gemm_kernel<2>
+                                      : g.npairs == 3 ? gemm_kernel<3>
+                                                      : gemm_kernel<4>;
+    cudaError_t e = set_smem_once(kern, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // pairs of CTAs (2-CTA clusters), as many as can be resident at once, each walking tiles
     cudaLaunchConfig_t cfg = {};
@@ -575,25 +590,24 @@ cudaError_t launch_gemm(const GemmOperands& g, cudaStream_t s) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     static std::mutex mu;
-    static int max_pairs[64] = {};
+    static int max_pairs[kMaxPairs][64] = {};
     int dev = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     int pairs = 0;
     {
         std::lock_guard<std::mutex> lock(mu);
-        if (dev >= 0 && dev < 64) pairs = max_pairs[dev];
+        if (dev >= 0 && dev < 64) pairs = max_pairs[g.npairs - 1][dev];
     }
     if (pairs <= 0) {
         cfg.gridDim = dim3(2);
-        if ((e = cudaOccupancyMaxActiveClusters(&pairs, gemm_kernel, &cfg)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg)) != cudaSuccess) return e;
         if (pairs <= 0) return cudaErrorLaunchOutOfResources;
         std::lock_guard<std::mutex> lock(mu);
-        if (dev >= 0 && dev < 64) max_pairs[dev] = pairs;
+        if (dev >= 0 && dev < 64) max_pairs[g.npairs - 1][dev] = pairs;
     }
     const int ntiles = a.batch * a.mt * a.nt * a.splits;
     cfg.gridDim = dim3(2u * (unsigned)(ntiles < pairs ? ntiles : pairs));
-    return cudaLaunchKernelEx(&cfg, gemm_kernel, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6],
-                              maps[7], a);
+    return cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7], a);
 }
 
 }  // namespace rglru
