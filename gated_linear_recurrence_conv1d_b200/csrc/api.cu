@@ -330,7 +330,7 @@ rglru_status rglru_layer_plan(const rglru_dims* dims, const rglru_projections* p
 static rglru_status check_mqa(const rglru_mqa_dims* d, bool decode) {
     if (!d || d->batch <= 0 || d->q_heads <= 0 || d->head_dim <= 0 || d->window <= 0) return RGLRU_ERR_INVALID_ARG;
     if (!decode && d->seq_len <= 0) return RGLRU_ERR_INVALID_ARG;
-    if (!(d->scale == d->scale) || !(d->rope_base > 0.0f)) return RGLRU_ERR_INVALID_ARG;
+    if (!(d->scale > 0.0f) || !(d->rope_base > 0.0f)) return RGLRU_ERR_INVALID_ARG;
     if (!rglru::mqa_supported(d)) return RGLRU_ERR_UNSUPPORTED;
     if (!decode && (long long)d->batch * d->seq_len * d->q_heads * d->head_dim > (1LL << 40)) return RGLRU_ERR_UNSUPPORTED;
     if (d->batch > (1 << 16) || (!decode && d->seq_len > (1 << 30))) return RGLRU_ERR_UNSUPPORTED;

@@ -168,8 +168,8 @@ constexpr uint32_t P_BYTES = BQ * BKV * 2;           // 16384: [128 queries x 64
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;          // 2 stages
 constexpr uint32_t OFF_V = OFF_K + 2 * KT_BYTES;     // 2 stages
-constexpr uint32_t OFF_P = OFF_V + 2 * VT_BYTES;
-constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
+constexpr uint32_t OFF_P = OFF_V + 2 * VT_BYTES;     // 2 buffers (tile parity)
+constexpr uint32_t OFF_BAR = OFF_P + 2 * P_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 // TMEM: [0,128) Q (A operand, bf16 pairs), [128,256) S double buffer, [256,512) O (fp32)
@@ -186,9 +186,9 @@ struct Bars {
     __device__ __forceinline__ uint32_t v_empty(int i) const { return base + 64 + 8u * i; }
     __device__ __forceinline__ uint32_t s_full(int i) const { return base + 80 + 8u * i; }
     __device__ __forceinline__ uint32_t s_free(int i) const { return base + 96 + 8u * i; }
-    __device__ __forceinline__ uint32_t p_full() const { return base + 112; }
-    __device__ __forceinline__ uint32_t o_done() const { return base + 120; }   // a P V finished
-    __device__ __forceinline__ uint32_t mma_done() const { return base + 128; }
+    __device__ __forceinline__ uint32_t p_full(int i) const { return base + 112 + 8u * i; }
+    __device__ __forceinline__ uint32_t o_done(int i) const { return base + 128 + 8u * i; }   // P V on buffer i finished
+    __device__ __forceinline__ uint32_t mma_done() const { return base + 144; }
 };
 
 __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, const PrefArgs& a, volatile int* abort, unsigned where) {
@@ -234,8 +234,8 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const Bars bars{sbase + OFF_BAR};
-    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 144);
-    volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_BAR + 160);
+    volatile uint32_t* tmem_base_s = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 160);
+    volatile int* abort = reinterpret_cast<volatile int*>(smem + OFF_BAR + 176);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // blockIdx.x = query tile, y = head, z = row
     const int t0 = blockIdx.x * BQ, h = blockIdx.y, b = blockIdx.z;
@@ -254,9 +254,9 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             mbar_init(bars.v_empty(i), 1);
             mbar_init(bars.s_full(i), 1);
             mbar_init(bars.s_free(i), kSmWarps);
+            mbar_init(bars.p_full(i), kSmWarps);
+            mbar_init(bars.o_done(i), 1);
         }
-        mbar_init(bars.p_full(), kSmWarps);
-        mbar_init(bars.o_done(), 1);
         mbar_init(bars.mma_done(), 1);
         *abort = 0;
         fence_barrier_init();
@@ -329,18 +329,18 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
                 __syncwarp();
             }
             if (j >= 1) {                                    // O += P_{j-1} V_{j-1}
-                const int jj = j - 1, s = jj & 1;
-                if (!wait_w(bars.p_full(), jj & 1, 6)) break;
+                const int jj = j - 1, s = jj & 1;             // P and V buffers of tile jj
+                if (!wait_w(bars.p_full(s), (jj >> 1) & 1, 6)) break;
                 if (!wait_w(bars.v_full(s), (jj >> 1) & 1, 7)) break;
                 tc_fence_after();
                 if (elect_one()) {
 #pragma unroll
                     for (int ks = 0; ks < BKV / 16; ++ks) {
-                        const uint64_t ad = desc_k_sw128(sbase + OFF_P + ks * 32);
+                        const uint64_t ad = desc_k_sw128(sbase + OFF_P + s * P_BYTES + ks * 32);
                         const uint64_t bd = desc_v(sbase + OFF_V + s * VT_BYTES + ks * 2048);
                         mma_ss(tm + TM_O, ad, bd, id_o, (jj > 0 || ks > 0) ? 1u : 0u);
                     }
-                    mma_commit(bars.o_done());
+                    mma_commit(bars.o_done(s));
                     mma_commit(bars.v_empty(s));
                 }
                 __syncwarp();
@@ -406,25 +406,40 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.s_free(s));
+            // scores stay unscaled (scale > 0: the maximum commutes with it); a tile inside every
+            // query's window (the same for the whole CTA) needs no mask
             float mx = -INFINITY;
+            if (key0 >= t0 + BQ - a.w && key0 + BKV - 1 <= t0) {
 #pragma unroll
-            for (int i = 0; i < BKV; ++i) {
-                const int key = key0 + i;
-                const bool in = t < a.T && key >= lo_key && key <= t;
-                sv[i] = in ? sv[i] * a.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, sv[i]);
+                for (int i = 0; i < BKV; ++i) mx = fmaxf(mx, sv[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < BKV; ++i) {
+                    const int key = key0 + i;
+                    const bool in = t < a.T && key >= lo_key && key <= t;
+                    sv[i] = in ? sv[i] : -INFINITY;
+                    mx = fmaxf(mx, sv[i]);
+                }
             }
+            mx *= a.scale_log2;
             // the reference maximum moves (and the accumulator is rescaled) only when the
             // tile's maximum passes it by more than 8 (a factor 256 in P)
             const bool move = mx > m_ref + 8.0f;
             const bool any_move = __any_sync(0xffffffffu, move);
             const float m_new = move ? mx : m_ref;
-            // P of the previous tile must be consumed (and O complete) before P and O change
-            if (pv_issued > 0) {
-                ok = __all_sync(0xffffffffu, wait_b(bars.o_done(), (pv_issued - 1) & 1, a, abort, 10));
+            // P buffer s was last read by the P V of tile j - 2; O may be rescaled only once the
+            // P V of tile j - 1 (and so every earlier one) is complete
+            if (pv_issued >= 2) {
+                const int jj = pv_issued - 2;                 // == j - 2
+                ok = __all_sync(0xffffffffu, wait_b(bars.o_done(jj & 1), (jj >> 1) & 1, a, abort, 10));
                 if (!ok) break;
-                tc_fence_after();
             }
+            if (any_move && pv_issued > 0) {
+                const int jj = pv_issued - 1;
+                ok = __all_sync(0xffffffffu, wait_b(bars.o_done(jj & 1), (jj >> 1) & 1, a, abort, 12));
+                if (!ok) break;
+            }
+            tc_fence_after();
             if (any_move && pv_issued > 0) {
                 const float f = (move && m_ref != -INFINITY) ? exp2f(m_ref - m_new) : 1.0f;
 #pragma unroll 1
@@ -441,13 +456,13 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             }
             m_ref = m_new;
             // P in bf16: row r, 64 keys = 128 bytes, 16-byte chunks swizzled by (r & 7)
-            uint8_t* prow = smem + OFF_P + (r >> 3) * 1024 + (r & 7) * 128;
+            uint8_t* prow = smem + OFF_P + s * P_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 float p[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    p[i] = (m_ref == -INFINITY) ? 0.f : exp2f(sv[8 * c + i] - m_ref);
+                    p[i] = (m_ref == -INFINITY) ? 0.f : exp2f(fmaf(sv[8 * c + i], a.scale_log2, -m_ref));
                     l += p[i];
                 }
                 uint4 pk;
@@ -460,12 +475,14 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bars.p_full());
+            if (lane == 0) mbar_arrive(bars.p_full(s));
             ++pv_issued;
         }
         // the last P V, then out = O / l
-        if (ok && pv_issued > 0)
-            ok = __all_sync(0xffffffffu, wait_b(bars.o_done(), (pv_issued - 1) & 1, a, abort, 11));
+        if (ok && pv_issued > 0) {
+            const int jj = pv_issued - 1;                     // the last P V (every earlier one is done too)
+            ok = __all_sync(0xffffffffu, wait_b(bars.o_done(jj & 1), (jj >> 1) & 1, a, abort, 11));
+        }
         if (ok) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.0f / l : 0.f;

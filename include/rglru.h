@@ -239,7 +239,7 @@ typedef struct {
     int q_heads;      /* H */
     int head_dim;     /* d, 256 */
     int window;       /* w */
-    float scale;      /* score scale, e.g. 1 / sqrt(head_dim) */
+    float scale;      /* score scale > 0, e.g. 1 / sqrt(head_dim) */
     float rope_base;  /* e.g. 10000 */
 } rglru_mqa_dims;
 

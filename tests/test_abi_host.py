@@ -147,7 +147,9 @@ def test_mqa_rejects_bad_arguments():
     for bad, code in ((binding.make_mqa_dims(2, 64, 4, 128, 32), 2),     # head_dim
                       (binding.make_mqa_dims(2, 64, 17, 256, 32), 2),    # too many query heads
                       (binding.make_mqa_dims(2, 64, 4, 256, 0), 1),      # window
-                      (binding.make_mqa_dims(0, 64, 4, 256, 8), 1)):     # batch
+                      (binding.make_mqa_dims(0, 64, 4, 256, 8), 1),      # batch
+                      (binding.make_mqa_dims(2, 64, 4, 256, 32, scale=0.0), 1),    # score scale not > 0
+                      (binding.make_mqa_dims(2, 64, 4, 256, 32, scale=-0.5), 1)):
         assert binding.mqa_workspace_size(bad) == 0
         rc = lib.rglru_mqa_prefill(ctypes.byref(bad), ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE + 0x100),
                                    ctypes.c_void_p(FAKE + 0x200), 0, ctypes.c_void_p(FAKE + 0x300), None,
