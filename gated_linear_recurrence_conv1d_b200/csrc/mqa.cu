@@ -456,13 +456,16 @@ mqa_prefill_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_const
             }
             m_ref = m_new;
             // P in bf16: row r, 64 keys = 128 bytes, 16-byte chunks swizzled by (r & 7)
+            // (m_ref is -inf only while every score so far, this tile's included, is masked: then
+            // the exponent is -inf and p = 0)
             uint8_t* prow = smem + OFF_P + s * P_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
+            const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 float p[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    p[i] = (m_ref == -INFINITY) ? 0.f : exp2f(fmaf(sv[8 * c + i], a.scale_log2, -m_ref));
+                    p[i] = ex2_approx(fmaf(sv[8 * c + i], a.scale_log2, neg_m));
                     l += p[i];
                 }
                 uint4 pk;
