@@ -16,7 +16,8 @@
 //   * a persistent pair of CTAs (a 2-CTA cluster on neighbouring SMs) walks output tiles of
 //     256 x 256 (batch, m-tile, n-tile, k-slice) with tcgen05.mma.cta_group::2 (M = 256, N = 256,
 //     K = 16 per instruction): each CTA holds half of A (128 rows) and half of B (128 columns)
-//     of every 64-wide K block in a 6-stage ring (32 KB a stage), so a CTA moves 2/3 of the
+//     of every 64-wide K block, two K blocks to a stage of a 3-stage ring (64 KB a stage: the
+//     loads and the MMAs of a stage share one barrier round trip), so a CTA moves 2/3 of the
 //     bytes a 128 x 256 tile would for the same flops and has more of them in flight; the
 //     leader CTA's MMA warp issues for both, its commits arrive on both CTAs' barriers, and
 //     its ring barriers count both CTAs' TMA bytes (the partner's loads complete on the
@@ -44,10 +45,11 @@ using namespace sm100;
 
 constexpr int BM = 128, BN = 256, BK = 64;         // BM rows per CTA (256 per pair), BN columns
 constexpr int BNH = BN / 2;                        // B columns a CTA loads
-constexpr int STAGES = 6;
-constexpr uint32_t TILE_A = BM * BK * 2;           // 16384
+constexpr int KPS = 2;                             // 64-wide K blocks per ring stage
+constexpr int STAGES = 3;
+constexpr uint32_t TILE_A = BM * BK * 2;           // 16384: a CTA's half of A for one K block
 constexpr uint32_t TILE_B = BNH * BK * 2;          // 16384
-constexpr uint32_t STAGE_BYTES = TILE_A + TILE_B;
+constexpr uint32_t STAGE_BYTES = KPS * (TILE_A + TILE_B);   // [A blocks][B blocks]
 constexpr uint32_t OFF_BAR = STAGES * STAGE_BYTES;
 // per epilogue warp, a [32 rows x 32 columns] fp32 staging tile (rows of 128 B, 16-byte chunks
 // XOR-swizzled by the row): the warp's accumulator rows go in row by row and come out as whole
@@ -334,46 +336,52 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
                 }
                 int pi = 0, local = 0;
                 if (k_beg < k_end) pi = pair_of(a, k_beg, local);
-                for (int kb = k_beg; kb < k_end; ++kb) {
+                for (int kb = k_beg; kb < k_end; kb += KPS) {
                     if (!wait_c(empty(s), ph ^ 1, a, abort, 1)) {
                         ok = false;
                         break;
                     }
-                    const int k0 = local * BK;
-                    const CUtensorMap* ma = &ma0;
-                    const CUtensorMap* mb = &mb0;
-                    int arr = ar[0], acc_ = ac[0], brr = br[0], bcc = bc[0];
-#pragma unroll
-                    for (int i = 1; i < NP; ++i)
-                        if (pi == i) {
-                            ma = i == 1 ? &ma1 : i == 2 ? &ma2 : &ma3;
-                            mb = i == 1 ? &mb1 : i == 2 ? &mb2 : &mb3;
-                            arr = ar[i];
-                            acc_ = ac[i];
-                            brr = br[i];
-                            bcc = bc[i];
-                        }
-                    const uint32_t sa = sbase + s * STAGE_BYTES, sb = sa + TILE_A;
+                    const int nb = min(KPS, k_end - kb);     // K blocks in this stage
                     const uint32_t fb = fb0 + 8u * s;
-                    if (rank == 0) mbar_arrive_expect_tx(full(s), 2 * STAGE_BYTES);
-                    if (akm) {
-                        tma_load_2d_pair(sa, ma, acc_ + k0, arr, fb);
-                    } else {
-                        tma_load_2d_pair(sa, ma, acc_, arr + k0, fb);
-                        tma_load_2d_pair(sa + 8192, ma, acc_ + 64, arr + k0, fb);
-                    }
-                    if (bkm) {
-                        tma_load_2d_pair(sb, mb, bcc + k0, brr, fb);
-                    } else {
-                        tma_load_2d_pair(sb, mb, bcc, brr + k0, fb);
-                        tma_load_2d_pair(sb + 8192, mb, bcc + 64, brr + k0, fb);
+                    if (rank == 0) mbar_arrive_expect_tx(full(s), 2u * (uint32_t)nb * (TILE_A + TILE_B));
+#pragma unroll
+                    for (int j = 0; j < KPS; ++j) {
+                        if (j >= nb) break;
+                        const int k0 = local * BK;
+                        const CUtensorMap* ma = &ma0;
+                        const CUtensorMap* mb = &mb0;
+                        int arr = ar[0], acc_ = ac[0], brr = br[0], bcc = bc[0];
+#pragma unroll
+                        for (int i = 1; i < NP; ++i)
+                            if (pi == i) {
+                                ma = i == 1 ? &ma1 : i == 2 ? &ma2 : &ma3;
+                                mb = i == 1 ? &mb1 : i == 2 ? &mb2 : &mb3;
+                                arr = ar[i];
+                                acc_ = ac[i];
+                                brr = br[i];
+                                bcc = bc[i];
+                            }
+                        const uint32_t sa = sbase + s * STAGE_BYTES + j * TILE_A;
+                        const uint32_t sb = sbase + s * STAGE_BYTES + KPS * TILE_A + j * TILE_B;
+                        if (akm) {
+                            tma_load_2d_pair(sa, ma, acc_ + k0, arr, fb);
+                        } else {
+                            tma_load_2d_pair(sa, ma, acc_, arr + k0, fb);
+                            tma_load_2d_pair(sa + 8192, ma, acc_ + 64, arr + k0, fb);
+                        }
+                        if (bkm) {
+                            tma_load_2d_pair(sb, mb, bcc + k0, brr, fb);
+                        } else {
+                            tma_load_2d_pair(sb, mb, bcc, brr + k0, fb);
+                            tma_load_2d_pair(sb + 8192, mb, bcc + 64, brr + k0, fb);
+                        }
+                        advance(pi, local);
                     }
                     ++issued;
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1;
                     }
-                    advance(pi, local);
                 }
             }
             // never leave the pair with a bulk copy still writing shared memory: the leader sees
@@ -396,7 +404,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
             uint32_t ph = 0;
             bool ok = true;
             const uint64_t da0 = akm ? desc_k_sw128(sbase) : desc_mn_sw128(sbase);
-            const uint64_t db0 = bkm ? desc_k_sw128(sbase + TILE_A) : desc_mn_sw128(sbase + TILE_A);
+            const uint64_t db0 = bkm ? desc_k_sw128(sbase + KPS * TILE_A) : desc_mn_sw128(sbase + KPS * TILE_A);
             for (int t = pair; t < ntiles && ok; t += npair, ++tc) {
                 int b, m0, n0, sp;
                 tile_of(t, b, m0, n0, sp);
@@ -405,20 +413,26 @@ gemm_kernel(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUt
                 if (!__all_sync(0xffffffffu, wait_c(acc_empty(ai), ((tc >> 1) & 1) ^ 1, a, abort, 2))) break;
                 tc_fence_after();
                 const uint32_t d = tm + ai * BN;
-                for (int kb = k_beg; kb < k_end; ++kb) {
+                for (int kb = k_beg; kb < k_end; kb += KPS) {
                     if (!__all_sync(0xffffffffu, wait_c(full(s), ph, a, abort, 3))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    const int nb = min(KPS, k_end - kb);
                     if (elect_one()) {
-                        // stage s's descriptors: the stage base's plus the stage offset / 16; the
-                        // same offsets address the partner's halves
-                        const uint64_t ad = da0 + (uint64_t)((s * STAGE_BYTES) >> 4);
-                        const uint64_t bd = db0 + (uint64_t)((s * STAGE_BYTES) >> 4);
+                        // block j of stage s: the stage base's descriptor plus the byte offset / 16;
+                        // the same offsets address the partner's halves
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)
-                            mma_ss_pair(d, ad + kk * a_step, bd + kk * b_step, id, (kb > k_beg || kk > 0) ? 1u : 0u);
+                        for (int j = 0; j < KPS; ++j) {
+                            if (j >= nb) break;
+                            const uint64_t ad = da0 + (uint64_t)((s * STAGE_BYTES + j * TILE_A) >> 4);
+                            const uint64_t bd = db0 + (uint64_t)((s * STAGE_BYTES + j * TILE_B) >> 4);
+#pragma unroll
+                            for (int kk = 0; kk < BK / 16; ++kk)
+                                mma_ss_pair(d, ad + kk * a_step, bd + kk * b_step, id,
+                                            (kb > k_beg || j > 0 || kk > 0) ? 1u : 0u);
+                        }
                         mma_commit_pair(empty(s));
                     }
                     __syncwarp();
