@@ -827,8 +827,8 @@ mqa_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
 #pragma unroll
                 for (int h = 0; h < kMaxH; ++h) {
                     const float mn = fmaxf(M[h], mt[h]);
-                    const float fo = mn == -INFINITY ? 0.f : exp2f(M[h] - mn);
-                    const float fn = mn == -INFINITY ? 0.f : exp2f(mt[h] - mn);
+                    const float fo = mn == -INFINITY ? 0.f : ex2_approx(M[h] - mn);
+                    const float fn = mn == -INFINITY ? 0.f : ex2_approx(mt[h] - mn);
                     acc0[h] = fmaf(acc0[h], fo, o0[h] * fn);
                     acc1[h] = fmaf(acc1[h], fo, o1[h] * fn);
                     M[h] = mn;
@@ -897,7 +897,7 @@ mqa_decode_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_consta
                 const uint32_t pch = (uint32_t)((r & 63) >> 3);
 #pragma unroll
                 for (int h = 0; h < kMaxH; ++h) {
-                    const float p = s[h] == -INFINITY ? 0.f : exp2f(s[h] - m[h]);
+                    const float p = s[h] == -INFINITY ? 0.f : ex2_approx(s[h] - m[h]);
                     *reinterpret_cast<__nv_bfloat16*>(pbuf + pcol + (uint32_t)h * 128 + ((pch ^ (uint32_t)(h & 7)) << 4)) =
                         __float2bfloat16_rn(p);
                     float v = p;
