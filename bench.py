@@ -875,8 +875,10 @@ def main():
     elif args.extras_only:
         import torch
         dev = torch.device("cuda", torch.cuda.current_device())
-        print(json.dumps({"backward": bench_backward(args, dev), "layer": bench_layer(args, dev),
-                          "mqa": bench_mqa(args, dev)}))
+        out = {} if args.no_backward else {"backward": bench_backward(args, dev)}
+        out["layer"] = bench_layer(args, dev)
+        out["mqa"] = bench_mqa(args, dev)
+        print(json.dumps(out))
     else:
         run_ours(args)
 
