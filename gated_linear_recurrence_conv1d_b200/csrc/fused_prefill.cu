@@ -734,13 +734,10 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                                         (((cl & (HALF - 1)) + 4 * p4) >> 2)
                                   : nullptr;
                 uint2 fw[3];                              // final window (the tail of the row), bf16
-                if ((rm & 0xFFu) == 0) {
-                    if (has_last) conv_tokens<false, true>(xtw, bhi, xcw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
-                    else conv_tokens<false, false>(xtw, bhi, xcw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
-                } else {
-                    if (has_last) conv_tokens<true, true>(xtw, bhi, xcw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
-                    else conv_tokens<true, false>(xtw, bhi, xcw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
-                }
+                if ((rm & 0xFFu) == 0 && !has_last)
+                    conv_tokens<false, false>(xtw, bhi, xcw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
+                else
+                    conv_tokens<true, true>(xtw, bhi, xcw, cchunk, rm, jlast, w, cb, h0, h1, h2, fw);
                 // final conv history of the sequence (this CTA's channels), as soon as the row's
                 // last token is convolved: the conv read the copy taken before the launch
                 if (write_tail) {
