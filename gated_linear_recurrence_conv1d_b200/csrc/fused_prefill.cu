@@ -85,8 +85,8 @@ constexpr bool kSplitGate = true;
 // producer (tickets and x tiles), 13 MMA.  14 warps: at most 4 per SM sub-partition, so 128
 // registers a thread.
 constexpr int kEpiGroup = 4, kEpiWarps = G * kEpiGroup;
-constexpr int kWarpProd = kEpiWarps, kWarpMma = kWarpProd + 1;
-constexpr int kThreads = (kWarpMma + 1) * 32;   // 448
+constexpr int kWarpProd = kEpiWarps, kWarpMma = kWarpProd + 1, kWarpStore = kWarpMma + 1;
+constexpr int kThreads = (kWarpStore + 1) * 32;   // 480: 15 warps, still at most 4 per SM sub-partition
 constexpr int kSlots = 4;               // TMEM accumulator slots (item n uses slot n % 4)
 
 constexpr uint32_t KBLK_BYTES = L * 128;               // one 64-channel K block of the B tile
@@ -756,23 +756,8 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             return true;
         };
 
-        // y tile of the group's item n into its stage, by one thread, once the stage's previous
-        // out tile has been read by its store; false: no load (the end, or a failed wait)
-        const bool y_loader = !SAVE && q == 0 && lane == 0;
-        auto load_y = [&](int n) -> bool {
-            if (!wait_bar(bars.tk(n % RING), (n / RING) & 1, wc, 3)) return false;
-            const int kn = slot[n % RING];
-            if (kn < 0) return false;
-            mbar_arrive_expect_tx(bars.y_full(st), Y_BYTES);
-            tma_load_3d(sbase + OFF_Y + st * Y_BYTES, &map_y, head * DH + half * HALF, (kn / a.B) * L, kn % a.B,
-                        bars.y_full(st));
-            return true;
-        };
-
         int n = eg;
         bool have = conv_item(n);
-        int y_pending = -1;                              // item whose y load is in flight, or -1
-        if (have && y_loader && load_y(n)) y_pending = n;
         while (have) {
             const uint32_t ph = (n / G) & 1;
             const int sl = n % kSlots;
@@ -873,7 +858,6 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
             } else {
                 // ---- pass 2: h_t from the carry, merged with GeLU(y_t)
                 if (!wait_bar_warp(bars.y_full(st), ph, wc, 16)) break;
-                if (y_loader) y_pending = -1;
                 if (tanh_form) pass2<true>(dcol, yt, carry);
                 else pass2<false>(dcol, yt, carry);
                 // the TMEM slot is read: the MMA of a later item may overwrite it
@@ -881,33 +865,83 @@ fused_prefill_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars.slot_free(sl));
 
-                // ---- out tile -> global (TMA store clips the ragged tail); then the next y
+                // ---- the out tile is complete: the store warp writes it and loads the next y
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars.out_ready(st));
-                if (q == 0 && lane == 0) {
-                    if (wait_bar(bars.out_ready(st), ph, wc, 17)) {
-                        tma_store_3d(&map_out, sbase + OFF_Y + st * Y_BYTES, head * DH + half * HALF, t0, b);
-                        bulk_commit();
-                        bulk_wait_read0();               // the tile is free for the next y
-                        if (have_next && load_y(n + G)) y_pending = n + G;
-                    }
-                }
             }
             n += G;
             have = have_next;
         }
-        // no tensor-memory access of this warp may still be in flight when TMEM is released, and
-        // no bulk copy may still write this CTA's shared memory when it exits
+        // no tensor-memory access of this warp may still be in flight when TMEM is released
         tmem_wait_ld();
-        if (q == 0 && lane == 0) {
-            bulk_wait0();
-            if (y_pending >= 0) {
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait_sleep(bars.y_full(st), (y_pending / G) & 1, 100000u) &&
-                       globaltimer_ns() - t0 < a.timeout_ns) {
+    } else if (warp == kWarpStore) {
+        // ================================ out stores and y loads ==============================
+        // one thread serves the three stages: as a stage's item completes its second pass, its
+        // out tile goes to global memory by TMA (which clips the ragged tail) and, once the tile
+        // has been read, the y tile of the stage's next item comes in -- so that no epilogue
+        // warp waits for a store
+        if (!SAVE && lane == 0) {
+            int nxt[G], kb[G];                           // stage's item and its (row, chunk), or -1
+            bool done[G];
+            int pending_y[G];                            // item whose y load is in flight, or -1
+            auto issue_y = [&](int st, int m) -> bool {  // y of item m into stage st; false: the end
+                if (!wait_bar(bars.tk(m % RING), (m / RING) & 1, wc, 30)) return false;
+                const int km = slot[m % RING];
+                if (km < 0) return false;
+                mbar_arrive_expect_tx(bars.y_full(st), Y_BYTES);
+                tma_load_3d(sbase + OFF_Y + st * Y_BYTES, &map_y, head * DH + half * HALF, (km / a.B) * L, km % a.B,
+                            bars.y_full(st));
+                kb[st] = km;
+                pending_y[st] = m;
+                return true;
+            };
+            int live = 0;
+            for (int st = 0; st < G; ++st) {
+                nxt[st] = st;
+                pending_y[st] = -1;
+                done[st] = !issue_y(st, st);
+                live += done[st] ? 0 : 1;
+            }
+            uint64_t t_last = globaltimer_ns();
+            while (live > 0) {
+                bool progress = false;
+                for (int st = 0; st < G; ++st) {
+                    if (done[st]) continue;
+                    const int m = nxt[st];
+                    if (!mbar_try_wait(bars.out_ready(st), (m / G) & 1)) continue;
+                    progress = true;
+                    pending_y[st] = -1;                  // its second pass consumed the y tile
+                    tma_store_3d(&map_out, sbase + OFF_Y + st * Y_BYTES, head * DH + half * HALF,
+                                 (kb[st] / a.B) * L, kb[st] % a.B);
+                    bulk_commit();
+                    bulk_wait_read0();                   // the tile is free for the next y
+                    nxt[st] = m + G;
+                    if (!issue_y(st, m + G)) {
+                        done[st] = true;
+                        --live;
+                    }
+                }
+                if (progress) {
+                    t_last = globaltimer_ns();
+                } else {
+                    __nanosleep(64);
+                    if (*abort || *(volatile unsigned*)&a.status->code != 0) break;
+                    if (globaltimer_ns() - t_last > a.timeout_ns) {
+                        latch_status(a.status, RGLRU_ERR_TIMEOUT, 31, blockIdx.x, (unsigned)live);
+                        *abort = 1;
+                        break;
+                    }
                 }
             }
+            // no bulk copy may still read or write this CTA's shared memory when it exits
+            bulk_wait0();
+            const uint64_t t0w = globaltimer_ns();
+            for (int st = 0; st < G; ++st)
+                if (pending_y[st] >= 0)
+                    while (!mbar_try_wait_sleep(bars.y_full(st), (pending_y[st] / G) & 1, 100000u) &&
+                           globaltimer_ns() - t0w < a.timeout_ns) {
+                    }
         }
     }
 
