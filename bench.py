@@ -58,8 +58,8 @@ NCU_TRAFFIC = {
     # the packed workload's is that capture
     # scaled by the algorithmic bytes (every item moves the same tiles), the packed workload itself
     # being above the size a multi-pass capture may hold on the device
-    ("fused_prefill.cu", "36d84f7a96280daa", "rg2b_bf16"): 235977728,
-    ("fused_prefill.cu", "36d84f7a96280daa", "packed_bf16"): 4483364376,
+    ("fused_prefill.cu", "bf5e2316ce3e1637", "rg2b_bf16"): 236076288,
+    ("fused_prefill.cu", "bf5e2316ce3e1637", "packed_bf16"): 4485236927,
 }
 
 

@@ -17,11 +17,12 @@
 //     so that hi + lo is the fp32 value to 2^-16 -- and, for the CTA's own 128 channels, in fp32
 //     for the epilogue (the i_t x_t term of the update);
 //   * warp roles: an x producer (tickets and the TMA of the [35 tokens x 256 channels] x tile
-//     with its 3-token halo), 2 conv warps (16 tokens each; a lane convolves 8 channels with
-//     packed fp32x2 FMAs), one MMA warp (D = W^T . xc^T for both gates, M = 128 channels, N = 32
-//     tokens, K = 256 x 2 parts; an elected lane issues) and 3 epilogue groups of 4 warps, group
-//     g taking the items n = g (mod 3) and loading their y tiles; 3 stages of shared-memory tiles
-//     and TMEM accumulators;
+//     with its 3-token halo), one MMA warp (D = W^T . xc^T for both gates, M = 128 channels, N =
+//     32 tokens, K = 256 x 2 parts; an elected lane issues), 3 groups of 4 warps, group g taking
+//     the items n = g (mod 3): it convolves its next item (a lane 8 channels x 8 tokens with
+//     packed fp32x2 FMAs) and runs the epilogue of its current one, and a store warp that writes
+//     each finished out tile by TMA and loads the stage's next y tile; 3 stages of shared-memory
+//     tiles, 4 TMEM accumulator slots;
 //   * transposed orientation: a TMEM lane is an output channel and the 32 columns are tokens,
 //     so an epilogue thread owns one channel.  Its first pass turns the gate contractions into
 //     a_t and the normalised input u_t, 8 tokens at a time, writes them back over the stage's
@@ -81,12 +82,12 @@ constexpr int kConvBatch = 4;           // x rows a conv lane loads ahead of the
 constexpr bool kSplitGate = true;
 
 // warp roles: 0-11 three groups of 4 (TMEM lane quarter = warp % 4, group = warp / 4): a group
-// convolves its next item, runs the epilogue of its current one and loads its y tiles; 12 x
-// producer (tickets and x tiles), 13 MMA.  14 warps: at most 4 per SM sub-partition, so 128
+// convolves its next item and runs the epilogue of its current one; 12 x producer (tickets and x
+// tiles), 13 MMA, 14 out stores and y loads.  15 warps: at most 4 per SM sub-partition, so 128
 // registers a thread.
 constexpr int kEpiGroup = 4, kEpiWarps = G * kEpiGroup;
 constexpr int kWarpProd = kEpiWarps, kWarpMma = kWarpProd + 1, kWarpStore = kWarpMma + 1;
-constexpr int kThreads = (kWarpStore + 1) * 32;   // 480: 15 warps, still at most 4 per SM sub-partition
+constexpr int kThreads = (kWarpStore + 1) * 32;   // 480
 constexpr int kSlots = 4;               // TMEM accumulator slots (item n uses slot n % 4)
 
 constexpr uint32_t KBLK_BYTES = L * 128;               // one 64-channel K block of the B tile
