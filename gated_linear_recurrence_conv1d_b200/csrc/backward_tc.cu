@@ -54,8 +54,8 @@ constexpr int kChunk = 64;       // tokens per chunk of the reverse scan
 // Resident blocks per SM asked of the three streaming kernels (their register caps) and the
 // conv transpose's prefetch depth, set by measurement on B200 (rg2b_bf16): more resident warps
 // hide the scans' load latency better than deeper per-thread batches.
-constexpr int kAggMinBlocks = 12, kOutMinBlocks = 12, kConvTMinBlocks = 6;
-constexpr int kPFC = 8;          // positions a conv-transpose batch loads ahead
+constexpr int kAggMinBlocks = 12, kOutMinBlocks = 12, kConvTMinBlocks = 4;
+constexpr int kPFC = 4;          // positions a conv-transpose batch loads ahead
 
 struct Layout {
     size_t ga, gx, hprev, dxc, xc_hi, xc_lo, dga_hi, dga_lo, dgx_hi, dgx_lo;
@@ -360,91 +360,117 @@ __device__ __forceinline__ bool window_reads(const uint8_t* rrow, int s, int t) 
     return true;
 }
 
-// Thread = (row b, block of kTB positions, channel pair ch, ch + 1); one walk over the block's
+// Thread = (row b, block of kTB positions, channels ch .. ch + 3); one walk over the block's
 // positions s with the last three x and the next three dxc in registers: the parameter gradients
 // of token t = s (the taps that read x_{s-3..s}) and dx_s (the taps of the tokens s..s+3 that
 // read x_s).  A window reads position s for token t when no segment starts in (s, t]: L below is
-// the last segment start at or before the current token.  Every value is a channel pair.
+// the last segment start at or before the current token.  Values are four channels as two pairs.
 __device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 
+// Four channels as two packed pairs.
+struct F4 {
+    float2 lo, hi;
+};
+__device__ __forceinline__ F4 f4fma(F4 x, F4 y, F4 z) { return {f2fma(x.lo, y.lo, z.lo), f2fma(x.hi, y.hi, z.hi)}; }
+__device__ __forceinline__ F4 f4add(F4 x, F4 y) {
+    return {make_float2(x.lo.x + y.lo.x, x.lo.y + y.lo.y), make_float2(x.hi.x + y.hi.x, x.hi.y + y.hi.y)};
+}
+__device__ __forceinline__ F4 f4zero() { return {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}; }
+__device__ __forceinline__ F4 f4_bf16x4(uint2 v) {
+    return {__bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x)),
+            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y))};
+}
+
 __global__ void __launch_bounds__(128, kConvTMinBlocks) bwd_convT_kernel(ConvTArgs a) {
-    const int ch = 2 * (blockIdx.x * 128 + threadIdx.x), tb = blockIdx.y, b = blockIdx.z;
+    const int ch = 4 * (blockIdx.x * 128 + threadIdx.x), tb = blockIdx.y, b = blockIdx.z;
     if (ch >= a.W) return;
     const int T = a.T;
     const int t0 = tb * kTB, t1 = min(T, t0 + kTB);
     const long long W = a.W;
     const uint8_t* rrow = a.reset ? a.reset + (size_t)b * T : nullptr;
     const size_t rowe = (size_t)b * T * W + ch;             // element (b, 0, ch)
-    const __nv_bfloat162* xr = reinterpret_cast<const __nv_bfloat162*>(a.x + rowe);
-    const float2* dr = reinterpret_cast<const float2*>(a.dxc + rowe);
+    const uint2* xr = reinterpret_cast<const uint2*>(a.x + rowe);        // 4 bf16: 8 bytes
+    const float4* dr = reinterpret_cast<const float4*>(a.dxc + rowe);
     float* dxr = a.dx + rowe;                               // caller's buffer: 4-byte aligned only
-    const long long W2 = W / 2;                             // row pitch in channel pairs
-    float2 cw[kConvWidth];
+    const long long W4 = W / 4;                             // row pitch in channel quads
+    F4 cw[kConvWidth];
 #pragma unroll
-    for (int k = 0; k < kConvWidth; ++k) cw[k] = make_float2(a.conv_w[(size_t)k * W + ch], a.conv_w[(size_t)k * W + ch + 1]);
-    auto xval = [&](int s) -> float2 {                      // x_s, the initial history for s < 0
-        if (s >= 0) return __bfloat1622float2(xr[s * W2]);
-        if (!a.tail0) return make_float2(0.f, 0.f);
-        return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(a.tail0 + ((size_t)b * kHist + (kHist + s)) * W + ch));
+    for (int k = 0; k < kConvWidth; ++k) {
+        const float* c = a.conv_w + (size_t)k * W + ch;
+        cw[k] = {make_float2(c[0], c[1]), make_float2(c[2], c[3])};
+    }
+    auto xval = [&](int s) -> F4 {                          // x_s, the initial history for s < 0
+        if (s >= 0) return f4_bf16x4(xr[s * W4]);
+        if (!a.tail0) return f4zero();
+        const __nv_bfloat162* tp = reinterpret_cast<const __nv_bfloat162*>(a.tail0 + ((size_t)b * kHist + (kHist + s)) * W + ch);
+        return {__bfloat1622float2(tp[0]), __bfloat1622float2(tp[1])};
     };
-    auto dxcv = [&](int t) -> float2 { return t >= 0 && t < T ? dr[t * W2] : make_float2(0.f, 0.f); };
+    auto dxcv = [&](int t) -> F4 {
+        if (t < 0 || t >= T) return f4zero();
+        const float4 v = dr[t * W4];
+        return {make_float2(v.x, v.y), make_float2(v.z, v.w)};
+    };
     auto rs = [&](int p) -> bool { return rrow && p >= 0 && p < T && rrow[p] != 0; };
 
     int L = -kHist - 1;                                     // no segment start within reach
     for (int p = max(0, t0 - kHist); p < t0; ++p)
         if (rs(p)) L = p;
-    float2 xa = xval(t0 - 3), xb = xval(t0 - 2), xcc = xval(t0 - 1);   // x_{t-3}, x_{t-2}, x_{t-1}
-    const float2 z2 = make_float2(0.f, 0.f);
-    float2 s_cw[kConvWidth] = {z2, z2, z2, z2}, s_cb = z2;
+    F4 xa = xval(t0 - 3), xb = xval(t0 - 2), xcc = xval(t0 - 1);   // x_{t-3}, x_{t-2}, x_{t-1}
+    F4 s_cw[kConvWidth] = {f4zero(), f4zero(), f4zero(), f4zero()}, s_cb = f4zero();
     const int sb = tb == 0 ? -kHist : t0;                   // the first block also owns the history
-    float2 d0 = dxcv(sb), d1 = dxcv(sb + 1), d2 = dxcv(sb + 2);
+    F4 d0 = dxcv(sb), d1 = dxcv(sb + 1), d2 = dxcv(sb + 2);
     bool q0 = rs(sb), q1 = rs(sb + 1), q2 = rs(sb + 2);
     // positions in batches of kPFC: the batch's loads are issued together, ahead of its arithmetic
     for (int s0 = sb; s0 < t1; s0 += kPFC) {
-        float2 dn[kPFC], xn[kPFC];
+        F4 dn[kPFC], xn[kPFC];
         bool qn[kPFC];
 #pragma unroll
         for (int j = 0; j < kPFC; ++j) {
             const int s = s0 + j;
             dn[j] = dxcv(s + 3);
             qn[j] = rs(s + 3);
-            xn[j] = s >= t0 && s < t1 ? __bfloat1622float2(xr[s * W2]) : z2;
+            xn[j] = s >= t0 && s < t1 ? f4_bf16x4(xr[s * W4]) : f4zero();
         }
 #pragma unroll
         for (int j = 0; j < kPFC; ++j) {
             const int s = s0 + j;
             if (s >= t1) break;
-            const float2 d3 = dn[j];
+            const F4 d3 = dn[j];
             const bool q3 = qn[j];
             if (s >= t0) {                                  // token t = s: its four taps
-                const float2 xs = xn[j];
+                const F4 xs = xn[j];
                 if (q0) L = s;
-                s_cb = make_float2(s_cb.x + d0.x, s_cb.y + d0.y);
-                if (s - 3 >= L) s_cw[0] = f2fma(d0, xa, s_cw[0]);
-                if (s - 2 >= L) s_cw[1] = f2fma(d0, xb, s_cw[1]);
-                if (s - 1 >= L) s_cw[2] = f2fma(d0, xcc, s_cw[2]);
-                s_cw[3] = f2fma(d0, xs, s_cw[3]);
+                s_cb = f4add(s_cb, d0);
+                if (s - 3 >= L) s_cw[0] = f4fma(d0, xa, s_cw[0]);
+                if (s - 2 >= L) s_cw[1] = f4fma(d0, xb, s_cw[1]);
+                if (s - 1 >= L) s_cw[2] = f4fma(d0, xcc, s_cw[2]);
+                s_cw[3] = f4fma(d0, xs, s_cw[3]);
                 xa = xb; xb = xcc; xcc = xs;
             }
             // dx_s: tap k of token s + 3 - k, while no segment starts in (s, s + 3 - k]
             const bool ok1 = !q1, ok2 = ok1 && !q2, ok3 = ok2 && !q3;
-            float2 acc = z2;
-            if (ok3 && s + 3 >= 0 && s + 3 < T) acc = f2fma(cw[0], d3, acc);
-            if (ok2 && s + 2 >= 0 && s + 2 < T) acc = f2fma(cw[1], d2, acc);
-            if (ok1 && s + 1 >= 0 && s + 1 < T) acc = f2fma(cw[2], d1, acc);
-            if (s >= 0) acc = f2fma(cw[3], d0, acc);
+            F4 acc = f4zero();
+            if (ok3 && s + 3 >= 0 && s + 3 < T) acc = f4fma(cw[0], d3, acc);
+            if (ok2 && s + 2 >= 0 && s + 2 < T) acc = f4fma(cw[1], d2, acc);
+            if (ok1 && s + 1 >= 0 && s + 1 < T) acc = f4fma(cw[2], d1, acc);
+            if (s >= 0) acc = f4fma(cw[3], d0, acc);
             if (a.dtail_final && s >= T - kHist && window_reads(rrow, s, T - 1)) {
                 const float* df = a.dtail_final + ((size_t)b * kHist + (s - (T - kHist))) * W + ch;
-                acc = make_float2(acc.x + df[0], acc.y + df[1]);
+                acc = f4add(acc, {make_float2(df[0], df[1]), make_float2(df[2], df[3])});
             }
             if (s >= 0) {
-                dxr[s * W] = acc.x;
-                dxr[s * W + 1] = acc.y;
+                float* o = dxr + (size_t)s * W;
+                o[0] = acc.lo.x;
+                o[1] = acc.lo.y;
+                o[2] = acc.hi.x;
+                o[3] = acc.hi.y;
             } else if (a.dtail0) {
                 float* dt = a.dtail0 + ((size_t)b * kHist + (kHist + s)) * W + ch;
-                dt[0] = acc.x;
-                dt[1] = acc.y;
+                dt[0] = acc.lo.x;
+                dt[1] = acc.lo.y;
+                dt[2] = acc.hi.x;
+                dt[3] = acc.hi.y;
             }
             d0 = d1; d1 = d2; d2 = d3;
             q0 = q1; q1 = q2; q2 = q3;
@@ -452,8 +478,9 @@ __global__ void __launch_bounds__(128, kConvTMinBlocks) bwd_convT_kernel(ConvTAr
     }
     const size_t pb = (size_t)a.B * a.ntb * W, pi = ((size_t)b * a.ntb + tb) * W + ch;
 #pragma unroll
-    for (int k = 0; k < kConvWidth; ++k) *reinterpret_cast<float2*>(a.part + k * pb + pi) = s_cw[k];
-    *reinterpret_cast<float2*>(a.part + 4 * pb + pi) = s_cb;
+    for (int k = 0; k < kConvWidth; ++k)
+        *reinterpret_cast<float4*>(a.part + k * pb + pi) = make_float4(s_cw[k].lo.x, s_cw[k].lo.y, s_cw[k].hi.x, s_cw[k].hi.y);
+    *reinterpret_cast<float4*>(a.part + 4 * pb + pi) = make_float4(s_cb.lo.x, s_cb.lo.y, s_cb.hi.x, s_cb.hi.y);
 }
 
 // ---------------------------------------------------------------- 6. fixed-order sums -------
@@ -613,7 +640,7 @@ cudaError_t launch_backward_tc(const rglru_dims* d, const rglru_params* p, const
     ca.tail0 = st0 ? static_cast<const __nv_bfloat16*>(st0->conv_tail) : nullptr;
     ca.reset = reset; ca.dtail_final = dtail_final; ca.dxc = f32(l.dxc);
     ca.dx = grads->dx; ca.dtail0 = grads->dtail0; ca.part = f32(l.part_conv);
-    bwd_convT_kernel<<<dim3((W + 255) / 256, l.ntb, B), 128, 0, s>>>(ca);
+    bwd_convT_kernel<<<dim3((W + 511) / 512, l.ntb, B), 128, 0, s>>>(ca);   // 4 channels a thread
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
